@@ -1,0 +1,219 @@
+"""CPU oracle of the Video Sparse Attention forward path (test infrastructure).
+
+Only the test suite, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The CUDA library never loads it.
+
+The arithmetic lives in ``vsa_oracle.c`` (plain C, built with gcc,
+``-ffp-contract=off``); this module builds it on demand and wraps each
+function for numpy arrays.  bf16 tensors travel as uint16 bit patterns.
+Each step follows the statement cited in the C file's header:
+
+* ``geometry``/``tile``/``untile``/``pool``/``score``/``topk``: "FastVideo VSA"
+  (vLLM-Omni user guide), introduction and section "Choose top-k";
+* ``map_to_index``: FastVideo commit log, examples/inference/basic/README.md;
+* ``attn_rows``: "FastVideo VSA", introduction and section "Verify routing
+  and fallback" (non-causal, scale head_size^-1/2), computed in fp64.
+
+Pins (tests/test_oracle_*.py) check every function against results fixed by
+the pages or by mathematics, never against itself.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "vsa_oracle.c")
+_LIB = os.path.join(_HERE, "libvsa_oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile vsa_oracle.c into libvsa_oracle.so next to it."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-ffp-contract=off", "-fPIC", "-shared",
+               "-Wall", "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        i = ctypes.c_int
+        L = ctypes.c_long
+        geo = [i] * 7
+        lib.oracle_geometry.argtypes = geo + [P]
+        lib.oracle_block_valid_counts.argtypes = geo + [P]
+        lib.oracle_tile.argtypes = geo + [P, P, i, i, i]
+        lib.oracle_untile.argtypes = geo + [P, P, i, i, i]
+        lib.oracle_pool.argtypes = geo + [P, P, i, i, i]
+        lib.oracle_score.argtypes = [P, P, P, i, i, i, i]
+        lib.oracle_topk.argtypes = [P, i, i, i, i, P, P]
+        lib.oracle_map_to_index.argtypes = [P, i, i, i, i, P, P]
+        lib.oracle_attn_rows.argtypes = geo + [P, P, P, P, P, i, i, i, i, P, L, P, P]
+        lib.oracle_max_threads.argtypes = []
+        for f in ("oracle_geometry", "oracle_block_valid_counts", "oracle_tile", "oracle_untile",
+                  "oracle_pool", "oracle_score", "oracle_topk", "oracle_map_to_index",
+                  "oracle_attn_rows", "oracle_max_threads"):
+            getattr(lib, f).restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise ValueError(f"oracle {what} failed with code {rc}")
+
+
+@dataclass(frozen=True)
+class Geometry:
+    n_prefix: int
+    T: int
+    Hg: int
+    Wg: int
+    bt: int
+    bh: int
+    bw: int
+    bs: int
+    nT: int
+    nH: int
+    nW: int
+    n_pre: int
+    NB: int
+    S: int
+    Sp: int
+
+    @property
+    def args(self):
+        return (self.n_prefix, self.T, self.Hg, self.Wg, self.bt, self.bh, self.bw)
+
+
+def geometry(T, Hg, Wg, block=(4, 8, 8), n_prefix=0) -> Geometry:
+    out = np.zeros(8, dtype=np.int64)
+    _check(_load().oracle_geometry(n_prefix, T, Hg, Wg, *block, _ptr(out)), "geometry")
+    bs, nT, nH, nW, n_pre, NB, S, Sp = (int(x) for x in out)
+    return Geometry(n_prefix, T, Hg, Wg, *block, bs, nT, nH, nW, n_pre, NB, S, Sp)
+
+
+def geometry_of(wl) -> Geometry:
+    return geometry(wl.T, wl.Hg, wl.Wg, wl.block, wl.n_prefix)
+
+
+def block_valid_counts(g: Geometry) -> np.ndarray:
+    out = np.zeros(g.NB, dtype=np.int32)
+    _check(_load().oracle_block_valid_counts(*g.args, _ptr(out)), "block_valid_counts")
+    return out
+
+
+def tile(g: Geometry, x: np.ndarray) -> np.ndarray:
+    """x [B,S,H,D] bf16 bits -> [B,H,Sp,D] bf16 bits."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    B, S, H, D = x.shape
+    assert S == g.S
+    out = np.empty((B, H, g.Sp, D), dtype=np.uint16)
+    _check(_load().oracle_tile(*g.args, _ptr(x), _ptr(out), B, H, D), "tile")
+    return out
+
+
+def untile(g: Geometry, xt: np.ndarray) -> np.ndarray:
+    """xt [B,H,Sp,D] -> [B,S,H,D] (padded rows dropped). Works for any 2-byte dtype."""
+    xt = np.ascontiguousarray(xt)
+    assert xt.dtype.itemsize == 2
+    B, H, Sp, D = xt.shape
+    assert Sp == g.Sp
+    src = xt.view(np.uint16)
+    out = np.empty((B, g.S, H, D), dtype=np.uint16)
+    _check(_load().oracle_untile(*g.args, _ptr(src), _ptr(out), B, H, D), "untile")
+    return out.view(xt.dtype)
+
+
+def pool(g: Geometry, xt: np.ndarray) -> np.ndarray:
+    """Tiled xt [B,H,Sp,D] bf16 bits -> fp32 block means [B,H,NB,D]."""
+    xt = np.ascontiguousarray(xt, dtype=np.uint16)
+    B, H, Sp, D = xt.shape
+    out = np.empty((B, H, g.NB, D), dtype=np.float32)
+    _check(_load().oracle_pool(*g.args, _ptr(xt), _ptr(out), B, H, D), "pool")
+    return out
+
+
+def score(qbar: np.ndarray, kbar: np.ndarray) -> np.ndarray:
+    qbar = np.ascontiguousarray(qbar, dtype=np.float32)
+    kbar = np.ascontiguousarray(kbar, dtype=np.float32)
+    B, H, NB, D = qbar.shape
+    assert kbar.shape == qbar.shape
+    out = np.empty((B, H, NB, NB), dtype=np.float32)
+    _check(_load().oracle_score(_ptr(qbar), _ptr(kbar), _ptr(out), B, H, NB, D), "score")
+    return out
+
+
+def topk(s: np.ndarray, k: int):
+    """Block scores [B,H,NB,NB] -> (q2k_idx [B,H,NB,k] ascending, q2k_num [B,H,NB])."""
+    s = np.ascontiguousarray(s, dtype=np.float32)
+    B, H, NB, NB2 = s.shape
+    assert NB == NB2
+    idx = np.empty((B, H, NB, max(k, 1)), dtype=np.int32)
+    num = np.empty((B, H, NB), dtype=np.int32)
+    _check(_load().oracle_topk(_ptr(s), B, H, NB, k, _ptr(idx), _ptr(num)), "topk")
+    return idx, num
+
+
+def map_to_index(m: np.ndarray):
+    """Bool map [B,H,NQ,NK] -> (q2k_idx [B,H,NQ,NK] ascending, -1 padded; q2k_num)."""
+    m = np.ascontiguousarray(m, dtype=np.uint8)
+    B, H, NQ, NK = m.shape
+    idx = np.empty((B, H, NQ, NK), dtype=np.int32)
+    num = np.empty((B, H, NQ), dtype=np.int32)
+    _check(_load().oracle_map_to_index(_ptr(m), B, H, NQ, NK, _ptr(idx), _ptr(num)), "map_to_index")
+    return idx, num
+
+
+def attn_rows(g: Geometry, qt, kt, vt, idx, num, rows):
+    """fp64 attention for flat rows of [B,H,Sp]; returns (o [n,D] f64, lse [n] f64)."""
+    qt = np.ascontiguousarray(qt, dtype=np.uint16)
+    kt = np.ascontiguousarray(kt, dtype=np.uint16)
+    vt = np.ascontiguousarray(vt, dtype=np.uint16)
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    num = np.ascontiguousarray(num, dtype=np.int32)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    B, H, Sp, D = qt.shape
+    max_k = idx.shape[-1]
+    o = np.empty((len(rows), D), dtype=np.float64)
+    lse = np.empty(len(rows), dtype=np.float64)
+    _check(_load().oracle_attn_rows(*g.args, _ptr(qt), _ptr(kt), _ptr(vt), _ptr(idx), _ptr(num),
+                                    max_k, B, H, D, _ptr(rows), len(rows), _ptr(o), _ptr(lse)),
+           "attn_rows")
+    return o, lse
+
+
+def attn(g: Geometry, qt, kt, vt, idx, num):
+    """fp64 attention over every row: (o [B,H,Sp,D], lse [B,H,Sp])."""
+    B, H, Sp, D = qt.shape
+    rows = np.arange(B * H * Sp, dtype=np.int64)
+    o, lse = attn_rows(g, qt, kt, vt, idx, num, rows)
+    return o.reshape(B, H, Sp, D), lse.reshape(B, H, Sp)
+
+
+def max_threads() -> int:
+    return int(_load().oracle_max_threads())
+
+
+def coarse(g: Geometry, qt, kt, k: int):
+    """pool -> score -> top-k, the whole coarse stage on tiled Q and K."""
+    qbar = pool(g, qt)
+    kbar = pool(g, kt)
+    return topk(score(qbar, kbar), k), (qbar, kbar)

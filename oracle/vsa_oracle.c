@@ -1,0 +1,332 @@
+/*
+ * vsa_oracle.c -- plain CPU oracle of the Video Sparse Attention forward path.
+ *
+ * TEST INFRASTRUCTURE.  Only the test suite, the package smoke check and the
+ * CPU-baseline leg of the benchmark load this library.  It shares no code,
+ * header, table or helper with the CUDA library, and neither calls the other.
+ *
+ * What it computes, step by step, and where each step is stated:
+ *
+ *  geometry  "FastVideo VSA" (vLLM-Omni user guide), section "Choose top-k":
+ *            the post-patch latent grid (T, H, W) is cut into blocks of
+ *            (4, 8, 8) tokens; num_blocks counts the zero-padded grid, e.g.
+ *            (31, 22, 40) -> 8 * 3 * 5 = 120.  A prefix of n_prefix tokens
+ *            (the tile-64 layout of the FastVideo commit log,
+ *            examples/inference/basic/README.md) is cut into contiguous tiles
+ *            placed before the video blocks.
+ *  tile      same page, introduction: tokens are regrouped so that every
+ *            spatiotemporal block is contiguous.  Blocks are in raster order
+ *            over (bT, bH, bW); tokens inside a block in raster order over
+ *            (lt, lh, lw); padding sits at its grid coordinates and is zero.
+ *  pool      same page, introduction ("for every query block, VSA scores the
+ *            key/value blocks"): a block is summarised by the mean of its
+ *            valid tokens.  Sum in slot order in fp32, then one fp32 division.
+ *  score     block score = pooled q . pooled k, one fused multiply-add per
+ *            channel in channel order, fp32 (no scale: ranking ignores it).
+ *  top-k     same page, sections "Enable the backend" and "Choose top-k":
+ *            each query block keeps its topk highest-scoring key blocks,
+ *            0 < topk <= num_blocks; ties go to the lower block index; the
+ *            kept indices are written in ascending order.
+ *  map       FastVideo commit log: a bool block map [B,H,NQ,NK] is compacted
+ *            into q2k_idx (ascending, -1 padded) and q2k_num (may be 0).
+ *  attention "FastVideo VSA", sections introduction and "Verify routing and
+ *            fallback": non-causal attention of every query token of a block
+ *            against the valid tokens of its selected blocks only, scale
+ *            head_size^-1/2, equal Q/KV lengths and head counts, no mask.
+ *            Computed in double from the bf16 inputs.  A row with count 0
+ *            gives o = 0 and lse = -inf (commit log: zero-count rows).
+ *  untile    inverse of tile; padded rows are dropped.
+ *
+ * bf16 tensors are passed as their raw 16-bit patterns.  Build with
+ * -ffp-contract=off so that every fp32 operation rounds as written.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_OK 0
+#define ORACLE_ERR_ARG 1
+#define ORACLE_ERR_INDEX 2
+#define ORACLE_ERR_NOMEM 3
+
+typedef struct {
+    int n_prefix, T, Hg, Wg, bt, bh, bw;
+    int bs;           /* tokens per block */
+    int nT, nH, nW;   /* blocks along each grid axis */
+    int n_pre;        /* prefix tiles */
+    int NB;           /* total blocks */
+    long S;           /* real tokens */
+    long Sp;          /* padded tokens = NB * bs */
+} geom_t;
+
+static int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+static int geom_init(geom_t *g, int n_prefix, int T, int Hg, int Wg, int bt, int bh, int bw) {
+    if (n_prefix < 0 || T < 1 || Hg < 1 || Wg < 1 || bt < 1 || bh < 1 || bw < 1) return ORACLE_ERR_ARG;
+    g->n_prefix = n_prefix; g->T = T; g->Hg = Hg; g->Wg = Wg;
+    g->bt = bt; g->bh = bh; g->bw = bw;
+    g->bs = bt * bh * bw;
+    g->nT = ceil_div(T, bt); g->nH = ceil_div(Hg, bh); g->nW = ceil_div(Wg, bw);
+    g->n_pre = ceil_div(n_prefix, g->bs);
+    g->NB = g->n_pre + g->nT * g->nH * g->nW;
+    g->S = (long)n_prefix + (long)T * Hg * Wg;
+    g->Sp = (long)g->NB * g->bs;
+    return ORACLE_OK;
+}
+
+/* out[0..7] = bs, nT, nH, nW, n_pre, NB, S, Sp */
+int oracle_geometry(int n_prefix, int T, int Hg, int Wg, int bt, int bh, int bw, long *out) {
+    geom_t g;
+    int rc = geom_init(&g, n_prefix, T, Hg, Wg, bt, bh, bw);
+    if (rc) return rc;
+    out[0] = g.bs; out[1] = g.nT; out[2] = g.nH; out[3] = g.nW; out[4] = g.n_pre;
+    out[5] = g.NB; out[6] = g.S; out[7] = g.Sp;
+    return ORACLE_OK;
+}
+
+/* Position in the tiled sequence of untiled token s. */
+static long tiled_pos_of_token(const geom_t *g, long s) {
+    if (s < g->n_prefix) return s; /* prefix tiles are contiguous and come first */
+    long v = s - g->n_prefix;
+    int x = (int)(v % g->Wg);
+    int y = (int)((v / g->Wg) % g->Hg);
+    int t = (int)(v / ((long)g->Wg * g->Hg));
+    int bT = t / g->bt, lt = t % g->bt;
+    int bH = y / g->bh, lh = y % g->bh;
+    int bW = x / g->bw, lw = x % g->bw;
+    long blk = (long)g->n_pre + ((long)bT * g->nH + bH) * g->nW + bW;
+    long slot = ((long)lt * g->bh + lh) * g->bw + lw;
+    return blk * g->bs + slot;
+}
+
+/* Whether slot `slot` of block `blk` holds a real token (else it is padding). */
+static int slot_is_valid(const geom_t *g, int blk, int slot) {
+    if (blk < g->n_pre) return (long)blk * g->bs + slot < g->n_prefix;
+    int vb = blk - g->n_pre;
+    int bW = vb % g->nW, bH = (vb / g->nW) % g->nH, bT = vb / (g->nW * g->nH);
+    int lw = slot % g->bw, lh = (slot / g->bw) % g->bh, lt = slot / (g->bw * g->bh);
+    return bT * g->bt + lt < g->T && bH * g->bh + lh < g->Hg && bW * g->bw + lw < g->Wg;
+}
+
+static int block_valid_count(const geom_t *g, int blk) {
+    int c = 0;
+    for (int s = 0; s < g->bs; ++s) c += slot_is_valid(g, blk, s);
+    return c;
+}
+
+int oracle_block_valid_counts(int n_prefix, int T, int Hg, int Wg, int bt, int bh, int bw, int *counts) {
+    geom_t g;
+    int rc = geom_init(&g, n_prefix, T, Hg, Wg, bt, bh, bw);
+    if (rc) return rc;
+    for (int b = 0; b < g.NB; ++b) counts[b] = block_valid_count(&g, b);
+    return ORACLE_OK;
+}
+
+static float bf16_to_f32(uint16_t h) {
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+/* tile: x [B,S,H,D] -> xt [B,H,Sp,D]; padded rows are zero. */
+int oracle_tile(int n_prefix, int T, int Hg, int Wg, int bt, int bh, int bw,
+                const uint16_t *x, uint16_t *xt, int B, int H, int D) {
+    geom_t g;
+    int rc = geom_init(&g, n_prefix, T, Hg, Wg, bt, bh, bw);
+    if (rc) return rc;
+    memset(xt, 0, sizeof(uint16_t) * (size_t)B * H * g.Sp * D);
+    for (int b = 0; b < B; ++b)
+        for (long s = 0; s < g.S; ++s) {
+            long p = tiled_pos_of_token(&g, s);
+            for (int h = 0; h < H; ++h)
+                memcpy(xt + (((size_t)b * H + h) * g.Sp + p) * D,
+                       x + (((size_t)b * g.S + s) * H + h) * D, sizeof(uint16_t) * D);
+        }
+    return ORACLE_OK;
+}
+
+/* untile: xt [B,H,Sp,D] -> x [B,S,H,D]; padded rows are dropped. */
+int oracle_untile(int n_prefix, int T, int Hg, int Wg, int bt, int bh, int bw,
+                  const uint16_t *xt, uint16_t *x, int B, int H, int D) {
+    geom_t g;
+    int rc = geom_init(&g, n_prefix, T, Hg, Wg, bt, bh, bw);
+    if (rc) return rc;
+    for (int b = 0; b < B; ++b)
+        for (long s = 0; s < g.S; ++s) {
+            long p = tiled_pos_of_token(&g, s);
+            for (int h = 0; h < H; ++h)
+                memcpy(x + (((size_t)b * g.S + s) * H + h) * D,
+                       xt + (((size_t)b * H + h) * g.Sp + p) * D, sizeof(uint16_t) * D);
+        }
+    return ORACLE_OK;
+}
+
+/* pool: xt [B,H,Sp,D] -> pooled [B,H,NB,D] fp32 mean over the valid slots,
+ * summed in slot order with one fp32 rounding per addition. */
+int oracle_pool(int n_prefix, int T, int Hg, int Wg, int bt, int bh, int bw,
+                const uint16_t *xt, float *pooled, int B, int H, int D) {
+    geom_t g;
+    int rc = geom_init(&g, n_prefix, T, Hg, Wg, bt, bh, bw);
+    if (rc) return rc;
+#pragma omp parallel for schedule(static)
+    for (int bhh = 0; bhh < B * H; ++bhh)
+        for (int blk = 0; blk < g.NB; ++blk) {
+            int count = block_valid_count(&g, blk);
+            for (int d = 0; d < D; ++d) {
+                float s = 0.0f;
+                for (int slot = 0; slot < g.bs; ++slot)
+                    if (slot_is_valid(&g, blk, slot))
+                        s = s + bf16_to_f32(xt[((size_t)bhh * g.Sp + (size_t)blk * g.bs + slot) * D + d]);
+                pooled[((size_t)bhh * g.NB + blk) * D + d] = s / (float)count;
+            }
+        }
+    return ORACLE_OK;
+}
+
+/* score: s[b,h,i,j] = sum_d qbar[i,d] * kbar[j,d], fused multiply-add in d order. */
+int oracle_score(const float *qbar, const float *kbar, float *s, int B, int H, int NB, int D) {
+#pragma omp parallel for schedule(static)
+    for (int bhh = 0; bhh < B * H; ++bhh)
+        for (int i = 0; i < NB; ++i)
+            for (int j = 0; j < NB; ++j) {
+                const float *qi = qbar + ((size_t)bhh * NB + i) * D;
+                const float *kj = kbar + ((size_t)bhh * NB + j) * D;
+                float acc = 0.0f;
+                for (int d = 0; d < D; ++d) acc = fmaf(qi[d], kj[d], acc);
+                s[((size_t)bhh * NB + i) * NB + j] = acc;
+            }
+    return ORACLE_OK;
+}
+
+typedef struct { float v; int j; } scored_t;
+
+/* Descending score; equal scores keep the lower block index first. */
+static int by_score_then_index(const void *a, const void *b) {
+    const scored_t *x = (const scored_t *)a, *y = (const scored_t *)b;
+    if (x->v > y->v) return -1;
+    if (x->v < y->v) return 1;
+    return (x->j > y->j) - (x->j < y->j);
+}
+
+static int by_index(const void *a, const void *b) {
+    int x = *(const int *)a, y = *(const int *)b;
+    return (x > y) - (x < y);
+}
+
+/* top-k: s [B,H,NB,NB] -> idx [B,H,NB,topk] ascending, num [B,H,NB] = topk. */
+int oracle_topk(const float *s, int B, int H, int NB, int topk, int32_t *idx, int32_t *num) {
+    if (topk < 1 || topk > NB) return ORACLE_ERR_ARG;
+    scored_t *row = (scored_t *)malloc(sizeof(scored_t) * NB);
+    int *keep = (int *)malloc(sizeof(int) * topk);
+    if (!row || !keep) { free(row); free(keep); return ORACLE_ERR_NOMEM; }
+    for (long r = 0; r < (long)B * H * NB; ++r) {
+        for (int j = 0; j < NB; ++j) { row[j].v = s[r * NB + j]; row[j].j = j; }
+        qsort(row, NB, sizeof(scored_t), by_score_then_index);
+        for (int t = 0; t < topk; ++t) keep[t] = row[t].j;
+        qsort(keep, topk, sizeof(int), by_index);
+        for (int t = 0; t < topk; ++t) idx[r * topk + t] = keep[t];
+        num[r] = topk;
+    }
+    free(row);
+    free(keep);
+    return ORACLE_OK;
+}
+
+/* map_to_index: map [B,H,NQ,NK] bool -> idx [B,H,NQ,NK] (ascending, -1 padded), num. */
+int oracle_map_to_index(const uint8_t *map, int B, int H, int NQ, int NK, int32_t *idx, int32_t *num) {
+    for (long r = 0; r < (long)B * H * NQ; ++r) {
+        int c = 0;
+        for (int j = 0; j < NK; ++j)
+            if (map[r * NK + j]) idx[r * NK + c++] = j;
+        for (int j = c; j < NK; ++j) idx[r * NK + j] = -1;
+        num[r] = c;
+    }
+    return ORACLE_OK;
+}
+
+/*
+ * attention on selected blocks, for an explicit list of query rows.
+ *   q, k, v : tiled [B,H,Sp,D] bf16 bits
+ *   idx     : [B,H,NB,max_k] block ids; num: [B,H,NB] counts
+ *   rows    : flat indices into [B,H,Sp]; o_rows [n_rows, D], lse_rows [n_rows]
+ * For query token i of block r: keys are the valid slots of blocks
+ * idx[r, 0..num[r]-1]; o_i = sum_j softmax_j(scale q_i.k_j) v_j,
+ * lse_i = log sum_j exp(scale q_i.k_j), scale = 1/sqrt(D).
+ */
+int oracle_attn_rows(int n_prefix, int T, int Hg, int Wg, int bt, int bh, int bw,
+                     const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                     const int32_t *idx, const int32_t *num, int max_k,
+                     int B, int H, int D, const int64_t *rows, long n_rows,
+                     double *o_rows, double *lse_rows) {
+    geom_t g;
+    int rc = geom_init(&g, n_prefix, T, Hg, Wg, bt, bh, bw);
+    if (rc) return rc;
+    (void)B; (void)H; /* rows are flat indices into [B,H,Sp] */
+    if (D < 1 || D > 512 || max_k < 1) return ORACLE_ERR_ARG;
+    const double scale = 1.0 / sqrt((double)D);
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 4) reduction(| : bad)
+    for (long n = 0; n < n_rows; ++n) {
+        long flat = rows[n];
+        long i = flat % g.Sp;
+        long bhh = flat / g.Sp;
+        int rblk = (int)(i / g.bs);
+        int cnt = num[bhh * g.NB + rblk];
+        double *o = o_rows + (size_t)n * D;
+        for (int d = 0; d < D; ++d) o[d] = 0.0;
+        if (cnt <= 0 || cnt > max_k) {
+            lse_rows[n] = -INFINITY;
+            if (cnt != 0) bad = 1;
+            continue;
+        }
+        double qi[512];
+        for (int d = 0; d < D; ++d) qi[d] = bf16_to_f32(q[((size_t)bhh * g.Sp + i) * D + d]);
+        double *logit = (double *)malloc(sizeof(double) * (size_t)cnt * g.bs);
+        long *key = (long *)malloc(sizeof(long) * (size_t)cnt * g.bs);
+        long nk = 0;
+        for (int t = 0; t < cnt; ++t) {
+            int kb = idx[(bhh * g.NB + rblk) * (long)max_k + t];
+            if (kb < 0 || kb >= g.NB) { bad = 1; continue; }
+            for (int slot = 0; slot < g.bs; ++slot) {
+                if (!slot_is_valid(&g, kb, slot)) continue;
+                long j = (long)kb * g.bs + slot;
+                const uint16_t *kj = k + ((size_t)bhh * g.Sp + j) * D;
+                double dot = 0.0;
+                for (int d = 0; d < D; ++d) dot += qi[d] * (double)bf16_to_f32(kj[d]);
+                logit[nk] = scale * dot;
+                key[nk] = j;
+                ++nk;
+            }
+        }
+        if (nk == 0) {
+            lse_rows[n] = -INFINITY;
+        } else {
+            double m = -INFINITY;
+            for (long t = 0; t < nk; ++t) if (logit[t] > m) m = logit[t];
+            double l = 0.0;
+            for (long t = 0; t < nk; ++t) {
+                double p = exp(logit[t] - m);
+                l += p;
+                const uint16_t *vj = v + ((size_t)bhh * g.Sp + key[t]) * D;
+                for (int d = 0; d < D; ++d) o[d] += p * (double)bf16_to_f32(vj[d]);
+            }
+            for (int d = 0; d < D; ++d) o[d] /= l;
+            lse_rows[n] = m + log(l);
+        }
+        free(logit);
+        free(key);
+    }
+    return bad ? ORACLE_ERR_INDEX : ORACLE_OK;
+}
+
+/* Highest thread count OpenMP will use here (1 without OpenMP). */
+int oracle_max_threads(void) {
+#ifdef _OPENMP
+    extern int omp_get_max_threads(void);
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
