@@ -1,0 +1,261 @@
+"""Video Sparse Attention forward path on B200 -- Python binding of libvsa.so.
+
+The binding only marshals arguments: torch CUDA tensors become device
+pointers, the current torch stream becomes the launch stream, and outputs are
+allocated with torch when the caller does not pass them.  Every step of the
+path runs in the CUDA library (include/vsa.h).  There is no fallback: if
+libvsa.so is missing or a call fails, a ``VSAError`` is raised.
+
+Path ("FastVideo VSA", vLLM-Omni user guide, introduction):
+    tile(q, k, v) -> coarse_topk(qbar, kbar) -> sparse_attn_fwd -> untile(o)
+or, with a caller-supplied bool block map (FastVideo commit log),
+    tile -> map_to_index(map) -> sparse_attn_fwd -> untile.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libvsa.so")
+
+# Every symbol include/vsa.h declares.
+SYMBOLS = (
+    "vsa_plan_create", "vsa_plan_create_prefix", "vsa_plan_destroy", "vsa_plan_sizes",
+    "vsa_plan_describe", "vsa_tile", "vsa_untile", "vsa_coarse_topk", "vsa_map_to_index",
+    "vsa_sparse_attn_fwd", "vsa_get_status", "vsa_strerror",
+)
+
+VSA_OK = 0
+VSA_ERR_INVALID_ARG = 1
+VSA_ERR_UNSUPPORTED = 2
+VSA_ERR_TOPK = 3
+VSA_ERR_CUDA = 4
+VSA_ERR_BAD_INDEX = 5
+VSA_ERR_TIMEOUT = 6
+VSA_ERR_NO_DEVICE = 7
+
+_lib = None
+
+
+class VSAError(RuntimeError):
+    def __init__(self, code: int, what: str = ""):
+        self.code = code
+        msg = _lib.vsa_strerror(code).decode() if _lib is not None else f"status {code}"
+        super().__init__(f"{what}: {msg} (code {code})" if what else f"{msg} (code {code})")
+
+
+def lib():
+    """Load libvsa.so (built in-tree); raise if it is absent."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run `python -m block_sparse_video_gather_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        L.vsa_plan_create.argtypes = [i, i, i, i, i, i, P]
+        L.vsa_plan_create_prefix.argtypes = [i, i, i, i, i, i, i, P]
+        L.vsa_plan_destroy.argtypes = [P]
+        L.vsa_plan_destroy.restype = None
+        L.vsa_plan_sizes.argtypes = [P, P, P, P, P]
+        L.vsa_plan_describe.argtypes = [P, i, ctypes.c_char_p, sz]
+        L.vsa_tile.argtypes = [P, P, P, P, i, i, i, P]
+        L.vsa_untile.argtypes = [P, P, P, i, i, i, P]
+        L.vsa_coarse_topk.argtypes = [P, P, P, i, i, i, i, P, P, P]
+        L.vsa_map_to_index.argtypes = [P, i, i, i, i, P, P, P]
+        L.vsa_sparse_attn_fwd.argtypes = [P, P, P, P, P, P, i, i, i, i, P, P, P]
+        L.vsa_get_status.argtypes = [P, P]
+        L.vsa_strerror.argtypes = [i]
+        L.vsa_strerror.restype = ctypes.c_char_p
+        for name in SYMBOLS:
+            if name not in ("vsa_plan_destroy", "vsa_strerror"):
+                getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _check(rc: int, what: str):
+    if rc != VSA_OK:
+        raise VSAError(rc, what)
+
+
+class Plan:
+    """Geometry of one latent grid: block partition, padding, block count."""
+
+    def __init__(self, T: int, Hg: int, Wg: int, block=(4, 8, 8), n_prefix: int = 0):
+        L = lib()
+        h = ctypes.c_void_p()
+        _check(L.vsa_plan_create_prefix(n_prefix, T, Hg, Wg, *block, ctypes.byref(h)), "vsa_plan_create")
+        self._h = h
+        nb, bs = ctypes.c_int(), ctypes.c_int()
+        s, sp = ctypes.c_int64(), ctypes.c_int64()
+        _check(L.vsa_plan_sizes(h, ctypes.byref(nb), ctypes.byref(s), ctypes.byref(sp), ctypes.byref(bs)),
+               "vsa_plan_sizes")
+        self.T, self.Hg, self.Wg, self.block, self.n_prefix = T, Hg, Wg, tuple(block), n_prefix
+        self.NB, self.S, self.Sp, self.bs = nb.value, s.value, sp.value, bs.value
+
+    @classmethod
+    def of(cls, wl) -> "Plan":
+        return cls(wl.T, wl.Hg, wl.Wg, wl.block, wl.n_prefix)
+
+    @property
+    def handle(self):
+        return self._h
+
+    def describe(self, topk: int) -> str:
+        buf = ctypes.create_string_buffer(512)
+        _check(lib().vsa_plan_describe(self._h, topk, buf, len(buf)), "vsa_plan_describe")
+        return buf.value.decode()
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value and _lib is not None:
+            _lib.vsa_plan_destroy(h)
+            self._h = None
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _ptr(t, dtype, what):
+    torch = _torch()
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{what} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{what} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{what} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(_torch().cuda.current_stream().cuda_stream)
+
+
+def tile(plan: Plan, x, pooled: bool = False, out=None, pooled_out=None):
+    """x [B,S,H,D] bf16 -> x_tiled [B,H,Sp,D] (and fp32 block means [B,H,NB,D])."""
+    torch = _torch()
+    B, S, H, D = x.shape
+    if out is None:
+        out = torch.empty((B, H, plan.Sp, D), dtype=torch.bfloat16, device=x.device)
+    if pooled and pooled_out is None:
+        pooled_out = torch.empty((B, H, plan.NB, D), dtype=torch.float32, device=x.device)
+    if S != plan.S:
+        raise ValueError(f"x has {S} tokens, plan expects {plan.S}")
+    _check(lib().vsa_tile(plan.handle, _ptr(x, torch.bfloat16, "x"), _ptr(out, torch.bfloat16, "x_tiled"),
+                          _ptr(pooled_out, torch.float32, "pooled") if pooled else None, B, H, D, _stream()),
+           "vsa_tile")
+    return (out, pooled_out) if pooled else out
+
+
+def untile(plan: Plan, xt, out=None):
+    """x_tiled [B,H,Sp,D] bf16 -> x [B,S,H,D] (padded rows dropped)."""
+    torch = _torch()
+    B, H, Sp, D = xt.shape
+    if Sp != plan.Sp:
+        raise ValueError(f"x_tiled has {Sp} rows, plan expects {plan.Sp}")
+    if out is None:
+        out = torch.empty((B, plan.S, H, D), dtype=torch.bfloat16, device=xt.device)
+    _check(lib().vsa_untile(plan.handle, _ptr(xt, torch.bfloat16, "x_tiled"), _ptr(out, torch.bfloat16, "x"),
+                            B, H, D, _stream()), "vsa_untile")
+    return out
+
+
+def coarse_topk(plan: Plan, qbar, kbar, topk: int, idx_out=None, num_out=None):
+    """Block scores + per-row top-k -> (q2k_idx [B,H,NB,topk], q2k_num [B,H,NB])."""
+    torch = _torch()
+    B, H, NB, D = qbar.shape
+    if idx_out is None:
+        idx_out = torch.empty((B, H, NB, max(topk, 1)), dtype=torch.int32, device=qbar.device)
+    if num_out is None:
+        num_out = torch.empty((B, H, NB), dtype=torch.int32, device=qbar.device)
+    _check(lib().vsa_coarse_topk(plan.handle, _ptr(qbar, torch.float32, "qbar"), _ptr(kbar, torch.float32, "kbar"),
+                                 B, H, D, topk, _ptr(idx_out, torch.int32, "q2k_idx"),
+                                 _ptr(num_out, torch.int32, "q2k_num"), _stream()), "vsa_coarse_topk")
+    return idx_out, num_out
+
+
+def map_to_index(block_map, idx_out=None, num_out=None):
+    """Bool map [B,H,NQ,NK] -> (q2k_idx [B,H,NQ,NK] ascending then -1, q2k_num [B,H,NQ])."""
+    torch = _torch()
+    m = block_map.view(torch.uint8) if block_map.dtype == torch.bool else block_map
+    B, H, NQ, NK = m.shape
+    if idx_out is None:
+        idx_out = torch.empty((B, H, NQ, NK), dtype=torch.int32, device=m.device)
+    if num_out is None:
+        num_out = torch.empty((B, H, NQ), dtype=torch.int32, device=m.device)
+    _check(lib().vsa_map_to_index(_ptr(m, torch.uint8, "map"), B, H, NQ, NK, _ptr(idx_out, torch.int32, "q2k_idx"),
+                                  _ptr(num_out, torch.int32, "q2k_num"), _stream()), "vsa_map_to_index")
+    return idx_out, num_out
+
+
+def sparse_attn_fwd(plan: Plan, q, k, v, q2k_idx, q2k_num, o_out=None, lse_out=None):
+    """Attention of every query block over its selected blocks (tiled layout) -> (o, lse)."""
+    torch = _torch()
+    B, H, Sp, D = q.shape
+    max_k = q2k_idx.shape[-1]
+    if o_out is None:
+        o_out = torch.empty_like(q)
+    if lse_out is None:
+        lse_out = torch.empty((B, H, Sp), dtype=torch.float32, device=q.device)
+    _check(lib().vsa_sparse_attn_fwd(plan.handle, _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
+                                     _ptr(v, torch.bfloat16, "v"), _ptr(q2k_idx, torch.int32, "q2k_idx"),
+                                     _ptr(q2k_num, torch.int32, "q2k_num"), max_k, B, H, D,
+                                     _ptr(o_out, torch.bfloat16, "o"), _ptr(lse_out, torch.float32, "lse"),
+                                     _stream()), "vsa_sparse_attn_fwd")
+    return o_out, lse_out
+
+
+def get_status(stream=None) -> int:
+    """Synchronise the stream, then read and clear the device status word."""
+    torch = _torch()
+    st = ctypes.c_int(0)
+    s = ctypes.c_void_p((stream or torch.cuda.current_stream()).cuda_stream)
+    _check(lib().vsa_get_status(s, ctypes.byref(st)), "vsa_get_status")
+    return st.value
+
+
+class Forward:
+    """The whole forward path with its intermediates allocated once.
+
+    __call__(q, k, v[, block_map]) runs tile(q) with pooling, tile(k) with
+    pooling, tile(v), the coarse stage (or map_to_index when a block map is
+    given), the fine stage and untile(o); it returns o [B,S,H,D] and the tiled
+    lse [B,H,Sp].
+    """
+
+    def __init__(self, plan: Plan, B: int, H: int, topk: int | None, device="cuda", D: int = 128):
+        torch = _torch()
+        self.plan, self.B, self.H, self.D, self.topk = plan, B, H, D, topk
+        t = dict(dtype=torch.bfloat16, device=device)
+        self.qt = torch.empty((B, H, plan.Sp, D), **t)
+        self.kt = torch.empty((B, H, plan.Sp, D), **t)
+        self.vt = torch.empty((B, H, plan.Sp, D), **t)
+        self.ot = torch.empty((B, H, plan.Sp, D), **t)
+        self.o = torch.empty((B, plan.S, H, D), **t)
+        self.lse = torch.empty((B, H, plan.Sp), dtype=torch.float32, device=device)
+        self.qbar = torch.empty((B, H, plan.NB, D), dtype=torch.float32, device=device)
+        self.kbar = torch.empty((B, H, plan.NB, D), dtype=torch.float32, device=device)
+        width = topk if topk is not None else plan.NB
+        self.idx = torch.empty((B, H, plan.NB, width), dtype=torch.int32, device=device)
+        self.num = torch.empty((B, H, plan.NB), dtype=torch.int32, device=device)
+
+    def __call__(self, q, k, v, block_map=None):
+        p = self.plan
+        tile(p, q, pooled=True, out=self.qt, pooled_out=self.qbar)
+        tile(p, k, pooled=True, out=self.kt, pooled_out=self.kbar)
+        tile(p, v, out=self.vt)
+        if block_map is None:
+            coarse_topk(p, self.qbar, self.kbar, self.topk, idx_out=self.idx, num_out=self.num)
+        else:
+            map_to_index(block_map, idx_out=self.idx, num_out=self.num)
+        sparse_attn_fwd(p, self.qt, self.kt, self.vt, self.idx, self.num, o_out=self.ot, lse_out=self.lse)
+        untile(p, self.ot, out=self.o)
+        return self.o, self.lse
+
+    # kernels launched by one call: 3 tiles, 1 index stage, 1 attention, 1 untile
+    launches_per_call = 6

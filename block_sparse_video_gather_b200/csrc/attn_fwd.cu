@@ -1,0 +1,505 @@
+// attn_fwd.cu -- fine stage of VSA: block-sparse flash attention forward on
+// the 5th-generation tensor cores (tcgen05, TMEM accumulators, TMA loads).
+//
+// "FastVideo VSA" (vLLM-Omni user guide), introduction and section "Verify
+// routing and fallback": each query block attends only to the tokens of its
+// selected key/value blocks; non-causal; scale head_size^-1/2.  FastVideo
+// commit log (examples/inference/basic/README.md): rows carry different
+// counts, including zero.
+//
+// Work item: one (b*h, query block) of 256 tokens = two 128-row Q tiles.
+// Each selected key block is two 128-key tiles.  Persistent CTAs, one per SM,
+// take items in head-major order so the K/V of a head stay hot in L2.
+//
+// Warp roles (384 threads):
+//   warp 0      TMA producer: Q (64 KB per item), K and V tiles (32 KB each)
+//               into a 2-stage ring, completion counted on mbarriers.
+//   warp 1      TMEM owner (512 columns) and single-thread MMA issuer.
+//   warps 4-7   softmax + epilogue of Q tile 0 (one thread per query row)
+//   warps 8-11  softmax + epilogue of Q tile 1
+//
+// Tensor memory (128 lanes x 512 fp32 columns):
+//   [  0,128) S0 = Q0 K^T   (P0 = bf16 softmax numerators, aliased on [0,64))
+//   [128,256) S1 = Q1 K^T   (P1 on [128,192))
+//   [256,384) O0            [384,512) O1
+// Per KV tile the MMA thread issues, in order:
+//   PV0(t)  S0(t+1)  PV1(t)  S1(t+1)
+// so softmax of tile 0 overlaps the tensor-core work of tile 1 and back.
+// S MMAs: A = Q (K-major, smem), B = K tile (K-major, smem).
+// PV MMAs: A = P (TMEM), B = V tile (MN-major, smem); O accumulates in TMEM.
+//
+// Online softmax in the log2 domain with a lazy maximum: the running max used
+// for the exponentials only moves when a row's new tile max exceeds it by more
+// than 8 (a factor 256), and only then is that row of O rescaled in TMEM.
+// Numerators stay <= 256, safe in bf16 and fp32; o = O / l and
+// lse = (m + log2 l) ln 2 use the same maximum, so the result is exact.
+//
+// Every mbarrier wait is bounded (globaltimer); on expiry the kernel records
+// VSA_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace vsa {
+
+namespace {
+
+constexpr int kThreads = 384;
+constexpr int kStages = 2;
+constexpr uint32_t kHalfBytes = 128 * 128;      // 128 rows x 64 bf16 (one 128-B swizzle column)
+constexpr uint32_t kTileBytes = 2 * kHalfBytes;  // 128 rows x 128 bf16
+constexpr uint32_t kQBytes = 2 * kTileBytes;     // two Q tiles
+constexpr uint32_t kSmemQ = 0;
+constexpr uint32_t kSmemK = kSmemQ + kQBytes;
+constexpr uint32_t kSmemV = kSmemK + kStages * kTileBytes;
+constexpr uint32_t kSmemBar = kSmemV + kStages * kTileBytes;
+constexpr uint32_t kSmemTotal = kSmemBar + 256 + 1024;  // barriers + 1 KB alignment slack
+constexpr uint64_t kTimeoutNs = 2000000000ull;          // 2 s per wait
+
+constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, 0, 0);   // Q (K-major) x K (K-major)
+constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, 0, 1);  // P (TMEM) x V (MN-major)
+
+struct Barriers {
+  uint64_t q_full, q_empty;
+  uint64_t k_full[kStages], k_empty[kStages];
+  uint64_t v_full[kStages], v_empty[kStages];
+  uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(Barriers) <= 256, "barrier block too large");
+
+struct Params {
+  const int32_t* idx;
+  const int32_t* num;
+  int max_k;
+  int BH;
+  uint16_t* o;
+  float* lse;
+  unsigned int* status;
+  float scale_log2;
+  Geo g;
+};
+
+// Number of selected blocks of an item (clamped into [0, max_k]).
+__device__ __forceinline__ int item_blocks(const Params& p, int item, bool report) {
+  int c = __ldg(p.num + item);
+  if (c < 0 || c > p.max_k) {
+    if (report) atomicCAS(p.status, 0u, (unsigned)VSA_ERR_BAD_INDEX);
+    c = c < 0 ? 0 : p.max_k;
+  }
+  return c;
+}
+
+// Block id of selection j of an item; -1 if out of range.
+__device__ __forceinline__ int item_block_id(const Params& p, int item, int j) {
+  const int kb = __ldg(p.idx + static_cast<long long>(item) * p.max_k + j);
+  return (kb >= 0 && kb < p.g.NB) ? kb : -1;
+}
+
+// Validity bits of the 128 key columns of tile `half` of block kb (bit c of
+// word c/32 set = slot half*128 + c holds a real token).  Returns true when
+// every column is real.
+__device__ __forceinline__ bool key_tile_mask(const Geo& g, int kb, int half, uint32_t (&w)[4]) {
+  if (kb < 0) {
+    w[0] = w[1] = w[2] = w[3] = 0u;
+    return false;
+  }
+  const int first = half * 128;
+  if (kb < g.n_pre) {
+    const int lim = g.n_prefix - kb * g.bs - first;  // real columns of this tile
+    if (lim >= 128) return true;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int n = min(max(lim - 32 * i, 0), 32);
+      w[i] = n >= 32 ? 0xffffffffu : ((1u << n) - 1u);
+    }
+    return false;
+  }
+  int vt, vh, vw;
+  video_block_extent(g, kb - g.n_pre, vt, vh, vw);
+  if (vt == g.bt && vh == g.bh && vw == g.bw) return true;
+  const uint32_t rowbits = vw >= 32 ? 0xffffffffu : ((1u << vw) - 1u);
+  const int rows_per_word = 32 >> g.lbw;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t word = 0;
+    const int row0 = (first + 32 * i) >> g.lbw;
+    for (int r = 0; r < rows_per_word; ++r) {
+      const int R = row0 + r;
+      const int lh = R & (g.bh - 1);
+      const int lt = R >> g.lbh;
+      if (lt < vt && lh < vh) word |= rowbits << (r << g.lbw);
+    }
+    w[i] = word;
+  }
+  return false;
+}
+
+// Warp-uniform bounded wait: all lanes wait, then agree.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Barriers* bars, unsigned int* status) {
+  bool ok = mbar_wait(bar, parity, &bars->abort, status, kTimeoutNs);
+  return __all_sync(0xffffffffu, ok);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte alignment for the 128-byte swizzle atoms
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem + kSmemQ;
+  uint8_t* sK = smem + kSmemK;
+  uint8_t* sV = smem + kSmemV;
+  Barriers* bars = reinterpret_cast<Barriers*>(smem + kSmemBar);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const Geo& g = p.g;
+  const int total_items = p.BH * g.NB;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    mbar_init(&bars->q_empty, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->k_empty[s], 1);
+      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->v_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->s_full[i], 1);
+      mbar_init(&bars->p_full[i], 128);
+      mbar_init(&bars->o_full[i], 1);
+      mbar_init(&bars->o_empty[i], 128);
+    }
+    mbar_init(&bars->drain, 1);
+    bars->abort = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      const uint64_t pol_kv = policy_evict_last();
+      const uint64_t pol_q = policy_evict_first();
+      int kit = 0, vit = 0, qit = 0;
+      for (int item = blockIdx.x; item < total_items; item += gridDim.x) {
+        const int nb = item_blocks(p, item, false);
+        if (nb == 0) continue;
+        const int bh = item / g.NB, qb = item - bh * g.NB;
+        const long long base = static_cast<long long>(bh) * g.Sp;
+        if (!mbar_wait(&bars->q_empty, (qit & 1) ^ 1, &bars->abort, p.status, kTimeoutNs)) break;
+        mbar_arrive_expect_tx(&bars->q_full, kQBytes);
+        const int qrow = static_cast<int>(base + static_cast<long long>(qb) * 256);
+        for (int i = 0; i < 2; ++i)
+          for (int hf = 0; hf < 2; ++hf)
+            tma_load_2d(sQ + i * kTileBytes + hf * kHalfBytes, &tm_q, hf * 64, qrow + i * 128, &bars->q_full, pol_q);
+        ++qit;
+        bool stop = false;
+        for (int t = 0; t < 2 * nb && !stop; ++t) {
+          const int kb0 = item_block_id(p, item, t >> 1);
+          const int kb = kb0 < 0 ? 0 : kb0;  // unusable ids load block 0; the softmax masks them out
+          const int krow = static_cast<int>(base + static_cast<long long>(kb) * 256 + (t & 1) * 128);
+          const int sk = kit % kStages;
+          if (!mbar_wait(&bars->k_empty[sk], ((kit / kStages) & 1) ^ 1, &bars->abort, p.status, kTimeoutNs)) {
+            stop = true;
+            break;
+          }
+          mbar_arrive_expect_tx(&bars->k_full[sk], kTileBytes);
+          for (int hf = 0; hf < 2; ++hf)
+            tma_load_2d(sK + sk * kTileBytes + hf * kHalfBytes, &tm_k, hf * 64, krow, &bars->k_full[sk], pol_kv);
+          ++kit;
+          const int sv = vit % kStages;
+          if (!mbar_wait(&bars->v_empty[sv], ((vit / kStages) & 1) ^ 1, &bars->abort, p.status, kTimeoutNs)) {
+            stop = true;
+            break;
+          }
+          mbar_arrive_expect_tx(&bars->v_full[sv], kTileBytes);
+          for (int hf = 0; hf < 2; ++hf)
+            tma_load_2d(sV + sv * kTileBytes + hf * kHalfBytes, &tm_v, hf * 64, krow, &bars->v_full[sv], pol_kv);
+          ++vit;
+        }
+        if (stop) break;
+      }
+      // Drain: every issued copy must land before the CTA's shared memory is released.
+      if (qit > 0) mbar_wait_drain(&bars->q_full, (qit - 1) & 1, kTimeoutNs);
+      for (int s = 0; s < kStages; ++s) {
+        if (kit > s) {
+          const int last = kit - 1 - ((kit - 1 - s) % kStages);
+          mbar_wait_drain(&bars->k_full[s], (last / kStages) & 1, kTimeoutNs);
+        }
+        if (vit > s) {
+          const int last = vit - 1 - ((vit - 1 - s) % kStages);
+          mbar_wait_drain(&bars->v_full[s], (last / kStages) & 1, kTimeoutNs);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t qaddr = smem_u32(sQ), kaddr = smem_u32(sK), vaddr = smem_u32(sV);
+      int kit = 0, vit = 0, qit = 0, tiles = 0, items = 0;
+      bool ok = true;
+      auto issue_s = [&](int i, int sk) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+          const uint64_t a = sdesc_sw128(qaddr + i * kTileBytes + off, 16, 1024);
+          const uint64_t b = sdesc_sw128(kaddr + sk * kTileBytes + off, 16, 1024);
+          mma_ss(tmem + i * 128, a, b, kIdescS, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int i, int sv, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t b = sdesc_sw128(vaddr + sv * kTileBytes + kk * 2048, kHalfBytes, 1024);
+          mma_ts(tmem + 256 + i * 128, tmem + i * 128 + kk * 8, b, kIdescPV, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      for (int item = blockIdx.x; item < total_items && ok; item += gridDim.x) {
+        const int nb = item_blocks(p, item, true);
+        if (nb == 0) continue;
+        const int n = 2 * nb;
+        if (!(ok = mbar_wait(&bars->q_full, qit & 1, &bars->abort, p.status, kTimeoutNs))) break;
+        ++qit;
+        tc_fence_after();
+        int sk = kit % kStages;
+        if (!(ok = mbar_wait(&bars->k_full[sk], (kit / kStages) & 1, &bars->abort, p.status, kTimeoutNs))) break;
+        tc_fence_after();
+        issue_s(0, sk);
+        mma_commit(&bars->s_full[0]);
+        issue_s(1, sk);
+        mma_commit(&bars->s_full[1]);
+        mma_commit(&bars->k_empty[sk]);
+        ++kit;
+        for (int t = 0; t < n; ++t) {
+          const int sv = vit % kStages;
+          if (!(ok = mbar_wait(&bars->v_full[sv], (vit / kStages) & 1, &bars->abort, p.status, kTimeoutNs))) break;
+          if (!(ok = mbar_wait(&bars->p_full[0], tiles & 1, &bars->abort, p.status, kTimeoutNs))) break;
+          if (t == 0 && !(ok = mbar_wait(&bars->o_empty[0], (items & 1) ^ 1, &bars->abort, p.status, kTimeoutNs)))
+            break;
+          tc_fence_after();
+          issue_pv(0, sv, t > 0);
+          if (t == n - 1) mma_commit(&bars->o_full[0]);
+          const bool more = t + 1 < n;
+          sk = kit % kStages;
+          if (more) {
+            if (!(ok = mbar_wait(&bars->k_full[sk], (kit / kStages) & 1, &bars->abort, p.status, kTimeoutNs))) break;
+            tc_fence_after();
+            issue_s(0, sk);
+            mma_commit(&bars->s_full[0]);
+          }
+          if (!(ok = mbar_wait(&bars->p_full[1], tiles & 1, &bars->abort, p.status, kTimeoutNs))) break;
+          if (t == 0 && !(ok = mbar_wait(&bars->o_empty[1], (items & 1) ^ 1, &bars->abort, p.status, kTimeoutNs)))
+            break;
+          tc_fence_after();
+          issue_pv(1, sv, t > 0);
+          mma_commit(&bars->v_empty[sv]);
+          ++vit;
+          if (t == n - 1) mma_commit(&bars->o_full[1]);
+          if (more) {
+            issue_s(1, sk);
+            mma_commit(&bars->s_full[1]);
+            mma_commit(&bars->k_empty[sk]);
+            ++kit;
+          }
+          ++tiles;
+        }
+        if (!ok) break;
+        mma_commit(&bars->q_empty);
+        ++items;
+      }
+      // Drain: wait for every MMA issued by this thread before TMEM and smem go away.
+      mma_commit(&bars->drain);
+      mbar_wait_drain(&bars->drain, 0, kTimeoutNs);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int wg = (warp - 4) >> 2;  // Q tile
+    const int quarter = warp & 3;    // TMEM lane quarter of this warp
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_off + wg * 128;
+    const uint32_t tO = tmem + lane_off + 256 + wg * 128;
+    const float sl2 = p.scale_log2;
+    int tiles = 0, items = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < total_items && ok; item += gridDim.x) {
+      const int nb = item_blocks(p, item, false);
+      const int bh = item / g.NB, qb = item - bh * g.NB;
+      const long long row = static_cast<long long>(bh) * g.Sp + static_cast<long long>(qb) * 256 + wg * 128 + r;
+      uint4* orow = reinterpret_cast<uint4*>(p.o + row * 128);
+      if (nb == 0) {
+#pragma unroll
+        for (int c = 0; c < 16; ++c) orow[c] = make_uint4(0, 0, 0, 0);
+        p.lse[row] = -INFINITY;
+        continue;
+      }
+      const int n = 2 * nb;
+      float m_used = -INFINITY, l = 0.0f;
+      for (int t = 0; t < n; ++t) {
+        const int kb = item_block_id(p, item, t >> 1);
+        if (kb < 0 && wg == 0 && r == 0) atomicCAS(p.status, 0u, (unsigned)VSA_ERR_BAD_INDEX);
+        uint32_t mw[4];
+        const bool full = key_tile_mask(g, kb, t & 1, mw);
+        if (!(ok = warp_wait(&bars->s_full[wg], tiles & 1, bars, p.status))) break;
+        tc_fence_after();
+        uint32_t sv[128];
+        tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+        tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
+        tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
+        tmem_wait_ld();
+        if (!full) {
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (!((mw[c >> 5] >> (c & 31)) & 1u)) sv[c] = 0xff800000u;  // -inf
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(sv[c]));
+        const float mt = mx * sl2;
+        const bool grow = mt > m_used + 8.0f;  // false while the tile is fully masked
+        const bool rescale = grow && t > 0 && m_used != -INFINITY;
+        const float alpha = rescale ? ex2_approx(m_used - mt) : 1.0f;
+        if (grow) m_used = mt;
+        const float msub = (m_used == -INFINITY) ? 0.0f : m_used;
+        uint32_t pk[64];
+        float lsum = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          const float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * j]), sl2, -msub));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * j + 1]), sl2, -msub));
+          lsum += p0 + p1;
+          pk[j] = pack_bf16x2(p0, p1);
+        }
+        l = l * alpha + lsum;
+        tmem_st32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+        tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+        // Rescale this row of O when its maximum moved (warp-uniform branch;
+        // rows that did not move use alpha = 1).  PV(t-1) is complete: the
+        // s_full commit just waited on follows it in issue order.
+        if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t ov[32];
+            tmem_ld32(tO + c * 32, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha);
+            tmem_st32(tO + c * 32, ov);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bars->p_full[wg]);
+        ++tiles;
+      }
+      if (!ok) break;
+      // epilogue: O / l -> bf16 row, lse
+      if (!(ok = warp_wait(&bars->o_full[wg], items & 1, bars, p.status))) break;
+      tc_fence_after();
+      const float inv = l > 0.0f ? 1.0f / l : 0.0f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t ov[32];
+        tmem_ld32(tO + c * 32, ov);
+        tmem_wait_ld();
+        uint4 w[4];
+        uint32_t* wp = reinterpret_cast<uint32_t*>(w);
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          wp[j] = pack_bf16x2(__uint_as_float(ov[2 * j]) * inv, __uint_as_float(ov[2 * j + 1]) * inv);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) orow[c * 4 + j] = w[j];
+      }
+      tc_fence_before();
+      mbar_arrive(&bars->o_empty[wg]);
+      p.lse[row] = l > 0.0f ? (m_used + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+      ++items;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// [rows, 128] bf16 row-major viewed as a 2-D tensor; box = 64 columns x box_rows rows, 128-B swizzle.
+bool make_tmap(CUtensorMap* tm, const void* base, unsigned long long rows, unsigned box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {128, rows};
+  cuuint64_t strides[1] = {128 * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_attn_fwd(const Geo& g, const AttnArgs& a, cudaStream_t stream) {
+  if (g.bs != 256) return cudaErrorNotSupported;
+  const unsigned long long rows = static_cast<unsigned long long>(a.BH) * g.Sp;
+  if (rows >= (1ull << 31)) return cudaErrorInvalidValue;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap(&tq, a.q, rows, 128) || !make_tmap(&tk, a.k, rows, 128) || !make_tmap(&tv, a.v, rows, 128))
+    return cudaErrorInvalidValue;
+  Params p;
+  p.idx = a.idx;
+  p.num = a.num;
+  p.max_k = a.max_k;
+  p.BH = a.BH;
+  p.o = a.o;
+  p.lse = a.lse;
+  p.status = a.status;
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / 11.313708498984761);  // log2(e) / sqrt(128)
+  p.g = g;
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTotal);
+  if (e != cudaSuccess) return e;
+  const long long items = static_cast<long long>(a.BH) * g.NB;
+  const int grid = static_cast<int>(items < a.num_sms ? items : a.num_sms);
+  attn_fwd_kernel<<<grid, kThreads, kSmemTotal, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace vsa

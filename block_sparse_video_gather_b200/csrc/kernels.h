@@ -1,0 +1,38 @@
+// kernels.h -- internal launch entry points of the VSA kernels (not public ABI).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace vsa {
+
+// tile.cu
+cudaError_t launch_tile(const Geo& g, int B, int H, const uint16_t* x, uint16_t* xt, float* pooled,
+                        cudaStream_t stream);
+cudaError_t launch_untile(const Geo& g, int B, int H, const uint16_t* xt, uint16_t* x, cudaStream_t stream);
+
+// coarse.cu
+cudaError_t launch_score_topk(int BH, int NB, int topk, const float* qbar, const float* kbar, int32_t* idx,
+                              int32_t* num, cudaStream_t stream);
+cudaError_t launch_map_to_index(const uint8_t* map, long long rows, int NK, int32_t* idx, int32_t* num,
+                                cudaStream_t stream);
+
+// attn_fwd.cu
+struct AttnArgs {
+  const uint16_t* q;
+  const uint16_t* k;
+  const uint16_t* v;
+  const int32_t* idx;
+  const int32_t* num;
+  int max_k;
+  int BH;
+  uint16_t* o;
+  float* lse;
+  unsigned int* status;
+  int num_sms;
+};
+cudaError_t launch_attn_fwd(const Geo& g, const AttnArgs& a, cudaStream_t stream);
+
+}  // namespace vsa

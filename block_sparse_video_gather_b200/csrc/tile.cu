@@ -1,0 +1,150 @@
+// tile.cu -- token reorder into spatiotemporal blocks, its inverse, and the
+// per-block mean pooling of the coarse stage.
+//
+// "FastVideo VSA" (vLLM-Omni user guide), introduction and section "Choose
+// top-k": the post-patch latent grid is cut into (4, 8, 8) blocks over the
+// zero-padded grid; each block is summarised for scoring.
+//
+// One CTA per (b, h, block).  A token row of one head is D = 128 bf16 =
+// 256 B, moved as 16 lanes x 16 B, so a warp covers two rows per access and
+// the tiled side is one contiguous 32-64 KB run per CTA.  When pooling, the
+// block is also staged in shared memory and thread d sums channel d over
+// the slots in slot order in fp32 (the order the coarse stage is defined
+// with), then divides once by the real-token count.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace vsa {
+
+namespace {
+
+constexpr int kTileThreads = 256;
+constexpr int kRowChunks = 16;  // 16 B chunks per 256 B row (D = 128)
+
+// Token index of slot `slot` of block `blk`, or -1 for a padded slot.
+__device__ __forceinline__ long long token_of_slot(const Geo& g, int blk, int slot) {
+  if (blk < g.n_pre) {
+    long long s = static_cast<long long>(blk) * g.bs + slot;
+    return s < g.n_prefix ? s : -1;
+  }
+  int vb = blk - g.n_pre;
+  int bW = vb % g.nW, bH = (vb / g.nW) % g.nH, bT = vb / (g.nW * g.nH);
+  int lw = slot & (g.bw - 1);
+  int lh = (slot >> g.lbw) & (g.bh - 1);
+  int lt = slot >> (g.lbw + g.lbh);
+  int t = bT * g.bt + lt, y = bH * g.bh + lh, x = bW * g.bw + lw;
+  if (t >= g.T || y >= g.Hg || x >= g.Wg) return -1;
+  return g.n_prefix + (static_cast<long long>(t) * g.Hg + y) * g.Wg + x;
+}
+
+__device__ __forceinline__ int block_real_count(const Geo& g, int blk) {
+  if (blk < g.n_pre) return min(g.bs, g.n_prefix - blk * g.bs);
+  int vt, vh, vw;
+  video_block_extent(g, blk - g.n_pre, vt, vh, vw);
+  return vt * vh * vw;
+}
+
+template <int BS, bool POOL>
+__global__ void __launch_bounds__(kTileThreads) tile_kernel(Geo g, int H, const uint4* __restrict__ x,
+                                                            uint4* __restrict__ xt, float* __restrict__ pooled) {
+  extern __shared__ __align__(16) uint4 stage[];  // [BS][16] when POOL
+  const int blk = blockIdx.x;
+  const int bh = blockIdx.y;
+  const int b = bh / H, h = bh - b * H;
+  const int chunk = threadIdx.x & (kRowChunks - 1);
+  const int row0 = threadIdx.x >> 4;  // 0..15
+  constexpr int kIters = BS / 16;
+
+  uint4 v[kIters];
+#pragma unroll
+  for (int i = 0; i < kIters; ++i) {
+    const int slot = row0 + 16 * i;
+    const long long s = token_of_slot(g, blk, slot);
+    if (s >= 0) {
+      const long long src = ((static_cast<long long>(b) * g.S + s) * H + h) * kRowChunks + chunk;
+      v[i] = __ldcs(x + src);
+    } else {
+      v[i] = make_uint4(0, 0, 0, 0);
+    }
+  }
+  const long long dst0 = (static_cast<long long>(bh) * g.Sp + static_cast<long long>(blk) * BS) * kRowChunks;
+#pragma unroll
+  for (int i = 0; i < kIters; ++i) {
+    const int slot = row0 + 16 * i;
+    xt[dst0 + slot * kRowChunks + chunk] = v[i];
+    if (POOL) stage[slot * kRowChunks + chunk] = v[i];
+  }
+  if (POOL) {
+    __syncthreads();
+    if (threadIdx.x < 128) {
+      const int d = threadIdx.x;
+      const __nv_bfloat16* st = reinterpret_cast<const __nv_bfloat16*>(stage);
+      float s = 0.0f;
+#pragma unroll 8
+      for (int slot = 0; slot < BS; ++slot) s = __fadd_rn(s, __bfloat162float(st[slot * 128 + d]));
+      const float mean = __fdiv_rn(s, static_cast<float>(block_real_count(g, blk)));
+      pooled[(static_cast<long long>(bh) * g.NB + blk) * 128 + d] = mean;
+    }
+  }
+}
+
+template <int BS>
+__global__ void __launch_bounds__(kTileThreads) untile_kernel(Geo g, int H, const uint4* __restrict__ xt,
+                                                              uint4* __restrict__ x) {
+  const int blk = blockIdx.x;
+  const int bh = blockIdx.y;
+  const int b = bh / H, h = bh - b * H;
+  const int chunk = threadIdx.x & (kRowChunks - 1);
+  const int row0 = threadIdx.x >> 4;
+  constexpr int kIters = BS / 16;
+  const long long src0 = (static_cast<long long>(bh) * g.Sp + static_cast<long long>(blk) * BS) * kRowChunks;
+  uint4 v[kIters];
+#pragma unroll
+  for (int i = 0; i < kIters; ++i) v[i] = __ldcs(xt + src0 + (row0 + 16 * i) * kRowChunks + chunk);
+#pragma unroll
+  for (int i = 0; i < kIters; ++i) {
+    const long long s = token_of_slot(g, blk, row0 + 16 * i);
+    if (s >= 0) x[((static_cast<long long>(b) * g.S + s) * H + h) * kRowChunks + chunk] = v[i];
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_tile(const Geo& g, int B, int H, const uint16_t* x, uint16_t* xt, float* pooled,
+                        cudaStream_t stream) {
+  dim3 grid(g.NB, B * H);
+  const uint4* xi = reinterpret_cast<const uint4*>(x);
+  uint4* xo = reinterpret_cast<uint4*>(xt);
+  if (g.bs == 256) {
+    if (pooled) {
+      const int smem = 256 * 256;
+      cudaError_t e = cudaFuncSetAttribute(tile_kernel<256, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return e;
+      tile_kernel<256, true><<<grid, kTileThreads, smem, stream>>>(g, H, xi, xo, pooled);
+    } else {
+      tile_kernel<256, false><<<grid, kTileThreads, 0, stream>>>(g, H, xi, xo, nullptr);
+    }
+  } else {
+    if (pooled) {
+      tile_kernel<64, true><<<grid, kTileThreads, 64 * 256, stream>>>(g, H, xi, xo, pooled);
+    } else {
+      tile_kernel<64, false><<<grid, kTileThreads, 0, stream>>>(g, H, xi, xo, nullptr);
+    }
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_untile(const Geo& g, int B, int H, const uint16_t* xt, uint16_t* x, cudaStream_t stream) {
+  dim3 grid(g.NB, B * H);
+  const uint4* xi = reinterpret_cast<const uint4*>(xt);
+  uint4* xo = reinterpret_cast<uint4*>(x);
+  if (g.bs == 256)
+    untile_kernel<256><<<grid, kTileThreads, 0, stream>>>(g, H, xi, xo);
+  else
+    untile_kernel<64><<<grid, kTileThreads, 0, stream>>>(g, H, xi, xo);
+  return cudaGetLastError();
+}
+
+}  // namespace vsa

@@ -1,0 +1,163 @@
+/*
+ * vsa.h -- C ABI of the Video Sparse Attention (VSA) forward path on B200.
+ *
+ * The method ("FastVideo VSA", vLLM-Omni user guide, introduction): the
+ * post-patch latent grid of a video DiT is cut into spatiotemporal blocks;
+ * every query block scores all key/value blocks on block-pooled Q and K,
+ * keeps its top-k, and runs attention against the tokens of those blocks
+ * only.  The forward path is four calls, in stream order:
+ *
+ *   vsa_tile(q), vsa_tile(k) (with pooled means), vsa_tile(v)
+ *   vsa_coarse_topk(qbar, kbar)          -> q2k_idx, q2k_num
+ *      (or vsa_map_to_index(bool map)    -> q2k_idx, q2k_num)
+ *   vsa_sparse_attn_fwd(q, k, v, index)  -> o, lse      (tiled layout)
+ *   vsa_untile(o)
+ *
+ * Conventions shared by every call
+ *  - bf16 tensors are passed as pointers to their raw 16-bit patterns.
+ *  - Untiled layout: [B, S, H, D] (token-major, heads inside), S = n_prefix +
+ *    T*Hg*Wg tokens, video tokens in (t, y, x) raster order after the prefix.
+ *  - Tiled layout: [B, H, Sp, D], Sp = NB * block_tokens.  Block b holds rows
+ *    [b*bs, (b+1)*bs).  Prefix tiles come first and hold the prefix tokens in
+ *    order.  Video blocks follow in raster order over (bT, bH, bW); inside a
+ *    block, token (lt, lh, lw) sits at slot (lt*bh + lh)*bw + lw.  Slots whose
+ *    grid coordinates fall outside (T, Hg, Wg) are padding and hold zeros.
+ *  - D must be 128 (the only head size the B200 kernels are built for).
+ *  - Every device pointer must be 16-byte aligned and every buffer is owned
+ *    by the caller; the library allocates no device memory in any call.
+ *  - Every call is asynchronous on `stream` and returns an int status.  A
+ *    non-zero return means nothing was launched.  Errors found on the device
+ *    (bad block ids, counts above max_k, a pipeline wait that ran out) are
+ *    recorded in a per-device status word read by vsa_get_status().
+ *  - Nothing falls back: unsupported input is an error, never rerouted.
+ */
+#ifndef VSA_H
+#define VSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define VSA_API __attribute__((visibility("default")))
+#else
+#define VSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st *vsa_stream_t;
+
+/* Opaque, host-only description of one video geometry. */
+typedef struct vsa_plan *vsa_plan_t;
+
+enum vsa_status {
+    VSA_OK = 0,
+    VSA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, non-positive size */
+    VSA_ERR_UNSUPPORTED = 2,   /* D != 128, block tokens not 64 or 256, odd tile count, not sm_100 */
+    VSA_ERR_TOPK = 3,          /* topk <= 0 or topk > num_blocks */
+    VSA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
+    VSA_ERR_BAD_INDEX = 5,     /* device: a block id outside [0, NB) or a count outside [0, max_k] */
+    VSA_ERR_TIMEOUT = 6,       /* device: a pipeline wait ran out; the kernel stopped early */
+    VSA_ERR_NO_DEVICE = 7      /* no usable CUDA device */
+};
+
+/*
+ * Geometry ("FastVideo VSA", section "Choose top-k": blocks of (4, 8, 8)
+ * tokens over the zero-padded latent grid; num_blocks = ceil(T/bt) *
+ * ceil(Hg/bh) * ceil(Wg/bw), e.g. (31, 22, 40) -> 120).
+ *
+ * vsa_plan_create_prefix adds n_prefix tokens ahead of the grid, tiled in
+ * order into ceil(n_prefix / bs) contiguous tiles (the tile-64 layout of
+ * the FastVideo commit log, examples/inference/basic/README.md).
+ * Block sizes: bt*bh*bw must be 64 or 256 and each of bt, bh, bw a power of
+ * two.  Returns VSA_ERR_INVALID_ARG / VSA_ERR_UNSUPPORTED on bad sizes.
+ * The plan is host memory owned by the caller; free it with vsa_plan_destroy.
+ */
+VSA_API int vsa_plan_create(int T, int Hg, int Wg, int bt, int bh, int bw, vsa_plan_t *out);
+VSA_API int vsa_plan_create_prefix(int n_prefix, int T, int Hg, int Wg, int bt, int bh, int bw,
+                           vsa_plan_t *out);
+VSA_API void vsa_plan_destroy(vsa_plan_t plan);
+
+/* Sizes of a plan: block count NB, real tokens S, padded tokens Sp, tokens per block. */
+VSA_API int vsa_plan_sizes(vsa_plan_t plan, int *num_blocks, int64_t *seq_len, int64_t *padded_len,
+                   int *block_tokens);
+
+/*
+ * The routing fields the page logs ("FastVideo VSA", section "Choose
+ * top-k"): seq_len, dit_seq_shape, block_size, num_blocks, topk and
+ * keep_ratio, written as one NUL-terminated line into buf (at most n bytes).
+ */
+VSA_API int vsa_plan_describe(vsa_plan_t plan, int topk, char *buf, size_t n);
+
+/*
+ * Tile: x [B,S,H,D] bf16 -> x_tiled [B,H,Sp,D] bf16 (padding zero-filled).
+ * If pooled is not NULL it also receives the per-block mean of the real
+ * tokens, [B,H,NB,D] fp32, summed in slot order in fp32 and divided once by
+ * the real-token count (the block summary the coarse stage scores; "FastVideo
+ * VSA", introduction).  x and x_tiled must not overlap.
+ */
+VSA_API int vsa_tile(vsa_plan_t plan, const uint16_t *x, uint16_t *x_tiled, float *pooled,
+             int B, int H, int D, vsa_stream_t stream);
+
+/* Untile: x_tiled [B,H,Sp,D] -> x [B,S,H,D]; padded rows are dropped. */
+VSA_API int vsa_untile(vsa_plan_t plan, const uint16_t *x_tiled, uint16_t *x, int B, int H, int D,
+               vsa_stream_t stream);
+
+/*
+ * Coarse stage ("FastVideo VSA", introduction and section "Choose top-k"):
+ * score[i][j] = qbar[i] . kbar[j] (fp32, one fused multiply-add per channel
+ * in channel order) for every (b, h); every query block i keeps the topk
+ * largest scores, ties to the lower block index, written to
+ * q2k_idx [B,H,NB,topk] in ascending block order; q2k_num [B,H,NB] = topk.
+ * qbar, kbar: [B,H,NB,D] fp32 as produced by vsa_tile.  0 < topk <= NB,
+ * else VSA_ERR_TOPK.
+ */
+VSA_API int vsa_coarse_topk(vsa_plan_t plan, const float *qbar, const float *kbar, int B, int H, int D,
+                    int topk, int32_t *q2k_idx, int32_t *q2k_num, vsa_stream_t stream);
+
+/*
+ * Bool block map -> index (FastVideo commit log: map_to_index):
+ * map [B,H,NQ,NK] (one byte per entry, non-zero = selected) ->
+ * q2k_idx [B,H,NQ,NK] (selected ids ascending, then -1), q2k_num [B,H,NQ]
+ * (0 allowed).
+ */
+VSA_API int vsa_map_to_index(const uint8_t *map, int B, int H, int NQ, int NK, int32_t *q2k_idx,
+                     int32_t *q2k_num, vsa_stream_t stream);
+
+/*
+ * Fine stage ("FastVideo VSA", introduction and section "Verify routing and
+ * fallback"; FastVideo commit log for non-uniform and zero-count rows):
+ * for every query token i of block r, attention over the real tokens of
+ * blocks q2k_idx[r, 0 .. q2k_num[r]-1] with scale D^-1/2, non-causal.
+ *   q, k, v  : tiled [B,H,Sp,D] bf16
+ *   q2k_idx  : [B,H,NB,max_k] int32;  q2k_num: [B,H,NB] int32
+ *   o        : tiled [B,H,Sp,D] bf16; lse: [B,H,Sp] fp32, natural log of
+ *              sum_j exp(scale q.k_j).  A row of count 0 gives o = 0 and
+ *              lse = -inf.  Padded query rows are computed like any other.
+ * bf16 products, fp32 accumulation and fp32 online softmax.
+ * Block ids outside [0, NB) are skipped and counts outside [0, max_k] are
+ * clamped; both set VSA_ERR_BAD_INDEX in the device status word.
+ * For 64-token blocks the block count must be even.
+ */
+VSA_API int vsa_sparse_attn_fwd(vsa_plan_t plan, const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                        const int32_t *q2k_idx, const int32_t *q2k_num, int max_k,
+                        int B, int H, int D, uint16_t *o, float *lse, vsa_stream_t stream);
+
+/*
+ * Synchronise `stream`, then read and clear the status word of the current
+ * device: *device_status receives VSA_OK or the first device-detected error
+ * (VSA_ERR_BAD_INDEX, VSA_ERR_TIMEOUT) since the last read.
+ */
+VSA_API int vsa_get_status(vsa_stream_t stream, int *device_status);
+
+/* Static text for a status code. */
+VSA_API const char *vsa_strerror(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VSA_H */

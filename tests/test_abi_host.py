@@ -1,0 +1,143 @@
+"""Host-side checks of the C ABI (no kernel is launched by any test here).
+
+Every call below either fails argument validation -- which returns before
+any CUDA call -- or only touches host state (plans, strings).
+"""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import block_sparse_video_gather_b200 as vsa
+from block_sparse_video_gather_b200 import build as vsa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "vsa.h")
+FAKE = 0x100000  # an aligned, non-null address; never dereferenced (validation fails first)
+
+
+@pytest.fixture(scope="module")
+def L():
+    vsa_build.build()
+    return vsa.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(vsa_[a-z_]+)\s*\(", text)))
+
+
+def test_header_and_binding_agree():
+    assert declared_functions() == sorted(vsa.SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_library_exports_nothing_else(L):
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", vsa.LIB_PATH], capture_output=True, text=True).stdout
+    exported = sorted({ln.split()[-1] for ln in out.splitlines() if " T " in ln and ln.split()[-1].startswith("vsa_")})
+    assert exported == declared_functions()
+
+
+def test_strerror(L):
+    for code in range(8):
+        assert L.vsa_strerror(code)
+    assert b"unknown" in L.vsa_strerror(99)
+
+
+def _plan(*args):
+    p = vsa.Plan(*args)
+    return p
+
+
+def test_plan_sizes_match_oracle_geometry():
+    import oracle
+    from block_sparse_video_gather_b200 import workloads
+    for wl in workloads.WORKLOADS.values():
+        p = vsa.Plan.of(wl)
+        g = oracle.geometry_of(wl)
+        assert (p.NB, p.S, p.Sp, p.bs) == (g.NB, g.S, g.Sp, g.bs)
+
+
+def test_describe_reproduces_route_log_fields():
+    """Fields of the routing log printed on "FastVideo VSA", section "Choose top-k"."""
+    gold = {}
+    for line in open(os.path.join(ROOT, "tests", "golden", "fastwan_route.txt")):
+        if line.strip() and not line.startswith("#"):
+            k, *v = line.split()
+            gold[k] = v
+    p = vsa.Plan(31, 22, 40)
+    s = p.describe(64)
+    assert f"seq_len={gold['seq_len'][0]}" in s
+    assert "dit_seq_shape=({}, {}, {})".format(*gold["dit_seq_shape"]) in s
+    assert "block_size=({}, {}, {})".format(*gold["block_size"]) in s
+    assert f"num_blocks={gold['num_blocks'][0]}" in s
+    assert f"topk={gold['topk'][0]}" in s
+    assert f"keep_ratio={gold['keep_ratio_percent'][0]}%" in s
+
+
+@pytest.mark.parametrize("args,code", [
+    ((0, 8, 8, 4, 8, 8), vsa.VSA_ERR_INVALID_ARG),
+    ((4, 8, 8, 0, 8, 8), vsa.VSA_ERR_INVALID_ARG),
+    ((4, 8, 8, 3, 8, 8), vsa.VSA_ERR_UNSUPPORTED),   # not a power of two
+    ((4, 8, 8, 4, 8, 4), vsa.VSA_ERR_UNSUPPORTED),   # 128 tokens per block
+    ((4, 8, 8, 1, 1, 64), vsa.VSA_ERR_UNSUPPORTED),  # bw > 32
+])
+def test_plan_rejects_bad_geometry(L, args, code):
+    h = ctypes.c_void_p()
+    assert L.vsa_plan_create(*args, ctypes.byref(h)) == code
+    assert not h.value
+
+
+def test_plan_rejects_null_out(L):
+    assert L.vsa_plan_create(4, 8, 8, 4, 8, 8, None) == vsa.VSA_ERR_INVALID_ARG
+
+
+def test_describe_rejects_bad_topk(L):
+    p = vsa.Plan(31, 22, 40)
+    buf = ctypes.create_string_buffer(256)
+    assert L.vsa_plan_describe(p.handle, 0, buf, 256) == vsa.VSA_ERR_TOPK
+    assert L.vsa_plan_describe(p.handle, 121, buf, 256) == vsa.VSA_ERR_TOPK
+
+
+def test_calls_reject_invalid_arguments(L):
+    p = vsa.Plan(8, 16, 16)
+    h = p.handle
+    F, M = ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE + 8)  # aligned / misaligned
+    # tile / untile
+    assert L.vsa_tile(None, F, F, None, 1, 2, 128, None) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_tile(h, None, F, None, 1, 2, 128, None) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_tile(h, M, F, None, 1, 2, 128, None) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_tile(h, F, F, M, 1, 2, 128, None) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_tile(h, F, F, None, 0, 2, 128, None) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_tile(h, F, F, None, 1, 2, 64, None) == vsa.VSA_ERR_UNSUPPORTED
+    assert L.vsa_untile(h, F, M, 1, 2, 128, None) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_untile(h, F, F, 1, 2, 96, None) == vsa.VSA_ERR_UNSUPPORTED
+    # coarse stage: topk must satisfy 0 < topk <= NB (NB = 8 here)
+    assert L.vsa_coarse_topk(h, F, F, 1, 2, 128, 0, F, F, None) == vsa.VSA_ERR_TOPK
+    assert L.vsa_coarse_topk(h, F, F, 1, 2, 128, 9, F, F, None) == vsa.VSA_ERR_TOPK
+    assert L.vsa_coarse_topk(h, F, M, 1, 2, 128, 4, F, F, None) == vsa.VSA_ERR_INVALID_ARG
+    # map compaction
+    assert L.vsa_map_to_index(None, 1, 1, 4, 4, F, F, None) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_map_to_index(F, 1, 1, 0, 4, F, F, None) == vsa.VSA_ERR_INVALID_ARG
+    # fine stage
+    assert L.vsa_sparse_attn_fwd(h, F, F, F, F, F, 0, 1, 2, 128, F, F, None) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_sparse_attn_fwd(h, F, F, M, F, F, 4, 1, 2, 128, F, F, None) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_sparse_attn_fwd(h, F, F, F, F, F, 4, 1, 2, 256, F, F, None) == vsa.VSA_ERR_UNSUPPORTED
+    odd = vsa.Plan(4, 4, 12, (4, 4, 4))  # 3 tiles of 64: the tile count must be even
+    assert L.vsa_sparse_attn_fwd(odd.handle, F, F, F, F, F, 4, 1, 2, 128, F, F, None) == vsa.VSA_ERR_UNSUPPORTED
+    assert L.vsa_get_status(None, None) == vsa.VSA_ERR_INVALID_ARG
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path")
+def test_valid_call_without_gpu_reports_no_device(L):
+    p = vsa.Plan(8, 16, 16)
+    F = ctypes.c_void_p(FAKE)
+    assert L.vsa_tile(p.handle, F, F, None, 1, 2, 128, None) == vsa.VSA_ERR_NO_DEVICE
