@@ -1,0 +1,393 @@
+"""Benchmark of the VSA forward path on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload fastwan] [--impl ours|reference]
+
+A step is one pass of the whole forward path over one batch of seeded
+synthetic input: tile(q), tile(k) with pooled means, tile(v), block scores +
+top-k, block-sparse attention, untile(o).  The metric is effective TFLOP/s
+over the selected blocks (4 * D * bs^2 FLOPs per selected block pair), with
+ms per step beside it.  ``value`` is timed with the inputs already in HBM;
+``e2e`` times the same call with pinned host inputs copied in and o copied
+back inside every step.
+
+Several GPUs run independent replicas of the same workload (the path has no
+exchange step); the time is the maximum over ranks and ``value`` counts the
+work of all ranks.  ``--impl reference`` times the CPU oracle (rank 0 only)
+on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_video_gather_b200 import workloads  # noqa: E402
+
+PROFILE = os.path.join(ROOT, "profiles", "attn_fwd_fastwan.md")
+ATTN_SOURCES = [os.path.join(ROOT, "block_sparse_video_gather_b200", "csrc", f)
+                for f in ("attn_fwd.cu", "common.cuh")]
+WORKLOAD_TEXT = {
+    "tiny": "tiny grid 8x16x16, B1 H2 D128, block 4x8x8, topk 4",
+    "fastwan": "FastWan2.2-TI2V-5B latent grid 31x22x40, B1 H24 D128, block 4x8x8, topk 64",
+    "wan81": "Wan2.1-1.3B 81-frame latent grid 21x30x52, B1 H12 D128, block 4x8x8, topk 32",
+    "long": "Wan2.1-1.3B 321-frame latent grid 81x30x52, B1 H12 D128, block 4x8x8, topk 59",
+}
+
+
+def selected_flops(wl, num: np.ndarray) -> float:
+    """4 * D * bs^2 per selected (query block, key block) pair, padding included."""
+    return 4.0 * wl.D * wl.block_tokens ** 2 * float(np.asarray(num, dtype=np.int64).sum())
+
+
+def uniform_flops(wl) -> float:
+    return 4.0 * wl.D * wl.block_tokens ** 2 * wl.B * wl.H * wl.num_blocks * wl.topk
+
+
+def attn_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ATTN_SOURCES:
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profile_traffic(workload: str):
+    """DRAM bytes per attention launch from the committed ncu summary, or None when
+    the summary is absent, for another workload, or older than the kernel source."""
+    if not os.path.exists(PROFILE):
+        return None
+    text = open(PROFILE).read()
+    m_src = re.search(r"source_hash:\s*([0-9a-f]+)", text)
+    m_wl = re.search(r"bench_workload:\s*(\w+)", text)
+    m_b = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not (m_src and m_wl and m_b) or m_src.group(1) != attn_source_hash() or m_wl.group(1) != workload:
+        return None
+    return float(m_b.group(1))
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return d.get("bf16_tflops"), d.get("bf16_tflops_sustained"), d.get("hbm_gbs"), "measured"
+    return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in out.splitlines():
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[3:7]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}: launch N>1 with torch.distributed.run")
+    return world, rank, local
+
+
+def run_reference(args, wl, world, rank):
+    """The CPU oracle on a bounded sample of the workload (rank 0 only)."""
+    if rank != 0:
+        return
+    import oracle
+    g = oracle.geometry_of(wl)
+    inp = workloads.make_inputs(wl)
+    total_rows = wl.B * wl.H * g.Sp
+    rng = np.random.default_rng(1)
+    sample_rows = min(total_rows, args.ref_rows)
+
+    def step():
+        t0 = time.perf_counter()
+        qt, kt, vt = (oracle.tile(g, inp[n]) for n in ("q", "k", "v"))
+        qbar, kbar = oracle.pool(g, qt), oracle.pool(g, kt)
+        idx, num = oracle.topk(oracle.score(qbar, kbar), wl.topk)
+        t1 = time.perf_counter()
+        rows = np.sort(rng.choice(total_rows, size=sample_rows, replace=False))
+        o, _ = oracle.attn_rows(g, qt, kt, vt, idx, num, rows)
+        t2 = time.perf_counter()
+        ot = np.zeros((wl.B, wl.H, g.Sp, wl.D), dtype=np.uint16)
+        oracle.untile(g, ot)
+        t3 = time.perf_counter()
+        return (t1 - t0) + (t2 - t1) * total_rows / sample_rows + (t3 - t2), num
+
+    for _ in range(args.warmup):
+        step()
+    times = []
+    for _ in range(args.steps):
+        t, num = step()
+        times.append(t)
+    est = float(np.mean(times))
+    flops = selected_flops(wl, num)
+    value = flops / est / 1e12
+    cores = oracle.max_threads()
+    sample = (f"per step: oracle tile/pool/score/top-k/untile over the whole workload, attention on "
+              f"{sample_rows} of {total_rows} query rows drawn at random, scaled to all rows")
+    line = {
+        "impl": "reference", "metric": "VSA sparse-attn fwd effective TFLOP/s (selected blocks) on 1 B200",
+        "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": est * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic (seeded)",
+        "config": {"workload": WORKLOAD_TEXT.get(args.workload, args.workload)},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline_sample(wl, seconds_hint=20.0):
+    """Oracle throughput on a bounded sample of the workload (about 10-30 s of CPU work)."""
+    import oracle
+    g = oracle.geometry_of(wl)
+    inp = workloads.make_inputs(wl)
+    t0 = time.perf_counter()
+    qt, kt, vt = (oracle.tile(g, inp[n]) for n in ("q", "k", "v"))
+    qbar, kbar = oracle.pool(g, qt), oracle.pool(g, kt)
+    idx, num = oracle.topk(oracle.score(qbar, kbar), wl.topk)
+    oracle.untile(g, qt)
+    t_front = time.perf_counter() - t0
+    total_rows = wl.B * wl.H * g.Sp
+    rng = np.random.default_rng(2)
+    n = 256
+    t_attn, done = 0.0, 0
+    while t_attn < seconds_hint * 0.5 and done < total_rows:
+        rows = np.sort(rng.choice(total_rows, size=min(n, total_rows), replace=False))
+        t1 = time.perf_counter()
+        oracle.attn_rows(g, qt, kt, vt, idx, num, rows)
+        t_attn += time.perf_counter() - t1
+        done += len(rows)
+        n *= 2
+    est = t_front + t_attn * total_rows / done
+    value = selected_flops(wl, num) / est / 1e12
+    return {"value": value, "unit": "TFLOP/s", "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": (f"oracle tile+pool+score+top-k+untile over the whole workload ({t_front:.1f} s) and "
+                       f"attention on {done} of {total_rows} query rows ({t_attn:.1f} s), scaled to all rows; "
+                       f"estimated {est:.0f} s per step")}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="fastwan", choices=list(WORKLOAD_TEXT))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ref-rows", type=int, default=2048, help="query rows per reference step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be at least 3")
+    wl = workloads.WORKLOADS[args.workload]
+    world, rank, local = dist_setup(args)
+
+    if args.impl == "reference":
+        run_reference(args, wl, world, rank)
+        return
+
+    import torch
+    import block_sparse_video_gather_b200 as vsa
+    from block_sparse_video_gather_b200 import build as vsa_build
+
+    torch.cuda.set_device(local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+        pg = dist
+    if rank == 0:
+        vsa_build.build()
+    if pg:
+        pg.barrier()
+    vsa.lib()
+
+    inp = workloads.make_inputs(wl)
+    host = {n: torch.from_numpy(inp[n].view(np.int16)).view(torch.bfloat16).pin_memory() for n in ("q", "k", "v")}
+    dev = {n: host[n].to("cuda", non_blocking=False) for n in host}
+    plan = vsa.Plan.of(wl)
+    fwd = vsa.Forward(plan, wl.B, wl.H, wl.topk)
+    o_host = torch.empty(fwd.o.shape, dtype=torch.bfloat16).pin_memory()
+
+    stream = torch.cuda.current_stream()
+    attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+    front_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+
+    def step(i=None):
+        p = fwd.plan
+        if i is not None:
+            front_ev[i].record(stream)
+        vsa.tile(p, dev["q"], pooled=True, out=fwd.qt, pooled_out=fwd.qbar)
+        vsa.tile(p, dev["k"], pooled=True, out=fwd.kt, pooled_out=fwd.kbar)
+        vsa.tile(p, dev["v"], out=fwd.vt)
+        vsa.coarse_topk(p, fwd.qbar, fwd.kbar, wl.topk, idx_out=fwd.idx, num_out=fwd.num)
+        if i is not None:
+            attn_ev[i][0].record(stream)
+        vsa.sparse_attn_fwd(p, fwd.qt, fwd.kt, fwd.vt, fwd.idx, fwd.num, o_out=fwd.ot, lse_out=fwd.lse)
+        if i is not None:
+            attn_ev[i][1].record(stream)
+        vsa.untile(p, fwd.ot, out=fwd.o)
+
+    def sync_all():
+        torch.cuda.synchronize()
+        if pg:
+            pg.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(x: float) -> float:
+        if not pg:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert vsa.get_status() == vsa.VSA_OK
+    flops = selected_flops(wl, fwd.num.cpu().numpy())
+
+    props = torch.cuda.get_device_properties(local)
+    gpu_id = str(getattr(props, "uuid", local))
+    if gpu_id and not gpu_id.startswith("GPU-") and len(gpu_id) >= 32:
+        gpu_id = "GPU-" + gpu_id
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    time.sleep(0.3)
+
+    # ---- device-resident timing
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sync_all()
+    t0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    t1.record(stream)
+    sync_all()
+    clocks = sampler.stop()
+    elapsed = max_over_ranks(t0.elapsed_time(t1) / 1e3)
+    attn_s = [a.elapsed_time(b) / 1e3 for a, b in attn_ev]
+    front_s = [f.elapsed_time(a[0]) / 1e3 for f, a in zip(front_ev, attn_ev)]
+    attn_avg = max_over_ranks(float(np.mean(attn_s)))
+    assert vsa.get_status() == vsa.VSA_OK
+
+    # ---- end to end through the public API with pinned host buffers
+    for _ in range(3):
+        for n in dev:
+            dev[n].copy_(host[n], non_blocking=True)
+        fwd(dev["q"], dev["k"], dev["v"])
+        o_host.copy_(fwd.o, non_blocking=True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sync_all()
+    e0.record(stream)
+    for _ in range(args.steps):
+        for n in dev:
+            dev[n].copy_(host[n], non_blocking=True)
+        fwd(dev["q"], dev["k"], dev["v"])
+        o_host.copy_(fwd.o, non_blocking=True)
+    e1.record(stream)
+    sync_all()
+    e2e_elapsed = max_over_ranks(e0.elapsed_time(e1) / 1e3)
+    assert vsa.get_status() == vsa.VSA_OK
+    h2d = sum(host[n].numel() * 2 for n in host)
+    d2h = o_host.numel() * 2
+
+    if rank == 0:
+        burst, sustained, hbm, peak_kind = measured_peaks()
+        peak = burst
+        achieved = flops / attn_avg / 1e12
+        traffic = profile_traffic(args.workload)
+        line = {
+            "metric": "VSA sparse-attn fwd effective TFLOP/s (selected blocks) on 1 B200",
+            "value": world * flops * args.steps / elapsed / 1e12,
+            "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": elapsed / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded; the recipe in block_sparse_video_gather_b200/workloads.py)",
+            "config": {
+                "workload": WORKLOAD_TEXT[args.workload],
+                "B": wl.B, "H": wl.H, "D": wl.D, "grid": [wl.T, wl.Hg, wl.Wg], "block": list(wl.block),
+                "num_blocks": wl.num_blocks, "topk": wl.topk, "selected_block_tflop_per_step": flops / 1e12,
+                "attn_ms": attn_avg * 1e3, "front_ms": float(np.mean(front_s)) * 1e3,
+                "l2": "inputs larger than L2: q/k/v %.0f MB and tiled q/k/v %.0f MB per step" % (
+                    h2d / 1e6, 3 * fwd.qt.numel() * 2 / 1e6),
+                "parallelism": f"replicas x{world}",
+            },
+            "roofline": {
+                "bound": "tensor", "kernel": "attn_fwd_kernel", "achieved": achieved,
+                "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "peak_source": f"{peak_kind} bf16 burst (MEASURED_PEAKS.json)" if peak_kind == "measured"
+                else "fallback 1.59 PFLOP/s",
+                "traffic": traffic,
+            },
+            "clocks": clocks,
+            "e2e": {"value": world * flops * args.steps / e2e_elapsed / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_elapsed / args.steps * 1e3},
+            "gpu_launches": args.steps * vsa.Forward.launches_per_call,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline_sample(wl)
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

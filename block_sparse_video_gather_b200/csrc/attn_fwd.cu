@@ -57,9 +57,21 @@ constexpr uint32_t kSmemV = kSmemK + kStages * kTileBytes;
 constexpr uint32_t kSmemBar = kSmemV + kStages * kTileBytes;
 constexpr uint32_t kSmemTotal = kSmemBar + 256 + 1024;  // barriers + 1 KB alignment slack
 constexpr uint64_t kTimeoutNs = 2000000000ull;          // 2 s per wait
+// Register split: launched at 168 per thread (384 x 168 = 64512); warpgroup 0
+// (producer, MMA issuer, two idle warps) gives back down to 104 and the two
+// softmax warpgroups take 200 each: 128 x 104 + 256 x 200 = 64512.
+constexpr int kRegsLaunch = 168, kRegsLow = 104, kRegsHigh = 200;
+static_assert(kThreads * kRegsLaunch == 128 * kRegsLow + 256 * kRegsHigh, "register split must match the launch");
 
 constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, 0, 0);   // Q (K-major) x K (K-major)
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, 0, 1);  // P (TMEM) x V (MN-major)
+
+constexpr int kTileFull = 0, kTilePartial = 1, kTileEmpty = 2;
+// Exponential pairs, out of every 8, evaluated by polynomial on the FMA pipe.
+#ifndef VSA_POLY_PAIRS
+#define VSA_POLY_PAIRS 0
+#endif
+constexpr int kPolyPairsOf8 = VSA_POLY_PAIRS;
 
 struct Barriers {
   uint64_t q_full, q_empty;
@@ -101,29 +113,31 @@ __device__ __forceinline__ int item_block_id(const Params& p, int item, int j) {
 }
 
 // Validity bits of the 128 key columns of tile `half` of block kb (bit c of
-// word c/32 set = slot half*128 + c holds a real token).  Returns true when
-// every column is real.
-__device__ __forceinline__ bool key_tile_mask(const Geo& g, int kb, int half, uint32_t (&w)[4]) {
+// word c/32 set = slot half*128 + c holds a real token).  Returns kTileFull
+// when every column is real, kTileEmpty when none is, else kTilePartial.
+__device__ __forceinline__ int key_tile_mask(const Geo& g, int kb, int half, uint32_t (&w)[4]) {
   if (kb < 0) {
     w[0] = w[1] = w[2] = w[3] = 0u;
-    return false;
+    return kTileEmpty;
   }
   const int first = half * 128;
   if (kb < g.n_pre) {
     const int lim = g.n_prefix - kb * g.bs - first;  // real columns of this tile
-    if (lim >= 128) return true;
+    if (lim >= 128) return kTileFull;
+    if (lim <= 0) return kTileEmpty;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int n = min(max(lim - 32 * i, 0), 32);
       w[i] = n >= 32 ? 0xffffffffu : ((1u << n) - 1u);
     }
-    return false;
+    return kTilePartial;
   }
   int vt, vh, vw;
   video_block_extent(g, kb - g.n_pre, vt, vh, vw);
-  if (vt == g.bt && vh == g.bh && vw == g.bw) return true;
+  if (vt == g.bt && vh == g.bh && vw == g.bw) return kTileFull;
   const uint32_t rowbits = vw >= 32 ? 0xffffffffu : ((1u << vw) - 1u);
   const int rows_per_word = 32 >> g.lbw;
+  uint32_t any = 0;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     uint32_t word = 0;
@@ -135,8 +149,34 @@ __device__ __forceinline__ bool key_tile_mask(const Geo& g, int kb, int half, ui
       if (lt < vt && lh < vh) word |= rowbits << (r << g.lbw);
     }
     w[i] = word;
+    any |= word;
   }
-  return false;
+  return any ? kTilePartial : kTileEmpty;
+}
+
+// Set the masked columns of one row of S to -inf.  The mask is the same for
+// every thread, so the branches are uniform; columns are handled four at a
+// time whenever each group of four is all-real or all-padded.
+__device__ __forceinline__ void apply_key_mask(uint32_t (&sv)[128], const uint32_t (&mw)[4]) {
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    const uint32_t m = mw[w];
+    if (m == 0xffffffffu) continue;
+    // a nibble is mixed if not all four of its bits agree
+    const uint32_t x = (m ^ (m >> 1)) | (m ^ (m >> 2)) | (m ^ (m >> 3));
+    if ((x & 0x11111111u) == 0u) {
+#pragma unroll
+      for (int gi = 0; gi < 8; ++gi)
+        if (!((m >> (4 * gi)) & 1u)) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) sv[32 * w + 4 * gi + c] = 0xff800000u;
+        }
+    } else {
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        if (!((m >> c) & 1u)) sv[32 * w + c] = 0xff800000u;
+    }
+  }
 }
 
 // Warp-uniform bounded wait: all lanes wait, then agree.
@@ -190,6 +230,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
+  if (warp < 4) {
+  regs_dec<kRegsLow>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -253,24 +295,30 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t qaddr = smem_u32(sQ), kaddr = smem_u32(sK), vaddr = smem_u32(sV);
+      // Descriptors are built once; each MMA only adds a constant to the
+      // start-address field (smem addresses stay below 2^18, so the 14-bit
+      // field never carries).  A lean issue loop keeps the tensor core fed:
+      // rebuilding descriptors per instruction made this thread the bottleneck.
+      const uint64_t dq0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t dk0 = sdesc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t dv0 = sdesc_sw128(smem_u32(sV), kHalfBytes, 1024);
+      constexpr uint64_t kTileDesc = kTileBytes >> 4;
       int kit = 0, vit = 0, qit = 0, tiles = 0, items = 0;
       bool ok = true;
       auto issue_s = [&](int i, int sk) {
+        const uint32_t d = tmem + i * 128;
+        const uint64_t a = dq0 + i * kTileDesc, b = dk0 + sk * kTileDesc;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-          const uint64_t a = sdesc_sw128(qaddr + i * kTileBytes + off, 16, 1024);
-          const uint64_t b = sdesc_sw128(kaddr + sk * kTileBytes + off, 16, 1024);
-          mma_ss(tmem + i * 128, a, b, kIdescS, kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+          mma_ss(d, a + off, b + off, kIdescS, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int i, int sv, bool acc) {
+        const uint32_t d = tmem + 256 + i * 128, pa = tmem + i * 128;
+        const uint64_t b = dv0 + sv * kTileDesc;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t b = sdesc_sw128(vaddr + sv * kTileBytes + kk * 2048, kHalfBytes, 1024);
-          mma_ts(tmem + 256 + i * 128, tmem + i * 128 + kk * 8, b, kIdescPV, (acc || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < 8; ++kk) mma_ts(d, pa + kk * 8, b + kk * (2048 >> 4), kIdescPV, (acc || kk > 0) ? 1u : 0u);
       };
       for (int item = blockIdx.x; item < total_items && ok; item += gridDim.x) {
         const int nb = item_blocks(p, item, true);
@@ -329,7 +377,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(&bars->drain);
       mbar_wait_drain(&bars->drain, 0, kTimeoutNs);
     }
-  } else if (warp >= 4) {
+  }
+  } else {
+    regs_inc<kRegsHigh>();
     // ------------------------------------------------------------ softmax + epilogue
     const int wg = (warp - 4) >> 2;  // Q tile
     const int quarter = warp & 3;    // TMEM lane quarter of this warp
@@ -357,37 +407,79 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int kb = item_block_id(p, item, t >> 1);
         if (kb < 0 && wg == 0 && r == 0) atomicCAS(p.status, 0u, (unsigned)VSA_ERR_BAD_INDEX);
         uint32_t mw[4];
-        const bool full = key_tile_mask(g, kb, t & 1, mw);
+        const int mstate = key_tile_mask(g, kb, t & 1, mw);
         if (!(ok = warp_wait(&bars->s_full[wg], tiles & 1, bars, p.status))) break;
         tc_fence_after();
-        uint32_t sv[128];
-        tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-        tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
-        tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
-        tmem_wait_ld();
-        if (!full) {
-#pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (!((mw[c >> 5] >> (c & 31)) & 1u)) sv[c] = 0xff800000u;  // -inf
-        }
-        float mx = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(sv[c]));
-        const float mt = mx * sl2;
-        const bool grow = mt > m_used + 8.0f;  // false while the tile is fully masked
-        const bool rescale = grow && t > 0 && m_used != -INFINITY;
-        const float alpha = rescale ? ex2_approx(m_used - mt) : 1.0f;
-        if (grow) m_used = mt;
-        const float msub = (m_used == -INFINITY) ? 0.0f : m_used;
         uint32_t pk[64];
-        float lsum = 0.0f;
+        float lsum = 0.0f, alpha = 1.0f;
+        bool rescale = false;
+        if (mstate == kTileEmpty) {
+          // no real key: the numerators are all zero and the maximum does not move
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * j]), sl2, -msub));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * j + 1]), sl2, -msub));
-          lsum += p0 + p1;
-          pk[j] = pack_bf16x2(p0, p1);
+          for (int j = 0; j < 64; ++j) pk[j] = 0u;
+        } else {
+          uint32_t sv[128];
+          tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+          tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+          tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
+          tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
+          tmem_wait_ld();
+          if (mstate == kTilePartial) apply_key_mask(sv, mw);
+          float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < 128; c += 8) {
+            a0 = max3f(a0, __uint_as_float(sv[c + 0]), __uint_as_float(sv[c + 1]));
+            a1 = max3f(a1, __uint_as_float(sv[c + 2]), __uint_as_float(sv[c + 3]));
+            a2 = max3f(a2, __uint_as_float(sv[c + 4]), __uint_as_float(sv[c + 5]));
+            a3 = max3f(a3, __uint_as_float(sv[c + 6]), __uint_as_float(sv[c + 7]));
+          }
+          const float mt = max3f(a0, a1, fmaxf(a2, a3)) * sl2;
+          const bool grow = mt > m_used + 8.0f;
+          rescale = grow && t > 0 && m_used != -INFINITY;
+          alpha = rescale ? ex2_approx(m_used - mt) : 1.0f;
+          if (grow) m_used = mt;
+          const float msub = (m_used == -INFINITY) ? 0.0f : m_used;
+          const uint64_t c2 = f2pack(sl2, sl2), nm2 = f2pack(-msub, -msub);
+          uint64_t acc0 = 0, acc1 = 0, acc2 = 0, acc3 = 0;
+#pragma unroll
+          for (int j = 0; j < 64; ++j) {
+            const uint64_t x = fma2(u2pack(sv[2 * j], sv[2 * j + 1]), c2, nm2);
+            uint64_t pp;
+#ifdef VSA_EXP_BF16X2
+            {
+              float xa, xb;
+              f2unpack(x, xa, xb);
+              const uint32_t e = ex2_bf16x2(pack_bf16x2(xa, xb));
+              pk[j] = e;
+              pp = u2pack(e << 16, e & 0xffff0000u);
+            }
+#else
+            if ((j & 7) < kPolyPairsOf8) {
+              pp = exp2_poly2(x);
+            } else {
+              float xa, xb;
+              f2unpack(x, xa, xb);
+              pp = f2pack(ex2_approx(xa), ex2_approx(xb));
+            }
+            {
+              float p0, p1;
+              f2unpack(pp, p0, p1);
+              pk[j] = pack_bf16x2(p0, p1);
+            }
+#endif
+            switch (j & 3) {
+              case 0: acc0 = add2(acc0, pp); break;
+              case 1: acc1 = add2(acc1, pp); break;
+              case 2: acc2 = add2(acc2, pp); break;
+              default: acc3 = add2(acc3, pp); break;
+            }
+          }
+          float s0, s1, s2, s3, s4, s5, s6, s7;
+          f2unpack(acc0, s0, s1);
+          f2unpack(acc1, s2, s3);
+          f2unpack(acc2, s4, s5);
+          f2unpack(acc3, s6, s7);
+          lsum = ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
         }
         l = l * alpha + lsum;
         tmem_st32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));

@@ -260,12 +260,88 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       : "memory");
 }
 
+// Warpgroup register rebalancing (all four warps of a warpgroup execute it).
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ---------------------------------------------------------------------------
 // Small numerics
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Packed pairs of fp32 in one 64-bit register (sm_100 f32x2 arithmetic).
+__device__ __forceinline__ uint64_t f2pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t u2pack(uint32_t a, uint32_t b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t r, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ void u2unpack(uint64_t r, uint32_t& a, uint32_t& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(a), "=r"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 2^x for a pair, on the FMA/ALU pipes instead of the MUFU unit.
+// Split x = j + f with j = rint(x) (the 1.5*2^23 rounding constant), f in
+// [-1/2, 1/2]; 2^f by a degree-3 polynomial (least-relative-error fit,
+// |rel err| < 7.5e-5, far below the bf16 rounding of the numerators); then
+// j is added to the exponent field.  x is clamped to >= -125 so the result
+// stays a normal number (2^-125 for masked columns: negligible next to the
+// row maximum, which is >= 2^-8 whenever the row has a real key).
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+  float a, b;
+  f2unpack(x2, a, b);
+  a = fmaxf(a, -125.0f);
+  b = fmaxf(b, -125.0f);
+  const uint64_t x = f2pack(a, b);
+  const uint64_t r = add2(x, f2pack(12582912.0f, 12582912.0f));
+  const uint64_t jj = add2(r, f2pack(-12582912.0f, -12582912.0f));
+  const uint64_t f = fma2(jj, f2pack(-1.0f, -1.0f), x);
+  uint64_t p = fma2(f2pack(0.05517167f, 0.05517167f), f, f2pack(0.24261113f, 0.24261113f));
+  p = fma2(p, f, f2pack(0.69326097f, 0.69326097f));
+  p = fma2(p, f, f2pack(0.99992806f, 0.99992806f));
+  uint32_t p0, p1, r0, r1;
+  u2unpack(p, p0, p1);
+  u2unpack(r, r0, r1);
+  return u2pack(p0 + (r0 << 23), p1 + (r1 << 23));
+}
+
+// 2^x on a packed bf16 pair (one MUFU operation for both).
+__device__ __forceinline__ uint32_t ex2_bf16x2(uint32_t x) {
+  uint32_t y;
+  asm("ex2.approx.ftz.bf16x2 %0, %1;" : "=r"(y) : "r"(x));
   return y;
 }
 
