@@ -42,6 +42,8 @@ WORKLOAD_TEXT = {
     "fastwan": "FastWan2.2-TI2V-5B latent grid 31x22x40, B1 H24 D128, block 4x8x8, topk 64",
     "wan81": "Wan2.1-1.3B 81-frame latent grid 21x30x52, B1 H12 D128, block 4x8x8, topk 32",
     "long": "Wan2.1-1.3B 321-frame latent grid 81x30x52, B1 H12 D128, block 4x8x8, topk 59",
+    "tile64": ("non-uniform rows, 64-token tiles: 512 prefix + video 16x32x32, B1 H24 D128, tile 4x4x4, "
+               "bool block map (prefix rows dense, video rows prefix + 32, 5% rows empty)"),
 }
 
 
@@ -156,7 +158,10 @@ def run_reference(args, wl, world, rank):
         t0 = time.perf_counter()
         qt, kt, vt = (oracle.tile(g, inp[n]) for n in ("q", "k", "v"))
         qbar, kbar = oracle.pool(g, qt), oracle.pool(g, kt)
-        idx, num = oracle.topk(oracle.score(qbar, kbar), wl.topk)
+        if wl.map_driven:
+            idx, num = oracle.map_to_index(inp["map"])
+        else:
+            idx, num = oracle.topk(oracle.score(qbar, kbar), wl.topk)
         t1 = time.perf_counter()
         rows = np.sort(rng.choice(total_rows, size=sample_rows, replace=False))
         o, _ = oracle.attn_rows(g, qt, kt, vt, idx, num, rows)
@@ -198,7 +203,10 @@ def cpu_baseline_sample(wl, seconds_hint=20.0):
     t0 = time.perf_counter()
     qt, kt, vt = (oracle.tile(g, inp[n]) for n in ("q", "k", "v"))
     qbar, kbar = oracle.pool(g, qt), oracle.pool(g, kt)
-    idx, num = oracle.topk(oracle.score(qbar, kbar), wl.topk)
+    if wl.map_driven:
+        idx, num = oracle.map_to_index(inp["map"])
+    else:
+        idx, num = oracle.topk(oracle.score(qbar, kbar), wl.topk)
     oracle.untile(g, qt)
     t_front = time.perf_counter() - t0
     total_rows = wl.B * wl.H * g.Sp
@@ -258,6 +266,8 @@ def main():
 
     inp = workloads.make_inputs(wl)
     host = {n: torch.from_numpy(inp[n].view(np.int16)).view(torch.bfloat16).pin_memory() for n in ("q", "k", "v")}
+    if wl.map_driven:
+        host["map"] = torch.from_numpy(inp["map"].view(np.uint8)).pin_memory()
     dev = {n: host[n].to("cuda", non_blocking=False) for n in host}
     plan = vsa.Plan.of(wl)
     fwd = vsa.Forward(plan, wl.B, wl.H, wl.topk)
@@ -275,7 +285,10 @@ def main():
         vsa.tile(p, dev["q"], pooled=True, out=fwd.qt, pooled_out=fwd.qbar)
         vsa.tile(p, dev["k"], pooled=True, out=fwd.kt, pooled_out=fwd.kbar)
         vsa.tile(p, dev["v"], out=fwd.vt)
-        vsa.coarse_topk(p, fwd.qbar, fwd.kbar, wl.topk, idx_out=fwd.idx, num_out=fwd.num)
+        if wl.map_driven:
+            vsa.map_to_index(dev["map"], idx_out=fwd.idx, num_out=fwd.num)
+        else:
+            vsa.coarse_topk(p, fwd.qbar, fwd.kbar, wl.topk, idx_out=fwd.idx, num_out=fwd.num)
         if i is not None:
             attn_ev[i][0].record(stream)
         vsa.sparse_attn_fwd(p, fwd.qt, fwd.kt, fwd.vt, fwd.idx, fwd.num, o_out=fwd.ot, lse_out=fwd.lse)
@@ -329,7 +342,7 @@ def main():
     for _ in range(3):
         for n in dev:
             dev[n].copy_(host[n], non_blocking=True)
-        fwd(dev["q"], dev["k"], dev["v"])
+        fwd(dev["q"], dev["k"], dev["v"], dev.get("map"))
         o_host.copy_(fwd.o, non_blocking=True)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sync_all()
@@ -337,13 +350,13 @@ def main():
     for _ in range(args.steps):
         for n in dev:
             dev[n].copy_(host[n], non_blocking=True)
-        fwd(dev["q"], dev["k"], dev["v"])
+        fwd(dev["q"], dev["k"], dev["v"], dev.get("map"))
         o_host.copy_(fwd.o, non_blocking=True)
     e1.record(stream)
     sync_all()
     e2e_elapsed = max_over_ranks(e0.elapsed_time(e1) / 1e3)
     assert vsa.get_status() == vsa.VSA_OK
-    h2d = sum(host[n].numel() * 2 for n in host)
+    h2d = sum(host[n].numel() * host[n].element_size() for n in host)
     d2h = o_host.numel() * 2
 
     if rank == 0:
@@ -363,9 +376,10 @@ def main():
                 "workload": WORKLOAD_TEXT[args.workload],
                 "B": wl.B, "H": wl.H, "D": wl.D, "grid": [wl.T, wl.Hg, wl.Wg], "block": list(wl.block),
                 "num_blocks": wl.num_blocks, "topk": wl.topk, "selected_block_tflop_per_step": flops / 1e12,
+                "selected_pairs": int(fwd.num.sum().item()),
                 "attn_ms": attn_avg * 1e3, "front_ms": float(np.mean(front_s)) * 1e3,
                 "l2": "inputs larger than L2: q/k/v %.0f MB and tiled q/k/v %.0f MB per step" % (
-                    h2d / 1e6, 3 * fwd.qt.numel() * 2 / 1e6),
+                    sum(host[n].numel() * 2 for n in ("q", "k", "v")) / 1e6, 3 * fwd.qt.numel() * 2 / 1e6),
                 "parallelism": f"replicas x{world}",
             },
             "roofline": {

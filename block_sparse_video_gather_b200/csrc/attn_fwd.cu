@@ -154,6 +154,78 @@ __device__ __forceinline__ int key_tile_mask(const Geo& g, int kb, int half, uin
   return any ? kTilePartial : kTileEmpty;
 }
 
+// Validity bits of the 64 slots of block kb (two words), for 64-token
+// blocks.  Returns kTileFull / kTilePartial / kTileEmpty.
+__device__ __forceinline__ int block64_mask(const Geo& g, int kb, uint32_t& w0, uint32_t& w1) {
+  uint32_t w[4];
+  // slots 0..63 of the block are columns 0..63 of "tile 0" of a 128-column view
+  w[0] = w[1] = w[2] = w[3] = 0xffffffffu;
+  if (kb < 0) {
+    w0 = w1 = 0u;
+    return kTileEmpty;
+  }
+  if (kb < g.n_pre) {
+    const int lim = g.n_prefix - kb * g.bs;
+    if (lim <= 0) {
+      w0 = w1 = 0u;
+      return kTileEmpty;
+    }
+    if (lim >= 64) {
+      w0 = w1 = 0xffffffffu;
+      return kTileFull;
+    }
+    w0 = lim >= 32 ? 0xffffffffu : ((1u << lim) - 1u);
+    w1 = lim <= 32 ? 0u : ((1u << (lim - 32)) - 1u);
+    return kTilePartial;
+  }
+  int vt, vh, vw;
+  video_block_extent(g, kb - g.n_pre, vt, vh, vw);
+  if (vt == g.bt && vh == g.bh && vw == g.bw) {
+    w0 = w1 = 0xffffffffu;
+    return kTileFull;
+  }
+  const uint32_t rowbits = vw >= 32 ? 0xffffffffu : ((1u << vw) - 1u);
+  const int rows_per_word = 32 >> g.lbw;
+  uint32_t any = 0;
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    uint32_t word = 0;
+    const int row0 = (32 * i) >> g.lbw;
+    for (int r = 0; r < rows_per_word; ++r) {
+      const int R = row0 + r;
+      const int lh = R & (g.bh - 1);
+      const int lt = R >> g.lbh;
+      if (lt < vt && lh < vh) word |= rowbits << (r << g.lbw);
+    }
+    w[i] = word;
+    any |= word;
+  }
+  w0 = w[0];
+  w1 = w[1];
+  return any ? kTilePartial : kTileEmpty;
+}
+
+// Mask of 128-key tile t of an item.  256-token blocks: tile t is half t&1
+// of block list[t/2].  64-token blocks: tile t holds blocks list[2t] and
+// list[2t+1] (the second may be absent).
+template <int BS>
+__device__ __forceinline__ int item_tile_mask(const Geo& g, int kb_a, int kb_b, int t, uint32_t (&mw)[4]) {
+  if (BS == 256) return key_tile_mask(g, kb_a, t & 1, mw);
+  const int sa = block64_mask(g, kb_a, mw[0], mw[1]);
+  const int sb = block64_mask(g, kb_b, mw[2], mw[3]);
+  if (sa == kTileFull && sb == kTileFull) return kTileFull;
+  if (sa == kTileEmpty && sb == kTileEmpty) return kTileEmpty;
+  if (sa == kTileFull) mw[0] = mw[1] = 0xffffffffu;
+  if (sb == kTileFull) mw[2] = mw[3] = 0xffffffffu;
+  return kTilePartial;
+}
+
+// 128-key tiles of an item with nb selected blocks.
+template <int BS>
+__device__ __forceinline__ int item_tiles(int nb) {
+  return BS == 256 ? 2 * nb : (nb + 1) / 2;
+}
+
 // Set the masked columns of one row of S to -inf.  The mask is the same for
 // every thread, so the branches are uniform; columns are handled four at a
 // time whenever each group of four is all-real or all-padded.
@@ -185,6 +257,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Barrie
   return __all_sync(0xffffffffu, ok);
 }
 
+template <int BS>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ Params p) {
@@ -196,6 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sV = smem + kSmemV;
   Barriers* bars = reinterpret_cast<Barriers*>(smem + kSmemBar);
 
+  constexpr int kQTiles = BS == 256 ? 2 : 1;  // 128-row query tiles per item
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const Geo& g = p.g;
@@ -247,25 +321,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int bh = item / g.NB, qb = item - bh * g.NB;
         const long long base = static_cast<long long>(bh) * g.Sp;
         if (!mbar_wait(&bars->q_empty, (qit & 1) ^ 1, &bars->abort, p.status, kTimeoutNs)) break;
-        mbar_arrive_expect_tx(&bars->q_full, kQBytes);
-        const int qrow = static_cast<int>(base + static_cast<long long>(qb) * 256);
-        for (int i = 0; i < 2; ++i)
+        mbar_arrive_expect_tx(&bars->q_full, kQTiles * kTileBytes);
+        const int qrow = static_cast<int>(base + static_cast<long long>(qb) * BS);
+        for (int i = 0; i < kQTiles; ++i)
           for (int hf = 0; hf < 2; ++hf)
             tma_load_2d(sQ + i * kTileBytes + hf * kHalfBytes, &tm_q, hf * 64, qrow + i * 128, &bars->q_full, pol_q);
         ++qit;
         bool stop = false;
-        for (int t = 0; t < 2 * nb && !stop; ++t) {
-          const int kb0 = item_block_id(p, item, t >> 1);
-          const int kb = kb0 < 0 ? 0 : kb0;  // unusable ids load block 0; the softmax masks them out
-          const int krow = static_cast<int>(base + static_cast<long long>(kb) * 256 + (t & 1) * 128);
+        const int n = item_tiles<BS>(nb);
+        for (int t = 0; t < n && !stop; ++t) {
+          // Key rows of this tile: one 128-row box (256-token blocks) or two
+          // 64-row boxes (64-token blocks).  Unusable or absent blocks load
+          // block 0 -- finite data, masked out by the softmax -- so that no
+          // stale shared memory can reach the PV product.
+          int krow0, krow1 = 0;
+          if (BS == 256) {
+            const int kb0 = item_block_id(p, item, t >> 1);
+            const int kb = kb0 < 0 ? 0 : kb0;
+            krow0 = static_cast<int>(base + static_cast<long long>(kb) * 256 + (t & 1) * 128);
+          } else {
+            const int ka = item_block_id(p, item, 2 * t);
+            const int kb = 2 * t + 1 < nb ? item_block_id(p, item, 2 * t + 1) : -1;
+            krow0 = static_cast<int>(base + static_cast<long long>(ka < 0 ? 0 : ka) * 64);
+            krow1 = static_cast<int>(base + static_cast<long long>(kb < 0 ? 0 : kb) * 64);
+          }
           const int sk = kit % kStages;
           if (!mbar_wait(&bars->k_empty[sk], ((kit / kStages) & 1) ^ 1, &bars->abort, p.status, kTimeoutNs)) {
             stop = true;
             break;
           }
           mbar_arrive_expect_tx(&bars->k_full[sk], kTileBytes);
-          for (int hf = 0; hf < 2; ++hf)
-            tma_load_2d(sK + sk * kTileBytes + hf * kHalfBytes, &tm_k, hf * 64, krow, &bars->k_full[sk], pol_kv);
+          for (int hf = 0; hf < 2; ++hf) {
+            uint8_t* dst = sK + sk * kTileBytes + hf * kHalfBytes;
+            tma_load_2d(dst, &tm_k, hf * 64, krow0, &bars->k_full[sk], pol_kv);
+            if (BS == 64) tma_load_2d(dst + kHalfBytes / 2, &tm_k, hf * 64, krow1, &bars->k_full[sk], pol_kv);
+          }
           ++kit;
           const int sv = vit % kStages;
           if (!mbar_wait(&bars->v_empty[sv], ((vit / kStages) & 1) ^ 1, &bars->abort, p.status, kTimeoutNs)) {
@@ -273,8 +363,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           mbar_arrive_expect_tx(&bars->v_full[sv], kTileBytes);
-          for (int hf = 0; hf < 2; ++hf)
-            tma_load_2d(sV + sv * kTileBytes + hf * kHalfBytes, &tm_v, hf * 64, krow, &bars->v_full[sv], pol_kv);
+          for (int hf = 0; hf < 2; ++hf) {
+            uint8_t* dst = sV + sv * kTileBytes + hf * kHalfBytes;
+            tma_load_2d(dst, &tm_v, hf * 64, krow0, &bars->v_full[sv], pol_kv);
+            if (BS == 64) tma_load_2d(dst + kHalfBytes / 2, &tm_v, hf * 64, krow1, &bars->v_full[sv], pol_kv);
+          }
           ++vit;
         }
         if (stop) break;
@@ -323,7 +416,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int item = blockIdx.x; item < total_items && ok; item += gridDim.x) {
         const int nb = item_blocks(p, item, true);
         if (nb == 0) continue;
-        const int n = 2 * nb;
+        const int n = item_tiles<BS>(nb);
         if (!(ok = mbar_wait(&bars->q_full, qit & 1, &bars->abort, p.status, kTimeoutNs))) break;
         ++qit;
         tc_fence_after();
@@ -332,8 +425,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         issue_s(0, sk);
         mma_commit(&bars->s_full[0]);
-        issue_s(1, sk);
-        mma_commit(&bars->s_full[1]);
+        if (kQTiles == 2) {
+          issue_s(1, sk);
+          mma_commit(&bars->s_full[1]);
+        }
         mma_commit(&bars->k_empty[sk]);
         ++kit;
         for (int t = 0; t < n; ++t) {
@@ -353,17 +448,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             issue_s(0, sk);
             mma_commit(&bars->s_full[0]);
           }
-          if (!(ok = mbar_wait(&bars->p_full[1], tiles & 1, &bars->abort, p.status, kTimeoutNs))) break;
-          if (t == 0 && !(ok = mbar_wait(&bars->o_empty[1], (items & 1) ^ 1, &bars->abort, p.status, kTimeoutNs)))
-            break;
-          tc_fence_after();
-          issue_pv(1, sv, t > 0);
+          if (kQTiles == 2) {
+            if (!(ok = mbar_wait(&bars->p_full[1], tiles & 1, &bars->abort, p.status, kTimeoutNs))) break;
+            if (t == 0 && !(ok = mbar_wait(&bars->o_empty[1], (items & 1) ^ 1, &bars->abort, p.status, kTimeoutNs)))
+              break;
+            tc_fence_after();
+            issue_pv(1, sv, t > 0);
+          }
           mma_commit(&bars->v_empty[sv]);
           ++vit;
-          if (t == n - 1) mma_commit(&bars->o_full[1]);
+          if (kQTiles == 2 && t == n - 1) mma_commit(&bars->o_full[1]);
           if (more) {
-            issue_s(1, sk);
-            mma_commit(&bars->s_full[1]);
+            if (kQTiles == 2) {
+              issue_s(1, sk);
+              mma_commit(&bars->s_full[1]);
+            }
             mma_commit(&bars->k_empty[sk]);
             ++kit;
           }
@@ -382,6 +481,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_inc<kRegsHigh>();
     // ------------------------------------------------------------ softmax + epilogue
     const int wg = (warp - 4) >> 2;  // Q tile
+    // 64-token blocks: one query tile per item, held by the first warpgroup
+    // in the top 64 rows of its 128-row MMA tile; the second warpgroup idles.
+    const bool active = kQTiles == 2 || wg == 0;
     const int quarter = warp & 3;    // TMEM lane quarter of this warp
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
@@ -390,24 +492,35 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float sl2 = p.scale_log2;
     int tiles = 0, items = 0;
     bool ok = true;
-    for (int item = blockIdx.x; item < total_items && ok; item += gridDim.x) {
+    for (int item = blockIdx.x; item < total_items && ok && active; item += gridDim.x) {
       const int nb = item_blocks(p, item, false);
       const int bh = item / g.NB, qb = item - bh * g.NB;
-      const long long row = static_cast<long long>(bh) * g.Sp + static_cast<long long>(qb) * 256 + wg * 128 + r;
+      const long long row = static_cast<long long>(bh) * g.Sp + static_cast<long long>(qb) * BS + wg * 128 + r;
+      const bool real_row = BS == 256 || r < 64;
       uint4* orow = reinterpret_cast<uint4*>(p.o + row * 128);
       if (nb == 0) {
+        if (!real_row) continue;
 #pragma unroll
         for (int c = 0; c < 16; ++c) orow[c] = make_uint4(0, 0, 0, 0);
         p.lse[row] = -INFINITY;
         continue;
       }
-      const int n = 2 * nb;
+      const int n = item_tiles<BS>(nb);
       float m_used = -INFINITY, l = 0.0f;
       for (int t = 0; t < n; ++t) {
-        const int kb = item_block_id(p, item, t >> 1);
-        if (kb < 0 && wg == 0 && r == 0) atomicCAS(p.status, 0u, (unsigned)VSA_ERR_BAD_INDEX);
+        int kb_a, kb_b = -1;
+        if (BS == 256) {
+          kb_a = item_block_id(p, item, t >> 1);
+        } else {
+          kb_a = item_block_id(p, item, 2 * t);
+          if (2 * t + 1 < nb) {
+            kb_b = item_block_id(p, item, 2 * t + 1);
+            if (kb_b < 0 && r == 0) atomicCAS(p.status, 0u, (unsigned)VSA_ERR_BAD_INDEX);
+          }
+        }
+        if (kb_a < 0 && wg == 0 && r == 0) atomicCAS(p.status, 0u, (unsigned)VSA_ERR_BAD_INDEX);
         uint32_t mw[4];
-        const int mstate = key_tile_mask(g, kb, t & 1, mw);
+        const int mstate = item_tile_mask<BS>(g, kb_a, kb_b, t, mw);
         if (!(ok = warp_wait(&bars->s_full[wg], tiles & 1, bars, p.status))) break;
         tc_fence_after();
         uint32_t pk[64];
@@ -518,12 +631,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int j = 0; j < 16; ++j)
           wp[j] = pack_bf16x2(__uint_as_float(ov[2 * j]) * inv, __uint_as_float(ov[2 * j + 1]) * inv);
+        if (real_row) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) orow[c * 4 + j] = w[j];
+          for (int j = 0; j < 4; ++j) orow[c * 4 + j] = w[j];
+        }
       }
       tc_fence_before();
       mbar_arrive(&bars->o_empty[wg]);
-      p.lse[row] = l > 0.0f ? (m_used + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+      if (real_row) p.lse[row] = l > 0.0f ? (m_used + __log2f(l)) * 0.69314718055994531f : -INFINITY;
       ++items;
     }
   }
@@ -570,11 +685,12 @@ bool make_tmap(CUtensorMap* tm, const void* base, unsigned long long rows, unsig
 }  // namespace
 
 cudaError_t launch_attn_fwd(const Geo& g, const AttnArgs& a, cudaStream_t stream) {
-  if (g.bs != 256) return cudaErrorNotSupported;
+  if (g.bs != 256 && g.bs != 64) return cudaErrorNotSupported;
   const unsigned long long rows = static_cast<unsigned long long>(a.BH) * g.Sp;
   if (rows >= (1ull << 31)) return cudaErrorInvalidValue;
+  const unsigned kv_box = g.bs == 256 ? 128 : 64;
   CUtensorMap tq, tk, tv;
-  if (!make_tmap(&tq, a.q, rows, 128) || !make_tmap(&tk, a.k, rows, 128) || !make_tmap(&tv, a.v, rows, 128))
+  if (!make_tmap(&tq, a.q, rows, 128) || !make_tmap(&tk, a.k, rows, kv_box) || !make_tmap(&tv, a.v, rows, kv_box))
     return cudaErrorInvalidValue;
   Params p;
   p.idx = a.idx;
@@ -586,11 +702,12 @@ cudaError_t launch_attn_fwd(const Geo& g, const AttnArgs& a, cudaStream_t stream
   p.status = a.status;
   p.scale_log2 = static_cast<float>(1.4426950408889634 / 11.313708498984761);  // log2(e) / sqrt(128)
   p.g = g;
-  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTotal);
-  if (e != cudaSuccess) return e;
   const long long items = static_cast<long long>(a.BH) * g.NB;
   const int grid = static_cast<int>(items < a.num_sms ? items : a.num_sms);
-  attn_fwd_kernel<<<grid, kThreads, kSmemTotal, stream>>>(tq, tk, tv, p);
+  auto kern = g.bs == 256 ? attn_fwd_kernel<256> : attn_fwd_kernel<64>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTotal);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreads, kSmemTotal, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 

@@ -215,7 +215,6 @@ int vsa_sparse_attn_fwd(vsa_plan_t plan, const uint16_t* q, const uint16_t* k, c
   if (int rc = check_dims(B, H, D)) return rc;
   const vsa::Geo& g = plan->g;
   if (g.bs == 64 && (g.NB & 1)) return VSA_ERR_UNSUPPORTED;
-  if (g.bs != 256) return VSA_ERR_UNSUPPORTED;
   DeviceState* ds = nullptr;
   if (int rc = device_state(&ds)) return rc;
   vsa::AttnArgs a;

@@ -159,7 +159,7 @@ def test_attention_tiny_every_row():
     _attn_vs_oracle(wl, ref["idx"], ref["num"], what="tiny")
 
 
-@pytest.mark.parametrize("shape", [s for s in EDGE_SHAPES if s[3] == (4, 8, 8)])
+@pytest.mark.parametrize("shape", EDGE_SHAPES)
 def test_attention_oracle_indices_nonuniform_rows(shape):
     """Random selections with per-row counts 0..max_k (zero rows included), on grids
     with partial blocks along every axis."""
@@ -229,22 +229,30 @@ def _sample_rows(wl, n_per_head, seed):
     return np.concatenate(rows)
 
 
-@pytest.mark.parametrize("name", ["tiny", "fastwan", "wan81", "long"])
+@pytest.mark.parametrize("name", ["tiny", "fastwan", "wan81", "long", "tile64"])
 def test_full_path_full_size(name):
     """The launch configuration the benchmark times (vsa.Forward) at full size:
-    indices bit-exact, o/lse on sampled real rows, untile of o bit-exact."""
+    indices bit-exact, o/lse on sampled real rows, untile of o bit-exact.
+    tile64 takes its caller-supplied bool block map through map_to_index."""
     wl = workloads.WORKLOADS[name]
     ref = H.oracle_front(wl)
     inp = H.inputs(wl)
     plan = vsa.Plan.of(wl)
     fwd = vsa.Forward(plan, wl.B, wl.H, wl.topk)
-    o, lse = fwd(H.to_dev(inp["q"]), H.to_dev(inp["k"]), H.to_dev(inp["v"]))
+    bmap = torch.from_numpy(inp["map"]).cuda() if wl.map_driven else None
+    o, lse = fwd(H.to_dev(inp["q"]), H.to_dev(inp["k"]), H.to_dev(inp["v"]), bmap)
     torch.cuda.synchronize()
     assert vsa.get_status() == vsa.VSA_OK
     np.testing.assert_array_equal(fwd.idx.cpu().numpy(), ref["idx"])
     np.testing.assert_array_equal(fwd.num.cpu().numpy(), ref["num"])
     np.testing.assert_array_equal(H.from_dev(fwd.qt), ref["qt"])
     rows = _sample_rows(wl, 48 if name != "tiny" else 200, seed=16)
+    if wl.map_driven:  # include rows of zero-count tiles and of dense prefix tiles
+        g = ref["g"]
+        zero = np.flatnonzero(ref["num"].reshape(-1) == 0)[:8]
+        extra = [(z // g.NB) * g.Sp + (z % g.NB) * g.bs + np.arange(0, g.bs, 9) for z in zero]
+        extra += [bh * g.Sp + np.arange(0, g.n_pre * g.bs, 37) for bh in range(wl.B * wl.H)]
+        rows = np.unique(np.concatenate([rows] + extra))
     o_ref, lse_ref = oracle.attn_rows(ref["g"], ref["qt"], ref["kt"], ref["vt"], ref["idx"], ref["num"], rows)
     ot_bits = H.from_dev(fwd.ot).reshape(-1, 128)
     H.compare_o_lse(ot_bits[rows], lse.cpu().numpy().reshape(-1)[rows], o_ref, lse_ref, name)
