@@ -23,18 +23,36 @@ namespace {
 constexpr int kTileThreads = 256;
 constexpr int kRowChunks = 16;  // 16 B chunks per 256 B row (D = 128)
 
-// Token index of slot `slot` of block `blk`, or -1 for a padded slot.
-__device__ __forceinline__ long long token_of_slot(const Geo& g, int blk, int slot) {
-  if (blk < g.n_pre) {
-    long long s = static_cast<long long>(blk) * g.bs + slot;
-    return s < g.n_prefix ? s : -1;
-  }
-  int vb = blk - g.n_pre;
-  int bW = vb % g.nW, bH = (vb / g.nW) % g.nH, bT = vb / (g.nW * g.nH);
-  int lw = slot & (g.bw - 1);
-  int lh = (slot >> g.lbw) & (g.bh - 1);
-  int lt = slot >> (g.lbw + g.lbh);
-  int t = bT * g.bt + lt, y = bH * g.bh + lh, x = bW * g.bw + lw;
+// Where the tokens of one block live in the untiled sequence.  Computed
+// once per CTA (three divisions); each slot then costs shifts and two
+// multiply-adds.  Slot (lt, lh, lw) of a video block sits at grid point
+// (t0 + lt, y0 + lh, x0 + lw); slot s of a prefix tile is token p0 + s.
+struct BlockOrigin {
+  bool prefix;
+  long long p0;   // first token of a prefix tile
+  int plim;       // real tokens of a prefix tile
+  int t0, y0, x0; // grid origin of a video block
+};
+
+__device__ __forceinline__ BlockOrigin block_origin(const Geo& g, int blk) {
+  BlockOrigin o;
+  o.prefix = blk < g.n_pre;
+  o.p0 = static_cast<long long>(blk) * g.bs;
+  o.plim = g.n_prefix - blk * g.bs;
+  const int vb = blk - g.n_pre;
+  const int bW = vb % g.nW, bH = (vb / g.nW) % g.nH, bT = vb / (g.nW * g.nH);
+  o.t0 = bT * g.bt;
+  o.y0 = bH * g.bh;
+  o.x0 = bW * g.bw;
+  return o;
+}
+
+// Token index of slot `slot` of the block, or -1 for a padded slot.
+__device__ __forceinline__ long long token_of_slot(const Geo& g, const BlockOrigin& o, int slot) {
+  if (o.prefix) return slot < o.plim ? o.p0 + slot : -1;
+  const int x = o.x0 + (slot & (g.bw - 1));
+  const int y = o.y0 + ((slot >> g.lbw) & (g.bh - 1));
+  const int t = o.t0 + (slot >> (g.lbw + g.lbh));
   if (t >= g.T || y >= g.Hg || x >= g.Wg) return -1;
   return g.n_prefix + (static_cast<long long>(t) * g.Hg + y) * g.Wg + x;
 }
@@ -57,11 +75,12 @@ __global__ void __launch_bounds__(kTileThreads) tile_kernel(Geo g, int H, const 
   const int row0 = threadIdx.x >> 4;  // 0..15
   constexpr int kIters = BS / 16;
 
+  const BlockOrigin org = block_origin(g, blk);
   uint4 v[kIters];
 #pragma unroll
   for (int i = 0; i < kIters; ++i) {
     const int slot = row0 + 16 * i;
-    const long long s = token_of_slot(g, blk, slot);
+    const long long s = token_of_slot(g, org, slot);
     if (s >= 0) {
       const long long src = ((static_cast<long long>(b) * g.S + s) * H + h) * kRowChunks + chunk;
       v[i] = __ldcs(x + src);
@@ -103,9 +122,10 @@ __global__ void __launch_bounds__(kTileThreads) untile_kernel(Geo g, int H, cons
   uint4 v[kIters];
 #pragma unroll
   for (int i = 0; i < kIters; ++i) v[i] = __ldcs(xt + src0 + (row0 + 16 * i) * kRowChunks + chunk);
+  const BlockOrigin org = block_origin(g, blk);
 #pragma unroll
   for (int i = 0; i < kIters; ++i) {
-    const long long s = token_of_slot(g, blk, row0 + 16 * i);
+    const long long s = token_of_slot(g, org, row0 + 16 * i);
     if (s >= 0) x[((static_cast<long long>(b) * g.S + s) * H + h) * kRowChunks + chunk] = v[i];
   }
 }
