@@ -308,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   regs_dec<kRegsLow>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
@@ -320,12 +320,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (nb == 0) continue;
         const int bh = item / g.NB, qb = item - bh * g.NB;
         const long long base = static_cast<long long>(bh) * g.Sp;
-        if (!mbar_wait(&bars->q_empty, (qit & 1) ^ 1, &bars->abort, p.status, kTimeoutNs)) break;
-        mbar_arrive_expect_tx(&bars->q_full, kQTiles * kTileBytes);
+        if (!warp_wait(&bars->q_empty, (qit & 1) ^ 1, bars, p.status)) break;
+        mbar_arrive_expect_tx_w(&bars->q_full, kQTiles * kTileBytes);
         const int qrow = static_cast<int>(base + static_cast<long long>(qb) * BS);
         for (int i = 0; i < kQTiles; ++i)
           for (int hf = 0; hf < 2; ++hf)
-            tma_load_2d(sQ + i * kTileBytes + hf * kHalfBytes, &tm_q, hf * 64, qrow + i * 128, &bars->q_full, pol_q);
+            tma_load_2d_w(sQ + i * kTileBytes + hf * kHalfBytes, &tm_q, hf * 64, qrow + i * 128, &bars->q_full, pol_q);
         ++qit;
         bool stop = false;
         const int n = item_tiles<BS>(nb);
@@ -346,27 +346,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             krow1 = static_cast<int>(base + static_cast<long long>(kb < 0 ? 0 : kb) * 64);
           }
           const int sk = kit % kStages;
-          if (!mbar_wait(&bars->k_empty[sk], ((kit / kStages) & 1) ^ 1, &bars->abort, p.status, kTimeoutNs)) {
+          if (!warp_wait(&bars->k_empty[sk], ((kit / kStages) & 1) ^ 1, bars, p.status)) {
             stop = true;
             break;
           }
-          mbar_arrive_expect_tx(&bars->k_full[sk], kTileBytes);
+          mbar_arrive_expect_tx_w(&bars->k_full[sk], kTileBytes);
           for (int hf = 0; hf < 2; ++hf) {
             uint8_t* dst = sK + sk * kTileBytes + hf * kHalfBytes;
-            tma_load_2d(dst, &tm_k, hf * 64, krow0, &bars->k_full[sk], pol_kv);
-            if (BS == 64) tma_load_2d(dst + kHalfBytes / 2, &tm_k, hf * 64, krow1, &bars->k_full[sk], pol_kv);
+            tma_load_2d_w(dst, &tm_k, hf * 64, krow0, &bars->k_full[sk], pol_kv);
+            if (BS == 64) tma_load_2d_w(dst + kHalfBytes / 2, &tm_k, hf * 64, krow1, &bars->k_full[sk], pol_kv);
           }
           ++kit;
           const int sv = vit % kStages;
-          if (!mbar_wait(&bars->v_empty[sv], ((vit / kStages) & 1) ^ 1, &bars->abort, p.status, kTimeoutNs)) {
+          if (!warp_wait(&bars->v_empty[sv], ((vit / kStages) & 1) ^ 1, bars, p.status)) {
             stop = true;
             break;
           }
-          mbar_arrive_expect_tx(&bars->v_full[sv], kTileBytes);
+          mbar_arrive_expect_tx_w(&bars->v_full[sv], kTileBytes);
           for (int hf = 0; hf < 2; ++hf) {
             uint8_t* dst = sV + sv * kTileBytes + hf * kHalfBytes;
-            tma_load_2d(dst, &tm_v, hf * 64, krow0, &bars->v_full[sv], pol_kv);
-            if (BS == 64) tma_load_2d(dst + kHalfBytes / 2, &tm_v, hf * 64, krow1, &bars->v_full[sv], pol_kv);
+            tma_load_2d_w(dst, &tm_v, hf * 64, krow0, &bars->v_full[sv], pol_kv);
+            if (BS == 64) tma_load_2d_w(dst + kHalfBytes / 2, &tm_v, hf * 64, krow1, &bars->v_full[sv], pol_kv);
           }
           ++vit;
         }
@@ -387,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    {
       // Descriptors are built once; each MMA only adds a constant to the
       // start-address field (smem addresses stay below 2^18, so the 14-bit
       // field never carries).  A lean issue loop keeps the tensor core fed:
@@ -404,76 +404,76 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
-          mma_ss(d, a + off, b + off, kIdescS, kk > 0 ? 1u : 0u);
+          mma_ss_w(d, a + off, b + off, kIdescS, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int i, int sv, bool acc) {
         const uint32_t d = tmem + 256 + i * 128, pa = tmem + i * 128;
         const uint64_t b = dv0 + sv * kTileDesc;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) mma_ts(d, pa + kk * 8, b + kk * (2048 >> 4), kIdescPV, (acc || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < 8; ++kk) mma_ts_w(d, pa + kk * 8, b + kk * (2048 >> 4), kIdescPV, (acc || kk > 0) ? 1u : 0u);
       };
       for (int item = blockIdx.x; item < total_items && ok; item += gridDim.x) {
-        const int nb = item_blocks(p, item, true);
+        const int nb = item_blocks(p, item, lane == 0);
         if (nb == 0) continue;
         const int n = item_tiles<BS>(nb);
-        if (!(ok = mbar_wait(&bars->q_full, qit & 1, &bars->abort, p.status, kTimeoutNs))) break;
+        if (!(ok = warp_wait(&bars->q_full, qit & 1, bars, p.status))) break;
         ++qit;
         tc_fence_after();
         int sk = kit % kStages;
-        if (!(ok = mbar_wait(&bars->k_full[sk], (kit / kStages) & 1, &bars->abort, p.status, kTimeoutNs))) break;
+        if (!(ok = warp_wait(&bars->k_full[sk], (kit / kStages) & 1, bars, p.status))) break;
         tc_fence_after();
         issue_s(0, sk);
-        mma_commit(&bars->s_full[0]);
+        mma_commit_w(&bars->s_full[0]);
         if (kQTiles == 2) {
           issue_s(1, sk);
-          mma_commit(&bars->s_full[1]);
+          mma_commit_w(&bars->s_full[1]);
         }
-        mma_commit(&bars->k_empty[sk]);
+        mma_commit_w(&bars->k_empty[sk]);
         ++kit;
         for (int t = 0; t < n; ++t) {
           const int sv = vit % kStages;
-          if (!(ok = mbar_wait(&bars->v_full[sv], (vit / kStages) & 1, &bars->abort, p.status, kTimeoutNs))) break;
-          if (!(ok = mbar_wait(&bars->p_full[0], tiles & 1, &bars->abort, p.status, kTimeoutNs))) break;
-          if (t == 0 && !(ok = mbar_wait(&bars->o_empty[0], (items & 1) ^ 1, &bars->abort, p.status, kTimeoutNs)))
+          if (!(ok = warp_wait(&bars->v_full[sv], (vit / kStages) & 1, bars, p.status))) break;
+          if (!(ok = warp_wait(&bars->p_full[0], tiles & 1, bars, p.status))) break;
+          if (t == 0 && !(ok = warp_wait(&bars->o_empty[0], (items & 1) ^ 1, bars, p.status)))
             break;
           tc_fence_after();
           issue_pv(0, sv, t > 0);
-          if (t == n - 1) mma_commit(&bars->o_full[0]);
+          if (t == n - 1) mma_commit_w(&bars->o_full[0]);
           const bool more = t + 1 < n;
           sk = kit % kStages;
           if (more) {
-            if (!(ok = mbar_wait(&bars->k_full[sk], (kit / kStages) & 1, &bars->abort, p.status, kTimeoutNs))) break;
+            if (!(ok = warp_wait(&bars->k_full[sk], (kit / kStages) & 1, bars, p.status))) break;
             tc_fence_after();
             issue_s(0, sk);
-            mma_commit(&bars->s_full[0]);
+            mma_commit_w(&bars->s_full[0]);
           }
           if (kQTiles == 2) {
-            if (!(ok = mbar_wait(&bars->p_full[1], tiles & 1, &bars->abort, p.status, kTimeoutNs))) break;
-            if (t == 0 && !(ok = mbar_wait(&bars->o_empty[1], (items & 1) ^ 1, &bars->abort, p.status, kTimeoutNs)))
+            if (!(ok = warp_wait(&bars->p_full[1], tiles & 1, bars, p.status))) break;
+            if (t == 0 && !(ok = warp_wait(&bars->o_empty[1], (items & 1) ^ 1, bars, p.status)))
               break;
             tc_fence_after();
             issue_pv(1, sv, t > 0);
           }
-          mma_commit(&bars->v_empty[sv]);
+          mma_commit_w(&bars->v_empty[sv]);
           ++vit;
-          if (kQTiles == 2 && t == n - 1) mma_commit(&bars->o_full[1]);
+          if (kQTiles == 2 && t == n - 1) mma_commit_w(&bars->o_full[1]);
           if (more) {
             if (kQTiles == 2) {
               issue_s(1, sk);
-              mma_commit(&bars->s_full[1]);
+              mma_commit_w(&bars->s_full[1]);
             }
-            mma_commit(&bars->k_empty[sk]);
+            mma_commit_w(&bars->k_empty[sk]);
             ++kit;
           }
           ++tiles;
         }
         if (!ok) break;
-        mma_commit(&bars->q_empty);
+        mma_commit_w(&bars->q_empty);
         ++items;
       }
       // Drain: wait for every MMA issued by this thread before TMEM and smem go away.
-      mma_commit(&bars->drain);
+      mma_commit_w(&bars->drain);
       mbar_wait_drain(&bars->drain, 0, kTimeoutNs);
     }
   }
