@@ -236,6 +236,7 @@ def main():
     ap.add_argument("--workload", default="fastwan", choices=list(WORKLOAD_TEXT))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-rows", type=int, default=2048, help="query rows per reference step")
+    ap.add_argument("--dtype", default="bf16", choices=["bf16", "f16"], help="16-bit format of q, k, v, o")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -264,14 +265,15 @@ def main():
         pg.barrier()
     vsa.lib()
 
-    inp = workloads.make_inputs(wl)
-    host = {n: torch.from_numpy(inp[n].view(np.int16)).view(torch.bfloat16).pin_memory() for n in ("q", "k", "v")}
+    inp = workloads.make_inputs(wl, dtype=args.dtype)
+    tdt = torch.float16 if args.dtype == "f16" else torch.bfloat16
+    host = {n: torch.from_numpy(inp[n].view(np.int16)).view(tdt).pin_memory() for n in ("q", "k", "v")}
     if wl.map_driven:
         host["map"] = torch.from_numpy(inp["map"].view(np.uint8)).pin_memory()
     dev = {n: host[n].to("cuda", non_blocking=False) for n in host}
     plan = vsa.Plan.of(wl)
-    fwd = vsa.Forward(plan, wl.B, wl.H, wl.topk)
-    o_host = torch.empty(fwd.o.shape, dtype=torch.bfloat16).pin_memory()
+    fwd = vsa.Forward(plan, wl.B, wl.H, wl.topk, dtype=tdt)
+    o_host = torch.empty(fwd.o.shape, dtype=tdt).pin_memory()
 
     stream = torch.cuda.current_stream()
     attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -371,7 +373,7 @@ def main():
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": elapsed / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16", "data": "synthetic (seeded; the recipe in block_sparse_video_gather_b200/workloads.py)",
+            "dtype": args.dtype, "data": "synthetic (seeded; the recipe in block_sparse_video_gather_b200/workloads.py)",
             "config": {
                 "workload": WORKLOAD_TEXT[args.workload],
                 "B": wl.B, "H": wl.H, "D": wl.D, "grid": [wl.T, wl.Hg, wl.Wg], "block": list(wl.block),

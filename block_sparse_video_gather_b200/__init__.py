@@ -22,9 +22,12 @@ LIB_PATH = os.path.join(_PKG, "libvsa.so")
 # Every symbol include/vsa.h declares.
 SYMBOLS = (
     "vsa_plan_create", "vsa_plan_create_prefix", "vsa_plan_destroy", "vsa_plan_sizes",
-    "vsa_plan_describe", "vsa_tile", "vsa_untile", "vsa_coarse_topk", "vsa_map_to_index",
-    "vsa_sparse_attn_fwd", "vsa_get_status", "vsa_strerror",
+    "vsa_plan_describe", "vsa_tile", "vsa_tile_ex", "vsa_untile", "vsa_coarse_topk", "vsa_map_to_index",
+    "vsa_sparse_attn_fwd", "vsa_sparse_attn_fwd_ex", "vsa_get_status", "vsa_strerror",
 )
+
+VSA_BF16 = 0
+VSA_F16 = 1
 
 VSA_OK = 0
 VSA_ERR_INVALID_ARG = 1
@@ -60,6 +63,8 @@ def lib():
         L.vsa_plan_sizes.argtypes = [P, P, P, P, P]
         L.vsa_plan_describe.argtypes = [P, i, ctypes.c_char_p, sz]
         L.vsa_tile.argtypes = [P, P, P, P, i, i, i, P]
+        L.vsa_tile_ex.argtypes = [P, i, P, P, P, i, i, i, P]
+        L.vsa_sparse_attn_fwd_ex.argtypes = [P, i, P, P, P, P, P, i, i, i, i, P, P, P]
         L.vsa_untile.argtypes = [P, P, P, i, i, i, P]
         L.vsa_coarse_topk.argtypes = [P, P, P, i, i, i, i, P, P, P]
         L.vsa_map_to_index.argtypes = [P, i, i, i, i, P, P, P]
@@ -132,35 +137,47 @@ def _ptr(t, dtype, what):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _dtype_code(t, what):
+    """bf16 -> VSA_BF16, fp16 -> VSA_F16 (the two formats the kernels take)."""
+    torch = _torch()
+    if t.dtype == torch.bfloat16:
+        return VSA_BF16
+    if t.dtype == torch.float16:
+        return VSA_F16
+    raise ValueError(f"{what} must be bfloat16 or float16, got {t.dtype}")
+
+
 def _stream():
     return ctypes.c_void_p(_torch().cuda.current_stream().cuda_stream)
 
 
 def tile(plan: Plan, x, pooled: bool = False, out=None, pooled_out=None):
-    """x [B,S,H,D] bf16 -> x_tiled [B,H,Sp,D] (and fp32 block means [B,H,NB,D])."""
+    """x [B,S,H,D] bf16/fp16 -> x_tiled [B,H,Sp,D] (and fp32 block means [B,H,NB,D])."""
     torch = _torch()
     B, S, H, D = x.shape
+    code = _dtype_code(x, "x")
     if out is None:
-        out = torch.empty((B, H, plan.Sp, D), dtype=torch.bfloat16, device=x.device)
+        out = torch.empty((B, H, plan.Sp, D), dtype=x.dtype, device=x.device)
     if pooled and pooled_out is None:
         pooled_out = torch.empty((B, H, plan.NB, D), dtype=torch.float32, device=x.device)
     if S != plan.S:
         raise ValueError(f"x has {S} tokens, plan expects {plan.S}")
-    _check(lib().vsa_tile(plan.handle, _ptr(x, torch.bfloat16, "x"), _ptr(out, torch.bfloat16, "x_tiled"),
-                          _ptr(pooled_out, torch.float32, "pooled") if pooled else None, B, H, D, _stream()),
+    _check(lib().vsa_tile_ex(plan.handle, code, _ptr(x, x.dtype, "x"), _ptr(out, x.dtype, "x_tiled"),
+                             _ptr(pooled_out, torch.float32, "pooled") if pooled else None, B, H, D, _stream()),
            "vsa_tile")
     return (out, pooled_out) if pooled else out
 
 
 def untile(plan: Plan, xt, out=None):
-    """x_tiled [B,H,Sp,D] bf16 -> x [B,S,H,D] (padded rows dropped)."""
+    """x_tiled [B,H,Sp,D] bf16/fp16 -> x [B,S,H,D] (padded rows dropped)."""
     torch = _torch()
     B, H, Sp, D = xt.shape
+    _dtype_code(xt, "x_tiled")
     if Sp != plan.Sp:
         raise ValueError(f"x_tiled has {Sp} rows, plan expects {plan.Sp}")
     if out is None:
-        out = torch.empty((B, plan.S, H, D), dtype=torch.bfloat16, device=xt.device)
-    _check(lib().vsa_untile(plan.handle, _ptr(xt, torch.bfloat16, "x_tiled"), _ptr(out, torch.bfloat16, "x"),
+        out = torch.empty((B, plan.S, H, D), dtype=xt.dtype, device=xt.device)
+    _check(lib().vsa_untile(plan.handle, _ptr(xt, xt.dtype, "x_tiled"), _ptr(out, xt.dtype, "x"),
                             B, H, D, _stream()), "vsa_untile")
     return out
 
@@ -198,15 +215,16 @@ def sparse_attn_fwd(plan: Plan, q, k, v, q2k_idx, q2k_num, o_out=None, lse_out=N
     torch = _torch()
     B, H, Sp, D = q.shape
     max_k = q2k_idx.shape[-1]
+    code = _dtype_code(q, "q")
     if o_out is None:
         o_out = torch.empty_like(q)
     if lse_out is None:
         lse_out = torch.empty((B, H, Sp), dtype=torch.float32, device=q.device)
-    _check(lib().vsa_sparse_attn_fwd(plan.handle, _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
-                                     _ptr(v, torch.bfloat16, "v"), _ptr(q2k_idx, torch.int32, "q2k_idx"),
-                                     _ptr(q2k_num, torch.int32, "q2k_num"), max_k, B, H, D,
-                                     _ptr(o_out, torch.bfloat16, "o"), _ptr(lse_out, torch.float32, "lse"),
-                                     _stream()), "vsa_sparse_attn_fwd")
+    _check(lib().vsa_sparse_attn_fwd_ex(plan.handle, code, _ptr(q, q.dtype, "q"), _ptr(k, q.dtype, "k"),
+                                        _ptr(v, q.dtype, "v"), _ptr(q2k_idx, torch.int32, "q2k_idx"),
+                                        _ptr(q2k_num, torch.int32, "q2k_num"), max_k, B, H, D,
+                                        _ptr(o_out, q.dtype, "o"), _ptr(lse_out, torch.float32, "lse"),
+                                        _stream()), "vsa_sparse_attn_fwd")
     return o_out, lse_out
 
 
@@ -228,10 +246,10 @@ class Forward:
     lse [B,H,Sp].
     """
 
-    def __init__(self, plan: Plan, B: int, H: int, topk: int | None, device="cuda", D: int = 128):
+    def __init__(self, plan: Plan, B: int, H: int, topk: int | None, device="cuda", D: int = 128, dtype=None):
         torch = _torch()
         self.plan, self.B, self.H, self.D, self.topk = plan, B, H, D, topk
-        t = dict(dtype=torch.bfloat16, device=device)
+        t = dict(dtype=dtype or torch.bfloat16, device=device)
         self.qt = torch.empty((B, H, plan.Sp, D), **t)
         self.kt = torch.empty((B, H, plan.Sp, D), **t)
         self.vt = torch.empty((B, H, plan.Sp, D), **t)

@@ -63,8 +63,12 @@ constexpr uint64_t kTimeoutNs = 2000000000ull;          // 2 s per wait
 constexpr int kRegsLaunch = 168, kRegsLow = 104, kRegsHigh = 200;
 static_assert(kThreads * kRegsLaunch == 128 * kRegsLow + 256 * kRegsHigh, "register split must match the launch");
 
-constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, 0, 0);   // Q (K-major) x K (K-major)
-constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, 0, 1);  // P (TMEM) x V (MN-major)
+// Q (K-major) x K (K-major); P (TMEM) x V (MN-major); bf16 or fp16 operands.
+template <bool F16>
+struct Idesc {
+  static constexpr uint32_t S = F16 ? idesc_f16_f32(128, 128, 0, 0) : idesc_bf16_f32(128, 128, 0, 0);
+  static constexpr uint32_t PV = F16 ? idesc_f16_f32(128, 128, 0, 1) : idesc_bf16_f32(128, 128, 0, 1);
+};
 
 constexpr int kTileFull = 0, kTilePartial = 1, kTileEmpty = 2;
 // Exponential pairs, out of every 8, evaluated by polynomial on the FMA pipe.
@@ -257,7 +261,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Barrie
   return __all_sync(0xffffffffu, ok);
 }
 
-template <int BS>
+template <int BS, bool F16>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ Params p) {
@@ -404,14 +408,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
-          mma_ss_w(d, a + off, b + off, kIdescS, kk > 0 ? 1u : 0u);
+          mma_ss_w(d, a + off, b + off, Idesc<F16>::S, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int i, int sv, bool acc) {
         const uint32_t d = tmem + 256 + i * 128, pa = tmem + i * 128;
         const uint64_t b = dv0 + sv * kTileDesc;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) mma_ts_w(d, pa + kk * 8, b + kk * (2048 >> 4), kIdescPV, (acc || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < 8; ++kk) mma_ts_w(d, pa + kk * 8, b + kk * (2048 >> 4), Idesc<F16>::PV, (acc || kk > 0) ? 1u : 0u);
       };
       for (int item = blockIdx.x; item < total_items && ok; item += gridDim.x) {
         const int nb = item_blocks(p, item, lane == 0);
@@ -577,7 +581,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             {
               float p0, p1;
               f2unpack(pp, p0, p1);
-              pk[j] = pack_bf16x2(p0, p1);
+              pk[j] = pack_half2<F16>(p0, p1);
             }
 #endif
             switch (j & 3) {
@@ -630,7 +634,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t* wp = reinterpret_cast<uint32_t*>(w);
 #pragma unroll
         for (int j = 0; j < 16; ++j)
-          wp[j] = pack_bf16x2(__uint_as_float(ov[2 * j]) * inv, __uint_as_float(ov[2 * j + 1]) * inv);
+          wp[j] = pack_half2<F16>(__uint_as_float(ov[2 * j]) * inv, __uint_as_float(ov[2 * j + 1]) * inv);
         if (real_row) {
 #pragma unroll
           for (int j = 0; j < 4; ++j) orow[c * 4 + j] = w[j];
@@ -669,14 +673,14 @@ EncodeTiledFn get_encode_fn() {
 }
 
 // [rows, 128] bf16 row-major viewed as a 2-D tensor; box = 64 columns x box_rows rows, 128-B swizzle.
-bool make_tmap(CUtensorMap* tm, const void* base, unsigned long long rows, unsigned box_rows) {
+bool make_tmap(CUtensorMap* tm, const void* base, unsigned long long rows, unsigned box_rows, bool f16) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {128, rows};
   cuuint64_t strides[1] = {128 * 2};
   cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+  CUresult r = enc(tm, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -690,7 +694,8 @@ cudaError_t launch_attn_fwd(const Geo& g, const AttnArgs& a, cudaStream_t stream
   if (rows >= (1ull << 31)) return cudaErrorInvalidValue;
   const unsigned kv_box = g.bs == 256 ? 128 : 64;
   CUtensorMap tq, tk, tv;
-  if (!make_tmap(&tq, a.q, rows, 128) || !make_tmap(&tk, a.k, rows, kv_box) || !make_tmap(&tv, a.v, rows, kv_box))
+  if (!make_tmap(&tq, a.q, rows, 128, a.f16) || !make_tmap(&tk, a.k, rows, kv_box, a.f16) ||
+      !make_tmap(&tv, a.v, rows, kv_box, a.f16))
     return cudaErrorInvalidValue;
   Params p;
   p.idx = a.idx;
@@ -704,7 +709,8 @@ cudaError_t launch_attn_fwd(const Geo& g, const AttnArgs& a, cudaStream_t stream
   p.g = g;
   const long long items = static_cast<long long>(a.BH) * g.NB;
   const int grid = static_cast<int>(items < a.num_sms ? items : a.num_sms);
-  auto kern = g.bs == 256 ? attn_fwd_kernel<256> : attn_fwd_kernel<64>;
+  auto kern = g.bs == 256 ? (a.f16 ? attn_fwd_kernel<256, true> : attn_fwd_kernel<256, false>)
+                          : (a.f16 ? attn_fwd_kernel<64, true> : attn_fwd_kernel<64, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTotal);
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, kSmemTotal, stream>>>(tq, tk, tv, p);

@@ -10,7 +10,7 @@ namespace vsa {
 
 // tile.cu
 cudaError_t launch_tile(const Geo& g, int B, int H, const uint16_t* x, uint16_t* xt, float* pooled,
-                        cudaStream_t stream);
+                        bool f16, cudaStream_t stream);
 cudaError_t launch_untile(const Geo& g, int B, int H, const uint16_t* xt, uint16_t* x, cudaStream_t stream);
 
 // coarse.cu
@@ -32,6 +32,7 @@ struct AttnArgs {
   float* lse;
   unsigned int* status;
   int num_sms;
+  bool f16;  // fp16 tensors (else bf16)
 };
 cudaError_t launch_attn_fwd(const Geo& g, const AttnArgs& a, cudaStream_t stream);
 

@@ -12,6 +12,7 @@
 // the slots in slot order in fp32 (the order the coarse stage is defined
 // with), then divides once by the real-token count.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -64,7 +65,7 @@ __device__ __forceinline__ int block_real_count(const Geo& g, int blk) {
   return vt * vh * vw;
 }
 
-template <int BS, bool POOL>
+template <int BS, bool POOL, bool F16>
 __global__ void __launch_bounds__(kTileThreads) tile_kernel(Geo g, int H, const uint4* __restrict__ x,
                                                             uint4* __restrict__ xt, float* __restrict__ pooled) {
   extern __shared__ __align__(16) uint4 stage[];  // [BS][16] when POOL
@@ -99,10 +100,14 @@ __global__ void __launch_bounds__(kTileThreads) tile_kernel(Geo g, int H, const 
     __syncthreads();
     if (threadIdx.x < 128) {
       const int d = threadIdx.x;
-      const __nv_bfloat16* st = reinterpret_cast<const __nv_bfloat16*>(stage);
+      const uint16_t* st = reinterpret_cast<const uint16_t*>(stage);
       float s = 0.0f;
 #pragma unroll 8
-      for (int slot = 0; slot < BS; ++slot) s = __fadd_rn(s, __bfloat162float(st[slot * 128 + d]));
+      for (int slot = 0; slot < BS; ++slot) {
+        const uint16_t h = st[slot * 128 + d];
+        const float f = F16 ? __half2float(__ushort_as_half(h)) : __uint_as_float(static_cast<uint32_t>(h) << 16);
+        s = __fadd_rn(s, f);
+      }
       const float mean = __fdiv_rn(s, static_cast<float>(block_real_count(g, blk)));
       pooled[(static_cast<long long>(bh) * g.NB + blk) * 128 + d] = mean;
     }
@@ -132,28 +137,29 @@ __global__ void __launch_bounds__(kTileThreads) untile_kernel(Geo g, int H, cons
 
 }  // namespace
 
-cudaError_t launch_tile(const Geo& g, int B, int H, const uint16_t* x, uint16_t* xt, float* pooled,
-                        cudaStream_t stream) {
+template <int BS, bool F16>
+cudaError_t launch_tile_t(const Geo& g, int B, int H, const uint4* xi, uint4* xo, float* pooled, cudaStream_t stream) {
   dim3 grid(g.NB, B * H);
-  const uint4* xi = reinterpret_cast<const uint4*>(x);
-  uint4* xo = reinterpret_cast<uint4*>(xt);
-  if (g.bs == 256) {
-    if (pooled) {
-      const int smem = 256 * 256;
-      cudaError_t e = cudaFuncSetAttribute(tile_kernel<256, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      if (e != cudaSuccess) return e;
-      tile_kernel<256, true><<<grid, kTileThreads, smem, stream>>>(g, H, xi, xo, pooled);
-    } else {
-      tile_kernel<256, false><<<grid, kTileThreads, 0, stream>>>(g, H, xi, xo, nullptr);
-    }
+  if (pooled) {
+    const int smem = BS * 256;
+    cudaError_t e = cudaFuncSetAttribute(tile_kernel<BS, true, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    tile_kernel<BS, true, F16><<<grid, kTileThreads, smem, stream>>>(g, H, xi, xo, pooled);
   } else {
-    if (pooled) {
-      tile_kernel<64, true><<<grid, kTileThreads, 64 * 256, stream>>>(g, H, xi, xo, pooled);
-    } else {
-      tile_kernel<64, false><<<grid, kTileThreads, 0, stream>>>(g, H, xi, xo, nullptr);
-    }
+    tile_kernel<BS, false, false><<<grid, kTileThreads, 0, stream>>>(g, H, xi, xo, nullptr);
   }
   return cudaGetLastError();
+}
+
+cudaError_t launch_tile(const Geo& g, int B, int H, const uint16_t* x, uint16_t* xt, float* pooled, bool f16,
+                        cudaStream_t stream) {
+  const uint4* xi = reinterpret_cast<const uint4*>(x);
+  uint4* xo = reinterpret_cast<uint4*>(xt);
+  if (g.bs == 256)
+    return f16 ? launch_tile_t<256, true>(g, B, H, xi, xo, pooled, stream)
+               : launch_tile_t<256, false>(g, B, H, xi, xo, pooled, stream);
+  return f16 ? launch_tile_t<64, true>(g, B, H, xi, xo, pooled, stream)
+             : launch_tile_t<64, false>(g, B, H, xi, xo, pooled, stream);
 }
 
 cudaError_t launch_untile(const Geo& g, int B, int H, const uint16_t* xt, uint16_t* x, cudaStream_t stream) {

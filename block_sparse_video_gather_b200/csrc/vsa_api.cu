@@ -163,14 +163,21 @@ int vsa_plan_describe(vsa_plan_t plan, int topk, char* buf, size_t n) {
   return (w < 0 || static_cast<size_t>(w) >= n) ? VSA_ERR_INVALID_ARG : VSA_OK;
 }
 
-int vsa_tile(vsa_plan_t plan, const uint16_t* x, uint16_t* x_tiled, float* pooled, int B, int H, int D,
-             vsa_stream_t stream) {
+int vsa_tile_ex(vsa_plan_t plan, vsa_dtype_t dtype, const uint16_t* x, uint16_t* x_tiled, float* pooled, int B,
+                int H, int D, vsa_stream_t stream) {
   if (!plan || !aligned16(x) || !aligned16(x_tiled)) return VSA_ERR_INVALID_ARG;
   if (pooled && !aligned16(pooled)) return VSA_ERR_INVALID_ARG;
+  if (dtype != VSA_BF16 && dtype != VSA_F16) return VSA_ERR_INVALID_ARG;
   if (int rc = check_dims(B, H, D)) return rc;
   DeviceState* ds = nullptr;
   if (int rc = device_state(&ds)) return rc;
-  return from_cuda(vsa::launch_tile(plan->g, B, H, x, x_tiled, pooled, reinterpret_cast<cudaStream_t>(stream)));
+  return from_cuda(vsa::launch_tile(plan->g, B, H, x, x_tiled, pooled, dtype == VSA_F16,
+                                    reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int vsa_tile(vsa_plan_t plan, const uint16_t* x, uint16_t* x_tiled, float* pooled, int B, int H, int D,
+             vsa_stream_t stream) {
+  return vsa_tile_ex(plan, VSA_BF16, x, x_tiled, pooled, B, H, D, stream);
 }
 
 int vsa_untile(vsa_plan_t plan, const uint16_t* x_tiled, uint16_t* x, int B, int H, int D, vsa_stream_t stream) {
@@ -206,9 +213,10 @@ int vsa_map_to_index(const uint8_t* map, int B, int H, int NQ, int NK, int32_t* 
   return from_cuda(vsa::launch_map_to_index(map, rows, NK, q2k_idx, q2k_num, reinterpret_cast<cudaStream_t>(stream)));
 }
 
-int vsa_sparse_attn_fwd(vsa_plan_t plan, const uint16_t* q, const uint16_t* k, const uint16_t* v,
-                        const int32_t* q2k_idx, const int32_t* q2k_num, int max_k, int B, int H, int D, uint16_t* o,
-                        float* lse, vsa_stream_t stream) {
+int vsa_sparse_attn_fwd_ex(vsa_plan_t plan, vsa_dtype_t dtype, const uint16_t* q, const uint16_t* k,
+                           const uint16_t* v, const int32_t* q2k_idx, const int32_t* q2k_num, int max_k, int B, int H,
+                           int D, uint16_t* o, float* lse, vsa_stream_t stream) {
+  if (dtype != VSA_BF16 && dtype != VSA_F16) return VSA_ERR_INVALID_ARG;
   if (!plan || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return VSA_ERR_INVALID_ARG;
   if (!aligned16(q2k_idx) || !aligned16(q2k_num) || max_k < 1) return VSA_ERR_INVALID_ARG;
@@ -229,7 +237,14 @@ int vsa_sparse_attn_fwd(vsa_plan_t plan, const uint16_t* q, const uint16_t* k, c
   a.lse = lse;
   a.status = ds->status;
   a.num_sms = ds->num_sms;
+  a.f16 = dtype == VSA_F16;
   return from_cuda(vsa::launch_attn_fwd(g, a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int vsa_sparse_attn_fwd(vsa_plan_t plan, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                        const int32_t* q2k_idx, const int32_t* q2k_num, int max_k, int B, int H, int D, uint16_t* o,
+                        float* lse, vsa_stream_t stream) {
+  return vsa_sparse_attn_fwd_ex(plan, VSA_BF16, q, k, v, q2k_idx, q2k_num, max_k, B, H, D, o, lse, stream);
 }
 
 int vsa_get_status(vsa_stream_t stream, int* device_status) {

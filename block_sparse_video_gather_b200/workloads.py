@@ -25,8 +25,9 @@ Recipe (stated once, used by every test and by the benchmark):
   ``offset_ar > 0`` the offsets follow an AR(1) chain along the temporal
   block index, ``o[t] = a o[t-1] + sqrt(1 - a^2) e[t]``, which keeps the
   marginal N(0, offset_std**2);
-* the fp32 values are rounded to bf16 with round-to-nearest-even and kept
-  as their raw 16-bit patterns (numpy has no bf16 dtype);
+* the fp32 values are rounded to bf16 (or, on request, IEEE fp16) with
+  round-to-nearest-even and kept as their raw 16-bit patterns (numpy has no
+  bf16 dtype);
 * block maps (map-driven workloads only): prefix query tiles select every
   tile; a video query tile selects every prefix tile plus ``map_video_k``
   distinct video tiles chosen uniformly at random; then
@@ -162,7 +163,12 @@ def _block_offsets(wl: Workload, seq: np.random.SeedSequence) -> np.ndarray:
     return e
 
 
-def _tensor(wl: Workload, noise_seq, off_seq, threads: int) -> np.ndarray:
+def f32_to_f16_bits(x: np.ndarray) -> np.ndarray:
+    """Round finite fp32 values to IEEE fp16 (nearest even); return the bit patterns."""
+    return np.ascontiguousarray(x, dtype=np.float32).astype(np.float16).view(np.uint16)
+
+
+def _tensor(wl: Workload, noise_seq, off_seq, threads: int, dtype: str = "bf16") -> np.ndarray:
     B, S, H, D = wl.B, wl.seq_len, wl.H, wl.D
     x = _normal_fill(noise_seq, B * S * H * D, threads).reshape(B, S, H, D)
     if wl.offset_std > 0.0:
@@ -178,7 +184,7 @@ def _tensor(wl: Workload, noise_seq, off_seq, threads: int) -> np.ndarray:
             # [H, T, Hg, Wg, D] -> [T, Hg, Wg, H, D], one b at a time to bound memory
             ob = off[b][:, ti][:, :, yi][:, :, :, xi]
             video += np.transpose(ob, (1, 2, 3, 0, 4))
-    return f32_to_bf16_bits(x)
+    return f32_to_f16_bits(x) if dtype == "f16" else f32_to_bf16_bits(x)
 
 
 def _block_map(wl: Workload, seq: np.random.SeedSequence) -> np.ndarray:
@@ -202,17 +208,17 @@ def _block_map(wl: Workload, seq: np.random.SeedSequence) -> np.ndarray:
     return m
 
 
-def make_inputs(wl: Workload | str, threads: int = 8) -> dict:
-    """Q, K, V as bf16 bit patterns [B, S, H, D] (uint16) and, for map-driven
-    workloads, the bool block map [B, H, NB, NB]."""
+def make_inputs(wl: Workload | str, threads: int = 8, dtype: str = "bf16") -> dict:
+    """Q, K, V as bf16 (or fp16) bit patterns [B, S, H, D] (uint16) and, for
+    map-driven workloads, the bool block map [B, H, NB, NB]."""
     if isinstance(wl, str):
         wl = WORKLOADS[wl]
     root = np.random.SeedSequence(wl.seed)
     nq, nk, nv, oq, ok, ov, mp = root.spawn(7)
     out = {
-        "q": _tensor(wl, nq, oq, threads),
-        "k": _tensor(wl, nk, ok, threads),
-        "v": _tensor(wl, nv, ov, threads),
+        "q": _tensor(wl, nq, oq, threads, dtype),
+        "k": _tensor(wl, nk, ok, threads, dtype),
+        "v": _tensor(wl, nv, ov, threads, dtype),
         "map": _block_map(wl, mp) if wl.map_driven else None,
     }
     return out

@@ -53,6 +53,11 @@ typedef struct CUstream_st *vsa_stream_t;
 /* Opaque, host-only description of one video geometry. */
 typedef struct vsa_plan *vsa_plan_t;
 
+/* 16-bit floating-point formats of Q, K, V and o ("FastVideo VSA", section
+ * "Verify routing and fallback": the kernel takes FP16 or BF16 tensors).
+ * The calls without an _ex suffix are bf16. */
+typedef enum vsa_dtype { VSA_BF16 = 0, VSA_F16 = 1 } vsa_dtype_t;
+
 enum vsa_status {
     VSA_OK = 0,
     VSA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, non-positive size */
@@ -102,7 +107,12 @@ VSA_API int vsa_plan_describe(vsa_plan_t plan, int topk, char *buf, size_t n);
 VSA_API int vsa_tile(vsa_plan_t plan, const uint16_t *x, uint16_t *x_tiled, float *pooled,
              int B, int H, int D, vsa_stream_t stream);
 
-/* Untile: x_tiled [B,H,Sp,D] -> x [B,S,H,D]; padded rows are dropped. */
+/* vsa_tile for either 16-bit format (the pooled means are fp32 either way). */
+VSA_API int vsa_tile_ex(vsa_plan_t plan, vsa_dtype_t dtype, const uint16_t *x, uint16_t *x_tiled,
+                        float *pooled, int B, int H, int D, vsa_stream_t stream);
+
+/* Untile: x_tiled [B,H,Sp,D] -> x [B,S,H,D]; padded rows are dropped.  A pure
+ * 16-bit copy: the same call serves bf16 and fp16. */
 VSA_API int vsa_untile(vsa_plan_t plan, const uint16_t *x_tiled, uint16_t *x, int B, int H, int D,
                vsa_stream_t stream);
 
@@ -145,6 +155,13 @@ VSA_API int vsa_map_to_index(const uint8_t *map, int B, int H, int NQ, int NK, i
 VSA_API int vsa_sparse_attn_fwd(vsa_plan_t plan, const uint16_t *q, const uint16_t *k, const uint16_t *v,
                         const int32_t *q2k_idx, const int32_t *q2k_num, int max_k,
                         int B, int H, int D, uint16_t *o, float *lse, vsa_stream_t stream);
+
+/* vsa_sparse_attn_fwd for either 16-bit format: q, k, v and o share dtype
+ * (fp16: the softmax numerators are rounded to fp16 for the PV product). */
+VSA_API int vsa_sparse_attn_fwd_ex(vsa_plan_t plan, vsa_dtype_t dtype, const uint16_t *q, const uint16_t *k,
+                                   const uint16_t *v, const int32_t *q2k_idx, const int32_t *q2k_num,
+                                   int max_k, int B, int H, int D, uint16_t *o, float *lse,
+                                   vsa_stream_t stream);
 
 /*
  * Synchronise `stream`, then read and clear the status word of the current

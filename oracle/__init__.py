@@ -56,15 +56,16 @@ def _load():
         lib.oracle_block_valid_counts.argtypes = geo + [P]
         lib.oracle_tile.argtypes = geo + [P, P, i, i, i]
         lib.oracle_untile.argtypes = geo + [P, P, i, i, i]
-        lib.oracle_pool.argtypes = geo + [P, P, i, i, i]
+        lib.oracle_pool.argtypes = geo + [P, P, i, i, i, i]
+        lib.oracle_half_to_f32.argtypes = [P, P, L, i]
         lib.oracle_score.argtypes = [P, P, P, i, i, i, i]
         lib.oracle_topk.argtypes = [P, i, i, i, i, P, P]
         lib.oracle_map_to_index.argtypes = [P, i, i, i, i, P, P]
-        lib.oracle_attn_rows.argtypes = geo + [P, P, P, P, P, i, i, i, i, P, L, P, P]
+        lib.oracle_attn_rows.argtypes = geo + [P, P, P, P, P, i, i, i, i, P, L, P, P, i]
         lib.oracle_max_threads.argtypes = []
         for f in ("oracle_geometry", "oracle_block_valid_counts", "oracle_tile", "oracle_untile",
                   "oracle_pool", "oracle_score", "oracle_topk", "oracle_map_to_index",
-                  "oracle_attn_rows", "oracle_max_threads"):
+                  "oracle_attn_rows", "oracle_max_threads", "oracle_half_to_f32"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -142,12 +143,23 @@ def untile(g: Geometry, xt: np.ndarray) -> np.ndarray:
     return out.view(xt.dtype)
 
 
-def pool(g: Geometry, xt: np.ndarray) -> np.ndarray:
-    """Tiled xt [B,H,Sp,D] bf16 bits -> fp32 block means [B,H,NB,D]."""
+DTYPES = {"bf16": 0, "f16": 1}
+
+
+def half_to_f32(x: np.ndarray, dtype: str = "bf16") -> np.ndarray:
+    """16-bit patterns -> fp32 values (bf16 or IEEE fp16)."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    out = np.empty(x.shape, dtype=np.float32)
+    _check(_load().oracle_half_to_f32(_ptr(x), _ptr(out), x.size, DTYPES[dtype]), "half_to_f32")
+    return out
+
+
+def pool(g: Geometry, xt: np.ndarray, dtype: str = "bf16") -> np.ndarray:
+    """Tiled xt [B,H,Sp,D] 16-bit patterns -> fp32 block means [B,H,NB,D]."""
     xt = np.ascontiguousarray(xt, dtype=np.uint16)
     B, H, Sp, D = xt.shape
     out = np.empty((B, H, g.NB, D), dtype=np.float32)
-    _check(_load().oracle_pool(*g.args, _ptr(xt), _ptr(out), B, H, D), "pool")
+    _check(_load().oracle_pool(*g.args, _ptr(xt), _ptr(out), B, H, D, DTYPES[dtype]), "pool")
     return out
 
 
@@ -182,7 +194,7 @@ def map_to_index(m: np.ndarray):
     return idx, num
 
 
-def attn_rows(g: Geometry, qt, kt, vt, idx, num, rows):
+def attn_rows(g: Geometry, qt, kt, vt, idx, num, rows, dtype: str = "bf16"):
     """fp64 attention for flat rows of [B,H,Sp]; returns (o [n,D] f64, lse [n] f64)."""
     qt = np.ascontiguousarray(qt, dtype=np.uint16)
     kt = np.ascontiguousarray(kt, dtype=np.uint16)
@@ -195,16 +207,16 @@ def attn_rows(g: Geometry, qt, kt, vt, idx, num, rows):
     o = np.empty((len(rows), D), dtype=np.float64)
     lse = np.empty(len(rows), dtype=np.float64)
     _check(_load().oracle_attn_rows(*g.args, _ptr(qt), _ptr(kt), _ptr(vt), _ptr(idx), _ptr(num),
-                                    max_k, B, H, D, _ptr(rows), len(rows), _ptr(o), _ptr(lse)),
+                                    max_k, B, H, D, _ptr(rows), len(rows), _ptr(o), _ptr(lse), DTYPES[dtype]),
            "attn_rows")
     return o, lse
 
 
-def attn(g: Geometry, qt, kt, vt, idx, num):
+def attn(g: Geometry, qt, kt, vt, idx, num, dtype: str = "bf16"):
     """fp64 attention over every row: (o [B,H,Sp,D], lse [B,H,Sp])."""
     B, H, Sp, D = qt.shape
     rows = np.arange(B * H * Sp, dtype=np.int64)
-    o, lse = attn_rows(g, qt, kt, vt, idx, num, rows)
+    o, lse = attn_rows(g, qt, kt, vt, idx, num, rows, dtype)
     return o.reshape(B, H, Sp, D), lse.reshape(B, H, Sp)
 
 
@@ -212,8 +224,8 @@ def max_threads() -> int:
     return int(_load().oracle_max_threads())
 
 
-def coarse(g: Geometry, qt, kt, k: int):
+def coarse(g: Geometry, qt, kt, k: int, dtype: str = "bf16"):
     """pool -> score -> top-k, the whole coarse stage on tiled Q and K."""
-    qbar = pool(g, qt)
-    kbar = pool(g, kt)
+    qbar = pool(g, qt, dtype)
+    kbar = pool(g, kt, dtype)
     return topk(score(qbar, kbar), k), (qbar, kbar)

@@ -37,7 +37,8 @@
  *            gives o = 0 and lse = -inf (commit log: zero-count rows).
  *  untile    inverse of tile; padded rows are dropped.
  *
- * bf16 tensors are passed as their raw 16-bit patterns.  Build with
+ * bf16 / fp16 tensors are passed as their raw 16-bit patterns (the page
+ * names "FP16 or BF16" inputs; pool and attention take a dtype flag).  Build with
  * -ffp-contract=off so that every fp32 operation rounds as written.
  */
 #include <math.h>
@@ -130,6 +131,25 @@ static float bf16_to_f32(uint16_t h) {
     return f;
 }
 
+/* IEEE binary16 -> float: sign, 5-bit exponent (bias 15), 10-bit fraction;
+ * exponent 0 is subnormal (fraction * 2^-24), exponent 31 is inf/nan. */
+static float f16_to_f32(uint16_t h) {
+    const int sign = (h >> 15) & 1, e = (h >> 10) & 31, m = h & 1023;
+    double v;
+    if (e == 0) v = ldexp((double)m, -24);
+    else if (e == 31) v = m ? NAN : INFINITY;
+    else v = ldexp(1.0 + m / 1024.0, e - 15);
+    return (float)(sign ? -v : v);
+}
+
+/* dtype 0: bf16, 1: fp16 (the kernel takes "FP16 or BF16" inputs). */
+static float half_to_f32(uint16_t h, int dtype) { return dtype ? f16_to_f32(h) : bf16_to_f32(h); }
+
+int oracle_half_to_f32(const uint16_t *x, float *y, long n, int dtype) {
+    for (long i = 0; i < n; ++i) y[i] = half_to_f32(x[i], dtype);
+    return ORACLE_OK;
+}
+
 /* tile: x [B,S,H,D] -> xt [B,H,Sp,D]; padded rows are zero. */
 int oracle_tile(int n_prefix, int T, int Hg, int Wg, int bt, int bh, int bw,
                 const uint16_t *x, uint16_t *xt, int B, int H, int D) {
@@ -166,7 +186,7 @@ int oracle_untile(int n_prefix, int T, int Hg, int Wg, int bt, int bh, int bw,
 /* pool: xt [B,H,Sp,D] -> pooled [B,H,NB,D] fp32 mean over the valid slots,
  * summed in slot order with one fp32 rounding per addition. */
 int oracle_pool(int n_prefix, int T, int Hg, int Wg, int bt, int bh, int bw,
-                const uint16_t *xt, float *pooled, int B, int H, int D) {
+                const uint16_t *xt, float *pooled, int B, int H, int D, int dtype) {
     geom_t g;
     int rc = geom_init(&g, n_prefix, T, Hg, Wg, bt, bh, bw);
     if (rc) return rc;
@@ -178,7 +198,7 @@ int oracle_pool(int n_prefix, int T, int Hg, int Wg, int bt, int bh, int bw,
                 float s = 0.0f;
                 for (int slot = 0; slot < g.bs; ++slot)
                     if (slot_is_valid(&g, blk, slot))
-                        s = s + bf16_to_f32(xt[((size_t)bhh * g.Sp + (size_t)blk * g.bs + slot) * D + d]);
+                        s = s + half_to_f32(xt[((size_t)bhh * g.Sp + (size_t)blk * g.bs + slot) * D + d], dtype);
                 pooled[((size_t)bhh * g.NB + blk) * D + d] = s / (float)count;
             }
         }
@@ -259,7 +279,7 @@ int oracle_attn_rows(int n_prefix, int T, int Hg, int Wg, int bt, int bh, int bw
                      const uint16_t *q, const uint16_t *k, const uint16_t *v,
                      const int32_t *idx, const int32_t *num, int max_k,
                      int B, int H, int D, const int64_t *rows, long n_rows,
-                     double *o_rows, double *lse_rows) {
+                     double *o_rows, double *lse_rows, int dtype) {
     geom_t g;
     int rc = geom_init(&g, n_prefix, T, Hg, Wg, bt, bh, bw);
     if (rc) return rc;
@@ -282,7 +302,7 @@ int oracle_attn_rows(int n_prefix, int T, int Hg, int Wg, int bt, int bh, int bw
             continue;
         }
         double qi[512];
-        for (int d = 0; d < D; ++d) qi[d] = bf16_to_f32(q[((size_t)bhh * g.Sp + i) * D + d]);
+        for (int d = 0; d < D; ++d) qi[d] = half_to_f32(q[((size_t)bhh * g.Sp + i) * D + d], dtype);
         double *logit = (double *)malloc(sizeof(double) * (size_t)cnt * g.bs);
         long *key = (long *)malloc(sizeof(long) * (size_t)cnt * g.bs);
         long nk = 0;
@@ -294,7 +314,7 @@ int oracle_attn_rows(int n_prefix, int T, int Hg, int Wg, int bt, int bh, int bw
                 long j = (long)kb * g.bs + slot;
                 const uint16_t *kj = k + ((size_t)bhh * g.Sp + j) * D;
                 double dot = 0.0;
-                for (int d = 0; d < D; ++d) dot += qi[d] * (double)bf16_to_f32(kj[d]);
+                for (int d = 0; d < D; ++d) dot += qi[d] * (double)half_to_f32(kj[d], dtype);
                 logit[nk] = scale * dot;
                 key[nk] = j;
                 ++nk;
@@ -310,7 +330,7 @@ int oracle_attn_rows(int n_prefix, int T, int Hg, int Wg, int bt, int bh, int bw
                 double p = exp(logit[t] - m);
                 l += p;
                 const uint16_t *vj = v + ((size_t)bhh * g.Sp + key[t]) * D;
-                for (int d = 0; d < D; ++d) o[d] += p * (double)bf16_to_f32(vj[d]);
+                for (int d = 0; d < D; ++d) o[d] += p * (double)half_to_f32(vj[d], dtype);
             }
             for (int d = 0; d < D; ++d) o[d] /= l;
             lse_rows[n] = m + log(l);

@@ -134,6 +134,10 @@ def test_calls_reject_invalid_arguments(L):
     odd = vsa.Plan(4, 4, 12, (4, 4, 4))  # 3 tiles of 64: the tile count must be even
     assert L.vsa_sparse_attn_fwd(odd.handle, F, F, F, F, F, 4, 1, 2, 128, F, F, None) == vsa.VSA_ERR_UNSUPPORTED
     assert L.vsa_get_status(None, None) == vsa.VSA_ERR_INVALID_ARG
+    # dtype must be one of the two 16-bit formats
+    assert L.vsa_tile_ex(h, 7, F, F, None, 1, 2, 128, None) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_sparse_attn_fwd_ex(h, 2, F, F, F, F, F, 4, 1, 2, 128, F, F, None) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_sparse_attn_fwd_ex(h, vsa.VSA_F16, F, F, F, F, F, 4, 1, 2, 96, F, F, None) == vsa.VSA_ERR_UNSUPPORTED
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path")
