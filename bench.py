@@ -237,6 +237,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-rows", type=int, default=2048, help="query rows per reference step")
     ap.add_argument("--dtype", default="bf16", choices=["bf16", "f16"], help="16-bit format of q, k, v, o")
+    ap.add_argument("--gate", action="store_true",
+                    help="add the gate-compress branch (pooled v, block-level attention, gated sum in untile)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -265,14 +267,15 @@ def main():
         pg.barrier()
     vsa.lib()
 
-    inp = workloads.make_inputs(wl, dtype=args.dtype)
+    inp = workloads.make_inputs(wl, dtype=args.dtype, gate=args.gate)
     tdt = torch.float16 if args.dtype == "f16" else torch.bfloat16
-    host = {n: torch.from_numpy(inp[n].view(np.int16)).view(tdt).pin_memory() for n in ("q", "k", "v")}
+    tensors = ("q", "k", "v", "gate") if args.gate else ("q", "k", "v")
+    host = {n: torch.from_numpy(inp[n].view(np.int16)).view(tdt).pin_memory() for n in tensors}
     if wl.map_driven:
         host["map"] = torch.from_numpy(inp["map"].view(np.uint8)).pin_memory()
     dev = {n: host[n].to("cuda", non_blocking=False) for n in host}
     plan = vsa.Plan.of(wl)
-    fwd = vsa.Forward(plan, wl.B, wl.H, wl.topk, dtype=tdt)
+    fwd = vsa.Forward(plan, wl.B, wl.H, wl.topk, dtype=tdt, gated=args.gate)
     o_host = torch.empty(fwd.o.shape, dtype=tdt).pin_memory()
 
     stream = torch.cuda.current_stream()
@@ -286,9 +289,17 @@ def main():
             front_ev[i].record(stream)
         vsa.tile(p, dev["q"], pooled=True, out=fwd.qt, pooled_out=fwd.qbar)
         vsa.tile(p, dev["k"], pooled=True, out=fwd.kt, pooled_out=fwd.kbar)
-        vsa.tile(p, dev["v"], out=fwd.vt)
+        if args.gate:
+            vsa.tile(p, dev["v"], pooled=True, out=fwd.vt, pooled_out=fwd.vbar)
+        else:
+            vsa.tile(p, dev["v"], out=fwd.vt)
         if wl.map_driven:
             vsa.map_to_index(dev["map"], idx_out=fwd.idx, num_out=fwd.num)
+            if args.gate:
+                vsa.coarse_compress(p, fwd.qbar, fwd.kbar, fwd.vbar, 0, o_out=fwd.oc)
+        elif args.gate:
+            vsa.coarse_compress(p, fwd.qbar, fwd.kbar, fwd.vbar, wl.topk, o_out=fwd.oc, idx_out=fwd.idx,
+                                num_out=fwd.num)
         else:
             vsa.coarse_topk(p, fwd.qbar, fwd.kbar, wl.topk, idx_out=fwd.idx, num_out=fwd.num)
         if i is not None:
@@ -296,7 +307,10 @@ def main():
         vsa.sparse_attn_fwd(p, fwd.qt, fwd.kt, fwd.vt, fwd.idx, fwd.num, o_out=fwd.ot, lse_out=fwd.lse)
         if i is not None:
             attn_ev[i][1].record(stream)
-        vsa.untile(p, fwd.ot, out=fwd.o)
+        if args.gate:
+            vsa.untile_gate(p, fwd.ot, fwd.oc, dev["gate"], out=fwd.o)
+        else:
+            vsa.untile(p, fwd.ot, out=fwd.o)
 
     def sync_all():
         torch.cuda.synchronize()
@@ -344,7 +358,7 @@ def main():
     for _ in range(3):
         for n in dev:
             dev[n].copy_(host[n], non_blocking=True)
-        fwd(dev["q"], dev["k"], dev["v"], dev.get("map"))
+        fwd(dev["q"], dev["k"], dev["v"], dev.get("map"), gate=dev.get("gate"))
         o_host.copy_(fwd.o, non_blocking=True)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sync_all()
@@ -352,7 +366,7 @@ def main():
     for _ in range(args.steps):
         for n in dev:
             dev[n].copy_(host[n], non_blocking=True)
-        fwd(dev["q"], dev["k"], dev["v"], dev.get("map"))
+        fwd(dev["q"], dev["k"], dev["v"], dev.get("map"), gate=dev.get("gate"))
         o_host.copy_(fwd.o, non_blocking=True)
     e1.record(stream)
     sync_all()
@@ -383,6 +397,7 @@ def main():
                 "l2": "inputs larger than L2: q/k/v %.0f MB and tiled q/k/v %.0f MB per step" % (
                     sum(host[n].numel() * 2 for n in ("q", "k", "v")) / 1e6, 3 * fwd.qt.numel() * 2 / 1e6),
                 "parallelism": f"replicas x{world}",
+                "gate_compress": bool(args.gate),
             },
             "roofline": {
                 "bound": "tensor", "kernel": "attn_fwd_kernel", "achieved": achieved,
@@ -395,7 +410,7 @@ def main():
             "e2e": {"value": world * flops * args.steps / e2e_elapsed / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_elapsed / args.steps * 1e3},
-            "gpu_launches": args.steps * vsa.Forward.launches_per_call,
+            "gpu_launches": args.steps * fwd.launches(wl.map_driven),
         }
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline_sample(wl)

@@ -10,6 +10,9 @@ Path ("FastVideo VSA", vLLM-Omni user guide, introduction):
     tile(q, k, v) -> coarse_topk(qbar, kbar) -> sparse_attn_fwd -> untile(o)
 or, with a caller-supplied bool block map (FastVideo commit log),
     tile -> map_to_index(map) -> sparse_attn_fwd -> untile.
+With the gate-compress branch ("FastVideo VSA", section "Checkpoint
+behavior"), v is pooled too, coarse_compress adds the block-level branch to
+the selection, and untile_gate sums the two branches under the caller's gate.
 """
 from __future__ import annotations
 
@@ -24,6 +27,7 @@ SYMBOLS = (
     "vsa_plan_create", "vsa_plan_create_prefix", "vsa_plan_destroy", "vsa_plan_sizes",
     "vsa_plan_describe", "vsa_tile", "vsa_tile_ex", "vsa_untile", "vsa_coarse_topk", "vsa_map_to_index",
     "vsa_sparse_attn_fwd", "vsa_sparse_attn_fwd_ex", "vsa_get_status", "vsa_strerror",
+    "vsa_coarse_compress", "vsa_untile_gate",
 )
 
 VSA_BF16 = 0
@@ -68,6 +72,8 @@ def lib():
         L.vsa_untile.argtypes = [P, P, P, i, i, i, P]
         L.vsa_coarse_topk.argtypes = [P, P, P, i, i, i, i, P, P, P]
         L.vsa_map_to_index.argtypes = [P, i, i, i, i, P, P, P]
+        L.vsa_coarse_compress.argtypes = [P, P, P, P, i, i, i, i, P, P, P, P]
+        L.vsa_untile_gate.argtypes = [P, i, P, P, P, P, i, i, i, P]
         L.vsa_sparse_attn_fwd.argtypes = [P, P, P, P, P, P, i, i, i, i, P, P, P]
         L.vsa_get_status.argtypes = [P, P]
         L.vsa_strerror.argtypes = [i]
@@ -196,6 +202,45 @@ def coarse_topk(plan: Plan, qbar, kbar, topk: int, idx_out=None, num_out=None):
     return idx_out, num_out
 
 
+def coarse_compress(plan: Plan, qbar, kbar, vbar, topk: int = 0, o_out=None, idx_out=None, num_out=None):
+    """Compression branch o_compress [B,H,NB,D] fp32: attention among the block
+    means.  With topk > 0 the same launch also writes the selection of
+    coarse_topk; returns (o_compress, q2k_idx, q2k_num) then, else o_compress."""
+    torch = _torch()
+    B, H, NB, D = qbar.shape
+    if o_out is None:
+        o_out = torch.empty((B, H, NB, D), dtype=torch.float32, device=qbar.device)
+    if topk > 0:
+        if idx_out is None:
+            idx_out = torch.empty((B, H, NB, topk), dtype=torch.int32, device=qbar.device)
+        if num_out is None:
+            num_out = torch.empty((B, H, NB), dtype=torch.int32, device=qbar.device)
+        ip, nump = _ptr(idx_out, torch.int32, "q2k_idx"), _ptr(num_out, torch.int32, "q2k_num")
+    else:
+        ip = nump = None
+    _check(lib().vsa_coarse_compress(plan.handle, _ptr(qbar, torch.float32, "qbar"), _ptr(kbar, torch.float32, "kbar"),
+                                     _ptr(vbar, torch.float32, "vbar"), B, H, D, topk, ip, nump,
+                                     _ptr(o_out, torch.float32, "o_compress"), _stream()), "vsa_coarse_compress")
+    return (o_out, idx_out, num_out) if topk > 0 else o_out
+
+
+def untile_gate(plan: Plan, ot, o_compress, gate, out=None):
+    """o [B,S,H,D] = untile(ot) + gate * o_compress of each token's block (gate untiled, same dtype)."""
+    torch = _torch()
+    B, H, Sp, D = ot.shape
+    code = _dtype_code(ot, "o_tiled")
+    if Sp != plan.Sp:
+        raise ValueError(f"o_tiled has {Sp} rows, plan expects {plan.Sp}")
+    if tuple(gate.shape) != (B, plan.S, H, D):
+        raise ValueError(f"gate must be [B,S,H,D] = {(B, plan.S, H, D)}, got {tuple(gate.shape)}")
+    if out is None:
+        out = torch.empty((B, plan.S, H, D), dtype=ot.dtype, device=ot.device)
+    _check(lib().vsa_untile_gate(plan.handle, code, _ptr(ot, ot.dtype, "o_tiled"),
+                                 _ptr(o_compress, torch.float32, "o_compress"), _ptr(gate, ot.dtype, "gate"),
+                                 _ptr(out, ot.dtype, "o"), B, H, D, _stream()), "vsa_untile_gate")
+    return out
+
+
 def map_to_index(block_map, idx_out=None, num_out=None):
     """Bool map [B,H,NQ,NK] -> (q2k_idx [B,H,NQ,NK] ascending then -1, q2k_num [B,H,NQ])."""
     torch = _torch()
@@ -244,11 +289,18 @@ class Forward:
     pooling, tile(v), the coarse stage (or map_to_index when a block map is
     given), the fine stage and untile(o); it returns o [B,S,H,D] and the tiled
     lse [B,H,Sp].
+
+    gated=True adds the gate-compress branch: v is pooled as well, the coarse
+    stage also computes o_compress (coarse_compress), and untile_gate replaces
+    untile, so __call__(q, k, v, gate=g) returns o_fine + g * o_compress per
+    token (g [B,S,H,D], same dtype as q).  The launch count stays six (with a
+    block map: map_to_index plus a compress-only coarse launch, seven).
     """
 
-    def __init__(self, plan: Plan, B: int, H: int, topk: int | None, device="cuda", D: int = 128, dtype=None):
+    def __init__(self, plan: Plan, B: int, H: int, topk: int | None, device="cuda", D: int = 128, dtype=None,
+                 gated: bool = False):
         torch = _torch()
-        self.plan, self.B, self.H, self.D, self.topk = plan, B, H, D, topk
+        self.plan, self.B, self.H, self.D, self.topk, self.gated = plan, B, H, D, topk, gated
         t = dict(dtype=dtype or torch.bfloat16, device=device)
         self.qt = torch.empty((B, H, plan.Sp, D), **t)
         self.kt = torch.empty((B, H, plan.Sp, D), **t)
@@ -261,19 +313,40 @@ class Forward:
         width = topk if topk is not None else plan.NB
         self.idx = torch.empty((B, H, plan.NB, width), dtype=torch.int32, device=device)
         self.num = torch.empty((B, H, plan.NB), dtype=torch.int32, device=device)
+        if gated:
+            self.vbar = torch.empty((B, H, plan.NB, D), dtype=torch.float32, device=device)
+            self.oc = torch.empty((B, H, plan.NB, D), dtype=torch.float32, device=device)
 
-    def __call__(self, q, k, v, block_map=None):
+    def __call__(self, q, k, v, block_map=None, gate=None):
         p = self.plan
+        if self.gated != (gate is not None):
+            raise ValueError("a gate is required exactly when the Forward was built with gated=True")
         tile(p, q, pooled=True, out=self.qt, pooled_out=self.qbar)
         tile(p, k, pooled=True, out=self.kt, pooled_out=self.kbar)
-        tile(p, v, out=self.vt)
+        if self.gated:
+            tile(p, v, pooled=True, out=self.vt, pooled_out=self.vbar)
+        else:
+            tile(p, v, out=self.vt)
         if block_map is None:
-            coarse_topk(p, self.qbar, self.kbar, self.topk, idx_out=self.idx, num_out=self.num)
+            if self.gated:
+                coarse_compress(p, self.qbar, self.kbar, self.vbar, self.topk, o_out=self.oc, idx_out=self.idx,
+                                num_out=self.num)
+            else:
+                coarse_topk(p, self.qbar, self.kbar, self.topk, idx_out=self.idx, num_out=self.num)
         else:
             map_to_index(block_map, idx_out=self.idx, num_out=self.num)
+            if self.gated:
+                coarse_compress(p, self.qbar, self.kbar, self.vbar, 0, o_out=self.oc)
         sparse_attn_fwd(p, self.qt, self.kt, self.vt, self.idx, self.num, o_out=self.ot, lse_out=self.lse)
-        untile(p, self.ot, out=self.o)
+        if self.gated:
+            untile_gate(p, self.ot, self.oc, gate, out=self.o)
+        else:
+            untile(p, self.ot, out=self.o)
         return self.o, self.lse
 
-    # kernels launched by one call: 3 tiles, 1 index stage, 1 attention, 1 untile
+    def launches(self, block_map: bool = False) -> int:
+        """Kernels one call launches: 3 tiles, the index stage, attention, untile
+        (+1 compress-only coarse launch when a gated call takes a block map)."""
+        return 6 + (1 if (self.gated and block_map) else 0)
+
     launches_per_call = 6

@@ -17,6 +17,15 @@
 // bitwise search (each step: count keys >= candidate, warp reduction), and
 // writes the selected ids in ascending order with ballots; ties at the
 // threshold go to the lower block index.
+//
+// Compression branch ("FastVideo VSA", section "Checkpoint behavior": the
+// learned gate_compress projection; FastVideo commit log: the gate-compress
+// branch pools per tile).  The same CTA turns its 16 score rows into softmax
+// weights over all blocks, exp(scale (s - max)), kept in shared memory in
+// place of the keys, and every thread accumulates one channel of eight rows
+// against the pooled V of the head streamed in block order:
+// o_compress[r] = sum_c w_rc vbar[c] / sum_c w_rc.  The weights come from the
+// very fp32 scores the selection ranks.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -35,13 +44,22 @@ __device__ __forceinline__ uint32_t order_key(float x) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Inverse of order_key (the score back from its key; -0 comes back as +0).
+__device__ __forceinline__ float key_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+template <bool SELECT, bool COMPRESS>
 __global__ void __launch_bounds__(kThreads) score_topk_kernel(int NB, int topk, const float* __restrict__ qbar,
                                                               const float* __restrict__ kbar,
-                                                              int32_t* __restrict__ idx, int32_t* __restrict__ num) {
+                                                              int32_t* __restrict__ idx, int32_t* __restrict__ num,
+                                                              const float* __restrict__ vbar,
+                                                              float* __restrict__ o_compress, float scale) {
   extern __shared__ __align__(16) float sm[];
   float* q_s = sm;                               // [kRows][128]
   float* k_s = q_s + kRows * 128;                // [kChunk][129]
   uint32_t* keys = reinterpret_cast<uint32_t*>(k_s + kChunk * kKStride);  // [kRows][NB]
+  float* wsum = reinterpret_cast<float*>(keys + kRows * NB);              // [kRows]
 
   const int bh = blockIdx.y;
   const int r0 = blockIdx.x * kRows;
@@ -87,7 +105,7 @@ __global__ void __launch_bounds__(kThreads) score_topk_kernel(int NB, int topk, 
 
   const int warp = tid >> 5, lane = tid & 31;
   const uint32_t lt_mask = (1u << lane) - 1u;
-  for (int r = warp; r < kRows; r += kThreads / 32) {
+  for (int r = warp; SELECT && r < kRows; r += kThreads / 32) {
     const int row = r0 + r;
     if (row >= NB) break;
     const uint32_t* key = keys + r * NB;
@@ -120,6 +138,43 @@ __global__ void __launch_bounds__(kThreads) score_topk_kernel(int NB, int topk, 
     }
     if (lane == 0) num[static_cast<long long>(bh) * NB + row] = topk;
   }
+  if (!COMPRESS) return;
+
+  __syncthreads();  // the selection is done reading the keys
+  float* w = reinterpret_cast<float*>(keys);
+  for (int r = warp; r < kRows; r += kThreads / 32) {
+    uint32_t* key = keys + r * NB;
+    uint32_t kmax = 0;
+    for (int j = lane; j < NB; j += 32) kmax = max(kmax, key[j]);
+    const float m = key_value(__reduce_max_sync(0xffffffffu, kmax));
+    float l = 0.0f;
+    for (int j = lane; j < NB; j += 32) {
+      const float e = expf((key_value(key[j]) - m) * scale);
+      w[r * NB + j] = e;  // same word, same thread: the key is read before it is overwritten
+      l += e;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+    if (lane == 0) wsum[r] = l;
+  }
+  __syncthreads();
+  const int d = tid & 127;
+  const int rbase = (tid >> 7) * (kRows / 2);  // rows rbase .. rbase + 7
+  const float* vh = vbar + static_cast<long long>(bh) * NB * 128 + d;
+  const float* wr = w + rbase * NB;
+  float acc[kRows / 2];
+#pragma unroll
+  for (int i = 0; i < kRows / 2; ++i) acc[i] = 0.0f;
+  for (int c = 0; c < NB; ++c) {
+    const float vv = __ldg(vh + static_cast<long long>(c) * 128);
+#pragma unroll
+    for (int i = 0; i < kRows / 2; ++i) acc[i] = __fmaf_rn(wr[i * NB + c], vv, acc[i]);
+  }
+#pragma unroll
+  for (int i = 0; i < kRows / 2; ++i) {
+    const int row = r0 + rbase + i;
+    if (row < NB) o_compress[(static_cast<long long>(bh) * NB + row) * 128 + d] = __fdiv_rn(acc[i], wsum[rbase + i]);
+  }
 }
 
 __global__ void __launch_bounds__(256) map_to_index_kernel(const uint8_t* __restrict__ map, long long rows, int NK,
@@ -145,18 +200,34 @@ __global__ void __launch_bounds__(256) map_to_index_kernel(const uint8_t* __rest
 }  // namespace
 
 size_t score_topk_smem_bytes(int NB) {
-  return sizeof(float) * (kRows * 128 + kChunk * kKStride) + sizeof(uint32_t) * kRows * static_cast<size_t>(NB);
+  return sizeof(float) * (kRows * 128 + kChunk * kKStride) + sizeof(uint32_t) * kRows * static_cast<size_t>(NB) +
+         sizeof(float) * kRows;
+}
+
+template <bool SELECT, bool COMPRESS>
+cudaError_t launch_coarse_t(int BH, int NB, int topk, const float* qbar, const float* kbar, int32_t* idx,
+                            int32_t* num, const float* vbar, float* o_compress, float scale, cudaStream_t stream) {
+  const size_t smem = score_topk_smem_bytes(NB);
+  cudaError_t e = cudaFuncSetAttribute(score_topk_kernel<SELECT, COMPRESS>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  dim3 grid((NB + kRows - 1) / kRows, BH);
+  score_topk_kernel<SELECT, COMPRESS><<<grid, kThreads, smem, stream>>>(NB, topk, qbar, kbar, idx, num, vbar,
+                                                                          o_compress, scale);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_score_topk(int BH, int NB, int topk, const float* qbar, const float* kbar, int32_t* idx,
                               int32_t* num, cudaStream_t stream) {
-  const size_t smem = score_topk_smem_bytes(NB);
-  cudaError_t e = cudaFuncSetAttribute(score_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  dim3 grid((NB + kRows - 1) / kRows, BH);
-  score_topk_kernel<<<grid, kThreads, smem, stream>>>(NB, topk, qbar, kbar, idx, num);
-  return cudaGetLastError();
+  return launch_coarse_t<true, false>(BH, NB, topk, qbar, kbar, idx, num, nullptr, nullptr, 0.0f, stream);
+}
+
+cudaError_t launch_coarse_compress(int BH, int NB, int topk, const float* qbar, const float* kbar,
+                                   const float* vbar, int32_t* idx, int32_t* num, float* o_compress, float scale,
+                                   cudaStream_t stream) {
+  if (topk > 0)
+    return launch_coarse_t<true, true>(BH, NB, topk, qbar, kbar, idx, num, vbar, o_compress, scale, stream);
+  return launch_coarse_t<false, true>(BH, NB, 0, qbar, kbar, nullptr, nullptr, vbar, o_compress, scale, stream);
 }
 
 cudaError_t launch_map_to_index(const uint8_t* map, long long rows, int NK, int32_t* idx, int32_t* num,

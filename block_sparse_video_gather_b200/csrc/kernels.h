@@ -12,10 +12,17 @@ namespace vsa {
 cudaError_t launch_tile(const Geo& g, int B, int H, const uint16_t* x, uint16_t* xt, float* pooled,
                         bool f16, cudaStream_t stream);
 cudaError_t launch_untile(const Geo& g, int B, int H, const uint16_t* xt, uint16_t* x, cudaStream_t stream);
+// x = x_tiled + gate * o_compress[block], untiled; gate in the untiled layout.
+cudaError_t launch_untile_gate(const Geo& g, int B, int H, const uint16_t* xt, const float* o_compress,
+                               const uint16_t* gate, uint16_t* x, bool f16, cudaStream_t stream);
 
 // coarse.cu
 cudaError_t launch_score_topk(int BH, int NB, int topk, const float* qbar, const float* kbar, int32_t* idx,
                               int32_t* num, cudaStream_t stream);
+// topk == 0: the compression branch alone (idx, num unused).
+cudaError_t launch_coarse_compress(int BH, int NB, int topk, const float* qbar, const float* kbar,
+                                   const float* vbar, int32_t* idx, int32_t* num, float* o_compress, float scale,
+                                   cudaStream_t stream);
 cudaError_t launch_map_to_index(const uint8_t* map, long long rows, int NK, int32_t* idx, int32_t* num,
                                 cudaStream_t stream);
 

@@ -135,6 +135,60 @@ __global__ void __launch_bounds__(kTileThreads) untile_kernel(Geo g, int H, cons
   }
 }
 
+// The two 16-bit values of a packed word as fp32 (exact), for either format.
+template <bool F16>
+__device__ __forceinline__ float half_lo(uint32_t w) {
+  return F16 ? __half2float(__ushort_as_half(static_cast<unsigned short>(w & 0xFFFFu))) : bf16_lo(w);
+}
+template <bool F16>
+__device__ __forceinline__ float half_hi(uint32_t w) {
+  return F16 ? __half2float(__ushort_as_half(static_cast<unsigned short>(w >> 16))) : bf16_hi(w);
+}
+
+// Untile fused with the gated sum of the compression branch:
+// x[token] = x_tiled[slot] + gate[token] * o_compress[block], one fp32 fused
+// multiply-add per channel, rounded once to the 16-bit format.  A thread owns
+// 8 channels (one 16-byte chunk) of 16 rows; its 8 o_compress values are
+// loaded once.
+template <int BS, bool F16>
+__global__ void __launch_bounds__(kTileThreads) untile_gate_kernel(Geo g, int H, const uint4* __restrict__ xt,
+                                                                   const float* __restrict__ o_compress,
+                                                                   const uint4* __restrict__ gate,
+                                                                   uint4* __restrict__ x) {
+  const int blk = blockIdx.x;
+  const int bh = blockIdx.y;
+  const int b = bh / H, h = bh - b * H;
+  const int chunk = threadIdx.x & (kRowChunks - 1);
+  const int row0 = threadIdx.x >> 4;
+  constexpr int kIters = BS / 16;
+  const long long src0 = (static_cast<long long>(bh) * g.Sp + static_cast<long long>(blk) * BS) * kRowChunks;
+  uint4 v[kIters];
+#pragma unroll
+  for (int i = 0; i < kIters; ++i) v[i] = __ldcs(xt + src0 + (row0 + 16 * i) * kRowChunks + chunk);
+  const float4* cp = reinterpret_cast<const float4*>(o_compress + (static_cast<long long>(bh) * g.NB + blk) * 128) +
+                     2 * chunk;
+  const float4 c0 = __ldg(cp), c1 = __ldg(cp + 1);
+  const float c[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+  const BlockOrigin org = block_origin(g, blk);
+#pragma unroll
+  for (int i = 0; i < kIters; ++i) {
+    const long long s = token_of_slot(g, org, row0 + 16 * i);
+    if (s < 0) continue;
+    const long long dst = ((static_cast<long long>(b) * g.S + s) * H + h) * kRowChunks + chunk;
+    const uint4 gv = __ldcs(gate + dst);
+    const uint32_t ow[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+    const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+    uint32_t r[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float lo = __fmaf_rn(half_lo<F16>(gw[k]), c[2 * k], half_lo<F16>(ow[k]));
+      const float hi = __fmaf_rn(half_hi<F16>(gw[k]), c[2 * k + 1], half_hi<F16>(ow[k]));
+      r[k] = pack_half2<F16>(lo, hi);
+    }
+    __stcs(x + dst, make_uint4(r[0], r[1], r[2], r[3]));
+  }
+}
+
 }  // namespace
 
 template <int BS, bool F16>
@@ -170,6 +224,22 @@ cudaError_t launch_untile(const Geo& g, int B, int H, const uint16_t* xt, uint16
     untile_kernel<256><<<grid, kTileThreads, 0, stream>>>(g, H, xi, xo);
   else
     untile_kernel<64><<<grid, kTileThreads, 0, stream>>>(g, H, xi, xo);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_untile_gate(const Geo& g, int B, int H, const uint16_t* xt, const float* o_compress,
+                               const uint16_t* gate, uint16_t* x, bool f16, cudaStream_t stream) {
+  dim3 grid(g.NB, B * H);
+  const uint4* xi = reinterpret_cast<const uint4*>(xt);
+  const uint4* gi = reinterpret_cast<const uint4*>(gate);
+  uint4* xo = reinterpret_cast<uint4*>(x);
+  if (g.bs == 256) {
+    if (f16) untile_gate_kernel<256, true><<<grid, kTileThreads, 0, stream>>>(g, H, xi, o_compress, gi, xo);
+    else untile_gate_kernel<256, false><<<grid, kTileThreads, 0, stream>>>(g, H, xi, o_compress, gi, xo);
+  } else {
+    if (f16) untile_gate_kernel<64, true><<<grid, kTileThreads, 0, stream>>>(g, H, xi, o_compress, gi, xo);
+    else untile_gate_kernel<64, false><<<grid, kTileThreads, 0, stream>>>(g, H, xi, o_compress, gi, xo);
+  }
   return cudaGetLastError();
 }
 

@@ -4,6 +4,7 @@
 // call launches nothing.  Device-detected errors land in one status word per
 // device (a __device__ variable of this library); vsa_get_status reads and
 // clears it.
+#include <cmath>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -200,6 +201,35 @@ int vsa_coarse_topk(vsa_plan_t plan, const float* qbar, const float* kbar, int B
   if (int rc = device_state(&ds)) return rc;
   return from_cuda(vsa::launch_score_topk(B * H, NB, topk, qbar, kbar, q2k_idx, q2k_num,
                                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int vsa_coarse_compress(vsa_plan_t plan, const float* qbar, const float* kbar, const float* vbar, int B, int H,
+                        int D, int topk, int32_t* q2k_idx, int32_t* q2k_num, float* o_compress, vsa_stream_t stream) {
+  if (!plan || !aligned16(qbar) || !aligned16(kbar) || !aligned16(vbar) || !aligned16(o_compress))
+    return VSA_ERR_INVALID_ARG;
+  if (int rc = check_dims(B, H, D)) return rc;
+  const int NB = plan->g.NB;
+  if (topk < 0 || topk > NB) return VSA_ERR_TOPK;
+  if (topk > 0 && (!aligned16(q2k_idx) || !aligned16(q2k_num))) return VSA_ERR_INVALID_ARG;
+  if (topk == 0 && (q2k_idx || q2k_num)) return VSA_ERR_INVALID_ARG;
+  if (NB > 2048) return VSA_ERR_UNSUPPORTED;  // scores of 16 rows must fit in shared memory
+  DeviceState* ds = nullptr;
+  if (int rc = device_state(&ds)) return rc;
+  const float scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+  return from_cuda(vsa::launch_coarse_compress(B * H, NB, topk, qbar, kbar, vbar, q2k_idx, q2k_num, o_compress,
+                                               scale, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int vsa_untile_gate(vsa_plan_t plan, vsa_dtype_t dtype, const uint16_t* o_tiled, const float* o_compress,
+                    const uint16_t* gate, uint16_t* o, int B, int H, int D, vsa_stream_t stream) {
+  if (dtype != VSA_BF16 && dtype != VSA_F16) return VSA_ERR_INVALID_ARG;
+  if (!plan || !aligned16(o_tiled) || !aligned16(o_compress) || !aligned16(gate) || !aligned16(o))
+    return VSA_ERR_INVALID_ARG;
+  if (int rc = check_dims(B, H, D)) return rc;
+  DeviceState* ds = nullptr;
+  if (int rc = device_state(&ds)) return rc;
+  return from_cuda(vsa::launch_untile_gate(plan->g, B, H, o_tiled, o_compress, gate, o, dtype == VSA_F16,
+                                           reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int vsa_map_to_index(const uint8_t* map, int B, int H, int NQ, int NK, int32_t* q2k_idx, int32_t* q2k_num,

@@ -28,6 +28,9 @@ Recipe (stated once, used by every test and by the benchmark):
 * the fp32 values are rounded to bf16 (or, on request, IEEE fp16) with
   round-to-nearest-even and kept as their raw 16-bit patterns (numpy has no
   bf16 dtype);
+* gate (only when asked for): i.i.d. N(0, 1) in the untiled [B, S, H, D]
+  layout, rounded the same way -- a stand-in for the output of a learned
+  gate_compress projection ("FastVideo VSA", section "Checkpoint behavior");
 * block maps (map-driven workloads only): prefix query tiles select every
   tile; a video query tile selects every prefix tile plus ``map_video_k``
   distinct video tiles chosen uniformly at random; then
@@ -208,17 +211,22 @@ def _block_map(wl: Workload, seq: np.random.SeedSequence) -> np.ndarray:
     return m
 
 
-def make_inputs(wl: Workload | str, threads: int = 8, dtype: str = "bf16") -> dict:
-    """Q, K, V as bf16 (or fp16) bit patterns [B, S, H, D] (uint16) and, for
-    map-driven workloads, the bool block map [B, H, NB, NB]."""
+def make_inputs(wl: Workload | str, threads: int = 8, dtype: str = "bf16", gate: bool = False) -> dict:
+    """Q, K, V as bf16 (or fp16) bit patterns [B, S, H, D] (uint16), for
+    map-driven workloads the bool block map [B, H, NB, NB], and on request
+    the gate [B, S, H, D] (same format)."""
     if isinstance(wl, str):
         wl = WORKLOADS[wl]
     root = np.random.SeedSequence(wl.seed)
-    nq, nk, nv, oq, ok, ov, mp = root.spawn(7)
+    # children are numbered: the eighth (gate) leaves the first seven unchanged
+    nq, nk, nv, oq, ok, ov, mp, ng = root.spawn(8)
     out = {
         "q": _tensor(wl, nq, oq, threads, dtype),
         "k": _tensor(wl, nk, ok, threads, dtype),
         "v": _tensor(wl, nv, ov, threads, dtype),
         "map": _block_map(wl, mp) if wl.map_driven else None,
     }
+    if gate:
+        g = _normal_fill(ng, wl.B * wl.seq_len * wl.H * wl.D, threads).reshape(wl.B, wl.seq_len, wl.H, wl.D)
+        out["gate"] = f32_to_f16_bits(g) if dtype == "f16" else f32_to_bf16_bits(g)
     return out

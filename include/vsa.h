@@ -129,6 +129,42 @@ VSA_API int vsa_coarse_topk(vsa_plan_t plan, const float *qbar, const float *kba
                     int topk, int32_t *q2k_idx, int32_t *q2k_num, vsa_stream_t stream);
 
 /*
+ * Coarse stage with its compression branch ("FastVideo VSA", section
+ * "Checkpoint behavior": checkpoints carry a learned gate_compress
+ * projection; FastVideo commit log: the gate-compress branch pools per tile).
+ * The pages print no formula; this call computes the plainest reading:
+ *   o_compress[r] = sum_c softmax_c(D^-1/2 qbar[r] . kbar[c]) vbar[c]
+ * over all NB blocks of each (b, h), from the fp32 scores vsa_coarse_topk
+ * ranks (fp32 weights and accumulation).
+ *   qbar, kbar, vbar : [B,H,NB,D] fp32 block means (vsa_tile / vsa_tile_ex
+ *                      with pooled output, for q, k and v)
+ *   o_compress       : [B,H,NB,D] fp32, caller-owned
+ *   topk > 0         : also the selection of vsa_coarse_topk into q2k_idx
+ *                      [B,H,NB,topk] / q2k_num [B,H,NB], same results bit for bit;
+ *   topk == 0        : the branch alone (selection from a block map);
+ *                      q2k_idx and q2k_num must then be NULL.
+ * Errors: VSA_ERR_TOPK for topk < 0 or topk > NB; VSA_ERR_INVALID_ARG for a
+ * null or misaligned pointer, or index outputs given with topk == 0;
+ * VSA_ERR_UNSUPPORTED for NB > 2048 or D != 128.
+ */
+VSA_API int vsa_coarse_compress(vsa_plan_t plan, const float *qbar, const float *kbar, const float *vbar,
+                                int B, int H, int D, int topk, int32_t *q2k_idx, int32_t *q2k_num,
+                                float *o_compress, vsa_stream_t stream);
+
+/*
+ * Untile fused with the gated sum of the two branches (same reading as
+ * vsa_coarse_compress): for every real token s of block r,
+ *   o[b,s,h,:] = o_tiled[b,h,slot(s),:] + gate[b,s,h,:] * o_compress[b,h,r,:]
+ * one fp32 fused multiply-add per channel, rounded once to dtype.
+ *   o_tiled    : tiled [B,H,Sp,D] (the fine stage's o), dtype
+ *   o_compress : [B,H,NB,D] fp32 (vsa_coarse_compress)
+ *   gate       : [B,S,H,D] dtype, untiled (the caller's gate_compress projection)
+ *   o          : [B,S,H,D] dtype, caller-owned; must not overlap the inputs
+ */
+VSA_API int vsa_untile_gate(vsa_plan_t plan, vsa_dtype_t dtype, const uint16_t *o_tiled, const float *o_compress,
+                            const uint16_t *gate, uint16_t *o, int B, int H, int D, vsa_stream_t stream);
+
+/*
  * Bool block map -> index (FastVideo commit log: map_to_index):
  * map [B,H,NQ,NK] (one byte per entry, non-zero = selected) ->
  * q2k_idx [B,H,NQ,NK] (selected ids ascending, then -1), q2k_num [B,H,NQ]

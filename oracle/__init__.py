@@ -12,7 +12,12 @@ Each step follows the statement cited in the C file's header:
   (vLLM-Omni user guide), introduction and section "Choose top-k";
 * ``map_to_index``: FastVideo commit log, examples/inference/basic/README.md;
 * ``attn_rows``: "FastVideo VSA", introduction and section "Verify routing
-  and fallback" (non-causal, scale head_size^-1/2), computed in fp64.
+  and fallback" (non-causal, scale head_size^-1/2), computed in fp64;
+* ``compress``/``gate_rows``: "FastVideo VSA", section "Checkpoint behavior"
+  (learned gate_compress projection) and the FastVideo commit log (the
+  gate-compress branch pools per tile); the formula is a reading, stated in
+  the C file: dense attention among block means, broadcast to the block's
+  tokens, times the caller's gate, added to the sparse branch.
 
 Pins (tests/test_oracle_*.py) check every function against results fixed by
 the pages or by mathematics, never against itself.
@@ -62,10 +67,13 @@ def _load():
         lib.oracle_topk.argtypes = [P, i, i, i, i, P, P]
         lib.oracle_map_to_index.argtypes = [P, i, i, i, i, P, P]
         lib.oracle_attn_rows.argtypes = geo + [P, P, P, P, P, i, i, i, i, P, L, P, P, i]
+        lib.oracle_compress.argtypes = [P, P, P, i, i, i, i, P]
+        lib.oracle_gate_rows.argtypes = geo + [P, L, P, P, P, i, i, i, P, i]
         lib.oracle_max_threads.argtypes = []
         for f in ("oracle_geometry", "oracle_block_valid_counts", "oracle_tile", "oracle_untile",
                   "oracle_pool", "oracle_score", "oracle_topk", "oracle_map_to_index",
-                  "oracle_attn_rows", "oracle_max_threads", "oracle_half_to_f32"):
+                  "oracle_attn_rows", "oracle_max_threads", "oracle_half_to_f32", "oracle_compress",
+                  "oracle_gate_rows"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -229,3 +237,29 @@ def coarse(g: Geometry, qt, kt, k: int, dtype: str = "bf16"):
     qbar = pool(g, qt, dtype)
     kbar = pool(g, kt, dtype)
     return topk(score(qbar, kbar), k), (qbar, kbar)
+
+
+def compress(qbar: np.ndarray, kbar: np.ndarray, vbar: np.ndarray) -> np.ndarray:
+    """Compression branch: fp64 attention among block means, [B,H,NB,D] each -> [B,H,NB,D] f64."""
+    qbar = np.ascontiguousarray(qbar, dtype=np.float32)
+    kbar = np.ascontiguousarray(kbar, dtype=np.float32)
+    vbar = np.ascontiguousarray(vbar, dtype=np.float32)
+    B, H, NB, D = qbar.shape
+    assert kbar.shape == qbar.shape and vbar.shape == qbar.shape
+    out = np.empty((B, H, NB, D), dtype=np.float64)
+    _check(_load().oracle_compress(_ptr(qbar), _ptr(kbar), _ptr(vbar), B, H, NB, D, _ptr(out)), "compress")
+    return out
+
+
+def gate_rows(g: Geometry, rows, o_fine, gate, o_compress, dtype: str = "bf16") -> np.ndarray:
+    """o_fine [n,D] + gate (untiled [B,S,H,D] 16-bit) * o_compress of each row's block; f64 [n,D]."""
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    o_fine = np.ascontiguousarray(o_fine, dtype=np.float64)
+    gate = np.ascontiguousarray(gate, dtype=np.uint16)
+    o_compress = np.ascontiguousarray(o_compress, dtype=np.float64)
+    B, S, H, D = gate.shape
+    assert S == g.S and o_fine.shape == (len(rows), D)
+    out = np.empty((len(rows), D), dtype=np.float64)
+    _check(_load().oracle_gate_rows(*g.args, _ptr(rows), len(rows), _ptr(o_fine), _ptr(gate), _ptr(o_compress),
+                                    B, H, D, _ptr(out), DTYPES[dtype]), "gate_rows")
+    return out

@@ -36,6 +36,15 @@
  *            Computed in double from the bf16 inputs.  A row with count 0
  *            gives o = 0 and lse = -inf (commit log: zero-count rows).
  *  untile    inverse of tile; padded rows are dropped.
+ *  compress  "FastVideo VSA", section "Checkpoint behavior", and the FastVideo
+ *            commit log (the gate-compress branch pools per tile): the pages
+ *            name a learned gate_compress projection and a branch that pools
+ *            per block but print no formula.  Reading taken: the branch is
+ *            dense attention among the pooled blocks of a head,
+ *            o_c[r] = sum_c softmax_c(scale qbar_r . kbar_c) vbar_c, in double
+ *            from the fp32 block means; every token of block r receives
+ *            o_c[r], scaled channel-wise by the caller's gate and added to the
+ *            sparse branch: o_i = o_fine_i + gate_i * o_c[block(i)].
  *
  * bf16 / fp16 tensors are passed as their raw 16-bit patterns (the page
  * names "FP16 or BF16" inputs; pool and attention take a dtype flag).  Build with
@@ -338,6 +347,84 @@ int oracle_attn_rows(int n_prefix, int T, int Hg, int Wg, int bt, int bh, int bw
         free(logit);
         free(key);
     }
+    return bad ? ORACLE_ERR_INDEX : ORACLE_OK;
+}
+
+/*
+ * compression branch: dense attention among the block means of each head.
+ *   qbar, kbar, vbar : [B,H,NB,D] fp32 block means
+ *   out              : [B,H,NB,D] double
+ * out[r] = sum_c a_rc vbar[c], a_rc = exp(z_rc - max_c z) / sum_c exp(z_rc - max_c z),
+ * z_rc = scale * sum_d qbar[r,d] kbar[c,d] (double), scale = 1/sqrt(D).
+ */
+int oracle_compress(const float *qbar, const float *kbar, const float *vbar, int B, int H, int NB, int D,
+                    double *out) {
+    if (B < 1 || H < 1 || NB < 1 || D < 1) return ORACLE_ERR_ARG;
+    const double scale = 1.0 / sqrt((double)D);
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (long row = 0; row < (long)B * H * NB; ++row) {
+        long bhh = row / NB;
+        const float *qr = qbar + (size_t)row * D;
+        const float *kh = kbar + (size_t)bhh * NB * D;
+        const float *vh = vbar + (size_t)bhh * NB * D;
+        double *o = out + (size_t)row * D;
+        double *z = (double *)malloc(sizeof(double) * (size_t)NB);
+        if (!z) { bad = 1; continue; }
+        double m = -INFINITY;
+        for (int c = 0; c < NB; ++c) {
+            double dot = 0.0;
+            for (int d = 0; d < D; ++d) dot += (double)qr[d] * (double)kh[(size_t)c * D + d];
+            z[c] = scale * dot;
+            if (z[c] > m) m = z[c];
+        }
+        for (int d = 0; d < D; ++d) o[d] = 0.0;
+        double l = 0.0;
+        for (int c = 0; c < NB; ++c) {
+            double p = exp(z[c] - m);
+            l += p;
+            for (int d = 0; d < D; ++d) o[d] += p * (double)vh[(size_t)c * D + d];
+        }
+        for (int d = 0; d < D; ++d) o[d] /= l;
+        free(z);
+    }
+    return bad ? ORACLE_ERR_NOMEM : ORACLE_OK;
+}
+
+/*
+ * gated sum of the two branches for an explicit list of real tokens.
+ *   rows       : flat indices into the tiled [B,H,Sp]; the token of each must be real
+ *   o_fine     : [n_rows, D] double, the sparse branch of those rows
+ *   gate       : untiled [B,S,H,D] 16-bit patterns (bf16 or fp16)
+ *   o_compress : [B,H,NB,D] double (oracle_compress)
+ *   out        : [n_rows, D] double = o_fine + gate * o_compress[block of the row]
+ */
+int oracle_gate_rows(int n_prefix, int T, int Hg, int Wg, int bt, int bh, int bw,
+                     const int64_t *rows, long n_rows, const double *o_fine, const uint16_t *gate,
+                     const double *o_compress, int B, int H, int D, double *out, int dtype) {
+    geom_t g;
+    int rc = geom_init(&g, n_prefix, T, Hg, Wg, bt, bh, bw);
+    if (rc) return rc;
+    if (D < 1) return ORACLE_ERR_ARG;
+    /* tiled slot -> real token index (or -1), built by walking the tokens */
+    long *token_of_slot = (long *)malloc(sizeof(long) * (size_t)g.Sp);
+    if (!token_of_slot) return ORACLE_ERR_NOMEM;
+    for (long i = 0; i < g.Sp; ++i) token_of_slot[i] = -1;
+    for (long s = 0; s < g.S; ++s) token_of_slot[tiled_pos_of_token(&g, s)] = s;
+    int bad = 0;
+    for (long n = 0; n < n_rows; ++n) {
+        long flat = rows[n];
+        long i = flat % g.Sp;
+        long bhh = flat / g.Sp;
+        long b = bhh / H, h = bhh % H;
+        long s = token_of_slot[i];
+        if (s < 0 || b >= B) { bad = 1; continue; }
+        const uint16_t *gi = gate + (((size_t)b * g.S + s) * H + h) * D;
+        const double *oc = o_compress + ((size_t)bhh * g.NB + i / g.bs) * D;
+        for (int d = 0; d < D; ++d)
+            out[(size_t)n * D + d] = o_fine[(size_t)n * D + d] + (double)half_to_f32(gi[d], dtype) * oc[d];
+    }
+    free(token_of_slot);
     return bad ? ORACLE_ERR_INDEX : ORACLE_OK;
 }
 

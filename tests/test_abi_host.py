@@ -138,6 +138,19 @@ def test_calls_reject_invalid_arguments(L):
     assert L.vsa_tile_ex(h, 7, F, F, None, 1, 2, 128, None) == vsa.VSA_ERR_INVALID_ARG
     assert L.vsa_sparse_attn_fwd_ex(h, 2, F, F, F, F, F, 4, 1, 2, 128, F, F, None) == vsa.VSA_ERR_INVALID_ARG
     assert L.vsa_sparse_attn_fwd_ex(h, vsa.VSA_F16, F, F, F, F, F, 4, 1, 2, 96, F, F, None) == vsa.VSA_ERR_UNSUPPORTED
+    # compression branch: 0 <= topk <= NB; index outputs exactly when topk > 0
+    assert L.vsa_coarse_compress(h, F, F, F, 1, 2, 128, -1, None, None, F, None) == vsa.VSA_ERR_TOPK
+    assert L.vsa_coarse_compress(h, F, F, F, 1, 2, 128, 9, F, F, F, None) == vsa.VSA_ERR_TOPK
+    assert L.vsa_coarse_compress(h, F, F, F, 1, 2, 128, 0, F, None, F, None) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_coarse_compress(h, F, F, F, 1, 2, 128, 4, None, F, F, None) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_coarse_compress(h, F, F, M, 1, 2, 128, 4, F, F, F, None) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_coarse_compress(h, F, F, F, 1, 2, 128, 4, F, F, None, None) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_coarse_compress(h, F, F, F, 1, 2, 64, 4, F, F, F, None) == vsa.VSA_ERR_UNSUPPORTED
+    # gated untile
+    assert L.vsa_untile_gate(h, 5, F, F, F, F, 1, 2, 128, None) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_untile_gate(h, vsa.VSA_BF16, F, F, M, F, 1, 2, 128, None) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_untile_gate(h, vsa.VSA_BF16, F, None, F, F, 1, 2, 128, None) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_untile_gate(h, vsa.VSA_F16, F, F, F, F, 1, 2, 96, None) == vsa.VSA_ERR_UNSUPPORTED
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path")
