@@ -237,6 +237,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-rows", type=int, default=2048, help="query rows per reference step")
     ap.add_argument("--dtype", default="bf16", choices=["bf16", "f16"], help="16-bit format of q, k, v, o")
+    ap.add_argument("--unfused", action="store_true",
+                    help="run the front end as separate tile / coarse launches instead of one")
     ap.add_argument("--gate", action="store_true",
                     help="add the gate-compress branch (pooled v, block-level attention, gated sum in untile)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -275,7 +277,7 @@ def main():
         host["map"] = torch.from_numpy(inp["map"].view(np.uint8)).pin_memory()
     dev = {n: host[n].to("cuda", non_blocking=False) for n in host}
     plan = vsa.Plan.of(wl)
-    fwd = vsa.Forward(plan, wl.B, wl.H, wl.topk, dtype=tdt, gated=args.gate)
+    fwd = vsa.Forward(plan, wl.B, wl.H, wl.topk, dtype=tdt, gated=args.gate, fused=not args.unfused)
     o_host = torch.empty(fwd.o.shape, dtype=tdt).pin_memory()
 
     stream = torch.cuda.current_stream()
@@ -284,33 +286,15 @@ def main():
     front_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
 
     def step(i=None):
-        p = fwd.plan
         if i is not None:
             front_ev[i].record(stream)
-        vsa.tile(p, dev["q"], pooled=True, out=fwd.qt, pooled_out=fwd.qbar)
-        vsa.tile(p, dev["k"], pooled=True, out=fwd.kt, pooled_out=fwd.kbar)
-        if args.gate:
-            vsa.tile(p, dev["v"], pooled=True, out=fwd.vt, pooled_out=fwd.vbar)
-        else:
-            vsa.tile(p, dev["v"], out=fwd.vt)
-        if wl.map_driven:
-            vsa.map_to_index(dev["map"], idx_out=fwd.idx, num_out=fwd.num)
-            if args.gate:
-                vsa.coarse_compress(p, fwd.qbar, fwd.kbar, fwd.vbar, 0, o_out=fwd.oc)
-        elif args.gate:
-            vsa.coarse_compress(p, fwd.qbar, fwd.kbar, fwd.vbar, wl.topk, o_out=fwd.oc, idx_out=fwd.idx,
-                                num_out=fwd.num)
-        else:
-            vsa.coarse_topk(p, fwd.qbar, fwd.kbar, wl.topk, idx_out=fwd.idx, num_out=fwd.num)
+        fwd.front(dev["q"], dev["k"], dev["v"], dev.get("map"))
         if i is not None:
             attn_ev[i][0].record(stream)
-        vsa.sparse_attn_fwd(p, fwd.qt, fwd.kt, fwd.vt, fwd.idx, fwd.num, o_out=fwd.ot, lse_out=fwd.lse)
+        fwd.fine()
         if i is not None:
             attn_ev[i][1].record(stream)
-        if args.gate:
-            vsa.untile_gate(p, fwd.ot, fwd.oc, dev["gate"], out=fwd.o)
-        else:
-            vsa.untile(p, fwd.ot, out=fwd.o)
+        fwd.back(dev.get("gate"))
 
     def sync_all():
         torch.cuda.synchronize()
@@ -398,6 +382,7 @@ def main():
                     sum(host[n].numel() * 2 for n in ("q", "k", "v")) / 1e6, 3 * fwd.qt.numel() * 2 / 1e6),
                 "parallelism": f"replicas x{world}",
                 "gate_compress": bool(args.gate),
+                "front_end": "separate launches" if args.unfused else "one launch (tile + coarse)",
             },
             "roofline": {
                 "bound": "tensor", "kernel": "attn_fwd_kernel", "achieved": achieved,

@@ -27,7 +27,7 @@ SYMBOLS = (
     "vsa_plan_create", "vsa_plan_create_prefix", "vsa_plan_destroy", "vsa_plan_sizes",
     "vsa_plan_describe", "vsa_tile", "vsa_tile_ex", "vsa_untile", "vsa_coarse_topk", "vsa_map_to_index",
     "vsa_sparse_attn_fwd", "vsa_sparse_attn_fwd_ex", "vsa_get_status", "vsa_strerror",
-    "vsa_coarse_compress", "vsa_untile_gate",
+    "vsa_coarse_compress", "vsa_untile_gate", "vsa_tile_coarse",
 )
 
 VSA_BF16 = 0
@@ -74,6 +74,7 @@ def lib():
         L.vsa_map_to_index.argtypes = [P, i, i, i, i, P, P, P]
         L.vsa_coarse_compress.argtypes = [P, P, P, P, i, i, i, i, P, P, P, P]
         L.vsa_untile_gate.argtypes = [P, i, P, P, P, P, i, i, i, P]
+        L.vsa_tile_coarse.argtypes = [P, i, P, P, P, i, i, i, i] + [P] * 11
         L.vsa_sparse_attn_fwd.argtypes = [P, P, P, P, P, P, i, i, i, i, P, P, P]
         L.vsa_get_status.argtypes = [P, P]
         L.vsa_strerror.argtypes = [i]
@@ -224,6 +225,45 @@ def coarse_compress(plan: Plan, qbar, kbar, vbar, topk: int = 0, o_out=None, idx
     return (o_out, idx_out, num_out) if topk > 0 else o_out
 
 
+def workspace(B: int, H: int, device="cuda"):
+    """The zeroed 2*B*H int32 workspace tile_coarse synchronises its CTAs with."""
+    return _torch().zeros(2 * B * H, dtype=_torch().int32, device=device)
+
+
+def tile_coarse(plan: Plan, q, k, v, topk: int, ws, gated: bool = False, out: dict | None = None):
+    """Front end in one launch: tile q, k, v with block means, then the coarse
+    stage (topk > 0) and, when gated, the compression branch.  Returns a dict
+    with qt, kt, vt, qbar, kbar (+ vbar, oc when gated; + idx, num when topk > 0);
+    tensors given in `out` are written in place."""
+    torch = _torch()
+    B, S, H, D = q.shape
+    code = _dtype_code(q, "q")
+    if S != plan.S:
+        raise ValueError(f"q has {S} tokens, plan expects {plan.S}")
+    o = dict(out or {})
+    for n in ("qt", "kt", "vt"):
+        if n not in o:
+            o[n] = torch.empty((B, H, plan.Sp, D), dtype=q.dtype, device=q.device)
+    names = ["qbar", "kbar"] + (["vbar", "oc"] if gated else [])
+    for n in names:
+        if n not in o:
+            o[n] = torch.empty((B, H, plan.NB, D), dtype=torch.float32, device=q.device)
+    if topk > 0:
+        if "idx" not in o:
+            o["idx"] = torch.empty((B, H, plan.NB, topk), dtype=torch.int32, device=q.device)
+        if "num" not in o:
+            o["num"] = torch.empty((B, H, plan.NB), dtype=torch.int32, device=q.device)
+    f32, i32 = torch.float32, torch.int32
+    _check(lib().vsa_tile_coarse(
+        plan.handle, code, _ptr(q, q.dtype, "q"), _ptr(k, q.dtype, "k"), _ptr(v, q.dtype, "v"), B, H, D, topk,
+        _ptr(o["qt"], q.dtype, "q_tiled"), _ptr(o["kt"], q.dtype, "k_tiled"), _ptr(o["vt"], q.dtype, "v_tiled"),
+        _ptr(o["qbar"], f32, "qbar"), _ptr(o["kbar"], f32, "kbar"), _ptr(o["vbar"], f32, "vbar") if gated else None,
+        _ptr(o["idx"], i32, "q2k_idx") if topk > 0 else None, _ptr(o["num"], i32, "q2k_num") if topk > 0 else None,
+        _ptr(o["oc"], f32, "o_compress") if gated else None, _ptr(ws, i32, "workspace"), _stream()),
+        "vsa_tile_coarse")
+    return o
+
+
 def untile_gate(plan: Plan, ot, o_compress, gate, out=None):
     """o [B,S,H,D] = untile(ot) + gate * o_compress of each token's block (gate untiled, same dtype)."""
     torch = _torch()
@@ -285,22 +325,26 @@ def get_status(stream=None) -> int:
 class Forward:
     """The whole forward path with its intermediates allocated once.
 
-    __call__(q, k, v[, block_map]) runs tile(q) with pooling, tile(k) with
-    pooling, tile(v), the coarse stage (or map_to_index when a block map is
+    __call__(q, k, v[, block_map]) runs the front end (tile q, k, v with
+    block means and the coarse stage, or map_to_index when a block map is
     given), the fine stage and untile(o); it returns o [B,S,H,D] and the tiled
-    lse [B,H,Sp].
+    lse [B,H,Sp].  The three stages are also callable one by one (front,
+    fine, back).
+
+    fused=True (default) runs the front end as one launch (tile_coarse);
+    fused=False as separate tile / coarse launches.
 
     gated=True adds the gate-compress branch: v is pooled as well, the coarse
-    stage also computes o_compress (coarse_compress), and untile_gate replaces
-    untile, so __call__(q, k, v, gate=g) returns o_fine + g * o_compress per
-    token (g [B,S,H,D], same dtype as q).  The launch count stays six (with a
-    block map: map_to_index plus a compress-only coarse launch, seven).
+    stage also computes o_compress, and untile_gate replaces untile, so
+    __call__(q, k, v, gate=g) returns o_fine + g * o_compress per token
+    (g [B,S,H,D], same dtype as q).
     """
 
     def __init__(self, plan: Plan, B: int, H: int, topk: int | None, device="cuda", D: int = 128, dtype=None,
-                 gated: bool = False):
+                 gated: bool = False, fused: bool = True):
         torch = _torch()
-        self.plan, self.B, self.H, self.D, self.topk, self.gated = plan, B, H, D, topk, gated
+        self.plan, self.B, self.H, self.D, self.topk = plan, B, H, D, topk
+        self.gated, self.fused = gated, fused
         t = dict(dtype=dtype or torch.bfloat16, device=device)
         self.qt = torch.empty((B, H, plan.Sp, D), **t)
         self.kt = torch.empty((B, H, plan.Sp, D), **t)
@@ -316,11 +360,21 @@ class Forward:
         if gated:
             self.vbar = torch.empty((B, H, plan.NB, D), dtype=torch.float32, device=device)
             self.oc = torch.empty((B, H, plan.NB, D), dtype=torch.float32, device=device)
+        if fused:
+            self.ws = workspace(B, H, device)
 
-    def __call__(self, q, k, v, block_map=None, gate=None):
+    def front(self, q, k, v, block_map=None):
         p = self.plan
-        if self.gated != (gate is not None):
-            raise ValueError("a gate is required exactly when the Forward was built with gated=True")
+        if self.fused:
+            out = dict(qt=self.qt, kt=self.kt, vt=self.vt, qbar=self.qbar, kbar=self.kbar)
+            if self.gated:
+                out.update(vbar=self.vbar, oc=self.oc)
+            if block_map is None:
+                out.update(idx=self.idx, num=self.num)
+            tile_coarse(p, q, k, v, self.topk if block_map is None else 0, self.ws, self.gated, out)
+            if block_map is not None:
+                map_to_index(block_map, idx_out=self.idx, num_out=self.num)
+            return
         tile(p, q, pooled=True, out=self.qt, pooled_out=self.qbar)
         tile(p, k, pooled=True, out=self.kt, pooled_out=self.kbar)
         if self.gated:
@@ -337,16 +391,26 @@ class Forward:
             map_to_index(block_map, idx_out=self.idx, num_out=self.num)
             if self.gated:
                 coarse_compress(p, self.qbar, self.kbar, self.vbar, 0, o_out=self.oc)
-        sparse_attn_fwd(p, self.qt, self.kt, self.vt, self.idx, self.num, o_out=self.ot, lse_out=self.lse)
+
+    def fine(self):
+        sparse_attn_fwd(self.plan, self.qt, self.kt, self.vt, self.idx, self.num, o_out=self.ot, lse_out=self.lse)
+
+    def back(self, gate=None):
         if self.gated:
-            untile_gate(p, self.ot, self.oc, gate, out=self.o)
+            untile_gate(self.plan, self.ot, self.oc, gate, out=self.o)
         else:
-            untile(p, self.ot, out=self.o)
+            untile(self.plan, self.ot, out=self.o)
+
+    def __call__(self, q, k, v, block_map=None, gate=None):
+        if self.gated != (gate is not None):
+            raise ValueError("a gate is required exactly when the Forward was built with gated=True")
+        self.front(q, k, v, block_map)
+        self.fine()
+        self.back(gate)
         return self.o, self.lse
 
     def launches(self, block_map: bool = False) -> int:
-        """Kernels one call launches: 3 tiles, the index stage, attention, untile
-        (+1 compress-only coarse launch when a gated call takes a block map)."""
-        return 6 + (1 if (self.gated and block_map) else 0)
-
-    launches_per_call = 6
+        """Kernels one call launches."""
+        if self.fused:
+            return 3 + (1 if block_map else 0)  # front (+ map_to_index), attention, untile
+        return 6 + (1 if (self.gated and block_map) else 0)  # 3 tiles, index stage (+compress), attention, untile

@@ -1,0 +1,296 @@
+// items.cuh -- the per-CTA work items of the front end, shared by the
+// standalone tile / coarse kernels and the fused front-end kernel: tiling
+// (with block means) of one (b*h, block), and scoring + selection (+ the
+// compression branch) of 8 query blocks of one head.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+
+namespace vsa {
+namespace items {
+
+constexpr int kTileThreads = 256;
+constexpr int kRowChunks = 16;  // 16 B chunks per 256 B row (D = 128)
+
+// Where the tokens of one block live in the untiled sequence.  Computed
+// once per CTA (three divisions); each slot then costs shifts and two
+// multiply-adds.  Slot (lt, lh, lw) of a video block sits at grid point
+// (t0 + lt, y0 + lh, x0 + lw); slot s of a prefix tile is token p0 + s.
+struct BlockOrigin {
+  bool prefix;
+  long long p0;   // first token of a prefix tile
+  int plim;       // real tokens of a prefix tile
+  int t0, y0, x0; // grid origin of a video block
+};
+
+__device__ __forceinline__ BlockOrigin block_origin(const Geo& g, int blk) {
+  BlockOrigin o;
+  o.prefix = blk < g.n_pre;
+  o.p0 = static_cast<long long>(blk) * g.bs;
+  o.plim = g.n_prefix - blk * g.bs;
+  const int vb = blk - g.n_pre;
+  const int bW = vb % g.nW, bH = (vb / g.nW) % g.nH, bT = vb / (g.nW * g.nH);
+  o.t0 = bT * g.bt;
+  o.y0 = bH * g.bh;
+  o.x0 = bW * g.bw;
+  return o;
+}
+
+// Token index of slot `slot` of the block, or -1 for a padded slot.
+__device__ __forceinline__ long long token_of_slot(const Geo& g, const BlockOrigin& o, int slot) {
+  if (o.prefix) return slot < o.plim ? o.p0 + slot : -1;
+  const int x = o.x0 + (slot & (g.bw - 1));
+  const int y = o.y0 + ((slot >> g.lbw) & (g.bh - 1));
+  const int t = o.t0 + (slot >> (g.lbw + g.lbh));
+  if (t >= g.T || y >= g.Hg || x >= g.Wg) return -1;
+  return g.n_prefix + (static_cast<long long>(t) * g.Hg + y) * g.Wg + x;
+}
+
+__device__ __forceinline__ int block_real_count(const Geo& g, int blk) {
+  if (blk < g.n_pre) return min(g.bs, g.n_prefix - blk * g.bs);
+  int vt, vh, vw;
+  video_block_extent(g, blk - g.n_pre, vt, vh, vw);
+  return vt * vh * vw;
+}
+
+// Tile one (b*h, block): copy its BS token rows into the tiled layout
+// (padding zero-filled) and, with POOL, write the block's fp32 channel means.
+// `stage` is BS * 256 bytes of shared memory (used only with POOL).
+template <int BS, bool POOL, bool F16>
+__device__ __forceinline__ void tile_item(const Geo& g, int H, int blk, int bh, const uint4* __restrict__ x,
+                                          uint4* __restrict__ xt, float* __restrict__ pooled, uint4* stage) {
+  const int b = bh / H, h = bh - b * H;
+  const int chunk = threadIdx.x & (kRowChunks - 1);
+  const int row0 = threadIdx.x >> 4;  // 0..15
+  constexpr int kIters = BS / 16;
+
+  const BlockOrigin org = block_origin(g, blk);
+  uint4 v[kIters];
+#pragma unroll
+  for (int i = 0; i < kIters; ++i) {
+    const int slot = row0 + 16 * i;
+    const long long s = token_of_slot(g, org, slot);
+    if (s >= 0) {
+      const long long src = ((static_cast<long long>(b) * g.S + s) * H + h) * kRowChunks + chunk;
+      v[i] = __ldcs(x + src);
+    } else {
+      v[i] = make_uint4(0, 0, 0, 0);
+    }
+  }
+  const long long dst0 = (static_cast<long long>(bh) * g.Sp + static_cast<long long>(blk) * BS) * kRowChunks;
+#pragma unroll
+  for (int i = 0; i < kIters; ++i) {
+    const int slot = row0 + 16 * i;
+    xt[dst0 + slot * kRowChunks + chunk] = v[i];
+    if (POOL) stage[slot * kRowChunks + chunk] = v[i];
+  }
+  if (POOL) {
+    __syncthreads();
+    if (threadIdx.x < 128) {
+      const int d = threadIdx.x;
+      const uint16_t* st = reinterpret_cast<const uint16_t*>(stage);
+      float s = 0.0f;
+#pragma unroll 8
+      for (int slot = 0; slot < BS; ++slot) {
+        const uint16_t h = st[slot * 128 + d];
+        const float f = F16 ? __half2float(__ushort_as_half(h)) : __uint_as_float(static_cast<uint32_t>(h) << 16);
+        s = __fadd_rn(s, f);
+      }
+      const float mean = __fdiv_rn(s, static_cast<float>(block_real_count(g, blk)));
+      pooled[(static_cast<long long>(bh) * g.NB + blk) * 128 + d] = mean;
+    }
+  }
+}
+
+
+constexpr int kRows = 8;       // query blocks per score item (one per warp in the selection)
+constexpr int kChunk = 64;     // key blocks per shared-memory chunk
+constexpr int kKStride = 132;  // row stride (floats): 16-byte rows, float4 reads of a warp take 4 wavefronts
+constexpr int kThreads = 256;
+constexpr int kGroups = kThreads / kChunk;      // row groups (4)
+constexpr int kRowsPerGroup = kRows / kGroups;  // rows per thread (2)
+
+// fp32 loads: read-only path for inputs of the launch, L2-only for data
+// that other CTAs of the same launch wrote.
+template <bool COHERENT>
+__device__ __forceinline__ float ldf(const float* p) {
+  return COHERENT ? __ldcg(p) : __ldg(p);
+}
+
+// 16-byte global -> shared copy through L2 (cp.async.cg); a source size of
+// 0 writes zeros.  All copies of a thread stay in flight until cp_async_wait.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(gsrc),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+}
+
+__host__ __device__ constexpr size_t score_smem_bytes_c(int NB) {
+  return sizeof(float) * (kRows * 128 + kChunk * kKStride) + sizeof(uint32_t) * kRows * static_cast<size_t>(NB) +
+         sizeof(float) * kRows;
+}
+inline size_t score_smem_bytes(int NB) { return score_smem_bytes_c(NB); }
+
+// Monotone map fp32 -> uint32 (larger score -> larger key); -0 counts as +0.
+__device__ __forceinline__ uint32_t order_key(float x) {
+  uint32_t u = __float_as_uint(x == 0.0f ? 0.0f : x);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Inverse of order_key (the score back from its key; -0 comes back as +0).
+__device__ __forceinline__ float key_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+// Scores, selection and compression branch of query blocks r0 .. r0+7 of
+// head bh.  `sm` is score_smem_bytes(NB) of shared memory.  COHERENT: the
+// block means were written by other CTAs of the same launch, so they are
+// read through L2 only (never the read-only path).
+//
+// A thread owns one key block of the current chunk and kRowsPerGroup query
+// blocks; each score is one fused-multiply-add chain over the channels in
+// order (four channels per step: one 16-byte load of the key row, one
+// broadcast 16-byte load per query row).  Block means reach shared memory by
+// cp.async through L2, every copy of a chunk in flight at once.
+template <bool SELECT, bool COMPRESS, bool COHERENT>
+__device__ __forceinline__ void score_item(int NB, int topk, int r0, int bh, const float* qbar, const float* kbar,
+                                           int32_t* __restrict__ idx, int32_t* __restrict__ num, const float* vbar,
+                                           float* __restrict__ o_compress, float scale, float* sm) {
+  float* q_s = sm;                               // [kRows][128]
+  float* k_s = q_s + kRows * 128;                // [kChunk][kKStride]
+  uint32_t* keys = reinterpret_cast<uint32_t*>(k_s + kChunk * kKStride);  // [kRows][NB]
+  float* wsum = reinterpret_cast<float*>(keys + kRows * NB);              // [kRows]
+
+  const int tid = threadIdx.x;
+  const float* qh = qbar + static_cast<long long>(bh) * NB * 128;
+  const float* kh = kbar + static_cast<long long>(bh) * NB * 128;
+
+  static_assert(kRows * 128 == 4 * kThreads, "one 16-byte copy of query means per thread");
+  {
+    const int i = 4 * tid;
+    const bool ok = r0 + (i >> 7) < NB;
+    cp_async16(q_s + i, ok ? qh + static_cast<long long>(r0) * 128 + i : qh, ok);  // rows past NB read as 0
+  }
+
+  constexpr int kCopies = kChunk * 128 / (4 * kThreads);  // 16-byte copies per thread per chunk (8)
+  const int j_loc = tid % kChunk;
+  const int rg = tid / kChunk;  // owns query rows rg*kRowsPerGroup ..
+  for (int c0 = 0; c0 < NB; c0 += kChunk) {
+    const int nrow = min(kChunk, NB - c0);
+    __syncthreads();  // the previous chunk is no longer read
+#pragma unroll
+    for (int it = 0; it < kCopies; ++it) {
+      const int i4 = tid + it * kThreads;  // 16-byte unit in the chunk; 32 per key row
+      const int jr = i4 >> 5;
+      if (jr < nrow) cp_async16(k_s + jr * kKStride + 4 * (i4 & 31), kh + static_cast<long long>(c0) * 128 + 4 * i4, true);
+    }
+    cp_async_wait();
+    __syncthreads();
+    if (j_loc < nrow) {
+      float acc[kRowsPerGroup];
+#pragma unroll
+      for (int r = 0; r < kRowsPerGroup; ++r) acc[r] = 0.0f;
+      const float* kr = k_s + j_loc * kKStride;
+      const float* q0 = q_s + (rg * kRowsPerGroup) * 128;
+#pragma unroll 4
+      for (int d = 0; d < 128; d += 4) {
+        const float4 kv = *reinterpret_cast<const float4*>(kr + d);
+#pragma unroll
+        for (int r = 0; r < kRowsPerGroup; ++r) {
+          const float4 qv = *reinterpret_cast<const float4*>(q0 + r * 128 + d);
+          acc[r] = __fmaf_rn(qv.x, kv.x, acc[r]);
+          acc[r] = __fmaf_rn(qv.y, kv.y, acc[r]);
+          acc[r] = __fmaf_rn(qv.z, kv.z, acc[r]);
+          acc[r] = __fmaf_rn(qv.w, kv.w, acc[r]);
+        }
+      }
+      const int j = c0 + j_loc;
+#pragma unroll
+      for (int r = 0; r < kRowsPerGroup; ++r) keys[(rg * kRowsPerGroup + r) * NB + j] = order_key(acc[r]);
+    }
+  }
+  __syncthreads();
+
+  const int warp = tid >> 5, lane = tid & 31;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  for (int r = warp; SELECT && r < kRows; r += kThreads / 32) {
+    const int row = r0 + r;
+    if (row >= NB) break;
+    const uint32_t* key = keys + r * NB;
+    // k-th largest key: the largest v with #{key >= v} >= topk
+    uint32_t tau = 0;
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = tau | (1u << bit);
+      unsigned cnt = 0;
+      for (int j = lane; j < NB; j += 32) cnt += key[j] >= cand;
+      cnt = __reduce_add_sync(0xffffffffu, cnt);
+      if (cnt >= static_cast<unsigned>(topk)) tau = cand;
+    }
+    unsigned gt = 0;
+    for (int j = lane; j < NB; j += 32) gt += key[j] > tau;
+    gt = __reduce_add_sync(0xffffffffu, gt);
+    const int need = topk - static_cast<int>(gt);  // ties at tau to take, lowest ids first
+    int32_t* out = idx + (static_cast<long long>(bh) * NB + row) * topk;
+    int pos = 0, ties = 0;
+    for (int base = 0; base < NB; base += 32) {
+      const int j = base + lane;
+      const uint32_t u = (j < NB) ? key[j] : 0u;
+      const bool is_gt = (j < NB) && u > tau;
+      const bool is_eq = (j < NB) && u == tau;
+      const uint32_t eq = __ballot_sync(0xffffffffu, is_eq);
+      const bool sel = is_gt || (is_eq && ties + __popc(eq & lt_mask) < need);
+      const uint32_t sm_ = __ballot_sync(0xffffffffu, sel);
+      if (sel) out[pos + __popc(sm_ & lt_mask)] = j;
+      pos += __popc(sm_);
+      ties += __popc(eq);
+    }
+    if (lane == 0) num[static_cast<long long>(bh) * NB + row] = topk;
+  }
+  if (!COMPRESS) return;
+
+  __syncthreads();  // the selection is done reading the keys
+  float* w = reinterpret_cast<float*>(keys);
+  for (int r = warp; r < kRows; r += kThreads / 32) {
+    uint32_t* key = keys + r * NB;
+    uint32_t kmax = 0;
+    for (int j = lane; j < NB; j += 32) kmax = max(kmax, key[j]);
+    const float m = key_value(__reduce_max_sync(0xffffffffu, kmax));
+    float l = 0.0f;
+    for (int j = lane; j < NB; j += 32) {
+      const float e = expf((key_value(key[j]) - m) * scale);
+      w[r * NB + j] = e;  // same word, same thread: the key is read before it is overwritten
+      l += e;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+    if (lane == 0) wsum[r] = l;
+  }
+  __syncthreads();
+  const int d = tid & 127;
+  const int rbase = (tid >> 7) * (kRows / 2);  // rows rbase .. rbase + kRows/2 - 1
+  const float* vh = vbar + static_cast<long long>(bh) * NB * 128 + d;
+  const float* wr = w + rbase * NB;
+  float acc[kRows / 2];
+#pragma unroll
+  for (int i = 0; i < kRows / 2; ++i) acc[i] = 0.0f;
+  for (int c = 0; c < NB; ++c) {
+    const float vv = ldf<COHERENT>(vh + static_cast<long long>(c) * 128);
+#pragma unroll
+    for (int i = 0; i < kRows / 2; ++i) acc[i] = __fmaf_rn(wr[i * NB + c], vv, acc[i]);
+  }
+#pragma unroll
+  for (int i = 0; i < kRows / 2; ++i) {
+    const int row = r0 + rbase + i;
+    if (row < NB) o_compress[(static_cast<long long>(bh) * NB + row) * 128 + d] = __fdiv_rn(acc[i], wsum[rbase + i]);
+  }
+}
+
+
+}  // namespace items
+}  // namespace vsa

@@ -26,6 +26,23 @@ cudaError_t launch_coarse_compress(int BH, int NB, int topk, const float* qbar, 
 cudaError_t launch_map_to_index(const uint8_t* map, long long rows, int NK, int32_t* idx, int32_t* num,
                                 cudaStream_t stream);
 
+// front.cu: tile q, k, v (+ block means) and the coarse stage in one launch.
+struct FrontArgs {
+  Geo g;
+  int H, BH;
+  int topk;                        // 0: no selection
+  const uint4 *q, *k, *v;          // [B,S,H,D] 16-bit
+  uint4 *qt, *kt, *vt;             // [B,H,Sp,D]
+  float *qbar, *kbar, *vbar;       // [B,H,NB,D]; vbar null: no compression branch
+  int32_t *idx, *num;              // selection (topk > 0)
+  float* o_compress;               // [B,H,NB,D] (with vbar)
+  float scale;                     // D^-1/2
+  int *arrive, *done;              // [B*H] each, zero on entry, zero again on exit
+  unsigned int* status;
+  bool f16;
+};
+cudaError_t launch_front(const FrontArgs& a, cudaStream_t stream);
+
 // attn_fwd.cu
 struct AttnArgs {
   const uint16_t* q;

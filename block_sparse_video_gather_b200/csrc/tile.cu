@@ -15,103 +15,21 @@
 #include <cuda_fp16.h>
 
 #include "common.cuh"
+#include "items.cuh"
 #include "kernels.h"
 
 namespace vsa {
 
 namespace {
 
-constexpr int kTileThreads = 256;
-constexpr int kRowChunks = 16;  // 16 B chunks per 256 B row (D = 128)
+using namespace items;
 
-// Where the tokens of one block live in the untiled sequence.  Computed
-// once per CTA (three divisions); each slot then costs shifts and two
-// multiply-adds.  Slot (lt, lh, lw) of a video block sits at grid point
-// (t0 + lt, y0 + lh, x0 + lw); slot s of a prefix tile is token p0 + s.
-struct BlockOrigin {
-  bool prefix;
-  long long p0;   // first token of a prefix tile
-  int plim;       // real tokens of a prefix tile
-  int t0, y0, x0; // grid origin of a video block
-};
-
-__device__ __forceinline__ BlockOrigin block_origin(const Geo& g, int blk) {
-  BlockOrigin o;
-  o.prefix = blk < g.n_pre;
-  o.p0 = static_cast<long long>(blk) * g.bs;
-  o.plim = g.n_prefix - blk * g.bs;
-  const int vb = blk - g.n_pre;
-  const int bW = vb % g.nW, bH = (vb / g.nW) % g.nH, bT = vb / (g.nW * g.nH);
-  o.t0 = bT * g.bt;
-  o.y0 = bH * g.bh;
-  o.x0 = bW * g.bw;
-  return o;
-}
-
-// Token index of slot `slot` of the block, or -1 for a padded slot.
-__device__ __forceinline__ long long token_of_slot(const Geo& g, const BlockOrigin& o, int slot) {
-  if (o.prefix) return slot < o.plim ? o.p0 + slot : -1;
-  const int x = o.x0 + (slot & (g.bw - 1));
-  const int y = o.y0 + ((slot >> g.lbw) & (g.bh - 1));
-  const int t = o.t0 + (slot >> (g.lbw + g.lbh));
-  if (t >= g.T || y >= g.Hg || x >= g.Wg) return -1;
-  return g.n_prefix + (static_cast<long long>(t) * g.Hg + y) * g.Wg + x;
-}
-
-__device__ __forceinline__ int block_real_count(const Geo& g, int blk) {
-  if (blk < g.n_pre) return min(g.bs, g.n_prefix - blk * g.bs);
-  int vt, vh, vw;
-  video_block_extent(g, blk - g.n_pre, vt, vh, vw);
-  return vt * vh * vw;
-}
 
 template <int BS, bool POOL, bool F16>
 __global__ void __launch_bounds__(kTileThreads) tile_kernel(Geo g, int H, const uint4* __restrict__ x,
                                                             uint4* __restrict__ xt, float* __restrict__ pooled) {
   extern __shared__ __align__(16) uint4 stage[];  // [BS][16] when POOL
-  const int blk = blockIdx.x;
-  const int bh = blockIdx.y;
-  const int b = bh / H, h = bh - b * H;
-  const int chunk = threadIdx.x & (kRowChunks - 1);
-  const int row0 = threadIdx.x >> 4;  // 0..15
-  constexpr int kIters = BS / 16;
-
-  const BlockOrigin org = block_origin(g, blk);
-  uint4 v[kIters];
-#pragma unroll
-  for (int i = 0; i < kIters; ++i) {
-    const int slot = row0 + 16 * i;
-    const long long s = token_of_slot(g, org, slot);
-    if (s >= 0) {
-      const long long src = ((static_cast<long long>(b) * g.S + s) * H + h) * kRowChunks + chunk;
-      v[i] = __ldcs(x + src);
-    } else {
-      v[i] = make_uint4(0, 0, 0, 0);
-    }
-  }
-  const long long dst0 = (static_cast<long long>(bh) * g.Sp + static_cast<long long>(blk) * BS) * kRowChunks;
-#pragma unroll
-  for (int i = 0; i < kIters; ++i) {
-    const int slot = row0 + 16 * i;
-    xt[dst0 + slot * kRowChunks + chunk] = v[i];
-    if (POOL) stage[slot * kRowChunks + chunk] = v[i];
-  }
-  if (POOL) {
-    __syncthreads();
-    if (threadIdx.x < 128) {
-      const int d = threadIdx.x;
-      const uint16_t* st = reinterpret_cast<const uint16_t*>(stage);
-      float s = 0.0f;
-#pragma unroll 8
-      for (int slot = 0; slot < BS; ++slot) {
-        const uint16_t h = st[slot * 128 + d];
-        const float f = F16 ? __half2float(__ushort_as_half(h)) : __uint_as_float(static_cast<uint32_t>(h) << 16);
-        s = __fadd_rn(s, f);
-      }
-      const float mean = __fdiv_rn(s, static_cast<float>(block_real_count(g, blk)));
-      pooled[(static_cast<long long>(bh) * g.NB + blk) * 128 + d] = mean;
-    }
-  }
+  tile_item<BS, POOL, F16>(g, H, blockIdx.x, blockIdx.y, x, xt, pooled, stage);
 }
 
 template <int BS>

@@ -196,7 +196,7 @@ int vsa_coarse_topk(vsa_plan_t plan, const float* qbar, const float* kbar, int B
   if (int rc = check_dims(B, H, D)) return rc;
   const int NB = plan->g.NB;
   if (topk < 1 || topk > NB) return VSA_ERR_TOPK;
-  if (NB > 2048) return VSA_ERR_UNSUPPORTED;  // scores of 16 rows must fit in shared memory
+  if (NB > 2048) return VSA_ERR_UNSUPPORTED;  // scores of 8 rows must fit in shared memory
   DeviceState* ds = nullptr;
   if (int rc = device_state(&ds)) return rc;
   return from_cuda(vsa::launch_score_topk(B * H, NB, topk, qbar, kbar, q2k_idx, q2k_num,
@@ -212,12 +212,55 @@ int vsa_coarse_compress(vsa_plan_t plan, const float* qbar, const float* kbar, c
   if (topk < 0 || topk > NB) return VSA_ERR_TOPK;
   if (topk > 0 && (!aligned16(q2k_idx) || !aligned16(q2k_num))) return VSA_ERR_INVALID_ARG;
   if (topk == 0 && (q2k_idx || q2k_num)) return VSA_ERR_INVALID_ARG;
-  if (NB > 2048) return VSA_ERR_UNSUPPORTED;  // scores of 16 rows must fit in shared memory
+  if (NB > 2048) return VSA_ERR_UNSUPPORTED;  // scores of 8 rows must fit in shared memory
   DeviceState* ds = nullptr;
   if (int rc = device_state(&ds)) return rc;
   const float scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
   return from_cuda(vsa::launch_coarse_compress(B * H, NB, topk, qbar, kbar, vbar, q2k_idx, q2k_num, o_compress,
                                                scale, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int vsa_tile_coarse(vsa_plan_t plan, vsa_dtype_t dtype, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                    int B, int H, int D, int topk, uint16_t* q_tiled, uint16_t* k_tiled, uint16_t* v_tiled,
+                    float* qbar, float* kbar, float* vbar, int32_t* q2k_idx, int32_t* q2k_num, float* o_compress,
+                    int32_t* workspace, vsa_stream_t stream) {
+  if (dtype != VSA_BF16 && dtype != VSA_F16) return VSA_ERR_INVALID_ARG;
+  if (!plan || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q_tiled) || !aligned16(k_tiled) ||
+      !aligned16(v_tiled) || !aligned16(qbar) || !aligned16(kbar) || !aligned16(workspace))
+    return VSA_ERR_INVALID_ARG;
+  if ((vbar == nullptr) != (o_compress == nullptr)) return VSA_ERR_INVALID_ARG;
+  if (vbar && (!aligned16(vbar) || !aligned16(o_compress))) return VSA_ERR_INVALID_ARG;
+  if (int rc = check_dims(B, H, D)) return rc;
+  const int NB = plan->g.NB;
+  if (topk < 0 || topk > NB) return VSA_ERR_TOPK;
+  if (topk > 0 && (!aligned16(q2k_idx) || !aligned16(q2k_num))) return VSA_ERR_INVALID_ARG;
+  if (topk == 0 && (q2k_idx || q2k_num)) return VSA_ERR_INVALID_ARG;
+  if (NB > 2048) return VSA_ERR_UNSUPPORTED;  // scores of 8 rows must fit in shared memory
+  DeviceState* ds = nullptr;
+  if (int rc = device_state(&ds)) return rc;
+  vsa::FrontArgs a;
+  a.g = plan->g;
+  a.H = H;
+  a.BH = B * H;
+  a.topk = topk;
+  a.q = reinterpret_cast<const uint4*>(q);
+  a.k = reinterpret_cast<const uint4*>(k);
+  a.v = reinterpret_cast<const uint4*>(v);
+  a.qt = reinterpret_cast<uint4*>(q_tiled);
+  a.kt = reinterpret_cast<uint4*>(k_tiled);
+  a.vt = reinterpret_cast<uint4*>(v_tiled);
+  a.qbar = qbar;
+  a.kbar = kbar;
+  a.vbar = vbar;
+  a.idx = q2k_idx;
+  a.num = q2k_num;
+  a.o_compress = o_compress;
+  a.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+  a.arrive = workspace;
+  a.done = workspace + static_cast<long long>(B) * H;
+  a.status = ds->status;
+  a.f16 = dtype == VSA_F16;
+  return from_cuda(vsa::launch_front(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int vsa_untile_gate(vsa_plan_t plan, vsa_dtype_t dtype, const uint16_t* o_tiled, const float* o_compress,

@@ -165,6 +165,34 @@ VSA_API int vsa_untile_gate(vsa_plan_t plan, vsa_dtype_t dtype, const uint16_t *
                             const uint16_t *gate, uint16_t *o, int B, int H, int D, vsa_stream_t stream);
 
 /*
+ * The front end in one launch: vsa_tile_ex of q, k and v (block means of q
+ * and k always, of v when vbar is not NULL) followed, per head, by the coarse
+ * stage of vsa_coarse_topk (topk > 0) and/or the compression branch of
+ * vsa_coarse_compress (vbar and o_compress not NULL).  Every output is bit
+ * for bit the one the separate calls write.  topk == 0 with vbar == NULL
+ * tiles only (selection from a block map).
+ *   q, k, v                : [B,S,H,D] dtype
+ *   q_tiled, k_tiled, v_tiled : [B,H,Sp,D] dtype, caller-owned
+ *   qbar, kbar (, vbar)    : [B,H,NB,D] fp32, caller-owned
+ *   q2k_idx, q2k_num       : as vsa_coarse_topk (NULL when topk == 0)
+ *   o_compress             : [B,H,NB,D] fp32 (NULL exactly when vbar is NULL)
+ *   workspace              : 2*B*H int32 of device memory, zero before the
+ *                            first call; each call leaves it zero unless it
+ *                            reports VSA_ERR_TIMEOUT, after which the caller
+ *                            zeroes it again.  Calls that share a workspace
+ *                            must not run concurrently.
+ * The scoring of a head waits (at most 2 s) for the tiling of that head
+ * inside the same launch; on expiry the status word holds VSA_ERR_TIMEOUT.
+ * Errors: as vsa_tile_ex and vsa_coarse_compress; VSA_ERR_INVALID_ARG for a
+ * null or misaligned workspace.
+ */
+VSA_API int vsa_tile_coarse(vsa_plan_t plan, vsa_dtype_t dtype, const uint16_t *q, const uint16_t *k,
+                            const uint16_t *v, int B, int H, int D, int topk, uint16_t *q_tiled,
+                            uint16_t *k_tiled, uint16_t *v_tiled, float *qbar, float *kbar, float *vbar,
+                            int32_t *q2k_idx, int32_t *q2k_num, float *o_compress, int32_t *workspace,
+                            vsa_stream_t stream);
+
+/*
  * Bool block map -> index (FastVideo commit log: map_to_index):
  * map [B,H,NQ,NK] (one byte per entry, non-zero = selected) ->
  * q2k_idx [B,H,NQ,NK] (selected ids ascending, then -1), q2k_num [B,H,NQ]

@@ -146,6 +146,17 @@ def test_calls_reject_invalid_arguments(L):
     assert L.vsa_coarse_compress(h, F, F, M, 1, 2, 128, 4, F, F, F, None) == vsa.VSA_ERR_INVALID_ARG
     assert L.vsa_coarse_compress(h, F, F, F, 1, 2, 128, 4, F, F, None, None) == vsa.VSA_ERR_INVALID_ARG
     assert L.vsa_coarse_compress(h, F, F, F, 1, 2, 64, 4, F, F, F, None) == vsa.VSA_ERR_UNSUPPORTED
+    # one-launch front end: workspace required; vbar and o_compress together
+    args = lambda topk, vb, idx, num, oc, ws: (h, vsa.VSA_BF16, F, F, F, 1, 2, 128, topk, F, F, F, F, F, vb, idx,
+                                                num, oc, ws, None)
+    assert L.vsa_tile_coarse(*args(4, None, F, F, None, None)) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_tile_coarse(*args(4, None, F, F, None, M)) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_tile_coarse(*args(4, F, F, F, None, F)) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_tile_coarse(*args(4, None, F, F, F, F)) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_tile_coarse(*args(9, None, F, F, None, F)) == vsa.VSA_ERR_TOPK
+    assert L.vsa_tile_coarse(*args(-1, None, None, None, None, F)) == vsa.VSA_ERR_TOPK
+    assert L.vsa_tile_coarse(*args(0, None, F, None, None, F)) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_tile_coarse(*args(4, None, None, F, None, F)) == vsa.VSA_ERR_INVALID_ARG
     # gated untile
     assert L.vsa_untile_gate(h, 5, F, F, F, F, 1, 2, 128, None) == vsa.VSA_ERR_INVALID_ARG
     assert L.vsa_untile_gate(h, vsa.VSA_BF16, F, F, M, F, 1, 2, 128, None) == vsa.VSA_ERR_INVALID_ARG
