@@ -27,7 +27,7 @@ SYMBOLS = (
     "vsa_plan_create", "vsa_plan_create_prefix", "vsa_plan_destroy", "vsa_plan_sizes",
     "vsa_plan_describe", "vsa_tile", "vsa_tile_ex", "vsa_untile", "vsa_coarse_topk", "vsa_map_to_index",
     "vsa_sparse_attn_fwd", "vsa_sparse_attn_fwd_ex", "vsa_get_status", "vsa_strerror",
-    "vsa_coarse_compress", "vsa_untile_gate", "vsa_tile_coarse",
+    "vsa_coarse_compress", "vsa_untile_gate", "vsa_tile_coarse", "vsa_tile_coarse_static",
 )
 
 VSA_BF16 = 0
@@ -75,6 +75,7 @@ def lib():
         L.vsa_coarse_compress.argtypes = [P, P, P, P, i, i, i, i, P, P, P, P]
         L.vsa_untile_gate.argtypes = [P, i, P, P, P, P, i, i, i, P]
         L.vsa_tile_coarse.argtypes = [P, i, P, P, P, i, i, i, i] + [P] * 11
+        L.vsa_tile_coarse_static.argtypes = [P, i, P, P, P, i, i, i, i] + [P] * 10
         L.vsa_sparse_attn_fwd.argtypes = [P, P, P, P, P, P, i, i, i, i, P, P, P]
         L.vsa_get_status.argtypes = [P, P]
         L.vsa_strerror.argtypes = [i]
@@ -234,7 +235,8 @@ def tile_coarse(plan: Plan, q, k, v, topk: int, ws, gated: bool = False, out: di
     """Front end in one launch: tile q, k, v with block means, then the coarse
     stage (topk > 0) and, when gated, the compression branch.  Returns a dict
     with qt, kt, vt, qbar, kbar (+ vbar, oc when gated; + idx, num when topk > 0);
-    tensors given in `out` are written in place."""
+    tensors given in `out` are written in place.  ws=None runs
+    vsa_tile_coarse_static (the library's own counters, B*H <= 4096)."""
     torch = _torch()
     B, S, H, D = q.shape
     code = _dtype_code(q, "q")
@@ -254,13 +256,16 @@ def tile_coarse(plan: Plan, q, k, v, topk: int, ws, gated: bool = False, out: di
         if "num" not in o:
             o["num"] = torch.empty((B, H, plan.NB), dtype=torch.int32, device=q.device)
     f32, i32 = torch.float32, torch.int32
-    _check(lib().vsa_tile_coarse(
+    args = [
         plan.handle, code, _ptr(q, q.dtype, "q"), _ptr(k, q.dtype, "k"), _ptr(v, q.dtype, "v"), B, H, D, topk,
         _ptr(o["qt"], q.dtype, "q_tiled"), _ptr(o["kt"], q.dtype, "k_tiled"), _ptr(o["vt"], q.dtype, "v_tiled"),
         _ptr(o["qbar"], f32, "qbar"), _ptr(o["kbar"], f32, "kbar"), _ptr(o["vbar"], f32, "vbar") if gated else None,
         _ptr(o["idx"], i32, "q2k_idx") if topk > 0 else None, _ptr(o["num"], i32, "q2k_num") if topk > 0 else None,
-        _ptr(o["oc"], f32, "o_compress") if gated else None, _ptr(ws, i32, "workspace"), _stream()),
-        "vsa_tile_coarse")
+        _ptr(o["oc"], f32, "o_compress") if gated else None]
+    if ws is None:
+        _check(lib().vsa_tile_coarse_static(*args, _stream()), "vsa_tile_coarse_static")
+    else:
+        _check(lib().vsa_tile_coarse(*args, _ptr(ws, i32, "workspace"), _stream()), "vsa_tile_coarse")
     return o
 
 

@@ -90,6 +90,42 @@ int from_cuda(cudaError_t e) {
   return VSA_ERR_CUDA;
 }
 
+// Library-owned scratch of vsa_tile_coarse_static: the fused front end's
+// 2 int32 arrival counters per (b, h), for at most kStaticMaxHeads heads
+// (32 KB per device).  Its address is looked up once per device, with that
+// device current.
+constexpr int kStaticMaxHeads = 4096;
+static __device__ __align__(256) int g_front_scratch[2 * kStaticMaxHeads];
+
+struct StaticScratch {
+  bool ready = false;
+  int* ptr = nullptr;
+};
+std::mutex g_scratch_mu;
+StaticScratch g_scratch[kMaxDevices];
+
+int static_scratch(int** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
+    cudaGetLastError();
+    return VSA_ERR_NO_DEVICE;
+  }
+  if (dev >= kMaxDevices) return VSA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  StaticScratch& s = g_scratch[dev];
+  if (!s.ready) {
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_front_scratch) != cudaSuccess || addr == nullptr) {
+      cudaGetLastError();
+      return VSA_ERR_CUDA;
+    }
+    s.ptr = static_cast<int*>(addr);
+    s.ready = true;
+  }
+  *out = s.ptr;
+  return VSA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -261,6 +297,38 @@ int vsa_tile_coarse(vsa_plan_t plan, vsa_dtype_t dtype, const uint16_t* q, const
   a.status = ds->status;
   a.f16 = dtype == VSA_F16;
   return from_cuda(vsa::launch_front(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int vsa_tile_coarse_static(vsa_plan_t plan, vsa_dtype_t dtype, const uint16_t* q, const uint16_t* k,
+                           const uint16_t* v, int B, int H, int D, int topk, uint16_t* q_tiled, uint16_t* k_tiled,
+                           uint16_t* v_tiled, float* qbar, float* kbar, float* vbar, int32_t* q2k_idx,
+                           int32_t* q2k_num, float* o_compress, vsa_stream_t stream) {
+  // the checks of vsa_tile_coarse, so that a rejected call touches no device memory
+  if (dtype != VSA_BF16 && dtype != VSA_F16) return VSA_ERR_INVALID_ARG;
+  if (!plan || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q_tiled) || !aligned16(k_tiled) ||
+      !aligned16(v_tiled) || !aligned16(qbar) || !aligned16(kbar))
+    return VSA_ERR_INVALID_ARG;
+  if ((vbar == nullptr) != (o_compress == nullptr)) return VSA_ERR_INVALID_ARG;
+  if (vbar && (!aligned16(vbar) || !aligned16(o_compress))) return VSA_ERR_INVALID_ARG;
+  if (int rc = check_dims(B, H, D)) return rc;
+  if (static_cast<long long>(B) * H > kStaticMaxHeads) return VSA_ERR_UNSUPPORTED;
+  const int NB = plan->g.NB;
+  if (topk < 0 || topk > NB) return VSA_ERR_TOPK;
+  if (topk > 0 && (!aligned16(q2k_idx) || !aligned16(q2k_num))) return VSA_ERR_INVALID_ARG;
+  if (topk == 0 && (q2k_idx || q2k_num)) return VSA_ERR_INVALID_ARG;
+  if (NB > 2048) return VSA_ERR_UNSUPPORTED;
+  DeviceState* ds = nullptr;
+  if (int rc = device_state(&ds)) return rc;
+  int* scratch = nullptr;
+  if (int rc = static_scratch(&scratch)) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // the counters must start at zero (a call that timed out may leave them set)
+  if (cudaMemsetAsync(scratch, 0, sizeof(int) * 2 * static_cast<size_t>(B) * H, s) != cudaSuccess) {
+    cudaGetLastError();
+    return VSA_ERR_CUDA;
+  }
+  return vsa_tile_coarse(plan, dtype, q, k, v, B, H, D, topk, q_tiled, k_tiled, v_tiled, qbar, kbar, vbar, q2k_idx,
+                         q2k_num, o_compress, scratch, stream);
 }
 
 int vsa_untile_gate(vsa_plan_t plan, vsa_dtype_t dtype, const uint16_t* o_tiled, const float* o_compress,

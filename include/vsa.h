@@ -193,6 +193,25 @@ VSA_API int vsa_tile_coarse(vsa_plan_t plan, vsa_dtype_t dtype, const uint16_t *
                             vsa_stream_t stream);
 
 /*
+ * vsa_tile_coarse without a caller workspace: the arrival counters live in
+ * a static device array of the library (2 int32 per (b, h), B*H <= 4096,
+ * 32 KB per device), cleared by an asynchronous memset on `stream` before
+ * each launch.  The call allocates no memory.  The pages have no
+ * counterpart: it is an API convenience of this library.
+ *   Same arguments, outputs and errors as vsa_tile_coarse, minus workspace;
+ *   VSA_ERR_UNSUPPORTED when B*H > 4096.
+ *   Calls on one device share the one array: calls that may overlap (other
+ *   streams, other host threads) race on it and must be serialised by the
+ *   caller.
+ *   The first call on a device looks up the array's address (host-side
+ *   set-up); make that first call before any stream capture.
+ */
+VSA_API int vsa_tile_coarse_static(vsa_plan_t plan, vsa_dtype_t dtype, const uint16_t *q, const uint16_t *k,
+                                   const uint16_t *v, int B, int H, int D, int topk, uint16_t *q_tiled,
+                                   uint16_t *k_tiled, uint16_t *v_tiled, float *qbar, float *kbar, float *vbar,
+                                   int32_t *q2k_idx, int32_t *q2k_num, float *o_compress, vsa_stream_t stream);
+
+/*
  * Bool block map -> index (FastVideo commit log: map_to_index):
  * map [B,H,NQ,NK] (one byte per entry, non-zero = selected) ->
  * q2k_idx [B,H,NQ,NK] (selected ids ascending, then -1), q2k_num [B,H,NQ]
