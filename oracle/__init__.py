@@ -13,6 +13,9 @@ Each step follows the statement cited in the C file's header:
 * ``map_to_index``: FastVideo commit log, examples/inference/basic/README.md;
 * ``attn_rows``: "FastVideo VSA", introduction and section "Verify routing
   and fallback" (non-causal, scale head_size^-1/2), computed in fp64;
+* ``attn_bwd_q_rows``/``attn_bwd_kv``: gradients of the attention step with
+  the selection fixed (definition of softmax attention's derivative; the
+  commit log keeps the grad path separate), in fp64, real query rows only;
 * ``compress``/``gate_rows``: "FastVideo VSA", section "Checkpoint behavior"
   (learned gate_compress projection) and the FastVideo commit log (the
   gate-compress branch pools per tile); the formula is a reading, stated in
@@ -69,11 +72,13 @@ def _load():
         lib.oracle_attn_rows.argtypes = geo + [P, P, P, P, P, i, i, i, i, P, L, P, P, i]
         lib.oracle_compress.argtypes = [P, P, P, i, i, i, i, P]
         lib.oracle_gate_rows.argtypes = geo + [P, L, P, P, P, i, i, i, P, i]
+        lib.oracle_attn_bwd_q_rows.argtypes = geo + [P, P, P, P, P, P, i, i, i, i, P, L, P, i]
+        lib.oracle_attn_bwd_kv.argtypes = geo + [P, P, P, P, P, P, i, i, i, i, P, P, i]
         lib.oracle_max_threads.argtypes = []
         for f in ("oracle_geometry", "oracle_block_valid_counts", "oracle_tile", "oracle_untile",
                   "oracle_pool", "oracle_score", "oracle_topk", "oracle_map_to_index",
                   "oracle_attn_rows", "oracle_max_threads", "oracle_half_to_f32", "oracle_compress",
-                  "oracle_gate_rows"):
+                  "oracle_gate_rows", "oracle_attn_bwd_q_rows", "oracle_attn_bwd_kv"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -263,3 +268,29 @@ def gate_rows(g: Geometry, rows, o_fine, gate, o_compress, dtype: str = "bf16") 
     _check(_load().oracle_gate_rows(*g.args, _ptr(rows), len(rows), _ptr(o_fine), _ptr(gate), _ptr(o_compress),
                                     B, H, D, _ptr(out), DTYPES[dtype]), "gate_rows")
     return out
+
+
+def attn_bwd_q_rows(g: Geometry, qt, kt, vt, dot, idx, num, rows, dtype: str = "bf16") -> np.ndarray:
+    """dq (fp64 [n, D]) of flat query rows of [B,H,Sp]; padded rows give 0."""
+    arrs = [np.ascontiguousarray(a, dtype=np.uint16) for a in (qt, kt, vt, dot)]
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    num = np.ascontiguousarray(num, dtype=np.int32)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    B, H, Sp, D = arrs[0].shape
+    out = np.empty((len(rows), D), dtype=np.float64)
+    _check(_load().oracle_attn_bwd_q_rows(*g.args, *[_ptr(a) for a in arrs], _ptr(idx), _ptr(num), idx.shape[-1],
+                                          B, H, D, _ptr(rows), len(rows), _ptr(out), DTYPES[dtype]), "attn_bwd_q_rows")
+    return out
+
+
+def attn_bwd_kv(g: Geometry, qt, kt, vt, dot, idx, num, dtype: str = "bf16"):
+    """(dk, dv) fp64 [B,H,Sp,D] over all key rows (small problems only)."""
+    arrs = [np.ascontiguousarray(a, dtype=np.uint16) for a in (qt, kt, vt, dot)]
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    num = np.ascontiguousarray(num, dtype=np.int32)
+    B, H, Sp, D = arrs[0].shape
+    dk = np.empty((B, H, Sp, D), dtype=np.float64)
+    dv = np.empty((B, H, Sp, D), dtype=np.float64)
+    _check(_load().oracle_attn_bwd_kv(*g.args, *[_ptr(a) for a in arrs], _ptr(idx), _ptr(num), idx.shape[-1],
+                                      B, H, D, _ptr(dk), _ptr(dv), DTYPES[dtype]), "attn_bwd_kv")
+    return dk, dv

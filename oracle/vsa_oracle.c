@@ -36,6 +36,15 @@
  *            Computed in double from the bf16 inputs.  A row with count 0
  *            gives o = 0 and lse = -inf (commit log: zero-count rows).
  *  untile    inverse of tile; padded rows are dropped.
+ *  backward  the gradients of the attention step with the selection held
+ *            fixed (the commit log keeps the grad path on its own kernels; the
+ *            pages print no formula, so this is the definition): with
+ *            P_ij = softmax_j(scale q_i.k_j) over row i's keys,
+ *            dv_j = sum_i P_ij do_i, dP_ij = do_i.v_j,
+ *            dS_ij = P_ij (dP_ij - sum_l P_il dP_il),
+ *            dq_i = scale sum_j dS_ij k_j, dk_j = scale sum_i dS_ij q_i,
+ *            summed over the real query rows only (padded rows are not
+ *            outputs of the method), in double.
  *  compress  "FastVideo VSA", section "Checkpoint behavior", and the FastVideo
  *            commit log (the gate-compress branch pools per tile): the pages
  *            name a learned gate_compress projection and a branch that pools
@@ -346,6 +355,143 @@ int oracle_attn_rows(int n_prefix, int T, int Hg, int Wg, int bt, int bh, int bw
         }
         free(logit);
         free(key);
+    }
+    return bad ? ORACLE_ERR_INDEX : ORACLE_OK;
+}
+
+/* Softmax of one query row over its selected keys, in double.  Fills the key
+ * rows (tiled indices) and P; returns the key count, -1 on a bad block id. */
+static long row_softmax(const geom_t *g, const uint16_t *q, const uint16_t *k, const int32_t *idx,
+                        const int32_t *num, int max_k, int D, long bhh, long i, int dtype,
+                        long *key, double *p) {
+    int rblk = (int)(i / g->bs);
+    int cnt = num[bhh * g->NB + rblk];
+    if (cnt < 0 || cnt > max_k) return -1;
+    const double scale = 1.0 / sqrt((double)D);
+    const uint16_t *qi = q + ((size_t)bhh * g->Sp + i) * D;
+    long nk = 0;
+    for (int t = 0; t < cnt; ++t) {
+        int kb = idx[(bhh * g->NB + rblk) * (long)max_k + t];
+        if (kb < 0 || kb >= g->NB) return -1;
+        for (int slot = 0; slot < g->bs; ++slot) {
+            if (!slot_is_valid(g, kb, slot)) continue;
+            long j = (long)kb * g->bs + slot;
+            const uint16_t *kj = k + ((size_t)bhh * g->Sp + j) * D;
+            double dot = 0.0;
+            for (int d = 0; d < D; ++d) dot += (double)half_to_f32(qi[d], dtype) * (double)half_to_f32(kj[d], dtype);
+            p[nk] = scale * dot;
+            key[nk] = j;
+            ++nk;
+        }
+    }
+    double m = -INFINITY;
+    for (long t = 0; t < nk; ++t) if (p[t] > m) m = p[t];
+    double l = 0.0;
+    for (long t = 0; t < nk; ++t) { p[t] = exp(p[t] - m); l += p[t]; }
+    for (long t = 0; t < nk; ++t) p[t] /= l;
+    return nk;
+}
+
+/* dP_ij = do_i . v_j for the row's keys, and delta_i = sum_j P_ij dP_ij. */
+static double row_dp(const uint16_t *v, const uint16_t *dO, long bhh, long i, long Sp, int D, int dtype,
+                     const long *key, const double *p, long nk, double *dp) {
+    const uint16_t *doi = dO + ((size_t)bhh * Sp + i) * D;
+    double delta = 0.0;
+    for (long t = 0; t < nk; ++t) {
+        const uint16_t *vj = v + ((size_t)bhh * Sp + key[t]) * D;
+        double x = 0.0;
+        for (int d = 0; d < D; ++d) x += (double)half_to_f32(doi[d], dtype) * (double)half_to_f32(vj[d], dtype);
+        dp[t] = x;
+        delta += p[t] * x;
+    }
+    return delta;
+}
+
+static long max_keys(const geom_t *g, int max_k) { return (long)max_k * g->bs; }
+
+/*
+ * backward, query side: dq for an explicit list of query rows (flat indices
+ * into [B,H,Sp]); padded rows give dq = 0.  dq_rows [n_rows, D] double.
+ */
+int oracle_attn_bwd_q_rows(int n_prefix, int T, int Hg, int Wg, int bt, int bh, int bw,
+                           const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint16_t *dO,
+                           const int32_t *idx, const int32_t *num, int max_k, int B, int H, int D,
+                           const int64_t *rows, long n_rows, double *dq_rows, int dtype) {
+    geom_t g;
+    int rc = geom_init(&g, n_prefix, T, Hg, Wg, bt, bh, bw);
+    if (rc) return rc;
+    (void)B; (void)H;
+    if (D < 1 || max_k < 1) return ORACLE_ERR_ARG;
+    const double scale = 1.0 / sqrt((double)D);
+    int bad = 0;
+#pragma omp parallel reduction(| : bad)
+    {
+        long *key = (long *)malloc(sizeof(long) * (size_t)max_keys(&g, max_k));
+        double *p = (double *)malloc(sizeof(double) * (size_t)max_keys(&g, max_k));
+        double *dp = (double *)malloc(sizeof(double) * (size_t)max_keys(&g, max_k));
+        if (!key || !p || !dp) bad = 1;
+#pragma omp for schedule(dynamic, 4)
+        for (long n = 0; n < n_rows; ++n) {
+            double *out = dq_rows + (size_t)n * D;
+            for (int d = 0; d < D; ++d) out[d] = 0.0;
+            if (bad) continue;
+            long i = rows[n] % g.Sp, bhh = rows[n] / g.Sp;
+            if (!slot_is_valid(&g, (int)(i / g.bs), (int)(i % g.bs))) continue;
+            long nk = row_softmax(&g, q, k, idx, num, max_k, D, bhh, i, dtype, key, p);
+            if (nk < 0) { bad = 1; continue; }
+            double delta = row_dp(v, dO, bhh, i, g.Sp, D, dtype, key, p, nk, dp);
+            for (long t = 0; t < nk; ++t) {
+                double ds = p[t] * (dp[t] - delta) * scale;
+                const uint16_t *kj = k + ((size_t)bhh * g.Sp + key[t]) * D;
+                for (int d = 0; d < D; ++d) out[d] += ds * (double)half_to_f32(kj[d], dtype);
+            }
+        }
+        free(key); free(p); free(dp);
+    }
+    return bad ? ORACLE_ERR_INDEX : ORACLE_OK;
+}
+
+/*
+ * backward, key side: dk and dv [B,H,Sp,D] double for every key row, summed
+ * over every real query row of the head (small problems only: the cost is
+ * the whole attention, twice).  Padded key rows get 0.
+ */
+int oracle_attn_bwd_kv(int n_prefix, int T, int Hg, int Wg, int bt, int bh, int bw,
+                       const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint16_t *dO,
+                       const int32_t *idx, const int32_t *num, int max_k, int B, int H, int D,
+                       double *dk, double *dv, int dtype) {
+    geom_t g;
+    int rc = geom_init(&g, n_prefix, T, Hg, Wg, bt, bh, bw);
+    if (rc) return rc;
+    if (D < 1 || max_k < 1) return ORACLE_ERR_ARG;
+    const double scale = 1.0 / sqrt((double)D);
+    memset(dk, 0, sizeof(double) * (size_t)B * H * g.Sp * D);
+    memset(dv, 0, sizeof(double) * (size_t)B * H * g.Sp * D);
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (long bhh = 0; bhh < (long)B * H; ++bhh) {
+        long *key = (long *)malloc(sizeof(long) * (size_t)max_keys(&g, max_k));
+        double *p = (double *)malloc(sizeof(double) * (size_t)max_keys(&g, max_k));
+        double *dp = (double *)malloc(sizeof(double) * (size_t)max_keys(&g, max_k));
+        if (!key || !p || !dp) { bad = 1; free(key); free(p); free(dp); continue; }
+        for (long i = 0; i < g.Sp; ++i) {
+            if (!slot_is_valid(&g, (int)(i / g.bs), (int)(i % g.bs))) continue;
+            long nk = row_softmax(&g, q, k, idx, num, max_k, D, bhh, i, dtype, key, p);
+            if (nk < 0) { bad = 1; continue; }
+            double delta = row_dp(v, dO, bhh, i, g.Sp, D, dtype, key, p, nk, dp);
+            const uint16_t *doi = dO + ((size_t)bhh * g.Sp + i) * D;
+            const uint16_t *qi = q + ((size_t)bhh * g.Sp + i) * D;
+            for (long t = 0; t < nk; ++t) {
+                double *dvj = dv + ((size_t)bhh * g.Sp + key[t]) * D;
+                double *dkj = dk + ((size_t)bhh * g.Sp + key[t]) * D;
+                double ds = p[t] * (dp[t] - delta) * scale;
+                for (int d = 0; d < D; ++d) {
+                    dvj[d] += p[t] * (double)half_to_f32(doi[d], dtype);
+                    dkj[d] += ds * (double)half_to_f32(qi[d], dtype);
+                }
+            }
+        }
+        free(key); free(p); free(dp);
     }
     return bad ? ORACLE_ERR_INDEX : ORACLE_OK;
 }
