@@ -36,7 +36,7 @@ from block_sparse_video_gather_b200 import workloads  # noqa: E402
 
 PROFILE = os.path.join(ROOT, "profiles", "attn_fwd_fastwan.md")
 ATTN_SOURCES = [os.path.join(ROOT, "block_sparse_video_gather_b200", "csrc", f)
-                for f in ("attn_fwd.cu", "common.cuh")]
+                for f in ("attn_fwd.cu", "common.cuh", "tiles.cuh")]
 WORKLOAD_TEXT = {
     "tiny": "tiny grid 8x16x16, B1 H2 D128, block 4x8x8, topk 4",
     "fastwan": "FastWan2.2-TI2V-5B latent grid 31x22x40, B1 H24 D128, block 4x8x8, topk 64",

@@ -28,6 +28,7 @@ SYMBOLS = (
     "vsa_plan_describe", "vsa_tile", "vsa_tile_ex", "vsa_untile", "vsa_coarse_topk", "vsa_map_to_index",
     "vsa_sparse_attn_fwd", "vsa_sparse_attn_fwd_ex", "vsa_get_status", "vsa_strerror",
     "vsa_coarse_compress", "vsa_untile_gate", "vsa_tile_coarse", "vsa_tile_coarse_static",
+    "vsa_sparse_attn_bwd_workspace", "vsa_sparse_attn_bwd",
 )
 
 VSA_BF16 = 0
@@ -76,6 +77,8 @@ def lib():
         L.vsa_untile_gate.argtypes = [P, i, P, P, P, P, i, i, i, P]
         L.vsa_tile_coarse.argtypes = [P, i, P, P, P, i, i, i, i] + [P] * 11
         L.vsa_tile_coarse_static.argtypes = [P, i, P, P, P, i, i, i, i] + [P] * 10
+        L.vsa_sparse_attn_bwd_workspace.argtypes = [P, i, i, i, P]
+        L.vsa_sparse_attn_bwd.argtypes = [P, i, P, P, P, P, P, P, P, P, i, i, i, i, P, P, P, P, P]
         L.vsa_sparse_attn_fwd.argtypes = [P, P, P, P, P, P, i, i, i, i, P, P, P]
         L.vsa_get_status.argtypes = [P, P]
         L.vsa_strerror.argtypes = [i]
@@ -316,6 +319,33 @@ def sparse_attn_fwd(plan: Plan, q, k, v, q2k_idx, q2k_num, o_out=None, lse_out=N
                                         _ptr(o_out, q.dtype, "o"), _ptr(lse_out, torch.float32, "lse"),
                                         _stream()), "vsa_sparse_attn_fwd")
     return o_out, lse_out
+
+
+def bwd_workspace_bytes(plan: Plan, B: int, H: int, max_k: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().vsa_sparse_attn_bwd_workspace(plan.handle, B, H, max_k, ctypes.byref(n)),
+           "vsa_sparse_attn_bwd_workspace")
+    return n.value
+
+
+def sparse_attn_bwd(plan: Plan, q, k, v, o, lse, do, q2k_idx, q2k_num, dq=None, dk=None, dv=None, workspace=None):
+    """Gradients of the fine stage (tiled layout) -> (dq, dk, dv), selection fixed."""
+    torch = _torch()
+    B, H, Sp, D = q.shape
+    max_k = q2k_idx.shape[-1]
+    code = _dtype_code(q, "q")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    if workspace is None:
+        workspace = torch.empty(bwd_workspace_bytes(plan, B, H, max_k), dtype=torch.uint8, device=q.device)
+    t = q.dtype
+    _check(lib().vsa_sparse_attn_bwd(
+        plan.handle, code, _ptr(q, t, "q"), _ptr(k, t, "k"), _ptr(v, t, "v"), _ptr(o, t, "o"),
+        _ptr(lse, torch.float32, "lse"), _ptr(do, t, "do"), _ptr(q2k_idx, torch.int32, "q2k_idx"),
+        _ptr(q2k_num, torch.int32, "q2k_num"), max_k, B, H, D, _ptr(dq, t, "dq"), _ptr(dk, t, "dk"),
+        _ptr(dv, t, "dv"), _ptr(workspace, torch.uint8, "workspace"), _stream()), "vsa_sparse_attn_bwd")
+    return dq, dk, dv
 
 
 def get_status(stream=None) -> int:

@@ -1,0 +1,686 @@
+// attn_bwd.cu -- gradients of the fine stage (dq, dk, dv) with the block
+// selection held fixed, on the 5th-generation tensor cores.
+//
+// The attention step is "FastVideo VSA" (vLLM-Omni user guide, introduction
+// and section "Verify routing and fallback"); the FastVideo commit log keeps
+// the grad path on separate kernels and prints no formula.  With
+// P = softmax(scale q k^T) over each row's selected keys, recomputed from the
+// forward's lse:
+//   dv = P^T do,  dP = do v^T,  dS = P (dP - delta),  delta_i = do_i . o_i,
+//   dq = scale dS k,  dk = scale dS^T q.
+// Padded query rows and padded key rows take no part (P = 0 there), so their
+// gradients are zero whatever do holds at padded rows.
+//
+// Four launches:
+//   bwd_prep  delta_i = do_i . o_i and lse2_i = lse_i log2(e) per tiled row.
+//   k2q       the transposed selection: for each key block, the query blocks
+//             that list it (a repeated id is listed again), ascending; rows are
+//             placed in order, so the lists do not depend on thread timing.
+//   bwd_dkdv  one CTA per (b*h, key block, 128-key half).  K and V stay in
+//             shared memory; the query tiles of every listed query block
+//             stream through a 2-stage ring (Q, dO, lse2, delta).
+//             TMEM: S^T [0,128) with P^T (16-bit) written back on [0,64);
+//             dP^T [128,256) with dS^T on [128,192); dV [256,384); dK [384,512).
+//             Per query tile: S^T = K Q^T, dP^T = V dO^T, then
+//             dV += P^T dO and dK += dS^T Q (P^T, dS^T read from TMEM).
+//   bwd_dq    one CTA per (b*h, query block, 128-row half).  Q and dO stay;
+//             the K and V tiles of the selected blocks stream.  TMEM: S [0,128),
+//             dP [128,256), dQ [256,384), dS (16-bit) [384,448).  Per key tile:
+//             S = Q K^T, dP = dO V^T, then dQ += dS K.
+// Operands use the two forms of the forward kernel: K-major x K-major for the
+// products over the head dimension, TMEM (A) x MN-major shared memory (B) for
+// the products over keys or queries.  A tile in shared memory is the TMA image
+// of 128 rows x 128 channels (two 64-channel boxes, 128-byte swizzle) and is
+// read either way through its descriptor.
+//
+// Warp roles (256 threads): warp 0 TMA producer, warp 1 TMEM owner and MMA
+// issuer, warps 4-7 one thread per TMEM lane (tile row) for the elementwise
+// step and the epilogue.  Every mbarrier wait is bounded; on expiry the kernel
+// records VSA_ERR_TIMEOUT, drains its copies and MMAs, frees TMEM and returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tiles.cuh"
+
+namespace vsa {
+
+namespace {
+
+using namespace tiles;
+
+constexpr int kThreads = 256;
+constexpr uint32_t kHalfBytes = 128 * 128;      // 128 rows x 64 16-bit channels
+constexpr uint32_t kTileBytes = 2 * kHalfBytes;  // 128 rows x 128 channels
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <bool F16>
+struct Idesc {
+  static constexpr uint32_t KK = F16 ? idesc_f16_f32(128, 128, 0, 0) : idesc_bf16_f32(128, 128, 0, 0);
+  static constexpr uint32_t TM = F16 ? idesc_f16_f32(128, 128, 0, 1) : idesc_bf16_f32(128, 128, 0, 1);
+};
+
+// Word i of four, without dynamic indexing (which would put the array in local memory).
+__device__ __forceinline__ uint32_t pick4(const uint32_t (&w)[4], int i) {
+  return i == 0 ? w[0] : (i == 1 ? w[1] : (i == 2 ? w[2] : w[3]));
+}
+
+// All 128 validity bits of a tile (key_tile_mask sets them only for a
+// partial tile; a full or empty one is reported by its return value).
+__device__ __forceinline__ int tile_bits(const Geo& g, int blk, int half, uint32_t (&w)[4]) {
+  const int st = key_tile_mask(g, blk, half, w);
+  if (st != kTilePartial) w[0] = w[1] = w[2] = w[3] = (st == kTileFull) ? 0xffffffffu : 0u;
+  return st;
+}
+
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+struct BwdBarriers {
+  uint64_t a_full;            // resident tiles (K,V for dkdv; Q,dO for dq)
+  uint64_t full[2], empty[2];  // streamed stages
+  uint64_t s_full, ds_full, done, drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ __forceinline__ bool wwait(uint64_t* bar, uint32_t parity, BwdBarriers* b, unsigned int* status) {
+  bool ok = mbar_wait(bar, parity, &b->abort, status, kTimeoutNs);
+  return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ void init_barriers(BwdBarriers* b) {
+  mbar_init(&b->a_full, 1);
+  for (int s = 0; s < 2; ++s) {
+    mbar_init(&b->full[s], 1);
+    mbar_init(&b->empty[s], 1);
+  }
+  mbar_init(&b->s_full, 1);
+  mbar_init(&b->ds_full, 128);
+  mbar_init(&b->done, 1);
+  mbar_init(&b->drain, 1);
+  b->abort = 0;
+  fence_barrier_init();
+  fence_proxy_async_smem();
+}
+
+// 128 fp32 TMEM columns of this thread's lane, scaled, to one 16-bit row in
+// global memory.  `load` must be the same for the whole warp (the TMEM load
+// is a warp-wide instruction); `zero` may differ per thread.
+template <bool F16>
+__device__ __forceinline__ void store_row(uint32_t taddr, float scale, uint16_t* dst, bool load, bool zero) {
+  uint4* out = reinterpret_cast<uint4*>(dst);
+  zero = zero || !load;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t v[32];
+    if (load) {
+      tmem_ld32(taddr + c * 32, v);
+      tmem_wait_ld();
+    }
+    uint32_t w[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      w[j] = zero ? 0u : pack_half2<F16>(__uint_as_float(v[2 * j]) * scale, __uint_as_float(v[2 * j + 1]) * scale);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) out[c * 4 + j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+  }
+}
+
+struct BwdParams {
+  Geo g;
+  int BH, max_k;
+  const int32_t* idx;
+  const int32_t* num;
+  const int32_t* k2q_off;  // [BH][NB + 1]
+  const int32_t* k2q;      // [BH][NB * max_k]
+  const float* lse2;       // [BH * Sp]
+  const float* delta;      // [BH * Sp]
+  uint16_t* dq;
+  uint16_t* dk;
+  uint16_t* dv;
+  unsigned int* status;
+  float scale;       // D^-1/2
+  float scale_log2;  // D^-1/2 log2(e)
+};
+
+// ---------------------------------------------------------------------------
+// dk, dv
+// ---------------------------------------------------------------------------
+constexpr uint32_t kKV_K = 0, kKV_V = kTileBytes, kKV_Stage = 2 * kTileBytes;
+constexpr uint32_t kKV_StageBytes = 2 * kTileBytes;   // Q + dO
+constexpr uint32_t kKV_L = kKV_Stage + 2 * kKV_StageBytes;  // lse2, delta: 2 stages x 1 KB
+constexpr uint32_t kKV_Bar = kKV_L + 2 * 1024;
+constexpr uint32_t kKV_Smem = kKV_Bar + 256 + 1024;
+
+template <bool F16>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                         const __grid_constant__ BwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  BwdBarriers* bars = reinterpret_cast<BwdBarriers*>(smem + kKV_Bar);
+  const Geo& g = p.g;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int item = blockIdx.x;
+  const int half = item & 1;
+  const int kb = (item >> 1) % g.NB;
+  const int bh = (item >> 1) / g.NB;
+  const int32_t* offs = p.k2q_off + static_cast<long long>(bh) * (g.NB + 1);
+  const int lo = __ldg(offs + kb), hi = __ldg(offs + kb + 1);
+  const int32_t* list = p.k2q + static_cast<long long>(bh) * g.NB * p.max_k + lo;
+  const int nq = 2 * (hi - lo);  // query tiles
+  const long long base = static_cast<long long>(bh) * g.Sp;
+
+  if (threadIdx.x == 0) init_barriers(bars);
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    const uint64_t pol_last = policy_evict_last();
+    int issued = 0;
+    bool kv = false;
+    if (nq > 0) {
+      const int krow = static_cast<int>(base + static_cast<long long>(kb) * 256 + half * 128);
+      mbar_arrive_expect_tx_w(&bars->a_full, 2 * kTileBytes);
+      for (int hf = 0; hf < 2; ++hf) {
+        tma_load_2d_w(smem + kKV_K + hf * kHalfBytes, &tm_k, hf * 64, krow, &bars->a_full, pol_last);
+        tma_load_2d_w(smem + kKV_V + hf * kHalfBytes, &tm_v, hf * 64, krow, &bars->a_full, pol_last);
+      }
+      kv = true;
+      for (int u = 0; u < nq; ++u) {
+        const int s = u & 1;
+        if (!wwait(&bars->empty[s], ((u >> 1) & 1) ^ 1, bars, p.status)) break;
+        const int qb = __ldg(list + (u >> 1));
+        const long long qrow = base + static_cast<long long>(qb) * 256 + (u & 1) * 128;
+        uint8_t* st = smem + kKV_Stage + s * kKV_StageBytes;
+        mbar_arrive_expect_tx_w(&bars->full[s], 2 * kTileBytes + 1024);
+        for (int hf = 0; hf < 2; ++hf) {
+          tma_load_2d_w(st + hf * kHalfBytes, &tm_q, hf * 64, static_cast<int>(qrow), &bars->full[s], pol_last);
+          tma_load_2d_w(st + kTileBytes + hf * kHalfBytes, &tm_do, hf * 64, static_cast<int>(qrow), &bars->full[s],
+                        pol_last);
+        }
+        if (lane == 0) {
+          bulk_load(smem + kKV_L + s * 1024, p.lse2 + qrow, 512, &bars->full[s]);
+          bulk_load(smem + kKV_L + s * 1024 + 512, p.delta + qrow, 512, &bars->full[s]);
+        }
+        __syncwarp();
+        ++issued;
+      }
+    }
+    // drain every copy in flight before shared memory is released
+    if (kv) mbar_wait_drain(&bars->a_full, 0, kTimeoutNs);
+    for (int s = 0; s < 2; ++s)
+      if (issued > s) {
+        const int last = issued - 1 - ((issued - 1 - s) & 1);
+        mbar_wait_drain(&bars->full[s], (last >> 1) & 1, kTimeoutNs);
+      }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint64_t dK = sdesc_sw128(smem_u32(smem + kKV_K), 16, 1024);
+    const uint64_t dV = sdesc_sw128(smem_u32(smem + kKV_V), 16, 1024);
+    const uint64_t dSt = sdesc_sw128(smem_u32(smem + kKV_Stage), 16, 1024);                 // K-major view
+    const uint64_t mSt = sdesc_sw128(smem_u32(smem + kKV_Stage), kHalfBytes, 1024);         // MN-major view
+    constexpr uint64_t kStage = kKV_StageBytes >> 4, kTile = kTileBytes >> 4;
+    bool ok = true;
+    if (nq > 0) ok = wwait(&bars->a_full, 0, bars, p.status);
+    for (int u = 0; u < nq && ok; ++u) {
+      const int s = u & 1;
+      if (!(ok = wwait(&bars->full[s], (u >> 1) & 1, bars, p.status))) break;
+      tc_fence_after();
+      const uint64_t q_k = dSt + s * kStage, do_k = q_k + kTile;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t off = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+        mma_ss_w(tmem + 0, dK + off, q_k + off, Idesc<F16>::KK, kk > 0 ? 1u : 0u);
+      }
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t off = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+        mma_ss_w(tmem + 128, dV + off, do_k + off, Idesc<F16>::KK, kk > 0 ? 1u : 0u);
+      }
+      mma_commit_w(&bars->s_full);
+      if (!(ok = wwait(&bars->ds_full, u & 1, bars, p.status))) break;
+      tc_fence_after();
+      const uint64_t q_m = mSt + s * kStage, do_m = q_m + kTile;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_ts_w(tmem + 256, tmem + 0 + kk * 8, do_m + kk * (2048 >> 4), Idesc<F16>::TM, (u > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_ts_w(tmem + 384, tmem + 128 + kk * 8, q_m + kk * (2048 >> 4), Idesc<F16>::TM, (u > 0 || kk > 0) ? 1u : 0u);
+      mma_commit_w(&bars->empty[s]);
+    }
+    mma_commit_w(&bars->done);
+    mma_commit_w(&bars->drain);
+    mbar_wait_drain(&bars->drain, 0, kTimeoutNs);
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ elementwise + epilogue
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;  // key row of the tile
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_off, tP = tS + 128;
+    uint32_t kw[4];
+    tile_bits(g, kb, half, kw);
+    const bool kvalid = (pick4(kw, r >> 5) >> (r & 31)) & 1u;
+    const float c2 = p.scale_log2;
+    bool ok = true;
+    for (int u = 0; u < nq && ok; ++u) {
+      const int s = u & 1;
+      const int qb = __ldg(list + (u >> 1));
+      uint32_t qw[4];
+      tile_bits(g, qb, u & 1, qw);
+      if (!kvalid) qw[0] = qw[1] = qw[2] = qw[3] = 0u;
+      if (!(ok = wwait(&bars->full[s], (u >> 1) & 1, bars, p.status))) break;
+      if (!(ok = wwait(&bars->s_full, u & 1, bars, p.status))) break;
+      tc_fence_after();
+      const float* L2 = reinterpret_cast<const float*>(smem + kKV_L + s * 1024);
+      const float* DL = L2 + 128;
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t sv[32], dv[32];
+        tmem_ld32(tS + ch * 32, sv);
+        tmem_ld32(tP + ch * 32, dv);
+        tmem_wait_ld();
+        const uint32_t m = pick4(qw, ch);
+        uint32_t pk[16], dk16[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          float pr[2], dr[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int c = 2 * j + e;
+            const int q = ch * 32 + c;
+            const float x = __fmaf_rn(__uint_as_float(sv[c]), c2, -L2[q]);
+            const float pp = ((m >> c) & 1u) ? ex2_approx(x) : 0.0f;
+            pr[e] = pp;
+            dr[e] = pp * (__uint_as_float(dv[c]) - DL[q]);
+          }
+          pk[j] = pack_half2<F16>(pr[0], pr[1]);
+          dk16[j] = pack_half2<F16>(dr[0], dr[1]);
+        }
+        tmem_st16(tS + ch * 16, pk);
+        tmem_st16(tP + ch * 16, dk16);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars->ds_full);
+    }
+    if (ok && nq > 0) ok = wwait(&bars->done, 0, bars, p.status);
+    tc_fence_after();
+    const long long row = base + static_cast<long long>(kb) * 256 + half * 128 + r;
+    const bool load = ok && nq > 0;  // warp-uniform
+    store_row<F16>(tS + 256, 1.0f, p.dv + row * 128, load, false);
+    store_row<F16>(tS + 384, p.scale, p.dk + row * 128, load, false);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dq
+// ---------------------------------------------------------------------------
+constexpr uint32_t kQ_Q = 0, kQ_DO = kTileBytes, kQ_K = 2 * kTileBytes;  // K stages: 2 x 32 KB
+constexpr uint32_t kQ_V = kQ_K + 2 * kTileBytes;                          // V stages: 2 x 32 KB
+constexpr uint32_t kQ_Bar = kQ_V + 2 * kTileBytes;
+constexpr uint32_t kQ_Smem = kQ_Bar + 256 + 1024;
+
+__device__ __forceinline__ int dq_block(const BwdParams& p, long long row_item, int j) {
+  const int kb = __ldg(p.idx + row_item * p.max_k + j);
+  return (kb >= 0 && kb < p.g.NB) ? kb : -1;
+}
+
+template <bool F16>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                       const __grid_constant__ BwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  BwdBarriers* bars = reinterpret_cast<BwdBarriers*>(smem + kQ_Bar);
+  const Geo& g = p.g;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int item = blockIdx.x;
+  const int half = item & 1;
+  const int qb = (item >> 1) % g.NB;
+  const int bh = (item >> 1) / g.NB;
+  const long long row_item = static_cast<long long>(bh) * g.NB + qb;
+  int nb = __ldg(p.num + row_item);
+  if (nb < 0 || nb > p.max_k) {
+    if (threadIdx.x == 0 && half == 0) atomicCAS(p.status, 0u, (unsigned)VSA_ERR_BAD_INDEX);
+    nb = nb < 0 ? 0 : p.max_k;
+  }
+  const int n = 2 * nb;  // key tiles
+  const long long base = static_cast<long long>(bh) * g.Sp;
+
+  if (threadIdx.x == 0) init_barriers(bars);
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    const uint64_t pol_last = policy_evict_last(), pol_first = policy_evict_first();
+    int issued = 0;
+    bool qd = false;
+    if (n > 0) {
+      const int qrow = static_cast<int>(base + static_cast<long long>(qb) * 256 + half * 128);
+      mbar_arrive_expect_tx_w(&bars->a_full, 2 * kTileBytes);
+      for (int hf = 0; hf < 2; ++hf) {
+        tma_load_2d_w(smem + kQ_Q + hf * kHalfBytes, &tm_q, hf * 64, qrow, &bars->a_full, pol_first);
+        tma_load_2d_w(smem + kQ_DO + hf * kHalfBytes, &tm_do, hf * 64, qrow, &bars->a_full, pol_first);
+      }
+      qd = true;
+      for (int t = 0; t < n; ++t) {
+        const int s = t & 1;
+        if (!wwait(&bars->empty[s], ((t >> 1) & 1) ^ 1, bars, p.status)) break;
+        const int kb0 = dq_block(p, row_item, t >> 1);
+        const int kb = kb0 < 0 ? 0 : kb0;  // unusable ids load block 0; the elementwise step masks it out
+        const int krow = static_cast<int>(base + static_cast<long long>(kb) * 256 + (t & 1) * 128);
+        mbar_arrive_expect_tx_w(&bars->full[s], 2 * kTileBytes);
+        for (int hf = 0; hf < 2; ++hf) {
+          tma_load_2d_w(smem + kQ_K + s * kTileBytes + hf * kHalfBytes, &tm_k, hf * 64, krow, &bars->full[s],
+                        pol_last);
+          tma_load_2d_w(smem + kQ_V + s * kTileBytes + hf * kHalfBytes, &tm_v, hf * 64, krow, &bars->full[s],
+                        pol_last);
+        }
+        ++issued;
+      }
+    }
+    if (qd) mbar_wait_drain(&bars->a_full, 0, kTimeoutNs);
+    for (int s = 0; s < 2; ++s)
+      if (issued > s) {
+        const int last = issued - 1 - ((issued - 1 - s) & 1);
+        mbar_wait_drain(&bars->full[s], (last >> 1) & 1, kTimeoutNs);
+      }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint64_t dQ = sdesc_sw128(smem_u32(smem + kQ_Q), 16, 1024);
+    const uint64_t dDO = sdesc_sw128(smem_u32(smem + kQ_DO), 16, 1024);
+    const uint64_t dK = sdesc_sw128(smem_u32(smem + kQ_K), 16, 1024);
+    const uint64_t dV = sdesc_sw128(smem_u32(smem + kQ_V), 16, 1024);
+    const uint64_t mK = sdesc_sw128(smem_u32(smem + kQ_K), kHalfBytes, 1024);
+    constexpr uint64_t kTile = kTileBytes >> 4;
+    bool ok = true;
+    if (n > 0) ok = wwait(&bars->a_full, 0, bars, p.status);
+    for (int t = 0; t < n && ok; ++t) {
+      const int s = t & 1;
+      if (!(ok = wwait(&bars->full[s], (t >> 1) & 1, bars, p.status))) break;
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t off = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+        mma_ss_w(tmem + 0, dQ + off, dK + s * kTile + off, Idesc<F16>::KK, kk > 0 ? 1u : 0u);
+      }
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t off = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+        mma_ss_w(tmem + 128, dDO + off, dV + s * kTile + off, Idesc<F16>::KK, kk > 0 ? 1u : 0u);
+      }
+      mma_commit_w(&bars->s_full);
+      if (!(ok = wwait(&bars->ds_full, t & 1, bars, p.status))) break;
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_ts_w(tmem + 256, tmem + 384 + kk * 8, mK + s * kTile + kk * (2048 >> 4), Idesc<F16>::TM,
+                 (t > 0 || kk > 0) ? 1u : 0u);
+      mma_commit_w(&bars->empty[s]);
+    }
+    mma_commit_w(&bars->done);
+    mma_commit_w(&bars->drain);
+    mbar_wait_drain(&bars->drain, 0, kTimeoutNs);
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ elementwise + epilogue
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;  // query row of the tile
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_off, tP = tS + 128, tDS = tS + 384;
+    uint32_t rw[4];
+    tile_bits(g, qb, half, rw);
+    const bool rvalid = (pick4(rw, r >> 5) >> (r & 31)) & 1u;
+    const long long row = base + static_cast<long long>(qb) * 256 + half * 128 + r;
+    const float nl2 = rvalid ? -__ldg(p.lse2 + row) : 0.0f;
+    const float dl = rvalid ? __ldg(p.delta + row) : 0.0f;
+    const float c2 = p.scale_log2;
+    bool ok = true;
+    for (int t = 0; t < n && ok; ++t) {
+      const int kb = dq_block(p, row_item, t >> 1);
+      if (kb < 0 && r == 0 && half == 0 && (t & 1) == 0) atomicCAS(p.status, 0u, (unsigned)VSA_ERR_BAD_INDEX);
+      uint32_t kw[4];
+      tile_bits(g, kb, t & 1, kw);
+      if (!rvalid) kw[0] = kw[1] = kw[2] = kw[3] = 0u;
+      if (!(ok = wwait(&bars->s_full, t & 1, bars, p.status))) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t sv[32], dv[32];
+        tmem_ld32(tS + ch * 32, sv);
+        tmem_ld32(tP + ch * 32, dv);
+        tmem_wait_ld();
+        const uint32_t m = pick4(kw, ch);
+        uint32_t dk16[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          float dr[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int c = 2 * j + e;
+            const float x = __fmaf_rn(__uint_as_float(sv[c]), c2, nl2);
+            const float pp = ((m >> c) & 1u) ? ex2_approx(x) : 0.0f;
+            dr[e] = pp * (__uint_as_float(dv[c]) - dl);
+          }
+          dk16[j] = pack_half2<F16>(dr[0], dr[1]);
+        }
+        tmem_st16(tDS + ch * 16, dk16);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars->ds_full);
+    }
+    if (ok && n > 0) ok = wwait(&bars->done, 0, bars, p.status);
+    tc_fence_after();
+    store_row<F16>(tS + 256, p.scale, p.dq + row * 128, ok && n > 0, !rvalid);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// preparation: delta and lse2 per tiled row; transposed selection per head
+// ---------------------------------------------------------------------------
+template <bool F16>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const uint4* __restrict__ o, const uint4* __restrict__ dO,
+                                                       const float* __restrict__ lse, float* __restrict__ lse2,
+                                                       float* __restrict__ delta, long long rows) {
+  const long long row = static_cast<long long>(blockIdx.x) * 16 + (threadIdx.x >> 4);
+  const int chunk = threadIdx.x & 15;
+  float acc = 0.0f;
+  if (row < rows) {
+    const uint4 a = __ldg(o + row * 16 + chunk), b = __ldg(dO + row * 16 + chunk);
+    const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float alo, ahi, blo, bhi;
+      if (F16) {
+        alo = __half2float(__ushort_as_half(static_cast<unsigned short>(aw[k] & 0xFFFFu)));
+        ahi = __half2float(__ushort_as_half(static_cast<unsigned short>(aw[k] >> 16)));
+        blo = __half2float(__ushort_as_half(static_cast<unsigned short>(bw[k] & 0xFFFFu)));
+        bhi = __half2float(__ushort_as_half(static_cast<unsigned short>(bw[k] >> 16)));
+      } else {
+        alo = bf16_lo(aw[k]);
+        ahi = bf16_hi(aw[k]);
+        blo = bf16_lo(bw[k]);
+        bhi = bf16_hi(bw[k]);
+      }
+      acc = __fmaf_rn(alo, blo, acc);
+      acc = __fmaf_rn(ahi, bhi, acc);
+    }
+  }
+#pragma unroll
+  for (int off = 8; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (row < rows && chunk == 0) {
+    delta[row] = acc;
+    lse2[row] = __ldg(lse + row) * kLog2e;
+  }
+}
+
+// One CTA per (b*h).  Counts per key block, offsets, then rows in order.
+__global__ void __launch_bounds__(256) k2q_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ num,
+                                                  int NB, int max_k, int32_t* __restrict__ k2q_off,
+                                                  int32_t* __restrict__ k2q, unsigned int* status) {
+  extern __shared__ int kq_sm[];
+  int* cnt = kq_sm;        // [NB]
+  int* cur = kq_sm + NB;   // [NB]
+  const int bh = blockIdx.x;
+  const int32_t* ih = idx + static_cast<long long>(bh) * NB * max_k;
+  const int32_t* nh = num + static_cast<long long>(bh) * NB;
+  int32_t* list = k2q + static_cast<long long>(bh) * NB * max_k;
+  for (int c = threadIdx.x; c < NB; c += blockDim.x) {
+    cnt[c] = 0;
+    cur[c] = 0;
+  }
+  __syncthreads();
+  bool bad = false;
+  for (long long e = threadIdx.x; e < static_cast<long long>(NB) * max_k; e += blockDim.x) {
+    const int r = static_cast<int>(e / max_k), t = static_cast<int>(e - static_cast<long long>(r) * max_k);
+    int c = nh[r];
+    if (c < 0 || c > max_k) {
+      bad = true;
+      c = c < 0 ? 0 : max_k;
+    }
+    if (t >= c) continue;
+    const int kb = ih[e];
+    if (kb < 0 || kb >= NB) {
+      bad = true;
+      continue;
+    }
+    atomicAdd(&cnt[kb], 1);
+  }
+  if (bad) atomicCAS(status, 0u, (unsigned)VSA_ERR_BAD_INDEX);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0;
+    int32_t* off = k2q_off + static_cast<long long>(bh) * (NB + 1);
+    for (int c = 0; c < NB; ++c) {
+      const int x = cnt[c];
+      cnt[c] = run;
+      off[c] = run;
+      run += x;
+    }
+    off[NB] = run;
+  }
+  __syncthreads();
+  for (int r = 0; r < NB; ++r) {
+    int c = nh[r];
+    c = c < 0 ? 0 : (c > max_k ? max_k : c);
+    for (int t = threadIdx.x; t < c; t += blockDim.x) {
+      const int kb = ih[static_cast<long long>(r) * max_k + t];
+      if (kb < 0 || kb >= NB) continue;
+      list[cnt[kb] + atomicAdd(&cur[kb], 1)] = r;
+    }
+    __syncthreads();
+  }
+}
+
+}  // namespace
+
+size_t attn_bwd_workspace_bytes(const Geo& g, int BH, int max_k) {
+  const size_t rows = static_cast<size_t>(BH) * g.Sp;
+  size_t b = 2 * rows * sizeof(float);                                   // lse2, delta
+  b += static_cast<size_t>(BH) * (g.NB + 1) * sizeof(int32_t);           // k2q offsets
+  b = (b + 15) & ~size_t(15);
+  b += static_cast<size_t>(BH) * g.NB * max_k * sizeof(int32_t);        // k2q lists
+  return b;
+}
+
+cudaError_t launch_attn_bwd(const Geo& g, const AttnBwdArgs& a, cudaStream_t stream) {
+  if (g.bs != 256) return cudaErrorNotSupported;
+  const unsigned long long rows = static_cast<unsigned long long>(a.BH) * g.Sp;
+  if (rows >= (1ull << 31)) return cudaErrorInvalidValue;
+  uint8_t* ws = static_cast<uint8_t*>(a.workspace);
+  float* lse2 = reinterpret_cast<float*>(ws);
+  float* delta = lse2 + rows;
+  int32_t* k2q_off = reinterpret_cast<int32_t*>(delta + rows);
+  size_t off_bytes = 2 * rows * sizeof(float) + static_cast<size_t>(a.BH) * (g.NB + 1) * sizeof(int32_t);
+  off_bytes = (off_bytes + 15) & ~size_t(15);
+  int32_t* k2q = reinterpret_cast<int32_t*>(ws + off_bytes);
+
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_tmap(&tq, a.q, rows, 128, a.f16) || !make_tmap(&tk, a.k, rows, 128, a.f16) ||
+      !make_tmap(&tv, a.v, rows, 128, a.f16) || !make_tmap(&tdo, a.dO, rows, 128, a.f16))
+    return cudaErrorInvalidValue;
+
+  const unsigned prep_blocks = static_cast<unsigned>((rows + 15) / 16);
+  if (a.f16)
+    bwd_prep_kernel<true><<<prep_blocks, 256, 0, stream>>>(reinterpret_cast<const uint4*>(a.o),
+                                                           reinterpret_cast<const uint4*>(a.dO), a.lse, lse2, delta,
+                                                           static_cast<long long>(rows));
+  else
+    bwd_prep_kernel<false><<<prep_blocks, 256, 0, stream>>>(reinterpret_cast<const uint4*>(a.o),
+                                                            reinterpret_cast<const uint4*>(a.dO), a.lse, lse2, delta,
+                                                            static_cast<long long>(rows));
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  k2q_kernel<<<a.BH, 256, 2 * g.NB * sizeof(int), stream>>>(a.idx, a.num, g.NB, a.max_k, k2q_off, k2q, a.status);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+  BwdParams p;
+  p.g = g;
+  p.BH = a.BH;
+  p.max_k = a.max_k;
+  p.idx = a.idx;
+  p.num = a.num;
+  p.k2q_off = k2q_off;
+  p.k2q = k2q;
+  p.lse2 = lse2;
+  p.delta = delta;
+  p.dq = a.dq;
+  p.dk = a.dk;
+  p.dv = a.dv;
+  p.status = a.status;
+  p.scale = static_cast<float>(1.0 / 11.313708498984761);            // 128^-1/2
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / 11.313708498984761);
+  const unsigned items = static_cast<unsigned>(2ull * a.BH * g.NB);
+  auto kv = a.f16 ? attn_bwd_dkdv_kernel<true> : attn_bwd_dkdv_kernel<false>;
+  auto dq = a.f16 ? attn_bwd_dq_kernel<true> : attn_bwd_dq_kernel<false>;
+  if ((e = cudaFuncSetAttribute(kv, cudaFuncAttributeMaxDynamicSharedMemorySize, kKV_Smem)) != cudaSuccess) return e;
+  if ((e = cudaFuncSetAttribute(dq, cudaFuncAttributeMaxDynamicSharedMemorySize, kQ_Smem)) != cudaSuccess) return e;
+  kv<<<items, kThreads, kKV_Smem, stream>>>(tq, tk, tv, tdo, p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  dq<<<items, kThreads, kQ_Smem, stream>>>(tq, tk, tv, tdo, p);
+  return cudaGetLastError();
+}
+
+}  // namespace vsa

@@ -60,4 +60,20 @@ struct AttnArgs {
 };
 cudaError_t launch_attn_fwd(const Geo& g, const AttnArgs& a, cudaStream_t stream);
 
+// attn_bwd.cu
+struct AttnBwdArgs {
+  const uint16_t *q, *k, *v, *o, *dO;  // tiled [B,H,Sp,D]
+  const float* lse;                    // [B,H,Sp]
+  const int32_t* idx;
+  const int32_t* num;
+  int max_k;
+  int BH;
+  uint16_t *dq, *dk, *dv;  // tiled [B,H,Sp,D]
+  void* workspace;         // attn_bwd_workspace_bytes
+  unsigned int* status;
+  bool f16;
+};
+size_t attn_bwd_workspace_bytes(const Geo& g, int BH, int max_k);
+cudaError_t launch_attn_bwd(const Geo& g, const AttnBwdArgs& a, cudaStream_t stream);
+
 }  // namespace vsa

@@ -388,6 +388,46 @@ int vsa_sparse_attn_fwd(vsa_plan_t plan, const uint16_t* q, const uint16_t* k, c
   return vsa_sparse_attn_fwd_ex(plan, VSA_BF16, q, k, v, q2k_idx, q2k_num, max_k, B, H, D, o, lse, stream);
 }
 
+int vsa_sparse_attn_bwd_workspace(vsa_plan_t plan, int B, int H, int max_k, size_t* bytes) {
+  if (!plan || !bytes || B < 1 || H < 1 || max_k < 1) return VSA_ERR_INVALID_ARG;
+  *bytes = vsa::attn_bwd_workspace_bytes(plan->g, B * H, max_k);
+  return VSA_OK;
+}
+
+int vsa_sparse_attn_bwd(vsa_plan_t plan, vsa_dtype_t dtype, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                        const uint16_t* o, const float* lse, const uint16_t* dO, const int32_t* q2k_idx,
+                        const int32_t* q2k_num, int max_k, int B, int H, int D, uint16_t* dq, uint16_t* dk,
+                        uint16_t* dv, void* workspace, vsa_stream_t stream) {
+  if (dtype != VSA_BF16 && dtype != VSA_F16) return VSA_ERR_INVALID_ARG;
+  if (!plan || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      !aligned16(dO) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
+    return VSA_ERR_INVALID_ARG;
+  if (!aligned16(q2k_idx) || !aligned16(q2k_num) || max_k < 1) return VSA_ERR_INVALID_ARG;
+  if (int rc = check_dims(B, H, D)) return rc;
+  const vsa::Geo& g = plan->g;
+  if (g.bs != 256) return VSA_ERR_UNSUPPORTED;
+  DeviceState* ds = nullptr;
+  if (int rc = device_state(&ds)) return rc;
+  vsa::AttnBwdArgs a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.dO = dO;
+  a.lse = lse;
+  a.idx = q2k_idx;
+  a.num = q2k_num;
+  a.max_k = max_k;
+  a.BH = B * H;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.workspace = workspace;
+  a.status = ds->status;
+  a.f16 = dtype == VSA_F16;
+  return from_cuda(vsa::launch_attn_bwd(g, a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int vsa_get_status(vsa_stream_t stream, int* device_status) {
   if (!device_status) return VSA_ERR_INVALID_ARG;
   DeviceState* ds = nullptr;

@@ -247,6 +247,31 @@ VSA_API int vsa_sparse_attn_fwd_ex(vsa_plan_t plan, vsa_dtype_t dtype, const uin
                                    vsa_stream_t stream);
 
 /*
+ * Backward of the fine stage with the selection held fixed (the FastVideo
+ * commit log keeps the grad path on separate kernels; the pages print no
+ * formula, so this is the derivative of the fine stage): with
+ * P = softmax(D^-1/2 q k^T) over each row's selected real keys,
+ *   dv = P^T do,  dS = P (do v^T - rowsum(do * o)),
+ *   dq = D^-1/2 dS k,  dk = D^-1/2 dS^T q.
+ *   q, k, v, o, dO : tiled [B,H,Sp,D] dtype (o and lse from the forward call
+ *                    with the same q2k_idx / q2k_num)
+ *   lse            : [B,H,Sp] fp32 from the forward call
+ *   dq, dk, dv     : tiled [B,H,Sp,D] dtype, caller-owned; padded rows get 0
+ *                    and the dO of padded rows is ignored
+ *   workspace      : device memory of vsa_sparse_attn_bwd_workspace bytes,
+ *                    caller-owned, contents need not be initialised
+ * 16-bit operands (P, dS rounded to dtype for the tensor cores), fp32
+ * accumulation.  256-token blocks only (VSA_ERR_UNSUPPORTED otherwise).
+ * Block ids outside [0, NB) and counts outside [0, max_k] are skipped /
+ * clamped and set VSA_ERR_BAD_INDEX in the device status word.
+ */
+VSA_API int vsa_sparse_attn_bwd_workspace(vsa_plan_t plan, int B, int H, int max_k, size_t *bytes);
+VSA_API int vsa_sparse_attn_bwd(vsa_plan_t plan, vsa_dtype_t dtype, const uint16_t *q, const uint16_t *k,
+                                const uint16_t *v, const uint16_t *o, const float *lse, const uint16_t *dO,
+                                const int32_t *q2k_idx, const int32_t *q2k_num, int max_k, int B, int H, int D,
+                                uint16_t *dq, uint16_t *dk, uint16_t *dv, void *workspace, vsa_stream_t stream);
+
+/*
  * Synchronise `stream`, then read and clear the status word of the current
  * device: *device_status receives VSA_OK or the first device-detected error
  * (VSA_ERR_BAD_INDEX, VSA_ERR_TIMEOUT) since the last read.

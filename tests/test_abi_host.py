@@ -157,6 +157,17 @@ def test_calls_reject_invalid_arguments(L):
     assert L.vsa_tile_coarse(*args(-1, None, None, None, None, F)) == vsa.VSA_ERR_TOPK
     assert L.vsa_tile_coarse(*args(0, None, F, None, None, F)) == vsa.VSA_ERR_INVALID_ARG
     assert L.vsa_tile_coarse(*args(4, None, None, F, None, F)) == vsa.VSA_ERR_INVALID_ARG
+    # backward: dtype, pointers, sizes, block size
+    bw = lambda dt, ws, mk, D, plan=h: (plan, dt, F, F, F, F, F, F, F, F, mk, 1, 2, D, F, F, F, ws, None)
+    assert L.vsa_sparse_attn_bwd(*bw(3, F, 4, 128)) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_sparse_attn_bwd(*bw(vsa.VSA_BF16, None, 4, 128)) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_sparse_attn_bwd(*bw(vsa.VSA_BF16, M, 4, 128)) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_sparse_attn_bwd(*bw(vsa.VSA_BF16, F, 0, 128)) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_sparse_attn_bwd(*bw(vsa.VSA_F16, F, 4, 64)) == vsa.VSA_ERR_UNSUPPORTED
+    t64 = vsa.Plan(4, 4, 8, (4, 4, 4))
+    assert L.vsa_sparse_attn_bwd(*bw(vsa.VSA_BF16, F, 4, 128, t64.handle)) == vsa.VSA_ERR_UNSUPPORTED
+    assert L.vsa_sparse_attn_bwd_workspace(h, 1, 2, 0, ctypes.byref(ctypes.c_size_t())) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_sparse_attn_bwd_workspace(h, 1, 2, 4, None) == vsa.VSA_ERR_INVALID_ARG
     # gated untile
     assert L.vsa_untile_gate(h, 5, F, F, F, F, 1, 2, 128, None) == vsa.VSA_ERR_INVALID_ARG
     assert L.vsa_untile_gate(h, vsa.VSA_BF16, F, F, M, F, 1, 2, 128, None) == vsa.VSA_ERR_INVALID_ARG
@@ -169,3 +180,10 @@ def test_valid_call_without_gpu_reports_no_device(L):
     p = vsa.Plan(8, 16, 16)
     F = ctypes.c_void_p(FAKE)
     assert L.vsa_tile(p.handle, F, F, None, 1, 2, 128, None) == vsa.VSA_ERR_NO_DEVICE
+
+
+def test_backward_workspace_size_is_host_only():
+    p = vsa.Plan(31, 22, 40)
+    a = vsa.bwd_workspace_bytes(p, 1, 24, 64)
+    b = vsa.bwd_workspace_bytes(p, 1, 24, 65)
+    assert a > 2 * 24 * p.Sp * 4 and b > a and a % 4 == 0

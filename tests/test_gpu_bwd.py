@@ -1,0 +1,147 @@
+"""GPU parity of the fine stage's backward (vsa_sparse_attn_bwd) against the
+fp64 oracle (gradients of the attention step of "FastVideo VSA" with the
+selection fixed).
+
+Tolerances, relative to the size of each gradient (16-bit operands P and dS,
+16-bit outputs, fp32 accumulation; delta is formed from the 16-bit o of the
+forward): max-abs error <= 2.5e-2 x max |ref| and mean-abs error <= 8e-3 x
+mean |ref|, per tensor.
+"""
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_video_gather_b200 as vsa
+import oracle
+from block_sparse_video_gather_b200 import build as vsa_build
+from block_sparse_video_gather_b200 import workloads
+from tests import gpu_helpers as H
+
+pytestmark = pytest.mark.gpu
+
+MAX_REL = 2.5e-2
+MEAN_REL = 8e-3
+TDT = {"bf16": torch.bfloat16, "f16": torch.float16}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    vsa_build.build()
+    vsa.lib()
+
+
+def _dev(bits, dtype):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(TDT[dtype])
+
+
+def _host(t):
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def _vals(bits, dtype):
+    return oracle.half_to_f32(bits, dtype).astype(np.float64)
+
+
+def _check(name, got, ref):
+    err = np.abs(got - ref)
+    mx, mn = float(err.max()), float(err.mean())
+    rmx, rmn = float(np.abs(ref).max()), float(np.abs(ref).mean())
+    print(f"{name}: max {mx:.3e} (ref {rmx:.3e}, ratio {mx / max(rmx, 1e-30):.3e}) "
+          f"mean {mn:.3e} (ref {rmn:.3e}, ratio {mn / max(rmn, 1e-30):.3e})")
+    assert mx <= MAX_REL * rmx, name
+    assert mn <= MEAN_REL * rmn, name
+
+
+def _problem(wl, dtype, k, seed, zero_rows=True, garbage_pad=False):
+    g = oracle.geometry_of(wl)
+    inp = workloads.make_inputs(wl, dtype=dtype)
+    qt, kt, vt = (oracle.tile(g, inp[n]) for n in ("q", "k", "v"))
+    rng = np.random.default_rng(seed)
+    to16 = workloads.f32_to_f16_bits if dtype == "f16" else workloads.f32_to_bf16_bits
+    do = oracle.tile(g, to16(rng.standard_normal(inp["q"].shape).astype(np.float32)))
+    if garbage_pad:  # the dO of padded rows must be ignored
+        pad = ~H.real_rows(wl)
+        do[:, :, pad] = to16(np.full((1,), 7.0, np.float32))[0]
+    if k is None:
+        (idx, num), _ = oracle.coarse(g, qt, kt, wl.topk, dtype)
+    else:
+        k = min(k, g.NB)
+        num = rng.integers(0 if zero_rows else 1, k + 1, size=(wl.B, wl.H, g.NB)).astype(np.int32)
+        idx = np.full((wl.B, wl.H, g.NB, k), -1, dtype=np.int32)
+        for pos in np.ndindex(wl.B, wl.H, g.NB):
+            idx[pos][:num[pos]] = np.sort(rng.permutation(g.NB)[:num[pos]])
+    return g, qt, kt, vt, do, idx, num
+
+
+def _gpu_bwd(wl, dtype, qt, kt, vt, do, idx, num):
+    plan = vsa.Plan.of(wl)
+    q, k, v, d = (_dev(x, dtype) for x in (qt, kt, vt, do))
+    ti, tn = torch.from_numpy(idx).cuda(), torch.from_numpy(num).cuda()
+    o, lse = vsa.sparse_attn_fwd(plan, q, k, v, ti, tn)
+    dq, dk, dv = vsa.sparse_attn_bwd(plan, q, k, v, o, lse, d, ti, tn)
+    torch.cuda.synchronize()
+    assert vsa.get_status() == vsa.VSA_OK
+    return _host(dq), _host(dk), _host(dv)
+
+
+CASES = [
+    # name, workload kwargs, k (None: oracle top-k), dtype, garbage in padded dO
+    ("tiny", None, None, "bf16", False),
+    ("ragged-empty-rows", dict(T=5, Hg=9, Wg=11, H=2), 3, "bf16", True),
+    ("batch2-f16", dict(T=6, Hg=12, Wg=20, B=2, H=2), 4, "f16", False),
+    ("prefix", dict(T=4, Hg=16, Wg=16, n_prefix=300, H=3), 5, "bf16", True),
+    ("all-blocks", dict(T=8, Hg=8, Wg=16, H=2), 0, "bf16", False),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
+def test_bwd_matches_oracle_everywhere(case):
+    name, kw, k, dtype, garbage = case
+    wl = workloads.WORKLOADS[name] if kw is None else workloads.custom(topk=1, **kw)
+    if k == 0:  # every block selected: dense attention over the real tokens
+        g = oracle.geometry_of(wl)
+        k = g.NB
+        g, qt, kt, vt, do, _, _ = _problem(wl, dtype, k, seed=7)
+        idx = np.broadcast_to(np.arange(g.NB, dtype=np.int32), (wl.B, wl.H, g.NB, g.NB)).copy()
+        num = np.full((wl.B, wl.H, g.NB), g.NB, dtype=np.int32)
+    else:
+        g, qt, kt, vt, do, idx, num = _problem(wl, dtype, k, seed=7, garbage_pad=garbage)
+    dq, dk, dv = _gpu_bwd(wl, dtype, qt, kt, vt, do, idx, num)
+    real = H.real_rows(wl)
+    rows = np.arange(wl.B * wl.H * g.Sp, dtype=np.int64)
+    ref_dq = oracle.attn_bwd_q_rows(g, qt, kt, vt, do, idx, num, rows, dtype).reshape(dq.shape)
+    ref_dk, ref_dv = oracle.attn_bwd_kv(g, qt, kt, vt, do, idx, num, dtype)
+    _check(f"{name} dq", _vals(dq, dtype)[:, :, real], ref_dq[:, :, real])
+    _check(f"{name} dk", _vals(dk, dtype)[:, :, real], ref_dk[:, :, real])
+    _check(f"{name} dv", _vals(dv, dtype)[:, :, real], ref_dv[:, :, real])
+    pad = ~real
+    for t in (dq, dk, dv):
+        assert (t[:, :, pad] == 0).all()
+
+
+def test_bwd_full_size_fastwan():
+    """The benchmark workload: dq on sampled rows against the oracle; dk and dv
+    through identities that hold at any size: sum over keys of dk is 0 and sum
+    of dv is the sum of do over rows with a non-empty selection."""
+    wl = workloads.WORKLOADS["fastwan"]
+    g, qt, kt, vt, do, idx, num = _problem(wl, "bf16", None, seed=11)
+    dq, dk, dv = _gpu_bwd(wl, "bf16", qt, kt, vt, do, idx, num)
+    real = np.flatnonzero(H.real_rows(wl))
+    rng = np.random.default_rng(12)
+    rows = np.concatenate([bh * g.Sp + np.unique(np.concatenate([rng.choice(real, 24, replace=False),
+                                                                 real[:2], real[-2:]]))
+                           for bh in range(wl.H)])
+    ref = oracle.attn_bwd_q_rows(g, qt, kt, vt, do, idx, num, rows)
+    _check("fastwan dq rows", _vals(dq, "bf16").reshape(-1, 128)[rows], ref)
+    realm = H.real_rows(wl)
+    dkv = _vals(dk, "bf16")[0][:, realm]
+    dvv = _vals(dv, "bf16")[0][:, realm]
+    dov = _vals(do, "bf16")[0][:, realm]
+    for h in range(wl.H):
+        s = dkv[h].sum(axis=0)
+        assert np.abs(s).max() <= 2e-2 * np.abs(dkv[h]).sum(axis=0).max(), h
+        # every fastwan row has topk > 0 selections
+        np.testing.assert_allclose(dvv[h].sum(axis=0), dov[h].sum(axis=0), rtol=0,
+                                   atol=2e-2 * np.abs(dov[h]).sum(axis=0).max())
