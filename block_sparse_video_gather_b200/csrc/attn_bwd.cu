@@ -12,7 +12,7 @@
 // gradients are zero whatever do holds at padded rows.
 //
 // Four launches:
-//   bwd_prep  delta_i = do_i . o_i and lse2_i = lse_i log2(e) per tiled row.
+//   bwd_prep  -delta_i = -do_i . o_i and -lse_i log2(e) per tiled row.
 //   k2q       the transposed selection: for each key block, the query blocks
 //             that list it (a repeated id is listed again), ascending; rows are
 //             placed in order, so the lists do not depend on thread timing.
@@ -33,9 +33,11 @@
 // of 128 rows x 128 channels (two 64-channel boxes, 128-byte swizzle) and is
 // read either way through its descriptor.
 //
-// Warp roles (256 threads): warp 0 TMA producer, warp 1 TMEM owner and MMA
-// issuer, warps 4-7 one thread per TMEM lane (tile row) for the elementwise
-// step and the epilogue.  Every mbarrier wait is bounded; on expiry the kernel
+// Warp roles (384 threads): warp 0 TMA producer, warp 1 TMEM owner and MMA
+// issuer, warps 4-11 two warpgroups for the elementwise step and the
+// epilogue: a thread owns one TMEM lane (tile row), warpgroup w the columns
+// [64w, 64w + 64) of it.  In dkdv, P^T and dS^T are written back over S^T and
+// dP^T, so both warpgroups finish reading before either writes (named barrier).  Every mbarrier wait is bounded; on expiry the kernel
 // records VSA_ERR_TIMEOUT, drains its copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -50,11 +52,16 @@ namespace {
 
 using namespace tiles;
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
 constexpr uint32_t kHalfBytes = 128 * 128;      // 128 rows x 64 16-bit channels
 constexpr uint32_t kTileBytes = 2 * kHalfBytes;  // 128 rows x 128 channels
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
+// Register split: launched at 168 per thread (384 x 168 = 64512); warpgroup 0
+// (producer, MMA issuer, two idle warps) gives back down to 104 and the two
+// elementwise warpgroups take 200 each: 128 x 104 + 256 x 200 = 64512.
+constexpr int kRegsLaunch = 168, kRegsLow = 104, kRegsHigh = 200;
+static_assert(kThreads * kRegsLaunch == 128 * kRegsLow + 256 * kRegsHigh, "register split must match the launch");
 
 template <bool F16>
 struct Idesc {
@@ -75,6 +82,39 @@ __device__ __forceinline__ int tile_bits(const Geo& g, int blk, int half, uint32
   return st;
 }
 
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// Barrier among the 256 threads of the two elementwise warpgroups.
+__device__ __forceinline__ void wg_pair_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+// P and dS for 32 columns of this thread's row: x = s c2 + nl, P = 2^x (0 where
+// m has no bit), dS = P (dp + nd).  nl, nd: two columns per 64-bit word.
+template <bool F16>
+__device__ __forceinline__ void p_ds32(const uint32_t (&sv)[32], const uint32_t (&dv)[32], uint64_t c2,
+                                       const uint64_t* nl, const uint64_t* nd, uint32_t m, uint32_t (&pk)[16],
+                                       uint32_t (&dk)[16]) {
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const uint64_t x = fma2(u2pack(sv[2 * j], sv[2 * j + 1]), c2, nl[j]);
+    float xa, xb;
+    f2unpack(x, xa, xb);
+    float pa = ex2_approx(xa), pb = ex2_approx(xb);
+    if (m != 0xffffffffu) {
+      pa = ((m >> (2 * j)) & 1u) ? pa : 0.0f;
+      pb = ((m >> (2 * j + 1)) & 1u) ? pb : 0.0f;
+    }
+    const uint64_t ds = mul2(f2pack(pa, pb), add2(u2pack(dv[2 * j], dv[2 * j + 1]), nd[j]));
+    float da, db;
+    f2unpack(ds, da, db);
+    pk[j] = pack_half2<F16>(pa, pb);
+    dk[j] = pack_half2<F16>(da, db);
+  }
+}
+
 __device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
@@ -85,8 +125,10 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint3
 
 struct BwdBarriers {
   uint64_t a_full;            // resident tiles (K,V for dkdv; Q,dO for dq)
-  uint64_t full[2], empty[2];  // streamed stages
-  uint64_t s_full, ds_full, done, drain;
+  uint64_t full[2], empty[2];  // streamed stages (dq: the V ring)
+  uint64_t kfull[3], kempty[3];  // dq: the K ring
+  uint32_t mask[3][4];            // validity bits of the streamed tile of each stage (written by the producer)
+  uint64_t s_full, s_free, ds_full, ds_free, done, drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -102,8 +144,14 @@ __device__ __forceinline__ void init_barriers(BwdBarriers* b) {
     mbar_init(&b->full[s], 1);
     mbar_init(&b->empty[s], 1);
   }
+  for (int s = 0; s < 3; ++s) {
+    mbar_init(&b->kfull[s], 1);
+    mbar_init(&b->kempty[s], 1);
+  }
   mbar_init(&b->s_full, 1);
-  mbar_init(&b->ds_full, 128);
+  mbar_init(&b->s_free, 256);
+  mbar_init(&b->ds_full, 256);
+  mbar_init(&b->ds_free, 1);
   mbar_init(&b->done, 1);
   mbar_init(&b->drain, 1);
   b->abort = 0;
@@ -134,6 +182,27 @@ __device__ __forceinline__ void store_row(uint32_t taddr, float scale, uint16_t*
   }
 }
 
+// Columns [c0, c0 + 64) of this thread's lane (fp32, scaled) to 64 16-bit values at dst.
+template <bool F16>
+__device__ __forceinline__ void store_half_row(uint32_t taddr, float scale, uint16_t* dst, bool load, bool zero) {
+  uint4* out = reinterpret_cast<uint4*>(dst);
+  zero = zero || !load;
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    uint32_t v[32];
+    if (load) {
+      tmem_ld32(taddr + c * 32, v);
+      tmem_wait_ld();
+    }
+    uint32_t w[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      w[j] = zero ? 0u : pack_half2<F16>(__uint_as_float(v[2 * j]) * scale, __uint_as_float(v[2 * j + 1]) * scale);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) out[c * 4 + j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+  }
+}
+
 struct BwdParams {
   Geo g;
   int BH, max_k;
@@ -141,8 +210,8 @@ struct BwdParams {
   const int32_t* num;
   const int32_t* k2q_off;  // [BH][NB + 1]
   const int32_t* k2q;      // [BH][NB * max_k]
-  const float* lse2;       // [BH * Sp]
-  const float* delta;      // [BH * Sp]
+  const float* nlse2;      // [BH * Sp]  -lse log2(e)
+  const float* ndelta;     // [BH * Sp]  -(do . o)
   uint16_t* dq;
   uint16_t* dk;
   uint16_t* dv;
@@ -190,6 +259,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
+  if (warp < 4) {
+  regs_dec<kRegsLow>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     const uint64_t pol_last = policy_evict_last();
@@ -209,6 +280,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int qb = __ldg(list + (u >> 1));
         const long long qrow = base + static_cast<long long>(qb) * 256 + (u & 1) * 128;
         uint8_t* st = smem + kKV_Stage + s * kKV_StageBytes;
+        {  // query-tile validity for the elementwise warps, published by the arrive below
+          uint32_t w[4];
+          tile_bits(g, qb, u & 1, w);
+          if (lane < 4) bars->mask[s][lane] = pick4(w, lane);
+          __syncwarp();
+        }
         mbar_arrive_expect_tx_w(&bars->full[s], 2 * kTileBytes + 1024);
         for (int hf = 0; hf < 2; ++hf) {
           tma_load_2d_w(st + hf * kHalfBytes, &tm_q, hf * 64, static_cast<int>(qrow), &bars->full[s], pol_last);
@@ -216,8 +293,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         pol_last);
         }
         if (lane == 0) {
-          bulk_load(smem + kKV_L + s * 1024, p.lse2 + qrow, 512, &bars->full[s]);
-          bulk_load(smem + kKV_L + s * 1024 + 512, p.delta + qrow, 512, &bars->full[s]);
+          bulk_load(smem + kKV_L + s * 1024, p.nlse2 + qrow, 512, &bars->full[s]);
+          bulk_load(smem + kKV_L + s * 1024 + 512, p.ndelta + qrow, 512, &bars->full[s]);
         }
         __syncwarp();
         ++issued;
@@ -269,8 +346,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     mma_commit_w(&bars->done);
     mma_commit_w(&bars->drain);
     mbar_wait_drain(&bars->drain, 0, kTimeoutNs);
-  } else if (warp >= 4) {
+  }
+  } else {
+    regs_inc<kRegsHigh>();
     // ------------------------------------------------------------ elementwise + epilogue
+    const int wg = (warp - 4) >> 2;     // query columns [64 wg, 64 wg + 64)
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // key row of the tile
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
@@ -278,44 +358,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t kw[4];
     tile_bits(g, kb, half, kw);
     const bool kvalid = (pick4(kw, r >> 5) >> (r & 31)) & 1u;
-    const float c2 = p.scale_log2;
+    const uint64_t c2 = f2pack(p.scale_log2, p.scale_log2);
     bool ok = true;
     for (int u = 0; u < nq && ok; ++u) {
       const int s = u & 1;
-      const int qb = __ldg(list + (u >> 1));
-      uint32_t qw[4];
-      tile_bits(g, qb, u & 1, qw);
-      if (!kvalid) qw[0] = qw[1] = qw[2] = qw[3] = 0u;
       if (!(ok = wwait(&bars->full[s], (u >> 1) & 1, bars, p.status))) break;
+      uint32_t qw[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) qw[i] = bars->mask[s][i];
       if (!(ok = wwait(&bars->s_full, u & 1, bars, p.status))) break;
       tc_fence_after();
-      const float* L2 = reinterpret_cast<const float*>(smem + kKV_L + s * 1024);
-      const float* DL = L2 + 128;
-#pragma unroll 1
-      for (int ch = 0; ch < 4; ++ch) {
+      const uint64_t* NL = reinterpret_cast<const uint64_t*>(smem + kKV_L + s * 1024);
+      const uint64_t* ND = NL + 64;
+      uint32_t pk[2][16], dk16[2][16];
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        const int ch = 2 * wg + cc;
         uint32_t sv[32], dv[32];
         tmem_ld32(tS + ch * 32, sv);
         tmem_ld32(tP + ch * 32, dv);
         tmem_wait_ld();
-        const uint32_t m = pick4(qw, ch);
-        uint32_t pk[16], dk16[16];
+        p_ds32<F16>(sv, dv, c2, NL + 16 * ch, ND + 16 * ch, kvalid ? pick4(qw, ch) : 0u, pk[cc], dk16[cc]);
+      }
+      wg_pair_sync();  // every column of S^T and dP^T has been read
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          float pr[2], dr[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int c = 2 * j + e;
-            const int q = ch * 32 + c;
-            const float x = __fmaf_rn(__uint_as_float(sv[c]), c2, -L2[q]);
-            const float pp = ((m >> c) & 1u) ? ex2_approx(x) : 0.0f;
-            pr[e] = pp;
-            dr[e] = pp * (__uint_as_float(dv[c]) - DL[q]);
-          }
-          pk[j] = pack_half2<F16>(pr[0], pr[1]);
-          dk16[j] = pack_half2<F16>(dr[0], dr[1]);
-        }
-        tmem_st16(tS + ch * 16, pk);
-        tmem_st16(tP + ch * 16, dk16);
+      for (int cc = 0; cc < 2; ++cc) {
+        const int ch = 2 * wg + cc;
+        tmem_st16(tS + ch * 16, pk[cc]);
+        tmem_st16(tP + ch * 16, dk16[cc]);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -325,8 +395,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const long long row = base + static_cast<long long>(kb) * 256 + half * 128 + r;
     const bool load = ok && nq > 0;  // warp-uniform
-    store_row<F16>(tS + 256, 1.0f, p.dv + row * 128, load, false);
-    store_row<F16>(tS + 384, p.scale, p.dk + row * 128, load, false);
+    if (wg == 0)
+      store_row<F16>(tS + 256, 1.0f, p.dv + row * 128, load, false);
+    else
+      store_row<F16>(tS + 384, p.scale, p.dk + row * 128, load, false);
   }
 
   tc_fence_before();
@@ -341,8 +413,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------
 // dq
 // ---------------------------------------------------------------------------
-constexpr uint32_t kQ_Q = 0, kQ_DO = kTileBytes, kQ_K = 2 * kTileBytes;  // K stages: 2 x 32 KB
-constexpr uint32_t kQ_V = kQ_K + 2 * kTileBytes;                          // V stages: 2 x 32 KB
+// K is read by the first MMA of a tile and by its last (dQ += dS K), V only by
+// the first: three K stages and two V stages keep the next copies in flight.
+constexpr uint32_t kQ_Q = 0, kQ_DO = kTileBytes, kQ_K = 2 * kTileBytes;  // K stages: 3 x 32 KB
+constexpr uint32_t kQ_V = kQ_K + 3 * kTileBytes;                          // V stages: 2 x 32 KB
 constexpr uint32_t kQ_Bar = kQ_V + 2 * kTileBytes;
 constexpr uint32_t kQ_Smem = kQ_Bar + 256 + 1024;
 
@@ -384,10 +458,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
+  if (warp < 4) {
+  regs_dec<kRegsLow>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     const uint64_t pol_last = policy_evict_last(), pol_first = policy_evict_first();
-    int issued = 0;
+    int issued = 0, issued_k = 0;  // V and K copies issued
     bool qd = false;
     if (n > 0) {
       const int qrow = static_cast<int>(base + static_cast<long long>(qb) * 256 + half * 128);
@@ -398,18 +474,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       qd = true;
       for (int t = 0; t < n; ++t) {
-        const int s = t & 1;
-        if (!wwait(&bars->empty[s], ((t >> 1) & 1) ^ 1, bars, p.status)) break;
         const int kb0 = dq_block(p, row_item, t >> 1);
         const int kb = kb0 < 0 ? 0 : kb0;  // unusable ids load block 0; the elementwise step masks it out
         const int krow = static_cast<int>(base + static_cast<long long>(kb) * 256 + (t & 1) * 128);
-        mbar_arrive_expect_tx_w(&bars->full[s], 2 * kTileBytes);
-        for (int hf = 0; hf < 2; ++hf) {
-          tma_load_2d_w(smem + kQ_K + s * kTileBytes + hf * kHalfBytes, &tm_k, hf * 64, krow, &bars->full[s],
-                        pol_last);
-          tma_load_2d_w(smem + kQ_V + s * kTileBytes + hf * kHalfBytes, &tm_v, hf * 64, krow, &bars->full[s],
-                        pol_last);
+        const int ks = t % 3, vs = t & 1;
+        if (!wwait(&bars->kempty[ks], ((t / 3) & 1) ^ 1, bars, p.status)) break;
+        {  // key-tile validity for the elementwise warps, published by the arrive below
+          uint32_t w[4];
+          tile_bits(g, kb0, t & 1, w);
+          if (lane < 4) bars->mask[ks][lane] = pick4(w, lane);
+          if (kb0 < 0 && lane == 0 && half == 0 && (t & 1) == 0) atomicCAS(p.status, 0u, (unsigned)VSA_ERR_BAD_INDEX);
+          __syncwarp();
         }
+        mbar_arrive_expect_tx_w(&bars->kfull[ks], kTileBytes);
+        for (int hf = 0; hf < 2; ++hf)
+          tma_load_2d_w(smem + kQ_K + ks * kTileBytes + hf * kHalfBytes, &tm_k, hf * 64, krow, &bars->kfull[ks],
+                        pol_last);
+        if (!wwait(&bars->empty[vs], ((t >> 1) & 1) ^ 1, bars, p.status)) {
+          ++issued_k;
+          break;
+        }
+        mbar_arrive_expect_tx_w(&bars->full[vs], kTileBytes);
+        for (int hf = 0; hf < 2; ++hf)
+          tma_load_2d_w(smem + kQ_V + vs * kTileBytes + hf * kHalfBytes, &tm_v, hf * 64, krow, &bars->full[vs],
+                        pol_last);
+        ++issued_k;
         ++issued;
       }
     }
@@ -419,6 +508,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int last = issued - 1 - ((issued - 1 - s) & 1);
         mbar_wait_drain(&bars->full[s], (last >> 1) & 1, kTimeoutNs);
       }
+    for (int s = 0; s < 3; ++s)
+      if (issued_k > s) {
+        const int last = issued_k - 1 - ((issued_k - 1 - s) % 3);
+        mbar_wait_drain(&bars->kfull[s], (last / 3) & 1, kTimeoutNs);
+      }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     const uint64_t dQ = sdesc_sw128(smem_u32(smem + kQ_Q), 16, 1024);
@@ -427,36 +521,57 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t dV = sdesc_sw128(smem_u32(smem + kQ_V), 16, 1024);
     const uint64_t mK = sdesc_sw128(smem_u32(smem + kQ_K), kHalfBytes, 1024);
     constexpr uint64_t kTile = kTileBytes >> 4;
-    bool ok = true;
-    if (n > 0) ok = wwait(&bars->a_full, 0, bars, p.status);
-    for (int t = 0; t < n && ok; ++t) {
-      const int s = t & 1;
-      if (!(ok = wwait(&bars->full[s], (t >> 1) & 1, bars, p.status))) break;
-      tc_fence_after();
+    // S(t+1) and dP(t+1) are issued as soon as the elementwise warps have read
+    // S(t) and dP(t) (s_free), so the tensor core works while they form dS(t).
+    auto issue_sdp = [&](int t) {  // S(t), dP(t); V(t) is released when they complete
+      const int ks = t % 3, vs = t & 1;
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const uint32_t off = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
-        mma_ss_w(tmem + 0, dQ + off, dK + s * kTile + off, Idesc<F16>::KK, kk > 0 ? 1u : 0u);
+        mma_ss_w(tmem + 0, dQ + off, dK + ks * kTile + off, Idesc<F16>::KK, kk > 0 ? 1u : 0u);
       }
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const uint32_t off = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
-        mma_ss_w(tmem + 128, dDO + off, dV + s * kTile + off, Idesc<F16>::KK, kk > 0 ? 1u : 0u);
+        mma_ss_w(tmem + 128, dDO + off, dV + vs * kTile + off, Idesc<F16>::KK, kk > 0 ? 1u : 0u);
       }
       mma_commit_w(&bars->s_full);
+      mma_commit_w(&bars->empty[vs]);
+    };
+    auto wait_kv = [&](int t) {
+      return wwait(&bars->kfull[t % 3], (t / 3) & 1, bars, p.status) &&
+             wwait(&bars->full[t & 1], (t >> 1) & 1, bars, p.status);
+    };
+    bool ok = true;
+    if (n > 0) ok = wwait(&bars->a_full, 0, bars, p.status) && wait_kv(0);
+    if (ok && n > 0) {
+      tc_fence_after();
+      issue_sdp(0);
+    }
+    for (int t = 0; t < n && ok; ++t) {
+      if (!(ok = wwait(&bars->s_free, t & 1, bars, p.status))) break;
+      if (t + 1 < n) {
+        if (!(ok = wait_kv(t + 1))) break;
+        tc_fence_after();
+        issue_sdp(t + 1);
+      }
       if (!(ok = wwait(&bars->ds_full, t & 1, bars, p.status))) break;
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
-        mma_ts_w(tmem + 256, tmem + 384 + kk * 8, mK + s * kTile + kk * (2048 >> 4), Idesc<F16>::TM,
+        mma_ts_w(tmem + 256, tmem + 384 + kk * 8, mK + (t % 3) * kTile + kk * (2048 >> 4), Idesc<F16>::TM,
                  (t > 0 || kk > 0) ? 1u : 0u);
-      mma_commit_w(&bars->empty[s]);
+      mma_commit_w(&bars->kempty[t % 3]);
+      mma_commit_w(&bars->ds_free);
     }
     mma_commit_w(&bars->done);
     mma_commit_w(&bars->drain);
     mbar_wait_drain(&bars->drain, 0, kTimeoutNs);
-  } else if (warp >= 4) {
+  }
+  } else {
+    regs_inc<kRegsHigh>();
     // ------------------------------------------------------------ elementwise + epilogue
+    const int wg = (warp - 4) >> 2;     // key columns [64 wg, 64 wg + 64)
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // query row of the tile
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
@@ -465,47 +580,47 @@ __global__ void __launch_bounds__(kThreads, 1)
     tile_bits(g, qb, half, rw);
     const bool rvalid = (pick4(rw, r >> 5) >> (r & 31)) & 1u;
     const long long row = base + static_cast<long long>(qb) * 256 + half * 128 + r;
-    const float nl2 = rvalid ? -__ldg(p.lse2 + row) : 0.0f;
-    const float dl = rvalid ? __ldg(p.delta + row) : 0.0f;
-    const float c2 = p.scale_log2;
+    const float nl = rvalid ? __ldg(p.nlse2 + row) : 0.0f;
+    const float nd = rvalid ? __ldg(p.ndelta + row) : 0.0f;
+    uint64_t nl2[16], nd2[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      nl2[j] = f2pack(nl, nl);
+      nd2[j] = f2pack(nd, nd);
+    }
+    const uint64_t c2 = f2pack(p.scale_log2, p.scale_log2);
     bool ok = true;
     for (int t = 0; t < n && ok; ++t) {
-      const int kb = dq_block(p, row_item, t >> 1);
-      if (kb < 0 && r == 0 && half == 0 && (t & 1) == 0) atomicCAS(p.status, 0u, (unsigned)VSA_ERR_BAD_INDEX);
-      uint32_t kw[4];
-      tile_bits(g, kb, t & 1, kw);
-      if (!rvalid) kw[0] = kw[1] = kw[2] = kw[3] = 0u;
       if (!(ok = wwait(&bars->s_full, t & 1, bars, p.status))) break;
+      // the key tile's validity bits: written before its copy was announced on kfull
+      if (!(ok = wwait(&bars->kfull[t % 3], (t / 3) & 1, bars, p.status))) break;
+      uint32_t kw[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) kw[i] = bars->mask[t % 3][i];
       tc_fence_after();
-#pragma unroll 1
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t sv[32], dv[32];
-        tmem_ld32(tS + ch * 32, sv);
-        tmem_ld32(tP + ch * 32, dv);
-        tmem_wait_ld();
-        const uint32_t m = pick4(kw, ch);
-        uint32_t dk16[16];
+      uint32_t sv[2][32], dv[2][32], pk[16], dk16[2][16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          float dr[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int c = 2 * j + e;
-            const float x = __fmaf_rn(__uint_as_float(sv[c]), c2, nl2);
-            const float pp = ((m >> c) & 1u) ? ex2_approx(x) : 0.0f;
-            dr[e] = pp * (__uint_as_float(dv[c]) - dl);
-          }
-          dk16[j] = pack_half2<F16>(dr[0], dr[1]);
-        }
-        tmem_st16(tDS + ch * 16, dk16);
+      for (int cc = 0; cc < 2; ++cc) {
+        tmem_ld32(tS + (2 * wg + cc) * 32, sv[cc]);
+        tmem_ld32(tP + (2 * wg + cc) * 32, dv[cc]);
       }
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&bars->s_free);  // S and dP may be overwritten by the next tile
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc)
+        p_ds32<F16>(sv[cc], dv[cc], c2, nl2, nd2, rvalid ? pick4(kw, 2 * wg + cc) : 0u, pk, dk16[cc]);
+      if (t > 0 && !(ok = wwait(&bars->ds_free, (t - 1) & 1, bars, p.status))) break;  // dQ(t-1) read dS
+      tc_fence_after();
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) tmem_st16(tDS + (2 * wg + cc) * 16, dk16[cc]);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars->ds_full);
     }
     if (ok && n > 0) ok = wwait(&bars->done, 0, bars, p.status);
     tc_fence_after();
-    store_row<F16>(tS + 256, p.scale, p.dq + row * 128, ok && n > 0, !rvalid);
+    store_half_row<F16>(tS + 256 + 64 * wg, p.scale, p.dq + row * 128 + 64 * wg, ok && n > 0, !rvalid);
   }
 
   tc_fence_before();
@@ -522,8 +637,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------
 template <bool F16>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint4* __restrict__ o, const uint4* __restrict__ dO,
-                                                       const float* __restrict__ lse, float* __restrict__ lse2,
-                                                       float* __restrict__ delta, long long rows) {
+                                                       const float* __restrict__ lse, float* __restrict__ nlse2,
+                                                       float* __restrict__ ndelta, long long rows) {
   const long long row = static_cast<long long>(blockIdx.x) * 16 + (threadIdx.x >> 4);
   const int chunk = threadIdx.x & 15;
   float acc = 0.0f;
@@ -551,8 +666,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint4* __restrict__
 #pragma unroll
   for (int off = 8; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
   if (row < rows && chunk == 0) {
-    delta[row] = acc;
-    lse2[row] = __ldg(lse + row) * kLog2e;
+    ndelta[row] = -acc;
+    nlse2[row] = -__ldg(lse + row) * kLog2e;
   }
 }
 
@@ -664,8 +779,8 @@ cudaError_t launch_attn_bwd(const Geo& g, const AttnBwdArgs& a, cudaStream_t str
   p.num = a.num;
   p.k2q_off = k2q_off;
   p.k2q = k2q;
-  p.lse2 = lse2;
-  p.delta = delta;
+  p.nlse2 = lse2;
+  p.ndelta = delta;
   p.dq = a.dq;
   p.dk = a.dk;
   p.dv = a.dv;
