@@ -228,6 +228,190 @@ def cpu_baseline_sample(wl, seconds_hint=20.0):
                        f"estimated {est:.0f} s per step")}
 
 
+BWD_SOURCES = [os.path.join(ROOT, "block_sparse_video_gather_b200", "csrc", f)
+               for f in ("attn_bwd.cu", "common.cuh", "tiles.cuh")]
+BWD_PROFILE = os.path.join(ROOT, "profiles", "attn_bwd_fastwan.md")
+
+
+def bwd_traffic(workload: str):
+    """DRAM bytes per backward call from the committed ncu summary (None if absent or stale)."""
+    if not os.path.exists(BWD_PROFILE):
+        return None
+    h = hashlib.sha256()
+    for f in BWD_SOURCES:
+        h.update(open(f, "rb").read())
+    text = open(BWD_PROFILE).read()
+    m_src = re.search(r"source_hash:\s*([0-9a-f]+)", text)
+    m_wl = re.search(r"bench_workload:\s*(\w+)", text)
+    m_b = re.search(r"traffic_bytes_per_call:\s*([0-9.eE+]+)", text)
+    if not (m_src and m_wl and m_b) or m_src.group(1) != h.hexdigest()[:16] or m_wl.group(1) != workload:
+        return None
+    return float(m_b.group(1))
+
+
+def bwd_cpu_baseline(wl, inp, do_untiled, idx, num, flops, seconds_hint=20.0):
+    """Oracle backward on a bounded sample: dq of sampled query rows, scaled to all rows.
+    The oracle's key side costs the same per query row (softmax, dP, then one
+    accumulation), so the full backward is estimated at twice the dq cost."""
+    import oracle
+    g = oracle.geometry_of(wl)
+    qt, kt, vt = (oracle.tile(g, inp[n]) for n in ("q", "k", "v"))
+    dot = oracle.tile(g, do_untiled)
+    total_rows = wl.B * wl.H * g.Sp
+    rng = np.random.default_rng(3)
+    n, t, done = 128, 0.0, 0
+    while t < seconds_hint * 0.5 and done < total_rows:
+        rows = np.sort(rng.choice(total_rows, size=min(n, total_rows), replace=False))
+        t1 = time.perf_counter()
+        oracle.attn_bwd_q_rows(g, qt, kt, vt, dot, idx, num, rows)
+        t += time.perf_counter() - t1
+        done += len(rows)
+        n *= 2
+    est = 2.0 * t * total_rows / done
+    return {"value": flops / est / 1e12, "unit": "TFLOP/s", "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": (f"oracle dq on {done} of {total_rows} query rows ({t:.1f} s), scaled to all rows and "
+                       f"doubled for dk/dv; estimated {est:.0f} s per backward")}
+
+
+def run_backward(args, wl, world, rank, local, pg):
+    """One step = one vsa_sparse_attn_bwd call (prep, transposed index, dk/dv, dq) on
+    inputs resident in HBM; the selection, o and lse come from a forward call."""
+    import torch
+    import block_sparse_video_gather_b200 as vsa
+    if wl.block_tokens != 256 or wl.map_driven:
+        raise SystemExit("the backward bench takes a top-k workload with 256-token blocks")
+    inp = workloads.make_inputs(wl, dtype=args.dtype)
+    tdt = torch.float16 if args.dtype == "f16" else torch.bfloat16
+    plan = vsa.Plan.of(wl)
+    rng = np.random.default_rng(5)
+    to16 = workloads.f32_to_f16_bits if args.dtype == "f16" else workloads.f32_to_bf16_bits
+    do_untiled = to16(rng.standard_normal(inp["q"].shape).astype(np.float32))  # gradient of the untiled o
+    dev16 = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).cuda().view(tdt)
+    fwd = vsa.Forward(plan, wl.B, wl.H, wl.topk, dtype=tdt)
+    fwd(dev16(inp["q"]), dev16(inp["k"]), dev16(inp["v"]))
+    do = vsa.tile(plan, dev16(do_untiled))  # tiled; padded rows zero
+    ws = torch.empty(vsa.bwd_workspace_bytes(plan, wl.B, wl.H, fwd.idx.shape[-1]), dtype=torch.uint8, device="cuda")
+    dq, dk, dv = (torch.empty_like(fwd.qt) for _ in range(3))
+    stream = torch.cuda.current_stream()
+
+    def step():
+        vsa.sparse_attn_bwd(plan, fwd.qt, fwd.kt, fwd.vt, fwd.ot, fwd.lse, do, fwd.idx, fwd.num, dq, dk, dv, ws)
+
+    def sync_all():
+        torch.cuda.synchronize()
+        if pg:
+            pg.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(x: float) -> float:
+        if not pg:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert vsa.get_status() == vsa.VSA_OK
+    fwd_flops = selected_flops(wl, fwd.num.cpu().numpy())
+    flops = 2.5 * fwd_flops  # the usual count: five products of the forward's size, two of them repeated
+    mma_flops = 3.5 * fwd_flops  # what the two kernels execute: 4 (dk/dv) + 3 (dq) products of half that size
+
+    props = torch.cuda.get_device_properties(local)
+    gpu_id = str(getattr(props, "uuid", local))
+    if gpu_id and not gpu_id.startswith("GPU-") and len(gpu_id) >= 32:
+        gpu_id = "GPU-" + gpu_id
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    time.sleep(0.3)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sync_all()
+    t0.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    t1.record(stream)
+    sync_all()
+    clocks = sampler.stop()
+    elapsed = max_over_ranks(t0.elapsed_time(t1) / 1e3)
+    call_avg = max_over_ranks(float(np.mean([a.elapsed_time(b) / 1e3 for a, b in ev])))
+    assert vsa.get_status() == vsa.VSA_OK
+
+    # end to end: tiled q, k, v, o, do, lse and the selection copied in, dq, dk, dv copied out
+    host_in = {n: t.cpu().pin_memory() for n, t in (("q", fwd.qt), ("k", fwd.kt), ("v", fwd.vt), ("o", fwd.ot),
+                                                     ("do", do), ("lse", fwd.lse), ("idx", fwd.idx),
+                                                     ("num", fwd.num))}
+    dev_in = {n: torch.empty_like(t, device="cuda") for n, t in host_in.items()}
+    host_out = [torch.empty(dq.shape, dtype=tdt).pin_memory() for _ in range(3)]
+
+    def e2e_step():
+        for n in dev_in:
+            dev_in[n].copy_(host_in[n], non_blocking=True)
+        vsa.sparse_attn_bwd(plan, dev_in["q"], dev_in["k"], dev_in["v"], dev_in["o"], dev_in["lse"], dev_in["do"],
+                            dev_in["idx"], dev_in["num"], dq, dk, dv, ws)
+        for h, d in zip(host_out, (dq, dk, dv)):
+            h.copy_(d, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sync_all()
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    sync_all()
+    e2e_elapsed = max_over_ranks(e0.elapsed_time(e1) / 1e3)
+    assert vsa.get_status() == vsa.VSA_OK
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+
+    if rank == 0:
+        burst, _, _, peak_kind = measured_peaks()
+        achieved = mma_flops / call_avg / 1e12
+        line = {
+            "metric": "VSA sparse-attn bwd effective TFLOP/s (selected blocks) on 1 B200",
+            "value": world * flops * args.steps / elapsed / 1e12,
+            "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": elapsed / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": args.dtype, "data": "synthetic (seeded; the recipe in block_sparse_video_gather_b200/workloads.py)",
+            "config": {
+                "workload": WORKLOAD_TEXT[args.workload], "pass": "backward of the fine stage (selection fixed)",
+                "B": wl.B, "H": wl.H, "D": wl.D, "grid": [wl.T, wl.Hg, wl.Wg], "block": list(wl.block),
+                "num_blocks": wl.num_blocks, "topk": wl.topk,
+                "flop_count": "2.5 x the forward's selected-block FLOPs",
+                "tflop_per_step": flops / 1e12, "call_ms": call_avg * 1e3,
+                "l2": "inputs larger than L2: tiled q, k, v, o, do %.0f MB per step" % (5 * fwd.qt.numel() * 2 / 1e6),
+                "parallelism": f"replicas x{world}",
+            },
+            "roofline": {
+                "bound": "tensor", "kernel": "attn_bwd (prep + k2q + dkdv + dq, one call)", "achieved": achieved,
+                "peak": burst, "unit": "TFLOP/s", "frac": achieved / burst,
+                "flops_counted": "products the kernels execute: 3.5 x the forward's selected-block FLOPs",
+                "peak_source": f"{peak_kind} bf16 burst (MEASURED_PEAKS.json)" if peak_kind == "measured"
+                else "fallback 1.59 PFLOP/s",
+                "traffic": bwd_traffic(args.workload),
+            },
+            "clocks": clocks,
+            "e2e": {"value": world * flops * args.steps / e2e_elapsed / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_elapsed / args.steps * 1e3},
+            "gpu_launches": args.steps * 4,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = bwd_cpu_baseline(wl, inp, do_untiled, fwd.idx.cpu().numpy(),
+                                                    fwd.num.cpu().numpy(), flops)
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -237,6 +421,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-rows", type=int, default=2048, help="query rows per reference step")
     ap.add_argument("--dtype", default="bf16", choices=["bf16", "f16"], help="16-bit format of q, k, v, o")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the fine stage's backward (dq, dk, dv) instead of the forward step")
     ap.add_argument("--unfused", action="store_true",
                     help="run the front end as separate tile / coarse launches instead of one")
     ap.add_argument("--gate", action="store_true",
@@ -268,6 +454,10 @@ def main():
     if pg:
         pg.barrier()
     vsa.lib()
+
+    if args.backward:
+        run_backward(args, wl, world, rank, local, pg)
+        return
 
     inp = workloads.make_inputs(wl, dtype=args.dtype, gate=args.gate)
     tdt = torch.float16 if args.dtype == "f16" else torch.bfloat16
