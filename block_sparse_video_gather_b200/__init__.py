@@ -430,22 +430,85 @@ class Forward:
     def fine(self):
         sparse_attn_fwd(self.plan, self.qt, self.kt, self.vt, self.idx, self.num, o_out=self.ot, lse_out=self.lse)
 
-    def back(self, gate=None):
+    def back(self, gate=None, out=None):
+        out = self.o if out is None else out
         if self.gated:
-            untile_gate(self.plan, self.ot, self.oc, gate, out=self.o)
+            untile_gate(self.plan, self.ot, self.oc, gate, out=out)
         else:
-            untile(self.plan, self.ot, out=self.o)
+            untile(self.plan, self.ot, out=out)
+        return out
 
-    def __call__(self, q, k, v, block_map=None, gate=None):
+    def __call__(self, q, k, v, block_map=None, gate=None, out=None):
+        """One forward step; o goes to `out` when given (else to self.o)."""
         if self.gated != (gate is not None):
             raise ValueError("a gate is required exactly when the Forward was built with gated=True")
         self.front(q, k, v, block_map)
         self.fine()
-        self.back(gate)
-        return self.o, self.lse
+        return self.back(gate, out), self.lse
 
     def launches(self, block_map: bool = False) -> int:
         """Kernels one call launches."""
         if self.fused:
             return 3 + (1 if block_map else 0)  # front (+ map_to_index), attention, untile
         return 6 + (1 if (self.gated and block_map) else 0)  # 3 tiles, index stage (+compress), attention, untile
+
+
+class HostPipeline:
+    """Forward steps on pinned host tensors with the copies overlapped.
+
+    submit(q, k, v, o[, block_map, gate]) enqueues one step: the inputs go to
+    the device on a copy stream (into one of two input slots), the forward runs
+    on a compute stream once they have landed, and o comes back on a second
+    copy stream (from one of two output slots).  While step i computes, step
+    i+1's inputs and step i-1's output are in flight.  Calls return at once;
+    synchronize() waits for every submitted step.  The host tensors must stay
+    untouched until then.
+    """
+
+    def __init__(self, fwd: Forward, device="cuda"):
+        torch = _torch()
+        self.fwd = fwd
+        self.h2d, self.comp, self.d2h = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+        self.slots_out = [torch.empty_like(fwd.o) for _ in range(2)]
+        self.slots_in = [None, None]
+        ev = lambda: [torch.cuda.Event(), torch.cuda.Event()]
+        self.ev_in, self.ev_used, self.ev_out, self.ev_back = ev(), ev(), ev(), ev()
+        self.n = 0
+
+    def _inputs(self, s, named):
+        torch = _torch()
+        if self.slots_in[s] is None:
+            self.slots_in[s] = {k: torch.empty(t.shape, dtype=t.dtype, device="cuda") for k, t in named.items()}
+        return self.slots_in[s]
+
+    def submit(self, q, k, v, o, block_map=None, gate=None):
+        torch = _torch()
+        s = self.n & 1
+        named = {"q": q, "k": k, "v": v}
+        if block_map is not None:
+            named["map"] = block_map
+        if gate is not None:
+            named["gate"] = gate
+        dev = self._inputs(s, named)
+        with torch.cuda.stream(self.h2d):
+            if self.n >= 2:
+                self.h2d.wait_event(self.ev_used[s])  # step n-2 no longer reads this slot
+            for name, src in named.items():
+                dev[name].copy_(src, non_blocking=True)
+            self.ev_in[s].record(self.h2d)
+        with torch.cuda.stream(self.comp):
+            self.comp.wait_event(self.ev_in[s])
+            if self.n >= 2:
+                self.comp.wait_event(self.ev_back[s])  # step n-2's output has left this slot
+            self.fwd(dev["q"], dev["k"], dev["v"], dev.get("map"), dev.get("gate"), out=self.slots_out[s])
+            self.ev_used[s].record(self.comp)
+            self.ev_out[s].record(self.comp)
+        with torch.cuda.stream(self.d2h):
+            self.d2h.wait_event(self.ev_out[s])
+            o.copy_(self.slots_out[s], non_blocking=True)
+            self.ev_back[s].record(self.d2h)
+        self.n += 1
+
+    def synchronize(self):
+        for st in (self.h2d, self.comp, self.d2h):
+            st.synchronize()
