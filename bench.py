@@ -278,8 +278,6 @@ def run_backward(args, wl, world, rank, local, pg):
     inputs resident in HBM; the selection, o and lse come from a forward call."""
     import torch
     import block_sparse_video_gather_b200 as vsa
-    if wl.block_tokens != 256 or wl.map_driven:
-        raise SystemExit("the backward bench takes a top-k workload with 256-token blocks")
     inp = workloads.make_inputs(wl, dtype=args.dtype)
     tdt = torch.float16 if args.dtype == "f16" else torch.bfloat16
     plan = vsa.Plan.of(wl)
@@ -288,7 +286,8 @@ def run_backward(args, wl, world, rank, local, pg):
     do_untiled = to16(rng.standard_normal(inp["q"].shape).astype(np.float32))  # gradient of the untiled o
     dev16 = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).cuda().view(tdt)
     fwd = vsa.Forward(plan, wl.B, wl.H, wl.topk, dtype=tdt)
-    fwd(dev16(inp["q"]), dev16(inp["k"]), dev16(inp["v"]))
+    bmap = torch.from_numpy(inp["map"]).cuda() if wl.map_driven else None
+    fwd(dev16(inp["q"]), dev16(inp["k"]), dev16(inp["v"]), bmap)
     do = vsa.tile(plan, dev16(do_untiled))  # tiled; padded rows zero
     ws = torch.empty(vsa.bwd_workspace_bytes(plan, wl.B, wl.H, fwd.idx.shape[-1]), dtype=torch.uint8, device="cuda")
     dq, dk, dv = (torch.empty_like(fwd.qt) for _ in range(3))

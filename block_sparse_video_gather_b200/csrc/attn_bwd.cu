@@ -27,6 +27,9 @@
 //             the K and V tiles of the selected blocks stream.  TMEM: S [0,128),
 //             dP [128,256), dQ [256,384), dS (16-bit) [384,448).  Per key tile:
 //             S = Q K^T, dP = dO V^T, then dQ += dS K.
+// 64-token blocks use the forward's tile-64 arrangement: the resident block
+// sits in the top half of a 128-row tile, the streamed 128-wide tiles pair two
+// listed blocks (64-row boxes).
 // Operands use the two forms of the forward kernel: K-major x K-major for the
 // products over the head dimension, TMEM (A) x MN-major shared memory (B) for
 // the products over keys or queries.  A tile in shared memory is the TMA image
@@ -229,24 +232,31 @@ constexpr uint32_t kKV_L = kKV_Stage + 2 * kKV_StageBytes;  // lse2, delta: 2 st
 constexpr uint32_t kKV_Bar = kKV_L + 2 * 1024;
 constexpr uint32_t kKV_Smem = kKV_Bar + 256 + 1024;
 
-template <bool F16>
+// 64-token blocks (BS = 64): an item is one key block in the top half of the
+// 128-row tile (the 128-row box also brings the next block's rows, finite and
+// masked), and each streamed 128-column query tile holds two listed query
+// blocks, loaded as 64-row boxes (tm_qs, tm_dos).  For BS = 256 the streamed
+// maps are the 128-row ones.
+template <int BS, bool F16>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+    attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_dos,
                          const __grid_constant__ BwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   BwdBarriers* bars = reinterpret_cast<BwdBarriers*>(smem + kKV_Bar);
   const Geo& g = p.g;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int kHalves = BS == 256 ? 2 : 1;
   const int item = blockIdx.x;
-  const int half = item & 1;
-  const int kb = (item >> 1) % g.NB;
-  const int bh = (item >> 1) / g.NB;
+  const int half = BS == 256 ? (item & 1) : 0;
+  const int kb = (item / kHalves) % g.NB;
+  const int bh = (item / kHalves) / g.NB;
   const int32_t* offs = p.k2q_off + static_cast<long long>(bh) * (g.NB + 1);
   const int lo = __ldg(offs + kb), hi = __ldg(offs + kb + 1);
   const int32_t* list = p.k2q + static_cast<long long>(bh) * g.NB * p.max_k + lo;
-  const int nq = 2 * (hi - lo);  // query tiles
+  const int len = hi - lo;
+  const int nq = BS == 256 ? 2 * len : (len + 1) / 2;  // query tiles
   const long long base = static_cast<long long>(bh) * g.Sp;
 
   if (threadIdx.x == 0) init_barriers(bars);
@@ -267,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int issued = 0;
     bool kv = false;
     if (nq > 0) {
-      const int krow = static_cast<int>(base + static_cast<long long>(kb) * 256 + half * 128);
+      const int krow = static_cast<int>(base + static_cast<long long>(kb) * BS + half * 128);
       mbar_arrive_expect_tx_w(&bars->a_full, 2 * kTileBytes);
       for (int hf = 0; hf < 2; ++hf) {
         tma_load_2d_w(smem + kKV_K + hf * kHalfBytes, &tm_k, hf * 64, krow, &bars->a_full, pol_last);
@@ -277,24 +287,48 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int u = 0; u < nq; ++u) {
         const int s = u & 1;
         if (!wwait(&bars->empty[s], ((u >> 1) & 1) ^ 1, bars, p.status)) break;
-        const int qb = __ldg(list + (u >> 1));
-        const long long qrow = base + static_cast<long long>(qb) * 256 + (u & 1) * 128;
-        uint8_t* st = smem + kKV_Stage + s * kKV_StageBytes;
-        {  // query-tile validity for the elementwise warps, published by the arrive below
-          uint32_t w[4];
+        // rows of the tile's query blocks: one 128-row box, or two 64-row boxes
+        // (an absent second block loads block 0, finite and masked)
+        long long qrow0, qrow1 = 0;
+        uint32_t w[4];
+        if (BS == 256) {
+          const int qb = __ldg(list + (u >> 1));
+          qrow0 = base + static_cast<long long>(qb) * 256 + (u & 1) * 128;
           tile_bits(g, qb, u & 1, w);
-          if (lane < 4) bars->mask[s][lane] = pick4(w, lane);
-          __syncwarp();
+        } else {
+          const int qa = __ldg(list + 2 * u);
+          const int qc = 2 * u + 1 < len ? __ldg(list + 2 * u + 1) : -1;
+          qrow0 = base + static_cast<long long>(qa) * 64;
+          qrow1 = base + static_cast<long long>(qc < 0 ? 0 : qc) * 64;
+          block64_mask(g, qa, w[0], w[1]);
+          block64_mask(g, qc, w[2], w[3]);
         }
+        uint8_t* st = smem + kKV_Stage + s * kKV_StageBytes;
+        if (lane < 4) bars->mask[s][lane] = pick4(w, lane);  // published by the arrive below
+        __syncwarp();
         mbar_arrive_expect_tx_w(&bars->full[s], 2 * kTileBytes + 1024);
         for (int hf = 0; hf < 2; ++hf) {
-          tma_load_2d_w(st + hf * kHalfBytes, &tm_q, hf * 64, static_cast<int>(qrow), &bars->full[s], pol_last);
-          tma_load_2d_w(st + kTileBytes + hf * kHalfBytes, &tm_do, hf * 64, static_cast<int>(qrow), &bars->full[s],
+          tma_load_2d_w(st + hf * kHalfBytes, &tm_qs, hf * 64, static_cast<int>(qrow0), &bars->full[s], pol_last);
+          tma_load_2d_w(st + kTileBytes + hf * kHalfBytes, &tm_dos, hf * 64, static_cast<int>(qrow0), &bars->full[s],
                         pol_last);
+          if (BS == 64) {
+            tma_load_2d_w(st + hf * kHalfBytes + kHalfBytes / 2, &tm_qs, hf * 64, static_cast<int>(qrow1),
+                          &bars->full[s], pol_last);
+            tma_load_2d_w(st + kTileBytes + hf * kHalfBytes + kHalfBytes / 2, &tm_dos, hf * 64,
+                          static_cast<int>(qrow1), &bars->full[s], pol_last);
+          }
         }
         if (lane == 0) {
-          bulk_load(smem + kKV_L + s * 1024, p.nlse2 + qrow, 512, &bars->full[s]);
-          bulk_load(smem + kKV_L + s * 1024 + 512, p.ndelta + qrow, 512, &bars->full[s]);
+          uint8_t* L = smem + kKV_L + s * 1024;
+          if (BS == 256) {
+            bulk_load(L, p.nlse2 + qrow0, 512, &bars->full[s]);
+            bulk_load(L + 512, p.ndelta + qrow0, 512, &bars->full[s]);
+          } else {
+            bulk_load(L, p.nlse2 + qrow0, 256, &bars->full[s]);
+            bulk_load(L + 256, p.nlse2 + qrow1, 256, &bars->full[s]);
+            bulk_load(L + 512, p.ndelta + qrow0, 256, &bars->full[s]);
+            bulk_load(L + 768, p.ndelta + qrow1, 256, &bars->full[s]);
+          }
         }
         __syncwarp();
         ++issued;
@@ -356,7 +390,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tS = tmem + lane_off, tP = tS + 128;
     uint32_t kw[4];
-    tile_bits(g, kb, half, kw);
+    if (BS == 256) {
+      tile_bits(g, kb, half, kw);
+    } else {
+      block64_mask(g, kb, kw[0], kw[1]);
+      kw[2] = kw[3] = 0u;  // rows 64..127 belong to the next block
+    }
     const bool kvalid = (pick4(kw, r >> 5) >> (r & 31)) & 1u;
     const uint64_t c2 = f2pack(p.scale_log2, p.scale_log2);
     bool ok = true;
@@ -393,12 +432,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok && nq > 0) ok = wwait(&bars->done, 0, bars, p.status);
     tc_fence_after();
-    const long long row = base + static_cast<long long>(kb) * 256 + half * 128 + r;
+    const long long row = base + static_cast<long long>(kb) * BS + half * 128 + r;
     const bool load = ok && nq > 0;  // warp-uniform
-    if (wg == 0)
-      store_row<F16>(tS + 256, 1.0f, p.dv + row * 128, load, false);
-    else
-      store_row<F16>(tS + 384, p.scale, p.dk + row * 128, load, false);
+    if (BS == 256 || quarter < 2) {  // for 64-token blocks, lanes 64..127 are the next block's rows
+      if (wg == 0)
+        store_row<F16>(tS + 256, 1.0f, p.dv + row * 128, load, false);
+      else
+        store_row<F16>(tS + 384, p.scale, p.dk + row * 128, load, false);
+    }
   }
 
   tc_fence_before();
@@ -425,27 +466,31 @@ __device__ __forceinline__ int dq_block(const BwdParams& p, long long row_item, 
   return (kb >= 0 && kb < p.g.NB) ? kb : -1;
 }
 
-template <bool F16>
+// 64-token blocks (BS = 64): an item is one query block in the top half of
+// the 128-row tile, and each streamed 128-key tile holds two selected blocks,
+// loaded as 64-row boxes (tm_ks, tm_vs).
+template <int BS, bool F16>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ks,
+                       const __grid_constant__ CUtensorMap tm_vs, const __grid_constant__ CUtensorMap tm_do,
                        const __grid_constant__ BwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   BwdBarriers* bars = reinterpret_cast<BwdBarriers*>(smem + kQ_Bar);
   const Geo& g = p.g;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int kHalves = BS == 256 ? 2 : 1;
   const int item = blockIdx.x;
-  const int half = item & 1;
-  const int qb = (item >> 1) % g.NB;
-  const int bh = (item >> 1) / g.NB;
+  const int half = BS == 256 ? (item & 1) : 0;
+  const int qb = (item / kHalves) % g.NB;
+  const int bh = (item / kHalves) / g.NB;
   const long long row_item = static_cast<long long>(bh) * g.NB + qb;
   int nb = __ldg(p.num + row_item);
   if (nb < 0 || nb > p.max_k) {
     if (threadIdx.x == 0 && half == 0) atomicCAS(p.status, 0u, (unsigned)VSA_ERR_BAD_INDEX);
     nb = nb < 0 ? 0 : p.max_k;
   }
-  const int n = 2 * nb;  // key tiles
+  const int n = BS == 256 ? 2 * nb : (nb + 1) / 2;  // key tiles
   const long long base = static_cast<long long>(bh) * g.Sp;
 
   if (threadIdx.x == 0) init_barriers(bars);
@@ -466,7 +511,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int issued = 0, issued_k = 0;  // V and K copies issued
     bool qd = false;
     if (n > 0) {
-      const int qrow = static_cast<int>(base + static_cast<long long>(qb) * 256 + half * 128);
+      const int qrow = static_cast<int>(base + static_cast<long long>(qb) * BS + half * 128);
       mbar_arrive_expect_tx_w(&bars->a_full, 2 * kTileBytes);
       for (int hf = 0; hf < 2; ++hf) {
         tma_load_2d_w(smem + kQ_Q + hf * kHalfBytes, &tm_q, hf * 64, qrow, &bars->a_full, pol_first);
@@ -474,30 +519,46 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       qd = true;
       for (int t = 0; t < n; ++t) {
-        const int kb0 = dq_block(p, row_item, t >> 1);
-        const int kb = kb0 < 0 ? 0 : kb0;  // unusable ids load block 0; the elementwise step masks it out
-        const int krow = static_cast<int>(base + static_cast<long long>(kb) * 256 + (t & 1) * 128);
+        // rows of the tile's key blocks: one 128-row box, or two 64-row boxes;
+        // unusable or absent ids load block 0, which the elementwise step masks out
+        int krow0, krow1 = 0;
+        uint32_t w[4];
+        bool bad;
+        if (BS == 256) {
+          const int kb0 = dq_block(p, row_item, t >> 1);
+          krow0 = static_cast<int>(base + static_cast<long long>(kb0 < 0 ? 0 : kb0) * 256 + (t & 1) * 128);
+          tile_bits(g, kb0, t & 1, w);
+          bad = kb0 < 0 && half == 0 && (t & 1) == 0;
+        } else {
+          const int ka = dq_block(p, row_item, 2 * t);
+          const int kc = 2 * t + 1 < nb ? dq_block(p, row_item, 2 * t + 1) : -1;
+          krow0 = static_cast<int>(base + static_cast<long long>(ka < 0 ? 0 : ka) * 64);
+          krow1 = static_cast<int>(base + static_cast<long long>(kc < 0 ? 0 : kc) * 64);
+          block64_mask(g, ka, w[0], w[1]);
+          block64_mask(g, kc, w[2], w[3]);
+          bad = ka < 0 || (2 * t + 1 < nb && kc < 0);
+        }
         const int ks = t % 3, vs = t & 1;
         if (!wwait(&bars->kempty[ks], ((t / 3) & 1) ^ 1, bars, p.status)) break;
-        {  // key-tile validity for the elementwise warps, published by the arrive below
-          uint32_t w[4];
-          tile_bits(g, kb0, t & 1, w);
-          if (lane < 4) bars->mask[ks][lane] = pick4(w, lane);
-          if (kb0 < 0 && lane == 0 && half == 0 && (t & 1) == 0) atomicCAS(p.status, 0u, (unsigned)VSA_ERR_BAD_INDEX);
-          __syncwarp();
-        }
+        if (lane < 4) bars->mask[ks][lane] = pick4(w, lane);  // published by the arrive below
+        if (bad && lane == 0) atomicCAS(p.status, 0u, (unsigned)VSA_ERR_BAD_INDEX);
+        __syncwarp();
         mbar_arrive_expect_tx_w(&bars->kfull[ks], kTileBytes);
-        for (int hf = 0; hf < 2; ++hf)
-          tma_load_2d_w(smem + kQ_K + ks * kTileBytes + hf * kHalfBytes, &tm_k, hf * 64, krow, &bars->kfull[ks],
-                        pol_last);
+        for (int hf = 0; hf < 2; ++hf) {
+          uint8_t* dst = smem + kQ_K + ks * kTileBytes + hf * kHalfBytes;
+          tma_load_2d_w(dst, &tm_ks, hf * 64, krow0, &bars->kfull[ks], pol_last);
+          if (BS == 64) tma_load_2d_w(dst + kHalfBytes / 2, &tm_ks, hf * 64, krow1, &bars->kfull[ks], pol_last);
+        }
         if (!wwait(&bars->empty[vs], ((t >> 1) & 1) ^ 1, bars, p.status)) {
           ++issued_k;
           break;
         }
         mbar_arrive_expect_tx_w(&bars->full[vs], kTileBytes);
-        for (int hf = 0; hf < 2; ++hf)
-          tma_load_2d_w(smem + kQ_V + vs * kTileBytes + hf * kHalfBytes, &tm_v, hf * 64, krow, &bars->full[vs],
-                        pol_last);
+        for (int hf = 0; hf < 2; ++hf) {
+          uint8_t* dst = smem + kQ_V + vs * kTileBytes + hf * kHalfBytes;
+          tma_load_2d_w(dst, &tm_vs, hf * 64, krow0, &bars->full[vs], pol_last);
+          if (BS == 64) tma_load_2d_w(dst + kHalfBytes / 2, &tm_vs, hf * 64, krow1, &bars->full[vs], pol_last);
+        }
         ++issued_k;
         ++issued;
       }
@@ -577,9 +638,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tS = tmem + lane_off, tP = tS + 128, tDS = tS + 384;
     uint32_t rw[4];
-    tile_bits(g, qb, half, rw);
+    if (BS == 256) {
+      tile_bits(g, qb, half, rw);
+    } else {
+      block64_mask(g, qb, rw[0], rw[1]);
+      rw[2] = rw[3] = 0u;  // rows 64..127 belong to the next block
+    }
     const bool rvalid = (pick4(rw, r >> 5) >> (r & 31)) & 1u;
-    const long long row = base + static_cast<long long>(qb) * 256 + half * 128 + r;
+    const long long row = base + static_cast<long long>(qb) * BS + half * 128 + r;
     const float nl = rvalid ? __ldg(p.nlse2 + row) : 0.0f;
     const float nd = rvalid ? __ldg(p.ndelta + row) : 0.0f;
     uint64_t nl2[16], nd2[16];
@@ -620,7 +686,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok && n > 0) ok = wwait(&bars->done, 0, bars, p.status);
     tc_fence_after();
-    store_half_row<F16>(tS + 256 + 64 * wg, p.scale, p.dq + row * 128 + 64 * wg, ok && n > 0, !rvalid);
+    if (BS == 256 || quarter < 2)  // for 64-token blocks, lanes 64..127 are the next block's rows
+      store_half_row<F16>(tS + 256 + 64 * wg, p.scale, p.dq + row * 128 + 64 * wg, ok && n > 0, !rvalid);
   }
 
   tc_fence_before();
@@ -740,8 +807,38 @@ size_t attn_bwd_workspace_bytes(const Geo& g, int BH, int max_k) {
   return b;
 }
 
+template <int BS, bool F16>
+cudaError_t launch_bwd_kernels(const Geo& g, const AttnBwdArgs& a, const BwdParams& p, cudaStream_t stream) {
+  const unsigned long long rows = static_cast<unsigned long long>(a.BH) * g.Sp;
+  CUtensorMap tq, tk, tv, tdo, tqs, tks, tvs, tdos;
+  if (!make_tmap(&tq, a.q, rows, 128, F16) || !make_tmap(&tk, a.k, rows, 128, F16) ||
+      !make_tmap(&tv, a.v, rows, 128, F16) || !make_tmap(&tdo, a.dO, rows, 128, F16))
+    return cudaErrorInvalidValue;
+  if (BS == 256) {
+    tqs = tq;
+    tks = tk;
+    tvs = tv;
+    tdos = tdo;
+  } else if (!make_tmap(&tqs, a.q, rows, 64, F16) || !make_tmap(&tks, a.k, rows, 64, F16) ||
+             !make_tmap(&tvs, a.v, rows, 64, F16) || !make_tmap(&tdos, a.dO, rows, 64, F16)) {
+    return cudaErrorInvalidValue;
+  }
+  const unsigned items = static_cast<unsigned>((BS == 256 ? 2ull : 1ull) * a.BH * g.NB);
+  cudaError_t e;
+  if ((e = cudaFuncSetAttribute(attn_bwd_dkdv_kernel<BS, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                kKV_Smem)) != cudaSuccess)
+    return e;
+  if ((e = cudaFuncSetAttribute(attn_bwd_dq_kernel<BS, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                kQ_Smem)) != cudaSuccess)
+    return e;
+  attn_bwd_dkdv_kernel<BS, F16><<<items, kThreads, kKV_Smem, stream>>>(tqs, tk, tv, tdos, p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  attn_bwd_dq_kernel<BS, F16><<<items, kThreads, kQ_Smem, stream>>>(tq, tks, tvs, tdo, p);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_attn_bwd(const Geo& g, const AttnBwdArgs& a, cudaStream_t stream) {
-  if (g.bs != 256) return cudaErrorNotSupported;
+  if (g.bs != 256 && g.bs != 64) return cudaErrorNotSupported;
   const unsigned long long rows = static_cast<unsigned long long>(a.BH) * g.Sp;
   if (rows >= (1ull << 31)) return cudaErrorInvalidValue;
   uint8_t* ws = static_cast<uint8_t*>(a.workspace);
@@ -751,11 +848,6 @@ cudaError_t launch_attn_bwd(const Geo& g, const AttnBwdArgs& a, cudaStream_t str
   size_t off_bytes = 2 * rows * sizeof(float) + static_cast<size_t>(a.BH) * (g.NB + 1) * sizeof(int32_t);
   off_bytes = (off_bytes + 15) & ~size_t(15);
   int32_t* k2q = reinterpret_cast<int32_t*>(ws + off_bytes);
-
-  CUtensorMap tq, tk, tv, tdo;
-  if (!make_tmap(&tq, a.q, rows, 128, a.f16) || !make_tmap(&tk, a.k, rows, 128, a.f16) ||
-      !make_tmap(&tv, a.v, rows, 128, a.f16) || !make_tmap(&tdo, a.dO, rows, 128, a.f16))
-    return cudaErrorInvalidValue;
 
   const unsigned prep_blocks = static_cast<unsigned>((rows + 15) / 16);
   if (a.f16)
@@ -787,15 +879,9 @@ cudaError_t launch_attn_bwd(const Geo& g, const AttnBwdArgs& a, cudaStream_t str
   p.status = a.status;
   p.scale = static_cast<float>(1.0 / 11.313708498984761);            // 128^-1/2
   p.scale_log2 = static_cast<float>(1.4426950408889634 / 11.313708498984761);
-  const unsigned items = static_cast<unsigned>(2ull * a.BH * g.NB);
-  auto kv = a.f16 ? attn_bwd_dkdv_kernel<true> : attn_bwd_dkdv_kernel<false>;
-  auto dq = a.f16 ? attn_bwd_dq_kernel<true> : attn_bwd_dq_kernel<false>;
-  if ((e = cudaFuncSetAttribute(kv, cudaFuncAttributeMaxDynamicSharedMemorySize, kKV_Smem)) != cudaSuccess) return e;
-  if ((e = cudaFuncSetAttribute(dq, cudaFuncAttributeMaxDynamicSharedMemorySize, kQ_Smem)) != cudaSuccess) return e;
-  kv<<<items, kThreads, kKV_Smem, stream>>>(tq, tk, tv, tdo, p);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  dq<<<items, kThreads, kQ_Smem, stream>>>(tq, tk, tv, tdo, p);
-  return cudaGetLastError();
+  if (g.bs == 256)
+    return a.f16 ? launch_bwd_kernels<256, true>(g, a, p, stream) : launch_bwd_kernels<256, false>(g, a, p, stream);
+  return a.f16 ? launch_bwd_kernels<64, true>(g, a, p, stream) : launch_bwd_kernels<64, false>(g, a, p, stream);
 }
 
 }  // namespace vsa

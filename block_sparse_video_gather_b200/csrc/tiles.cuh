@@ -54,6 +54,57 @@ __device__ __forceinline__ int key_tile_mask(const Geo& g, int kb, int half, uin
   return any ? kTilePartial : kTileEmpty;
 }
 
+// Validity bits of the 64 slots of block kb (two words), for 64-token
+// blocks.  Returns kTileFull / kTilePartial / kTileEmpty.
+__device__ __forceinline__ int block64_mask(const Geo& g, int kb, uint32_t& w0, uint32_t& w1) {
+  uint32_t w[4];
+  // slots 0..63 of the block are columns 0..63 of "tile 0" of a 128-column view
+  w[0] = w[1] = w[2] = w[3] = 0xffffffffu;
+  if (kb < 0) {
+    w0 = w1 = 0u;
+    return kTileEmpty;
+  }
+  if (kb < g.n_pre) {
+    const int lim = g.n_prefix - kb * g.bs;
+    if (lim <= 0) {
+      w0 = w1 = 0u;
+      return kTileEmpty;
+    }
+    if (lim >= 64) {
+      w0 = w1 = 0xffffffffu;
+      return kTileFull;
+    }
+    w0 = lim >= 32 ? 0xffffffffu : ((1u << lim) - 1u);
+    w1 = lim <= 32 ? 0u : ((1u << (lim - 32)) - 1u);
+    return kTilePartial;
+  }
+  int vt, vh, vw;
+  video_block_extent(g, kb - g.n_pre, vt, vh, vw);
+  if (vt == g.bt && vh == g.bh && vw == g.bw) {
+    w0 = w1 = 0xffffffffu;
+    return kTileFull;
+  }
+  const uint32_t rowbits = vw >= 32 ? 0xffffffffu : ((1u << vw) - 1u);
+  const int rows_per_word = 32 >> g.lbw;
+  uint32_t any = 0;
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    uint32_t word = 0;
+    const int row0 = (32 * i) >> g.lbw;
+    for (int r = 0; r < rows_per_word; ++r) {
+      const int R = row0 + r;
+      const int lh = R & (g.bh - 1);
+      const int lt = R >> g.lbh;
+      if (lt < vt && lh < vh) word |= rowbits << (r << g.lbw);
+    }
+    w[i] = word;
+    any |= word;
+  }
+  w0 = w[0];
+  w1 = w[1];
+  return any ? kTilePartial : kTileEmpty;
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);

@@ -405,7 +405,6 @@ int vsa_sparse_attn_bwd(vsa_plan_t plan, vsa_dtype_t dtype, const uint16_t* q, c
   if (!aligned16(q2k_idx) || !aligned16(q2k_num) || max_k < 1) return VSA_ERR_INVALID_ARG;
   if (int rc = check_dims(B, H, D)) return rc;
   const vsa::Geo& g = plan->g;
-  if (g.bs != 256) return VSA_ERR_UNSUPPORTED;
   DeviceState* ds = nullptr;
   if (int rc = device_state(&ds)) return rc;
   vsa::AttnBwdArgs a;

@@ -261,7 +261,8 @@ VSA_API int vsa_sparse_attn_fwd_ex(vsa_plan_t plan, vsa_dtype_t dtype, const uin
  *   workspace      : device memory of vsa_sparse_attn_bwd_workspace bytes,
  *                    caller-owned, contents need not be initialised
  * 16-bit operands (P, dS rounded to dtype for the tensor cores), fp32
- * accumulation.  256-token blocks only (VSA_ERR_UNSUPPORTED otherwise).
+ * accumulation.  Both block sizes (256 tokens, and the 64-token tiles of the
+ * FastVideo commit log's layout).
  * Block ids outside [0, NB) and counts outside [0, max_k] are skipped /
  * clamped and set VSA_ERR_BAD_INDEX in the device status word.
  */

@@ -93,6 +93,9 @@ CASES = [
     ("batch2-f16", dict(T=6, Hg=12, Wg=20, B=2, H=2), 4, "f16", False),
     ("prefix", dict(T=4, Hg=16, Wg=16, n_prefix=300, H=3), 5, "bf16", True),
     ("all-blocks", dict(T=8, Hg=8, Wg=16, H=2), 0, "bf16", False),
+    # 64-token tiles (the commit log's layout): prefix tiles, partial tiles
+    ("tile64-prefix", dict(T=6, Hg=8, Wg=12, block=(4, 4, 4), n_prefix=100, H=3), 7, "bf16", True),
+    ("tile64-ragged-f16", dict(T=5, Hg=9, Wg=11, block=(4, 4, 4), H=2), 5, "f16", False),
 ]
 
 
@@ -119,6 +122,52 @@ def test_bwd_matches_oracle_everywhere(case):
     pad = ~real
     for t in (dq, dk, dv):
         assert (t[:, :, pad] == 0).all()
+
+
+def _gpu_bwd_map(wl, qt, kt, vt, do, bmap):
+    """Forward through the block map on the GPU, then the backward; returns the selection too."""
+    plan = vsa.Plan.of(wl)
+    q, k, v, d = (_dev(x, "bf16") for x in (qt, kt, vt, do))
+    ti, tn = vsa.map_to_index(torch.from_numpy(bmap).cuda())
+    o, lse = vsa.sparse_attn_fwd(plan, q, k, v, ti, tn)
+    dq, dk, dv = vsa.sparse_attn_bwd(plan, q, k, v, o, lse, d, ti, tn)
+    torch.cuda.synchronize()
+    assert vsa.get_status() == vsa.VSA_OK
+    return _host(dq), _host(dk), _host(dv), ti.cpu().numpy(), tn.cpu().numpy()
+
+
+def test_bwd_full_size_tile64():
+    """The tile-64 workload (block map with dense prefix rows and empty rows): dq on
+    sampled rows (incl. prefix and empty rows) against the oracle; dk, dv through the
+    sum identities over the rows with a non-empty selection."""
+    wl = workloads.WORKLOADS["tile64"]
+    g = oracle.geometry_of(wl)
+    inp = workloads.make_inputs(wl)
+    qt, kt, vt = (oracle.tile(g, inp[n]) for n in ("q", "k", "v"))
+    rng = np.random.default_rng(13)
+    do = oracle.tile(g, workloads.f32_to_bf16_bits(rng.standard_normal(inp["q"].shape).astype(np.float32)))
+    dq, dk, dv, idx, num = _gpu_bwd_map(wl, qt, kt, vt, do, inp["map"])
+    ridx, rnum = oracle.map_to_index(inp["map"])
+    np.testing.assert_array_equal(idx, ridx)
+    real = np.flatnonzero(H.real_rows(wl))
+    rows = []
+    for bh in range(wl.B * wl.H):
+        pick = rng.choice(real, 24, replace=False)
+        zero = np.flatnonzero(num.reshape(-1, g.NB)[bh] == 0)[:2]
+        extra = [z * g.bs + np.arange(0, g.bs, 21) for z in zero] + [np.arange(0, g.n_pre * g.bs, 97)]
+        rows.append(bh * g.Sp + np.unique(np.concatenate([pick] + extra)))
+    rows = np.concatenate(rows)
+    ref = oracle.attn_bwd_q_rows(g, qt, kt, vt, do, idx, num, rows)
+    _check("tile64 dq rows", _vals(dq, "bf16").reshape(-1, 128)[rows], ref)
+    realm = H.real_rows(wl)
+    dkv = _vals(dk, "bf16")[0][:, realm]
+    dvv = _vals(dv, "bf16")[0][:, realm]
+    dov = _vals(do, "bf16")[0]
+    for h in range(wl.H):
+        rows_h = realm & (np.repeat(num[0, h], g.bs) > 0)
+        assert np.abs(dkv[h].sum(axis=0)).max() <= 2e-2 * np.abs(dkv[h]).sum(axis=0).max(), h
+        np.testing.assert_allclose(dvv[h].sum(axis=0), dov[h][rows_h].sum(axis=0), rtol=0,
+                                   atol=2e-2 * np.abs(dov[h][rows_h]).sum(axis=0).max())
 
 
 def test_bwd_full_size_fastwan():
