@@ -73,12 +73,6 @@ struct Idesc {
   static constexpr uint32_t PV = F16 ? idesc_f16_f32(128, 128, 0, 1) : idesc_bf16_f32(128, 128, 0, 1);
 };
 
-// Exponential pairs, out of every 8, evaluated by polynomial on the FMA pipe.
-#ifndef VSA_POLY_PAIRS
-#define VSA_POLY_PAIRS 0
-#endif
-constexpr int kPolyPairsOf8 = VSA_POLY_PAIRS;
-
 struct Barriers {
   uint64_t q_full, q_empty;
   uint64_t k_full[kStages], k_empty[kStages];
@@ -471,18 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < 64; ++j) {
             const uint64_t x = fma2(u2pack(sv[2 * j], sv[2 * j + 1]), c2, nm2);
             uint64_t pp;
-#ifdef VSA_EXP_BF16X2
             {
-              float xa, xb;
-              f2unpack(x, xa, xb);
-              const uint32_t e = ex2_bf16x2(pack_bf16x2(xa, xb));
-              pk[j] = e;
-              pp = u2pack(e << 16, e & 0xffff0000u);
-            }
-#else
-            if ((j & 7) < kPolyPairsOf8) {
-              pp = exp2_poly2(x);
-            } else {
               float xa, xb;
               f2unpack(x, xa, xb);
               pp = f2pack(ex2_approx(xa), ex2_approx(xb));
@@ -492,7 +475,6 @@ __global__ void __launch_bounds__(kThreads, 1)
               f2unpack(pp, p0, p1);
               pk[j] = pack_half2<F16>(p0, p1);
             }
-#endif
             switch (j & 3) {
               case 0: acc0 = add2(acc0, pp); break;
               case 1: acc1 = add2(acc1, pp); break;

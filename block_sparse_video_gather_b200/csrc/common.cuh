@@ -368,38 +368,6 @@ __device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
   return d;
 }
 
-// 2^x for a pair, on the FMA/ALU pipes instead of the MUFU unit.
-// Split x = j + f with j = rint(x) (the 1.5*2^23 rounding constant), f in
-// [-1/2, 1/2]; 2^f by a degree-3 polynomial (least-relative-error fit,
-// |rel err| < 7.5e-5, far below the bf16 rounding of the numerators); then
-// j is added to the exponent field.  x is clamped to >= -125 so the result
-// stays a normal number (2^-125 for masked columns: negligible next to the
-// row maximum, which is >= 2^-8 whenever the row has a real key).
-__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
-  float a, b;
-  f2unpack(x2, a, b);
-  a = fmaxf(a, -125.0f);
-  b = fmaxf(b, -125.0f);
-  const uint64_t x = f2pack(a, b);
-  const uint64_t r = add2(x, f2pack(12582912.0f, 12582912.0f));
-  const uint64_t jj = add2(r, f2pack(-12582912.0f, -12582912.0f));
-  const uint64_t f = fma2(jj, f2pack(-1.0f, -1.0f), x);
-  uint64_t p = fma2(f2pack(0.05517167f, 0.05517167f), f, f2pack(0.24261113f, 0.24261113f));
-  p = fma2(p, f, f2pack(0.69326097f, 0.69326097f));
-  p = fma2(p, f, f2pack(0.99992806f, 0.99992806f));
-  uint32_t p0, p1, r0, r1;
-  u2unpack(p, p0, p1);
-  u2unpack(r, r0, r1);
-  return u2pack(p0 + (r0 << 23), p1 + (r1 << 23));
-}
-
-// 2^x on a packed bf16 pair (one MUFU operation for both).
-__device__ __forceinline__ uint32_t ex2_bf16x2(uint32_t x) {
-  uint32_t y;
-  asm("ex2.approx.ftz.bf16x2 %0, %1;" : "=r"(y) : "r"(x));
-  return y;
-}
-
 // Two fp32 -> packed bf16x2 (round to nearest even); `lo` lands in bits [0,16).
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
