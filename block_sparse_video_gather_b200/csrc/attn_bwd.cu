@@ -17,12 +17,13 @@
 //             that list it (a repeated id is listed again), ascending; rows are
 //             placed in order, so the lists do not depend on thread timing.
 //   bwd_dkdv  one CTA per (b*h, key block, 128-key half).  K and V stay in
-//             shared memory; the query tiles of every listed query block
-//             stream through a 2-stage ring (Q, dO, lse2, delta).
-//             TMEM: S^T [0,128) with P^T (16-bit) written back on [0,64);
-//             dP^T [128,256) with dS^T on [128,192); dV [256,384); dK [384,512).
-//             Per query tile: S^T = K Q^T, dP^T = V dO^T, then
-//             dV += P^T dO and dK += dS^T Q (P^T, dS^T read from TMEM).
+//             shared memory; the 64-row query tiles of every listed query
+//             block stream through a 4-stage ring (Q, dO, -lse log2 e, -delta).
+//             TMEM: two buffers of S^T (64 columns, P^T written back on the
+//             first 32) and dP^T (dS^T on the first 32), dV [256,384),
+//             dK [384,512).  Per query tile: S^T = K Q^T, dP^T = V dO^T (N = 64),
+//             then dV += P^T dO and dK += dS^T Q; the next tiles' S^T, dP^T
+//             run while the elementwise warps work on the current one.
 //   bwd_dq    one CTA per (b*h, query block, 128-row half).  Q and dO stay;
 //             the K and V tiles of the selected blocks stream.  TMEM: S [0,128),
 //             dP [128,256), dQ [256,384), dS (16-bit) [384,448).  Per key tile:
@@ -128,13 +129,16 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint3
 
 struct BwdBarriers {
   uint64_t a_full;            // resident tiles (K,V for dkdv; Q,dO for dq)
-  uint64_t full[2], empty[2];  // streamed stages (dq: the V ring)
+  uint64_t full[4], empty[4];  // streamed stages (dkdv: Q/dO ring; dq: the V ring)
   uint64_t kfull[3], kempty[3];  // dq: the K ring
   uint32_t mask[3][4];            // validity bits of the streamed tile of each stage (written by the producer)
   uint64_t s_full, s_free, ds_full, ds_free, done, drain;
+  uint64_t sbuf[2];               // dkdv: S^T / dP^T buffer b holds a finished tile
   uint32_t tmem_base;
   int abort;
 };
+
+static_assert(sizeof(BwdBarriers) <= 256, "barrier block too large");
 
 __device__ __forceinline__ bool wwait(uint64_t* bar, uint32_t parity, BwdBarriers* b, unsigned int* status) {
   bool ok = mbar_wait(bar, parity, &b->abort, status, kTimeoutNs);
@@ -143,10 +147,12 @@ __device__ __forceinline__ bool wwait(uint64_t* bar, uint32_t parity, BwdBarrier
 
 __device__ __forceinline__ void init_barriers(BwdBarriers* b) {
   mbar_init(&b->a_full, 1);
-  for (int s = 0; s < 2; ++s) {
+  for (int s = 0; s < 4; ++s) {
     mbar_init(&b->full[s], 1);
     mbar_init(&b->empty[s], 1);
   }
+  mbar_init(&b->sbuf[0], 1);
+  mbar_init(&b->sbuf[1], 1);
   for (int s = 0; s < 3; ++s) {
     mbar_init(&b->kfull[s], 1);
     mbar_init(&b->kempty[s], 1);
@@ -226,28 +232,42 @@ struct BwdParams {
 // ---------------------------------------------------------------------------
 // dk, dv
 // ---------------------------------------------------------------------------
+// Query tiles of 64 rows: S^T and dP^T take 64 TMEM columns each, so both are
+// double-buffered next to dV and dK ([0,64)+64b: S^T of buffer b, P^T written
+// back on its first 32 columns; [128,192)+64b: dP^T, dS^T on its first 32;
+// [256,384) dV; [384,512) dK).  The MMA warp issues S^T(u+2), dP^T(u+2) right
+// after dV(u), dK(u) (which read buffer u&1 first), so the tensor core computes
+// the next tiles while the elementwise warps work on the current one.
+constexpr uint32_t kQ64Bytes = 64 * 128 * 2;           // 64 rows x 128 channels: two 8 KB halves
+constexpr int kKVStages = 4;
 constexpr uint32_t kKV_K = 0, kKV_V = kTileBytes, kKV_Stage = 2 * kTileBytes;
-constexpr uint32_t kKV_StageBytes = 2 * kTileBytes;   // Q + dO
-constexpr uint32_t kKV_L = kKV_Stage + 2 * kKV_StageBytes;  // lse2, delta: 2 stages x 1 KB
-constexpr uint32_t kKV_Bar = kKV_L + 2 * 1024;
+constexpr uint32_t kKV_StageBytes = 2 * kQ64Bytes;     // Q + dO
+constexpr uint32_t kKV_L = kKV_Stage + kKVStages * kKV_StageBytes;  // -lse log2 e, -delta: 64 + 64 floats a stage
+constexpr uint32_t kKV_Bar = kKV_L + kKVStages * 512;
 constexpr uint32_t kKV_Smem = kKV_Bar + 256 + 1024;
+
+template <bool F16>
+struct Idesc64 {
+  static constexpr uint32_t KK = F16 ? idesc_f16_f32(128, 64, 0, 0) : idesc_bf16_f32(128, 64, 0, 0);
+};
 
 // 64-token blocks (BS = 64): an item is one key block in the top half of the
 // 128-row tile (the 128-row box also brings the next block's rows, finite and
-// masked), and each streamed 128-column query tile holds two listed query
-// blocks, loaded as 64-row boxes (tm_qs, tm_dos).  For BS = 256 the streamed
-// maps are the 128-row ones.
+// masked).  A 256-token query block is four 64-row query tiles; a 64-token
+// block is one.
 template <int BS, bool F16>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_constant__ CUtensorMap tm_k,
-                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_dos,
+    attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q64, const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do64,
                          const __grid_constant__ BwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   BwdBarriers* bars = reinterpret_cast<BwdBarriers*>(smem + kKV_Bar);
+  uint32_t* maskw = &bars->mask[0][0];  // [stage][2]
   const Geo& g = p.g;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int kHalves = BS == 256 ? 2 : 1;
+  constexpr int kTilesPerBlock = BS / 64;
   const int item = blockIdx.x;
   const int half = BS == 256 ? (item & 1) : 0;
   const int kb = (item / kHalves) % g.NB;
@@ -255,8 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int32_t* offs = p.k2q_off + static_cast<long long>(bh) * (g.NB + 1);
   const int lo = __ldg(offs + kb), hi = __ldg(offs + kb + 1);
   const int32_t* list = p.k2q + static_cast<long long>(bh) * g.NB * p.max_k + lo;
-  const int len = hi - lo;
-  const int nq = BS == 256 ? 2 * len : (len + 1) / 2;  // query tiles
+  const int nq = kTilesPerBlock * (hi - lo);  // 64-row query tiles
   const long long base = static_cast<long long>(bh) * g.Sp;
 
   if (threadIdx.x == 0) init_barriers(bars);
@@ -284,51 +303,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_2d_w(smem + kKV_V + hf * kHalfBytes, &tm_v, hf * 64, krow, &bars->a_full, pol_last);
       }
       kv = true;
+      // the next tile's query block id and validity bits are prepared before
+      // its stage is free, so that only the copies follow the wait
+      int qb_next = __ldg(list);
       for (int u = 0; u < nq; ++u) {
-        const int s = u & 1;
-        if (!wwait(&bars->empty[s], ((u >> 1) & 1) ^ 1, bars, p.status)) break;
-        // rows of the tile's query blocks: one 128-row box, or two 64-row boxes
-        // (an absent second block loads block 0, finite and masked)
-        long long qrow0, qrow1 = 0;
+        const int s = u % kKVStages;
+        const int qb = qb_next;
+        if (u + 1 < nq) qb_next = __ldg(list + (u + 1) / kTilesPerBlock);
+        const int qq = u % kTilesPerBlock;  // 64-row part of the query block
+        const long long qrow = base + static_cast<long long>(qb) * BS + 64 * qq;
         uint32_t w[4];
         if (BS == 256) {
-          const int qb = __ldg(list + (u >> 1));
-          qrow0 = base + static_cast<long long>(qb) * 256 + (u & 1) * 128;
-          tile_bits(g, qb, u & 1, w);
+          tile_bits(g, qb, qq >> 1, w);
         } else {
-          const int qa = __ldg(list + 2 * u);
-          const int qc = 2 * u + 1 < len ? __ldg(list + 2 * u + 1) : -1;
-          qrow0 = base + static_cast<long long>(qa) * 64;
-          qrow1 = base + static_cast<long long>(qc < 0 ? 0 : qc) * 64;
-          block64_mask(g, qa, w[0], w[1]);
-          block64_mask(g, qc, w[2], w[3]);
+          block64_mask(g, qb, w[0], w[1]);
         }
-        uint8_t* st = smem + kKV_Stage + s * kKV_StageBytes;
-        if (lane < 4) bars->mask[s][lane] = pick4(w, lane);  // published by the arrive below
+        const uint32_t w0 = pick4(w, BS == 256 ? 2 * (qq & 1) : 0), w1 = pick4(w, BS == 256 ? 2 * (qq & 1) + 1 : 1);
+        if (!wwait(&bars->empty[s], ((u / kKVStages) & 1) ^ 1, bars, p.status)) break;
+        if (lane < 2) maskw[2 * s + lane] = lane ? w1 : w0;  // published by the arrive below
         __syncwarp();
-        mbar_arrive_expect_tx_w(&bars->full[s], 2 * kTileBytes + 1024);
+        uint8_t* st = smem + kKV_Stage + s * kKV_StageBytes;
+        mbar_arrive_expect_tx_w(&bars->full[s], kKV_StageBytes + 512);
         for (int hf = 0; hf < 2; ++hf) {
-          tma_load_2d_w(st + hf * kHalfBytes, &tm_qs, hf * 64, static_cast<int>(qrow0), &bars->full[s], pol_last);
-          tma_load_2d_w(st + kTileBytes + hf * kHalfBytes, &tm_dos, hf * 64, static_cast<int>(qrow0), &bars->full[s],
-                        pol_last);
-          if (BS == 64) {
-            tma_load_2d_w(st + hf * kHalfBytes + kHalfBytes / 2, &tm_qs, hf * 64, static_cast<int>(qrow1),
-                          &bars->full[s], pol_last);
-            tma_load_2d_w(st + kTileBytes + hf * kHalfBytes + kHalfBytes / 2, &tm_dos, hf * 64,
-                          static_cast<int>(qrow1), &bars->full[s], pol_last);
-          }
+          tma_load_2d_w(st + hf * (kQ64Bytes / 2), &tm_q64, hf * 64, static_cast<int>(qrow), &bars->full[s], pol_last);
+          tma_load_2d_w(st + kQ64Bytes + hf * (kQ64Bytes / 2), &tm_do64, hf * 64, static_cast<int>(qrow),
+                        &bars->full[s], pol_last);
         }
         if (lane == 0) {
-          uint8_t* L = smem + kKV_L + s * 1024;
-          if (BS == 256) {
-            bulk_load(L, p.nlse2 + qrow0, 512, &bars->full[s]);
-            bulk_load(L + 512, p.ndelta + qrow0, 512, &bars->full[s]);
-          } else {
-            bulk_load(L, p.nlse2 + qrow0, 256, &bars->full[s]);
-            bulk_load(L + 256, p.nlse2 + qrow1, 256, &bars->full[s]);
-            bulk_load(L + 512, p.ndelta + qrow0, 256, &bars->full[s]);
-            bulk_load(L + 768, p.ndelta + qrow1, 256, &bars->full[s]);
-          }
+          bulk_load(smem + kKV_L + s * 512, p.nlse2 + qrow, 256, &bars->full[s]);
+          bulk_load(smem + kKV_L + s * 512 + 256, p.ndelta + qrow, 256, &bars->full[s]);
         }
         __syncwarp();
         ++issued;
@@ -336,46 +339,61 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // drain every copy in flight before shared memory is released
     if (kv) mbar_wait_drain(&bars->a_full, 0, kTimeoutNs);
-    for (int s = 0; s < 2; ++s)
+    for (int s = 0; s < kKVStages; ++s)
       if (issued > s) {
-        const int last = issued - 1 - ((issued - 1 - s) & 1);
-        mbar_wait_drain(&bars->full[s], (last >> 1) & 1, kTimeoutNs);
+        const int last = issued - 1 - ((issued - 1 - s) % kKVStages);
+        mbar_wait_drain(&bars->full[s], (last / kKVStages) & 1, kTimeoutNs);
       }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     const uint64_t dK = sdesc_sw128(smem_u32(smem + kKV_K), 16, 1024);
     const uint64_t dV = sdesc_sw128(smem_u32(smem + kKV_V), 16, 1024);
-    const uint64_t dSt = sdesc_sw128(smem_u32(smem + kKV_Stage), 16, 1024);                 // K-major view
-    const uint64_t mSt = sdesc_sw128(smem_u32(smem + kKV_Stage), kHalfBytes, 1024);         // MN-major view
-    constexpr uint64_t kStage = kKV_StageBytes >> 4, kTile = kTileBytes >> 4;
+    const uint64_t dSt = sdesc_sw128(smem_u32(smem + kKV_Stage), 16, 1024);              // K-major view
+    const uint64_t mSt = sdesc_sw128(smem_u32(smem + kKV_Stage), kQ64Bytes / 2, 1024);   // MN-major view
+    constexpr uint64_t kStage = kKV_StageBytes >> 4, kQ64 = kQ64Bytes >> 4;
+    auto issue_sdp = [&](int u) {  // S^T(u), dP^T(u) into buffer u&1
+      const int s = u % kKVStages, b = u & 1;
+      const uint64_t q_k = dSt + s * kStage, do_k = q_k + kQ64;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t ok_ = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;        // 128-row K/V tile
+        const uint32_t oq = ((kk >> 2) * (kQ64Bytes / 2) + (kk & 3) * 32) >> 4;   // 64-row Q/dO tile
+        mma_ss_w(tmem + 64 * b, dK + ok_, q_k + oq, Idesc64<F16>::KK, kk > 0 ? 1u : 0u);
+      }
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t ok_ = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+        const uint32_t oq = ((kk >> 2) * (kQ64Bytes / 2) + (kk & 3) * 32) >> 4;
+        mma_ss_w(tmem + 128 + 64 * b, dV + ok_, do_k + oq, Idesc64<F16>::KK, kk > 0 ? 1u : 0u);
+      }
+      mma_commit_w(&bars->sbuf[b]);
+    };
     bool ok = true;
     if (nq > 0) ok = wwait(&bars->a_full, 0, bars, p.status);
-    for (int u = 0; u < nq && ok; ++u) {
-      const int s = u & 1;
-      if (!(ok = wwait(&bars->full[s], (u >> 1) & 1, bars, p.status))) break;
+    for (int u = 0; u < 2 && u < nq && ok; ++u) {
+      if (!(ok = wwait(&bars->full[u], 0, bars, p.status))) break;
       tc_fence_after();
-      const uint64_t q_k = dSt + s * kStage, do_k = q_k + kTile;
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t off = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
-        mma_ss_w(tmem + 0, dK + off, q_k + off, Idesc<F16>::KK, kk > 0 ? 1u : 0u);
-      }
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t off = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
-        mma_ss_w(tmem + 128, dV + off, do_k + off, Idesc<F16>::KK, kk > 0 ? 1u : 0u);
-      }
-      mma_commit_w(&bars->s_full);
+      issue_sdp(u);
+    }
+    for (int u = 0; u < nq && ok; ++u) {
+      const int s = u % kKVStages, b = u & 1;
       if (!(ok = wwait(&bars->ds_full, u & 1, bars, p.status))) break;
       tc_fence_after();
-      const uint64_t q_m = mSt + s * kStage, do_m = q_m + kTile;
+      const uint64_t q_m = mSt + s * kStage, do_m = q_m + kQ64;
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_ts_w(tmem + 256, tmem + 0 + kk * 8, do_m + kk * (2048 >> 4), Idesc<F16>::TM, (u > 0 || kk > 0) ? 1u : 0u);
+      for (int kk = 0; kk < 4; ++kk)
+        mma_ts_w(tmem + 256, tmem + 64 * b + kk * 8, do_m + kk * (2048 >> 4), Idesc<F16>::TM,
+                 (u > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_ts_w(tmem + 384, tmem + 128 + kk * 8, q_m + kk * (2048 >> 4), Idesc<F16>::TM, (u > 0 || kk > 0) ? 1u : 0u);
+      for (int kk = 0; kk < 4; ++kk)
+        mma_ts_w(tmem + 384, tmem + 128 + 64 * b + kk * 8, q_m + kk * (2048 >> 4), Idesc<F16>::TM,
+                 (u > 0 || kk > 0) ? 1u : 0u);
       mma_commit_w(&bars->empty[s]);
+      if (u + 2 < nq) {  // buffer b is free once dV(u), dK(u) have read it (tensor core order)
+        if (!(ok = wwait(&bars->full[(u + 2) % kKVStages], ((u + 2) / kKVStages) & 1, bars, p.status))) break;
+        tc_fence_after();
+        issue_sdp(u + 2);
+      }
     }
     mma_commit_w(&bars->done);
     mma_commit_w(&bars->drain);
@@ -384,11 +402,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     regs_inc<kRegsHigh>();
     // ------------------------------------------------------------ elementwise + epilogue
-    const int wg = (warp - 4) >> 2;     // query columns [64 wg, 64 wg + 64)
+    const int wg = (warp - 4) >> 2;     // query columns [32 wg, 32 wg + 32) of the 64-row tile
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // key row of the tile
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t tS = tmem + lane_off, tP = tS + 128;
+    const uint32_t tL = tmem + lane_off;
     uint32_t kw[4];
     if (BS == 256) {
       tile_bits(g, kb, half, kw);
@@ -400,32 +418,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t c2 = f2pack(p.scale_log2, p.scale_log2);
     bool ok = true;
     for (int u = 0; u < nq && ok; ++u) {
-      const int s = u & 1;
-      if (!(ok = wwait(&bars->full[s], (u >> 1) & 1, bars, p.status))) break;
-      uint32_t qw[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) qw[i] = bars->mask[s][i];
-      if (!(ok = wwait(&bars->s_full, u & 1, bars, p.status))) break;
+      const int s = u % kKVStages, b = u & 1;
+      if (!(ok = wwait(&bars->full[s], (u / kKVStages) & 1, bars, p.status))) break;
+      const uint32_t m = kvalid ? maskw[2 * s + wg] : 0u;
+      if (!(ok = wwait(&bars->sbuf[b], (u >> 1) & 1, bars, p.status))) break;
       tc_fence_after();
-      const uint64_t* NL = reinterpret_cast<const uint64_t*>(smem + kKV_L + s * 1024);
-      const uint64_t* ND = NL + 64;
-      uint32_t pk[2][16], dk16[2][16];
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        const int ch = 2 * wg + cc;
+      const uint64_t* NL = reinterpret_cast<const uint64_t*>(smem + kKV_L + s * 512);
+      const uint64_t* ND = NL + 32;
+      uint32_t pk[16], dk16[16];
+      {
         uint32_t sv[32], dv[32];
-        tmem_ld32(tS + ch * 32, sv);
-        tmem_ld32(tP + ch * 32, dv);
+        tmem_ld32(tL + 64 * b + 32 * wg, sv);
+        tmem_ld32(tL + 128 + 64 * b + 32 * wg, dv);
         tmem_wait_ld();
-        p_ds32<F16>(sv, dv, c2, NL + 16 * ch, ND + 16 * ch, kvalid ? pick4(qw, ch) : 0u, pk[cc], dk16[cc]);
+        p_ds32<F16>(sv, dv, c2, NL + 16 * wg, ND + 16 * wg, m, pk, dk16);
       }
-      wg_pair_sync();  // every column of S^T and dP^T has been read
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        const int ch = 2 * wg + cc;
-        tmem_st16(tS + ch * 16, pk[cc]);
-        tmem_st16(tP + ch * 16, dk16[cc]);
-      }
+      wg_pair_sync();  // both halves of S^T and dP^T have been read
+      tmem_st16(tL + 64 * b + 16 * wg, pk);
+      tmem_st16(tL + 128 + 64 * b + 16 * wg, dk16);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars->ds_full);
@@ -436,9 +446,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool load = ok && nq > 0;  // warp-uniform
     if (BS == 256 || quarter < 2) {  // for 64-token blocks, lanes 64..127 are the next block's rows
       if (wg == 0)
-        store_row<F16>(tS + 256, 1.0f, p.dv + row * 128, load, false);
+        store_row<F16>(tL + 256, 1.0f, p.dv + row * 128, load, false);
       else
-        store_row<F16>(tS + 384, p.scale, p.dk + row * 128, load, false);
+        store_row<F16>(tL + 384, p.scale, p.dk + row * 128, load, false);
     }
   }
 
@@ -810,17 +820,16 @@ size_t attn_bwd_workspace_bytes(const Geo& g, int BH, int max_k) {
 template <int BS, bool F16>
 cudaError_t launch_bwd_kernels(const Geo& g, const AttnBwdArgs& a, const BwdParams& p, cudaStream_t stream) {
   const unsigned long long rows = static_cast<unsigned long long>(a.BH) * g.Sp;
-  CUtensorMap tq, tk, tv, tdo, tqs, tks, tvs, tdos;
+  CUtensorMap tq, tk, tv, tdo, tks, tvs, tq64, tdo64;
   if (!make_tmap(&tq, a.q, rows, 128, F16) || !make_tmap(&tk, a.k, rows, 128, F16) ||
       !make_tmap(&tv, a.v, rows, 128, F16) || !make_tmap(&tdo, a.dO, rows, 128, F16))
     return cudaErrorInvalidValue;
+  if (!make_tmap(&tq64, a.q, rows, 64, F16) || !make_tmap(&tdo64, a.dO, rows, 64, F16))
+    return cudaErrorInvalidValue;
   if (BS == 256) {
-    tqs = tq;
     tks = tk;
     tvs = tv;
-    tdos = tdo;
-  } else if (!make_tmap(&tqs, a.q, rows, 64, F16) || !make_tmap(&tks, a.k, rows, 64, F16) ||
-             !make_tmap(&tvs, a.v, rows, 64, F16) || !make_tmap(&tdos, a.dO, rows, 64, F16)) {
+  } else if (!make_tmap(&tks, a.k, rows, 64, F16) || !make_tmap(&tvs, a.v, rows, 64, F16)) {
     return cudaErrorInvalidValue;
   }
   const unsigned items = static_cast<unsigned>((BS == 256 ? 2ull : 1ull) * a.BH * g.NB);
@@ -831,7 +840,7 @@ cudaError_t launch_bwd_kernels(const Geo& g, const AttnBwdArgs& a, const BwdPara
   if ((e = cudaFuncSetAttribute(attn_bwd_dq_kernel<BS, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 kQ_Smem)) != cudaSuccess)
     return e;
-  attn_bwd_dkdv_kernel<BS, F16><<<items, kThreads, kKV_Smem, stream>>>(tqs, tk, tv, tdos, p);
+  attn_bwd_dkdv_kernel<BS, F16><<<items, kThreads, kKV_Smem, stream>>>(tq64, tk, tv, tdo64, p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   attn_bwd_dq_kernel<BS, F16><<<items, kThreads, kQ_Smem, stream>>>(tq, tks, tvs, tdo, p);
   return cudaGetLastError();
