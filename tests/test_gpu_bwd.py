@@ -124,6 +124,26 @@ def test_bwd_matches_oracle_everywhere(case):
         assert (t[:, :, pad] == 0).all()
 
 
+def test_bwd_repeated_ids_count_twice():
+    """A row that lists a block twice sees its keys twice in the softmax (as the
+    forward does); the transposed lists carry the repeat, and dq, dk, dv match
+    the oracle, which walks the lists as given."""
+    wl = workloads.custom(T=8, Hg=8, Wg=16, H=2, topk=1)
+    g, qt, kt, vt, do, idx, num = _problem(wl, "bf16", 3, seed=9, zero_rows=False)
+    idx[0, 0, 1, :3] = [2, 2, 0]
+    num[0, 0, 1] = 3
+    idx[0, 1, 3, :2] = [1, 1]
+    num[0, 1, 3] = 2
+    dq, dk, dv = _gpu_bwd(wl, "bf16", qt, kt, vt, do, idx, num)
+    real = H.real_rows(wl)
+    rows = np.arange(wl.H * g.Sp, dtype=np.int64)
+    ref_dq = oracle.attn_bwd_q_rows(g, qt, kt, vt, do, idx, num, rows).reshape(dq.shape)
+    ref_dk, ref_dv = oracle.attn_bwd_kv(g, qt, kt, vt, do, idx, num)
+    _check("repeat dq", _vals(dq, "bf16")[:, :, real], ref_dq[:, :, real])
+    _check("repeat dk", _vals(dk, "bf16")[:, :, real], ref_dk[:, :, real])
+    _check("repeat dv", _vals(dv, "bf16")[:, :, real], ref_dv[:, :, real])
+
+
 def _gpu_bwd_map(wl, qt, kt, vt, do, bmap):
     """Forward through the block map on the GPU, then the backward; returns the selection too."""
     plan = vsa.Plan.of(wl)
