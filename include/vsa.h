@@ -5,7 +5,7 @@
  * post-patch latent grid of a video DiT is cut into spatiotemporal blocks;
  * every query block scores all key/value blocks on block-pooled Q and K,
  * keeps its top-k, and runs attention against the tokens of those blocks
- * only.  The forward path is four calls, in stream order:
+ * only.  The forward path, in stream order:
  *
  *   vsa_tile(q), vsa_tile(k) (with pooled means), vsa_tile(v)
  *   vsa_coarse_topk(qbar, kbar)          -> q2k_idx, q2k_num
@@ -13,8 +13,20 @@
  *   vsa_sparse_attn_fwd(q, k, v, index)  -> o, lse      (tiled layout)
  *   vsa_untile(o)
  *
+ * or, with the front end in one launch,
+ *
+ *   vsa_tile_coarse(q, k, v)             -> tiled q, k, v, means, q2k_idx, q2k_num
+ *   vsa_sparse_attn_fwd_ex(...)          -> o, lse
+ *   vsa_untile(o)
+ *
+ * The gate-compress branch adds pooled v to the front end,
+ * vsa_coarse_compress (or the compression outputs of vsa_tile_coarse) and
+ * vsa_untile_gate in place of vsa_untile.  vsa_sparse_attn_bwd gives the
+ * fine stage's gradients for a fixed selection.  The _ex calls and
+ * vsa_tile_coarse take bf16 or fp16.
+ *
  * Conventions shared by every call
- *  - bf16 tensors are passed as pointers to their raw 16-bit patterns.
+ *  - bf16 / fp16 tensors are passed as pointers to their raw 16-bit patterns.
  *  - Untiled layout: [B, S, H, D] (token-major, heads inside), S = n_prefix +
  *    T*Hg*Wg tokens, video tokens in (t, y, x) raster order after the prefix.
  *  - Tiled layout: [B, H, Sp, D], Sp = NB * block_tokens.  Block b holds rows
@@ -26,7 +38,7 @@
  *  - Every device pointer must be 16-byte aligned and every buffer is owned
  *    by the caller; the library allocates no device memory in any call.
  *  - Every call is asynchronous on `stream` and returns an int status.  A
- *    non-zero return means nothing was launched.  Errors found on the device
+ *    rejected argument returns before any device work is queued.  Errors found on the device
  *    (bad block ids, counts above max_k, a pipeline wait that ran out) are
  *    recorded in a per-device status word read by vsa_get_status().
  *  - Nothing falls back: unsupported input is an error, never rerouted.
