@@ -473,6 +473,7 @@ def main():
     attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(args.steps)]
     front_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    back_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
 
     def step(i=None):
         if i is not None:
@@ -484,6 +485,8 @@ def main():
         if i is not None:
             attn_ev[i][1].record(stream)
         fwd.back(dev.get("gate"))
+        if i is not None:
+            back_ev[i].record(stream)
 
     def sync_all():
         torch.cuda.synchronize()
@@ -524,6 +527,7 @@ def main():
     elapsed = max_over_ranks(t0.elapsed_time(t1) / 1e3)
     attn_s = [a.elapsed_time(b) / 1e3 for a, b in attn_ev]
     front_s = [f.elapsed_time(a[0]) / 1e3 for f, a in zip(front_ev, attn_ev)]
+    back_s = [a[1].elapsed_time(b) / 1e3 for a, b in zip(attn_ev, back_ev)]
     attn_avg = max_over_ranks(float(np.mean(attn_s)))
     assert vsa.get_status() == vsa.VSA_OK
 
@@ -580,6 +584,13 @@ def main():
                 "num_blocks": wl.num_blocks, "topk": wl.topk, "selected_block_tflop_per_step": flops / 1e12,
                 "selected_pairs": int(fwd.num.sum().item()),
                 "attn_ms": attn_avg * 1e3, "front_ms": float(np.mean(front_s)) * 1e3,
+                "back_ms": float(np.mean(back_s)) * 1e3,
+                # memory-bound stages: algorithmic bytes (untiled q, k, v read + tiled written; tiled o
+                # read + untiled o written, plus the gate when gated) over their event time
+                "front_gbs": (3 * host["q"].numel() * 2 + 3 * fwd.qt.numel() * 2) / float(np.mean(front_s)) / 1e9,
+                "back_gbs": (fwd.ot.numel() * 2 + fwd.o.numel() * 2 * (2 if args.gate else 1))
+                / float(np.mean(back_s)) / 1e9,
+                "hbm_peak_gbs": measured_peaks()[2],
                 "l2": "inputs larger than L2: q/k/v %.0f MB and tiled q/k/v %.0f MB per step" % (
                     sum(host[n].numel() * 2 for n in ("q", "k", "v")) / 1e6, 3 * fwd.qt.numel() * 2 / 1e6),
                 "parallelism": f"replicas x{world}",
