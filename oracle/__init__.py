@@ -16,6 +16,10 @@ Each step follows the statement cited in the C file's header:
 * ``attn_bwd_q_rows``/``attn_bwd_kv``: gradients of the attention step with
   the selection fixed (definition of softmax attention's derivative; the
   commit log keeps the grad path separate), in fp64, real query rows only;
+* ``quant_nvfp4``/``dequant_nvfp4``/``attn_rows_nvfp4``: FastVideo
+  "Optimizations" page, section "FP4 Flash Attention 4 (Blackwell only)" (Q
+  and K as NVFP4: E2M1 values, per-block E4M3 scales; V 16-bit); block length
+  16 and the amax/6 scale are NVFP4's own definition, stated in the C file;
 * ``compress``/``gate_rows``: "FastVideo VSA", section "Checkpoint behavior"
   (learned gate_compress projection) and the FastVideo commit log (the
   gate-compress branch pools per tile); the formula is a reading, stated in
@@ -74,11 +78,16 @@ def _load():
         lib.oracle_gate_rows.argtypes = geo + [P, L, P, P, P, i, i, i, P, i]
         lib.oracle_attn_bwd_q_rows.argtypes = geo + [P, P, P, P, P, P, i, i, i, i, P, L, P, i]
         lib.oracle_attn_bwd_kv.argtypes = geo + [P, P, P, P, P, P, i, i, i, i, P, P, i]
+        lib.oracle_quant_nvfp4.argtypes = [P, L, i, P, P, i]
+        lib.oracle_dequant_nvfp4.argtypes = [P, P, L, i, P]
+        lib.oracle_e4m3_round.argtypes = [P, L, P]
+        lib.oracle_attn_rows_nvfp4.argtypes = geo + [P, P, P, P, P, P, P, i, i, P, L, P, P, i]
         lib.oracle_max_threads.argtypes = []
         for f in ("oracle_geometry", "oracle_block_valid_counts", "oracle_tile", "oracle_untile",
                   "oracle_pool", "oracle_score", "oracle_topk", "oracle_map_to_index",
                   "oracle_attn_rows", "oracle_max_threads", "oracle_half_to_f32", "oracle_compress",
-                  "oracle_gate_rows", "oracle_attn_bwd_q_rows", "oracle_attn_bwd_kv"):
+                  "oracle_gate_rows", "oracle_attn_bwd_q_rows", "oracle_attn_bwd_kv", "oracle_quant_nvfp4",
+                  "oracle_dequant_nvfp4", "oracle_e4m3_round", "oracle_attn_rows_nvfp4"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -294,3 +303,50 @@ def attn_bwd_kv(g: Geometry, qt, kt, vt, dot, idx, num, dtype: str = "bf16"):
     _check(_load().oracle_attn_bwd_kv(*g.args, *[_ptr(a) for a in arrs], _ptr(idx), _ptr(num), idx.shape[-1],
                                       B, H, D, _ptr(dk), _ptr(dv), DTYPES[dtype]), "attn_bwd_kv")
     return dk, dv
+
+
+def quant_nvfp4(x: np.ndarray, dtype: str = "bf16"):
+    """16-bit rows [..., D] -> (codes [..., D/2] uint8, scales [..., D/16] uint8 E4M3)."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    D = x.shape[-1]
+    rows = x.size // D
+    codes = np.empty(x.shape[:-1] + (D // 2,), dtype=np.uint8)
+    sf = np.empty(x.shape[:-1] + (D // 16,), dtype=np.uint8)
+    _check(_load().oracle_quant_nvfp4(_ptr(x), rows, D, _ptr(codes), _ptr(sf), DTYPES[dtype]), "quant_nvfp4")
+    return codes, sf
+
+
+def dequant_nvfp4(codes: np.ndarray, sf: np.ndarray) -> np.ndarray:
+    """The values NVFP4 codes and scales stand for, fp64 [..., D]."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    sf = np.ascontiguousarray(sf, dtype=np.uint8)
+    D = codes.shape[-1] * 2
+    rows = codes.size // (D // 2)
+    y = np.empty(codes.shape[:-1] + (D,), dtype=np.float64)
+    _check(_load().oracle_dequant_nvfp4(_ptr(codes), _ptr(sf), rows, D, _ptr(y)), "dequant_nvfp4")
+    return y
+
+
+def e4m3_round(x: np.ndarray) -> np.ndarray:
+    """E4M3 bits of non-negative fp32 values (nearest, ties to even, capped at 448)."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    bits = np.empty(x.shape, dtype=np.uint8)
+    _check(_load().oracle_e4m3_round(_ptr(x), x.size, _ptr(bits)), "e4m3_round")
+    return bits
+
+
+def attn_rows_nvfp4(g: Geometry, qc, qs, kc, ks, vt, idx, num, rows, dtype: str = "bf16"):
+    """fp64 attention of flat rows of [B,H,Sp] with NVFP4 q, k (row-major codes/scales) and 16-bit v."""
+    qc, kc = (np.ascontiguousarray(a, dtype=np.uint8) for a in (qc, kc))
+    qs, ks = (np.ascontiguousarray(a, dtype=np.uint8) for a in (qs, ks))
+    vt = np.ascontiguousarray(vt, dtype=np.uint16)
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    num = np.ascontiguousarray(num, dtype=np.int32)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    D = vt.shape[-1]
+    o = np.empty((len(rows), D), dtype=np.float64)
+    lse = np.empty(len(rows), dtype=np.float64)
+    _check(_load().oracle_attn_rows_nvfp4(*g.args, _ptr(qc), _ptr(qs), _ptr(kc), _ptr(ks), _ptr(vt), _ptr(idx),
+                                          _ptr(num), idx.shape[-1], D, _ptr(rows), len(rows), _ptr(o), _ptr(lse),
+                                          DTYPES[dtype]), "attn_rows_nvfp4")
+    return o, lse

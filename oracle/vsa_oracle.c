@@ -293,6 +293,26 @@ int oracle_map_to_index(const uint8_t *map, int B, int H, int NQ, int NK, int32_
  * idx[r, 0..num[r]-1]; o_i = sum_j softmax_j(scale q_i.k_j) v_j,
  * lse_i = log sum_j exp(scale q_i.k_j), scale = 1/sqrt(D).
  */
+/* Where the q or k operand of the attention lives: 16-bit patterns, or NVFP4
+ * codes and scales (nvfp4_value below). */
+typedef struct {
+    const uint16_t *bits;
+    const uint8_t *codes, *sf;
+    int dtype;
+} operand_t;
+
+static double nvfp4_value(const uint8_t *codes, const uint8_t *sf, size_t row, int D, int d);
+
+/* Element d of tiled row `row` (flat over [B,H,Sp]) of an operand. */
+static double operand_value(const operand_t *op, size_t row, int D, int d) {
+    if (op->bits) return half_to_f32(op->bits[row * D + d], op->dtype);
+    return nvfp4_value(op->codes, op->sf, row, D, d);
+}
+
+static int attn_rows_core(const geom_t *gp, const operand_t *qop, const operand_t *kop, const uint16_t *v,
+                          const int32_t *idx, const int32_t *num, int max_k, int D, const int64_t *rows,
+                          long n_rows, double *o_rows, double *lse_rows, int dtype);
+
 int oracle_attn_rows(int n_prefix, int T, int Hg, int Wg, int bt, int bh, int bw,
                      const uint16_t *q, const uint16_t *k, const uint16_t *v,
                      const int32_t *idx, const int32_t *num, int max_k,
@@ -302,6 +322,14 @@ int oracle_attn_rows(int n_prefix, int T, int Hg, int Wg, int bt, int bh, int bw
     int rc = geom_init(&g, n_prefix, T, Hg, Wg, bt, bh, bw);
     if (rc) return rc;
     (void)B; (void)H; /* rows are flat indices into [B,H,Sp] */
+    const operand_t qop = {q, NULL, NULL, dtype}, kop = {k, NULL, NULL, dtype};
+    return attn_rows_core(&g, &qop, &kop, v, idx, num, max_k, D, rows, n_rows, o_rows, lse_rows, dtype);
+}
+
+static int attn_rows_core(const geom_t *gp, const operand_t *qop, const operand_t *kop, const uint16_t *v,
+                          const int32_t *idx, const int32_t *num, int max_k, int D, const int64_t *rows,
+                          long n_rows, double *o_rows, double *lse_rows, int dtype) {
+    const geom_t g = *gp;
     if (D < 1 || D > 512 || max_k < 1) return ORACLE_ERR_ARG;
     const double scale = 1.0 / sqrt((double)D);
     int bad = 0;
@@ -320,7 +348,7 @@ int oracle_attn_rows(int n_prefix, int T, int Hg, int Wg, int bt, int bh, int bw
             continue;
         }
         double qi[512];
-        for (int d = 0; d < D; ++d) qi[d] = half_to_f32(q[((size_t)bhh * g.Sp + i) * D + d], dtype);
+        for (int d = 0; d < D; ++d) qi[d] = operand_value(qop, (size_t)bhh * g.Sp + i, D, d);
         double *logit = (double *)malloc(sizeof(double) * (size_t)cnt * g.bs);
         long *key = (long *)malloc(sizeof(long) * (size_t)cnt * g.bs);
         long nk = 0;
@@ -330,9 +358,8 @@ int oracle_attn_rows(int n_prefix, int T, int Hg, int Wg, int bt, int bh, int bw
             for (int slot = 0; slot < g.bs; ++slot) {
                 if (!slot_is_valid(&g, kb, slot)) continue;
                 long j = (long)kb * g.bs + slot;
-                const uint16_t *kj = k + ((size_t)bhh * g.Sp + j) * D;
                 double dot = 0.0;
-                for (int d = 0; d < D; ++d) dot += qi[d] * (double)half_to_f32(kj[d], dtype);
+                for (int d = 0; d < D; ++d) dot += qi[d] * operand_value(kop, (size_t)bhh * g.Sp + j, D, d);
                 logit[nk] = scale * dot;
                 key[nk] = j;
                 ++nk;
@@ -572,6 +599,145 @@ int oracle_gate_rows(int n_prefix, int T, int Hg, int Wg, int bt, int bh, int bw
     }
     free(token_of_slot);
     return bad ? ORACLE_ERR_INDEX : ORACLE_OK;
+}
+
+/* ---------------------------------------------------------------------------
+ * NVFP4 Q and K.  FastVideo "Optimizations" page, section "FP4 Flash
+ * Attention 4 (Blackwell only)": Q and K are quantised to NVFP4 -- E2M1
+ * values with per-block E4M3 scale factors -- while V stays 16-bit.  The page
+ * fixes neither the block length nor how a scale is chosen; the readings
+ * taken are NVFP4's own definition:
+ *   - a block is 16 consecutive channels of one token;
+ *   - its scale is amax / 6 (6 = the largest E2M1 magnitude), one fp32
+ *     division, rounded to E4M3;
+ *   - each value becomes x * (1 / scale), one fp32 reciprocal and one fp32
+ *     multiply, rounded to E2M1; a scale that rounds to 0 gives 1/scale := 0.
+ * Both roundings take the nearest representable value, ties to the one whose
+ * last mantissa bit is 0, and stop at the largest finite value (448, 6); E2M1
+ * keeps the sign of its input, zero included.
+ * Formats: E4M3 = sign, 4 exponent bits (bias 7), 3 mantissa bits, step 2^-9
+ * below 2^-6; E2M1 = sign, 2 exponent bits (bias 1), 1 mantissa bit, step 0.5
+ * below 1: magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6.
+ * Storage: codes [rows, D/2] bytes, channel 2j in the low nibble of byte j and
+ * 2j+1 in the high nibble; scales [rows, D/16] bytes, block order.
+ * --------------------------------------------------------------------------- */
+
+/* v >= 0 rounded to the binary grid with `mbits` mantissa bits whose smallest
+ * normal binade is 2^emin (below it the step stays 2^(emin - mbits)); ties to
+ * the even multiple of the step. */
+static double round_to_grid(double v, int mbits, int emin) {
+    if (v == 0.0) return 0.0;
+    int e;
+    frexp(v, &e);         /* v = f 2^e with f in [1/2, 1): leading bit 2^(e-1) */
+    int lead = e - 1;
+    if (lead < emin) lead = emin;
+    const double step = ldexp(1.0, lead - mbits);
+    return nearbyint(v / step) * step; /* v / step is exact; default mode: half to even */
+}
+
+/* Bits of an E4M3 magnitude already on the grid (0 <= v <= 448). */
+static uint8_t e4m3_bits(double v) {
+    if (v < ldexp(1.0, -6)) return (uint8_t)(v / ldexp(1.0, -9));
+    int e;
+    frexp(v, &e);
+    const int lead = e - 1;
+    const int mant = (int)(v / ldexp(1.0, lead - 3)) - 8;
+    return (uint8_t)(((lead + 7) << 3) | mant);
+}
+
+static double e4m3_value(uint8_t b) {
+    const int ex = (b >> 3) & 15, mant = b & 7;
+    const double mag = ex == 0 ? ldexp((double)mant, -9) : ldexp(8.0 + mant, ex - 10);
+    return (b & 0x80) ? -mag : mag;
+}
+
+/* Bits of an E2M1 magnitude already on the grid (0 <= m <= 6). */
+static int e2m1_bits(double m) {
+    if (m < 1.0) return (int)(m / 0.5);
+    int e;
+    frexp(m, &e);
+    const int lead = e - 1;
+    const int mant = (int)(m / ldexp(1.0, lead - 1)) - 2;
+    return ((lead + 1) << 1) | mant;
+}
+
+static double e2m1_value(int c) {
+    const int ex = (c >> 1) & 3, mant = c & 1;
+    const double mag = ex == 0 ? 0.5 * mant : ldexp(2.0 + mant, ex - 2);
+    return (c & 8) ? -mag : mag;
+}
+
+static double nvfp4_value(const uint8_t *codes, const uint8_t *sf, size_t row, int D, int d) {
+    const uint8_t byte = codes[row * (size_t)(D / 2) + d / 2];
+    const int c = (d & 1) ? (byte >> 4) : (byte & 15);
+    return e2m1_value(c) * e4m3_value(sf[row * (size_t)(D / 16) + d / 16]);
+}
+
+int oracle_quant_nvfp4(const uint16_t *x, long rows, int D, uint8_t *codes, uint8_t *sf, int dtype) {
+    if (rows < 0 || D < 16 || D % 16) return ORACLE_ERR_ARG;
+#pragma omp parallel for schedule(static)
+    for (long r = 0; r < rows; ++r) {
+        for (int b = 0; b < D / 16; ++b) {
+            float xs[16], amax = 0.0f;
+            for (int j = 0; j < 16; ++j) {
+                xs[j] = half_to_f32(x[(size_t)r * D + 16 * b + j], dtype);
+                if (fabsf(xs[j]) > amax) amax = fabsf(xs[j]);
+            }
+            const float s32 = amax / 6.0f;
+            double s = round_to_grid((double)s32, 3, -6);
+            if (s > 448.0) s = 448.0;
+            const uint8_t sb = e4m3_bits(s);
+            sf[(size_t)r * (D / 16) + b] = sb;
+            const float sdec = (float)e4m3_value(sb);
+            const float inv = sdec == 0.0f ? 0.0f : 1.0f / sdec;
+            uint8_t *out = codes + (size_t)r * (D / 2) + 8 * b;
+            for (int j = 0; j < 16; ++j) {
+                const float y = xs[j] * inv;
+                double m = round_to_grid(fabs((double)y), 1, 0);
+                if (m > 6.0) m = 6.0;
+                const int c = e2m1_bits(m) | (signbit(y) ? 8 : 0);
+                if (j % 2 == 0)
+                    out[j / 2] = (uint8_t)c;
+                else
+                    out[j / 2] = (uint8_t)(out[j / 2] | (c << 4));
+            }
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* The values NVFP4 codes and scales stand for: y [rows, D] doubles. */
+int oracle_dequant_nvfp4(const uint8_t *codes, const uint8_t *sf, long rows, int D, double *y) {
+    if (rows < 0 || D < 16 || D % 16) return ORACLE_ERR_ARG;
+    for (long r = 0; r < rows; ++r)
+        for (int d = 0; d < D; ++d) y[(size_t)r * D + d] = nvfp4_value(codes, sf, (size_t)r, D, d);
+    return ORACLE_OK;
+}
+
+/* E4M3 bits of fp32 values (the scale rounding above, exposed for its pins). */
+int oracle_e4m3_round(const float *x, long n, uint8_t *bits) {
+    for (long i = 0; i < n; ++i) {
+        if (!(x[i] >= 0.0f)) return ORACLE_ERR_ARG;
+        double s = round_to_grid((double)x[i], 3, -6);
+        if (s > 448.0) s = 448.0;
+        bits[i] = e4m3_bits(s);
+    }
+    return ORACLE_OK;
+}
+
+/* Attention of explicit query rows with NVFP4 q and k (codes + scales in the
+ * storage above, tiled row order) and 16-bit v: the same definition as
+ * oracle_attn_rows, on the values the codes stand for. */
+int oracle_attn_rows_nvfp4(int n_prefix, int T, int Hg, int Wg, int bt, int bh, int bw,
+                           const uint8_t *qc, const uint8_t *qs, const uint8_t *kc, const uint8_t *ks,
+                           const uint16_t *v, const int32_t *idx, const int32_t *num, int max_k,
+                           int D, const int64_t *rows, long n_rows, double *o_rows, double *lse_rows, int dtype) {
+    geom_t g;
+    int rc = geom_init(&g, n_prefix, T, Hg, Wg, bt, bh, bw);
+    if (rc) return rc;
+    if (D < 16 || D % 16) return ORACLE_ERR_ARG;
+    const operand_t qop = {NULL, qc, qs, dtype}, kop = {NULL, kc, ks, dtype};
+    return attn_rows_core(&g, &qop, &kop, v, idx, num, max_k, D, rows, n_rows, o_rows, lse_rows, dtype);
 }
 
 /* Highest thread count OpenMP will use here (1 without OpenMP). */
