@@ -37,6 +37,9 @@ from block_sparse_video_gather_b200 import workloads  # noqa: E402
 PROFILE = os.path.join(ROOT, "profiles", "attn_fwd_fastwan.md")
 ATTN_SOURCES = [os.path.join(ROOT, "block_sparse_video_gather_b200", "csrc", f)
                 for f in ("attn_fwd.cu", "common.cuh", "tiles.cuh")]
+FP4_PROFILE = os.path.join(ROOT, "profiles", "attn_fwd_fp4_fastwan.md")
+FP4_SOURCES = [os.path.join(ROOT, "block_sparse_video_gather_b200", "csrc", f)
+               for f in ("fp4.cu", "common.cuh", "tiles.cuh")]
 WORKLOAD_TEXT = {
     "tiny": "tiny grid 8x16x16, B1 H2 D128, block 4x8x8, topk 4",
     "fastwan": "FastWan2.2-TI2V-5B latent grid 31x22x40, B1 H24 D128, block 4x8x8, topk 64",
@@ -56,23 +59,23 @@ def uniform_flops(wl) -> float:
     return 4.0 * wl.D * wl.block_tokens ** 2 * wl.B * wl.H * wl.num_blocks * wl.topk
 
 
-def attn_source_hash() -> str:
+def attn_source_hash(sources=None) -> str:
     h = hashlib.sha256()
-    for f in ATTN_SOURCES:
+    for f in sources or ATTN_SOURCES:
         h.update(open(f, "rb").read())
     return h.hexdigest()[:16]
 
 
-def profile_traffic(workload: str):
+def profile_traffic(workload: str, profile: str = PROFILE, sources=None):
     """DRAM bytes per attention launch from the committed ncu summary, or None when
     the summary is absent, for another workload, or older than the kernel source."""
-    if not os.path.exists(PROFILE):
+    if not os.path.exists(profile):
         return None
-    text = open(PROFILE).read()
+    text = open(profile).read()
     m_src = re.search(r"source_hash:\s*([0-9a-f]+)", text)
     m_wl = re.search(r"bench_workload:\s*(\w+)", text)
     m_b = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    if not (m_src and m_wl and m_b) or m_src.group(1) != attn_source_hash() or m_wl.group(1) != workload:
+    if not (m_src and m_wl and m_b) or m_src.group(1) != attn_source_hash(sources) or m_wl.group(1) != workload:
         return None
     return float(m_b.group(1))
 
@@ -162,9 +165,14 @@ def run_reference(args, wl, world, rank):
             idx, num = oracle.map_to_index(inp["map"])
         else:
             idx, num = oracle.topk(oracle.score(qbar, kbar), wl.topk)
+        if args.nvfp4:
+            (qc, qs), (kc, ks) = oracle.quant_nvfp4(qt), oracle.quant_nvfp4(kt)
         t1 = time.perf_counter()
         rows = np.sort(rng.choice(total_rows, size=sample_rows, replace=False))
-        o, _ = oracle.attn_rows(g, qt, kt, vt, idx, num, rows)
+        if args.nvfp4:
+            oracle.attn_rows_nvfp4(g, qc, qs, kc, ks, vt, idx, num, rows)
+        else:
+            oracle.attn_rows(g, qt, kt, vt, idx, num, rows)
         t2 = time.perf_counter()
         ot = np.zeros((wl.B, wl.H, g.Sp, wl.D), dtype=np.uint16)
         oracle.untile(g, ot)
@@ -181,8 +189,9 @@ def run_reference(args, wl, world, rank):
     flops = selected_flops(wl, num)
     value = flops / est / 1e12
     cores = oracle.max_threads()
-    sample = (f"per step: oracle tile/pool/score/top-k/untile over the whole workload, attention on "
-              f"{sample_rows} of {total_rows} query rows drawn at random, scaled to all rows")
+    sample = (f"per step: oracle tile/pool/score/top-k{'/NVFP4 quantisation of q, k' if args.nvfp4 else ''}/untile "
+              f"over the whole workload, attention on {sample_rows} of {total_rows} query rows drawn at random, "
+              f"scaled to all rows")
     line = {
         "impl": "reference", "metric": "VSA sparse-attn fwd effective TFLOP/s (selected blocks) on 1 B200",
         "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -195,7 +204,7 @@ def run_reference(args, wl, world, rank):
     print(json.dumps(line), flush=True)
 
 
-def cpu_baseline_sample(wl, seconds_hint=20.0):
+def cpu_baseline_sample(wl, seconds_hint=20.0, nvfp4=False):
     """Oracle throughput on a bounded sample of the workload (about 10-30 s of CPU work)."""
     import oracle
     g = oracle.geometry_of(wl)
@@ -207,6 +216,8 @@ def cpu_baseline_sample(wl, seconds_hint=20.0):
         idx, num = oracle.map_to_index(inp["map"])
     else:
         idx, num = oracle.topk(oracle.score(qbar, kbar), wl.topk)
+    if nvfp4:
+        (qc, qs), (kc, ks) = oracle.quant_nvfp4(qt), oracle.quant_nvfp4(kt)
     oracle.untile(g, qt)
     t_front = time.perf_counter() - t0
     total_rows = wl.B * wl.H * g.Sp
@@ -216,14 +227,18 @@ def cpu_baseline_sample(wl, seconds_hint=20.0):
     while t_attn < seconds_hint * 0.5 and done < total_rows:
         rows = np.sort(rng.choice(total_rows, size=min(n, total_rows), replace=False))
         t1 = time.perf_counter()
-        oracle.attn_rows(g, qt, kt, vt, idx, num, rows)
+        if nvfp4:
+            oracle.attn_rows_nvfp4(g, qc, qs, kc, ks, vt, idx, num, rows)
+        else:
+            oracle.attn_rows(g, qt, kt, vt, idx, num, rows)
         t_attn += time.perf_counter() - t1
         done += len(rows)
         n *= 2
     est = t_front + t_attn * total_rows / done
     value = selected_flops(wl, num) / est / 1e12
     return {"value": value, "unit": "TFLOP/s", "cores": oracle.max_threads(), "kind": "oracle",
-            "sample": (f"oracle tile+pool+score+top-k+untile over the whole workload ({t_front:.1f} s) and "
+            "sample": (f"oracle tile+pool+score+top-k{'+NVFP4 quantisation' if nvfp4 else ''}+untile over the "
+                       f"whole workload ({t_front:.1f} s) and "
                        f"attention on {done} of {total_rows} query rows ({t_attn:.1f} s), scaled to all rows; "
                        f"estimated {est:.0f} s per step")}
 
@@ -426,6 +441,8 @@ def main():
                     help="run the front end as separate tile / coarse launches instead of one")
     ap.add_argument("--gate", action="store_true",
                     help="add the gate-compress branch (pooled v, block-level attention, gated sum in untile)")
+    ap.add_argument("--nvfp4", action="store_true",
+                    help="NVFP4 q and k in the fine stage (quantisation + FP4 Q K^T), v and P 16-bit")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -466,13 +483,15 @@ def main():
         host["map"] = torch.from_numpy(inp["map"].view(np.uint8)).pin_memory()
     dev = {n: host[n].to("cuda", non_blocking=False) for n in host}
     plan = vsa.Plan.of(wl)
-    fwd = vsa.Forward(plan, wl.B, wl.H, wl.topk, dtype=tdt, gated=args.gate, fused=not args.unfused)
+    fwd = vsa.Forward(plan, wl.B, wl.H, wl.topk, dtype=tdt, gated=args.gate, fused=not args.unfused,
+                      nvfp4=args.nvfp4)
     o_host = torch.empty(fwd.o.shape, dtype=tdt).pin_memory()
 
     stream = torch.cuda.current_stream()
     attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(args.steps)]
     front_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    quant_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     back_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
 
     def step(i=None):
@@ -480,8 +499,11 @@ def main():
             front_ev[i].record(stream)
         fwd.front(dev["q"], dev["k"], dev["v"], dev.get("map"))
         if i is not None:
+            quant_ev[i].record(stream)
+        fwd.quantize()
+        if i is not None:
             attn_ev[i][0].record(stream)
-        fwd.fine()
+        fwd.attend()
         if i is not None:
             attn_ev[i][1].record(stream)
         fwd.back(dev.get("gate"))
@@ -526,7 +548,8 @@ def main():
     clocks = sampler.stop()
     elapsed = max_over_ranks(t0.elapsed_time(t1) / 1e3)
     attn_s = [a.elapsed_time(b) / 1e3 for a, b in attn_ev]
-    front_s = [f.elapsed_time(a[0]) / 1e3 for f, a in zip(front_ev, attn_ev)]
+    front_s = [f.elapsed_time(q) / 1e3 for f, q in zip(front_ev, quant_ev)]
+    quant_s = [q.elapsed_time(a[0]) / 1e3 for q, a in zip(quant_ev, attn_ev)]
     back_s = [a[1].elapsed_time(b) / 1e3 for a, b in zip(attn_ev, back_ev)]
     attn_avg = max_over_ranks(float(np.mean(attn_s)))
     assert vsa.get_status() == vsa.VSA_OK
@@ -568,8 +591,16 @@ def main():
     if rank == 0:
         burst, sustained, hbm, peak_kind = measured_peaks()
         peak = burst
+        peak_source = (f"{peak_kind} bf16 burst (MEASURED_PEAKS.json)" if peak_kind == "measured"
+                       else "fallback 1.59 PFLOP/s")
+        if args.nvfp4:
+            # half the flops (S = Q K^T) at the FP4 rate, 4x the bf16 rate (nominal 9 / 2.25 PFLOP/s),
+            # half (O += P V) at the bf16 rate: 2 / (1/(4P) + 1/P) = 1.6 P
+            peak = 1.6 * burst
+            peak_source += " x 1.6 (Q K^T at the nominal FP4:bf16 ratio 4, P V at bf16)"
         achieved = flops / attn_avg / 1e12
-        traffic = profile_traffic(args.workload)
+        traffic = (profile_traffic(args.workload, FP4_PROFILE, FP4_SOURCES) if args.nvfp4
+                   else profile_traffic(args.workload))
         line = {
             "metric": "VSA sparse-attn fwd effective TFLOP/s (selected blocks) on 1 B200",
             "value": world * flops * args.steps / elapsed / 1e12,
@@ -577,13 +608,15 @@ def main():
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": elapsed / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": args.dtype, "data": "synthetic (seeded; the recipe in block_sparse_video_gather_b200/workloads.py)",
+            "dtype": f"nvfp4 q,k + {args.dtype} v,p" if args.nvfp4 else args.dtype, "data": "synthetic (seeded; the recipe in block_sparse_video_gather_b200/workloads.py)",
             "config": {
                 "workload": WORKLOAD_TEXT[args.workload],
                 "B": wl.B, "H": wl.H, "D": wl.D, "grid": [wl.T, wl.Hg, wl.Wg], "block": list(wl.block),
                 "num_blocks": wl.num_blocks, "topk": wl.topk, "selected_block_tflop_per_step": flops / 1e12,
                 "selected_pairs": int(fwd.num.sum().item()),
                 "attn_ms": attn_avg * 1e3, "front_ms": float(np.mean(front_s)) * 1e3,
+                "quant_ms": float(np.mean(quant_s)) * 1e3,
+                "qk_format": "NVFP4 (E2M1, E4M3 scale per 16 channels)" if args.nvfp4 else args.dtype,
                 "back_ms": float(np.mean(back_s)) * 1e3,
                 # memory-bound stages: algorithmic bytes (untiled q, k, v read + tiled written; tiled o
                 # read + untiled o written, plus the gate when gated) over their event time
@@ -598,10 +631,9 @@ def main():
                 "front_end": "separate launches" if args.unfused else "one launch (tile + coarse)",
             },
             "roofline": {
-                "bound": "tensor", "kernel": "attn_fwd_kernel", "achieved": achieved,
-                "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                "peak_source": f"{peak_kind} bf16 burst (MEASURED_PEAKS.json)" if peak_kind == "measured"
-                else "fallback 1.59 PFLOP/s",
+                "bound": "tensor", "kernel": "attn_fwd_fp4_kernel" if args.nvfp4 else "attn_fwd_kernel",
+                "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "peak_source": peak_source,
                 "traffic": traffic,
             },
             "clocks": clocks,
@@ -613,7 +645,7 @@ def main():
             "gpu_launches": args.steps * fwd.launches(wl.map_driven),
         }
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline_sample(wl)
+            line["cpu_baseline"] = cpu_baseline_sample(wl, nvfp4=args.nvfp4)
         print(json.dumps(line), flush=True)
     if pg:
         pg.barrier()

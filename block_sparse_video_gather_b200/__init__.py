@@ -28,7 +28,7 @@ SYMBOLS = (
     "vsa_plan_describe", "vsa_tile", "vsa_tile_ex", "vsa_untile", "vsa_coarse_topk", "vsa_map_to_index",
     "vsa_sparse_attn_fwd", "vsa_sparse_attn_fwd_ex", "vsa_get_status", "vsa_strerror",
     "vsa_coarse_compress", "vsa_untile_gate", "vsa_tile_coarse", "vsa_tile_coarse_static",
-    "vsa_sparse_attn_bwd_workspace", "vsa_sparse_attn_bwd",
+    "vsa_sparse_attn_bwd_workspace", "vsa_sparse_attn_bwd", "vsa_quantize_nvfp4", "vsa_sparse_attn_fwd_nvfp4",
 )
 
 VSA_BF16 = 0
@@ -80,6 +80,8 @@ def lib():
         L.vsa_sparse_attn_bwd_workspace.argtypes = [P, i, i, i, P]
         L.vsa_sparse_attn_bwd.argtypes = [P, i, P, P, P, P, P, P, P, P, i, i, i, i, P, P, P, P, P]
         L.vsa_sparse_attn_fwd.argtypes = [P, P, P, P, P, P, i, i, i, i, P, P, P]
+        L.vsa_quantize_nvfp4.argtypes = [P, i, P, i, i, i, P, P, P]
+        L.vsa_sparse_attn_fwd_nvfp4.argtypes = [P, i, P, P, P, P, P, P, P, i, i, i, i, P, P, P]
         L.vsa_get_status.argtypes = [P, P]
         L.vsa_strerror.argtypes = [i]
         L.vsa_strerror.restype = ctypes.c_char_p
@@ -321,6 +323,52 @@ def sparse_attn_fwd(plan: Plan, q, k, v, q2k_idx, q2k_num, o_out=None, lse_out=N
     return o_out, lse_out
 
 
+def quantize_nvfp4(plan: Plan, xt, codes=None, scales=None):
+    """Tiled q or k [B,H,Sp,D] -> NVFP4 (codes [B,H,Sp,D/2] uint8, scales [B,H,Sp/128,1024] uint8 in the
+    tensor core's layout; see vsa_quantize_nvfp4)."""
+    torch = _torch()
+    B, H, Sp, D = xt.shape
+    code = _dtype_code(xt, "x_tiled")
+    if codes is None:
+        codes = torch.empty((B, H, Sp, D // 2), dtype=torch.uint8, device=xt.device)
+    if scales is None:
+        scales = torch.empty((B, H, Sp // 128, 64 * D // 8), dtype=torch.uint8, device=xt.device)
+    if codes.numel() != B * H * Sp * D // 2 or scales.numel() != B * H * Sp * D // 16:
+        raise ValueError("codes / scales have the wrong size")
+    _check(lib().vsa_quantize_nvfp4(plan.handle, code, _ptr(xt, xt.dtype, "x_tiled"), B, H, D,
+                                    _ptr(codes, torch.uint8, "codes"), _ptr(scales, torch.uint8, "scales"),
+                                    _stream()), "vsa_quantize_nvfp4")
+    return codes, scales
+
+
+def sparse_attn_fwd_nvfp4(plan: Plan, q_codes, q_scales, k_codes, k_scales, v, q2k_idx, q2k_num, o_out=None,
+                          lse_out=None):
+    """Fine stage with NVFP4 q, k (from quantize_nvfp4) and 16-bit v (tiled layout) -> (o, lse)."""
+    torch = _torch()
+    B, H, Sp, D = v.shape
+    max_k = q2k_idx.shape[-1]
+    code = _dtype_code(v, "v")
+    for t, n in ((q_codes, "q_codes"), (k_codes, "k_codes")):
+        if t.numel() != B * H * Sp * D // 2:
+            raise ValueError(f"{n} has the wrong size")
+    for t, n in ((q_scales, "q_scales"), (k_scales, "k_scales")):
+        if t.numel() != B * H * Sp * D // 16:
+            raise ValueError(f"{n} has the wrong size")
+    if o_out is None:
+        o_out = torch.empty_like(v)
+    if lse_out is None:
+        lse_out = torch.empty((B, H, Sp), dtype=torch.float32, device=v.device)
+    u8 = torch.uint8
+    _check(lib().vsa_sparse_attn_fwd_nvfp4(plan.handle, code, _ptr(q_codes, u8, "q_codes"),
+                                           _ptr(q_scales, u8, "q_scales"), _ptr(k_codes, u8, "k_codes"),
+                                           _ptr(k_scales, u8, "k_scales"), _ptr(v, v.dtype, "v"),
+                                           _ptr(q2k_idx, torch.int32, "q2k_idx"), _ptr(q2k_num, torch.int32, "q2k_num"),
+                                           max_k, B, H, D, _ptr(o_out, v.dtype, "o"),
+                                           _ptr(lse_out, torch.float32, "lse"), _stream()),
+           "vsa_sparse_attn_fwd_nvfp4")
+    return o_out, lse_out
+
+
 def bwd_workspace_bytes(plan: Plan, B: int, H: int, max_k: int) -> int:
     n = ctypes.c_size_t(0)
     _check(lib().vsa_sparse_attn_bwd_workspace(plan.handle, B, H, max_k, ctypes.byref(n)),
@@ -373,13 +421,17 @@ class Forward:
     stage also computes o_compress, and untile_gate replaces untile, so
     __call__(q, k, v, gate=g) returns o_fine + g * o_compress per token
     (g [B,S,H,D], same dtype as q).
+
+    nvfp4=True runs the fine stage with NVFP4 q and k: the tiled q and k are
+    quantised (two launches) and the FP4 attention kernel replaces the 16-bit
+    one; v stays 16-bit.
     """
 
     def __init__(self, plan: Plan, B: int, H: int, topk: int | None, device="cuda", D: int = 128, dtype=None,
-                 gated: bool = False, fused: bool = True):
+                 gated: bool = False, fused: bool = True, nvfp4: bool = False):
         torch = _torch()
         self.plan, self.B, self.H, self.D, self.topk = plan, B, H, D, topk
-        self.gated, self.fused = gated, fused
+        self.gated, self.fused, self.nvfp4 = gated, fused, nvfp4
         t = dict(dtype=dtype or torch.bfloat16, device=device)
         self.qt = torch.empty((B, H, plan.Sp, D), **t)
         self.kt = torch.empty((B, H, plan.Sp, D), **t)
@@ -397,6 +449,12 @@ class Forward:
             self.oc = torch.empty((B, H, plan.NB, D), dtype=torch.float32, device=device)
         if fused:
             self.ws = workspace(B, H, device)
+        if nvfp4:
+            u8 = dict(dtype=torch.uint8, device=device)
+            self.qc = torch.empty((B, H, plan.Sp, D // 2), **u8)
+            self.kc = torch.empty((B, H, plan.Sp, D // 2), **u8)
+            self.qs = torch.empty((B, H, plan.Sp // 128, 64 * D // 8), **u8)
+            self.ks = torch.empty((B, H, plan.Sp // 128, 64 * D // 8), **u8)
 
     def front(self, q, k, v, block_map=None):
         p = self.plan
@@ -427,8 +485,24 @@ class Forward:
             if self.gated:
                 coarse_compress(p, self.qbar, self.kbar, self.vbar, 0, o_out=self.oc)
 
+    def quantize(self):
+        """nvfp4: quantise the tiled q and k (nothing to do otherwise)."""
+        if self.nvfp4:
+            quantize_nvfp4(self.plan, self.qt, self.qc, self.qs)
+            quantize_nvfp4(self.plan, self.kt, self.kc, self.ks)
+
+    def attend(self):
+        """The fine-stage attention kernel alone."""
+        if self.nvfp4:
+            sparse_attn_fwd_nvfp4(self.plan, self.qc, self.qs, self.kc, self.ks, self.vt, self.idx, self.num,
+                                  o_out=self.ot, lse_out=self.lse)
+        else:
+            sparse_attn_fwd(self.plan, self.qt, self.kt, self.vt, self.idx, self.num, o_out=self.ot,
+                            lse_out=self.lse)
+
     def fine(self):
-        sparse_attn_fwd(self.plan, self.qt, self.kt, self.vt, self.idx, self.num, o_out=self.ot, lse_out=self.lse)
+        self.quantize()
+        self.attend()
 
     def back(self, gate=None, out=None):
         out = self.o if out is None else out
@@ -448,9 +522,10 @@ class Forward:
 
     def launches(self, block_map: bool = False) -> int:
         """Kernels one call launches."""
+        quant = 2 if self.nvfp4 else 0  # q and k quantisation
         if self.fused:
-            return 3 + (1 if block_map else 0)  # front (+ map_to_index), attention, untile
-        return 6 + (1 if (self.gated and block_map) else 0)  # 3 tiles, index stage (+compress), attention, untile
+            return 3 + quant + (1 if block_map else 0)  # front (+ map_to_index), attention, untile
+        return 6 + quant + (1 if (self.gated and block_map) else 0)  # 3 tiles, index stage (+compress), attention, untile
 
 
 class HostPipeline:

@@ -1,0 +1,758 @@
+// fp4.cu -- NVFP4 Q and K for the fine stage.
+//
+// FastVideo "Optimizations" page, section "FP4 Flash Attention 4 (Blackwell
+// only)": Q and K are quantised to NVFP4 -- E2M1 values with per-block E4M3
+// scale factors -- while V stays 16-bit.  Block length 16 (consecutive
+// channels of a token) and scale = E4M3(amax / 6) are NVFP4's own definition.
+//
+// Two kernels:
+//
+//   quant_nvfp4_kernel  tiled 16-bit rows -> E2M1 codes + E4M3 scales.  One
+//                       thread per 16-channel block: amax, scale = E4M3 of
+//                       fl32(amax / 6), codes = E2M1 of fl32(x * fl32(1/scale))
+//                       (hardware conversions: nearest, ties to even,
+//                       saturating), scales scattered into the layout the
+//                       tensor core reads (below).  HBM-bound.
+//
+//   attn_fwd_fp4_kernel the block-sparse attention forward with S = Q K^T as
+//                       a block-scaled FP4 product (tcgen05.mma
+//                       kind::mxf4nvf4, 16-channel blocks, E4M3 scales read
+//                       from tensor memory) and O += P V as a 16-bit product
+//                       (P in tensor memory, V in shared memory).
+//
+// Scale layout (the tensor core's): for each (b, h) and each 128-row tile t of
+// the tiled sequence, 1024 bytes; byte kh*512 + (r % 32)*16 + (r / 32)*4 + j
+// holds the scale of row 128t + r, channels 16(4kh + j) .. 16(4kh + j) + 15.
+// One 512-byte half is a 32 x 16-byte matrix that tcgen05.cp.32x128b.warpx4
+// moves into tensor memory, where lane r%32 (of every lane quarter), column
+// r/32, byte j holds the scale the MMA needs for row r and channel block j of
+// a 64-channel product.
+//
+// Attention work item: one (b*h, query block) as in the 16-bit kernel (two
+// 128-row Q tiles for 256-token blocks, one 64-row tile in the top half of a
+// 128-row MMA for 64-token blocks).  Keys are walked in steps of 64 (a quarter
+// of a 256-token block, or one 64-token block): tensor memory holds the two
+// O accumulators (2 x 128 columns) and the scale factors (32 columns), which
+// leaves 64 columns of S per Q tile.
+//
+// Warp roles (384 threads), as in the 16-bit kernel:
+//   warp 0      TMA producer: Q codes + scales once per item; per step the
+//               K codes (64 x 64 B) and the 1 KB of scales of their 128-row
+//               tile (K ring), and V (64 x 128 x 16-bit, V ring)
+//   warp 1      TMEM owner and MMA issuer (tcgen05.cp of scales, FP4 S MMAs,
+//               16-bit PV MMAs)
+//   warps 4-11  two softmax warpgroups, one per Q tile, one row per thread
+//
+// Tensor memory (128 lanes x 512 columns):
+//   [  0, 64) S0 (P0 as 16-bit numerators on [0,32))   [ 64,128) S1 (P1)
+//   [128,256) O0                                       [256,384) O1
+//   [384,400) Q scales: tile i at 384 + 8i, channel half kh at +4kh
+//   [400,416) K scales of the current and next step (8 columns each)
+// Per step u the MMA thread issues PV0(u), S0(u+1), PV1(u), S1(u+1), so one
+// warpgroup's softmax overlaps the other's tensor-core work.
+//
+// Every mbarrier wait is bounded (globaltimer); on expiry the kernel records
+// VSA_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tiles.cuh"
+
+namespace vsa {
+
+namespace {
+
+using namespace tiles;
+
+// ---------------------------------------------------------------------------
+// Conversions
+// ---------------------------------------------------------------------------
+
+// Eight fp32 values -> eight E2M1 codes in one word; value 0 in the low nibble
+// of byte 0.  Round to nearest, ties to even, saturate at +-6.
+__device__ __forceinline__ uint32_t e2m1x8(float x0, float x1, float x2, float x3, float x4, float x5, float x6,
+                                           float x7) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 c0, c1, c2, c3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c3, %8, %7;\n\t"
+      "mov.b32 %0, {c0, c1, c2, c3};\n\t}"
+      : "=r"(r)
+      : "f"(x0), "f"(x1), "f"(x2), "f"(x3), "f"(x4), "f"(x5), "f"(x6), "f"(x7));
+  return r;
+}
+
+// fp32 -> E4M3 bits (nearest, ties to even, saturating at 448).
+__device__ __forceinline__ uint32_t e4m3_of(float x) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(r) : "f"(x), "f"(0.0f));
+  return r & 0xffu;
+}
+
+// Value of non-negative E4M3 bits (exponent bias 7, 3 mantissa bits; step
+// 2^-9 below 2^-6), exact in fp32.
+__device__ __forceinline__ float e4m3_value(uint32_t b) {
+  const uint32_t ex = (b >> 3) & 15u, m = b & 7u;
+  return ex == 0 ? static_cast<float>(m) * 0.001953125f : __uint_as_float(((ex + 120u) << 23) | (m << 20));
+}
+
+// ---------------------------------------------------------------------------
+// Quantisation
+// ---------------------------------------------------------------------------
+
+// One thread per 16-channel block: 8 threads per 128-channel row, 32 rows per
+// 256-thread block.  rows is a multiple of 128 (whole scale tiles).
+template <bool F16>
+__global__ void __launch_bounds__(256) quant_nvfp4_kernel(const uint4* __restrict__ x, uint2* __restrict__ codes,
+                                                          uint32_t* __restrict__ sf, long long rows) {
+  const long long gid = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x;
+  const long long row = gid >> 3;
+  if (row >= rows) return;  // whole warps: rows is a multiple of 4
+  const int b = static_cast<int>(gid & 7);
+  const uint4 w0 = __ldg(x + 2 * gid), w1 = __ldg(x + 2 * gid + 1);
+  const uint32_t wd[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+  float f[16];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    if (F16) {
+      const __half2 h = *reinterpret_cast<const __half2*>(&wd[i]);
+      f[2 * i] = __low2float(h);
+      f[2 * i + 1] = __high2float(h);
+    } else {
+      f[2 * i] = bf16_lo(wd[i]);
+      f[2 * i + 1] = bf16_hi(wd[i]);
+    }
+  }
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
+  const uint32_t sb = e4m3_of(__fdiv_rn(amax, 6.0f));
+  const float s = e4m3_value(sb);
+  const float inv = s == 0.0f ? 0.0f : __frcp_rn(s);
+  float y[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) y[i] = __fmul_rn(f[i], inv);
+  codes[gid] = make_uint2(e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]),
+                          e2m1x8(y[8], y[9], y[10], y[11], y[12], y[13], y[14], y[15]));
+  // the four scales of a channel half (blocks 4kh .. 4kh+3) form one word
+  uint32_t word = sb;
+  word |= __shfl_down_sync(0xffffffffu, sb, 1) << 8;
+  word |= __shfl_down_sync(0xffffffffu, sb, 2) << 16;
+  word |= __shfl_down_sync(0xffffffffu, sb, 3) << 24;
+  if ((b & 3) == 0) {
+    const long long t = row >> 7;
+    const int r = static_cast<int>(row & 127);
+    sf[(t * 1024 + (b >> 2) * 512 + (r & 31) * 16 + (r >> 5) * 4) >> 2] = word;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Attention forward with FP4 Q K^T
+// ---------------------------------------------------------------------------
+
+constexpr int kThreads = 384;
+constexpr int kStages = 4;                        // K ring and V ring, in 64-key steps
+constexpr uint32_t kQTileBytes = 128 * 64;        // 128 rows x 64 B of codes
+constexpr uint32_t kSfTileBytes = 1024;           // scales of a 128-row tile
+constexpr uint32_t kKStepBytes = 64 * 64;         // 64 keys x 64 B of codes
+constexpr uint32_t kVHalfBytes = 64 * 128;        // 64 keys x 64 channels x 2 B
+constexpr uint32_t kVStepBytes = 2 * kVHalfBytes;  // 64 keys x 128 channels
+constexpr uint32_t kSmemQ = 0;
+constexpr uint32_t kSmemQsf = kSmemQ + 2 * kQTileBytes;
+constexpr uint32_t kSmemK = kSmemQsf + 2 * kSfTileBytes;
+constexpr uint32_t kSmemKsf = kSmemK + kStages * kKStepBytes;
+constexpr uint32_t kSmemV = kSmemKsf + kStages * kSfTileBytes;
+constexpr uint32_t kSmemBar = kSmemV + kStages * kVStepBytes;
+constexpr uint32_t kSmemTotal = kSmemBar + 256 + 1024;  // barriers + 1 KB alignment slack
+static_assert(kSmemK % 1024 == 0 && kSmemV % 1024 == 0 && kSmemBar % 1024 == 0, "1 KB-aligned sections");
+constexpr uint32_t kTmS = 0, kTmO = 128, kTmSfa = 384, kTmSfb = 400;
+constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s per wait
+constexpr int kRegsLaunch = 168, kRegsLow = 104, kRegsHigh = 200;
+static_assert(kThreads * kRegsLaunch == 128 * kRegsLow + 256 * kRegsHigh, "register split must match the launch");
+
+// S: E2M1 x E2M1 with UE4M3 block-16 scales, fp32 accumulate, M=128, N=64,
+// both K-major (K = 64 codes per instruction).  Fields: A/B format E2M1 = 1 at
+// bits 7 and 10, N>>3 at 17, scale format UE4M3 = 0 at 23, M>>4 at 24.
+constexpr uint32_t kIdescS = (1u << 7) | (1u << 10) | ((64u >> 3) << 17) | ((128u >> 4) << 24);
+template <bool F16>
+struct IdescPV {
+  static constexpr uint32_t v = F16 ? idesc_f16_f32(128, 128, 0, 1) : idesc_bf16_f32(128, 128, 0, 1);
+};
+
+// Shared-memory descriptor, K-major with 64-byte swizzle (layout type 4),
+// 8-row atoms of 64 B (SBO 512).
+__device__ __forceinline__ uint64_t sdesc_sw64(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(16u >> 4) << 16;
+  d |= static_cast<uint64_t>(512u >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(4) << 61;
+  return d;
+}
+
+// Source of tcgen05.cp.32x128b: 32 rows of 16 B, no swizzle, 8-row core
+// matrices 128 B apart.
+__device__ __forceinline__ uint64_t sdesc_rows16(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(128u >> 4) << 16;
+  d |= static_cast<uint64_t>(128u >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  return d;
+}
+
+// D[tmem] (+)= A[smem] * B[smem] with block scales from tensor memory.
+__device__ __forceinline__ void mma_fp4_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// 32 rows x 128 bits of shared memory -> 4 columns of tensor memory, copied
+// into every lane quarter.
+__device__ __forceinline__ void tmem_cp_32x128_w(uint32_t taddr, uint64_t src_desc) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;\n\t}" ::"r"(taddr),
+      "l"(src_desc)
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_load_w(void* smem_dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n\t}" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+struct Barriers {
+  uint64_t q_full, q_empty;
+  uint64_t k_full[kStages], k_empty[kStages];
+  uint64_t v_full[kStages], v_empty[kStages];
+  uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(Barriers) <= 256, "barrier block too large");
+
+struct Params {
+  const int32_t* idx;
+  const int32_t* num;
+  const uint8_t* q_sf;
+  const uint8_t* k_sf;
+  int max_k;
+  int BH;
+  uint16_t* o;
+  float* lse;
+  unsigned int* status;
+  float scale_log2;
+  Geo g;
+};
+
+__device__ __forceinline__ int item_blocks(const Params& p, int item, bool report) {
+  int c = __ldg(p.num + item);
+  if (c < 0 || c > p.max_k) {
+    if (report) atomicCAS(p.status, 0u, (unsigned)VSA_ERR_BAD_INDEX);
+    c = c < 0 ? 0 : p.max_k;
+  }
+  return c;
+}
+
+__device__ __forceinline__ int item_block_id(const Params& p, int item, int j) {
+  const int kb = __ldg(p.idx + static_cast<long long>(item) * p.max_k + j);
+  return (kb >= 0 && kb < p.g.NB) ? kb : -1;
+}
+
+// 64-key steps of an item with nb selected blocks.
+template <int BS>
+__device__ __forceinline__ int item_steps(int nb) {
+  return BS == 256 ? 4 * nb : nb;
+}
+
+// Step u of an item: selection index, first key row of the step inside its
+// head (kb < 0: block 0 stands in, masked), and which half (0/1) of its
+// 128-row scale tile the step's 64 keys are.
+template <int BS>
+__device__ __forceinline__ void step_keys(const Params& p, int item, int u, int& kb, int& key0, int& half) {
+  const int j = BS == 256 ? (u >> 2) : u;
+  kb = item_block_id(p, item, j);
+  const int kbl = kb < 0 ? 0 : kb;
+  key0 = BS == 256 ? kbl * 256 + (u & 3) * 64 : kbl * 64;
+  half = (key0 >> 6) & 1;
+}
+
+// Validity bits of the 64 keys of a step; returns kTileFull / kTilePartial / kTileEmpty.
+template <int BS>
+__device__ __forceinline__ int step_mask(const Geo& g, int kb, int u, uint32_t& m0, uint32_t& m1) {
+  if (BS == 64) {
+    const int st = block64_mask(g, kb, m0, m1);
+    if (st == kTileFull) m0 = m1 = 0xffffffffu;
+    return st;
+  }
+  uint32_t w[4];
+  const int st = key_tile_mask(g, kb, (u >> 1) & 1, w);
+  if (st == kTileFull) {
+    m0 = m1 = 0xffffffffu;
+    return kTileFull;
+  }
+  if (st == kTileEmpty) {
+    m0 = m1 = 0u;
+    return kTileEmpty;
+  }
+  m0 = (u & 1) ? w[2] : w[0];
+  m1 = (u & 1) ? w[3] : w[1];
+  if ((m0 & m1) == 0xffffffffu) return kTileFull;
+  if ((m0 | m1) == 0u) return kTileEmpty;
+  return kTilePartial;
+}
+
+// Masked columns of one row of S (64 columns) to -inf; uniform branches.
+__device__ __forceinline__ void apply_mask64(uint32_t (&sv)[64], uint32_t m0, uint32_t m1) {
+  const uint32_t mw[2] = {m0, m1};
+#pragma unroll
+  for (int w = 0; w < 2; ++w) {
+    const uint32_t m = mw[w];
+    if (m == 0xffffffffu) continue;
+#pragma unroll
+    for (int c = 0; c < 32; ++c)
+      if (!((m >> c) & 1u)) sv[32 * w + c] = 0xff800000u;
+  }
+}
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Barriers* bars, unsigned int* status) {
+  bool ok = mbar_wait(bar, parity, &bars->abort, status, kTimeoutNs);
+  return __all_sync(0xffffffffu, ok);
+}
+
+template <int BS, bool F16>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem + kSmemQ;
+  uint8_t* sQsf = smem + kSmemQsf;
+  uint8_t* sK = smem + kSmemK;
+  uint8_t* sKsf = smem + kSmemKsf;
+  uint8_t* sV = smem + kSmemV;
+  Barriers* bars = reinterpret_cast<Barriers*>(smem + kSmemBar);
+
+  constexpr int kQTiles = BS == 256 ? 2 : 1;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const Geo& g = p.g;
+  const int total_items = p.BH * g.NB;
+  const long long sf_tiles = g.Sp >> 7;  // 128-row scale tiles per head
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    mbar_init(&bars->q_empty, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->k_empty[s], 1);
+      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->v_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->s_full[i], 1);
+      mbar_init(&bars->p_full[i], 128);
+      mbar_init(&bars->o_full[i], 1);
+      mbar_init(&bars->o_empty[i], 128);
+    }
+    mbar_init(&bars->drain, 1);
+    bars->abort = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp < 4) {
+    regs_dec<kRegsLow>();
+    if (warp == 0) {
+      // ------------------------------------------------------------ producer
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      const uint64_t pol_kv = policy_evict_last();
+      const uint64_t pol_q = policy_evict_first();
+      int kit = 0, vit = 0, qit = 0;
+      for (int item = blockIdx.x; item < total_items; item += gridDim.x) {
+        const int nb = item_blocks(p, item, false);
+        if (nb == 0) continue;
+        const int bh = item / g.NB, qb = item - bh * g.NB;
+        const long long base = static_cast<long long>(bh) * g.Sp;
+        if (!warp_wait(&bars->q_empty, (qit & 1) ^ 1, bars, p.status)) break;
+        mbar_arrive_expect_tx_w(&bars->q_full, kQTiles * (kQTileBytes + kSfTileBytes));
+        const int q0 = qb * BS;  // first query row inside the head
+        for (int i = 0; i < kQTiles; ++i) {
+          tma_load_2d_w(sQ + i * kQTileBytes, &tm_q, 0, static_cast<int>(base + q0 + i * 128), &bars->q_full, pol_q);
+          const long long tile = bh * sf_tiles + ((q0 >> 7) + i);
+          bulk_load_w(sQsf + i * kSfTileBytes, p.q_sf + tile * kSfTileBytes, kSfTileBytes, &bars->q_full);
+        }
+        ++qit;
+        bool stop = false;
+        const int n = item_steps<BS>(nb);
+        for (int u = 0; u < n; ++u) {
+          int kb, key0, half;
+          step_keys<BS>(p, item, u, kb, key0, half);
+          const int sk = kit % kStages;
+          if (!warp_wait(&bars->k_empty[sk], ((kit / kStages) & 1) ^ 1, bars, p.status)) {
+            stop = true;
+            break;
+          }
+          mbar_arrive_expect_tx_w(&bars->k_full[sk], kKStepBytes + kSfTileBytes);
+          tma_load_2d_w(sK + sk * kKStepBytes, &tm_k, 0, static_cast<int>(base + key0), &bars->k_full[sk], pol_kv);
+          bulk_load_w(sKsf + sk * kSfTileBytes, p.k_sf + (bh * sf_tiles + (key0 >> 7)) * kSfTileBytes, kSfTileBytes,
+                      &bars->k_full[sk]);
+          ++kit;
+          const int sv = vit % kStages;
+          if (!warp_wait(&bars->v_empty[sv], ((vit / kStages) & 1) ^ 1, bars, p.status)) {
+            stop = true;
+            break;
+          }
+          mbar_arrive_expect_tx_w(&bars->v_full[sv], kVStepBytes);
+          for (int hf = 0; hf < 2; ++hf)
+            tma_load_2d_w(sV + sv * kVStepBytes + hf * kVHalfBytes, &tm_v, hf * 64, static_cast<int>(base + key0),
+                          &bars->v_full[sv], pol_kv);
+          ++vit;
+        }
+        if (stop) break;
+      }
+      if (qit > 0) mbar_wait_drain(&bars->q_full, (qit - 1) & 1, kTimeoutNs);
+      for (int s = 0; s < kStages; ++s) {
+        if (kit > s) {
+          const int last = kit - 1 - ((kit - 1 - s) % kStages);
+          mbar_wait_drain(&bars->k_full[s], (last / kStages) & 1, kTimeoutNs);
+        }
+        if (vit > s) {
+          const int last = vit - 1 - ((vit - 1 - s) % kStages);
+          mbar_wait_drain(&bars->v_full[s], (last / kStages) & 1, kTimeoutNs);
+        }
+      }
+    } else if (warp == 1) {
+      // ------------------------------------------------------------ MMA issuer
+      const uint64_t dq0 = sdesc_sw64(smem_u32(sQ));
+      const uint64_t dk0 = sdesc_sw64(smem_u32(sK));
+      const uint64_t dv0 = sdesc_sw128(smem_u32(sV), kVHalfBytes, 1024);
+      int kit = 0, vit = 0, qit = 0, steps = 0, items = 0;
+      bool ok = true;
+      auto copy_sfb = [&](int sk) {
+        const uint32_t dst = tmem + kTmSfb + 8 * (kit & 1);
+        tmem_cp_32x128_w(dst, sdesc_rows16(smem_u32(sKsf + sk * kSfTileBytes)));
+        tmem_cp_32x128_w(dst + 4, sdesc_rows16(smem_u32(sKsf + sk * kSfTileBytes + 512)));
+      };
+      // S_i = Q_i K^T for the step held in K stage sk (scales in buffer kit & 1)
+      auto issue_s = [&](int i, int sk, int khalf, uint32_t qshift) {
+        const uint32_t d = tmem + kTmS + 64 * i;
+#pragma unroll
+        for (int kh = 0; kh < 2; ++kh) {
+          const uint64_t a = dq0 + ((i * kQTileBytes + kh * 32) >> 4);
+          const uint64_t b = dk0 + ((sk * kKStepBytes + kh * 32) >> 4);
+          const uint32_t sfa = tmem + kTmSfa + 8 * i + 4 * kh + qshift;
+          const uint32_t sfb = tmem + kTmSfb + 8 * (kit & 1) + 4 * kh + 2 * khalf;
+          mma_fp4_w(d, a, b, kIdescS, sfa, sfb, kh > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int i, int sv, bool acc) {
+        const uint32_t d = tmem + kTmO + 128 * i, pa = tmem + kTmS + 64 * i;
+        const uint64_t b = dv0 + ((sv * kVStepBytes) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ts_w(d, pa + kk * 8, b + kk * (2048 >> 4), IdescPV<F16>::v, (acc || kk > 0) ? 1u : 0u);
+      };
+      for (int item = blockIdx.x; item < total_items && ok; item += gridDim.x) {
+        const int nb = item_blocks(p, item, lane == 0);
+        if (nb == 0) continue;
+        const int qb = item % g.NB;
+        // 64-token blocks: the item's rows are one half of their 128-row scale tile
+        const uint32_t qshift = BS == 64 ? 2u * static_cast<uint32_t>(qb & 1) : 0u;
+        const int n = item_steps<BS>(nb);
+        if (!(ok = warp_wait(&bars->q_full, qit & 1, bars, p.status))) break;
+        ++qit;
+        tc_fence_after();
+        for (int i = 0; i < kQTiles; ++i) {
+          tmem_cp_32x128_w(tmem + kTmSfa + 8 * i, sdesc_rows16(smem_u32(sQsf + i * kSfTileBytes)));
+          tmem_cp_32x128_w(tmem + kTmSfa + 8 * i + 4, sdesc_rows16(smem_u32(sQsf + i * kSfTileBytes + 512)));
+        }
+        int kb, key0, khalf;
+        step_keys<BS>(p, item, 0, kb, key0, khalf);
+        int sk = kit % kStages;
+        if (!(ok = warp_wait(&bars->k_full[sk], (kit / kStages) & 1, bars, p.status))) break;
+        tc_fence_after();
+        copy_sfb(sk);
+        issue_s(0, sk, khalf, qshift);
+        mma_commit_w(&bars->s_full[0]);
+        if (kQTiles == 2) {
+          issue_s(1, sk, khalf, qshift);
+          mma_commit_w(&bars->s_full[1]);
+        }
+        mma_commit_w(&bars->k_empty[sk]);
+        ++kit;
+        for (int u = 0; u < n; ++u) {
+          const int sv = vit % kStages;
+          if (!(ok = warp_wait(&bars->v_full[sv], (vit / kStages) & 1, bars, p.status))) break;
+          if (!(ok = warp_wait(&bars->p_full[0], steps & 1, bars, p.status))) break;
+          if (u == 0 && !(ok = warp_wait(&bars->o_empty[0], (items & 1) ^ 1, bars, p.status))) break;
+          tc_fence_after();
+          issue_pv(0, sv, u > 0);
+          if (u == n - 1) mma_commit_w(&bars->o_full[0]);
+          const bool more = u + 1 < n;
+          sk = kit % kStages;
+          if (more) {
+            step_keys<BS>(p, item, u + 1, kb, key0, khalf);
+            if (!(ok = warp_wait(&bars->k_full[sk], (kit / kStages) & 1, bars, p.status))) break;
+            tc_fence_after();
+            copy_sfb(sk);
+            issue_s(0, sk, khalf, qshift);
+            mma_commit_w(&bars->s_full[0]);
+          }
+          if (kQTiles == 2) {
+            if (!(ok = warp_wait(&bars->p_full[1], steps & 1, bars, p.status))) break;
+            if (u == 0 && !(ok = warp_wait(&bars->o_empty[1], (items & 1) ^ 1, bars, p.status))) break;
+            tc_fence_after();
+            issue_pv(1, sv, u > 0);
+          }
+          mma_commit_w(&bars->v_empty[sv]);
+          ++vit;
+          if (kQTiles == 2 && u == n - 1) mma_commit_w(&bars->o_full[1]);
+          if (more) {
+            if (kQTiles == 2) {
+              issue_s(1, sk, khalf, qshift);
+              mma_commit_w(&bars->s_full[1]);
+            }
+            mma_commit_w(&bars->k_empty[sk]);
+            ++kit;
+          }
+          ++steps;
+        }
+        if (!ok) break;
+        mma_commit_w(&bars->q_empty);
+        ++items;
+      }
+      mma_commit_w(&bars->drain);
+      mbar_wait_drain(&bars->drain, 0, kTimeoutNs);
+    }
+  } else {
+    regs_inc<kRegsHigh>();
+    // ------------------------------------------------------------ softmax + epilogue
+    const int wg = (warp - 4) >> 2;
+    const bool active = kQTiles == 2 || wg == 0;
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_off + kTmS + 64 * wg;
+    const uint32_t tO = tmem + lane_off + kTmO + 128 * wg;
+    const float sl2 = p.scale_log2;
+    int steps = 0, items = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < total_items && ok && active; item += gridDim.x) {
+      const int nb = item_blocks(p, item, false);
+      const int bh = item / g.NB, qb = item - bh * g.NB;
+      const long long row = static_cast<long long>(bh) * g.Sp + static_cast<long long>(qb) * BS + wg * 128 + r;
+      const bool real_row = BS == 256 || r < 64;
+      uint4* orow = reinterpret_cast<uint4*>(p.o + row * 128);
+      if (nb == 0) {
+        if (!real_row) continue;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) orow[c] = make_uint4(0, 0, 0, 0);
+        p.lse[row] = -INFINITY;
+        continue;
+      }
+      const int n = item_steps<BS>(nb);
+      float m_used = -INFINITY, l = 0.0f;
+      for (int u = 0; u < n; ++u) {
+        int kb, key0, khalf;
+        step_keys<BS>(p, item, u, kb, key0, khalf);
+        if (kb < 0 && wg == 0 && r == 0 && (BS == 64 || (u & 3) == 0))
+          atomicCAS(p.status, 0u, (unsigned)VSA_ERR_BAD_INDEX);
+        uint32_t m0, m1;
+        const int mstate = step_mask<BS>(g, kb, u, m0, m1);
+        if (!(ok = warp_wait(&bars->s_full[wg], steps & 1, bars, p.status))) break;
+        tc_fence_after();
+        uint32_t pk[32];
+        float lsum = 0.0f, alpha = 1.0f;
+        bool rescale = false;
+        if (mstate == kTileEmpty) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) pk[j] = 0u;
+        } else {
+          uint32_t sv[64];
+          tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+          tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+          tmem_wait_ld();
+          if (mstate == kTilePartial) apply_mask64(sv, m0, m1);
+          float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < 64; c += 8) {
+            a0 = max3f(a0, __uint_as_float(sv[c + 0]), __uint_as_float(sv[c + 1]));
+            a1 = max3f(a1, __uint_as_float(sv[c + 2]), __uint_as_float(sv[c + 3]));
+            a2 = max3f(a2, __uint_as_float(sv[c + 4]), __uint_as_float(sv[c + 5]));
+            a3 = max3f(a3, __uint_as_float(sv[c + 6]), __uint_as_float(sv[c + 7]));
+          }
+          const float mt = max3f(a0, a1, fmaxf(a2, a3)) * sl2;
+          const bool grow = mt > m_used + 8.0f;
+          rescale = grow && u > 0 && m_used != -INFINITY;
+          alpha = rescale ? ex2_approx(m_used - mt) : 1.0f;
+          if (grow) m_used = mt;
+          const float msub = (m_used == -INFINITY) ? 0.0f : m_used;
+          const uint64_t c2 = f2pack(sl2, sl2), nm2 = f2pack(-msub, -msub);
+          uint64_t acc0 = 0, acc1 = 0, acc2 = 0, acc3 = 0;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const uint64_t x = fma2(u2pack(sv[2 * j], sv[2 * j + 1]), c2, nm2);
+            float xa, xb;
+            f2unpack(x, xa, xb);
+            const float pa = ex2_approx(xa), pb = ex2_approx(xb);
+            pk[j] = pack_half2<F16>(pa, pb);
+            const uint64_t pp = f2pack(pa, pb);
+            switch (j & 3) {
+              case 0: acc0 = add2(acc0, pp); break;
+              case 1: acc1 = add2(acc1, pp); break;
+              case 2: acc2 = add2(acc2, pp); break;
+              default: acc3 = add2(acc3, pp); break;
+            }
+          }
+          float s0, s1, s2, s3, s4, s5, s6, s7;
+          f2unpack(acc0, s0, s1);
+          f2unpack(acc1, s2, s3);
+          f2unpack(acc2, s4, s5);
+          f2unpack(acc3, s6, s7);
+          lsum = ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
+        }
+        l = l * alpha + lsum;
+        tmem_st32(tS + 0, pk);
+        // PV(u-1) has completed: the s_full commit just waited on follows it.
+        if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t ov[32];
+            tmem_ld32(tO + c * 32, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha);
+            tmem_st32(tO + c * 32, ov);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bars->p_full[wg]);
+        ++steps;
+      }
+      if (!ok) break;
+      if (!(ok = warp_wait(&bars->o_full[wg], items & 1, bars, p.status))) break;
+      tc_fence_after();
+      const float inv = l > 0.0f ? 1.0f / l : 0.0f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t ov[32];
+        tmem_ld32(tO + c * 32, ov);
+        tmem_wait_ld();
+        uint4 w[4];
+        uint32_t* wp = reinterpret_cast<uint32_t*>(w);
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          wp[j] = pack_half2<F16>(__uint_as_float(ov[2 * j]) * inv, __uint_as_float(ov[2 * j + 1]) * inv);
+        if (real_row) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) orow[c * 4 + j] = w[j];
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bars->o_empty[wg]);
+      if (real_row) p.lse[row] = l > 0.0f ? (m_used + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+      ++items;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// TMA view of [rows, 64] bytes of E2M1 codes, 64-byte swizzle.
+bool make_tmap_codes(CUtensorMap* tm, const void* base, unsigned long long rows, unsigned box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {64, rows};
+  cuuint64_t strides[1] = {64};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_quant_nvfp4(long long rows, const uint16_t* x, uint8_t* codes, uint8_t* sf, bool f16,
+                               cudaStream_t stream) {
+  if (rows <= 0 || rows % 128 != 0) return cudaErrorInvalidValue;
+  const long long blocks = rows / 32;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  auto kern = f16 ? quant_nvfp4_kernel<true> : quant_nvfp4_kernel<false>;
+  kern<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(reinterpret_cast<const uint4*>(x),
+                                                         reinterpret_cast<uint2*>(codes),
+                                                         reinterpret_cast<uint32_t*>(sf), rows);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_fwd_nvfp4(const Geo& g, const AttnFp4Args& a, cudaStream_t stream) {
+  if (g.bs != 256 && g.bs != 64) return cudaErrorNotSupported;
+  if (g.Sp % 128 != 0) return cudaErrorNotSupported;
+  const unsigned long long rows = static_cast<unsigned long long>(a.BH) * g.Sp;
+  if (rows >= (1ull << 31)) return cudaErrorInvalidValue;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap_codes(&tq, a.q, rows, 128) || !make_tmap_codes(&tk, a.k, rows, 64) ||
+      !make_tmap(&tv, a.v, rows, 64, a.f16))
+    return cudaErrorInvalidValue;
+  Params p;
+  p.idx = a.idx;
+  p.num = a.num;
+  p.q_sf = a.q_sf;
+  p.k_sf = a.k_sf;
+  p.max_k = a.max_k;
+  p.BH = a.BH;
+  p.o = a.o;
+  p.lse = a.lse;
+  p.status = a.status;
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / 11.313708498984761);  // log2(e) / sqrt(128)
+  p.g = g;
+  const long long items = static_cast<long long>(a.BH) * g.NB;
+  const int grid = static_cast<int>(items < a.num_sms ? items : a.num_sms);
+  auto kern = g.bs == 256 ? (a.f16 ? attn_fwd_fp4_kernel<256, true> : attn_fwd_fp4_kernel<256, false>)
+                          : (a.f16 ? attn_fwd_fp4_kernel<64, true> : attn_fwd_fp4_kernel<64, false>);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTotal);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreads, kSmemTotal, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace vsa

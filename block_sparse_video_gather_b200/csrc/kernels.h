@@ -60,6 +60,26 @@ struct AttnArgs {
 };
 cudaError_t launch_attn_fwd(const Geo& g, const AttnArgs& a, cudaStream_t stream);
 
+// fp4.cu: NVFP4 codes + scales of tiled 16-bit rows (rows a multiple of 128),
+// and the fine stage with FP4 Q K^T.
+cudaError_t launch_quant_nvfp4(long long rows, const uint16_t* x, uint8_t* codes, uint8_t* sf, bool f16,
+                               cudaStream_t stream);
+struct AttnFp4Args {
+  const uint8_t *q, *q_sf;  // codes [B,H,Sp,64] bytes, scales (tensor-core layout)
+  const uint8_t *k, *k_sf;
+  const uint16_t* v;        // [B,H,Sp,D] 16-bit
+  const int32_t* idx;
+  const int32_t* num;
+  int max_k;
+  int BH;
+  uint16_t* o;
+  float* lse;
+  unsigned int* status;
+  int num_sms;
+  bool f16;  // v and o are fp16 (else bf16)
+};
+cudaError_t launch_attn_fwd_nvfp4(const Geo& g, const AttnFp4Args& a, cudaStream_t stream);
+
 // attn_bwd.cu
 struct AttnBwdArgs {
   const uint16_t *q, *k, *v, *o, *dO;  // tiled [B,H,Sp,D]

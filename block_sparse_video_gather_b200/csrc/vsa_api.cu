@@ -388,6 +388,52 @@ int vsa_sparse_attn_fwd(vsa_plan_t plan, const uint16_t* q, const uint16_t* k, c
   return vsa_sparse_attn_fwd_ex(plan, VSA_BF16, q, k, v, q2k_idx, q2k_num, max_k, B, H, D, o, lse, stream);
 }
 
+int vsa_quantize_nvfp4(vsa_plan_t plan, vsa_dtype_t dtype, const uint16_t* x_tiled, int B, int H, int D,
+                       uint8_t* codes, uint8_t* scales, vsa_stream_t stream) {
+  if (dtype != VSA_BF16 && dtype != VSA_F16) return VSA_ERR_INVALID_ARG;
+  if (!plan || !aligned16(x_tiled) || !aligned16(codes) || !aligned16(scales)) return VSA_ERR_INVALID_ARG;
+  if (int rc = check_dims(B, H, D)) return rc;
+  const vsa::Geo& g = plan->g;
+  if (g.Sp % 128 != 0) return VSA_ERR_UNSUPPORTED;
+  DeviceState* ds = nullptr;
+  if (int rc = device_state(&ds)) return rc;
+  const long long rows = static_cast<long long>(B) * H * g.Sp;
+  return from_cuda(vsa::launch_quant_nvfp4(rows, x_tiled, codes, scales, dtype == VSA_F16,
+                                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int vsa_sparse_attn_fwd_nvfp4(vsa_plan_t plan, vsa_dtype_t dtype, const uint8_t* q_codes, const uint8_t* q_scales,
+                              const uint8_t* k_codes, const uint8_t* k_scales, const uint16_t* v,
+                              const int32_t* q2k_idx, const int32_t* q2k_num, int max_k, int B, int H, int D,
+                              uint16_t* o, float* lse, vsa_stream_t stream) {
+  if (dtype != VSA_BF16 && dtype != VSA_F16) return VSA_ERR_INVALID_ARG;
+  if (!plan || !aligned16(q_codes) || !aligned16(q_scales) || !aligned16(k_codes) || !aligned16(k_scales) ||
+      !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return VSA_ERR_INVALID_ARG;
+  if (!aligned16(q2k_idx) || !aligned16(q2k_num) || max_k < 1) return VSA_ERR_INVALID_ARG;
+  if (int rc = check_dims(B, H, D)) return rc;
+  const vsa::Geo& g = plan->g;
+  if (g.Sp % 128 != 0) return VSA_ERR_UNSUPPORTED;
+  DeviceState* ds = nullptr;
+  if (int rc = device_state(&ds)) return rc;
+  vsa::AttnFp4Args a;
+  a.q = q_codes;
+  a.q_sf = q_scales;
+  a.k = k_codes;
+  a.k_sf = k_scales;
+  a.v = v;
+  a.idx = q2k_idx;
+  a.num = q2k_num;
+  a.max_k = max_k;
+  a.BH = B * H;
+  a.o = o;
+  a.lse = lse;
+  a.status = ds->status;
+  a.num_sms = ds->num_sms;
+  a.f16 = dtype == VSA_F16;
+  return from_cuda(vsa::launch_attn_fwd_nvfp4(g, a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int vsa_sparse_attn_bwd_workspace(vsa_plan_t plan, int B, int H, int max_k, size_t* bytes) {
   if (!plan || !bytes || B < 1 || H < 1 || max_k < 1) return VSA_ERR_INVALID_ARG;
   *bytes = vsa::attn_bwd_workspace_bytes(plan->g, B * H, max_k);

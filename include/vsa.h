@@ -23,7 +23,8 @@
  * vsa_coarse_compress (or the compression outputs of vsa_tile_coarse) and
  * vsa_untile_gate in place of vsa_untile.  vsa_sparse_attn_bwd gives the
  * fine stage's gradients for a fixed selection.  The _ex calls and
- * vsa_tile_coarse take bf16 or fp16.
+ * vsa_tile_coarse take bf16 or fp16.  For FP4 Q and K, vsa_quantize_nvfp4
+ * (tiled q, tiled k) and vsa_sparse_attn_fwd_nvfp4 replace the fine stage.
  *
  * Conventions shared by every call
  *  - bf16 / fp16 tensors are passed as pointers to their raw 16-bit patterns.
@@ -257,6 +258,42 @@ VSA_API int vsa_sparse_attn_fwd_ex(vsa_plan_t plan, vsa_dtype_t dtype, const uin
                                    const uint16_t *v, const int32_t *q2k_idx, const int32_t *q2k_num,
                                    int max_k, int B, int H, int D, uint16_t *o, float *lse,
                                    vsa_stream_t stream);
+
+/*
+ * NVFP4 quantisation of tiled Q or K (FastVideo "Optimizations" page, section
+ * "FP4 Flash Attention 4 (Blackwell only)": Q and K as NVFP4, E2M1 values with
+ * per-block E4M3 scale factors; block length and scale rule are NVFP4's own).
+ * For every 16-channel block of a row: s = E4M3(fl32(amax / 6)) and each
+ * value's code = E2M1(fl32(x * fl32(1 / s))) (1/s := 0 when s is 0); both
+ * roundings to nearest, ties to even, saturating (448, 6); E2M1 keeps the
+ * sign, zero included.
+ *   x_tiled : tiled [B,H,Sp,D] dtype
+ *   codes   : [B,H,Sp,D/2] bytes, caller-owned; channel 2j in the low nibble
+ *             of byte j, 2j+1 in the high nibble
+ *   scales  : B*H*Sp*D/16 bytes, caller-owned, in the tensor core's layout:
+ *             for each (b, h) and each 128-row tile t of the head's Sp rows,
+ *             1024 bytes; byte kh*512 + (r%32)*16 + (r/32)*4 + j holds the
+ *             scale of row 128t + r, channels 16(4kh + j) .. 16(4kh + j) + 15
+ * Sp must be a multiple of 128 (always for 256-token blocks; an even block
+ * count for 64-token blocks), else VSA_ERR_UNSUPPORTED.
+ */
+VSA_API int vsa_quantize_nvfp4(vsa_plan_t plan, vsa_dtype_t dtype, const uint16_t *x_tiled, int B, int H, int D,
+                               uint8_t *codes, uint8_t *scales, vsa_stream_t stream);
+
+/*
+ * Fine stage with NVFP4 Q and K (same page and section): the attention of
+ * vsa_sparse_attn_fwd_ex computed on the values the codes stand for,
+ * q_i = s_q * e2m1(code), k_j likewise; S = Q K^T runs as a block-scaled FP4
+ * product with fp32 accumulation, P and V stay 16-bit (dtype).
+ *   q_codes, q_scales, k_codes, k_scales : from vsa_quantize_nvfp4
+ *   v, o : tiled [B,H,Sp,D] dtype;  lse: [B,H,Sp] fp32
+ *   q2k_idx, q2k_num, max_k : as in vsa_sparse_attn_fwd
+ * Same error behaviour as vsa_sparse_attn_fwd; Sp must be a multiple of 128.
+ */
+VSA_API int vsa_sparse_attn_fwd_nvfp4(vsa_plan_t plan, vsa_dtype_t dtype, const uint8_t *q_codes,
+                                      const uint8_t *q_scales, const uint8_t *k_codes, const uint8_t *k_scales,
+                                      const uint16_t *v, const int32_t *q2k_idx, const int32_t *q2k_num, int max_k,
+                                      int B, int H, int D, uint16_t *o, float *lse, vsa_stream_t stream);
 
 /*
  * Backward of the fine stage with the selection held fixed (the FastVideo

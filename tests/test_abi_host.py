@@ -27,7 +27,7 @@ def L():
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(vsa_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(vsa_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_and_binding_agree():
@@ -171,6 +171,19 @@ def test_calls_reject_invalid_arguments(L):
     assert L.vsa_untile_gate(h, vsa.VSA_BF16, F, F, M, F, 1, 2, 128, None) == vsa.VSA_ERR_INVALID_ARG
     assert L.vsa_untile_gate(h, vsa.VSA_BF16, F, None, F, F, 1, 2, 128, None) == vsa.VSA_ERR_INVALID_ARG
     assert L.vsa_untile_gate(h, vsa.VSA_F16, F, F, F, F, 1, 2, 96, None) == vsa.VSA_ERR_UNSUPPORTED
+    # NVFP4: dtype, pointers, head size, whole 128-row scale tiles
+    assert L.vsa_quantize_nvfp4(h, 2, F, 1, 2, 128, F, F, None) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_quantize_nvfp4(h, vsa.VSA_BF16, F, 1, 2, 128, F, M, None) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_quantize_nvfp4(None, vsa.VSA_BF16, F, 1, 2, 128, F, F, None) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_quantize_nvfp4(h, vsa.VSA_BF16, F, 1, 2, 64, F, F, None) == vsa.VSA_ERR_UNSUPPORTED
+    assert L.vsa_quantize_nvfp4(odd.handle, vsa.VSA_BF16, F, 1, 2, 128, F, F, None) == vsa.VSA_ERR_UNSUPPORTED
+    f4 = lambda dt, qs, mk, D, plan=h: (plan, dt, F, qs, F, F, F, F, F, mk, 1, 2, D, F, F, None)
+    assert L.vsa_sparse_attn_fwd_nvfp4(*f4(3, F, 4, 128)) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_sparse_attn_fwd_nvfp4(*f4(vsa.VSA_BF16, M, 4, 128)) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_sparse_attn_fwd_nvfp4(*f4(vsa.VSA_BF16, None, 4, 128)) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_sparse_attn_fwd_nvfp4(*f4(vsa.VSA_BF16, F, 0, 128)) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_sparse_attn_fwd_nvfp4(*f4(vsa.VSA_F16, F, 4, 256)) == vsa.VSA_ERR_UNSUPPORTED
+    assert L.vsa_sparse_attn_fwd_nvfp4(*f4(vsa.VSA_BF16, F, 4, 128, odd.handle)) == vsa.VSA_ERR_UNSUPPORTED
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path")
