@@ -137,6 +137,30 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def sync_ranks(pg, device_sync=True):
+    """Every rank reaches this point with its device idle (barrier between two
+    device synchronisations; the barrier alone without a process group)."""
+    if device_sync:
+        import torch
+        torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    if device_sync:
+        import torch
+        torch.cuda.synchronize()
+
+
+def rank_max(x: float, pg, device="cuda") -> float:
+    """The largest x over all ranks (x itself without a process group): each
+    timed figure is the slowest rank's."""
+    if not pg:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
 def dist_setup(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -312,17 +336,10 @@ def run_backward(args, wl, world, rank, local, pg):
         vsa.sparse_attn_bwd(plan, fwd.qt, fwd.kt, fwd.vt, fwd.ot, fwd.lse, do, fwd.idx, fwd.num, dq, dk, dv, ws)
 
     def sync_all():
-        torch.cuda.synchronize()
-        if pg:
-            pg.barrier()
-        torch.cuda.synchronize()
+        sync_ranks(pg)
 
     def max_over_ranks(x: float) -> float:
-        if not pg:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        return float(t.item())
+        return rank_max(x, pg)
 
     for _ in range(args.warmup):
         step()
@@ -511,17 +528,10 @@ def main():
             back_ev[i].record(stream)
 
     def sync_all():
-        torch.cuda.synchronize()
-        if pg:
-            pg.barrier()
-        torch.cuda.synchronize()
+        sync_ranks(pg)
 
     def max_over_ranks(x: float) -> float:
-        if not pg:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        return float(t.item())
+        return rank_max(x, pg)
 
     for _ in range(args.warmup):
         step()
