@@ -1,9 +1,10 @@
 // fp4.cu -- NVFP4 Q and K for the fine stage.
 //
 // FastVideo "Optimizations" page, section "FP4 Flash Attention 4 (Blackwell
-// only)": Q and K are quantised to NVFP4 -- E2M1 values with per-block E4M3
-// scale factors -- while V stays 16-bit.  Block length 16 (consecutive
-// channels of a token) and scale = E4M3(amax / 6) are NVFP4's own definition.
+// only)": Q and K go to NVFP4 (4-bit E2M1 codes, each block of channels
+// sharing one 8-bit E4M3 scale) and V keeps its 16-bit format.  Block length
+// 16 (consecutive channels of a token) and scale = E4M3(amax / 6) are NVFP4's
+// own definition.
 //
 // Two kernels:
 //

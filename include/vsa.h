@@ -261,8 +261,8 @@ VSA_API int vsa_sparse_attn_fwd_ex(vsa_plan_t plan, vsa_dtype_t dtype, const uin
 
 /*
  * NVFP4 quantisation of tiled Q or K (FastVideo "Optimizations" page, section
- * "FP4 Flash Attention 4 (Blackwell only)": Q and K as NVFP4, E2M1 values with
- * per-block E4M3 scale factors; block length and scale rule are NVFP4's own).
+ * "FP4 Flash Attention 4 (Blackwell only)": Q and K as NVFP4: 4-bit E2M1 codes, one
+ * E4M3 scale per block of channels; block length and scale rule are NVFP4's own).
  * For every 16-channel block of a row: s = E4M3(fl32(amax / 6)) and each
  * value's code = E2M1(fl32(x * fl32(1 / s))) (1/s := 0 when s is 0); both
  * roundings to nearest, ties to even, saturating (448, 6); E2M1 keeps the

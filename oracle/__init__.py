@@ -18,7 +18,7 @@ Each step follows the statement cited in the C file's header:
   commit log keeps the grad path separate), in fp64, real query rows only;
 * ``quant_nvfp4``/``dequant_nvfp4``/``attn_rows_nvfp4``: FastVideo
   "Optimizations" page, section "FP4 Flash Attention 4 (Blackwell only)" (Q
-  and K as NVFP4: E2M1 values, per-block E4M3 scales; V 16-bit); block length
+  and K as NVFP4: 4-bit E2M1 codes, one E4M3 scale per block of channels; V 16-bit); block length
   16 and the amax/6 scale are NVFP4's own definition, stated in the C file;
 * ``compress``/``gate_rows``: "FastVideo VSA", section "Checkpoint behavior"
   (learned gate_compress projection) and the FastVideo commit log (the

@@ -603,8 +603,9 @@ int oracle_gate_rows(int n_prefix, int T, int Hg, int Wg, int bt, int bh, int bw
 
 /* ---------------------------------------------------------------------------
  * NVFP4 Q and K.  FastVideo "Optimizations" page, section "FP4 Flash
- * Attention 4 (Blackwell only)": Q and K are quantised to NVFP4 -- E2M1
- * values with per-block E4M3 scale factors -- while V stays 16-bit.  The page
+ * Attention 4 (Blackwell only)": Q and K go to NVFP4 -- 4-bit E2M1
+ * codes, each block of channels sharing one 8-bit E4M3 scale -- and V keeps
+ * its 16-bit format.  The page
  * fixes neither the block length nor how a scale is chosen; the readings
  * taken are NVFP4's own definition:
  *   - a block is 16 consecutive channels of one token;

@@ -2,8 +2,8 @@
 the quantised operands.
 
 Source: FastVideo "Optimizations" page, section "FP4 Flash Attention 4
-(Blackwell only)": Q and K are quantised to NVFP4 (E2M1 values with per-block
-E4M3 scale factors), V stays 16-bit.  Readings (NVFP4's own definition): blocks
+(Blackwell only)": Q and K go to NVFP4 (4-bit E2M1 codes, one E4M3 scale per
+block of channels), V keeps its 16-bit format.  Readings (NVFP4's own definition): blocks
 of 16 consecutive channels, scale = E4M3(fl32(amax / 6)), value codes =
 E2M1(fl32(x * fl32(1 / scale))), both roundings to nearest with ties to an even
 last mantissa bit, capped at the largest finite value, E2M1 keeping the sign.
