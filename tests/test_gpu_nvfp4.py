@@ -233,3 +233,17 @@ def test_full_path_nvfp4_full_size(name):
     o_ref, lse_ref = oracle.attn_rows_nvfp4(ref["g"], qc, qs, kc, ks, ref["vt"], ref["idx"], ref["num"], rows)
     ot_bits = H.from_dev(fwd.ot).reshape(-1, 128)
     H.compare_o_lse(ot_bits[rows], lse.cpu().numpy().reshape(-1)[rows], o_ref, lse_ref, name)
+
+
+@pytest.mark.parametrize("shape,H_,k", [((15, 14, 15, (4, 8, 8), 0), 24, 8), ((31, 22, 40, (4, 8, 8), 0), 2, 64)])
+def test_fp4_attention_many_items_per_cta(shape, H_, k):
+    """More items than CTAs and long selections on a grid with partial blocks:
+    exercises item-to-item hand-offs inside a CTA (every small case above has
+    at most one item per CTA)."""
+    wl = _wl(shape, H_=H_)
+    g = oracle.geometry_of(wl)
+    inp = workloads.make_inputs(wl)
+    qt, kt, vt = (oracle.tile(g, inp[n]) for n in ("q", "k", "v"))
+    idx, num = oracle.topk(oracle.score(oracle.pool(g, qt), oracle.pool(g, kt)), k)
+    rows = _sample_rows(wl, 24, seed=31)
+    _fp4_vs_oracle(wl, qt, kt, vt, idx, num, rows=rows, what=f"many items {shape} H{H_} k{k}")

@@ -257,3 +257,25 @@ def test_full_path_full_size(name):
     ot_bits = H.from_dev(fwd.ot).reshape(-1, 128)
     H.compare_o_lse(ot_bits[rows], lse.cpu().numpy().reshape(-1)[rows], o_ref, lse_ref, name)
     np.testing.assert_array_equal(H.from_dev(o), oracle.untile(ref["g"], H.from_dev(fwd.ot)))
+
+
+@pytest.mark.parametrize("shape,H_,k", [((15, 14, 15, (4, 8, 8), 0), 24, 8), ((31, 22, 40, (4, 8, 8), 0), 2, 64),
+                                        ((5, 6, 7, (4, 4, 4), 100), 24, 6)])
+def test_attention_many_items_per_cta(shape, H_, k):
+    """More items than CTAs and long selections on grids with partial blocks (both
+    block sizes): exercises item-to-item hand-offs inside a CTA."""
+    wl = _wl(shape, H_=H_)
+    g = oracle.geometry_of(wl)
+    inp = H.inputs(wl)
+    qt, kt = oracle.tile(g, inp["q"]), oracle.tile(g, inp["k"])
+    idx, num = oracle.topk(oracle.score(oracle.pool(g, qt), oracle.pool(g, kt)), k)
+    ref = dict(qt=qt, kt=kt, vt=oracle.tile(g, inp["v"]), g=g)
+    rows = _sample_rows(wl, 24, seed=32)
+    plan = vsa.Plan.of(wl)
+    q, kk, v = (H.to_dev(ref[n]) for n in ("qt", "kt", "vt"))
+    o, lse = vsa.sparse_attn_fwd(plan, q, kk, v, torch.from_numpy(idx).cuda(), torch.from_numpy(num).cuda())
+    torch.cuda.synchronize()
+    assert vsa.get_status() == vsa.VSA_OK
+    o_ref, lse_ref = oracle.attn_rows(g, ref["qt"], ref["kt"], ref["vt"], idx, num, rows)
+    H.compare_o_lse(H.from_dev(o).reshape(-1, 128)[rows], lse.cpu().numpy().reshape(-1)[rows], o_ref, lse_ref,
+                    f"many items {shape}")
