@@ -247,3 +247,18 @@ def test_fp4_attention_many_items_per_cta(shape, H_, k):
     idx, num = oracle.topk(oracle.score(oracle.pool(g, qt), oracle.pool(g, kt)), k)
     rows = _sample_rows(wl, 24, seed=31)
     _fp4_vs_oracle(wl, qt, kt, vt, idx, num, rows=rows, what=f"many items {shape} H{H_} k{k}")
+
+
+@pytest.mark.parametrize("shape", [SHAPES[1], SHAPES[5]])
+def test_fp4_attention_batch_of_two(shape):
+    wl = _wl(shape, H_=2, B=2)
+    g = oracle.geometry_of(wl)
+    inp = workloads.make_inputs(wl)
+    qt, kt, vt = (oracle.tile(g, inp[n]) for n in ("q", "k", "v"))
+    rng = np.random.default_rng(34)
+    max_k = min(4, g.NB)
+    num = rng.integers(0, max_k + 1, size=(2, 2, g.NB)).astype(np.int32)
+    idx = np.full((2, 2, g.NB, max_k), -1, dtype=np.int32)
+    for pos in np.ndindex(2, 2, g.NB):
+        idx[pos][:num[pos]] = np.sort(rng.permutation(g.NB)[:num[pos]])
+    _fp4_vs_oracle(wl, qt, kt, vt, idx, num, what=f"B2 {shape}")

@@ -279,3 +279,17 @@ def test_attention_many_items_per_cta(shape, H_, k):
     o_ref, lse_ref = oracle.attn_rows(g, ref["qt"], ref["kt"], ref["vt"], idx, num, rows)
     H.compare_o_lse(H.from_dev(o).reshape(-1, 128)[rows], lse.cpu().numpy().reshape(-1)[rows], o_ref, lse_ref,
                     f"many items {shape}")
+
+
+@pytest.mark.parametrize("shape", [EDGE_SHAPES[1], EDGE_SHAPES[6]])
+def test_attention_batch_of_two(shape):
+    """B = 2: the fine stage indexes (b, h) rows correctly (per-row counts 0..max_k)."""
+    wl = _wl(shape, H_=2, B=2)
+    g = oracle.geometry_of(wl)
+    rng = np.random.default_rng(33)
+    max_k = min(4, g.NB)
+    num = rng.integers(0, max_k + 1, size=(2, 2, g.NB)).astype(np.int32)
+    idx = np.full((2, 2, g.NB, max_k), -1, dtype=np.int32)
+    for pos in np.ndindex(2, 2, g.NB):
+        idx[pos][:num[pos]] = np.sort(rng.permutation(g.NB)[:num[pos]])
+    _attn_vs_oracle(wl, idx, num, what=f"B2 {shape}")
