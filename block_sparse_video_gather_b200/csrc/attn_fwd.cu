@@ -13,7 +13,8 @@
 //
 // Warp roles (384 threads):
 //   warp 0      TMA producer: Q (64 KB per item), K and V tiles (32 KB each)
-//               into a 2-stage ring, completion counted on mbarriers.
+//               into a 3-stage K ring and a 2-stage V ring (224 KB of shared
+//               memory in all), completion counted on mbarriers.
 //   warp 1      TMEM owner (512 columns) and single-thread MMA issuer.
 //   warps 4-7   softmax + epilogue of Q tile 0 (one thread per query row)
 //   warps 8-11  softmax + epilogue of Q tile 1
@@ -50,14 +51,16 @@ namespace {
 using namespace tiles;
 
 constexpr int kThreads = 384;
-constexpr int kStages = 2;
+// K tiles are needed first (by S) and V tiles a softmax later (by PV): the K
+// ring is one stage deeper so its loads start two tile periods ahead.
+constexpr int kStagesK = 3, kStagesV = 2;
 constexpr uint32_t kHalfBytes = 128 * 128;      // 128 rows x 64 bf16 (one 128-B swizzle column)
 constexpr uint32_t kTileBytes = 2 * kHalfBytes;  // 128 rows x 128 bf16
 constexpr uint32_t kQBytes = 2 * kTileBytes;     // two Q tiles
 constexpr uint32_t kSmemQ = 0;
 constexpr uint32_t kSmemK = kSmemQ + kQBytes;
-constexpr uint32_t kSmemV = kSmemK + kStages * kTileBytes;
-constexpr uint32_t kSmemBar = kSmemV + kStages * kTileBytes;
+constexpr uint32_t kSmemV = kSmemK + kStagesK * kTileBytes;
+constexpr uint32_t kSmemBar = kSmemV + kStagesV * kTileBytes;
 constexpr uint32_t kSmemTotal = kSmemBar + 256 + 1024;  // barriers + 1 KB alignment slack
 constexpr uint64_t kTimeoutNs = 2000000000ull;          // 2 s per wait
 // Register split: launched at 168 per thread (384 x 168 = 64512); warpgroup 0
@@ -75,8 +78,8 @@ struct Idesc {
 
 struct Barriers {
   uint64_t q_full, q_empty;
-  uint64_t k_full[kStages], k_empty[kStages];
-  uint64_t v_full[kStages], v_empty[kStages];
+  uint64_t k_full[kStagesK], k_empty[kStagesK];
+  uint64_t v_full[kStagesV], v_empty[kStagesV];
   uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
   uint64_t drain;
   uint32_t tmem_base;
@@ -185,9 +188,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
     mbar_init(&bars->q_empty, 1);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kStagesK; ++s) {
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->k_empty[s], 1);
+    }
+    for (int s = 0; s < kStagesV; ++s) {
       mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->v_empty[s], 1);
     }
@@ -252,8 +257,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             krow0 = static_cast<int>(base + static_cast<long long>(ka < 0 ? 0 : ka) * 64);
             krow1 = static_cast<int>(base + static_cast<long long>(kb < 0 ? 0 : kb) * 64);
           }
-          const int sk = kit % kStages;
-          if (!warp_wait(&bars->k_empty[sk], ((kit / kStages) & 1) ^ 1, bars, p.status)) {
+          const int sk = kit % kStagesK;
+          if (!warp_wait(&bars->k_empty[sk], ((kit / kStagesK) & 1) ^ 1, bars, p.status)) {
             stop = true;
             break;
           }
@@ -264,8 +269,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (BS == 64) tma_load_2d_w(dst + kHalfBytes / 2, &tm_k, hf * 64, krow1, &bars->k_full[sk], pol_kv);
           }
           ++kit;
-          const int sv = vit % kStages;
-          if (!warp_wait(&bars->v_empty[sv], ((vit / kStages) & 1) ^ 1, bars, p.status)) {
+          const int sv = vit % kStagesV;
+          if (!warp_wait(&bars->v_empty[sv], ((vit / kStagesV) & 1) ^ 1, bars, p.status)) {
             stop = true;
             break;
           }
@@ -281,16 +286,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // Drain: every issued copy must land before the CTA's shared memory is released.
       if (qit > 0) mbar_wait_drain(&bars->q_full, (qit - 1) & 1, kTimeoutNs);
-      for (int s = 0; s < kStages; ++s) {
+      for (int s = 0; s < kStagesK; ++s)
         if (kit > s) {
-          const int last = kit - 1 - ((kit - 1 - s) % kStages);
-          mbar_wait_drain(&bars->k_full[s], (last / kStages) & 1, kTimeoutNs);
+          const int last = kit - 1 - ((kit - 1 - s) % kStagesK);
+          mbar_wait_drain(&bars->k_full[s], (last / kStagesK) & 1, kTimeoutNs);
         }
+      for (int s = 0; s < kStagesV; ++s)
         if (vit > s) {
-          const int last = vit - 1 - ((vit - 1 - s) % kStages);
-          mbar_wait_drain(&bars->v_full[s], (last / kStages) & 1, kTimeoutNs);
+          const int last = vit - 1 - ((vit - 1 - s) % kStagesV);
+          mbar_wait_drain(&bars->v_full[s], (last / kStagesV) & 1, kTimeoutNs);
         }
-      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -327,8 +332,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = warp_wait(&bars->q_full, qit & 1, bars, p.status))) break;
         ++qit;
         tc_fence_after();
-        int sk = kit % kStages;
-        if (!(ok = warp_wait(&bars->k_full[sk], (kit / kStages) & 1, bars, p.status))) break;
+        int sk = kit % kStagesK;
+        if (!(ok = warp_wait(&bars->k_full[sk], (kit / kStagesK) & 1, bars, p.status))) break;
         tc_fence_after();
         issue_s(0, sk);
         mma_commit_w(&bars->s_full[0]);
@@ -339,8 +344,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit_w(&bars->k_empty[sk]);
         ++kit;
         for (int t = 0; t < n; ++t) {
-          const int sv = vit % kStages;
-          if (!(ok = warp_wait(&bars->v_full[sv], (vit / kStages) & 1, bars, p.status))) break;
+          const int sv = vit % kStagesV;
+          if (!(ok = warp_wait(&bars->v_full[sv], (vit / kStagesV) & 1, bars, p.status))) break;
           if (!(ok = warp_wait(&bars->p_full[0], tiles & 1, bars, p.status))) break;
           if (t == 0 && !(ok = warp_wait(&bars->o_empty[0], (items & 1) ^ 1, bars, p.status)))
             break;
@@ -348,9 +353,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           issue_pv(0, sv, t > 0);
           if (t == n - 1) mma_commit_w(&bars->o_full[0]);
           const bool more = t + 1 < n;
-          sk = kit % kStages;
+          sk = kit % kStagesK;
           if (more) {
-            if (!(ok = warp_wait(&bars->k_full[sk], (kit / kStages) & 1, bars, p.status))) break;
+            if (!(ok = warp_wait(&bars->k_full[sk], (kit / kStagesK) & 1, bars, p.status))) break;
             tc_fence_after();
             issue_s(0, sk);
             mma_commit_w(&bars->s_full[0]);
