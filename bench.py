@@ -652,9 +652,7 @@ def main():
                 "front_end": "separate launches" if args.unfused else "one launch (tile + coarse)",
             },
             "roofline": {
-                "bound": "tensor",
-                "kernel": (("attn_fwd_fp4_wide_kernel" if wl.block_tokens == 256 else "attn_fwd_fp4_kernel")
-                           if args.nvfp4 else "attn_fwd_kernel"),
+                "bound": "tensor", "kernel": "attn_fwd_fp4_kernel" if args.nvfp4 else "attn_fwd_kernel",
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "peak_source": peak_source,
                 "traffic": traffic,

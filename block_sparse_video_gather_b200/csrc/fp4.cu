@@ -29,31 +29,22 @@
 // r/32, byte j holds the scale the MMA needs for row r and channel block j of
 // a 64-channel product.
 //
-// Attention work item: one (b*h, query block) as in the 16-bit kernel, with
-// one kernel per block size:
-//
-//   attn_fwd_fp4_wide_kernel  256-token blocks (two 128-row Q tiles).  Keys in
-//                       128-row tiles and the 16-bit kernel's tensor-memory
-//                       map (S0, S1, O0, O1: all 512 columns); the scale
-//                       factors of each S product are parked in the other Q
-//                       tile's S columns while those hold nothing live.
-//   attn_fwd_fp4_kernel 64-token blocks (one 64-row Q tile in the top half of
-//                       a 128-row MMA).  Keys in 64-key steps, one selected
-//                       block each; tensor memory:
-//                         [  0, 64) S (P as 16-bit numerators on [0,32))
-//                         [128,256) O
-//                         [384,392) Q scales, channel half kh at +4kh
-//                         [400,416) K scales of the current and next step
+// Attention work item: one (b*h, query block) as in the 16-bit kernel (two
+// 128-row Q tiles for 256-token blocks, one 64-row tile in the top half of a
+// 128-row MMA for 64-token blocks), keys in 128-row tiles (half a 256-token
+// block, or two 64-token blocks), the same tensor-memory map (S0, S1, O0, O1:
+// all 512 columns) with the scale factors of each S product parked in the
+// other Q tile's S columns while those hold nothing live (details below).
 //
 // Warp roles (384 threads), as in the 16-bit kernel:
-//   warp 0      TMA producer: Q codes + scales once per item; per key step
-//               the K codes and the 1 KB of scales of their 128-row tile
-//               (K ring), and V (V ring)
+//   warp 0      TMA producer: Q codes + scales once per item; per key tile
+//               the K codes and the 1 KB scale tiles they belong to (K ring),
+//               and V (V ring)
 //   warp 1      TMEM owner and MMA issuer (tcgen05.cp of scales, FP4 S MMAs,
 //               16-bit PV MMAs)
-//   warps 4-11  softmax warpgroups, one per Q tile, one row per thread
-// With two Q tiles the MMA thread issues PV0(t), S0(t+1), PV1(t), S1(t+1) per
-// key tile, so one warpgroup's softmax overlaps the other's tensor-core work.
+//   warps 4-11  two softmax warpgroups, one per Q tile, one row per thread
+// Per key tile t the MMA thread issues PV0(t), S0(t+1), PV1(t), S1(t+1), so
+// one warpgroup's softmax overlaps the other's tensor-core work.
 //
 // Every mbarrier wait is bounded (globaltimer); on expiry the kernel records
 // VSA_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
@@ -157,31 +148,50 @@ __global__ void __launch_bounds__(256) quant_nvfp4_kernel(const uint4* __restric
 // ---------------------------------------------------------------------------
 // Attention forward with FP4 Q K^T
 // ---------------------------------------------------------------------------
+//
+// The 16-bit kernel's work item, warp roles, pipeline and tensor memory map:
+//   [  0,128) S0 (P0 on [0,64))     [128,256) S1 (P1 on [128,192))
+//   [256,384) O0                    [384,512) O1
+// Keys in 128-row tiles: half a 256-token block, or two selected 64-token
+// blocks (the second absent when the count is odd).  The scale factors of a
+// block-scaled product have no columns of their own.  Those of S0 = Q0 K^T
+// are copied to [192,216) (the Q tile's at +0, the key tile's at +8), those of
+// S1 to [64,80): columns of the other tile's S that hold nothing live between
+// the moment that tile's softmax has loaded its S (P only takes the first 64
+// columns) and the issue of its next S product.  The softmax warpgroups
+// signal the load (s_read); the MMA thread waits for it, copies the scales
+// (tcgen05.cp, ordered before the MMA that reads them) and issues the product.
+// With 64-token blocks there is one Q tile (its 64 rows in the top half of the
+// 128-row MMA) and S1 is never written, so no wait is needed; each block of a
+// key tile is its own N = 64 product, because its scales are one half of a
+// 128-row scale tile (two of the four columns the tensor core reads).
 
 constexpr int kThreads = 384;
-constexpr int kStages = 4;                        // K ring and V ring, in 64-key steps
-constexpr uint32_t kQTileBytes = 128 * 64;        // 128 rows x 64 B of codes
-constexpr uint32_t kSfTileBytes = 1024;           // scales of a 128-row tile
-constexpr uint32_t kKStepBytes = 64 * 64;         // 64 keys x 64 B of codes
-constexpr uint32_t kVHalfBytes = 64 * 128;        // 64 keys x 64 channels x 2 B
-constexpr uint32_t kVStepBytes = 2 * kVHalfBytes;  // 64 keys x 128 channels
+constexpr int kStagesK = 4, kStagesV = 3;
+constexpr uint32_t kQTileBytes = 128 * 64;       // 128 rows x 64 B of codes
+constexpr uint32_t kSfTileBytes = 1024;          // scales of a 128-row tile
+constexpr uint32_t kKTileBytes = 128 * 64;       // 128 keys x 64 B of codes
+constexpr uint32_t kKSfBytes = 2 * kSfTileBytes;  // a key tile's scale tiles (two for two 64-token blocks)
+constexpr uint32_t kVHalfBytes = 128 * 128;      // 128 keys x 64 channels x 2 B
+constexpr uint32_t kVTileBytes = 2 * kVHalfBytes;
 constexpr uint32_t kSmemQ = 0;
 constexpr uint32_t kSmemQsf = kSmemQ + 2 * kQTileBytes;
 constexpr uint32_t kSmemK = kSmemQsf + 2 * kSfTileBytes;
-constexpr uint32_t kSmemKsf = kSmemK + kStages * kKStepBytes;
-constexpr uint32_t kSmemV = kSmemKsf + kStages * kSfTileBytes;
-constexpr uint32_t kSmemBar = kSmemV + kStages * kVStepBytes;
+constexpr uint32_t kSmemKsf = kSmemK + kStagesK * kKTileBytes;
+constexpr uint32_t kSmemV = kSmemKsf + kStagesK * kKSfBytes;
+constexpr uint32_t kSmemBar = kSmemV + kStagesV * kVTileBytes;
 constexpr uint32_t kSmemTotal = kSmemBar + 256 + 1024;  // barriers + 1 KB alignment slack
 static_assert(kSmemK % 1024 == 0 && kSmemV % 1024 == 0 && kSmemBar % 1024 == 0, "1 KB-aligned sections");
-constexpr uint32_t kTmS = 0, kTmO = 128, kTmSfa = 384, kTmSfb = 400;
+constexpr uint32_t kTmO = 256;
 constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s per wait
 constexpr int kRegsLaunch = 168, kRegsLow = 104, kRegsHigh = 200;
 static_assert(kThreads * kRegsLaunch == 128 * kRegsLow + 256 * kRegsHigh, "register split must match the launch");
 
-// S: E2M1 x E2M1 with UE4M3 block-16 scales, fp32 accumulate, M=128, N=64,
-// both K-major (K = 64 codes per instruction).  Fields: A/B format E2M1 = 1 at
-// bits 7 and 10, N>>3 at 17, scale format UE4M3 = 0 at 23, M>>4 at 24.
-constexpr uint32_t kIdescS = (1u << 7) | (1u << 10) | ((64u >> 3) << 17) | ((128u >> 4) << 24);
+// S: E2M1 x E2M1 with UE4M3 block-16 scales, fp32 accumulate, M = 128, both
+// K-major (K = 64 codes per instruction).  Fields: A/B format E2M1 = 1 at bits
+// 7 and 10, N>>3 at 17, scale format UE4M3 = 0 at 23, M>>4 at 24.
+constexpr uint32_t idesc_s(uint32_t n) { return (1u << 7) | (1u << 10) | ((n >> 3) << 17) | ((128u >> 4) << 24); }
+
 template <bool F16>
 struct IdescPV {
   static constexpr uint32_t v = F16 ? idesc_f16_f32(128, 128, 0, 1) : idesc_bf16_f32(128, 128, 0, 1);
@@ -246,9 +256,9 @@ __device__ __forceinline__ void bulk_load_w(void* smem_dst, const void* src, uin
 
 struct Barriers {
   uint64_t q_full, q_empty;
-  uint64_t k_full[kStages], k_empty[kStages];
-  uint64_t v_full[kStages], v_empty[kStages];
-  uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
+  uint64_t k_full[kStagesK], k_empty[kStagesK];
+  uint64_t v_full[kStagesV], v_empty[kStagesV];
+  uint64_t s_full[2], s_read[2], p_full[2], o_full[2], o_empty[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -283,422 +293,39 @@ __device__ __forceinline__ int item_block_id(const Params& p, int item, int j) {
   return (kb >= 0 && kb < p.g.NB) ? kb : -1;
 }
 
-// Step u of an item (one selected 64-token block): its block id, the first
-// key row of the step inside its head (kb < 0: block 0 stands in, masked), and
-// which half (0/1) of its 128-row scale tile the block is.
-__device__ __forceinline__ void step_keys(const Params& p, int item, int u, int& kb, int& key0, int& half) {
-  kb = item_block_id(p, item, u);
-  const int kbl = kb < 0 ? 0 : kb;
-  key0 = kbl * 64;
-  half = kbl & 1;
+
+// 128-key tiles of an item with nb selected blocks.
+template <int BS>
+__device__ __forceinline__ int item_tiles(int nb) {
+  return BS == 256 ? 2 * nb : (nb + 1) / 2;
 }
 
-// Validity bits of the 64 keys of a step; returns kTileFull / kTilePartial / kTileEmpty.
-__device__ __forceinline__ int step_mask(const Geo& g, int kb, uint32_t& m0, uint32_t& m1) {
-  const int st = block64_mask(g, kb, m0, m1);
-  if (st == kTileFull) m0 = m1 = 0xffffffffu;
-  return st;
-}
-
-// Masked columns of one row of S (64 columns) to -inf; uniform branches.
-__device__ __forceinline__ void apply_mask64(uint32_t (&sv)[64], uint32_t m0, uint32_t m1) {
-  const uint32_t mw[2] = {m0, m1};
-#pragma unroll
-  for (int w = 0; w < 2; ++w) {
-    const uint32_t m = mw[w];
-    if (m == 0xffffffffu) continue;
-#pragma unroll
-    for (int c = 0; c < 32; ++c)
-      if (!((m >> c) & 1u)) sv[32 * w + c] = 0xff800000u;
-  }
-}
-
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Barriers* bars, unsigned int* status) {
-  bool ok = mbar_wait(bar, parity, &bars->abort, status, kTimeoutNs);
-  return __all_sync(0xffffffffu, ok);
-}
-
-template <bool F16>
-__global__ void __launch_bounds__(kThreads, 1)
-    attn_fwd_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ Params p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem + kSmemQ;
-  uint8_t* sQsf = smem + kSmemQsf;
-  uint8_t* sK = smem + kSmemK;
-  uint8_t* sKsf = smem + kSmemKsf;
-  uint8_t* sV = smem + kSmemV;
-  Barriers* bars = reinterpret_cast<Barriers*>(smem + kSmemBar);
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const Geo& g = p.g;
-  const int total_items = p.BH * g.NB;
-  const long long sf_tiles = g.Sp >> 7;  // 128-row scale tiles per head
-
-  if (threadIdx.x == 0) {
-    mbar_init(&bars->q_full, 1);
-    mbar_init(&bars->q_empty, 1);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bars->k_full[s], 1);
-      mbar_init(&bars->k_empty[s], 1);
-      mbar_init(&bars->v_full[s], 1);
-      mbar_init(&bars->v_empty[s], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars->s_full[i], 1);
-      mbar_init(&bars->p_full[i], 128);
-      mbar_init(&bars->o_full[i], 1);
-      mbar_init(&bars->o_empty[i], 128);
-    }
-    mbar_init(&bars->drain, 1);
-    bars->abort = 0;
-    fence_barrier_init();
-    fence_proxy_async_smem();
-  }
-  if (warp == 1) {
-    tmem_alloc(&bars->tmem_base, 512);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = bars->tmem_base;
-
-  if (warp < 4) {
-    regs_dec<kRegsLow>();
-    if (warp == 0) {
-      // ------------------------------------------------------------ producer
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-      const uint64_t pol_kv = policy_evict_last();
-      const uint64_t pol_q = policy_evict_first();
-      int kit = 0, vit = 0, qit = 0;
-      for (int item = blockIdx.x; item < total_items; item += gridDim.x) {
-        const int nb = item_blocks(p, item, false);
-        if (nb == 0) continue;
-        const int bh = item / g.NB, qb = item - bh * g.NB;
-        const long long base = static_cast<long long>(bh) * g.Sp;
-        if (!warp_wait(&bars->q_empty, (qit & 1) ^ 1, bars, p.status)) break;
-        mbar_arrive_expect_tx_w(&bars->q_full, kQTileBytes + kSfTileBytes);
-        // the block's 64 rows are the top of a 128-row box, its scales half of a scale tile
-        const int q0 = qb * 64;  // first query row inside the head
-        tma_load_2d_w(sQ, &tm_q, 0, static_cast<int>(base + q0), &bars->q_full, pol_q);
-        bulk_load_w(sQsf, p.q_sf + (bh * sf_tiles + (q0 >> 7)) * kSfTileBytes, kSfTileBytes, &bars->q_full);
-        ++qit;
-        bool stop = false;
-        for (int u = 0; u < nb; ++u) {
-          int kb, key0, half;
-          step_keys(p, item, u, kb, key0, half);
-          const int sk = kit % kStages;
-          if (!warp_wait(&bars->k_empty[sk], ((kit / kStages) & 1) ^ 1, bars, p.status)) {
-            stop = true;
-            break;
-          }
-          mbar_arrive_expect_tx_w(&bars->k_full[sk], kKStepBytes + kSfTileBytes);
-          tma_load_2d_w(sK + sk * kKStepBytes, &tm_k, 0, static_cast<int>(base + key0), &bars->k_full[sk], pol_kv);
-          bulk_load_w(sKsf + sk * kSfTileBytes, p.k_sf + (bh * sf_tiles + (key0 >> 7)) * kSfTileBytes, kSfTileBytes,
-                      &bars->k_full[sk]);
-          ++kit;
-          const int sv = vit % kStages;
-          if (!warp_wait(&bars->v_empty[sv], ((vit / kStages) & 1) ^ 1, bars, p.status)) {
-            stop = true;
-            break;
-          }
-          mbar_arrive_expect_tx_w(&bars->v_full[sv], kVStepBytes);
-          for (int hf = 0; hf < 2; ++hf)
-            tma_load_2d_w(sV + sv * kVStepBytes + hf * kVHalfBytes, &tm_v, hf * 64, static_cast<int>(base + key0),
-                          &bars->v_full[sv], pol_kv);
-          ++vit;
-        }
-        if (stop) break;
-      }
-      if (qit > 0) mbar_wait_drain(&bars->q_full, (qit - 1) & 1, kTimeoutNs);
-      for (int s = 0; s < kStages; ++s) {
-        if (kit > s) {
-          const int last = kit - 1 - ((kit - 1 - s) % kStages);
-          mbar_wait_drain(&bars->k_full[s], (last / kStages) & 1, kTimeoutNs);
-        }
-        if (vit > s) {
-          const int last = vit - 1 - ((vit - 1 - s) % kStages);
-          mbar_wait_drain(&bars->v_full[s], (last / kStages) & 1, kTimeoutNs);
-        }
-      }
-    } else if (warp == 1) {
-      // ------------------------------------------------------------ MMA issuer
-      const uint64_t dq0 = sdesc_sw64(smem_u32(sQ));
-      const uint64_t dk0 = sdesc_sw64(smem_u32(sK));
-      const uint64_t dv0 = sdesc_sw128(smem_u32(sV), kVHalfBytes, 1024);
-      int kit = 0, vit = 0, qit = 0, steps = 0, items = 0;
-      bool ok = true;
-      auto copy_sfb = [&](int sk) {
-        const uint32_t dst = tmem + kTmSfb + 8 * (kit & 1);
-        tmem_cp_32x128_w(dst, sdesc_rows16(smem_u32(sKsf + sk * kSfTileBytes)));
-        tmem_cp_32x128_w(dst + 4, sdesc_rows16(smem_u32(sKsf + sk * kSfTileBytes + 512)));
-      };
-      // S = Q K^T for the step held in K stage sk (scales in buffer kit & 1).
-      // The item's 64 query rows and the step's 64 keys are each one half of
-      // their 128-row scale tile: qshift and khalf pick the half's 2 columns.
-      auto issue_s = [&](int sk, int khalf, uint32_t qshift) {
-        const uint32_t d = tmem + kTmS;
-#pragma unroll
-        for (int kh = 0; kh < 2; ++kh) {
-          const uint64_t a = dq0 + ((kh * 32) >> 4);
-          const uint64_t b = dk0 + ((sk * kKStepBytes + kh * 32) >> 4);
-          const uint32_t sfa = tmem + kTmSfa + 4 * kh + qshift;
-          const uint32_t sfb = tmem + kTmSfb + 8 * (kit & 1) + 4 * kh + 2 * khalf;
-          mma_fp4_w(d, a, b, kIdescS, sfa, sfb, kh > 0 ? 1u : 0u);
-        }
-      };
-      auto issue_pv = [&](int sv, bool acc) {
-        const uint32_t d = tmem + kTmO, pa = tmem + kTmS;
-        const uint64_t b = dv0 + ((sv * kVStepBytes) >> 4);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ts_w(d, pa + kk * 8, b + kk * (2048 >> 4), IdescPV<F16>::v, (acc || kk > 0) ? 1u : 0u);
-      };
-      for (int item = blockIdx.x; item < total_items && ok; item += gridDim.x) {
-        const int nb = item_blocks(p, item, lane == 0);
-        if (nb == 0) continue;
-        const int qb = item % g.NB;
-        const uint32_t qshift = 2u * static_cast<uint32_t>(qb & 1);
-        if (!(ok = warp_wait(&bars->q_full, qit & 1, bars, p.status))) break;
-        ++qit;
-        tc_fence_after();
-        tmem_cp_32x128_w(tmem + kTmSfa, sdesc_rows16(smem_u32(sQsf)));
-        tmem_cp_32x128_w(tmem + kTmSfa + 4, sdesc_rows16(smem_u32(sQsf + 512)));
-        int kb, key0, khalf;
-        step_keys(p, item, 0, kb, key0, khalf);
-        int sk = kit % kStages;
-        if (!(ok = warp_wait(&bars->k_full[sk], (kit / kStages) & 1, bars, p.status))) break;
-        tc_fence_after();
-        copy_sfb(sk);
-        issue_s(sk, khalf, qshift);
-        mma_commit_w(&bars->s_full[0]);
-        mma_commit_w(&bars->k_empty[sk]);
-        ++kit;
-        for (int u = 0; u < nb; ++u) {
-          const int sv = vit % kStages;
-          if (!(ok = warp_wait(&bars->v_full[sv], (vit / kStages) & 1, bars, p.status))) break;
-          if (!(ok = warp_wait(&bars->p_full[0], steps & 1, bars, p.status))) break;
-          if (u == 0 && !(ok = warp_wait(&bars->o_empty[0], (items & 1) ^ 1, bars, p.status))) break;
-          tc_fence_after();
-          issue_pv(sv, u > 0);
-          if (u == nb - 1) mma_commit_w(&bars->o_full[0]);
-          mma_commit_w(&bars->v_empty[sv]);
-          ++vit;
-          if (u + 1 < nb) {
-            step_keys(p, item, u + 1, kb, key0, khalf);
-            sk = kit % kStages;
-            if (!(ok = warp_wait(&bars->k_full[sk], (kit / kStages) & 1, bars, p.status))) break;
-            tc_fence_after();
-            copy_sfb(sk);
-            issue_s(sk, khalf, qshift);
-            mma_commit_w(&bars->s_full[0]);
-            mma_commit_w(&bars->k_empty[sk]);
-            ++kit;
-          }
-          ++steps;
-        }
-        if (!ok) break;
-        mma_commit_w(&bars->q_empty);
-        ++items;
-      }
-      mma_commit_w(&bars->drain);
-      mbar_wait_drain(&bars->drain, 0, kTimeoutNs);
-    }
+// Blocks of key tile t: 256-token blocks, half t&1 of block kb_a (kb_b unused);
+// 64-token blocks, blocks kb_a and kb_b (-1 when the count is odd and t is
+// the last tile).  Unusable ids come back as -1.
+template <int BS>
+__device__ __forceinline__ void tile_blocks(const Params& p, int item, int nb, int t, int& kb_a, int& kb_b) {
+  if (BS == 256) {
+    kb_a = item_block_id(p, item, t >> 1);
+    kb_b = -1;
   } else {
-    regs_inc<kRegsHigh>();
-    // ------------------------------------------------------------ softmax + epilogue
-    // One query tile per item, held by the first warpgroup in the top 64 rows
-    // of its 128-row MMA tile; the second warpgroup idles.
-    const int wg = (warp - 4) >> 2;
-    const bool active = wg == 0;
-    const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t tS = tmem + lane_off + kTmS;
-    const uint32_t tO = tmem + lane_off + kTmO;
-    const float sl2 = p.scale_log2;
-    int steps = 0, items = 0;
-    bool ok = true;
-    for (int item = blockIdx.x; item < total_items && ok && active; item += gridDim.x) {
-      const int nb = item_blocks(p, item, false);
-      const int bh = item / g.NB, qb = item - bh * g.NB;
-      const long long row = static_cast<long long>(bh) * g.Sp + static_cast<long long>(qb) * 64 + r;
-      const bool real_row = r < 64;
-      uint4* orow = reinterpret_cast<uint4*>(p.o + row * 128);
-      if (nb == 0) {
-        if (!real_row) continue;
-#pragma unroll
-        for (int c = 0; c < 16; ++c) orow[c] = make_uint4(0, 0, 0, 0);
-        p.lse[row] = -INFINITY;
-        continue;
-      }
-      float m_used = -INFINITY, l = 0.0f;
-      for (int u = 0; u < nb; ++u) {
-        int kb, key0, khalf;
-        step_keys(p, item, u, kb, key0, khalf);
-        if (kb < 0 && r == 0) atomicCAS(p.status, 0u, (unsigned)VSA_ERR_BAD_INDEX);
-        uint32_t m0, m1;
-        const int mstate = step_mask(g, kb, m0, m1);
-        if (!(ok = warp_wait(&bars->s_full[0], steps & 1, bars, p.status))) break;
-        tc_fence_after();
-        uint32_t pk[32];
-        float lsum = 0.0f, alpha = 1.0f;
-        bool rescale = false;
-        if (mstate == kTileEmpty) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) pk[j] = 0u;
-        } else {
-          uint32_t sv[64];
-          tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-          tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-          tmem_wait_ld();
-          if (mstate == kTilePartial) apply_mask64(sv, m0, m1);
-          float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
-#pragma unroll
-          for (int c = 0; c < 64; c += 8) {
-            a0 = max3f(a0, __uint_as_float(sv[c + 0]), __uint_as_float(sv[c + 1]));
-            a1 = max3f(a1, __uint_as_float(sv[c + 2]), __uint_as_float(sv[c + 3]));
-            a2 = max3f(a2, __uint_as_float(sv[c + 4]), __uint_as_float(sv[c + 5]));
-            a3 = max3f(a3, __uint_as_float(sv[c + 6]), __uint_as_float(sv[c + 7]));
-          }
-          const float mt = max3f(a0, a1, fmaxf(a2, a3)) * sl2;
-          const bool grow = mt > m_used + 8.0f;
-          rescale = grow && u > 0 && m_used != -INFINITY;
-          alpha = rescale ? ex2_approx(m_used - mt) : 1.0f;
-          if (grow) m_used = mt;
-          const float msub = (m_used == -INFINITY) ? 0.0f : m_used;
-          const uint64_t c2 = f2pack(sl2, sl2), nm2 = f2pack(-msub, -msub);
-          uint64_t acc0 = 0, acc1 = 0, acc2 = 0, acc3 = 0;
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const uint64_t x = fma2(u2pack(sv[2 * j], sv[2 * j + 1]), c2, nm2);
-            float xa, xb;
-            f2unpack(x, xa, xb);
-            const float pa = ex2_approx(xa), pb = ex2_approx(xb);
-            pk[j] = pack_half2<F16>(pa, pb);
-            const uint64_t pp = f2pack(pa, pb);
-            switch (j & 3) {
-              case 0: acc0 = add2(acc0, pp); break;
-              case 1: acc1 = add2(acc1, pp); break;
-              case 2: acc2 = add2(acc2, pp); break;
-              default: acc3 = add2(acc3, pp); break;
-            }
-          }
-          float s0, s1, s2, s3, s4, s5, s6, s7;
-          f2unpack(acc0, s0, s1);
-          f2unpack(acc1, s2, s3);
-          f2unpack(acc2, s4, s5);
-          f2unpack(acc3, s6, s7);
-          lsum = ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
-        }
-        l = l * alpha + lsum;
-        tmem_st32(tS + 0, pk);
-        // PV(u-1) has completed: the s_full commit just waited on follows it.
-        if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t ov[32];
-            tmem_ld32(tO + c * 32, ov);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha);
-            tmem_st32(tO + c * 32, ov);
-          }
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&bars->p_full[0]);
-        ++steps;
-      }
-      if (!ok) break;
-      if (!(ok = warp_wait(&bars->o_full[0], items & 1, bars, p.status))) break;
-      tc_fence_after();
-      const float inv = l > 0.0f ? 1.0f / l : 0.0f;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t ov[32];
-        tmem_ld32(tO + c * 32, ov);
-        tmem_wait_ld();
-        uint4 w[4];
-        uint32_t* wp = reinterpret_cast<uint32_t*>(w);
-#pragma unroll
-        for (int j = 0; j < 16; ++j)
-          wp[j] = pack_half2<F16>(__uint_as_float(ov[2 * j]) * inv, __uint_as_float(ov[2 * j + 1]) * inv);
-        if (real_row) {
-#pragma unroll
-          for (int j = 0; j < 4; ++j) orow[c * 4 + j] = w[j];
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(&bars->o_empty[0]);
-      if (real_row) p.lse[row] = l > 0.0f ? (m_used + __log2f(l)) * 0.69314718055994531f : -INFINITY;
-      ++items;
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    __syncwarp();
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    kb_a = item_block_id(p, item, 2 * t);
+    kb_b = 2 * t + 1 < nb ? item_block_id(p, item, 2 * t + 1) : -1;
   }
 }
 
-// ---------------------------------------------------------------------------
-// Attention forward with FP4 Q K^T, 256-token blocks: 128-key steps
-// ---------------------------------------------------------------------------
-//
-// The same work item, warp roles and pipeline as the 16-bit kernel, with the
-// same tensor memory map:
-//   [  0,128) S0 (P0 on [0,64))     [128,256) S1 (P1 on [128,192))
-//   [256,384) O0                    [384,512) O1
-// The scale factors of a block-scaled product have no columns of their own.
-// Those of S0 = Q0 K^T are copied to [192,208) (Q0's at +0, the key tile's at
-// +8), those of S1 to [64,80): columns of the other tile's S that hold nothing
-// live between the moment that tile's softmax has loaded its S (P only takes
-// the first 64 columns) and the issue of its next S product.  The softmax
-// warpgroups signal the load (s_read); the MMA thread waits for it, copies
-// the scales (tcgen05.cp, ordered before the MMA that reads them) and issues
-// the product.
-namespace wide {
-
-constexpr int kStagesK = 4, kStagesV = 3;
-constexpr uint32_t kQTileBytes = 128 * 64;    // 128 rows x 64 B of codes
-constexpr uint32_t kSfTileBytes = 1024;       // scales of a 128-row tile
-constexpr uint32_t kKTileBytes = 128 * 64;    // 128 keys x 64 B of codes
-constexpr uint32_t kVHalfBytes = 128 * 128;   // 128 keys x 64 channels x 2 B
-constexpr uint32_t kVTileBytes = 2 * kVHalfBytes;
-constexpr uint32_t kSmemQ = 0;
-constexpr uint32_t kSmemQsf = kSmemQ + 2 * kQTileBytes;
-constexpr uint32_t kSmemK = kSmemQsf + 2 * kSfTileBytes;
-constexpr uint32_t kSmemKsf = kSmemK + kStagesK * kKTileBytes;
-constexpr uint32_t kSmemV = kSmemKsf + kStagesK * kSfTileBytes;
-constexpr uint32_t kSmemBar = kSmemV + kStagesV * kVTileBytes;
-constexpr uint32_t kSmemTotal = kSmemBar + 256 + 1024;  // barriers + 1 KB alignment slack
-static_assert(kSmemK % 1024 == 0 && kSmemV % 1024 == 0 && kSmemBar % 1024 == 0, "1 KB-aligned sections");
-constexpr uint32_t kTmO = 256;
-// M = 128, N = 128, K = 64 codes per instruction; fields as for kIdescS.
-constexpr uint32_t kIdescS = (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
-
-// First scale column of the product S_i (inside the other tile's S).
-__device__ __forceinline__ uint32_t sf_col(int i) { return i == 0 ? 192u : 64u; }
-
-struct Barriers {
-  uint64_t q_full, q_empty;
-  uint64_t k_full[kStagesK], k_empty[kStagesK];
-  uint64_t v_full[kStagesV], v_empty[kStagesV];
-  uint64_t s_full[2], s_read[2], p_full[2], o_full[2], o_empty[2];
-  uint64_t drain;
-  uint32_t tmem_base;
-  int abort;
-};
-static_assert(sizeof(Barriers) <= 256, "barrier block too large");
+// Validity bits of the 128 key columns of tile t; kTileFull / kTilePartial / kTileEmpty.
+template <int BS>
+__device__ __forceinline__ int tile_mask(const Geo& g, int kb_a, int kb_b, int t, uint32_t (&mw)[4]) {
+  if (BS == 256) return key_tile_mask(g, kb_a, t & 1, mw);
+  const int sa = block64_mask(g, kb_a, mw[0], mw[1]);
+  const int sb = block64_mask(g, kb_b, mw[2], mw[3]);
+  if (sa == kTileFull && sb == kTileFull) return kTileFull;
+  if (sa == kTileEmpty && sb == kTileEmpty) return kTileEmpty;
+  if (sa == kTileFull) mw[0] = mw[1] = 0xffffffffu;
+  if (sb == kTileFull) mw[2] = mw[3] = 0xffffffffu;
+  return kTilePartial;
+}
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Barriers* bars, unsigned int* status) {
   bool ok = mbar_wait(bar, parity, &bars->abort, status, kTimeoutNs);
@@ -717,10 +344,23 @@ __device__ __forceinline__ void apply_mask128(uint32_t (&sv)[128], const uint32_
   }
 }
 
-template <bool F16>
+// Scale-tile halves of the two blocks of 64-token key tile t (bit h for block
+// h; an absent or unusable block stands in as block 0).
+template <int BS>
+__device__ __forceinline__ uint32_t tile_halves(const Params& p, int item, int nb, int t) {
+  if (BS == 256) return 0u;
+  int kb_a, kb_b;
+  tile_blocks<BS>(p, item, nb, t, kb_a, kb_b);
+  return (static_cast<uint32_t>(kb_a < 0 ? 0 : kb_a) & 1u) | ((static_cast<uint32_t>(kb_b < 0 ? 0 : kb_b) & 1u) << 1);
+}
+
+// First scale column of the product S_i (inside the other tile's S).
+__device__ __forceinline__ uint32_t sf_col(int i) { return i == 0 ? 192u : 64u; }
+
+template <int BS, bool F16>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_fwd_fp4_wide_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ Params p) {
+    attn_fwd_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + kSmemQ;
@@ -730,6 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sV = smem + kSmemV;
   Barriers* bars = reinterpret_cast<Barriers*>(smem + kSmemBar);
 
+  constexpr int kQTiles = BS == 256 ? 2 : 1;  // 128-row query tiles per item
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const Geo& g = p.g;
@@ -784,29 +425,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int bh = item / g.NB, qb = item - bh * g.NB;
         const long long base = static_cast<long long>(bh) * g.Sp;
         if (!warp_wait(&bars->q_empty, (qit & 1) ^ 1, bars, p.status)) break;
-        mbar_arrive_expect_tx_w(&bars->q_full, 2 * (kQTileBytes + kSfTileBytes));
-        const int q0 = qb * 256;  // first query row inside the head
-        for (int i = 0; i < 2; ++i) {
+        mbar_arrive_expect_tx_w(&bars->q_full, kQTiles * (kQTileBytes + kSfTileBytes));
+        // a 64-token block's rows are the top of a 128-row box, its scales half of a scale tile
+        const int q0 = qb * BS;  // first query row inside the head
+        for (int i = 0; i < kQTiles; ++i) {
           tma_load_2d_w(sQ + i * kQTileBytes, &tm_q, 0, static_cast<int>(base + q0 + i * 128), &bars->q_full, pol_q);
           const long long tile = bh * sf_tiles + ((q0 >> 7) + i);
           bulk_load_w(sQsf + i * kSfTileBytes, p.q_sf + tile * kSfTileBytes, kSfTileBytes, &bars->q_full);
         }
         ++qit;
         bool stop = false;
-        const int n = 2 * nb;
+        const int n = item_tiles<BS>(nb);
         for (int t = 0; t < n; ++t) {
-          // an unusable block id loads block 0 (finite data, masked by the softmax)
-          const int kb = item_block_id(p, item, t >> 1);
-          const int key0 = (kb < 0 ? 0 : kb) * 256 + (t & 1) * 128;
+          // Key rows of this tile: one 128-row box, or two 64-row boxes.
+          // Unusable or absent blocks load block 0 -- finite data, masked out
+          // by the softmax -- so that no stale shared memory reaches P V.
+          int kb_a, kb_b;
+          tile_blocks<BS>(p, item, nb, t, kb_a, kb_b);
+          const int row_a = BS == 256 ? (kb_a < 0 ? 0 : kb_a) * 256 + (t & 1) * 128 : (kb_a < 0 ? 0 : kb_a) * 64;
+          const int row_b = (kb_b < 0 ? 0 : kb_b) * 64;
           const int sk = kit % kStagesK;
           if (!warp_wait(&bars->k_empty[sk], ((kit / kStagesK) & 1) ^ 1, bars, p.status)) {
             stop = true;
             break;
           }
-          mbar_arrive_expect_tx_w(&bars->k_full[sk], kKTileBytes + kSfTileBytes);
-          tma_load_2d_w(sK + sk * kKTileBytes, &tm_k, 0, static_cast<int>(base + key0), &bars->k_full[sk], pol_kv);
-          bulk_load_w(sKsf + sk * kSfTileBytes, p.k_sf + (bh * sf_tiles + (key0 >> 7)) * kSfTileBytes, kSfTileBytes,
-                      &bars->k_full[sk]);
+          uint8_t* kdst = sK + sk * kKTileBytes;
+          uint8_t* sfdst = sKsf + sk * kKSfBytes;
+          mbar_arrive_expect_tx_w(&bars->k_full[sk], kKTileBytes + (BS == 256 ? 1u : 2u) * kSfTileBytes);
+          tma_load_2d_w(kdst, &tm_k, 0, static_cast<int>(base + row_a), &bars->k_full[sk], pol_kv);
+          bulk_load_w(sfdst, p.k_sf + (bh * sf_tiles + (row_a >> 7)) * kSfTileBytes, kSfTileBytes, &bars->k_full[sk]);
+          if (BS == 64) {
+            tma_load_2d_w(kdst + kKTileBytes / 2, &tm_k, 0, static_cast<int>(base + row_b), &bars->k_full[sk], pol_kv);
+            bulk_load_w(sfdst + kSfTileBytes, p.k_sf + (bh * sf_tiles + (row_b >> 7)) * kSfTileBytes, kSfTileBytes,
+                        &bars->k_full[sk]);
+          }
           ++kit;
           const int sv = vit % kStagesV;
           if (!warp_wait(&bars->v_empty[sv], ((vit / kStagesV) & 1) ^ 1, bars, p.status)) {
@@ -814,9 +466,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           mbar_arrive_expect_tx_w(&bars->v_full[sv], kVTileBytes);
-          for (int hf = 0; hf < 2; ++hf)
-            tma_load_2d_w(sV + sv * kVTileBytes + hf * kVHalfBytes, &tm_v, hf * 64, static_cast<int>(base + key0),
-                          &bars->v_full[sv], pol_kv);
+          for (int hf = 0; hf < 2; ++hf) {
+            uint8_t* vdst = sV + sv * kVTileBytes + hf * kVHalfBytes;
+            tma_load_2d_w(vdst, &tm_v, hf * 64, static_cast<int>(base + row_a), &bars->v_full[sv], pol_kv);
+            if (BS == 64)
+              tma_load_2d_w(vdst + kVHalfBytes / 2, &tm_v, hf * 64, static_cast<int>(base + row_b), &bars->v_full[sv],
+                            pol_kv);
+          }
           ++vit;
         }
         if (stop) break;
@@ -841,24 +497,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       int kit = 0, vit = 0, qit = 0, tiles = 0, items = 0;
       int sn0 = 0, sn1 = 0;  // S products issued per Q tile
       bool ok = true;
-      // S_i = Q_i K^T for the key tile in K stage sk.  Its scales go into the
+      // S_i = Q_i K^T for key tile t in K stage sk.  Its scales go into the
       // other tile's S columns, free once that tile's softmax has loaded its
-      // latest S.
-      auto issue_s = [&](int i, int sk) -> bool {
+      // latest S (with one Q tile that S is never written).
+      // khalf: bit h = which half of its scale tile block h of a 64-token key tile is.
+      auto issue_s = [&](int i, int sk, uint32_t khalf, uint32_t qshift) -> bool {
         const int j = 1 - i, nj = i == 0 ? sn1 : sn0;
         if (nj > 0 && !warp_wait(&bars->s_read[j], (nj - 1) & 1, bars, p.status)) return false;
         tc_fence_after();
         const uint32_t sf = tmem + sf_col(i);
-        tmem_cp_32x128_w(sf + 0, sdesc_rows16(smem_u32(sQsf + i * kSfTileBytes)));
-        tmem_cp_32x128_w(sf + 4, sdesc_rows16(smem_u32(sQsf + i * kSfTileBytes + 512)));
-        tmem_cp_32x128_w(sf + 8, sdesc_rows16(smem_u32(sKsf + sk * kSfTileBytes)));
-        tmem_cp_32x128_w(sf + 12, sdesc_rows16(smem_u32(sKsf + sk * kSfTileBytes + 512)));
+        const uint8_t* qsf = sQsf + i * kSfTileBytes;
+        const uint8_t* ksf = sKsf + sk * kKSfBytes;
+        tmem_cp_32x128_w(sf + 0, sdesc_rows16(smem_u32(qsf)));
+        tmem_cp_32x128_w(sf + 4, sdesc_rows16(smem_u32(qsf + 512)));
+        tmem_cp_32x128_w(sf + 8, sdesc_rows16(smem_u32(ksf)));
+        tmem_cp_32x128_w(sf + 12, sdesc_rows16(smem_u32(ksf + 512)));
         const uint32_t d = tmem + 128 * i;
+        if (BS == 256) {
 #pragma unroll
-        for (int kh = 0; kh < 2; ++kh) {
-          const uint64_t a = dq0 + ((i * kQTileBytes + kh * 32) >> 4);
-          const uint64_t b = dk0 + ((sk * kKTileBytes + kh * 32) >> 4);
-          mma_fp4_w(d, a, b, kIdescS, sf + 4 * kh, sf + 8 + 4 * kh, kh > 0 ? 1u : 0u);
+          for (int kh = 0; kh < 2; ++kh) {
+            const uint64_t a = dq0 + ((i * kQTileBytes + kh * 32) >> 4);
+            const uint64_t b = dk0 + ((sk * kKTileBytes + kh * 32) >> 4);
+            mma_fp4_w(d, a, b, idesc_s(128), sf + 4 * kh, sf + 8 + 4 * kh, kh > 0 ? 1u : 0u);
+          }
+        } else {
+          // one N = 64 product per block; a block's scales are the half
+          // (kb & 1) of its scale tile, two columns in
+          tmem_cp_32x128_w(sf + 16, sdesc_rows16(smem_u32(ksf + kSfTileBytes)));
+          tmem_cp_32x128_w(sf + 20, sdesc_rows16(smem_u32(ksf + kSfTileBytes + 512)));
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int kh = 0; kh < 2; ++kh) {
+              const uint64_t a = dq0 + ((kh * 32) >> 4);
+              const uint64_t b = dk0 + ((sk * kKTileBytes + h * (kKTileBytes / 2) + kh * 32) >> 4);
+              mma_fp4_w(d + 64 * h, a, b, idesc_s(64), sf + 4 * kh + qshift, sf + 8 + 8 * h + 4 * kh + 2 * ((khalf >> h) & 1u),
+                        kh > 0 ? 1u : 0u);
+            }
         }
         if (i == 0) ++sn0; else ++sn1;
         return true;
@@ -873,17 +548,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int item = blockIdx.x; item < total_items && ok; item += gridDim.x) {
         const int nb = item_blocks(p, item, lane == 0);
         if (nb == 0) continue;
-        const int n = 2 * nb;
+        const int n = item_tiles<BS>(nb);
+        // 64-token blocks: the item's rows are one half of their 128-row scale tile
+        const uint32_t qshift = BS == 64 ? 2u * static_cast<uint32_t>((item % g.NB) & 1) : 0u;
         if (!(ok = warp_wait(&bars->q_full, qit & 1, bars, p.status))) break;
         ++qit;
         tc_fence_after();
         int sk = kit % kStagesK;
         if (!(ok = warp_wait(&bars->k_full[sk], (kit / kStagesK) & 1, bars, p.status))) break;
         tc_fence_after();
-        if (!(ok = issue_s(0, sk))) break;
+        uint32_t khalf = tile_halves<BS>(p, item, nb, 0);
+        if (!(ok = issue_s(0, sk, khalf, qshift))) break;
         mma_commit_w(&bars->s_full[0]);
-        if (!(ok = issue_s(1, sk))) break;
-        mma_commit_w(&bars->s_full[1]);
+        if (kQTiles == 2) {
+          if (!(ok = issue_s(1, sk, khalf, qshift))) break;
+          mma_commit_w(&bars->s_full[1]);
+        }
         mma_commit_w(&bars->k_empty[sk]);
         ++kit;
         for (int t = 0; t < n; ++t) {
@@ -897,21 +577,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool more = t + 1 < n;
           sk = kit % kStagesK;
           if (more) {
+            khalf = tile_halves<BS>(p, item, nb, t + 1);
             if (!(ok = warp_wait(&bars->k_full[sk], (kit / kStagesK) & 1, bars, p.status))) break;
             tc_fence_after();
-            if (!(ok = issue_s(0, sk))) break;
+            if (!(ok = issue_s(0, sk, khalf, qshift))) break;
             mma_commit_w(&bars->s_full[0]);
           }
-          if (!(ok = warp_wait(&bars->p_full[1], tiles & 1, bars, p.status))) break;
-          if (t == 0 && !(ok = warp_wait(&bars->o_empty[1], (items & 1) ^ 1, bars, p.status))) break;
-          tc_fence_after();
-          issue_pv(1, sv, t > 0);
+          if (kQTiles == 2) {
+            if (!(ok = warp_wait(&bars->p_full[1], tiles & 1, bars, p.status))) break;
+            if (t == 0 && !(ok = warp_wait(&bars->o_empty[1], (items & 1) ^ 1, bars, p.status))) break;
+            tc_fence_after();
+            issue_pv(1, sv, t > 0);
+          }
           mma_commit_w(&bars->v_empty[sv]);
           ++vit;
-          if (t == n - 1) mma_commit_w(&bars->o_full[1]);
+          if (kQTiles == 2 && t == n - 1) mma_commit_w(&bars->o_full[1]);
           if (more) {
-            if (!(ok = issue_s(1, sk))) break;
-            mma_commit_w(&bars->s_full[1]);
+            if (kQTiles == 2) {
+              if (!(ok = issue_s(1, sk, khalf, qshift))) break;
+              mma_commit_w(&bars->s_full[1]);
+            }
             mma_commit_w(&bars->k_empty[sk]);
             ++kit;
           }
@@ -929,6 +614,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_inc<kRegsHigh>();
     // ------------------------------------------------------------ softmax + epilogue
     const int wg = (warp - 4) >> 2;  // Q tile
+    // 64-token blocks: one query tile per item, held by the first warpgroup
+    // in the top 64 rows of its 128-row MMA tile; the second warpgroup idles.
+    const bool active = kQTiles == 2 || wg == 0;
     const int quarter = warp & 3;    // TMEM lane quarter of this warp
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
@@ -937,24 +625,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float sl2 = p.scale_log2;
     int tiles = 0, items = 0;
     bool ok = true;
-    for (int item = blockIdx.x; item < total_items && ok; item += gridDim.x) {
+    for (int item = blockIdx.x; item < total_items && ok && active; item += gridDim.x) {
       const int nb = item_blocks(p, item, false);
       const int bh = item / g.NB, qb = item - bh * g.NB;
-      const long long row = static_cast<long long>(bh) * g.Sp + static_cast<long long>(qb) * 256 + wg * 128 + r;
+      const long long row = static_cast<long long>(bh) * g.Sp + static_cast<long long>(qb) * BS + wg * 128 + r;
+      const bool real_row = BS == 256 || r < 64;
       uint4* orow = reinterpret_cast<uint4*>(p.o + row * 128);
       if (nb == 0) {
+        if (!real_row) continue;
 #pragma unroll
         for (int c = 0; c < 16; ++c) orow[c] = make_uint4(0, 0, 0, 0);
         p.lse[row] = -INFINITY;
         continue;
       }
-      const int n = 2 * nb;
+      const int n = item_tiles<BS>(nb);
       float m_used = -INFINITY, l = 0.0f;
       for (int t = 0; t < n; ++t) {
-        const int kb = item_block_id(p, item, t >> 1);
-        if (kb < 0 && wg == 0 && r == 0 && (t & 1) == 0) atomicCAS(p.status, 0u, (unsigned)VSA_ERR_BAD_INDEX);
+        int kb_a, kb_b;
+        tile_blocks<BS>(p, item, nb, t, kb_a, kb_b);
+        if (wg == 0 && r == 0) {
+          const bool bad = BS == 256 ? ((t & 1) == 0 && kb_a < 0) : (kb_a < 0 || (2 * t + 1 < nb && kb_b < 0));
+          if (bad) atomicCAS(p.status, 0u, (unsigned)VSA_ERR_BAD_INDEX);
+        }
         uint32_t mw[4];
-        const int mstate = key_tile_mask(g, kb, t & 1, mw);
+        const int mstate = tile_mask<BS>(g, kb_a, kb_b, t, mw);
         if (!(ok = warp_wait(&bars->s_full[wg], tiles & 1, bars, p.status))) break;
         tc_fence_after();
         uint32_t pk[64];
@@ -1050,12 +744,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int j = 0; j < 16; ++j)
           wp[j] = pack_half2<F16>(__uint_as_float(ov[2 * j]) * inv, __uint_as_float(ov[2 * j + 1]) * inv);
+        if (real_row) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) orow[c * 4 + j] = w[j];
+          for (int j = 0; j < 4; ++j) orow[c * 4 + j] = w[j];
+        }
       }
       tc_fence_before();
       mbar_arrive(&bars->o_empty[wg]);
-      p.lse[row] = l > 0.0f ? (m_used + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+      if (real_row) p.lse[row] = l > 0.0f ? (m_used + __log2f(l)) * 0.69314718055994531f : -INFINITY;
       ++items;
     }
   }
@@ -1069,7 +765,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-}  // namespace wide
 
 // TMA view of [rows, 64] bytes of E2M1 codes, 64-byte swizzle.
 bool make_tmap_codes(CUtensorMap* tm, const void* base, unsigned long long rows, unsigned box_rows) {
@@ -1104,7 +799,7 @@ cudaError_t launch_attn_fwd_nvfp4(const Geo& g, const AttnFp4Args& a, cudaStream
   if (g.Sp % 128 != 0) return cudaErrorNotSupported;
   const unsigned long long rows = static_cast<unsigned long long>(a.BH) * g.Sp;
   if (rows >= (1ull << 31)) return cudaErrorInvalidValue;
-  // 256-token blocks walk keys in 128-row tiles, 64-token blocks in 64-row steps
+  // key tiles: one 128-row box (256-token blocks) or two 64-row boxes (64-token blocks)
   const unsigned kv_box = g.bs == 256 ? 128 : 64;
   CUtensorMap tq, tk, tv;
   if (!make_tmap_codes(&tq, a.q, rows, 128) || !make_tmap_codes(&tk, a.k, rows, kv_box) ||
@@ -1124,14 +819,8 @@ cudaError_t launch_attn_fwd_nvfp4(const Geo& g, const AttnFp4Args& a, cudaStream
   p.g = g;
   const long long items = static_cast<long long>(a.BH) * g.NB;
   const int grid = static_cast<int>(items < a.num_sms ? items : a.num_sms);
-  if (g.bs == 256) {
-    auto kern = a.f16 ? wide::attn_fwd_fp4_wide_kernel<true> : wide::attn_fwd_fp4_wide_kernel<false>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, wide::kSmemTotal);
-    if (e != cudaSuccess) return e;
-    kern<<<grid, kThreads, wide::kSmemTotal, stream>>>(tq, tk, tv, p);
-    return cudaGetLastError();
-  }
-  auto kern = a.f16 ? attn_fwd_fp4_kernel<true> : attn_fwd_fp4_kernel<false>;
+  auto kern = g.bs == 256 ? (a.f16 ? attn_fwd_fp4_kernel<256, true> : attn_fwd_fp4_kernel<256, false>)
+                          : (a.f16 ? attn_fwd_fp4_kernel<64, true> : attn_fwd_fp4_kernel<64, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTotal);
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, kSmemTotal, stream>>>(tq, tk, tv, p);

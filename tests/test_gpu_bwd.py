@@ -190,11 +190,12 @@ def test_bwd_full_size_tile64():
                                    atol=2e-2 * np.abs(dov[h][rows_h]).sum(axis=0).max())
 
 
-def test_bwd_full_size_fastwan():
-    """The benchmark workload: dq on sampled rows against the oracle; dk and dv
-    through identities that hold at any size: sum over keys of dk is 0 and sum
-    of dv is the sum of do over rows with a non-empty selection."""
-    wl = workloads.WORKLOADS["fastwan"]
+@pytest.mark.parametrize("name", ["fastwan", "wan81", "long"])
+def test_bwd_full_size(name):
+    """The top-k workloads at full size: dq on sampled rows against the oracle;
+    dk and dv through identities that hold at any size: sum over keys of dk is 0
+    and sum of dv is the sum of do over rows with a non-empty selection."""
+    wl = workloads.WORKLOADS[name]
     g, qt, kt, vt, do, idx, num = _problem(wl, "bf16", None, seed=11)
     dq, dk, dv = _gpu_bwd(wl, "bf16", qt, kt, vt, do, idx, num)
     real = np.flatnonzero(H.real_rows(wl))
@@ -203,7 +204,7 @@ def test_bwd_full_size_fastwan():
                                                                  real[:2], real[-2:]]))
                            for bh in range(wl.H)])
     ref = oracle.attn_bwd_q_rows(g, qt, kt, vt, do, idx, num, rows)
-    _check("fastwan dq rows", _vals(dq, "bf16").reshape(-1, 128)[rows], ref)
+    _check(f"{name} dq rows", _vals(dq, "bf16").reshape(-1, 128)[rows], ref)
     realm = H.real_rows(wl)
     dkv = _vals(dk, "bf16")[0][:, realm]
     dvv = _vals(dv, "bf16")[0][:, realm]
@@ -211,6 +212,6 @@ def test_bwd_full_size_fastwan():
     for h in range(wl.H):
         s = dkv[h].sum(axis=0)
         assert np.abs(s).max() <= 2e-2 * np.abs(dkv[h]).sum(axis=0).max(), h
-        # every fastwan row has topk > 0 selections
+        # top-k workloads give every row topk > 0 selections
         np.testing.assert_allclose(dvv[h].sum(axis=0), dov[h].sum(axis=0), rtol=0,
                                    atol=2e-2 * np.abs(dov[h]).sum(axis=0).max())

@@ -44,7 +44,7 @@ def test_fp16_tile_pool_bit_exact(shape):
     np.testing.assert_array_equal(_host16(vsa.untile(plan, xt)), x)
 
 
-@pytest.mark.parametrize("name", ["tiny", "wan81"])
+@pytest.mark.parametrize("name", ["tiny", "wan81", "fastwan", "long"])
 def test_fp16_full_path(name):
     wl = workloads.WORKLOADS[name]
     g = oracle.geometry_of(wl)

@@ -213,7 +213,7 @@ def _sample_rows(wl, n_per_head, seed):
     return np.concatenate(rows)
 
 
-@pytest.mark.parametrize("name", ["fastwan", "wan81", "tile64"])
+@pytest.mark.parametrize("name", ["fastwan", "wan81", "tile64", "long"])
 def test_full_path_nvfp4_full_size(name):
     """Forward(nvfp4=True) at full size: the quantised q, k bit-exact, o/lse on
     sampled real rows against the oracle's NVFP4 attention."""
