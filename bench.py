@@ -260,7 +260,7 @@ def cpu_baseline_sample(wl, seconds_hint=20.0, nvfp4=False):
     n = 256
     t_attn, done = 0.0, 0
     while t_attn < seconds_hint * 0.5 and done < total_rows:
-        rows = np.sort(rng.choice(total_rows, size=min(n, total_rows), replace=False))
+        rows = np.sort(rng.choice(total_rows, size=min(n, total_rows - done), replace=False))
         t1 = time.perf_counter()
         if nvfp4:
             oracle.attn_rows_nvfp4(g, qc, qs, kc, ks, vt, idx, num, rows)
@@ -274,8 +274,9 @@ def cpu_baseline_sample(wl, seconds_hint=20.0, nvfp4=False):
     return {"value": value, "unit": "TFLOP/s", "cores": oracle.max_threads(), "kind": "oracle",
             "sample": (f"oracle tile+pool+score+top-k{'+NVFP4 quantisation' if nvfp4 else ''}+untile over the "
                        f"whole workload ({t_front:.1f} s) and "
-                       f"attention on {done} of {total_rows} query rows ({t_attn:.1f} s), scaled to all rows; "
-                       f"estimated {est:.0f} s per step")}
+                       f"attention on {done} sampled of {total_rows} query rows ({t_attn:.1f} s), scaled to all "
+                       f"rows; "
+                       f"estimated {est:.3g} s per step")}
 
 
 BWD_SOURCES = [os.path.join(ROOT, "block_sparse_video_gather_b200", "csrc", f)
@@ -311,7 +312,7 @@ def bwd_cpu_baseline(wl, inp, do_untiled, idx, num, flops, seconds_hint=20.0):
     rng = np.random.default_rng(3)
     n, t, done = 128, 0.0, 0
     while t < seconds_hint * 0.5 and done < total_rows:
-        rows = np.sort(rng.choice(total_rows, size=min(n, total_rows), replace=False))
+        rows = np.sort(rng.choice(total_rows, size=min(n, total_rows - done), replace=False))
         t1 = time.perf_counter()
         oracle.attn_bwd_q_rows(g, qt, kt, vt, dot, idx, num, rows)
         t += time.perf_counter() - t1
@@ -320,7 +321,7 @@ def bwd_cpu_baseline(wl, inp, do_untiled, idx, num, flops, seconds_hint=20.0):
     est = 2.0 * t * total_rows / done
     return {"value": flops / est / 1e12, "unit": "TFLOP/s", "cores": oracle.max_threads(), "kind": "oracle",
             "sample": (f"oracle dq on {done} of {total_rows} query rows ({t:.1f} s), scaled to all rows and "
-                       f"doubled for dk/dv; estimated {est:.0f} s per backward")}
+                       f"doubled for dk/dv; estimated {est:.3g} s per backward")}
 
 
 def run_backward(args, wl, world, rank, local, pg):
