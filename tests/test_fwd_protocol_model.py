@@ -25,67 +25,27 @@ out of order) must be caught; a harmless change (a later arrival) must not.
 The model is test infrastructure for the protocol's design; the GPU parity
 tests cover the kernels themselves.
 """
-import random
-
 import pytest
 
-
-class Hazard(AssertionError):
-    pass
+from tests.protocol_sim import Hazard, Sim
 
 
-class Bar:
-    """mbarrier: `count` arrivals and all expected copies complete a phase."""
-
-    def __init__(self, name, count):
-        self.name, self.count = name, count
-        self.pending, self.tx, self.done = count, 0, 0
-
-    def _maybe_complete(self):
-        if self.pending == 0 and self.tx == 0:
-            self.done += 1
-            self.pending = self.count
-
-    def arrive(self, n, tag):
-        if tag != self.done:
-            raise Hazard(f"{self.name}: arrival for phase {tag} while phase {self.done} is open")
-        if n > self.pending:
-            raise Hazard(f"{self.name}: {n} arrivals with {self.pending} pending")
-        self.pending -= n
-        self._maybe_complete()
-
-    def expect_tx(self, copies, tag):
-        self.tx += copies
-        self.arrive(1, tag)
-
-    def land(self):
-        self.tx -= 1
-        self._maybe_complete()
-
-    def passes(self, target):
-        # the hardware's parity test for "completion number `target` has happened"
-        return (self.done & 1) == (target & 1)
-
-
-class Model:
+class Model(Sim):
     def __init__(self, nbs, fp4, bs, seed, plant=None):
+        super().__init__(seed)
         self.nbs, self.fp4, self.bs, self.plant = nbs, fp4, bs, plant
-        self.rng = random.Random(seed)
         self.QT = 2 if bs == 256 else 1          # 128-row query tiles per item
         self.KS, self.VS = (4, 3) if fp4 else (3, 2)  # K and V ring stages
-        self.B = {}
         for n in ("q_full", "q_empty"):
-            self._bar(n)
+            self.bar(n)
         for s in range(self.KS):
-            self._bar(("k_full", s)), self._bar(("k_empty", s))
+            self.bar(("k_full", s)), self.bar(("k_empty", s))
         for s in range(self.VS):
-            self._bar(("v_full", s)), self._bar(("v_empty", s))
+            self.bar(("v_full", s)), self.bar(("v_empty", s))
         for i in range(2):
-            self._bar(("s_full", i)), self._bar(("o_full", i))
+            self.bar(("s_full", i)), self.bar(("o_full", i))
             for n in ("s_read", "p_full", "o_empty"):
-                self._bar((n, i), 128)
-        self.pipe, self.copies = [], []
-        self.smem, self.readers = {}, {}
+                self.bar((n, i), 128)
         self.s_val = [None, None]         # product index held by S_i
         self.s_loaded = [set(), set()]    # softmax warps that loaded it
         self.hi = [None, None]            # S_i's second half: ("S", u) or ("sf", owner, u)
@@ -93,9 +53,6 @@ class Model:
         self.p = [None, None]             # P_i: [state, item, tile, warps]
         self.o = [None, None]             # O_i: (item, last tile accumulated)
         self.o_read = [set(), set()]      # epilogue warps that read the final O_i
-
-    def _bar(self, name, count=1):
-        self.B[name] = Bar(name, count)
 
     def items(self):
         return [(it, nb) for it, nb in enumerate(self.nbs) if nb > 0]
@@ -206,17 +163,9 @@ class Model:
             items += 1
 
     # ---------------------------------------------------------------- effects
-    def read_smem(self, buf, version):
-        self.readers[buf] -= 1
-        if self.smem.get(buf) != version:
-            raise Hazard(f"read of {buf} expected {version}, holds {self.smem.get(buf)}")
-
     def tensor_op(self, op):
         kind = op[0]
-        if kind == "commit":
-            b = self.B[op[1]]
-            b.arrive(1, b.done)
-        elif kind == "cp":  # scales of S_i product u into the second half of S_j
+        if kind == "cp":  # scales of S_i product u into the second half of S_j
             _, i, u = op
             j = 1 - i
             if self.s_val[j] is not None and len(self.s_loaded[j]) < 4:
@@ -258,7 +207,7 @@ class Model:
         else:
             raise AssertionError(op)
 
-    def softmax_op(self, op):
+    def local_op(self, role, op):
         kind = op[0]
         if kind == "ld_S":
             _, i, w, g = op
@@ -286,61 +235,20 @@ class Model:
         else:
             raise AssertionError(op)
 
-    # ---------------------------------------------------------------- scheduler
-    def run(self, max_steps=5_000_000):
+    # ---------------------------------------------------------------- scheduler hooks
+    def roles(self):
         roles = {"producer": self.producer(), "mma": self.mma()}
         for i in range(self.QT):
             for w in range(4):
                 roles[("softmax", i, w)] = self.softmax_warp(i, w)
-        cur = {k: next(g, None) for k, g in roles.items()}
-        for _ in range(max_steps):
-            runnable = [k for k, op in cur.items()
-                        if op is not None and (op[0] != "wait" or self.B[op[1]].passes(op[2]))]
-            if self.pipe:
-                runnable.append("pipe")
-            if self.copies:
-                runnable.append("tma")
-            if not runnable:
-                blocked = {k: v for k, v in cur.items() if v is not None}
-                if blocked:
-                    raise Hazard(f"deadlock: {blocked}")
-                return
-            k = self.rng.choice(runnable)
-            if k == "pipe":
-                self.tensor_op(self.pipe.pop(0))
-                continue
-            if k == "tma":  # copies land in any order
-                buf, version, bar = self.copies.pop(self.rng.randrange(len(self.copies)))
-                if self.readers.get(buf, 0):
-                    raise Hazard(f"copy into {buf} lands while {self.readers[buf]} issued readers have not run")
-                self.smem[buf] = version
-                self.B[bar].land()
-                continue
-            op = cur[k]
-            if op[0] == "wait":
-                if self.B[op[1]].done != op[2]:
-                    raise Hazard(f"{k}: wait for completion {op[2]} of {op[1]} passed at {self.B[op[1]].done}")
-            elif op[0] == "arrive":
-                self.B[op[1]].arrive(op[2], op[3])
-            elif op[0] == "tma":
-                _, bar, tag, bufs = op
-                self.B[bar].expect_tx(len(bufs), tag)
-                self.copies.extend((buf, version, bar) for buf, version in bufs)
-            elif op[0] == "pipe":
-                pop = op[1]
-                if pop[0] == "S":
-                    for c in range(2 * self.QT):
-                        self.readers[("q", c)] = self.readers.get(("q", c), 0) + 1
-                    for c in range(2):
-                        self.readers[("k", pop[3], c)] = self.readers.get(("k", pop[3], c), 0) + 1
-                elif pop[0] == "PV":
-                    for c in range(2):
-                        self.readers[("v", pop[2], c)] = self.readers.get(("v", pop[2], c), 0) + 1
-                self.pipe.append(pop)
-            else:
-                self.softmax_op(op)
-            cur[k] = next(roles[k], None)
-        raise AssertionError("model did not finish")
+        return roles
+
+    def pipe_readers(self, op):
+        if op[0] == "S":
+            return [("q", c) for c in range(2 * self.QT)] + [("k", op[3], c) for c in range(2)]
+        if op[0] == "PV":
+            return [("v", op[2], c) for c in range(2)]
+        return ()
 
 
 ITEM_SETS = [
