@@ -137,6 +137,20 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+BAD_CLOCK_REASONS = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
+
+
+def clocks_rejected(clocks) -> bool:
+    """A timed region to measure again: a hardware or thermal slowdown was active,
+    or the SM clock sat well below its maximum with no reason given (a clock lock
+    left behind by another user).  sw_power_cap alone is kept."""
+    if not clocks:
+        return False
+    if BAD_CLOCK_REASONS & set(clocks["reasons"]):
+        return True
+    return not clocks["reasons"] and bool(clocks["sm_max_mhz"]) and clocks["sm_mhz"] < 0.85 * clocks["sm_max_mhz"]
+
+
 def sync_ranks(pg, device_sync=True):
     """Every rank reaches this point with its device idle (barrier between two
     device synchronisations; the barrier alone without a process group)."""
@@ -365,20 +379,25 @@ def run_backward(args, wl, world, rank, local, pg):
     gpu_id = str(getattr(props, "uuid", local))
     if gpu_id and not gpu_id.startswith("GPU-") and len(gpu_id) >= 32:
         gpu_id = "GPU-" + gpu_id
-    sampler = ClockSampler(gpu_id)
-    sampler.start()
-    time.sleep(0.3)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    sync_all()
-    t0.record(stream)
-    for i in range(args.steps):
-        ev[i][0].record(stream)
-        step()
-        ev[i][1].record(stream)
-    t1.record(stream)
-    sync_all()
-    clocks = sampler.stop()
+    for attempt in range(2):  # measured again, once, when the clocks show a slowdown
+        sampler = ClockSampler(gpu_id)
+        sampler.start()
+        time.sleep(0.3)
+        sync_all()
+        t0.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        t1.record(stream)
+        sync_all()
+        clocks = sampler.stop()
+        if attempt == 1 or rank_max(float(clocks_rejected(clocks)), pg) == 0.0:
+            break
+    if clocks is not None and attempt == 1:
+        clocks["remeasured"] = True
     elapsed = max_over_ranks(t0.elapsed_time(t1) / 1e3)
     call_avg = max_over_ranks(float(np.mean([a.elapsed_time(b) / 1e3 for a, b in ev])))
     assert vsa.get_status() == vsa.VSA_OK
@@ -555,19 +574,23 @@ def main():
     gpu_id = str(getattr(props, "uuid", local))
     if gpu_id and not gpu_id.startswith("GPU-") and len(gpu_id) >= 32:
         gpu_id = "GPU-" + gpu_id
-    sampler = ClockSampler(gpu_id)
-    sampler.start()
-    time.sleep(0.3)
-
-    # ---- device-resident timing
+    # ---- device-resident timing (measured again, once, when the clocks show a slowdown)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    sync_all()
-    t0.record(stream)
-    for i in range(args.steps):
-        step(i)
-    t1.record(stream)
-    sync_all()
-    clocks = sampler.stop()
+    for attempt in range(2):
+        sampler = ClockSampler(gpu_id)
+        sampler.start()
+        time.sleep(0.3)
+        sync_all()
+        t0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        t1.record(stream)
+        sync_all()
+        clocks = sampler.stop()
+        if attempt == 1 or rank_max(float(clocks_rejected(clocks)), pg) == 0.0:
+            break
+    if clocks is not None and attempt == 1:
+        clocks["remeasured"] = True
     elapsed = max_over_ranks(t0.elapsed_time(t1) / 1e3)
     attn_s = [a.elapsed_time(b) / 1e3 for a, b in attn_ev]
     front_s = [f.elapsed_time(q) / 1e3 for f, q in zip(front_ev, quant_ev)]
