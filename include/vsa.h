@@ -136,7 +136,8 @@ VSA_API int vsa_untile(vsa_plan_t plan, const uint16_t *x_tiled, uint16_t *x, in
  * largest scores, ties to the lower block index, written to
  * q2k_idx [B,H,NB,topk] in ascending block order; q2k_num [B,H,NB] = topk.
  * qbar, kbar: [B,H,NB,D] fp32 as produced by vsa_tile.  0 < topk <= NB,
- * else VSA_ERR_TOPK.
+ * else VSA_ERR_TOPK; VSA_ERR_UNSUPPORTED for NB > 2048 (the scores of eight
+ * query blocks are staged in shared memory) or D != 128.
  */
 VSA_API int vsa_coarse_topk(vsa_plan_t plan, const float *qbar, const float *kbar, int B, int H, int D,
                     int topk, int32_t *q2k_idx, int32_t *q2k_num, vsa_stream_t stream);

@@ -198,3 +198,16 @@ def test_backward_workspace_size_is_host_only():
     a = vsa.bwd_workspace_bytes(p, 1, 24, 64)
     b = vsa.bwd_workspace_bytes(p, 1, 24, 65)
     assert a > 2 * 24 * p.Sp * 4 and b > a and a % 4 == 0
+
+
+def test_coarse_calls_reject_more_than_2048_blocks(L):
+    """The coarse stage stages eight rows of NB scores in shared memory: NB <= 2048."""
+    big = vsa.Plan(64, 128, 72)  # 16 x 16 x 9 = 2304 blocks
+    assert big.NB == 2304
+    h = big.handle
+    F = ctypes.c_void_p(FAKE)
+    assert L.vsa_coarse_topk(h, F, F, 1, 2, 128, 4, F, F, None) == vsa.VSA_ERR_UNSUPPORTED
+    assert L.vsa_coarse_compress(h, F, F, F, 1, 2, 128, 4, F, F, F, None) == vsa.VSA_ERR_UNSUPPORTED
+    front = (h, vsa.VSA_BF16, F, F, F, 1, 2, 128, 4, F, F, F, F, F, None, F, F, None)
+    assert L.vsa_tile_coarse(*front, F, None) == vsa.VSA_ERR_UNSUPPORTED
+    assert L.vsa_tile_coarse_static(*front, None) == vsa.VSA_ERR_UNSUPPORTED
