@@ -31,11 +31,20 @@ Recipe (stated once, used by every test and by the benchmark):
 * gate (only when asked for): i.i.d. N(0, 1) in the untiled [B, S, H, D]
   layout, rounded the same way -- a stand-in for the output of a learned
   gate_compress projection ("FastVideo VSA", section "Checkpoint behavior");
+* forced-empty rows (``zero_row_frac > 0``): ``round(zero_row_frac * B * H *
+  NB)`` query rows, chosen uniformly at random, select nothing.  With a
+  computed selection (``prefix_dense``) they arrive as a row-keep byte mask
+  [B, H, NB] (0 = forced empty); with a block map, as cleared map rows;
 * block maps (map-driven workloads only): prefix query tiles select every
   tile; a video query tile selects every prefix tile plus ``map_video_k``
-  distinct video tiles chosen uniformly at random; then
-  ``round(zero_row_frac * B * H * NQ)`` rows, chosen uniformly at random,
-  are cleared to select nothing.
+  distinct video tiles chosen uniformly at random; then the forced-empty
+  rows are cleared.
+
+Selections: ``topk`` set and ``prefix_dense`` False -- the coarse stage's
+plain top-k over all blocks; ``prefix_dense`` -- prefix query tiles select
+every tile and a video query tile selects the prefix tiles plus its top-k
+video tiles, both computed by the coarse stage from the pooled scores;
+``topk`` None -- a caller-supplied bool block map.
 """
 from __future__ import annotations
 
@@ -60,6 +69,7 @@ class Workload:
     block: tuple  # (bt, bh, bw) tokens per block along (T, H, W)
     topk: int | None = None  # coarse-stage top-k; None for map-driven workloads
     n_prefix: int = 0  # tokens placed before the video grid, tiled contiguously
+    prefix_dense: bool = False  # prefix query tiles select all; video query tiles the prefix + top-k video tiles
     offset_std: float = 0.5
     offset_ar: float = 0.0
     map_video_k: int = 0
@@ -98,6 +108,13 @@ class Workload:
     def map_driven(self) -> bool:
         return self.topk is None
 
+    @property
+    def max_k(self) -> int:
+        """Row stride of q2k_idx: the longest possible row."""
+        if self.map_driven or self.prefix_dense:
+            return self.num_blocks
+        return self.topk
+
 
 WORKLOADS = {
     # B=1, H=2, grid (8,16,16) = 2048 tokens, 8 blocks, top-k 4.
@@ -106,10 +123,17 @@ WORKLOADS = {
     "fastwan": Workload("fastwan", B=1, H=24, D=128, T=31, Hg=22, Wg=40, block=(4, 8, 8), topk=64),
     # Wan2.1-1.3B, 81 frames: (21,30,52) = 32760 tokens -> 168 blocks, top-k 32.
     "wan81": Workload("wan81", B=1, H=12, D=128, T=21, Hg=30, Wg=52, block=(4, 8, 8), topk=32),
-    # Tile-64, non-uniform rows: 512 prefix tokens + (16,32,32) video, 264 tiles.
+    # Tile-64, non-uniform rows: 512 prefix tokens + (16,32,32) video, 264 tiles;
+    # prefix query tiles dense, video query tiles the prefix + their top-32 video
+    # tiles (computed), 5% of rows forced empty.
     "tile64": Workload("tile64", B=1, H=24, D=128, T=16, Hg=32, Wg=32, block=(4, 4, 4),
-                       topk=None, n_prefix=512, offset_std=0.0, map_video_k=32,
+                       topk=32, n_prefix=512, prefix_dense=True, offset_std=0.0,
                        zero_row_frac=0.05),
+    # The same layout with the selection as a caller-supplied bool block map
+    # (32 random video tiles per video row) compacted by map_to_index.
+    "tile64map": Workload("tile64map", B=1, H=24, D=128, T=16, Hg=32, Wg=32, block=(4, 4, 4),
+                          topk=None, n_prefix=512, offset_std=0.0, map_video_k=32,
+                          zero_row_frac=0.05),
     # Wan2.1-1.3B, 321 frames (4x horizon): (81,30,52) = 126360 tokens -> 588 blocks.
     "long": Workload("long", B=1, H=12, D=128, T=81, Hg=30, Wg=52, block=(4, 8, 8), topk=59,
                      offset_ar=0.9),
@@ -211,10 +235,22 @@ def _block_map(wl: Workload, seq: np.random.SeedSequence) -> np.ndarray:
     return m
 
 
+def _row_keep(wl: Workload, seq: np.random.SeedSequence) -> np.ndarray:
+    """[B, H, NB] uint8: 0 for the forced-empty rows, 1 elsewhere."""
+    n = wl.B * wl.H * wl.num_blocks
+    keep = np.ones(n, dtype=np.uint8)
+    nzero = int(round(wl.zero_row_frac * n))
+    if nzero > 0:
+        keep[np.random.default_rng(seq).permutation(n)[:nzero]] = 0
+    return keep.reshape(wl.B, wl.H, wl.num_blocks)
+
+
 def make_inputs(wl: Workload | str, threads: int = 8, dtype: str = "bf16", gate: bool = False) -> dict:
     """Q, K, V as bf16 (or fp16) bit patterns [B, S, H, D] (uint16), for
-    map-driven workloads the bool block map [B, H, NB, NB], and on request
-    the gate [B, S, H, D] (same format)."""
+    map-driven workloads the bool block map [B, H, NB, NB], for workloads
+    with forced-empty rows and a computed selection the row-keep mask
+    [B, H, NB] uint8 ("row_keep", else None), and on request the gate
+    [B, S, H, D] (same format)."""
     if isinstance(wl, str):
         wl = WORKLOADS[wl]
     root = np.random.SeedSequence(wl.seed)
@@ -225,6 +261,7 @@ def make_inputs(wl: Workload | str, threads: int = 8, dtype: str = "bf16", gate:
         "k": _tensor(wl, nk, ok, threads, dtype),
         "v": _tensor(wl, nv, ov, threads, dtype),
         "map": _block_map(wl, mp) if wl.map_driven else None,
+        "row_keep": _row_keep(wl, mp) if (not wl.map_driven and wl.zero_row_frac > 0) else None,
     }
     if gate:
         g = _normal_fill(ng, wl.B * wl.seq_len * wl.H * wl.D, threads).reshape(wl.B, wl.seq_len, wl.H, wl.D)

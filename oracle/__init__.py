@@ -11,9 +11,12 @@ Each step follows the statement cited in the C file's header:
 * ``geometry``/``tile``/``untile``/``pool``/``score``/``topk``: "FastVideo VSA"
   (vLLM-Omni user guide), introduction and section "Choose top-k";
 * ``map_to_index``: FastVideo commit log, examples/inference/basic/README.md;
+* ``topk_prefix``: the same commit log's tile-64 layout (prefix query tiles
+  dense, video query tiles the prefix plus a top-k of the video tiles, some
+  rows forced empty), with the block score and tie rule of ``topk``;
 * ``attn_rows``: "FastVideo VSA", introduction and section "Verify routing
   and fallback" (non-causal, scale head_size^-1/2), computed in fp64;
-* ``attn_bwd_q_rows``/``attn_bwd_kv``: gradients of the attention step with
+* ``attn_bwd_q_rows``/``attn_bwd_kv``/``attn_bwd_kv_blocks``: gradients of the attention step with
   the selection fixed (definition of softmax attention's derivative; the
   commit log keeps the grad path separate), in fp64, real query rows only;
 * ``quant_nvfp4``/``dequant_nvfp4``/``attn_rows_nvfp4``: FastVideo
@@ -73,6 +76,8 @@ def _load():
         lib.oracle_score.argtypes = [P, P, P, i, i, i, i]
         lib.oracle_topk.argtypes = [P, i, i, i, i, P, P]
         lib.oracle_map_to_index.argtypes = [P, i, i, i, i, P, P]
+        lib.oracle_topk_prefix.argtypes = [P, i, i, i, i, i, P, i, P, P]
+        lib.oracle_attn_bwd_kv_blocks.argtypes = geo + [P, P, P, P, P, P, i, i, i, i, P, L, P, P, i]
         lib.oracle_attn_rows.argtypes = geo + [P, P, P, P, P, i, i, i, i, P, L, P, P, i]
         lib.oracle_compress.argtypes = [P, P, P, i, i, i, i, P]
         lib.oracle_gate_rows.argtypes = geo + [P, L, P, P, P, i, i, i, P, i]
@@ -87,7 +92,8 @@ def _load():
                   "oracle_pool", "oracle_score", "oracle_topk", "oracle_map_to_index",
                   "oracle_attn_rows", "oracle_max_threads", "oracle_half_to_f32", "oracle_compress",
                   "oracle_gate_rows", "oracle_attn_bwd_q_rows", "oracle_attn_bwd_kv", "oracle_quant_nvfp4",
-                  "oracle_dequant_nvfp4", "oracle_e4m3_round", "oracle_attn_rows_nvfp4"):
+                  "oracle_dequant_nvfp4", "oracle_e4m3_round", "oracle_attn_rows_nvfp4", "oracle_topk_prefix",
+                  "oracle_attn_bwd_kv_blocks"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -206,6 +212,27 @@ def topk(s: np.ndarray, k: int):
     return idx, num
 
 
+def topk_prefix(s: np.ndarray, n_pre: int, k: int, row_keep=None, max_k: int | None = None):
+    """Top-k with dense prefix tiles (tile-64 layout): prefix query tiles list
+    every tile; a video query tile lists the n_pre prefix tiles and its k
+    best-scoring video tiles (ties to the lower index), ascending; rows whose
+    row_keep byte is 0 list nothing.  Returns (q2k_idx [B,H,NB,max_k] -1
+    padded, q2k_num [B,H,NB]); max_k defaults to NB (k when n_pre == 0)."""
+    s = np.ascontiguousarray(s, dtype=np.float32)
+    B, H, NB, NB2 = s.shape
+    assert NB == NB2
+    if max_k is None:
+        max_k = NB if n_pre > 0 else k
+    keep = None if row_keep is None else np.ascontiguousarray(row_keep, dtype=np.uint8)
+    if keep is not None:
+        assert keep.shape == (B, H, NB)
+    idx = np.empty((B, H, NB, max_k), dtype=np.int32)
+    num = np.empty((B, H, NB), dtype=np.int32)
+    _check(_load().oracle_topk_prefix(_ptr(s), B, H, NB, n_pre, k, None if keep is None else _ptr(keep), max_k,
+                                      _ptr(idx), _ptr(num)), "topk_prefix")
+    return idx, num
+
+
 def map_to_index(m: np.ndarray):
     """Bool map [B,H,NQ,NK] -> (q2k_idx [B,H,NQ,NK] ascending, -1 padded; q2k_num)."""
     m = np.ascontiguousarray(m, dtype=np.uint8)
@@ -302,6 +329,22 @@ def attn_bwd_kv(g: Geometry, qt, kt, vt, dot, idx, num, dtype: str = "bf16"):
     dv = np.empty((B, H, Sp, D), dtype=np.float64)
     _check(_load().oracle_attn_bwd_kv(*g.args, *[_ptr(a) for a in arrs], _ptr(idx), _ptr(num), idx.shape[-1],
                                       B, H, D, _ptr(dk), _ptr(dv), DTYPES[dtype]), "attn_bwd_kv")
+    return dk, dv
+
+
+def attn_bwd_kv_blocks(g: Geometry, qt, kt, vt, dot, idx, num, blocks, dtype: str = "bf16"):
+    """(dk, dv) fp64 [n, bs, D] of chosen key blocks (flat ids b*H*NB + h*NB + kb): every
+    real query row whose block lists the key block contributes (full-size problems)."""
+    arrs = [np.ascontiguousarray(a, dtype=np.uint16) for a in (qt, kt, vt, dot)]
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    num = np.ascontiguousarray(num, dtype=np.int32)
+    blocks = np.ascontiguousarray(blocks, dtype=np.int64)
+    B, H, Sp, D = arrs[0].shape
+    dk = np.empty((len(blocks), g.bs, D), dtype=np.float64)
+    dv = np.empty((len(blocks), g.bs, D), dtype=np.float64)
+    _check(_load().oracle_attn_bwd_kv_blocks(*g.args, *[_ptr(a) for a in arrs], _ptr(idx), _ptr(num),
+                                             idx.shape[-1], B, H, D, _ptr(blocks), len(blocks), _ptr(dk), _ptr(dv),
+                                             DTYPES[dtype]), "attn_bwd_kv_blocks")
     return dk, dv
 
 

@@ -29,6 +29,10 @@
  *            kept indices are written in ascending order.
  *  map       FastVideo commit log: a bool block map [B,H,NQ,NK] is compacted
  *            into q2k_idx (ascending, -1 padded) and q2k_num (may be 0).
+ *  prefix    FastVideo commit log, the tile-64 layout: prefix query tiles
+ *  top-k     attend every tile; a video query tile attends the prefix tiles
+ *            plus the top-k video tiles by the same block score (same tie
+ *            rule); rows the caller marks are forced empty (count 0).
  *  attention "FastVideo VSA", sections introduction and "Verify routing and
  *            fallback": non-causal attention of every query token of a block
  *            against the valid tokens of its selected blocks only, scale
@@ -266,6 +270,50 @@ int oracle_topk(const float *s, int B, int H, int NB, int topk, int32_t *idx, in
         qsort(keep, topk, sizeof(int), by_index);
         for (int t = 0; t < topk; ++t) idx[r * topk + t] = keep[t];
         num[r] = topk;
+    }
+    free(row);
+    free(keep);
+    return ORACLE_OK;
+}
+
+/*
+ * top-k with dense prefix tiles (FastVideo commit log: in the tile-64 layout
+ * the prefix query tiles attend every tile and a video query tile attends the
+ * prefix plus the top-k of the video tiles; some rows are forced empty).
+ *   s        : [B,H,NB,NB] block scores (oracle_score)
+ *   n_pre    : prefix tiles, blocks 0 .. n_pre-1
+ *   topk     : video tiles kept per video query tile, 0 < topk <= NB - n_pre
+ *   row_keep : [B,H,NB] bytes or NULL; a row whose byte is 0 selects nothing
+ *   max_k    : row stride of idx, at least the longest row (NB when n_pre > 0)
+ * A prefix query tile lists every tile (count NB).  A video query tile lists
+ * the prefix tiles, then the topk video tiles of highest score, ties to the
+ * lower index: count n_pre + topk, all ids ascending.  Unused entries are -1.
+ */
+int oracle_topk_prefix(const float *s, int B, int H, int NB, int n_pre, int topk, const uint8_t *row_keep,
+                       int max_k, int32_t *idx, int32_t *num) {
+    int nvid = NB - n_pre;
+    if (n_pre < 0 || nvid < 1 || topk < 1 || topk > nvid) return ORACLE_ERR_ARG;
+    if (max_k < (n_pre > 0 ? NB : topk)) return ORACLE_ERR_ARG;
+    scored_t *row = (scored_t *)malloc(sizeof(scored_t) * nvid);
+    int *keep = (int *)malloc(sizeof(int) * topk);
+    if (!row || !keep) { free(row); free(keep); return ORACLE_ERR_NOMEM; }
+    for (long r = 0; r < (long)B * H * NB; ++r) {
+        int32_t *out = idx + r * max_k;
+        int blk = (int)(r % NB), c = 0;
+        if (row_keep && !row_keep[r]) {
+            c = 0;
+        } else if (blk < n_pre) {
+            for (int j = 0; j < NB; ++j) out[c++] = j;
+        } else {
+            for (int j = 0; j < n_pre; ++j) out[c++] = j;
+            for (int j = 0; j < nvid; ++j) { row[j].v = s[r * NB + n_pre + j]; row[j].j = n_pre + j; }
+            qsort(row, nvid, sizeof(scored_t), by_score_then_index);
+            for (int t = 0; t < topk; ++t) keep[t] = row[t].j;
+            qsort(keep, topk, sizeof(int), by_index);
+            for (int t = 0; t < topk; ++t) out[c++] = keep[t];
+        }
+        for (int j = c; j < max_k; ++j) out[j] = -1;
+        num[r] = c;
     }
     free(row);
     free(keep);
@@ -515,6 +563,67 @@ int oracle_attn_bwd_kv(int n_prefix, int T, int Hg, int Wg, int bt, int bh, int 
                 for (int d = 0; d < D; ++d) {
                     dvj[d] += p[t] * (double)half_to_f32(doi[d], dtype);
                     dkj[d] += ds * (double)half_to_f32(qi[d], dtype);
+                }
+            }
+        }
+        free(key); free(p); free(dp);
+    }
+    return bad ? ORACLE_ERR_INDEX : ORACLE_OK;
+}
+
+/*
+ * backward, key side, for chosen key blocks: dk and dv of the bs slots of each
+ * block in `blocks` (flat ids bhh * NB + kb), out [n_blocks, bs, D] double.
+ * Every real query row of the head whose block lists kb (a repeated id counts
+ * each time) contributes, exactly as in oracle_attn_bwd_kv: the row's softmax
+ * over all its keys, then dv_j += P_ij do_i and dk_j += scale dS_ij q_i for
+ * the keys j of block kb.  Cost: the rows that select the block, not the
+ * whole attention, so it serves full-size problems.  Padded slots get 0.
+ */
+int oracle_attn_bwd_kv_blocks(int n_prefix, int T, int Hg, int Wg, int bt, int bh, int bw,
+                              const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint16_t *dO,
+                              const int32_t *idx, const int32_t *num, int max_k, int B, int H, int D,
+                              const int64_t *blocks, long n_blocks, double *dk, double *dv, int dtype) {
+    geom_t g;
+    int rc = geom_init(&g, n_prefix, T, Hg, Wg, bt, bh, bw);
+    if (rc) return rc;
+    if (D < 1 || max_k < 1) return ORACLE_ERR_ARG;
+    for (long n = 0; n < n_blocks; ++n)
+        if (blocks[n] < 0 || blocks[n] >= (long)B * H * g.NB) return ORACLE_ERR_ARG;
+    const double scale = 1.0 / sqrt((double)D);
+    memset(dk, 0, sizeof(double) * (size_t)n_blocks * g.bs * D);
+    memset(dv, 0, sizeof(double) * (size_t)n_blocks * g.bs * D);
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (long n = 0; n < n_blocks; ++n) {
+        long bhh = blocks[n] / g.NB;
+        int kb = (int)(blocks[n] % g.NB);
+        long *key = (long *)malloc(sizeof(long) * (size_t)max_keys(&g, max_k));
+        double *p = (double *)malloc(sizeof(double) * (size_t)max_keys(&g, max_k));
+        double *dp = (double *)malloc(sizeof(double) * (size_t)max_keys(&g, max_k));
+        if (!key || !p || !dp) { bad = 1; free(key); free(p); free(dp); continue; }
+        double *dkb = dk + (size_t)n * g.bs * D, *dvb = dv + (size_t)n * g.bs * D;
+        for (int r = 0; r < g.NB; ++r) {
+            int cnt = num[bhh * g.NB + r], listed = 0;
+            if (cnt < 0 || cnt > max_k) { bad = 1; break; }
+            for (int t = 0; t < cnt; ++t) listed |= idx[(bhh * g.NB + r) * (long)max_k + t] == kb;
+            if (!listed) continue;
+            for (int slot = 0; slot < g.bs; ++slot) {
+                if (!slot_is_valid(&g, r, slot)) continue;
+                long i = (long)r * g.bs + slot;
+                long nk = row_softmax(&g, q, k, idx, num, max_k, D, bhh, i, dtype, key, p);
+                if (nk < 0) { bad = 1; continue; }
+                double delta = row_dp(v, dO, bhh, i, g.Sp, D, dtype, key, p, nk, dp);
+                const uint16_t *doi = dO + ((size_t)bhh * g.Sp + i) * D;
+                const uint16_t *qi = q + ((size_t)bhh * g.Sp + i) * D;
+                for (long t = 0; t < nk; ++t) {
+                    if (key[t] / g.bs != kb) continue;
+                    long js = key[t] - (long)kb * g.bs;
+                    double ds = p[t] * (dp[t] - delta) * scale;
+                    for (int d = 0; d < D; ++d) {
+                        dvb[js * D + d] += p[t] * (double)half_to_f32(doi[d], dtype);
+                        dkb[js * D + d] += ds * (double)half_to_f32(qi[d], dtype);
+                    }
                 }
             }
         }

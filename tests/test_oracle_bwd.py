@@ -128,3 +128,74 @@ def test_single_key_row():
     np.testing.assert_allclose(dk, 0.0, atol=1e-15)
     assert np.array_equal(dv[0, 0, 0], f32(do[0, 0, 0]).astype(np.float64))
     assert (dv[0, 0, 1:] == 0).all()
+
+
+def _autograd_gather(qt, kt, vt, do, idx, num, g, valid, h):
+    """The same gradients by a second form: per query block, gather the key and
+    value rows of its listed blocks in list order (a repeated id appears
+    twice), mask padded keys, softmax, o = P V; torch autograd accumulates the
+    gradient of every gathered copy back onto its row."""
+    q = torch.tensor(f32(qt[0, h]), dtype=torch.float64, requires_grad=True)
+    k = torch.tensor(f32(kt[0, h]), dtype=torch.float64, requires_grad=True)
+    v = torch.tensor(f32(vt[0, h]), dtype=torch.float64, requires_grad=True)
+    dot = torch.tensor(f32(do[0, h]), dtype=torch.float64)
+    bs, D = g.bs, q.shape[1]
+    loss = torch.zeros((), dtype=torch.float64)
+    for r in range(g.NB):
+        ids = [int(x) for x in idx[0, h, r, :num[0, h, r]]]
+        if not ids:
+            continue
+        keys = torch.tensor(np.concatenate([np.arange(b * bs, (b + 1) * bs) for b in ids]))
+        real_k = torch.from_numpy(valid[keys.numpy()])
+        rows = torch.arange(r * bs, (r + 1) * bs)
+        real_q = torch.from_numpy(valid[rows.numpy()])
+        logits = (q[rows] @ k[keys].T) / np.sqrt(D)
+        p = torch.softmax(logits.masked_fill(~real_k[None, :], float("-inf")), dim=1)
+        o = p @ v[keys]
+        loss = loss + (o[real_q] * dot[rows][real_q]).sum()
+    loss.backward()
+    return k.grad.numpy(), v.grad.numpy()
+
+
+@pytest.mark.parametrize("shape", [((5, 9, 11), (4, 8, 8), 0), ((6, 8, 12), (4, 4, 4), 100)])
+def test_kv_blocks_match_autograd(shape):
+    """dk, dv of chosen key blocks (full-size checks use this form) equal the
+    fp64 autograd gradients, partial blocks and prefix tiles included."""
+    (T, Hg, Wg), block, npre = shape
+    g, qt, kt, vt, do, idx, num, valid = _problem(T, Hg, Wg, block, npre)
+    H = 2
+    blocks = np.array([h * g.NB + kb for h in range(H) for kb in range(g.NB)], dtype=np.int64)
+    dk, dv = oracle.attn_bwd_kv_blocks(g, qt, kt, vt, do, idx, num, blocks)
+    for h in range(H):
+        _, rk, rv = _autograd(qt, kt, vt, do, idx, num, g, valid, h)
+        got_k = dk[h * g.NB:(h + 1) * g.NB].reshape(g.Sp, -1)
+        got_v = dv[h * g.NB:(h + 1) * g.NB].reshape(g.Sp, -1)
+        np.testing.assert_allclose(got_k, rk, rtol=0, atol=1e-11)
+        np.testing.assert_allclose(got_v, rv, rtol=0, atol=1e-11)
+
+
+def test_kv_blocks_repeated_ids_count_twice():
+    """A block listed twice in a row counts twice (the gather form accumulates
+    both copies); a sample of blocks in any order gives the same rows."""
+    g, qt, kt, vt, do, idx, num, valid = _problem(5, 9, 11, (4, 8, 8), 0, H=1, D=32, k=3, zero_rows=False)
+    idx = idx.copy()
+    r = 1
+    idx[0, 0, r, :3] = [idx[0, 0, r, 0], idx[0, 0, r, 0], (idx[0, 0, r, 0] + 1) % g.NB]
+    num = num.copy()
+    num[0, 0, r] = 3
+    rk, rv = _autograd_gather(qt, kt, vt, do, idx, num, g, valid, 0)
+    order = np.array([5, 0, 3, 1], dtype=np.int64) % g.NB
+    dk, dv = oracle.attn_bwd_kv_blocks(g, qt, kt, vt, do, idx, num, order)
+    for n, kb in enumerate(order):
+        np.testing.assert_allclose(dk[n], rk[kb * g.bs:(kb + 1) * g.bs], rtol=0, atol=1e-11)
+        np.testing.assert_allclose(dv[n], rv[kb * g.bs:(kb + 1) * g.bs], rtol=0, atol=1e-11)
+    # and the whole-problem form agrees with the gather form on the repeated ids
+    fk, fv = oracle.attn_bwd_kv(g, qt, kt, vt, do, idx, num)
+    np.testing.assert_allclose(fk[0, 0], rk, rtol=0, atol=1e-11)
+    np.testing.assert_allclose(fv[0, 0], rv, rtol=0, atol=1e-11)
+
+
+def test_kv_blocks_rejects_out_of_range_block():
+    g, qt, kt, vt, do, idx, num, valid = _problem(4, 8, 8, H=1, D=16, k=1)
+    with pytest.raises(ValueError):
+        oracle.attn_bwd_kv_blocks(g, qt, kt, vt, do, idx, num, np.array([g.NB], np.int64))

@@ -70,7 +70,7 @@ def test_block_count_by_enumeration(name):
 def test_config_block_counts():
     """NB for the workloads as stated with them: 8, 120, 168, 264 tiles, 588."""
     got = {n: oracle.geometry_of(w).NB for n, w in workloads.WORKLOADS.items()}
-    assert got == {"tiny": 8, "fastwan": 120, "wan81": 168, "tile64": 264, "long": 588}
+    assert got == {"tiny": 8, "fastwan": 120, "wan81": 168, "tile64": 264, "tile64map": 264, "long": 588}
 
 
 @pytest.mark.parametrize("shape", SHAPES)
