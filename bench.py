@@ -46,7 +46,10 @@ WORKLOAD_TEXT = {
     "wan81": "Wan2.1-1.3B 81-frame latent grid 21x30x52, B1 H12 D128, block 4x8x8, topk 32",
     "long": "Wan2.1-1.3B 321-frame latent grid 81x30x52, B1 H12 D128, block 4x8x8, topk 59",
     "tile64": ("non-uniform rows, 64-token tiles: 512 prefix + video 16x32x32, B1 H24 D128, tile 4x4x4, "
-               "bool block map (prefix rows dense, video rows prefix + 32, 5% rows empty)"),
+               "computed selection: prefix query tiles dense, video query tiles the prefix + top-32 video tiles, "
+               "5% rows forced empty"),
+    "tile64map": ("non-uniform rows, 64-token tiles: 512 prefix + video 16x32x32, B1 H24 D128, tile 4x4x4, "
+                  "caller bool block map (prefix rows dense, video rows prefix + 32 random, 5% rows empty)"),
 }
 
 
@@ -57,6 +60,30 @@ def selected_flops(wl, num: np.ndarray) -> float:
 
 def uniform_flops(wl) -> float:
     return 4.0 * wl.D * wl.block_tokens ** 2 * wl.B * wl.H * wl.num_blocks * wl.topk
+
+
+def block_real_tokens(wl) -> np.ndarray:
+    """[NB] real (non-padding) tokens of each block: shape bookkeeping of the grid."""
+    bt, bh, bw = wl.block
+    nT, nH, nW = wl.grid_blocks
+    grid = np.zeros((nT * bt, nH * bh, nW * bw), dtype=np.int64)
+    grid[:wl.T, :wl.Hg, :wl.Wg] = 1
+    video = grid.reshape(nT, bt, nH, bh, nW, bw).sum(axis=(1, 3, 5)).reshape(-1)
+    bs = wl.block_tokens
+    pre = [min(bs, wl.n_prefix - i * bs) for i in range(wl.n_prefix_blocks)]
+    return np.concatenate([np.array(pre, dtype=np.int64), video])
+
+
+def real_token_flops(wl, idx: np.ndarray, num: np.ndarray) -> float:
+    """4 * D * (real query tokens) * (real key tokens) summed over the selected
+    (query block, key block) pairs: the work on real tokens only."""
+    real = block_real_tokens(wl)
+    idx = np.asarray(idx, dtype=np.int64)
+    num = np.asarray(num, dtype=np.int64)
+    pos = np.arange(idx.shape[-1])
+    listed = (pos < num[..., None]) & (idx >= 0)
+    keys = np.where(listed, real[np.clip(idx, 0, len(real) - 1)], 0).sum(axis=-1)  # [B,H,NB]
+    return 4.0 * wl.D * float((keys * real[None, None, :]).sum())
 
 
 def attn_source_hash(sources=None) -> str:
@@ -205,6 +232,11 @@ def run_reference(args, wl, world, rank):
     if wl.map_driven:
         _, num_all = oracle.map_to_index(inp["map"])
         flops = selected_flops(wl, num_all)
+    elif wl.prefix_dense:
+        qt_all, kt_all = oracle.tile(g, inp["q"]), oracle.tile(g, inp["k"])
+        _, num_all = oracle.topk_prefix(oracle.score(oracle.pool(g, qt_all), oracle.pool(g, kt_all)), g.n_pre,
+                                        wl.topk, inp["row_keep"], wl.max_k)
+        flops = selected_flops(wl, num_all)
     else:
         flops = uniform_flops(wl)
 
@@ -215,6 +247,10 @@ def run_reference(args, wl, world, rank):
         qt, kt, vt = (oracle.tile(g, head[n]) for n in ("q", "k", "v"))
         if wl.map_driven:
             idx, num = oracle.map_to_index(np.ascontiguousarray(inp["map"][:, h:h + 1]))
+        elif wl.prefix_dense:
+            qbar, kbar = oracle.pool(g, qt), oracle.pool(g, kt)
+            keep = None if inp["row_keep"] is None else np.ascontiguousarray(inp["row_keep"][:, h:h + 1])
+            idx, num = oracle.topk_prefix(oracle.score(qbar, kbar), g.n_pre, wl.topk, keep, wl.max_k)
         else:
             qbar, kbar = oracle.pool(g, qt), oracle.pool(g, kt)
             idx, num = oracle.topk(oracle.score(qbar, kbar), wl.topk)
@@ -263,6 +299,8 @@ def cpu_baseline_sample(wl, seconds_hint=20.0, nvfp4=False):
     qbar, kbar = oracle.pool(g, qt), oracle.pool(g, kt)
     if wl.map_driven:
         idx, num = oracle.map_to_index(inp["map"])
+    elif wl.prefix_dense:
+        idx, num = oracle.topk_prefix(oracle.score(qbar, kbar), g.n_pre, wl.topk, inp["row_keep"], wl.max_k)
     else:
         idx, num = oracle.topk(oracle.score(qbar, kbar), wl.topk)
     if nvfp4:
@@ -350,9 +388,10 @@ def run_backward(args, wl, world, rank, local, pg):
     to16 = workloads.f32_to_f16_bits if args.dtype == "f16" else workloads.f32_to_bf16_bits
     do_untiled = to16(rng.standard_normal(inp["q"].shape).astype(np.float32))  # gradient of the untiled o
     dev16 = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).cuda().view(tdt)
-    fwd = vsa.Forward(plan, wl.B, wl.H, wl.topk, dtype=tdt)
+    fwd = vsa.Forward(plan, wl.B, wl.H, wl.topk, dtype=tdt, prefix_dense=wl.prefix_dense)
     bmap = torch.from_numpy(inp["map"]).cuda() if wl.map_driven else None
-    fwd(dev16(inp["q"]), dev16(inp["k"]), dev16(inp["v"]), bmap)
+    keep = torch.from_numpy(inp["row_keep"]).cuda() if inp["row_keep"] is not None else None
+    fwd(dev16(inp["q"]), dev16(inp["k"]), dev16(inp["v"]), bmap, row_keep=keep)
     do = vsa.tile(plan, dev16(do_untiled))  # tiled; padded rows zero
     ws = torch.empty(vsa.bwd_workspace_bytes(plan, wl.B, wl.H, fwd.idx.shape[-1]), dtype=torch.uint8, device="cuda")
     dq, dk, dv = (torch.empty_like(fwd.qt) for _ in range(3))
@@ -529,11 +568,14 @@ def main():
     host = {n: torch.from_numpy(inp[n].view(np.int16)).view(tdt).pin_memory() for n in tensors}
     if wl.map_driven:
         host["map"] = torch.from_numpy(inp["map"].view(np.uint8)).pin_memory()
+    if inp["row_keep"] is not None:
+        host["row_keep"] = torch.from_numpy(inp["row_keep"]).pin_memory()
     dev = {n: host[n].to("cuda", non_blocking=False) for n in host}
     plan = vsa.Plan.of(wl)
     fwd = vsa.Forward(plan, wl.B, wl.H, wl.topk, dtype=tdt, gated=args.gate, fused=not args.unfused,
-                      nvfp4=args.nvfp4)
+                      nvfp4=args.nvfp4, prefix_dense=wl.prefix_dense)
     o_host = torch.empty(fwd.o.shape, dtype=tdt).pin_memory()
+    lse_host = torch.empty(fwd.lse.shape, dtype=torch.float32).pin_memory()
 
     stream = torch.cuda.current_stream()
     attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -545,7 +587,7 @@ def main():
     def step(i=None):
         if i is not None:
             front_ev[i].record(stream)
-        fwd.front(dev["q"], dev["k"], dev["v"], dev.get("map"))
+        fwd.front(dev["q"], dev["k"], dev["v"], dev.get("map"), dev.get("row_keep"))
         if i is not None:
             quant_ev[i].record(stream)
         fwd.quantize()
@@ -569,6 +611,17 @@ def main():
     torch.cuda.synchronize()
     assert vsa.get_status() == vsa.VSA_OK
     flops = selected_flops(wl, fwd.num.cpu().numpy())
+    flops_real = real_token_flops(wl, fwd.idx.cpu().numpy(), fwd.num.cpu().numpy())
+    fp4_cosine = None
+    if args.nvfp4 and not args.gate:
+        # the page's quality figure for FP4 attention: per-call cosine similarity of
+        # o against the 16-bit path on the same inputs (outside the timed region)
+        ref16 = vsa.Forward(plan, wl.B, wl.H, wl.topk, dtype=tdt, prefix_dense=wl.prefix_dense)
+        o16 = ref16(dev["q"], dev["k"], dev["v"], dev.get("map"), row_keep=dev.get("row_keep"))[0].float()
+        o4 = fwd.back(dev.get("gate"), out=torch.empty_like(fwd.o)).float()
+        fp4_cosine = float(torch.nn.functional.cosine_similarity(o4.reshape(1, -1), o16.reshape(1, -1)).item())
+        del ref16, o16, o4
+        torch.cuda.synchronize()
 
     props = torch.cuda.get_device_properties(local)
     gpu_id = str(getattr(props, "uuid", local))
@@ -603,7 +656,7 @@ def main():
     # copies its q, k, v in and its o out; vsa.HostPipeline overlaps step i's
     # compute with step i+1's upload and step i-1's download (two copy streams)
     pipe = vsa.HostPipeline(fwd)
-    extra = dict(block_map=host.get("map"), gate=host.get("gate"))
+    extra = dict(block_map=host.get("map"), gate=host.get("gate"), row_keep=host.get("row_keep"), lse=lse_host)
     for _ in range(3):
         pipe.submit(host["q"], host["k"], host["v"], o_host, **extra)
     pipe.synchronize()
@@ -623,15 +676,16 @@ def main():
     for _ in range(args.steps):
         for n in dev:
             dev[n].copy_(host[n], non_blocking=True)
-        fwd(dev["q"], dev["k"], dev["v"], dev.get("map"), gate=dev.get("gate"))
+        fwd(dev["q"], dev["k"], dev["v"], dev.get("map"), gate=dev.get("gate"), row_keep=dev.get("row_keep"))
         o_host.copy_(fwd.o, non_blocking=True)
+        lse_host.copy_(fwd.lse, non_blocking=True)
     s1.record(stream)
     sync_all()
     serial_elapsed = max_over_ranks(s0.elapsed_time(s1) / 1e3)
     e2e_elapsed = max_over_ranks(e0.elapsed_time(e1) / 1e3)
     assert vsa.get_status() == vsa.VSA_OK
     h2d = sum(host[n].numel() * host[n].element_size() for n in host)
-    d2h = o_host.numel() * 2
+    d2h = o_host.numel() * 2 + lse_host.numel() * 4  # o and lse: both outputs of the call
 
     if rank == 0:
         burst, sustained, hbm, peak_kind = measured_peaks()
@@ -644,6 +698,7 @@ def main():
             peak = 1.6 * burst
             peak_source += " x 1.6 (Q K^T at the nominal FP4:bf16 ratio 4, P V at bf16)"
         achieved = flops / attn_avg / 1e12
+        achieved_real = flops_real / attn_avg / 1e12
         traffic = (profile_traffic(args.workload, FP4_PROFILE, FP4_SOURCES) if args.nvfp4
                    else profile_traffic(args.workload))
         line = {
@@ -658,10 +713,14 @@ def main():
                 "workload": WORKLOAD_TEXT[args.workload],
                 "B": wl.B, "H": wl.H, "D": wl.D, "grid": [wl.T, wl.Hg, wl.Wg], "block": list(wl.block),
                 "num_blocks": wl.num_blocks, "topk": wl.topk, "selected_block_tflop_per_step": flops / 1e12,
+                "real_token_tflop_per_step": flops_real / 1e12,
+                "flop_count": ("4 * D * bs^2 per selected block pair, padded slots included (the value and the "
+                               "roofline); real_token_tflop_per_step counts real query x real key tokens only"),
                 "selected_pairs": int(fwd.num.sum().item()),
                 "attn_ms": attn_avg * 1e3, "front_ms": float(np.mean(front_s)) * 1e3,
                 "quant_ms": float(np.mean(quant_s)) * 1e3,
                 "qk_format": "NVFP4 (E2M1, E4M3 scale per 16 channels)" if args.nvfp4 else args.dtype,
+                "nvfp4_cosine_vs_16bit": fp4_cosine,
                 "back_ms": float(np.mean(back_s)) * 1e3,
                 # memory-bound stages: algorithmic bytes (untiled q, k, v read + tiled written; tiled o
                 # read + untiled o written, plus the gate when gated) over their event time
@@ -678,6 +737,7 @@ def main():
             "roofline": {
                 "bound": "tensor", "kernel": "attn_fwd_fp4_kernel" if args.nvfp4 else "attn_fwd_kernel",
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "achieved_real_tokens": achieved_real, "frac_real_tokens": achieved_real / peak,
                 "peak_source": peak_source,
                 "traffic": traffic,
             },

@@ -29,6 +29,7 @@ SYMBOLS = (
     "vsa_sparse_attn_fwd", "vsa_sparse_attn_fwd_ex", "vsa_get_status", "vsa_strerror",
     "vsa_coarse_compress", "vsa_untile_gate", "vsa_tile_coarse", "vsa_tile_coarse_static",
     "vsa_sparse_attn_bwd_workspace", "vsa_sparse_attn_bwd", "vsa_quantize_nvfp4", "vsa_sparse_attn_fwd_nvfp4",
+    "vsa_coarse_topk_prefix", "vsa_tile_coarse_prefix",
 )
 
 VSA_BF16 = 0
@@ -73,6 +74,8 @@ def lib():
         L.vsa_untile.argtypes = [P, P, P, i, i, i, P]
         L.vsa_coarse_topk.argtypes = [P, P, P, i, i, i, i, P, P, P]
         L.vsa_map_to_index.argtypes = [P, i, i, i, i, P, P, P]
+        L.vsa_coarse_topk_prefix.argtypes = [P, P, P, P, i, i, i, i, i, P, P, P]
+        L.vsa_tile_coarse_prefix.argtypes = [P, i, P, P, P, P, i, i, i, i, i] + [P] * 9
         L.vsa_coarse_compress.argtypes = [P, P, P, P, i, i, i, i, P, P, P, P]
         L.vsa_untile_gate.argtypes = [P, i, P, P, P, P, i, i, i, P]
         L.vsa_tile_coarse.argtypes = [P, i, P, P, P, i, i, i, i] + [P] * 11
@@ -209,6 +212,26 @@ def coarse_topk(plan: Plan, qbar, kbar, topk: int, idx_out=None, num_out=None):
     return idx_out, num_out
 
 
+def coarse_topk_prefix(plan: Plan, qbar, kbar, topk: int, row_keep=None, max_k: int | None = None, idx_out=None,
+                       num_out=None):
+    """Tile-64 selection: prefix query tiles take every block, video query tiles the
+    prefix plus their top-k video blocks; rows whose row_keep byte [B,H,NB] is 0 take
+    nothing -> (q2k_idx [B,H,NB,max_k] -1 padded, q2k_num [B,H,NB])."""
+    torch = _torch()
+    B, H, NB, D = qbar.shape
+    if max_k is None:
+        max_k = NB if plan.n_prefix > 0 else topk
+    if idx_out is None:
+        idx_out = torch.empty((B, H, NB, max_k), dtype=torch.int32, device=qbar.device)
+    if num_out is None:
+        num_out = torch.empty((B, H, NB), dtype=torch.int32, device=qbar.device)
+    _check(lib().vsa_coarse_topk_prefix(plan.handle, _ptr(qbar, torch.float32, "qbar"),
+                                        _ptr(kbar, torch.float32, "kbar"), _ptr(row_keep, torch.uint8, "row_keep"),
+                                        B, H, D, topk, max_k, _ptr(idx_out, torch.int32, "q2k_idx"),
+                                        _ptr(num_out, torch.int32, "q2k_num"), _stream()), "vsa_coarse_topk_prefix")
+    return idx_out, num_out
+
+
 def coarse_compress(plan: Plan, qbar, kbar, vbar, topk: int = 0, o_out=None, idx_out=None, num_out=None):
     """Compression branch o_compress [B,H,NB,D] fp32: attention among the block
     means.  With topk > 0 the same launch also writes the selection of
@@ -271,6 +294,39 @@ def tile_coarse(plan: Plan, q, k, v, topk: int, ws, gated: bool = False, out: di
         _check(lib().vsa_tile_coarse_static(*args, _stream()), "vsa_tile_coarse_static")
     else:
         _check(lib().vsa_tile_coarse(*args, _ptr(ws, i32, "workspace"), _stream()), "vsa_tile_coarse")
+    return o
+
+
+def tile_coarse_prefix(plan: Plan, q, k, v, topk: int, ws, row_keep=None, max_k: int | None = None,
+                       out: dict | None = None):
+    """Front end in one launch with the tile-64 selection (coarse_topk_prefix): tile q, k, v
+    with block means of q and k, then the selection.  Returns a dict with qt, kt, vt, qbar,
+    kbar, idx, num; tensors given in `out` are written in place."""
+    torch = _torch()
+    B, S, H, D = q.shape
+    code = _dtype_code(q, "q")
+    if S != plan.S:
+        raise ValueError(f"q has {S} tokens, plan expects {plan.S}")
+    if max_k is None:
+        max_k = plan.NB if plan.n_prefix > 0 else topk
+    o = dict(out or {})
+    for n in ("qt", "kt", "vt"):
+        if n not in o:
+            o[n] = torch.empty((B, H, plan.Sp, D), dtype=q.dtype, device=q.device)
+    for n in ("qbar", "kbar"):
+        if n not in o:
+            o[n] = torch.empty((B, H, plan.NB, D), dtype=torch.float32, device=q.device)
+    if "idx" not in o:
+        o["idx"] = torch.empty((B, H, plan.NB, max_k), dtype=torch.int32, device=q.device)
+    if "num" not in o:
+        o["num"] = torch.empty((B, H, plan.NB), dtype=torch.int32, device=q.device)
+    f32, i32 = torch.float32, torch.int32
+    _check(lib().vsa_tile_coarse_prefix(
+        plan.handle, code, _ptr(q, q.dtype, "q"), _ptr(k, q.dtype, "k"), _ptr(v, q.dtype, "v"),
+        _ptr(row_keep, torch.uint8, "row_keep"), B, H, D, topk, max_k,
+        _ptr(o["qt"], q.dtype, "q_tiled"), _ptr(o["kt"], q.dtype, "k_tiled"), _ptr(o["vt"], q.dtype, "v_tiled"),
+        _ptr(o["qbar"], f32, "qbar"), _ptr(o["kbar"], f32, "kbar"), _ptr(o["idx"], i32, "q2k_idx"),
+        _ptr(o["num"], i32, "q2k_num"), _ptr(ws, i32, "workspace"), _stream()), "vsa_tile_coarse_prefix")
     return o
 
 
@@ -414,6 +470,11 @@ class Forward:
     lse [B,H,Sp].  The three stages are also callable one by one (front,
     fine, back).
 
+    prefix_dense=True selects with the tile-64 rule (coarse_topk_prefix:
+    prefix query tiles take every block, video query tiles the prefix plus
+    their top-k video blocks); __call__ then takes the optional row-keep mask
+    [B,H,NB] uint8 (0 = row forced empty) as row_keep=.
+
     fused=True (default) runs the front end as one launch (tile_coarse);
     fused=False as separate tile / coarse launches.
 
@@ -428,10 +489,12 @@ class Forward:
     """
 
     def __init__(self, plan: Plan, B: int, H: int, topk: int | None, device="cuda", D: int = 128, dtype=None,
-                 gated: bool = False, fused: bool = True, nvfp4: bool = False):
+                 gated: bool = False, fused: bool = True, nvfp4: bool = False, prefix_dense: bool = False):
         torch = _torch()
+        if prefix_dense and (gated or topk is None):
+            raise ValueError("prefix_dense needs a top-k and no gate-compress branch")
         self.plan, self.B, self.H, self.D, self.topk = plan, B, H, D, topk
-        self.gated, self.fused, self.nvfp4 = gated, fused, nvfp4
+        self.gated, self.fused, self.nvfp4, self.prefix_dense = gated, fused, nvfp4, prefix_dense
         t = dict(dtype=dtype or torch.bfloat16, device=device)
         self.qt = torch.empty((B, H, plan.Sp, D), **t)
         self.kt = torch.empty((B, H, plan.Sp, D), **t)
@@ -441,7 +504,7 @@ class Forward:
         self.lse = torch.empty((B, H, plan.Sp), dtype=torch.float32, device=device)
         self.qbar = torch.empty((B, H, plan.NB, D), dtype=torch.float32, device=device)
         self.kbar = torch.empty((B, H, plan.NB, D), dtype=torch.float32, device=device)
-        width = topk if topk is not None else plan.NB
+        width = topk if (topk is not None and not (prefix_dense and plan.n_prefix > 0)) else plan.NB
         self.idx = torch.empty((B, H, plan.NB, width), dtype=torch.int32, device=device)
         self.num = torch.empty((B, H, plan.NB), dtype=torch.int32, device=device)
         if gated:
@@ -456,8 +519,24 @@ class Forward:
             self.qs = torch.empty((B, H, plan.Sp // 128, 64 * D // 8), **u8)
             self.ks = torch.empty((B, H, plan.Sp // 128, 64 * D // 8), **u8)
 
-    def front(self, q, k, v, block_map=None):
+    def front(self, q, k, v, block_map=None, row_keep=None):
         p = self.plan
+        if row_keep is not None and not self.prefix_dense:
+            raise ValueError("row_keep applies to the tile-64 selection (prefix_dense=True)")
+        if self.prefix_dense:
+            if block_map is not None:
+                raise ValueError("prefix_dense computes the selection; no block map")
+            if self.fused:
+                out = dict(qt=self.qt, kt=self.kt, vt=self.vt, qbar=self.qbar, kbar=self.kbar, idx=self.idx,
+                           num=self.num)
+                tile_coarse_prefix(p, q, k, v, self.topk, self.ws, row_keep, self.idx.shape[-1], out)
+            else:
+                tile(p, q, pooled=True, out=self.qt, pooled_out=self.qbar)
+                tile(p, k, pooled=True, out=self.kt, pooled_out=self.kbar)
+                tile(p, v, out=self.vt)
+                coarse_topk_prefix(p, self.qbar, self.kbar, self.topk, row_keep, self.idx.shape[-1],
+                                   idx_out=self.idx, num_out=self.num)
+            return
         if self.fused:
             out = dict(qt=self.qt, kt=self.kt, vt=self.vt, qbar=self.qbar, kbar=self.kbar)
             if self.gated:
@@ -512,11 +591,11 @@ class Forward:
             untile(self.plan, self.ot, out=out)
         return out
 
-    def __call__(self, q, k, v, block_map=None, gate=None, out=None):
+    def __call__(self, q, k, v, block_map=None, gate=None, out=None, row_keep=None):
         """One forward step; o goes to `out` when given (else to self.o)."""
         if self.gated != (gate is not None):
             raise ValueError("a gate is required exactly when the Forward was built with gated=True")
-        self.front(q, k, v, block_map)
+        self.front(q, k, v, block_map, row_keep)
         self.fine()
         return self.back(gate, out), self.lse
 
@@ -531,10 +610,11 @@ class Forward:
 class HostPipeline:
     """Forward steps on pinned host tensors with the copies overlapped.
 
-    submit(q, k, v, o[, block_map, gate]) enqueues one step: the inputs go to
-    the device on a copy stream (into one of two input slots), the forward runs
-    on a compute stream once they have landed, and o comes back on a second
-    copy stream (from one of two output slots).  While step i computes, step
+    submit(q, k, v, o[, block_map, gate, row_keep, lse]) enqueues one step:
+    the inputs go to the device on a copy stream (into one of two input
+    slots), the forward runs on a compute stream once they have landed, and o
+    (and lse, when a host tensor is given) come back on a second copy stream
+    (from one of two output slots).  While step i computes, step
     i+1's inputs and step i-1's output are in flight.  Calls return at once;
     synchronize() waits for every submitted step.  The host tensors must stay
     untouched until then.
@@ -545,6 +625,7 @@ class HostPipeline:
         self.fwd = fwd
         self.h2d, self.comp, self.d2h = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
         self.slots_out = [torch.empty_like(fwd.o) for _ in range(2)]
+        self.slots_lse = [torch.empty_like(fwd.lse) for _ in range(2)]
         self.slots_in = [None, None]
         ev = lambda: [torch.cuda.Event(), torch.cuda.Event()]
         self.ev_in, self.ev_used, self.ev_out, self.ev_back = ev(), ev(), ev(), ev()
@@ -556,7 +637,8 @@ class HostPipeline:
             self.slots_in[s] = {k: torch.empty(t.shape, dtype=t.dtype, device="cuda") for k, t in named.items()}
         return self.slots_in[s]
 
-    def submit(self, q, k, v, o, block_map=None, gate=None):
+    def submit(self, q, k, v, o, block_map=None, gate=None, row_keep=None, lse=None):
+        """lse: an optional pinned host tensor [B,H,Sp] fp32 that receives the step's lse."""
         torch = _torch()
         s = self.n & 1
         named = {"q": q, "k": k, "v": v}
@@ -564,6 +646,8 @@ class HostPipeline:
             named["map"] = block_map
         if gate is not None:
             named["gate"] = gate
+        if row_keep is not None:
+            named["row_keep"] = row_keep
         dev = self._inputs(s, named)
         with torch.cuda.stream(self.h2d):
             if self.n >= 2:
@@ -575,12 +659,17 @@ class HostPipeline:
             self.comp.wait_event(self.ev_in[s])
             if self.n >= 2:
                 self.comp.wait_event(self.ev_back[s])  # step n-2's output has left this slot
-            self.fwd(dev["q"], dev["k"], dev["v"], dev.get("map"), dev.get("gate"), out=self.slots_out[s])
+            self.fwd(dev["q"], dev["k"], dev["v"], dev.get("map"), dev.get("gate"), out=self.slots_out[s],
+                     row_keep=dev.get("row_keep"))
+            if lse is not None:
+                self.slots_lse[s].copy_(self.fwd.lse)
             self.ev_used[s].record(self.comp)
             self.ev_out[s].record(self.comp)
         with torch.cuda.stream(self.d2h):
             self.d2h.wait_event(self.ev_out[s])
             o.copy_(self.slots_out[s], non_blocking=True)
+            if lse is not None:
+                lse.copy_(self.slots_lse[s], non_blocking=True)
             self.ev_back[s].record(self.d2h)
         self.n += 1
 

@@ -869,7 +869,14 @@ cudaError_t launch_attn_bwd(const Geo& g, const AttnBwdArgs& a, cudaStream_t str
                                                             static_cast<long long>(rows));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  k2q_kernel<<<a.BH, 256, 2 * g.NB * sizeof(int), stream>>>(a.idx, a.num, g.NB, a.max_k, k2q_off, k2q, a.status);
+  // two int32 per key block of a head (counts, then write positions); above the
+  // default 48 KB the kernel opts in (the API caps NB at kBwdMaxBlocks)
+  const size_t k2q_smem = 2 * static_cast<size_t>(g.NB) * sizeof(int);
+  if (k2q_smem > 48 * 1024 &&
+      (e = cudaFuncSetAttribute(k2q_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(k2q_smem))) != cudaSuccess)
+    return e;
+  k2q_kernel<<<a.BH, 256, k2q_smem, stream>>>(a.idx, a.num, g.NB, a.max_k, k2q_off, k2q, a.status);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
   BwdParams p;

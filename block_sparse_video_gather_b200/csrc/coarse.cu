@@ -8,7 +8,10 @@
 // q2k_idx / q2k_num with rows of any length, zero included.
 //
 // score_topk: one CTA per (b*h, group of 8 query blocks); the work item is
-// score_item of items.cuh.  The pooled K of the head streams through shared
+// score_item of items.cuh.  The selection rule is either the VSA top-k over
+// every block or the tile-64 rule of the commit log (prefix query tiles
+// dense, video query tiles the prefix plus a top-k of the video tiles; rows
+// may be forced empty) -- see SelectRule in common.cuh.  The pooled K of the head streams through shared
 // memory in chunks of 64 blocks (copied with cp.async; 16-byte rows of 132
 // floats, read four channels at a time); a thread owns one key block and two query blocks and
 // runs two independent fused-multiply-add chains in channel order -- the
@@ -38,13 +41,14 @@ namespace {
 using namespace items;
 
 template <bool SELECT, bool COMPRESS>
-__global__ void __launch_bounds__(kThreads) score_topk_kernel(int NB, int topk, const float* __restrict__ qbar,
+__global__ void __launch_bounds__(kThreads) score_topk_kernel(int NB, int topk, SelectRule rule,
+                                                              const float* __restrict__ qbar,
                                                               const float* __restrict__ kbar,
                                                               int32_t* __restrict__ idx, int32_t* __restrict__ num,
                                                               const float* __restrict__ vbar,
                                                               float* __restrict__ o_compress, float scale) {
   extern __shared__ __align__(16) float sm[];
-  score_item<SELECT, COMPRESS, false>(NB, topk, blockIdx.x * kRows, blockIdx.y, qbar, kbar, idx, num, vbar,
+  score_item<SELECT, COMPRESS, false>(NB, topk, rule, blockIdx.x * kRows, blockIdx.y, qbar, kbar, idx, num, vbar,
                                       o_compress, scale, sm);
 }
 
@@ -72,29 +76,32 @@ __global__ void __launch_bounds__(256) map_to_index_kernel(const uint8_t* __rest
 
 
 template <bool SELECT, bool COMPRESS>
-cudaError_t launch_coarse_t(int BH, int NB, int topk, const float* qbar, const float* kbar, int32_t* idx,
-                            int32_t* num, const float* vbar, float* o_compress, float scale, cudaStream_t stream) {
+cudaError_t launch_coarse_t(int BH, int NB, int topk, const SelectRule& rule, const float* qbar, const float* kbar,
+                            int32_t* idx, int32_t* num, const float* vbar, float* o_compress, float scale,
+                            cudaStream_t stream) {
   const size_t smem = score_smem_bytes(NB);
   cudaError_t e = cudaFuncSetAttribute(score_topk_kernel<SELECT, COMPRESS>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   dim3 grid((NB + kRows - 1) / kRows, BH);
-  score_topk_kernel<SELECT, COMPRESS><<<grid, kThreads, smem, stream>>>(NB, topk, qbar, kbar, idx, num, vbar,
+  score_topk_kernel<SELECT, COMPRESS><<<grid, kThreads, smem, stream>>>(NB, topk, rule, qbar, kbar, idx, num, vbar,
                                                                           o_compress, scale);
   return cudaGetLastError();
 }
 
-cudaError_t launch_score_topk(int BH, int NB, int topk, const float* qbar, const float* kbar, int32_t* idx,
-                              int32_t* num, cudaStream_t stream) {
-  return launch_coarse_t<true, false>(BH, NB, topk, qbar, kbar, idx, num, nullptr, nullptr, 0.0f, stream);
+cudaError_t launch_score_topk(int BH, int NB, int topk, const SelectRule& rule, const float* qbar,
+                              const float* kbar, int32_t* idx, int32_t* num, cudaStream_t stream) {
+  return launch_coarse_t<true, false>(BH, NB, topk, rule, qbar, kbar, idx, num, nullptr, nullptr, 0.0f, stream);
 }
 
 cudaError_t launch_coarse_compress(int BH, int NB, int topk, const float* qbar, const float* kbar,
                                    const float* vbar, int32_t* idx, int32_t* num, float* o_compress, float scale,
                                    cudaStream_t stream) {
+  const SelectRule plain{topk, 0, nullptr};
   if (topk > 0)
-    return launch_coarse_t<true, true>(BH, NB, topk, qbar, kbar, idx, num, vbar, o_compress, scale, stream);
-  return launch_coarse_t<false, true>(BH, NB, 0, qbar, kbar, nullptr, nullptr, vbar, o_compress, scale, stream);
+    return launch_coarse_t<true, true>(BH, NB, topk, plain, qbar, kbar, idx, num, vbar, o_compress, scale, stream);
+  return launch_coarse_t<false, true>(BH, NB, 0, plain, qbar, kbar, nullptr, nullptr, vbar, o_compress, scale,
+                                      stream);
 }
 
 cudaError_t launch_map_to_index(const uint8_t* map, long long rows, int NK, int32_t* idx, int32_t* num,

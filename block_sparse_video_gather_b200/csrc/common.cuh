@@ -32,6 +32,22 @@ struct Geo {
   long long S, Sp;    // real and padded tokens
 };
 
+// What a query row of the coarse stage may select, and where its row of the
+// index goes.
+//   stride : entries per row of q2k_idx (at least the longest row); entries
+//            past a row's count are -1
+//   n_pre  : 0 -- top-k over every block (the VSA rule); > 0 -- the tile-64
+//            rule of the FastVideo commit log: query rows 0 .. n_pre-1 (the
+//            prefix tiles) take every block, any other row takes the n_pre
+//            prefix blocks plus its top-k among blocks n_pre .. NB-1
+//   keep   : [B*H, NB] bytes or null; a row whose byte is 0 selects nothing
+// With stride = topk, n_pre = 0 and keep = null this is the plain top-k.
+struct SelectRule {
+  int stride;
+  int n_pre;
+  const uint8_t* keep;
+};
+
 // Real extents (vt, vh, vw) of video block `vb` (0-based among video blocks).
 __device__ __forceinline__ void video_block_extent(const Geo& g, int vb, int& vt, int& vh, int& vw) {
   int bW = vb % g.nW;

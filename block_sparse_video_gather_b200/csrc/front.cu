@@ -131,7 +131,7 @@ __global__ void __launch_bounds__(kTileThreads, 3) front_kernel(FrontArgs a) {
   }
   __syncthreads();
   if (!s_ready) return;
-  score_item<SELECT, COMPRESS, true>(NB, a.topk, item * kRows, head, a.qbar, a.kbar, a.idx, a.num, a.vbar,
+  score_item<SELECT, COMPRESS, true>(NB, a.topk, a.rule, item * kRows, head, a.qbar, a.kbar, a.idx, a.num, a.vbar,
                                      a.o_compress, a.scale, reinterpret_cast<float*>(smem));
   if (threadIdx.x == 0) {
     // every score item of the head has passed its wait once the last one gets here

@@ -158,9 +158,15 @@ __device__ __forceinline__ float key_value(uint32_t k) {
 // order (four channels per step: one 16-byte load of the key row, one
 // broadcast 16-byte load per query row).  Block means reach shared memory by
 // cp.async through L2, every copy of a chunk in flight at once.
+//
+// The selection follows `rule` (common.cuh): a forced-empty row writes count
+// 0; a prefix query row under the tile-64 rule lists every block; any other
+// row lists the rule's n_pre prefix blocks, then its top-k among the blocks
+// n_pre .. NB-1 (every block under the plain rule), then -1 up to the stride.
 template <bool SELECT, bool COMPRESS, bool COHERENT>
-__device__ __forceinline__ void score_item(int NB, int topk, int r0, int bh, const float* qbar, const float* kbar,
-                                           int32_t* __restrict__ idx, int32_t* __restrict__ num, const float* vbar,
+__device__ __forceinline__ void score_item(int NB, int topk, const SelectRule& rule, int r0, int bh,
+                                           const float* qbar, const float* kbar, int32_t* __restrict__ idx,
+                                           int32_t* __restrict__ num, const float* vbar,
                                            float* __restrict__ o_compress, float scale, float* sm) {
   float* q_s = sm;                               // [kRows][128]
   float* k_s = q_s + kRows * 128;                // [kChunk][kKStride]
@@ -222,23 +228,36 @@ __device__ __forceinline__ void score_item(int NB, int topk, int r0, int bh, con
   for (int r = warp; SELECT && r < kRows; r += kThreads / 32) {
     const int row = r0 + r;
     if (row >= NB) break;
+    const long long rid = static_cast<long long>(bh) * NB + row;
+    int32_t* out = idx + rid * rule.stride;
+    if (rule.keep && __ldg(rule.keep + rid) == 0) {  // forced empty
+      for (int j = lane; j < rule.stride; j += 32) out[j] = -1;
+      if (lane == 0) num[rid] = 0;
+      continue;
+    }
+    if (row < rule.n_pre) {  // prefix query tile: every block
+      for (int j = lane; j < rule.stride; j += 32) out[j] = j < NB ? j : -1;
+      if (lane == 0) num[rid] = NB;
+      continue;
+    }
+    const int lo = rule.n_pre;  // candidates lo .. NB-1; blocks 0 .. lo-1 always listed
+    for (int j = lane; j < lo; j += 32) out[j] = j;
     const uint32_t* key = keys + r * NB;
     // k-th largest key: the largest v with #{key >= v} >= topk
     uint32_t tau = 0;
     for (int bit = 31; bit >= 0; --bit) {
       const uint32_t cand = tau | (1u << bit);
       unsigned cnt = 0;
-      for (int j = lane; j < NB; j += 32) cnt += key[j] >= cand;
+      for (int j = lo + lane; j < NB; j += 32) cnt += key[j] >= cand;
       cnt = __reduce_add_sync(0xffffffffu, cnt);
       if (cnt >= static_cast<unsigned>(topk)) tau = cand;
     }
     unsigned gt = 0;
-    for (int j = lane; j < NB; j += 32) gt += key[j] > tau;
+    for (int j = lo + lane; j < NB; j += 32) gt += key[j] > tau;
     gt = __reduce_add_sync(0xffffffffu, gt);
     const int need = topk - static_cast<int>(gt);  // ties at tau to take, lowest ids first
-    int32_t* out = idx + (static_cast<long long>(bh) * NB + row) * topk;
-    int pos = 0, ties = 0;
-    for (int base = 0; base < NB; base += 32) {
+    int pos = lo, ties = 0;
+    for (int base = lo; base < NB; base += 32) {
       const int j = base + lane;
       const uint32_t u = (j < NB) ? key[j] : 0u;
       const bool is_gt = (j < NB) && u > tau;
@@ -250,7 +269,8 @@ __device__ __forceinline__ void score_item(int NB, int topk, int r0, int bh, con
       pos += __popc(sm_);
       ties += __popc(eq);
     }
-    if (lane == 0) num[static_cast<long long>(bh) * NB + row] = topk;
+    for (int j = lo + topk + lane; j < rule.stride; j += 32) out[j] = -1;
+    if (lane == 0) num[rid] = lo + topk;
   }
   if (!COMPRESS) return;
 

@@ -17,8 +17,8 @@ cudaError_t launch_untile_gate(const Geo& g, int B, int H, const uint16_t* xt, c
                                const uint16_t* gate, uint16_t* x, bool f16, cudaStream_t stream);
 
 // coarse.cu
-cudaError_t launch_score_topk(int BH, int NB, int topk, const float* qbar, const float* kbar, int32_t* idx,
-                              int32_t* num, cudaStream_t stream);
+cudaError_t launch_score_topk(int BH, int NB, int topk, const SelectRule& rule, const float* qbar,
+                              const float* kbar, int32_t* idx, int32_t* num, cudaStream_t stream);
 // topk == 0: the compression branch alone (idx, num unused).
 cudaError_t launch_coarse_compress(int BH, int NB, int topk, const float* qbar, const float* kbar,
                                    const float* vbar, int32_t* idx, int32_t* num, float* o_compress, float scale,
@@ -31,6 +31,7 @@ struct FrontArgs {
   Geo g;
   int H, BH;
   int topk;                        // 0: no selection
+  SelectRule rule;                 // with topk > 0: stride, prefix rule, forced-empty rows
   const uint4 *q, *k, *v;          // [B,S,H,D] 16-bit
   uint4 *qt, *kt, *vt;             // [B,H,Sp,D]
   float *qbar, *kbar, *vbar;       // [B,H,NB,D]; vbar null: no compression branch
@@ -94,6 +95,9 @@ struct AttnBwdArgs {
   bool f16;
 };
 size_t attn_bwd_workspace_bytes(const Geo& g, int BH, int max_k);
+// The transposed selection of one head is built in shared memory (8 bytes per
+// key block): at most this many blocks per head.
+constexpr int kBwdMaxBlocks = 28672;
 cudaError_t launch_attn_bwd(const Geo& g, const AttnBwdArgs& a, cudaStream_t stream);
 
 }  // namespace vsa

@@ -235,7 +235,34 @@ int vsa_coarse_topk(vsa_plan_t plan, const float* qbar, const float* kbar, int B
   if (NB > 2048) return VSA_ERR_UNSUPPORTED;  // scores of 8 rows must fit in shared memory
   DeviceState* ds = nullptr;
   if (int rc = device_state(&ds)) return rc;
-  return from_cuda(vsa::launch_score_topk(B * H, NB, topk, qbar, kbar, q2k_idx, q2k_num,
+  const vsa::SelectRule plain{topk, 0, nullptr};
+  return from_cuda(vsa::launch_score_topk(B * H, NB, topk, plain, qbar, kbar, q2k_idx, q2k_num,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+namespace {
+// The tile-64 selection's arguments: 0 < topk <= video blocks, a row stride
+// that holds the longest row, an aligned (or absent) row-keep mask.
+int check_prefix_rule(const vsa::Geo& g, int topk, int max_k, const uint8_t* row_keep) {
+  if (topk < 1 || topk > g.NB - g.n_pre) return VSA_ERR_TOPK;
+  if (max_k < (g.n_pre > 0 ? g.NB : topk)) return VSA_ERR_INVALID_ARG;
+  if (row_keep && (reinterpret_cast<uintptr_t>(row_keep) & 15u)) return VSA_ERR_INVALID_ARG;
+  if (g.NB > 2048) return VSA_ERR_UNSUPPORTED;  // scores of 8 rows must fit in shared memory
+  return VSA_OK;
+}
+}  // namespace
+
+int vsa_coarse_topk_prefix(vsa_plan_t plan, const float* qbar, const float* kbar, const uint8_t* row_keep, int B,
+                           int H, int D, int topk, int max_k, int32_t* q2k_idx, int32_t* q2k_num,
+                           vsa_stream_t stream) {
+  if (!plan || !aligned16(qbar) || !aligned16(kbar) || !aligned16(q2k_idx) || !aligned16(q2k_num))
+    return VSA_ERR_INVALID_ARG;
+  if (int rc = check_dims(B, H, D)) return rc;
+  if (int rc = check_prefix_rule(plan->g, topk, max_k, row_keep)) return rc;
+  DeviceState* ds = nullptr;
+  if (int rc = device_state(&ds)) return rc;
+  const vsa::SelectRule rule{max_k, plan->g.n_pre, row_keep};
+  return from_cuda(vsa::launch_score_topk(B * H, plan->g.NB, topk, rule, qbar, kbar, q2k_idx, q2k_num,
                                           reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -279,6 +306,7 @@ int vsa_tile_coarse(vsa_plan_t plan, vsa_dtype_t dtype, const uint16_t* q, const
   a.H = H;
   a.BH = B * H;
   a.topk = topk;
+  a.rule = vsa::SelectRule{topk, 0, nullptr};
   a.q = reinterpret_cast<const uint4*>(q);
   a.k = reinterpret_cast<const uint4*>(k);
   a.v = reinterpret_cast<const uint4*>(v);
@@ -291,6 +319,45 @@ int vsa_tile_coarse(vsa_plan_t plan, vsa_dtype_t dtype, const uint16_t* q, const
   a.idx = q2k_idx;
   a.num = q2k_num;
   a.o_compress = o_compress;
+  a.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+  a.arrive = workspace;
+  a.done = workspace + static_cast<long long>(B) * H;
+  a.status = ds->status;
+  a.f16 = dtype == VSA_F16;
+  return from_cuda(vsa::launch_front(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int vsa_tile_coarse_prefix(vsa_plan_t plan, vsa_dtype_t dtype, const uint16_t* q, const uint16_t* k,
+                           const uint16_t* v, const uint8_t* row_keep, int B, int H, int D, int topk, int max_k,
+                           uint16_t* q_tiled, uint16_t* k_tiled, uint16_t* v_tiled, float* qbar, float* kbar,
+                           int32_t* q2k_idx, int32_t* q2k_num, int32_t* workspace, vsa_stream_t stream) {
+  if (dtype != VSA_BF16 && dtype != VSA_F16) return VSA_ERR_INVALID_ARG;
+  if (!plan || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q_tiled) || !aligned16(k_tiled) ||
+      !aligned16(v_tiled) || !aligned16(qbar) || !aligned16(kbar) || !aligned16(workspace) ||
+      !aligned16(q2k_idx) || !aligned16(q2k_num))
+    return VSA_ERR_INVALID_ARG;
+  if (int rc = check_dims(B, H, D)) return rc;
+  if (int rc = check_prefix_rule(plan->g, topk, max_k, row_keep)) return rc;
+  DeviceState* ds = nullptr;
+  if (int rc = device_state(&ds)) return rc;
+  vsa::FrontArgs a;
+  a.g = plan->g;
+  a.H = H;
+  a.BH = B * H;
+  a.topk = topk;
+  a.rule = vsa::SelectRule{max_k, plan->g.n_pre, row_keep};
+  a.q = reinterpret_cast<const uint4*>(q);
+  a.k = reinterpret_cast<const uint4*>(k);
+  a.v = reinterpret_cast<const uint4*>(v);
+  a.qt = reinterpret_cast<uint4*>(q_tiled);
+  a.kt = reinterpret_cast<uint4*>(k_tiled);
+  a.vt = reinterpret_cast<uint4*>(v_tiled);
+  a.qbar = qbar;
+  a.kbar = kbar;
+  a.vbar = nullptr;
+  a.idx = q2k_idx;
+  a.num = q2k_num;
+  a.o_compress = nullptr;
   a.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
   a.arrive = workspace;
   a.done = workspace + static_cast<long long>(B) * H;
@@ -451,6 +518,7 @@ int vsa_sparse_attn_bwd(vsa_plan_t plan, vsa_dtype_t dtype, const uint16_t* q, c
   if (!aligned16(q2k_idx) || !aligned16(q2k_num) || max_k < 1) return VSA_ERR_INVALID_ARG;
   if (int rc = check_dims(B, H, D)) return rc;
   const vsa::Geo& g = plan->g;
+  if (g.NB > vsa::kBwdMaxBlocks) return VSA_ERR_UNSUPPORTED;  // transposed selection in shared memory
   DeviceState* ds = nullptr;
   if (int rc = device_state(&ds)) return rc;
   vsa::AttnBwdArgs a;

@@ -9,7 +9,8 @@
  *
  *   vsa_tile(q), vsa_tile(k) (with pooled means), vsa_tile(v)
  *   vsa_coarse_topk(qbar, kbar)          -> q2k_idx, q2k_num
- *      (or vsa_map_to_index(bool map)    -> q2k_idx, q2k_num)
+ *      (or vsa_coarse_topk_prefix for the tile-64 layout's rule,
+ *       or vsa_map_to_index(bool map)    -> q2k_idx, q2k_num)
  *   vsa_sparse_attn_fwd(q, k, v, index)  -> o, lse      (tiled layout)
  *   vsa_untile(o)
  *
@@ -124,8 +125,10 @@ VSA_API int vsa_tile(vsa_plan_t plan, const uint16_t *x, uint16_t *x_tiled, floa
 VSA_API int vsa_tile_ex(vsa_plan_t plan, vsa_dtype_t dtype, const uint16_t *x, uint16_t *x_tiled,
                         float *pooled, int B, int H, int D, vsa_stream_t stream);
 
-/* Untile: x_tiled [B,H,Sp,D] -> x [B,S,H,D]; padded rows are dropped.  A pure
- * 16-bit copy: the same call serves bf16 and fp16. */
+/* Untile ("FastVideo VSA", introduction: the inverse of the regrouping into
+ * contiguous blocks, back to the model's token order): x_tiled [B,H,Sp,D] ->
+ * x [B,S,H,D]; padded rows are dropped.  A pure 16-bit copy: the same call
+ * serves bf16 and fp16. */
 VSA_API int vsa_untile(vsa_plan_t plan, const uint16_t *x_tiled, uint16_t *x, int B, int H, int D,
                vsa_stream_t stream);
 
@@ -226,6 +229,53 @@ VSA_API int vsa_tile_coarse_static(vsa_plan_t plan, vsa_dtype_t dtype, const uin
                                    int32_t *q2k_idx, int32_t *q2k_num, float *o_compress, vsa_stream_t stream);
 
 /*
+ * Coarse stage of the tile-64 layout (FastVideo commit log,
+ * examples/inference/basic/README.md: prefix query tiles attend every tile,
+ * video query tiles attend the prefix plus a top-k of the video tiles, and
+ * some rows select nothing).  With the plan's n_pre prefix tiles (blocks
+ * 0 .. n_pre-1) and the block scores of vsa_coarse_topk:
+ *   - a row whose row_keep byte is 0 selects nothing: count 0;
+ *   - a prefix query tile (row < n_pre) selects every block: count NB;
+ *   - a video query tile selects blocks 0 .. n_pre-1 and the topk video
+ *     blocks of highest score among n_pre .. NB-1 (ties to the lower block
+ *     index): count n_pre + topk.
+ * Ids are written ascending; entries past a row's count are -1.
+ *   qbar, kbar : [B,H,NB,D] fp32 block means (vsa_tile)
+ *   row_keep   : [B,H,NB] bytes (0 = forced empty) or NULL (every row kept)
+ *   max_k      : row stride of q2k_idx; at least NB when the plan has prefix
+ *                tiles, else at least topk
+ *   q2k_idx    : [B,H,NB,max_k] int32, q2k_num: [B,H,NB] int32, caller-owned
+ * Without prefix tiles and with every row kept this is vsa_coarse_topk with
+ * a row stride of max_k.
+ * Errors: VSA_ERR_TOPK unless 0 < topk <= NB - n_pre; VSA_ERR_INVALID_ARG for
+ * a max_k below the longest row or a null / misaligned pointer;
+ * VSA_ERR_UNSUPPORTED for NB > 2048 or D != 128.
+ */
+VSA_API int vsa_coarse_topk_prefix(vsa_plan_t plan, const float *qbar, const float *kbar, const uint8_t *row_keep,
+                                   int B, int H, int D, int topk, int max_k, int32_t *q2k_idx, int32_t *q2k_num,
+                                   vsa_stream_t stream);
+
+/*
+ * The front end in one launch with the selection of vsa_coarse_topk_prefix:
+ * vsa_tile_ex of q, k and v with the block means of q and k, then, per head,
+ * the tile-64 selection -- bit for bit the outputs of vsa_tile_ex and
+ * vsa_coarse_topk_prefix.
+ *   q, k, v                   : [B,S,H,D] dtype
+ *   row_keep, topk, max_k     : as vsa_coarse_topk_prefix
+ *   q_tiled, k_tiled, v_tiled : [B,H,Sp,D] dtype; qbar, kbar: [B,H,NB,D] fp32
+ *   q2k_idx, q2k_num          : [B,H,NB,max_k] / [B,H,NB] int32
+ *   workspace                 : as vsa_tile_coarse (2*B*H int32, zero before
+ *                               the first call, zero again after each call
+ *                               that did not report VSA_ERR_TIMEOUT)
+ * Errors: as vsa_tile_ex and vsa_coarse_topk_prefix.
+ */
+VSA_API int vsa_tile_coarse_prefix(vsa_plan_t plan, vsa_dtype_t dtype, const uint16_t *q, const uint16_t *k,
+                                   const uint16_t *v, const uint8_t *row_keep, int B, int H, int D, int topk,
+                                   int max_k, uint16_t *q_tiled, uint16_t *k_tiled, uint16_t *v_tiled, float *qbar,
+                                   float *kbar, int32_t *q2k_idx, int32_t *q2k_num, int32_t *workspace,
+                                   vsa_stream_t stream);
+
+/*
  * Bool block map -> index (FastVideo commit log: map_to_index):
  * map [B,H,NQ,NK] (one byte per entry, non-zero = selected) ->
  * q2k_idx [B,H,NQ,NK] (selected ids ascending, then -1), q2k_num [B,H,NQ]
@@ -315,6 +365,8 @@ VSA_API int vsa_sparse_attn_fwd_nvfp4(vsa_plan_t plan, vsa_dtype_t dtype, const 
  * FastVideo commit log's layout).
  * Block ids outside [0, NB) and counts outside [0, max_k] are skipped /
  * clamped and set VSA_ERR_BAD_INDEX in the device status word.
+ * VSA_ERR_UNSUPPORTED for NB > 28672 (the transposed selection of a head is
+ * built in shared memory, 8 bytes per block) or D != 128.
  */
 VSA_API int vsa_sparse_attn_bwd_workspace(vsa_plan_t plan, int B, int H, int max_k, size_t *bytes);
 VSA_API int vsa_sparse_attn_bwd(vsa_plan_t plan, vsa_dtype_t dtype, const uint16_t *q, const uint16_t *k,

@@ -77,7 +77,6 @@ def _load():
         lib.oracle_topk.argtypes = [P, i, i, i, i, P, P]
         lib.oracle_map_to_index.argtypes = [P, i, i, i, i, P, P]
         lib.oracle_topk_prefix.argtypes = [P, i, i, i, i, i, P, i, P, P]
-        lib.oracle_attn_bwd_kv_blocks.argtypes = geo + [P, P, P, P, P, P, i, i, i, i, P, L, P, P, i]
         lib.oracle_attn_rows.argtypes = geo + [P, P, P, P, P, i, i, i, i, P, L, P, P, i]
         lib.oracle_compress.argtypes = [P, P, P, i, i, i, i, P]
         lib.oracle_gate_rows.argtypes = geo + [P, L, P, P, P, i, i, i, P, i]
@@ -92,8 +91,7 @@ def _load():
                   "oracle_pool", "oracle_score", "oracle_topk", "oracle_map_to_index",
                   "oracle_attn_rows", "oracle_max_threads", "oracle_half_to_f32", "oracle_compress",
                   "oracle_gate_rows", "oracle_attn_bwd_q_rows", "oracle_attn_bwd_kv", "oracle_quant_nvfp4",
-                  "oracle_dequant_nvfp4", "oracle_e4m3_round", "oracle_attn_rows_nvfp4", "oracle_topk_prefix",
-                  "oracle_attn_bwd_kv_blocks"):
+                  "oracle_dequant_nvfp4", "oracle_e4m3_round", "oracle_attn_rows_nvfp4", "oracle_topk_prefix"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -332,19 +330,66 @@ def attn_bwd_kv(g: Geometry, qt, kt, vt, dot, idx, num, dtype: str = "bf16"):
     return dk, dv
 
 
+def slot_valid(g: Geometry) -> np.ndarray:
+    """[Sp] bool: which tiled slots hold a real token (the tile of an all-ones grid)."""
+    ones = np.full((1, g.S, 1, 8), 0x3F80, dtype=np.uint16)  # bf16 1.0
+    return tile(g, ones)[0, 0, :, 0] != 0
+
+
 def attn_bwd_kv_blocks(g: Geometry, qt, kt, vt, dot, idx, num, blocks, dtype: str = "bf16"):
-    """(dk, dv) fp64 [n, bs, D] of chosen key blocks (flat ids b*H*NB + h*NB + kb): every
-    real query row whose block lists the key block contributes (full-size problems)."""
-    arrs = [np.ascontiguousarray(a, dtype=np.uint16) for a in (qt, kt, vt, dot)]
+    """(dk, dv) fp64 [n, bs, D] of chosen key blocks (flat ids b*H*NB + h*NB + kb).
+
+    The definition of the key-side gradients (C file header, "backward"),
+    written with fp64 matrix products so that full-size problems finish: for
+    every query block r of the head whose list names a chosen block, over the
+    real query rows i of r and the real key slots j of r's listed blocks in
+    list order (a repeated id appears, and counts, twice):
+      P = softmax_j(scale q_i . k_j),  dP_ij = do_i . v_j,
+      dS = P (dP - rowsum(P dP)),
+    then dv_j += sum_i P_ij do_i and dk_j += scale sum_i dS_ij q_i for the
+    slots j of each chosen block.  Padded slots get 0."""
+    qt, kt, vt, dot = (np.ascontiguousarray(a, dtype=np.uint16) for a in (qt, kt, vt, dot))
     idx = np.ascontiguousarray(idx, dtype=np.int32)
     num = np.ascontiguousarray(num, dtype=np.int32)
     blocks = np.ascontiguousarray(blocks, dtype=np.int64)
-    B, H, Sp, D = arrs[0].shape
-    dk = np.empty((len(blocks), g.bs, D), dtype=np.float64)
-    dv = np.empty((len(blocks), g.bs, D), dtype=np.float64)
-    _check(_load().oracle_attn_bwd_kv_blocks(*g.args, *[_ptr(a) for a in arrs], _ptr(idx), _ptr(num),
-                                             idx.shape[-1], B, H, D, _ptr(blocks), len(blocks), _ptr(dk), _ptr(dv),
-                                             DTYPES[dtype]), "attn_bwd_kv_blocks")
+    B, H, Sp, D = qt.shape
+    NB, bs = g.NB, g.bs
+    if ((blocks < 0) | (blocks >= B * H * NB)).any():
+        raise ValueError("oracle attn_bwd_kv_blocks: block id out of range")
+    max_k = idx.shape[-1]
+    scale = 1.0 / np.sqrt(D)
+    valid = slot_valid(g)
+    dk = np.zeros((len(blocks), bs, D))
+    dv = np.zeros((len(blocks), bs, D))
+    wanted = {}
+    for n, fb in enumerate(blocks.tolist()):
+        wanted.setdefault(fb // NB, []).append((n, fb % NB))
+    for bhh, reqs in wanted.items():
+        b, h = divmod(bhh, H)
+        Q, K, V, dO = (half_to_f32(a[b, h], dtype).astype(np.float64) for a in (qt, kt, vt, dot))
+        for r in range(NB):
+            cnt = int(num[b, h, r])
+            if cnt < 0 or cnt > max_k:
+                raise ValueError("oracle attn_bwd_kv_blocks: count out of range")
+            ids = idx[b, h, r, :cnt]
+            if ((ids < 0) | (ids >= NB)).any():
+                raise ValueError("oracle attn_bwd_kv_blocks: block id out of range")
+            hits = [(n, kb) for n, kb in reqs if (ids == kb).any()]
+            if not hits:
+                continue
+            rows = np.arange(r * bs, (r + 1) * bs)[valid[r * bs:(r + 1) * bs]]
+            keys = np.concatenate([np.arange(kb * bs, (kb + 1) * bs) for kb in ids.tolist()])
+            keys = keys[valid[keys]]
+            s = (Q[rows] @ K[keys].T) * scale
+            p = np.exp(s - s.max(axis=1, keepdims=True))
+            p /= p.sum(axis=1, keepdims=True)
+            dp = dO[rows] @ V[keys].T
+            ds = p * (dp - (p * dp).sum(axis=1, keepdims=True))
+            for n, kb in hits:
+                cols = np.flatnonzero(keys // bs == kb)
+                slots = keys[cols] - kb * bs
+                np.add.at(dv[n], slots, p[:, cols].T @ dO[rows])
+                np.add.at(dk[n], slots, scale * (ds[:, cols].T @ Q[rows]))
     return dk, dv
 
 

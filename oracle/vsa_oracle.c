@@ -572,67 +572,6 @@ int oracle_attn_bwd_kv(int n_prefix, int T, int Hg, int Wg, int bt, int bh, int 
 }
 
 /*
- * backward, key side, for chosen key blocks: dk and dv of the bs slots of each
- * block in `blocks` (flat ids bhh * NB + kb), out [n_blocks, bs, D] double.
- * Every real query row of the head whose block lists kb (a repeated id counts
- * each time) contributes, exactly as in oracle_attn_bwd_kv: the row's softmax
- * over all its keys, then dv_j += P_ij do_i and dk_j += scale dS_ij q_i for
- * the keys j of block kb.  Cost: the rows that select the block, not the
- * whole attention, so it serves full-size problems.  Padded slots get 0.
- */
-int oracle_attn_bwd_kv_blocks(int n_prefix, int T, int Hg, int Wg, int bt, int bh, int bw,
-                              const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint16_t *dO,
-                              const int32_t *idx, const int32_t *num, int max_k, int B, int H, int D,
-                              const int64_t *blocks, long n_blocks, double *dk, double *dv, int dtype) {
-    geom_t g;
-    int rc = geom_init(&g, n_prefix, T, Hg, Wg, bt, bh, bw);
-    if (rc) return rc;
-    if (D < 1 || max_k < 1) return ORACLE_ERR_ARG;
-    for (long n = 0; n < n_blocks; ++n)
-        if (blocks[n] < 0 || blocks[n] >= (long)B * H * g.NB) return ORACLE_ERR_ARG;
-    const double scale = 1.0 / sqrt((double)D);
-    memset(dk, 0, sizeof(double) * (size_t)n_blocks * g.bs * D);
-    memset(dv, 0, sizeof(double) * (size_t)n_blocks * g.bs * D);
-    int bad = 0;
-#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
-    for (long n = 0; n < n_blocks; ++n) {
-        long bhh = blocks[n] / g.NB;
-        int kb = (int)(blocks[n] % g.NB);
-        long *key = (long *)malloc(sizeof(long) * (size_t)max_keys(&g, max_k));
-        double *p = (double *)malloc(sizeof(double) * (size_t)max_keys(&g, max_k));
-        double *dp = (double *)malloc(sizeof(double) * (size_t)max_keys(&g, max_k));
-        if (!key || !p || !dp) { bad = 1; free(key); free(p); free(dp); continue; }
-        double *dkb = dk + (size_t)n * g.bs * D, *dvb = dv + (size_t)n * g.bs * D;
-        for (int r = 0; r < g.NB; ++r) {
-            int cnt = num[bhh * g.NB + r], listed = 0;
-            if (cnt < 0 || cnt > max_k) { bad = 1; break; }
-            for (int t = 0; t < cnt; ++t) listed |= idx[(bhh * g.NB + r) * (long)max_k + t] == kb;
-            if (!listed) continue;
-            for (int slot = 0; slot < g.bs; ++slot) {
-                if (!slot_is_valid(&g, r, slot)) continue;
-                long i = (long)r * g.bs + slot;
-                long nk = row_softmax(&g, q, k, idx, num, max_k, D, bhh, i, dtype, key, p);
-                if (nk < 0) { bad = 1; continue; }
-                double delta = row_dp(v, dO, bhh, i, g.Sp, D, dtype, key, p, nk, dp);
-                const uint16_t *doi = dO + ((size_t)bhh * g.Sp + i) * D;
-                const uint16_t *qi = q + ((size_t)bhh * g.Sp + i) * D;
-                for (long t = 0; t < nk; ++t) {
-                    if (key[t] / g.bs != kb) continue;
-                    long js = key[t] - (long)kb * g.bs;
-                    double ds = p[t] * (dp[t] - delta) * scale;
-                    for (int d = 0; d < D; ++d) {
-                        dvb[js * D + d] += p[t] * (double)half_to_f32(doi[d], dtype);
-                        dkb[js * D + d] += ds * (double)half_to_f32(qi[d], dtype);
-                    }
-                }
-            }
-        }
-        free(key); free(p); free(dp);
-    }
-    return bad ? ORACLE_ERR_INDEX : ORACLE_OK;
-}
-
-/*
  * compression branch: dense attention among the block means of each head.
  *   qbar, kbar, vbar : [B,H,NB,D] fp32 block means
  *   out              : [B,H,NB,D] double

@@ -39,13 +39,15 @@ def inputs(wl: workloads.Workload):
 
 @functools.lru_cache(maxsize=4)
 def oracle_front(wl: workloads.Workload):
-    """Oracle tile of q, k, v and the coarse stage (or the map compaction)."""
+    """Oracle tile of q, k, v and the coarse stage (plain or tile-64 rule) or the map compaction."""
     g = oracle.geometry_of(wl)
     inp = inputs(wl)
     qt, kt, vt = (oracle.tile(g, inp[n]) for n in ("q", "k", "v"))
     qbar, kbar = oracle.pool(g, qt), oracle.pool(g, kt)
     if wl.map_driven:
         idx, num = oracle.map_to_index(inp["map"])
+    elif wl.prefix_dense:
+        idx, num = oracle.topk_prefix(oracle.score(qbar, kbar), g.n_pre, wl.topk, inp["row_keep"], wl.max_k)
     else:
         idx, num = oracle.topk(oracle.score(qbar, kbar), wl.topk)
     return dict(g=g, qt=qt, kt=kt, vt=vt, qbar=qbar, kbar=kbar, idx=idx, num=num)

@@ -211,3 +211,43 @@ def test_coarse_calls_reject_more_than_2048_blocks(L):
     front = (h, vsa.VSA_BF16, F, F, F, 1, 2, 128, 4, F, F, F, F, F, None, F, F, None)
     assert L.vsa_tile_coarse(*front, F, None) == vsa.VSA_ERR_UNSUPPORTED
     assert L.vsa_tile_coarse_static(*front, None) == vsa.VSA_ERR_UNSUPPORTED
+
+
+def test_prefix_selection_calls_reject_invalid_arguments(L):
+    """Tile-64 selection: 0 < topk <= video tiles, a row stride that holds the
+    longest row (NB with prefix tiles), aligned pointers, NB <= 2048."""
+    p = vsa.Plan(4, 8, 12, (4, 4, 4), n_prefix=130)  # 3 prefix tiles + 6 video tiles
+    assert p.NB == 9
+    h = p.handle
+    F, M = ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE + 8)
+    call = lambda topk, max_k, keep=None, qbar=F, plan=h: L.vsa_coarse_topk_prefix(
+        plan, qbar, F, keep, 1, 2, 128, topk, max_k, F, F, None)
+    assert call(0, 9) == vsa.VSA_ERR_TOPK
+    assert call(7, 9) == vsa.VSA_ERR_TOPK           # only 6 video tiles
+    assert call(2, 8) == vsa.VSA_ERR_INVALID_ARG    # prefix rows need all 9 entries
+    assert call(2, 9, keep=M) == vsa.VSA_ERR_INVALID_ARG
+    assert call(2, 9, qbar=M) == vsa.VSA_ERR_INVALID_ARG
+    assert call(2, 9, plan=None) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_coarse_topk_prefix(h, F, F, None, 1, 2, 64, 2, 9, F, F, None) == vsa.VSA_ERR_UNSUPPORTED
+    plain = vsa.Plan(8, 16, 16)  # no prefix: the stride only needs topk entries
+    assert call(3, 2, plan=plain.handle) == vsa.VSA_ERR_INVALID_ARG
+    assert call(9, 9, plan=plain.handle) == vsa.VSA_ERR_TOPK
+    big = vsa.Plan(64, 128, 72)
+    assert call(4, big.NB, plan=big.handle) == vsa.VSA_ERR_UNSUPPORTED
+    front = lambda topk, max_k, ws=F, dt=vsa.VSA_BF16: L.vsa_tile_coarse_prefix(
+        h, dt, F, F, F, None, 1, 2, 128, topk, max_k, F, F, F, F, F, F, F, ws, None)
+    assert front(7, 9) == vsa.VSA_ERR_TOPK
+    assert front(2, 8) == vsa.VSA_ERR_INVALID_ARG
+    assert front(2, 9, ws=None) == vsa.VSA_ERR_INVALID_ARG
+    assert front(2, 9, ws=M) == vsa.VSA_ERR_INVALID_ARG
+    assert front(2, 9, dt=5) == vsa.VSA_ERR_INVALID_ARG
+
+
+def test_backward_rejects_more_than_28672_blocks(L):
+    """The backward builds each head's transposed selection in shared memory
+    (8 bytes per block): NB <= 28672, checked before any launch."""
+    big = vsa.Plan(128, 128, 128, (4, 4, 4))  # 32 x 32 x 32 = 32768 tiles of 64
+    assert big.NB == 32768
+    F = ctypes.c_void_p(FAKE)
+    args = (big.handle, vsa.VSA_BF16, F, F, F, F, F, F, F, F, 4, 1, 2, 128, F, F, F, F, None)
+    assert L.vsa_sparse_attn_bwd(*args) == vsa.VSA_ERR_UNSUPPORTED

@@ -27,3 +27,26 @@ def test_slowdowns_and_leftover_clock_locks_are_measured_again():
     # well below the maximum with nothing to explain it: a lock someone left behind
     assert bench.clocks_rejected(_clocks(1100.0, 1965.0, []))
     assert not bench.clocks_rejected(_clocks(1800.0, 1965.0, []))
+
+
+def test_real_token_flops_count_real_query_and_key_tokens():
+    """Real-token FLOPs: 4 D (real query tokens) (real key tokens) per listed
+    pair; the block-pair count includes the padded slots."""
+    import numpy as np
+    import oracle
+    from block_sparse_video_gather_b200 import workloads
+    wl = workloads.custom(T=5, Hg=9, Wg=11, H=1, topk=2)  # partial blocks on every axis
+    real = bench.block_real_tokens(wl)
+    np.testing.assert_array_equal(real, oracle.block_valid_counts(oracle.geometry_of(wl)))
+    idx = np.array([[[[0, 3], [1, -1], [2, 2], [0, 1], [3, 0], [1, 2], [0, 3], [2, 1]]]], dtype=np.int32)
+    num = np.array([[[2, 1, 2, 0, 1, 2, 2, 2]]], dtype=np.int32)
+    want = 0
+    for r in range(8):
+        for t in range(num[0, 0, r]):
+            want += 4 * 128 * int(real[r]) * int(real[idx[0, 0, r, t]])
+    assert bench.real_token_flops(wl, idx, num) == want
+    assert bench.selected_flops(wl, num) == 4 * 128 * 256 ** 2 * int(num.sum())
+    # prefix tiles count their real tokens too (a partial last prefix tile)
+    wl64 = workloads.custom(T=4, Hg=8, Wg=8, block=(4, 4, 4), n_prefix=100, H=1)
+    np.testing.assert_array_equal(bench.block_real_tokens(wl64),
+                                  oracle.block_valid_counts(oracle.geometry_of(wl64)))

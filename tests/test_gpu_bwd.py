@@ -2,10 +2,15 @@
 fp64 oracle (gradients of the attention step of "FastVideo VSA" with the
 selection fixed).
 
-Tolerances, relative to the size of each gradient (16-bit operands P and dS,
-16-bit outputs, fp32 accumulation; delta is formed from the 16-bit o of the
-forward): max-abs error <= 2.5e-2 x max |ref| and mean-abs error <= 8e-3 x
-mean |ref|, per tensor.
+Tolerances, relative to the size of each gradient, per tensor: max-abs error
+<= 1e-2 x max |ref| and mean-abs error <= 5e-3 x mean |ref|.  Where they come
+from: the outputs are bf16, whose rounding alone costs up to 2^-9 (1.95e-3)
+of an element and on average about 2.3e-3 of the mean magnitude (the mean
+ratio every full-size case shows); the tensor-core operands P and dS are
+rounded to 16 bits (2^-9 each, random sign, summed over many rows in fp32),
+and delta = rowsum(do * o) uses the forward's 16-bit o.  Observed on a B200
+over every case here: max ratio <= 4.4e-3, mean ratio <= 3.1e-3; the bounds
+leave about 2x and 1.6x of margin.
 """
 import numpy as np
 import pytest
@@ -19,8 +24,8 @@ from tests import gpu_helpers as H
 
 pytestmark = pytest.mark.gpu
 
-MAX_REL = 2.5e-2
-MEAN_REL = 8e-3
+MAX_REL = 1e-2
+MEAN_REL = 5e-3
 TDT = {"bf16": torch.bfloat16, "f16": torch.float16}
 
 
@@ -144,11 +149,18 @@ def test_bwd_repeated_ids_count_twice():
     _check("repeat dv", _vals(dv, "bf16")[:, :, real], ref_dv[:, :, real])
 
 
-def _gpu_bwd_map(wl, qt, kt, vt, do, bmap):
-    """Forward through the block map on the GPU, then the backward; returns the selection too."""
+def _gpu_bwd_selected(wl, qt, kt, vt, do, inp):
+    """Forward with the workload's own selection on the GPU (the tile-64 rule with
+    its forced-empty rows, or the block map), then the backward; returns the
+    selection too."""
     plan = vsa.Plan.of(wl)
     q, k, v, d = (_dev(x, "bf16") for x in (qt, kt, vt, do))
-    ti, tn = vsa.map_to_index(torch.from_numpy(bmap).cuda())
+    if wl.map_driven:
+        ti, tn = vsa.map_to_index(torch.from_numpy(inp["map"]).cuda())
+    else:
+        qb, kb = vsa.tile(plan, _dev(inp["q"], "bf16"), pooled=True)[1], vsa.tile(plan, _dev(inp["k"], "bf16"),
+                                                                                 pooled=True)[1]
+        ti, tn = vsa.coarse_topk_prefix(plan, qb, kb, wl.topk, torch.from_numpy(inp["row_keep"]).cuda())
     o, lse = vsa.sparse_attn_fwd(plan, q, k, v, ti, tn)
     dq, dk, dv = vsa.sparse_attn_bwd(plan, q, k, v, o, lse, d, ti, tn)
     torch.cuda.synchronize()
@@ -156,19 +168,38 @@ def _gpu_bwd_map(wl, qt, kt, vt, do, bmap):
     return _host(dq), _host(dk), _host(dv), ti.cpu().numpy(), tn.cpu().numpy()
 
 
-def test_bwd_full_size_tile64():
-    """The tile-64 workload (block map with dense prefix rows and empty rows): dq on
-    sampled rows (incl. prefix and empty rows) against the oracle; dk, dv through the
-    sum identities over the rows with a non-empty selection."""
-    wl = workloads.WORKLOADS["tile64"]
+def _check_key_blocks(name, wl, g, qt, kt, vt, do, idx, num, dk, dv, heads, picks):
+    """dk and dv element by element on the chosen key blocks of the chosen heads
+    (every real query row whose block lists the key block contributes)."""
+    blocks = np.array([h * g.NB + kb for h in heads for kb in picks], dtype=np.int64)
+    ref_dk, ref_dv = oracle.attn_bwd_kv_blocks(g, qt, kt, vt, do, idx, num, blocks)
+    real = H.real_rows(wl)
+    got_k = _vals(dk, "bf16").reshape(wl.H, g.NB, g.bs, -1)
+    got_v = _vals(dv, "bf16").reshape(wl.H, g.NB, g.bs, -1)
+    gk = np.stack([got_k[h, kb] for h in heads for kb in picks])
+    gv = np.stack([got_v[h, kb] for h in heads for kb in picks])
+    m = np.stack([real[kb * g.bs:(kb + 1) * g.bs] for h in heads for kb in picks])
+    _check(f"{name} dk blocks", gk[m], ref_dk[m])
+    _check(f"{name} dv blocks", gv[m], ref_dv[m])
+    assert (gk[~m] == 0).all() and (gv[~m] == 0).all()
+
+
+@pytest.mark.parametrize("name", ["tile64", "tile64map"])
+def test_bwd_full_size_tile64(name):
+    """The tile-64 workloads (dense prefix rows, forced-empty rows; the computed
+    tile-64 selection and the block map): dq on sampled rows (incl. prefix and
+    empty rows), dk and dv element by element on sampled key blocks of two heads
+    (prefix tiles among them), against the oracle; plus the sum identities."""
+    wl = workloads.WORKLOADS[name]
     g = oracle.geometry_of(wl)
     inp = workloads.make_inputs(wl)
     qt, kt, vt = (oracle.tile(g, inp[n]) for n in ("q", "k", "v"))
     rng = np.random.default_rng(13)
     do = oracle.tile(g, workloads.f32_to_bf16_bits(rng.standard_normal(inp["q"].shape).astype(np.float32)))
-    dq, dk, dv, idx, num = _gpu_bwd_map(wl, qt, kt, vt, do, inp["map"])
-    ridx, rnum = oracle.map_to_index(inp["map"])
-    np.testing.assert_array_equal(idx, ridx)
+    dq, dk, dv, idx, num = _gpu_bwd_selected(wl, qt, kt, vt, do, inp)
+    ref = H.oracle_front(wl)
+    np.testing.assert_array_equal(idx, ref["idx"])
+    np.testing.assert_array_equal(num, ref["num"])
     real = np.flatnonzero(H.real_rows(wl))
     rows = []
     for bh in range(wl.B * wl.H):
@@ -177,8 +208,11 @@ def test_bwd_full_size_tile64():
         extra = [z * g.bs + np.arange(0, g.bs, 21) for z in zero] + [np.arange(0, g.n_pre * g.bs, 97)]
         rows.append(bh * g.Sp + np.unique(np.concatenate([pick] + extra)))
     rows = np.concatenate(rows)
-    ref = oracle.attn_bwd_q_rows(g, qt, kt, vt, do, idx, num, rows)
-    _check("tile64 dq rows", _vals(dq, "bf16").reshape(-1, 128)[rows], ref)
+    ref_dq = oracle.attn_bwd_q_rows(g, qt, kt, vt, do, idx, num, rows)
+    _check(f"{name} dq rows", _vals(dq, "bf16").reshape(-1, 128)[rows], ref_dq)
+    picks = [0, g.n_pre - 1, g.n_pre, 100, 171, g.NB - 1] + sorted(rng.choice(np.arange(g.n_pre, g.NB), 2,
+                                                                              replace=False).tolist())
+    _check_key_blocks(name, wl, g, qt, kt, vt, do, idx, num, dk, dv, [0, wl.H - 1], picks)
     realm = H.real_rows(wl)
     dkv = _vals(dk, "bf16")[0][:, realm]
     dvv = _vals(dv, "bf16")[0][:, realm]
@@ -192,9 +226,11 @@ def test_bwd_full_size_tile64():
 
 @pytest.mark.parametrize("name", ["fastwan", "wan81", "long"])
 def test_bwd_full_size(name):
-    """The top-k workloads at full size: dq on sampled rows against the oracle;
-    dk and dv through identities that hold at any size: sum over keys of dk is 0
-    and sum of dv is the sum of do over rows with a non-empty selection."""
+    """The top-k workloads at full size: dq on sampled rows, dk and dv element by
+    element on sampled key blocks of two heads (the partial corner block among
+    them), against the oracle; plus identities that hold at any size: the sum
+    over keys of dk is 0 and the sum of dv is the sum of do over rows with a
+    non-empty selection."""
     wl = workloads.WORKLOADS[name]
     g, qt, kt, vt, do, idx, num = _problem(wl, "bf16", None, seed=11)
     dq, dk, dv = _gpu_bwd(wl, "bf16", qt, kt, vt, do, idx, num)
@@ -205,6 +241,9 @@ def test_bwd_full_size(name):
                            for bh in range(wl.H)])
     ref = oracle.attn_bwd_q_rows(g, qt, kt, vt, do, idx, num, rows)
     _check(f"{name} dq rows", _vals(dq, "bf16").reshape(-1, 128)[rows], ref)
+    nblk = 8 if name != "long" else 4
+    picks = [0, g.NB - 1] + sorted(rng.choice(np.arange(1, g.NB - 1), nblk - 2, replace=False).tolist())
+    _check_key_blocks(name, wl, g, qt, kt, vt, do, idx, num, dk, dv, [0, wl.H - 1], picks)
     realm = H.real_rows(wl)
     dkv = _vals(dk, "bf16")[0][:, realm]
     dvv = _vals(dv, "bf16")[0][:, realm]

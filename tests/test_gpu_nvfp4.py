@@ -221,9 +221,10 @@ def test_full_path_nvfp4_full_size(name):
     ref = H.oracle_front(wl)
     inp = H.inputs(wl)
     plan = vsa.Plan.of(wl)
-    fwd = vsa.Forward(plan, wl.B, wl.H, wl.topk, nvfp4=True)
+    fwd = vsa.Forward(plan, wl.B, wl.H, wl.topk, nvfp4=True, prefix_dense=wl.prefix_dense)
     bmap = torch.from_numpy(inp["map"]).cuda() if wl.map_driven else None
-    o, lse = fwd(H.to_dev(inp["q"]), H.to_dev(inp["k"]), H.to_dev(inp["v"]), bmap)
+    keep = torch.from_numpy(inp["row_keep"]).cuda() if inp["row_keep"] is not None else None
+    o, lse = fwd(H.to_dev(inp["q"]), H.to_dev(inp["k"]), H.to_dev(inp["v"]), bmap, row_keep=keep)
     torch.cuda.synchronize()
     assert vsa.get_status() == vsa.VSA_OK
     (qc, qs), (kc, ks) = oracle.quant_nvfp4(ref["qt"]), oracle.quant_nvfp4(ref["kt"])
@@ -262,3 +263,28 @@ def test_fp4_attention_batch_of_two(shape):
     for pos in np.ndindex(2, 2, g.NB):
         idx[pos][:num[pos]] = np.sort(rng.permutation(g.NB)[:num[pos]])
     _fp4_vs_oracle(wl, qt, kt, vt, idx, num, what=f"B2 {shape}")
+
+
+@pytest.mark.parametrize("name", ["tiny", "fastwan", "wan81", "tile64", "long"])
+def test_fp4_cosine_to_bf16_per_call(name):
+    """The FastVideo "Optimizations" page (section "FP4 Flash Attention 4",
+    "Known Limitations") quotes a per-call cosine similarity of about 0.99 between
+    the FP4 and the BF16 attention output.  Here: the cosine of the NVFP4 fine
+    stage's o against the bf16 fine stage's o on the same inputs and selection,
+    over the real rows of one call, on every workload."""
+    wl = workloads.WORKLOADS[name]
+    inp = H.inputs(wl)
+    plan = vsa.Plan.of(wl)
+    bmap = torch.from_numpy(inp["map"]).cuda() if wl.map_driven else None
+    keep = torch.from_numpy(inp["row_keep"]).cuda() if inp["row_keep"] is not None else None
+    args = (H.to_dev(inp["q"]), H.to_dev(inp["k"]), H.to_dev(inp["v"]), bmap)
+    f16 = vsa.Forward(plan, wl.B, wl.H, wl.topk, prefix_dense=wl.prefix_dense)
+    f4 = vsa.Forward(plan, wl.B, wl.H, wl.topk, nvfp4=True, prefix_dense=wl.prefix_dense)
+    o16 = f16(*args, row_keep=keep)[0].float()
+    o4 = f4(*args, row_keep=keep)[0].float()
+    torch.cuda.synchronize()
+    assert vsa.get_status() == vsa.VSA_OK
+    assert torch.equal(f16.idx, f4.idx)
+    cos = float(torch.nn.functional.cosine_similarity(o4.reshape(1, -1), o16.reshape(1, -1)).item())
+    print(f"{name}: cosine(o_fp4, o_bf16) = {cos:.5f}")
+    assert cos >= 0.99, cos

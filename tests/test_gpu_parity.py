@@ -126,7 +126,7 @@ def test_map_to_index_bit_exact(shape):
 
 
 def test_map_to_index_tile64_workload():
-    wl = workloads.WORKLOADS["tile64"]
+    wl = workloads.WORKLOADS["tile64map"]
     m = H.inputs(wl)["map"]
     idx, num = vsa.map_to_index(torch.from_numpy(m).cuda())
     ref_idx, ref_num = oracle.map_to_index(m)
@@ -229,25 +229,28 @@ def _sample_rows(wl, n_per_head, seed):
     return np.concatenate(rows)
 
 
-@pytest.mark.parametrize("name", ["tiny", "fastwan", "wan81", "long", "tile64"])
+@pytest.mark.parametrize("name", ["tiny", "fastwan", "wan81", "long", "tile64", "tile64map"])
 def test_full_path_full_size(name):
     """The launch configuration the benchmark times (vsa.Forward) at full size:
     indices bit-exact, o/lse on sampled real rows, untile of o bit-exact.
-    tile64 takes its caller-supplied bool block map through map_to_index."""
+    tile64 computes the tile-64 selection (prefix tiles dense, video tiles the
+    prefix + top-32, forced-empty rows); tile64map takes a caller-supplied bool
+    block map through map_to_index."""
     wl = workloads.WORKLOADS[name]
     ref = H.oracle_front(wl)
     inp = H.inputs(wl)
     plan = vsa.Plan.of(wl)
-    fwd = vsa.Forward(plan, wl.B, wl.H, wl.topk)
+    fwd = vsa.Forward(plan, wl.B, wl.H, wl.topk, prefix_dense=wl.prefix_dense)
     bmap = torch.from_numpy(inp["map"]).cuda() if wl.map_driven else None
-    o, lse = fwd(H.to_dev(inp["q"]), H.to_dev(inp["k"]), H.to_dev(inp["v"]), bmap)
+    keep = torch.from_numpy(inp["row_keep"]).cuda() if inp["row_keep"] is not None else None
+    o, lse = fwd(H.to_dev(inp["q"]), H.to_dev(inp["k"]), H.to_dev(inp["v"]), bmap, row_keep=keep)
     torch.cuda.synchronize()
     assert vsa.get_status() == vsa.VSA_OK
     np.testing.assert_array_equal(fwd.idx.cpu().numpy(), ref["idx"])
     np.testing.assert_array_equal(fwd.num.cpu().numpy(), ref["num"])
     np.testing.assert_array_equal(H.from_dev(fwd.qt), ref["qt"])
     rows = _sample_rows(wl, 48 if name != "tiny" else 200, seed=16)
-    if wl.map_driven:  # include rows of zero-count tiles and of dense prefix tiles
+    if wl.map_driven or wl.prefix_dense:  # include rows of zero-count tiles and of dense prefix tiles
         g = ref["g"]
         zero = np.flatnonzero(ref["num"].reshape(-1) == 0)[:8]
         extra = [(z // g.NB) * g.Sp + (z % g.NB) * g.bs + np.arange(0, g.bs, 9) for z in zero]
