@@ -30,6 +30,7 @@ struct Geo {
   int n_pre;          // prefix tiles
   int NB;             // total blocks
   long long S, Sp;    // real and padded tokens
+  int vfull;          // 1: every video block is whole (T, Hg, Wg multiples of bt, bh, bw)
 };
 
 // What a query row of the coarse stage may select, and where its row of the

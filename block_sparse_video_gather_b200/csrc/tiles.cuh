@@ -32,6 +32,7 @@ __device__ __forceinline__ int key_tile_mask(const Geo& g, int kb, int half, uin
     }
     return kTilePartial;
   }
+  if (g.vfull) return kTileFull;
   int vt, vh, vw;
   video_block_extent(g, kb - g.n_pre, vt, vh, vw);
   if (vt == g.bt && vh == g.bh && vw == g.bw) return kTileFull;
@@ -77,6 +78,10 @@ __device__ __forceinline__ int block64_mask(const Geo& g, int kb, uint32_t& w0, 
     w0 = lim >= 32 ? 0xffffffffu : ((1u << lim) - 1u);
     w1 = lim <= 32 ? 0u : ((1u << (lim - 32)) - 1u);
     return kTilePartial;
+  }
+  if (g.vfull) {
+    w0 = w1 = 0xffffffffu;
+    return kTileFull;
   }
   int vt, vh, vw;
   video_block_extent(g, kb - g.n_pre, vt, vh, vw);

@@ -159,6 +159,7 @@ int vsa_plan_create_prefix(int n_prefix, int T, int Hg, int Wg, int bt, int bh, 
   g.NB = static_cast<int>(nvid + g.n_pre);
   g.S = static_cast<long long>(n_prefix) + static_cast<long long>(T) * Hg * Wg;
   g.Sp = static_cast<long long>(g.NB) * bs;
+  g.vfull = (T % bt == 0 && Hg % bh == 0 && Wg % bw == 0) ? 1 : 0;
   vsa_plan* p = new (std::nothrow) vsa_plan;
   if (!p) return VSA_ERR_INVALID_ARG;
   p->g = g;
