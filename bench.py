@@ -36,7 +36,15 @@ from block_sparse_video_gather_b200 import workloads  # noqa: E402
 
 PROFILE = os.path.join(ROOT, "profiles", "attn_fwd_fastwan.md")
 ATTN_SOURCES = [os.path.join(ROOT, "block_sparse_video_gather_b200", "csrc", f)
-                for f in ("attn_fwd.cu", "common.cuh", "tiles.cuh")]
+                for f in ("attn_fwd.cu", "fwd_common.cuh", "common.cuh", "tiles.cuh")]
+GROUPED_SOURCES = [os.path.join(ROOT, "block_sparse_video_gather_b200", "csrc", f)
+                   for f in ("attn_fwd_grouped.cu", "fwd_common.cuh", "common.cuh", "tiles.cuh")]
+# committed ncu summaries that carry the DRAM traffic of one fine-stage launch:
+# workload -> (summary, the kernel sources its source_hash covers)
+TRAFFIC_PROFILES = {
+    "fastwan": (PROFILE, ATTN_SOURCES),
+    "tile64": (os.path.join(ROOT, "profiles", "attn_fwd_grouped64_tile64.md"), GROUPED_SOURCES),
+}
 FP4_PROFILE = os.path.join(ROOT, "profiles", "attn_fwd_fp4_fastwan.md")
 FP4_SOURCES = [os.path.join(ROOT, "block_sparse_video_gather_b200", "csrc", f)
                for f in ("fp4.cu", "common.cuh", "tiles.cuh")]
@@ -531,10 +539,20 @@ def main():
     ap.add_argument("--nvfp4", action="store_true",
                     help="NVFP4 q and k in the fine stage (quantisation + FP4 Q K^T), v and P 16-bit")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="run the workload with this many heads (a smaller case of the same grid for profiler "
+                         "captures; the line then names the head count)")
+    ap.add_argument("--frames", type=int, default=None,
+                    help="run the workload with this many latent frames T (a smaller case for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")
     wl = workloads.WORKLOADS[args.workload]
+    if args.heads is not None or args.frames is not None:
+        import dataclasses
+        wl = dataclasses.replace(wl, H=args.heads or wl.H, T=args.frames or wl.T)
+        WORKLOAD_TEXT[args.workload] = (WORKLOAD_TEXT[args.workload] +
+                                        f" (profiling case: H={wl.H}, T={wl.T})")
     world, rank, local = dist_setup(args)
 
     if args.impl == "reference":
@@ -699,8 +717,12 @@ def main():
             peak_source += " x 1.6 (Q K^T at the nominal FP4:bf16 ratio 4, P V at bf16)"
         achieved = flops / attn_avg / 1e12
         achieved_real = flops_real / attn_avg / 1e12
-        traffic = (profile_traffic(args.workload, FP4_PROFILE, FP4_SOURCES) if args.nvfp4
-                   else profile_traffic(args.workload))
+        if args.nvfp4:
+            traffic = profile_traffic(args.workload, FP4_PROFILE, FP4_SOURCES)
+        elif args.workload in TRAFFIC_PROFILES and args.heads is None and args.frames is None:
+            traffic = profile_traffic(args.workload, *TRAFFIC_PROFILES[args.workload])
+        else:
+            traffic = None
         line = {
             "metric": "VSA sparse-attn fwd effective TFLOP/s (selected blocks) on 1 B200",
             "value": world * flops * args.steps / elapsed / 1e12,
@@ -735,7 +757,10 @@ def main():
                 "front_end": "separate launches" if args.unfused else "one launch (tile + coarse)",
             },
             "roofline": {
-                "bound": "tensor", "kernel": "attn_fwd_fp4_kernel" if args.nvfp4 else "attn_fwd_kernel",
+                "bound": "tensor",
+                "kernel": ("attn_fwd_fp4_kernel" if args.nvfp4 else
+                           "attn_fwd_grouped64_kernel" if (wl.block_tokens == 64 and wl.num_blocks <= 1024)
+                           else "attn_fwd_kernel"),
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "achieved_real_tokens": achieved_real, "frac_real_tokens": achieved_real / peak,
                 "peak_source": peak_source,

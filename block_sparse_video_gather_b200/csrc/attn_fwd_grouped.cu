@@ -1,0 +1,639 @@
+// attn_fwd_grouped.cu -- fine stage of VSA for 64-token blocks (the tile-64
+// layout of the FastVideo commit log, examples/inference/basic/README.md:
+// rows of any length, zero included), with four query blocks per work item
+// over the union of their selections.  "FastVideo VSA" (vLLM-Omni user
+// guide), introduction: each query block attends only to the tokens of its
+// selected blocks; non-causal; scale head_size^-1/2.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "fwd_common.cuh"
+#include "kernels.h"
+#include "tiles.cuh"
+
+namespace vsa {
+
+namespace {
+
+using namespace tiles;
+using namespace fwd;
+
+// ===========================================================================
+// 64-token blocks, grouped.
+//
+// A 64-row query block fills only half of an M = 128 product, and one block
+// per item leaves the second softmax warpgroup idle.  Here a work item is a
+// group of four consecutive query blocks of one head -- two 128-row Q tiles,
+// one per softmax warpgroup, exactly the 256-token kernel's schedule -- and
+// the key stream is the ascending union of the four selections, two 64-key
+// blocks per 128-key tile.  Each softmax warp serves one query block (warps
+// 0-1 of a warpgroup the first, 2-3 the second) and looks up, per key tile,
+// whether its block selected each half: unselected halves are masked, and a
+// warp whose block selected neither half skips the exponentials (P = 0).  The
+// tensor core computes every tile for both Q tiles; the softmax pays only for
+// the selected pairs.
+//
+// A fourth role builds the groups: warp 2 reads the four index rows, sets one
+// bit per (query block, selected block) in shared-memory bitmaps (double
+// buffered, two groups ahead), ORs them into the union, counts the tiles and
+// hands the group over on grp_full; the ten consuming warps (producer, MMA,
+// eight softmax warps) release it on grp_free.  Block ids outside [0, NB) are
+// skipped and counts outside [0, max_k] clamped (both reported); a list that
+// names a block twice puts the whole group in list order instead ("concat":
+// each query block's list, two ids per tile, only that block's rows unmasked),
+// so a repeated id counts twice as in the ungrouped kernel.
+//
+// The bitmaps hold kGroupMaxNB blocks: the host uses this kernel for
+// 64-token blocks when NB <= kGroupMaxNB.
+// ===========================================================================
+constexpr int kGroupBlocks = 4;
+constexpr int kGroupMaxWords = 32;
+static_assert(kGroupMaxNB == 32 * kGroupMaxWords, "bitmap capacity");
+
+struct GroupInfo {
+  int concat;   // 1: walk each list as given (a list repeats an id)
+  int n_tiles;  // 128-key tiles of the group's key stream
+  int nq;       // 128-row query tiles (1 for a group of two query blocks)
+  int cnt[kGroupBlocks];
+  int pad;
+  uint32_t bm[kGroupBlocks + 1][kGroupMaxWords];  // selection bitmaps; [kGroupBlocks] = union
+};
+
+struct GroupBarriers {
+  uint64_t q_full, q_empty;
+  uint64_t k_full[kStagesK], k_empty[kStagesK];
+  uint64_t v_full[kStagesV], v_empty[kStagesV];
+  uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
+  uint64_t grp_full[2], grp_free[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(GroupBarriers) <= 256, "barrier block too large");
+
+constexpr uint32_t kSmemGroups = kSmemBar + 256;
+constexpr uint32_t kSmemTotalG = kSmemGroups + 2 * sizeof(GroupInfo) + 1024;
+static_assert(kSmemTotalG <= 232448, "grouped kernel exceeds the shared memory of one CTA");
+constexpr uint32_t kGroupConsumers = 10;  // producer, MMA, 8 softmax warps: one arrival each
+
+__device__ __forceinline__ bool gwarp_wait(uint64_t* bar, uint32_t parity, GroupBarriers* bars,
+                                           unsigned int* status) {
+  bool ok = mbar_wait(bar, parity, &bars->abort, status, kTimeoutNs);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Block id at position t of index row `row`, or -1 when outside [0, NB).
+__device__ __forceinline__ int row_block_id(const Params& p, int row, int t) {
+  const int kb = __ldg(p.idx + static_cast<long long>(row) * p.max_k + t);
+  return (kb >= 0 && kb < p.g.NB) ? kb : -1;
+}
+
+// The key stream of one group: 128-key tile after 128-key tile, the two block
+// ids (-1: absent or unusable) and the query blocks of the group that use each.
+struct GroupWalk {
+  int a;       // union: bitmap word; concat: query block j
+  uint32_t b;  // union: bits of word a still to visit; concat: next pair of list j
+  __device__ __forceinline__ void init(const GroupInfo& gb) {
+    a = 0;
+    b = gb.concat ? 0u : gb.bm[kGroupBlocks][0];
+  }
+  __device__ __forceinline__ int pop_union(const GroupInfo& gb, int W) {
+    while (b == 0u) {
+      if (++a >= W) return -1;
+      b = gb.bm[kGroupBlocks][a];
+    }
+    const int bit = __ffs(b) - 1;
+    b &= b - 1u;
+    return a * 32 + bit;
+  }
+  // Next tile: ids ka, kb, and the one query block that uses them in list
+  // order (owner), or -1 for the union, where each query block's bitmap says.
+  __device__ __forceinline__ void next(const GroupInfo& gb, const Params& p, int row0, int W, int& ka,
+                                       int& kb, int& owner) {
+    if (!gb.concat) {
+      ka = pop_union(gb, W);
+      kb = pop_union(gb, W);
+      owner = -1;
+      return;
+    }
+    while (a < kGroupBlocks && 2 * static_cast<int>(b) >= gb.cnt[a]) {
+      ++a;
+      b = 0u;
+    }
+    if (a >= kGroupBlocks) {  // past the last list (not reached: n_tiles counts the pairs)
+      ka = kb = owner = -1;
+      return;
+    }
+    const int t = 2 * static_cast<int>(b);
+    ka = row_block_id(p, row0 + a, t);
+    kb = t + 1 < gb.cnt[a] ? row_block_id(p, row0 + a, t + 1) : -1;
+    owner = a;
+    ++b;
+  }
+};
+
+// Whether query block j of the group uses block kb of a tile (kb < 0: no).
+__device__ __forceinline__ bool group_uses(const GroupInfo& gb, int owner, int j, int kb) {
+  if (kb < 0) return false;
+  if (owner >= 0) return owner == j;
+  return (gb.bm[j][kb >> 5] >> (kb & 31)) & 1u;
+}
+
+// Softmax of one 128-column S row whose halves (two 64-key blocks) may be
+// unselected (ha / hb false: those columns are ignored); log2 domain with the
+// lazy maximum of the kernel above.  Writes the 16-bit numerators into pk
+// (zero for an unselected half, whose maximum and exponentials are skipped)
+// and returns their sum.  One body for every case keeps the loop's code small.
+template <bool F16>
+__device__ __forceinline__ float softmax_halves(uint32_t (&sv)[128], bool ha, bool hb, float sl2, int t,
+                                                float& m_used, float& alpha, bool& rescale, uint32_t (&pk)[64]) {
+  float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    if (h == 0 ? ha : hb) {
+#pragma unroll
+      for (int c = 64 * h; c < 64 * h + 64; c += 8) {
+        a0 = max3f(a0, __uint_as_float(sv[c + 0]), __uint_as_float(sv[c + 1]));
+        a1 = max3f(a1, __uint_as_float(sv[c + 2]), __uint_as_float(sv[c + 3]));
+        a2 = max3f(a2, __uint_as_float(sv[c + 4]), __uint_as_float(sv[c + 5]));
+        a3 = max3f(a3, __uint_as_float(sv[c + 6]), __uint_as_float(sv[c + 7]));
+      }
+    }
+  }
+  const float mt = max3f(a0, a1, fmaxf(a2, a3)) * sl2;
+  const bool grow = mt > m_used + 8.0f;
+  rescale = grow && t > 0 && m_used != -INFINITY;
+  alpha = rescale ? ex2_approx(m_used - mt) : 1.0f;
+  if (grow) m_used = mt;
+  const float msub = (m_used == -INFINITY) ? 0.0f : m_used;
+  const uint64_t c2 = f2pack(sl2, sl2), nm2 = f2pack(-msub, -msub);
+  uint64_t acc0 = 0, acc1 = 0, acc2 = 0, acc3 = 0;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    if (h == 0 ? ha : hb) {
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) {
+        const int j = 32 * h + jj;
+        const uint64_t x = fma2(u2pack(sv[2 * j], sv[2 * j + 1]), c2, nm2);
+        uint64_t pp;
+        {
+          float xa, xb;
+          f2unpack(x, xa, xb);
+          pp = f2pack(ex2_approx(xa), ex2_approx(xb));
+        }
+        {
+          float p0, p1;
+          f2unpack(pp, p0, p1);
+          pk[j] = pack_half2<F16>(p0, p1);
+        }
+        switch (jj & 3) {
+          case 0: acc0 = add2(acc0, pp); break;
+          case 1: acc1 = add2(acc1, pp); break;
+          case 2: acc2 = add2(acc2, pp); break;
+          default: acc3 = add2(acc3, pp); break;
+        }
+      }
+    } else {
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) pk[32 * h + jj] = 0u;
+    }
+  }
+  float s0, s1, s2, s3, s4, s5, s6, s7;
+  f2unpack(acc0, s0, s1);
+  f2unpack(acc1, s2, s3);
+  f2unpack(acc2, s4, s5);
+  f2unpack(acc3, s6, s7);
+  return ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
+}
+
+template <bool F16>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_grouped64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem + kSmemQ;
+  uint8_t* sK = smem + kSmemK;
+  uint8_t* sV = smem + kSmemV;
+  GroupBarriers* bars = reinterpret_cast<GroupBarriers*>(smem + kSmemBar);
+  GroupInfo* grp = reinterpret_cast<GroupInfo*>(smem + kSmemGroups);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const Geo& g = p.g;
+  const int ngq = (g.NB + kGroupBlocks - 1) / kGroupBlocks;  // groups per head
+  const int total_groups = p.BH * ngq;
+  const int W = (g.NB + 31) >> 5;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    mbar_init(&bars->q_empty, 1);
+    for (int s = 0; s < kStagesK; ++s) {
+      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->k_empty[s], 1);
+    }
+    for (int s = 0; s < kStagesV; ++s) {
+      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->v_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->s_full[i], 1);
+      mbar_init(&bars->p_full[i], 128);
+      mbar_init(&bars->o_full[i], 1);
+      mbar_init(&bars->o_empty[i], 128);
+      mbar_init(&bars->grp_full[i], 1);
+      mbar_init(&bars->grp_free[i], kGroupConsumers);
+    }
+    mbar_init(&bars->drain, 1);
+    bars->abort = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp < 4) {
+  regs_dec<kRegsLow>();
+  if (warp == 2) {
+    // ------------------------------------------------------------ group builder
+    int gl = 0;
+    for (int gi = blockIdx.x; gi < total_groups; gi += gridDim.x, ++gl) {
+      const int buf = gl & 1;
+      if (gl >= 2 && !gwarp_wait(&bars->grp_free[buf], ((gl >> 1) - 1) & 1, bars, p.status)) break;
+      GroupInfo& gb = grp[buf];
+      for (int i = lane; i < (kGroupBlocks + 1) * kGroupMaxWords; i += 32) (&gb.bm[0][0])[i] = 0u;
+      __syncwarp();
+      const int bh = gi / ngq, qb0 = (gi - bh * ngq) * kGroupBlocks;
+      const int nqb = min(kGroupBlocks, g.NB - qb0);
+      bool repeat = false, bad = false;
+      int cnts[kGroupBlocks];
+#pragma unroll
+      for (int j = 0; j < kGroupBlocks; ++j) {
+        int c = 0;
+        if (j < nqb) {
+          const long long row = static_cast<long long>(bh) * g.NB + qb0 + j;
+          c = __ldg(p.num + row);
+          if (c < 0 || c > p.max_k) {
+            bad = true;
+            c = c < 0 ? 0 : p.max_k;
+          }
+          for (int t = lane; t < c; t += 32) {
+            const int kb = __ldg(p.idx + row * p.max_k + t);
+            if (kb < 0 || kb >= g.NB) {
+              bad = true;
+              continue;
+            }
+            const uint32_t bit = 1u << (kb & 31);
+            if (atomicOr(&gb.bm[j][kb >> 5], bit) & bit) repeat = true;
+          }
+        }
+        cnts[j] = c;
+      }
+      __syncwarp();
+      repeat = __any_sync(0xffffffffu, repeat);
+      bad = __any_sync(0xffffffffu, bad);
+      if (bad && lane == 0) atomicCAS(p.status, 0u, (unsigned)VSA_ERR_BAD_INDEX);
+      int U = 0;
+      for (int w = lane; w < W; w += 32) {
+        const uint32_t u = gb.bm[0][w] | gb.bm[1][w] | gb.bm[2][w] | gb.bm[3][w];
+        gb.bm[kGroupBlocks][w] = u;
+        U += __popc(u);
+      }
+      U = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(U)));
+      if (lane == 0) {
+        int n = 0;
+        if (repeat) {
+#pragma unroll
+          for (int j = 0; j < kGroupBlocks; ++j) n += (cnts[j] + 1) / 2;
+        } else {
+          n = (U + 1) / 2;
+        }
+        gb.concat = repeat ? 1 : 0;
+        gb.n_tiles = n;
+        gb.nq = (nqb + 1) / 2;
+#pragma unroll
+        for (int j = 0; j < kGroupBlocks; ++j) gb.cnt[j] = cnts[j];
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->grp_full[buf]);
+    }
+  } else if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    const uint64_t pol_kv = policy_evict_last();
+    const uint64_t pol_q = policy_evict_first();
+    int kit = 0, vit = 0, qit = 0, gl = 0;
+    bool stop = false;
+    for (int gi = blockIdx.x; gi < total_groups && !stop; gi += gridDim.x, ++gl) {
+      const int buf = gl & 1;
+      if (!gwarp_wait(&bars->grp_full[buf], (gl >> 1) & 1, bars, p.status)) break;
+      const GroupInfo& gb = grp[buf];
+      const int n = gb.n_tiles, nq = gb.nq;
+      const int bh = gi / ngq, qb0 = (gi - bh * ngq) * kGroupBlocks;
+      const long long base = static_cast<long long>(bh) * g.Sp;
+      const int row0 = bh * g.NB + qb0;
+      if (n > 0) {
+        if (!gwarp_wait(&bars->q_empty, (qit & 1) ^ 1, bars, p.status)) break;
+        mbar_arrive_expect_tx_w(&bars->q_full, nq * kTileBytes);
+        const int qrow = static_cast<int>(base + static_cast<long long>(qb0) * 64);
+        for (int i = 0; i < nq; ++i)
+          for (int hf = 0; hf < 2; ++hf)
+            tma_load_2d_w(sQ + i * kTileBytes + hf * kHalfBytes, &tm_q, hf * 64, qrow + i * 128, &bars->q_full,
+                          pol_q);
+        ++qit;
+        GroupWalk walk;
+        walk.init(gb);
+        for (int t = 0; t < n; ++t) {
+          int ka, kb, owner;
+          walk.next(gb, p, row0, W, ka, kb, owner);
+          // absent or unusable blocks load block 0 (finite data, masked by every warp)
+          const int krow0 = static_cast<int>(base + static_cast<long long>(ka < 0 ? 0 : ka) * 64);
+          const int krow1 = static_cast<int>(base + static_cast<long long>(kb < 0 ? 0 : kb) * 64);
+          const int sk = kit % kStagesK;
+          if (!gwarp_wait(&bars->k_empty[sk], ((kit / kStagesK) & 1) ^ 1, bars, p.status)) {
+            stop = true;
+            break;
+          }
+          mbar_arrive_expect_tx_w(&bars->k_full[sk], kTileBytes);
+          for (int hf = 0; hf < 2; ++hf) {
+            uint8_t* dst = sK + sk * kTileBytes + hf * kHalfBytes;
+            tma_load_2d_w(dst, &tm_k, hf * 64, krow0, &bars->k_full[sk], pol_kv);
+            tma_load_2d_w(dst + kHalfBytes / 2, &tm_k, hf * 64, krow1, &bars->k_full[sk], pol_kv);
+          }
+          ++kit;
+          const int sv = vit % kStagesV;
+          if (!gwarp_wait(&bars->v_empty[sv], ((vit / kStagesV) & 1) ^ 1, bars, p.status)) {
+            stop = true;
+            break;
+          }
+          mbar_arrive_expect_tx_w(&bars->v_full[sv], kTileBytes);
+          for (int hf = 0; hf < 2; ++hf) {
+            uint8_t* dst = sV + sv * kTileBytes + hf * kHalfBytes;
+            tma_load_2d_w(dst, &tm_v, hf * 64, krow0, &bars->v_full[sv], pol_kv);
+            tma_load_2d_w(dst + kHalfBytes / 2, &tm_v, hf * 64, krow1, &bars->v_full[sv], pol_kv);
+          }
+          ++vit;
+        }
+        if (stop) break;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->grp_free[buf]);
+    }
+    // Drain: every issued copy must land before the CTA's shared memory is released.
+    if (qit > 0) mbar_wait_drain(&bars->q_full, (qit - 1) & 1, kTimeoutNs);
+    for (int s = 0; s < kStagesK; ++s)
+      if (kit > s) {
+        const int last = kit - 1 - ((kit - 1 - s) % kStagesK);
+        mbar_wait_drain(&bars->k_full[s], (last / kStagesK) & 1, kTimeoutNs);
+      }
+    for (int s = 0; s < kStagesV; ++s)
+      if (vit > s) {
+        const int last = vit - 1 - ((vit - 1 - s) % kStagesV);
+        mbar_wait_drain(&bars->v_full[s], (last / kStagesV) & 1, kTimeoutNs);
+      }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint64_t dq0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
+    const uint64_t dk0 = sdesc_sw128(smem_u32(sK), 16, 1024);
+    const uint64_t dv0 = sdesc_sw128(smem_u32(sV), kHalfBytes, 1024);
+    constexpr uint64_t kTileDesc = kTileBytes >> 4;
+    int kit = 0, vit = 0, qit = 0, gl = 0;
+    int tiles[2] = {0, 0}, items[2] = {0, 0};
+    bool ok = true;
+    auto issue_s = [&](int i, int sk) {
+      const uint32_t d = tmem + i * 128;
+      const uint64_t a = dq0 + i * kTileDesc, b = dk0 + sk * kTileDesc;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t off = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+        mma_ss_w(d, a + off, b + off, Idesc<F16>::S, kk > 0 ? 1u : 0u);
+      }
+    };
+    auto issue_pv = [&](int i, int sv, bool acc) {
+      const uint32_t d = tmem + 256 + i * 128, pa = tmem + i * 128;
+      const uint64_t b = dv0 + sv * kTileDesc;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_ts_w(d, pa + kk * 8, b + kk * (2048 >> 4), Idesc<F16>::PV, (acc || kk > 0) ? 1u : 0u);
+    };
+    for (int gi = blockIdx.x; gi < total_groups && ok; gi += gridDim.x, ++gl) {
+      const int buf = gl & 1;
+      if (!(ok = gwarp_wait(&bars->grp_full[buf], (gl >> 1) & 1, bars, p.status))) break;
+      const int n = grp[buf].n_tiles, nq = grp[buf].nq;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->grp_free[buf]);
+      if (n == 0) continue;
+      if (!(ok = gwarp_wait(&bars->q_full, qit & 1, bars, p.status))) break;
+      ++qit;
+      tc_fence_after();
+      int sk = kit % kStagesK;
+      if (!(ok = gwarp_wait(&bars->k_full[sk], (kit / kStagesK) & 1, bars, p.status))) break;
+      tc_fence_after();
+      issue_s(0, sk);
+      mma_commit_w(&bars->s_full[0]);
+      if (nq == 2) {
+        issue_s(1, sk);
+        mma_commit_w(&bars->s_full[1]);
+      }
+      mma_commit_w(&bars->k_empty[sk]);
+      // Q is read by the S products only: once the group's last S is issued,
+      // the next group's Q may load while the last P V products run
+      if (n == 1) mma_commit_w(&bars->q_empty);
+      ++kit;
+      for (int t = 0; t < n; ++t) {
+        const int sv = vit % kStagesV;
+        if (!(ok = gwarp_wait(&bars->v_full[sv], (vit / kStagesV) & 1, bars, p.status))) break;
+        if (!(ok = gwarp_wait(&bars->p_full[0], tiles[0] & 1, bars, p.status))) break;
+        if (t == 0 && !(ok = gwarp_wait(&bars->o_empty[0], (items[0] & 1) ^ 1, bars, p.status))) break;
+        tc_fence_after();
+        issue_pv(0, sv, t > 0);
+        ++tiles[0];
+        if (t == n - 1) mma_commit_w(&bars->o_full[0]);
+        const bool more = t + 1 < n;
+        sk = kit % kStagesK;
+        if (more) {
+          if (!(ok = gwarp_wait(&bars->k_full[sk], (kit / kStagesK) & 1, bars, p.status))) break;
+          tc_fence_after();
+          issue_s(0, sk);
+          mma_commit_w(&bars->s_full[0]);
+        }
+        if (nq == 2) {
+          if (!(ok = gwarp_wait(&bars->p_full[1], tiles[1] & 1, bars, p.status))) break;
+          if (t == 0 && !(ok = gwarp_wait(&bars->o_empty[1], (items[1] & 1) ^ 1, bars, p.status))) break;
+          tc_fence_after();
+          issue_pv(1, sv, t > 0);
+          ++tiles[1];
+        }
+        mma_commit_w(&bars->v_empty[sv]);
+        ++vit;
+        if (nq == 2 && t == n - 1) mma_commit_w(&bars->o_full[1]);
+        if (more) {
+          if (nq == 2) {
+            issue_s(1, sk);
+            mma_commit_w(&bars->s_full[1]);
+          }
+          mma_commit_w(&bars->k_empty[sk]);
+          if (t + 2 == n) mma_commit_w(&bars->q_empty);
+          ++kit;
+        }
+      }
+      if (!ok) break;
+      ++items[0];
+      if (nq == 2) ++items[1];
+    }
+    // Drain: wait for every MMA issued by this thread before TMEM and smem go away.
+    mma_commit_w(&bars->drain);
+    mbar_wait_drain(&bars->drain, 0, kTimeoutNs);
+  }
+  } else {
+    regs_inc<kRegsHigh>();
+    // ------------------------------------------------------------ softmax + epilogue
+    const int wg = (warp - 4) >> 2;  // Q tile
+    const int quarter = warp & 3;    // TMEM lane quarter of this warp
+    const int jq = 2 * wg + (quarter >> 1);  // query block of the group this warp serves
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_off + wg * 128;
+    const uint32_t tO = tmem + lane_off + 256 + wg * 128;
+    const float sl2 = p.scale_log2;
+    int tiles = 0, items = 0, gl = 0;
+    bool ok = true;
+    for (int gi = blockIdx.x; gi < total_groups && ok; gi += gridDim.x, ++gl) {
+      const int buf = gl & 1;
+      if (!(ok = gwarp_wait(&bars->grp_full[buf], (gl >> 1) & 1, bars, p.status))) break;
+      const GroupInfo& gb = grp[buf];
+      const int n = gb.n_tiles, nq = gb.nq;
+      const int bh = gi / ngq, qb0 = (gi - bh * ngq) * kGroupBlocks;
+      const int row0 = bh * g.NB + qb0;  // index row of the group's first query block (NB <= kGroupMaxNB)
+      if (wg >= nq || n == 0) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->grp_free[buf]);
+        if (wg < nq) {  // nothing selected by any query block of the group
+          const long long row = static_cast<long long>(bh) * g.Sp + static_cast<long long>(qb0) * 64 + wg * 128 + r;
+          uint4* orow = reinterpret_cast<uint4*>(p.o + row * 128);
+#pragma unroll
+          for (int c = 0; c < 16; ++c) orow[c] = make_uint4(0, 0, 0, 0);
+          p.lse[row] = -INFINITY;
+        }
+        continue;
+      }
+      float m_used = -INFINITY, l = 0.0f;
+      GroupWalk walk;
+      walk.init(gb);
+      for (int t = 0; t < n; ++t) {
+        int ka, kb, owner;
+        walk.next(gb, p, row0, W, ka, kb, owner);
+        // this warp's query block: which halves of the tile it selected
+        const int sa = group_uses(gb, owner, jq, ka) ? ka : -1;
+        const int sb = group_uses(gb, owner, jq, kb) ? kb : -1;
+        uint32_t w0 = 0, w1 = 0, w2 = 0, w3 = 0;
+        const int st_a = block64_mask(g, sa, w0, w1);
+        const int st_b = block64_mask(g, sb, w2, w3);
+        if (!(ok = gwarp_wait(&bars->s_full[wg], tiles & 1, bars, p.status))) break;
+        tc_fence_after();
+        uint32_t pk[64];
+        float lsum = 0.0f, alpha = 1.0f;
+        bool rescale = false;
+        const bool ha = st_a != kTileEmpty, hb = st_b != kTileEmpty;
+        if (ha || hb) {
+          uint32_t sv[128];  // an unselected half holds finite S values; the mask below overwrites them
+          tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+          tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+          tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
+          tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
+          tmem_wait_ld();
+          if (st_a == kTilePartial || st_b == kTilePartial) {
+            // padded slots of a selected block (an unselected half is skipped below)
+            const uint32_t mw[4] = {st_a == kTilePartial ? w0 : 0xffffffffu, st_a == kTilePartial ? w1 : 0xffffffffu,
+                                    st_b == kTilePartial ? w2 : 0xffffffffu, st_b == kTilePartial ? w3 : 0xffffffffu};
+            apply_key_mask(sv, mw);
+          }
+          lsum = softmax_halves<F16>(sv, ha, hb, sl2, t, m_used, alpha, rescale, pk);
+        } else {
+          // nothing selected in this tile by this warp's query block
+#pragma unroll
+          for (int j = 0; j < 64; ++j) pk[j] = 0u;
+        }
+        l = l * alpha + lsum;
+        tmem_st32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+        tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+        // Rescale this row of O when its maximum moved (warp-uniform branch).
+        // PV(t-1) is complete: the s_full commit just waited on follows it.
+        if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t ov[32];
+            tmem_ld32(tO + c * 32, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha);
+            tmem_st32(tO + c * 32, ov);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bars->p_full[wg]);
+        ++tiles;
+      }
+      if (!ok) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->grp_free[buf]);
+      // epilogue: O / l -> 16-bit row, lse
+      if (!(ok = gwarp_wait(&bars->o_full[wg], items & 1, bars, p.status))) break;
+      tc_fence_after();
+      const long long row = static_cast<long long>(bh) * g.Sp + static_cast<long long>(qb0) * 64 + wg * 128 + r;
+      uint4* orow = reinterpret_cast<uint4*>(p.o + row * 128);
+      const float inv = l > 0.0f ? 1.0f / l : 0.0f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t ov[32];
+        tmem_ld32(tO + c * 32, ov);
+        tmem_wait_ld();
+        uint4 w[4];
+        uint32_t* wp = reinterpret_cast<uint32_t*>(w);
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          wp[j] = pack_half2<F16>(__uint_as_float(ov[2 * j]) * inv, __uint_as_float(ov[2 * j + 1]) * inv);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) orow[c * 4 + j] = w[j];
+      }
+      tc_fence_before();
+      mbar_arrive(&bars->o_empty[wg]);
+      p.lse[row] = l > 0.0f ? (m_used + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+      ++items;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_attn_fwd_grouped64(const Geo& g, const CUtensorMap& tq, const CUtensorMap& tk,
+                                      const CUtensorMap& tv, const fwd::Params& p, int BH, int num_sms, bool f16,
+                                      cudaStream_t stream) {
+  const long long groups = static_cast<long long>(BH) * ((g.NB + kGroupBlocks - 1) / kGroupBlocks);
+  const int grid = static_cast<int>(groups < num_sms ? groups : num_sms);
+  auto kern = f16 ? attn_fwd_grouped64_kernel<true> : attn_fwd_grouped64_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTotalG);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreads, kSmemTotalG, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace vsa
