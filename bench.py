@@ -670,6 +670,22 @@ def main():
     attn_avg = max_over_ranks(float(np.mean(attn_s)))
     assert vsa.get_status() == vsa.VSA_OK
 
+    # ---- the same steps replayed from a CUDA graph of one step (launch gaps
+    # removed; reported beside the eager figure, which the roofline uses)
+    cg = fwd.graph(dev["q"], dev["k"], dev["v"], dev.get("map"), dev.get("gate"), row_keep=dev.get("row_keep"))
+    for _ in range(3):
+        cg.replay()
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sync_all()
+    g0.record(stream)
+    for _ in range(args.steps):
+        cg.replay()
+    g1.record(stream)
+    sync_all()
+    graph_elapsed = max_over_ranks(g0.elapsed_time(g1) / 1e3)
+    assert vsa.get_status() == vsa.VSA_OK
+    del cg
+
     # ---- end to end through the public API with pinned host buffers: every step
     # copies its q, k, v in and its o out; vsa.HostPipeline overlaps step i's
     # compute with step i+1's upload and step i-1's download (two copy streams)
@@ -773,6 +789,9 @@ def main():
                     "api": "vsa.HostPipeline (copies of neighbouring steps overlap the compute)",
                     "serial_ms_per_step": serial_elapsed / args.steps * 1e3},
             "gpu_launches": args.steps * fwd.launches(wl.map_driven),
+            "graph": {"value": world * flops * args.steps / graph_elapsed / 1e12, "unit": "TFLOP/s",
+                      "ms_per_step": graph_elapsed / args.steps * 1e3,
+                      "how": "the same step captured once in a CUDA graph (vsa.Forward.graph), replayed per step"},
         }
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline_sample(wl, nvfp4=args.nvfp4)

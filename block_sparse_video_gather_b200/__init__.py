@@ -599,6 +599,21 @@ class Forward:
         self.fine()
         return self.back(gate, out), self.lse
 
+    def graph(self, q, k, v, block_map=None, gate=None, row_keep=None):
+        """Capture one forward step on these device tensors in a CUDA graph and
+        return it (torch.cuda.CUDAGraph); replay() reruns the step's launches
+        with the inputs read from the same buffers and o / lse written to
+        self.o / self.lse.  One eager step runs first so that every host-side
+        set-up (device state, tensor-map encoder, kernel attributes) happens
+        outside the capture."""
+        torch = _torch()
+        self(q, k, v, block_map, gate, row_keep=row_keep)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self(q, k, v, block_map, gate, row_keep=row_keep)
+        return g
+
     def launches(self, block_map: bool = False) -> int:
         """Kernels one call launches."""
         quant = 2 if self.nvfp4 else 0  # q and k quantisation

@@ -43,3 +43,33 @@ def test_pipelined_steps_match_sequential_steps(gated):
         torch.cuda.synchronize()
         assert torch.equal(o.view(torch.int16), ref.cpu().view(torch.int16))
     assert not torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+
+
+@pytest.mark.parametrize("name", ["tiny", "tile64", "tile64map"])
+def test_graph_replay_matches_eager_steps(name):
+    """vsa.Forward.graph: a CUDA graph of one step, replayed after the inputs
+    change in place, gives bit for bit what an eager step gives (the one-launch
+    front end's counters are back at zero after each replay)."""
+    wl = workloads.WORKLOADS[name]
+    plan = vsa.Plan.of(wl)
+    fwd = vsa.Forward(plan, wl.B, wl.H, wl.topk, prefix_dense=wl.prefix_dense)
+    dev = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).cuda().view(torch.bfloat16)
+    inp = workloads.make_inputs(wl)
+    q, k, v = dev(inp["q"]), dev(inp["k"]), dev(inp["v"])
+    bmap = torch.from_numpy(inp["map"]).cuda() if wl.map_driven else None
+    keep = torch.from_numpy(inp["row_keep"]).cuda() if inp["row_keep"] is not None else None
+    g = fwd.graph(q, k, v, bmap, row_keep=keep)
+    fields = {f: getattr(wl, f) for f in wl.__dataclass_fields__ if f != "name"}
+    other = workloads.make_inputs(workloads.custom(name="other", **{**fields, "seed": 7}))
+    for src in (other, inp):
+        q.copy_(dev(src["q"])), k.copy_(dev(src["k"])), v.copy_(dev(src["v"]))
+        g.replay()
+        torch.cuda.synchronize()
+        got_o, got_lse, got_idx = fwd.o.clone(), fwd.lse.clone(), fwd.idx.clone()
+        ref_o, ref_lse = fwd(q, k, v, bmap, row_keep=keep)
+        torch.cuda.synchronize()
+        assert vsa.get_status() == vsa.VSA_OK
+        assert torch.equal(got_idx, fwd.idx)
+        assert torch.equal(got_o.view(torch.int16), ref_o.view(torch.int16))
+        assert torch.equal(got_lse.view(torch.int32), ref_lse.view(torch.int32))
+        assert int(fwd.ws.abs().sum()) == 0
