@@ -29,7 +29,7 @@ SYMBOLS = (
     "vsa_sparse_attn_fwd", "vsa_sparse_attn_fwd_ex", "vsa_get_status", "vsa_strerror",
     "vsa_coarse_compress", "vsa_untile_gate", "vsa_tile_coarse", "vsa_tile_coarse_static",
     "vsa_sparse_attn_bwd_workspace", "vsa_sparse_attn_bwd", "vsa_quantize_nvfp4", "vsa_sparse_attn_fwd_nvfp4",
-    "vsa_coarse_topk_prefix", "vsa_tile_coarse_prefix",
+    "vsa_coarse_topk_prefix", "vsa_tile_coarse_prefix", "vsa_sparse_attn_fwd_ws",
 )
 
 VSA_BF16 = 0
@@ -71,6 +71,7 @@ def lib():
         L.vsa_tile.argtypes = [P, P, P, P, i, i, i, P]
         L.vsa_tile_ex.argtypes = [P, i, P, P, P, i, i, i, P]
         L.vsa_sparse_attn_fwd_ex.argtypes = [P, i, P, P, P, P, P, i, i, i, i, P, P, P]
+        L.vsa_sparse_attn_fwd_ws.argtypes = [P, i, P, P, P, P, P, i, i, i, i, P, P, P, P]
         L.vsa_untile.argtypes = [P, P, P, i, i, i, P]
         L.vsa_coarse_topk.argtypes = [P, P, P, i, i, i, i, P, P, P]
         L.vsa_map_to_index.argtypes = [P, i, i, i, i, P, P, P]
@@ -361,8 +362,10 @@ def map_to_index(block_map, idx_out=None, num_out=None):
     return idx_out, num_out
 
 
-def sparse_attn_fwd(plan: Plan, q, k, v, q2k_idx, q2k_num, o_out=None, lse_out=None):
-    """Attention of every query block over its selected blocks (tiled layout) -> (o, lse)."""
+def sparse_attn_fwd(plan: Plan, q, k, v, q2k_idx, q2k_num, o_out=None, lse_out=None, workspace=None):
+    """Attention of every query block over its selected blocks (tiled layout) -> (o, lse).
+    workspace: optional zeroed int32 tensor of 4 entries (2 used) for the 64-token
+    kernel's shared work queue (vsa_sparse_attn_fwd_ws); left zero by every call."""
     torch = _torch()
     B, H, Sp, D = q.shape
     max_k = q2k_idx.shape[-1]
@@ -371,11 +374,14 @@ def sparse_attn_fwd(plan: Plan, q, k, v, q2k_idx, q2k_num, o_out=None, lse_out=N
         o_out = torch.empty_like(q)
     if lse_out is None:
         lse_out = torch.empty((B, H, Sp), dtype=torch.float32, device=q.device)
-    _check(lib().vsa_sparse_attn_fwd_ex(plan.handle, code, _ptr(q, q.dtype, "q"), _ptr(k, q.dtype, "k"),
-                                        _ptr(v, q.dtype, "v"), _ptr(q2k_idx, torch.int32, "q2k_idx"),
-                                        _ptr(q2k_num, torch.int32, "q2k_num"), max_k, B, H, D,
-                                        _ptr(o_out, q.dtype, "o"), _ptr(lse_out, torch.float32, "lse"),
-                                        _stream()), "vsa_sparse_attn_fwd")
+    args = (plan.handle, code, _ptr(q, q.dtype, "q"), _ptr(k, q.dtype, "k"), _ptr(v, q.dtype, "v"),
+            _ptr(q2k_idx, torch.int32, "q2k_idx"), _ptr(q2k_num, torch.int32, "q2k_num"), max_k, B, H, D,
+            _ptr(o_out, q.dtype, "o"), _ptr(lse_out, torch.float32, "lse"))
+    if workspace is None:
+        _check(lib().vsa_sparse_attn_fwd_ex(*args, _stream()), "vsa_sparse_attn_fwd")
+    else:
+        _check(lib().vsa_sparse_attn_fwd_ws(*args, _ptr(workspace, torch.int32, "workspace"), _stream()),
+               "vsa_sparse_attn_fwd_ws")
     return o_out, lse_out
 
 
@@ -512,6 +518,7 @@ class Forward:
             self.oc = torch.empty((B, H, plan.NB, D), dtype=torch.float32, device=device)
         if fused:
             self.ws = workspace(B, H, device)
+        self.fws = torch.zeros(4, dtype=torch.int32, device=device)  # the fine stage's work queue
         if nvfp4:
             u8 = dict(dtype=torch.uint8, device=device)
             self.qc = torch.empty((B, H, plan.Sp, D // 2), **u8)
@@ -577,7 +584,7 @@ class Forward:
                                   o_out=self.ot, lse_out=self.lse)
         else:
             sparse_attn_fwd(self.plan, self.qt, self.kt, self.vt, self.idx, self.num, o_out=self.ot,
-                            lse_out=self.lse)
+                            lse_out=self.lse, workspace=self.fws)
 
     def fine(self):
         self.quantize()

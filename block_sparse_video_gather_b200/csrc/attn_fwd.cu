@@ -458,6 +458,7 @@ cudaError_t launch_attn_fwd(const Geo& g, const AttnArgs& a, cudaStream_t stream
   p.status = a.status;
   p.scale_log2 = static_cast<float>(1.4426950408889634 / 11.313708498984761);  // log2(e) / sqrt(128)
   p.g = g;
+  p.queue = a.queue;
   if (g.bs == 64 && g.NB <= kGroupMaxNB)  // groups of four query blocks over their union
     return launch_attn_fwd_grouped64(g, tq, tk, tv, p, a.BH, a.num_sms, a.f16, stream);
   const long long items = static_cast<long long>(a.BH) * g.NB;

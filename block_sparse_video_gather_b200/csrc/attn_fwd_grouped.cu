@@ -44,6 +44,13 @@ using namespace fwd;
 // each query block's list, two ids per tile, only that block's rows unmasked),
 // so a repeated id counts twice as in the ungrouped kernel.
 //
+// Groups go to CTAs statically (every gridDim.x-th group) or, with a caller
+// workspace, through a shared queue: the builder takes tickets with an atomic
+// add, the groups holding prefix query tiles first (dense under the tile-64
+// rule, the longest), and publishes an end marker past the last group; the
+// last CTA to finish resets the counters.  Either way the consumers stop on
+// the end marker.
+//
 // The bitmaps hold kGroupMaxNB blocks: the host uses this kernel for
 // 64-token blocks when NB <= kGroupMaxNB.
 // ===========================================================================
@@ -56,7 +63,7 @@ struct GroupInfo {
   int n_tiles;  // 128-key tiles of the group's key stream
   int nq;       // 128-row query tiles (1 for a group of two query blocks)
   int cnt[kGroupBlocks];
-  int pad;
+  int gi;       // the group (b*h * groups per head + query block / 4), -1: no more groups
   uint32_t bm[kGroupBlocks + 1][kGroupMaxWords];  // selection bitmaps; [kGroupBlocks] = union
 };
 
@@ -81,6 +88,16 @@ __device__ __forceinline__ bool gwarp_wait(uint64_t* bar, uint32_t parity, Group
                                            unsigned int* status) {
   bool ok = mbar_wait(bar, parity, &bars->abort, status, kTimeoutNs);
   return __all_sync(0xffffffffu, ok);
+}
+
+// Group of ticket d of a shared queue: the groups holding prefix query tiles
+// (dense under the tile-64 rule, the longest) of every head first, then the
+// others head by head -- the longest work is handed out first.
+__device__ __forceinline__ int queue_group(const Geo& g, int BH, int ngq, int d) {
+  const int npq = min(ngq, (g.n_pre + kGroupBlocks - 1) / kGroupBlocks);
+  if (d < BH * npq) return (d / npq) * ngq + d % npq;
+  const int e = d - BH * npq, nv = ngq - npq;
+  return (e / nv) * ngq + npq + e % nv;
 }
 
 // Block id at position t of index row `row`, or -1 when outside [0, NB).
@@ -263,11 +280,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   regs_dec<kRegsLow>();
   if (warp == 2) {
     // ------------------------------------------------------------ group builder
-    int gl = 0;
-    for (int gi = blockIdx.x; gi < total_groups; gi += gridDim.x, ++gl) {
+    for (int gl = 0;; ++gl) {
+      // the next group: a ticket of the shared queue, or every gridDim.x-th group
+      int gi;
+      if (p.queue) {
+        int tk = 0;
+        if (lane == 0) tk = atomicAdd(p.queue, 1);
+        tk = __shfl_sync(0xffffffffu, tk, 0);
+        gi = tk < total_groups ? queue_group(g, p.BH, ngq, tk) : -1;
+      } else {
+        gi = blockIdx.x + gl * static_cast<int>(gridDim.x);
+        if (gi >= total_groups) gi = -1;
+      }
       const int buf = gl & 1;
       if (gl >= 2 && !gwarp_wait(&bars->grp_free[buf], ((gl >> 1) - 1) & 1, bars, p.status)) break;
       GroupInfo& gb = grp[buf];
+      if (gi < 0) {  // past the last group: an end marker for the consumers
+        if (lane == 0) gb.gi = -1;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->grp_full[buf]);
+        break;
+      }
       for (int i = lane; i < (kGroupBlocks + 1) * kGroupMaxWords; i += 32) (&gb.bm[0][0])[i] = 0u;
       __syncwarp();
       const int bh = gi / ngq, qb0 = (gi - bh * ngq) * kGroupBlocks;
@@ -315,6 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           n = (U + 1) / 2;
         }
+        gb.gi = gi;
         gb.concat = repeat ? 1 : 0;
         gb.n_tiles = n;
         gb.nq = (nqb + 1) / 2;
@@ -331,12 +365,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tm_v);
     const uint64_t pol_kv = policy_evict_last();
     const uint64_t pol_q = policy_evict_first();
-    int kit = 0, vit = 0, qit = 0, gl = 0;
+    int kit = 0, vit = 0, qit = 0;
     bool stop = false;
-    for (int gi = blockIdx.x; gi < total_groups && !stop; gi += gridDim.x, ++gl) {
+    for (int gl = 0; !stop; ++gl) {
       const int buf = gl & 1;
       if (!gwarp_wait(&bars->grp_full[buf], (gl >> 1) & 1, bars, p.status)) break;
       const GroupInfo& gb = grp[buf];
+      const int gi = gb.gi;
+      if (gi < 0) break;
       const int n = gb.n_tiles, nq = gb.nq;
       const int bh = gi / ngq, qb0 = (gi - bh * ngq) * kGroupBlocks;
       const long long base = static_cast<long long>(bh) * g.Sp;
@@ -406,7 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t dk0 = sdesc_sw128(smem_u32(sK), 16, 1024);
     const uint64_t dv0 = sdesc_sw128(smem_u32(sV), kHalfBytes, 1024);
     constexpr uint64_t kTileDesc = kTileBytes >> 4;
-    int kit = 0, vit = 0, qit = 0, gl = 0;
+    int kit = 0, vit = 0, qit = 0;
     int tiles[2] = {0, 0}, items[2] = {0, 0};
     bool ok = true;
     auto issue_s = [&](int i, int sk) {
@@ -425,9 +461,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int kk = 0; kk < 8; ++kk)
         mma_ts_w(d, pa + kk * 8, b + kk * (2048 >> 4), Idesc<F16>::PV, (acc || kk > 0) ? 1u : 0u);
     };
-    for (int gi = blockIdx.x; gi < total_groups && ok; gi += gridDim.x, ++gl) {
+    for (int gl = 0; ok; ++gl) {
       const int buf = gl & 1;
       if (!(ok = gwarp_wait(&bars->grp_full[buf], (gl >> 1) & 1, bars, p.status))) break;
+      if (grp[buf].gi < 0) break;
       const int n = grp[buf].n_tiles, nq = grp[buf].nq;
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->grp_free[buf]);
@@ -505,12 +542,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tS = tmem + lane_off + wg * 128;
     const uint32_t tO = tmem + lane_off + 256 + wg * 128;
     const float sl2 = p.scale_log2;
-    int tiles = 0, items = 0, gl = 0;
+    int tiles = 0, items = 0;
     bool ok = true;
-    for (int gi = blockIdx.x; gi < total_groups && ok; gi += gridDim.x, ++gl) {
+    for (int gl = 0; ok; ++gl) {
       const int buf = gl & 1;
       if (!(ok = gwarp_wait(&bars->grp_full[buf], (gl >> 1) & 1, bars, p.status))) break;
       const GroupInfo& gb = grp[buf];
+      const int gi = gb.gi;
+      if (gi < 0) break;
       const int n = gb.n_tiles, nq = gb.nq;
       const int bh = gi / ngq, qb0 = (gi - bh * ngq) * kGroupBlocks;
       const int row0 = bh * g.NB + qb0;  // index row of the group's first query block (NB <= kGroupMaxNB)
@@ -619,6 +658,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+  // the last CTA to finish leaves the queue's counters at zero for the next call
+  // (every CTA has taken its last ticket by now)
+  if (p.queue && threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(p.queue + 1, 1) == static_cast<int>(gridDim.x) - 1) {
+      p.queue[0] = 0;
+      p.queue[1] = 0;
+    }
   }
 }
 

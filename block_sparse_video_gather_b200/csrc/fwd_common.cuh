@@ -62,6 +62,10 @@ struct Params {
   unsigned int* status;
   float scale_log2;
   Geo g;
+  // grouped 64-token kernel: a shared group queue (2 int32 of caller memory,
+  // ticket and finished-CTA counters, zero on entry and again on exit), or
+  // null for a static assignment of groups to CTAs
+  int* queue;
 };
 
 // Number of selected blocks of an item (clamped into [0, max_k]).

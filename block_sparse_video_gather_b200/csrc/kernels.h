@@ -57,7 +57,8 @@ struct AttnArgs {
   float* lse;
   unsigned int* status;
   int num_sms;
-  bool f16;  // fp16 tensors (else bf16)
+  bool f16;    // fp16 tensors (else bf16)
+  int* queue;  // 2 int32 of caller memory for the grouped kernel's shared queue, or null
 };
 cudaError_t launch_attn_fwd(const Geo& g, const AttnArgs& a, cudaStream_t stream);
 

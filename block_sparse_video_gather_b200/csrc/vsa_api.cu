@@ -422,9 +422,10 @@ int vsa_map_to_index(const uint8_t* map, int B, int H, int NQ, int NK, int32_t* 
   return from_cuda(vsa::launch_map_to_index(map, rows, NK, q2k_idx, q2k_num, reinterpret_cast<cudaStream_t>(stream)));
 }
 
-int vsa_sparse_attn_fwd_ex(vsa_plan_t plan, vsa_dtype_t dtype, const uint16_t* q, const uint16_t* k,
-                           const uint16_t* v, const int32_t* q2k_idx, const int32_t* q2k_num, int max_k, int B, int H,
-                           int D, uint16_t* o, float* lse, vsa_stream_t stream) {
+namespace {
+int sparse_attn_fwd_impl(vsa_plan_t plan, vsa_dtype_t dtype, const uint16_t* q, const uint16_t* k,
+                         const uint16_t* v, const int32_t* q2k_idx, const int32_t* q2k_num, int max_k, int B, int H,
+                         int D, uint16_t* o, float* lse, int32_t* queue, vsa_stream_t stream) {
   if (dtype != VSA_BF16 && dtype != VSA_F16) return VSA_ERR_INVALID_ARG;
   if (!plan || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return VSA_ERR_INVALID_ARG;
@@ -447,7 +448,22 @@ int vsa_sparse_attn_fwd_ex(vsa_plan_t plan, vsa_dtype_t dtype, const uint16_t* q
   a.status = ds->status;
   a.num_sms = ds->num_sms;
   a.f16 = dtype == VSA_F16;
+  a.queue = queue;
   return from_cuda(vsa::launch_attn_fwd(g, a, reinterpret_cast<cudaStream_t>(stream)));
+}
+}  // namespace
+
+int vsa_sparse_attn_fwd_ex(vsa_plan_t plan, vsa_dtype_t dtype, const uint16_t* q, const uint16_t* k,
+                           const uint16_t* v, const int32_t* q2k_idx, const int32_t* q2k_num, int max_k, int B, int H,
+                           int D, uint16_t* o, float* lse, vsa_stream_t stream) {
+  return sparse_attn_fwd_impl(plan, dtype, q, k, v, q2k_idx, q2k_num, max_k, B, H, D, o, lse, nullptr, stream);
+}
+
+int vsa_sparse_attn_fwd_ws(vsa_plan_t plan, vsa_dtype_t dtype, const uint16_t* q, const uint16_t* k,
+                           const uint16_t* v, const int32_t* q2k_idx, const int32_t* q2k_num, int max_k, int B, int H,
+                           int D, uint16_t* o, float* lse, int32_t* workspace, vsa_stream_t stream) {
+  if (!aligned16(workspace)) return VSA_ERR_INVALID_ARG;
+  return sparse_attn_fwd_impl(plan, dtype, q, k, v, q2k_idx, q2k_num, max_k, B, H, D, o, lse, workspace, stream);
 }
 
 int vsa_sparse_attn_fwd(vsa_plan_t plan, const uint16_t* q, const uint16_t* k, const uint16_t* v,

@@ -311,6 +311,26 @@ VSA_API int vsa_sparse_attn_fwd_ex(vsa_plan_t plan, vsa_dtype_t dtype, const uin
                                    vsa_stream_t stream);
 
 /*
+ * vsa_sparse_attn_fwd_ex with a caller workspace that lets the 64-token
+ * fine stage (four query blocks per work item over the union of their
+ * selections) hand out its work items from a shared queue -- the items whose
+ * query blocks are prefix tiles (dense under the tile-64 rule) first -- instead
+ * of a fixed item-to-CTA assignment.  Same results bit for bit; the schedule
+ * is this library's, the pages have no counterpart.
+ *   workspace : 2 int32 of device memory, 16-byte aligned, caller-owned, zero
+ *               before the first call; each call leaves it zero unless it
+ *               reports VSA_ERR_TIMEOUT, after which the caller zeroes it
+ *               again.  Calls that share a workspace must not run
+ *               concurrently.  Unused by 256-token plans.
+ * Errors: as vsa_sparse_attn_fwd_ex; VSA_ERR_INVALID_ARG for a null or
+ * misaligned workspace.
+ */
+VSA_API int vsa_sparse_attn_fwd_ws(vsa_plan_t plan, vsa_dtype_t dtype, const uint16_t *q, const uint16_t *k,
+                                   const uint16_t *v, const int32_t *q2k_idx, const int32_t *q2k_num, int max_k,
+                                   int B, int H, int D, uint16_t *o, float *lse, int32_t *workspace,
+                                   vsa_stream_t stream);
+
+/*
  * NVFP4 quantisation of tiled Q or K (FastVideo "Optimizations" page, section
  * "FP4 Flash Attention 4 (Blackwell only)": Q and K as NVFP4: 4-bit E2M1 codes, one
  * E4M3 scale per block of channels; block length and scale rule are NVFP4's own).

@@ -251,3 +251,13 @@ def test_backward_rejects_more_than_28672_blocks(L):
     F = ctypes.c_void_p(FAKE)
     args = (big.handle, vsa.VSA_BF16, F, F, F, F, F, F, F, F, 4, 1, 2, 128, F, F, F, F, None)
     assert L.vsa_sparse_attn_bwd(*args) == vsa.VSA_ERR_UNSUPPORTED
+
+
+def test_fine_stage_with_workspace_checks_it(L):
+    p = vsa.Plan(8, 16, 16)
+    F, M = ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE + 8)
+    call = lambda ws: L.vsa_sparse_attn_fwd_ws(p.handle, vsa.VSA_BF16, F, F, F, F, F, 4, 1, 2, 128, F, F, ws, None)
+    assert call(None) == vsa.VSA_ERR_INVALID_ARG
+    assert call(M) == vsa.VSA_ERR_INVALID_ARG
+    assert L.vsa_sparse_attn_fwd_ws(p.handle, vsa.VSA_BF16, F, F, F, F, F, 4, 1, 2, 96, F, F, F, None) \
+        == vsa.VSA_ERR_UNSUPPORTED

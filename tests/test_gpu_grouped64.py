@@ -159,3 +159,44 @@ def test_beyond_bitmap_capacity_uses_the_per_block_kernel():
     real = np.flatnonzero(H.real_rows(wl))
     rows = np.unique(np.concatenate([rng.choice(real, 600, replace=False), real[:4], real[-4:]]))
     _run(wl, g, qt, kt, vt, idx, num, rows=rows, what="NB 2048")
+
+
+def test_shared_queue_gives_the_static_results_and_leaves_the_workspace_zero():
+    """vsa_sparse_attn_fwd_ws: groups handed out from a shared queue (prefix
+    groups first) give bit for bit the static assignment's results, on the full
+    tile64 workload, twice in a row; the workspace is zero after each call."""
+    wl = workloads.WORKLOADS["tile64"]
+    ref = H.oracle_front(wl)
+    plan = vsa.Plan.of(wl)
+    q, k, v = (H.to_dev(ref[n]) for n in ("qt", "kt", "vt"))
+    ti, tn = torch.from_numpy(ref["idx"]).cuda(), torch.from_numpy(ref["num"]).cuda()
+    o0, l0 = vsa.sparse_attn_fwd(plan, q, k, v, ti, tn)
+    ws = torch.zeros(4, dtype=torch.int32, device="cuda")
+    for _ in range(2):
+        o1, l1 = vsa.sparse_attn_fwd(plan, q, k, v, ti, tn, workspace=ws)
+        torch.cuda.synchronize()
+        assert vsa.get_status() == vsa.VSA_OK
+        assert int(ws.abs().sum()) == 0
+        assert torch.equal(o0.view(torch.int16), o1.view(torch.int16))
+        assert torch.equal(l0.view(torch.int32), l1.view(torch.int32))
+
+
+def test_shared_queue_on_small_grids():
+    """Fewer groups than SMs, a trailing group of two, repeated ids and empty rows
+    through the queue: against the oracle."""
+    wl, g, qt, kt, vt = _setup(12, 16, 16, npre=100, H_=3)
+    rng = np.random.default_rng(58)
+    idx, num = _random_lists(rng, 1, 3, g.NB, 9)
+    idx[0, 1, 3, :3] = [7, 7, 2]
+    num[0, 1, 3] = 3
+    num[0, 2, :4] = 0
+    plan = vsa.Plan.of(wl)
+    ws = torch.zeros(4, dtype=torch.int32, device="cuda")
+    o, lse = vsa.sparse_attn_fwd(plan, H.to_dev(qt), H.to_dev(kt), H.to_dev(vt), torch.from_numpy(idx).cuda(),
+                                 torch.from_numpy(num).cuda(), workspace=ws)
+    torch.cuda.synchronize()
+    assert vsa.get_status() == vsa.VSA_OK and int(ws.abs().sum()) == 0
+    rows = np.flatnonzero(np.tile(H.real_rows(wl), 3))
+    o_ref, lse_ref = oracle.attn_rows(g, qt, kt, vt, idx, num, rows)
+    H.compare_o_lse(H.from_dev(o).reshape(-1, 128)[rows], lse.cpu().numpy().reshape(-1)[rows], o_ref, lse_ref,
+                    "queue")

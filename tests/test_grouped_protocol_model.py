@@ -11,7 +11,9 @@ early without harm: it walks each tile before any softmax warp can reach
 it.  The softmax warps cannot.)  Groups carry their own number of
 key tiles (zero included) and of query tiles (one or two), so the MMA warp
 keeps per-tile counters for the p_full and o_empty phases, and a softmax
-warpgroup sits out the groups that have no second query tile.  Q is released
+warpgroup sits out the groups that have no second query tile.  With a shared
+queue (a caller workspace) the builder takes group tickets and, past the last
+group, publishes an end marker the consumers stop on.  Q is released
 (q_empty) once the group's last S product has been issued, so the next
 group's Q load overlaps the last P V products.  A softmax
 warp whose query block selected nothing in a tile does not load S at all.
@@ -28,29 +30,42 @@ from tests.test_fwd_protocol_model import Model as FwdModel
 
 
 class GroupedModel(FwdModel):
-    def __init__(self, groups, seed, plant=None, skip_every=3):
+    def __init__(self, groups, seed, plant=None, skip_every=3, sentinel=False):
         super().__init__([], False, 256, seed, plant)
         self.groups = groups            # [(key tiles, query tiles)]
         self.skip_every = skip_every    # which (warp, tile) pairs select nothing
+        # sentinel: the groups come from a shared queue; after the last one the
+        # builder publishes an end marker the consumers stop on
+        self.sentinel = sentinel
         for b in range(2):
             self.bar(("grp_full", b), 1)
             self.bar(("grp_free", b), 10)
         self.grp = [None, None]
 
+    def consumer_groups(self):
+        """Group slots a consumer walks: the groups, then (queue) the end marker."""
+        n = len(self.groups) + (1 if self.sentinel else 0)
+        for gl in range(n):
+            yield gl, (self.groups[gl] if gl < len(self.groups) else None)
+
     # ---------------------------------------------------------------- roles
     def builder(self):
-        for gl in range(len(self.groups)):
+        for gl in range(len(self.groups) + (1 if self.sentinel else 0)):
             b = gl & 1
             if gl >= 2 and self.plant != "builder_no_free_wait":
                 yield ("wait", ("grp_free", b), gl >> 1)
-            yield ("write_grp", b, gl)
+            yield ("write_grp", b, gl if gl < len(self.groups) else "end")
             yield ("arrive", ("grp_full", b), 1, gl >> 1)
 
     def producer(self):
         kit = vit = qit = 0
-        for gl, (n, nq) in enumerate(self.groups):
+        for gl, grp in self.consumer_groups():
             b = gl & 1
             yield ("wait", ("grp_full", b), (gl >> 1) + 1)
+            if grp is None:
+                yield ("read_grp", b, "end")
+                break
+            n, nq = grp
             yield ("read_grp", b, gl)
             if n > 0:
                 yield ("wait", "q_empty", qit)
@@ -74,9 +89,13 @@ class GroupedModel(FwdModel):
         if self.plant == "shared_counters":  # one counter for both query tiles, as the ungrouped kernel
             tiles, items = [0, 0], [0, 0]
         sn = [0, 0]
-        for gl, (n, nq) in enumerate(self.groups):
+        for gl, grp in self.consumer_groups():
             b = gl & 1
             yield ("wait", ("grp_full", b), (gl >> 1) + 1)
+            if grp is None:
+                yield ("read_grp", b, "end")
+                break
+            n, nq = grp
             yield ("read_grp", b, gl)
             yield ("arrive", ("grp_free", b), 1, gl >> 1)
             if n == 0:
@@ -134,9 +153,13 @@ class GroupedModel(FwdModel):
 
     def softmax_warp(self, i, w):
         tiles = items = 0
-        for gl, (n, nq) in enumerate(self.groups):
+        for gl, grp in self.consumer_groups():
             b = gl & 1
             yield ("wait", ("grp_full", b), (gl >> 1) + 1)
+            if grp is None:
+                yield ("read_grp", b, "end")
+                break
+            n, nq = grp
             yield ("read_grp", b, gl)
             if i >= nq or n == 0:
                 yield ("arrive", ("grp_free", b), 1, gl >> 1)
@@ -220,11 +243,18 @@ GROUP_SETS = [
 ]
 
 
+@pytest.mark.parametrize("sentinel", [False, True], ids=["static", "queue"])
 @pytest.mark.parametrize("groups", range(len(GROUP_SETS)))
 @pytest.mark.parametrize("skip_every", [2, 3, 5])
-def test_grouped_protocol_has_no_deadlock_alias_or_hazard(groups, skip_every):
+def test_grouped_protocol_has_no_deadlock_alias_or_hazard(groups, skip_every, sentinel):
     for seed in range(8):
-        GroupedModel(GROUP_SETS[groups], seed=100 * groups + seed, skip_every=skip_every).run()
+        GroupedModel(GROUP_SETS[groups], seed=100 * groups + seed, skip_every=skip_every, sentinel=sentinel).run()
+
+
+def test_queue_with_no_group_for_this_cta_ends_cleanly():
+    """A CTA whose first ticket is already past the end: only the end marker."""
+    for seed in range(10):
+        GroupedModel([], seed=seed, sentinel=True).run()
 
 
 @pytest.mark.parametrize("plant", [
