@@ -7,9 +7,10 @@
 // the FastVideo commit log for the gate-compress branch.
 //
 // One CTA per work item, two kinds:
-//   tile item   (tensor, b*h, block): tile_item of items.cuh; an item that
-//               pools announces its block means on the head's arrival
-//               counter (writes, fence, barrier, atomic add);
+//   tile item   (tensor, b*h, 256 tiled rows: one 256-token block or four
+//               64-token blocks): tile_item of items.cuh; an item that pools
+//               announces its block means on the head's arrival counter
+//               (writes, fence, barrier, atomic add);
 //   score item  (b*h, 8 query blocks): waits until every pooled item of its
 //               head has arrived, then score_item of items.cuh with loads
 //               through L2.
@@ -50,8 +51,10 @@ __global__ void __launch_bounds__(kTileThreads, 3) front_kernel(FrontArgs a) {
   const Geo& g = a.g;
   const int NB = g.NB;
   constexpr bool kScore = SELECT || COMPRESS;
+  constexpr int kBlocks = item_blocks<BS>();
+  const int nT = (NB + kBlocks - 1) / kBlocks;  // tile items per tensor and head
   // tile items per head segment: q, k (and v when the scoring needs its means)
-  const int nA = (COMPRESS || !kScore) ? 3 * NB : 2 * NB;
+  const int nA = (COMPRESS || !kScore) ? 3 * nT : 2 * nT;
   const int nB = kScore ? (NB + kRows - 1) / kRows : 0;
   const int per = nA + nB;
 
@@ -85,14 +88,14 @@ __global__ void __launch_bounds__(kTileThreads, 3) front_kernel(FrontArgs a) {
     }
   } else {  // v tiles that no score item waits for, after every score item
     const int vi = L - a.BH * per;
-    head = vi / NB;
-    item = 2 * NB + (vi - head * NB);
+    head = vi / nT;
+    item = 2 * nT + (vi - head * nT);
     is_tile = true;
   }
 
   if (is_tile) {
-    const int tensor = item / NB;  // 0 q, 1 k, 2 v
-    const int blk = item - tensor * NB;
+    const int tensor = item / nT;  // 0 q, 1 k, 2 v
+    const int blk = (item - tensor * nT) * kBlocks;
     if (tensor == 0) {
       tile_item<BS, true, F16>(g, a.H, blk, head, a.q, a.qt, a.qbar, smem);
     } else if (tensor == 1) {
@@ -116,7 +119,7 @@ __global__ void __launch_bounds__(kTileThreads, 3) front_kernel(FrontArgs a) {
   // score item: wait for the head's block means
   __shared__ int s_ready;
   if (threadIdx.x == 0) {
-    const int target = (COMPRESS ? 3 : 2) * NB;
+    const int target = (COMPRESS ? 3 : 2) * nT;
     const unsigned long long t0 = globaltimer_ns();
     int ready = 1;
     while (ld_acquire_gpu(a.arrive + head) < target) {
@@ -146,13 +149,14 @@ template <int BS, bool F16, bool SELECT, bool COMPRESS>
 cudaError_t launch_front_t(const FrontArgs& a, cudaStream_t stream) {
   constexpr bool kScore = SELECT || COMPRESS;
   const int NB = a.g.NB;
-  size_t smem = static_cast<size_t>(BS) * 256;
+  size_t smem = static_cast<size_t>(kItemRows) * 256;
   if (kScore) smem = smem > score_smem_bytes(NB) ? smem : score_smem_bytes(NB);
   cudaError_t e = cudaFuncSetAttribute(front_kernel<BS, F16, SELECT, COMPRESS>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const long long nB = kScore ? (NB + kRows - 1) / kRows : 0;
-  const long long grid = static_cast<long long>(a.BH) * (3LL * NB + nB);
+  const long long nT = (NB + item_blocks<BS>() - 1) / item_blocks<BS>();
+  const long long grid = static_cast<long long>(a.BH) * (3LL * nT + nB);
   if (grid > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
   front_kernel<BS, F16, SELECT, COMPRESS><<<static_cast<unsigned>(grid), kTileThreads, smem, stream>>>(a);
   return cudaGetLastError();

@@ -56,51 +56,71 @@ __device__ __forceinline__ int block_real_count(const Geo& g, int blk) {
   return vt * vh * vw;
 }
 
-// Tile one (b*h, block): copy its BS token rows into the tiled layout
-// (padding zero-filled) and, with POOL, write the block's fp32 channel means.
-// `stage` is BS * 256 bytes of shared memory (used only with POOL).
+// Token rows one tile item covers: one 256-token block or four 64-token
+// blocks, so every item moves 64 KB whatever the block size.
+constexpr int kItemRows = 256;
+template <int BS>
+__host__ __device__ constexpr int item_blocks() {
+  return kItemRows / BS;
+}
+
+// Tile blocks blk0 .. blk0 + item_blocks<BS>() - 1 (those below NB) of head
+// bh: copy their token rows into the tiled layout (padding zero-filled) and,
+// with POOL, write each block's fp32 channel means (channel d of a block is
+// summed over its slots in slot order, then divided once by its real-token
+// count).  `stage` is kItemRows * 256 bytes of shared memory (used only with
+// POOL).
 template <int BS, bool POOL, bool F16>
-__device__ __forceinline__ void tile_item(const Geo& g, int H, int blk, int bh, const uint4* __restrict__ x,
+__device__ __forceinline__ void tile_item(const Geo& g, int H, int blk0, int bh, const uint4* __restrict__ x,
                                           uint4* __restrict__ xt, float* __restrict__ pooled, uint4* stage) {
+  constexpr int kBlocks = item_blocks<BS>();
+  constexpr int kPer = BS / 16;  // row groups of one block per thread
   const int b = bh / H, h = bh - b * H;
   const int chunk = threadIdx.x & (kRowChunks - 1);
   const int row0 = threadIdx.x >> 4;  // 0..15
-  constexpr int kIters = BS / 16;
 
-  const BlockOrigin org = block_origin(g, blk);
-  uint4 v[kIters];
+  uint4 v[kBlocks * kPer];
 #pragma unroll
-  for (int i = 0; i < kIters; ++i) {
-    const int slot = row0 + 16 * i;
-    const long long s = token_of_slot(g, org, slot);
-    if (s >= 0) {
-      const long long src = ((static_cast<long long>(b) * g.S + s) * H + h) * kRowChunks + chunk;
-      v[i] = __ldcs(x + src);
-    } else {
-      v[i] = make_uint4(0, 0, 0, 0);
+  for (int j = 0; j < kBlocks; ++j) {
+    const int blk = blk0 + j;
+    const bool live = blk < g.NB;
+    const BlockOrigin org = block_origin(g, live ? blk : blk0);
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const long long s = live ? token_of_slot(g, org, row0 + 16 * i) : -1;
+      if (s >= 0) {
+        const long long src = ((static_cast<long long>(b) * g.S + s) * H + h) * kRowChunks + chunk;
+        v[j * kPer + i] = __ldcs(x + src);
+      } else {
+        v[j * kPer + i] = make_uint4(0, 0, 0, 0);
+      }
     }
   }
-  const long long dst0 = (static_cast<long long>(bh) * g.Sp + static_cast<long long>(blk) * BS) * kRowChunks;
+  const long long dst0 = (static_cast<long long>(bh) * g.Sp + static_cast<long long>(blk0) * BS) * kRowChunks;
 #pragma unroll
-  for (int i = 0; i < kIters; ++i) {
-    const int slot = row0 + 16 * i;
-    xt[dst0 + slot * kRowChunks + chunk] = v[i];
-    if (POOL) stage[slot * kRowChunks + chunk] = v[i];
+  for (int j = 0; j < kBlocks; ++j) {
+    if (blk0 + j >= g.NB) break;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int row = j * BS + row0 + 16 * i;
+      xt[dst0 + row * kRowChunks + chunk] = v[j * kPer + i];
+      if (POOL) stage[row * kRowChunks + chunk] = v[j * kPer + i];
+    }
   }
   if (POOL) {
     __syncthreads();
-    if (threadIdx.x < 128) {
-      const int d = threadIdx.x;
-      const uint16_t* st = reinterpret_cast<const uint16_t*>(stage);
+    const int d = threadIdx.x & 127;
+    const uint16_t* st = reinterpret_cast<const uint16_t*>(stage);
+    for (int j = threadIdx.x >> 7; j < kBlocks && blk0 + j < g.NB; j += kTileThreads / 128) {
       float s = 0.0f;
 #pragma unroll 8
       for (int slot = 0; slot < BS; ++slot) {
-        const uint16_t h = st[slot * 128 + d];
-        const float f = F16 ? __half2float(__ushort_as_half(h)) : __uint_as_float(static_cast<uint32_t>(h) << 16);
+        const uint16_t hv = st[(j * BS + slot) * 128 + d];
+        const float f = F16 ? __half2float(__ushort_as_half(hv)) : __uint_as_float(static_cast<uint32_t>(hv) << 16);
         s = __fadd_rn(s, f);
       }
-      const float mean = __fdiv_rn(s, static_cast<float>(block_real_count(g, blk)));
-      pooled[(static_cast<long long>(bh) * g.NB + blk) * 128 + d] = mean;
+      const float mean = __fdiv_rn(s, static_cast<float>(block_real_count(g, blk0 + j)));
+      pooled[(static_cast<long long>(bh) * g.NB + blk0 + j) * 128 + d] = mean;
     }
   }
 }

@@ -5,12 +5,14 @@
 // top-k": the post-patch latent grid is cut into (4, 8, 8) blocks over the
 // zero-padded grid; each block is summarised for scoring.
 //
-// One CTA per (b, h, block).  A token row of one head is D = 128 bf16 =
-// 256 B, moved as 16 lanes x 16 B, so a warp covers two rows per access and
-// the tiled side is one contiguous 32-64 KB run per CTA.  When pooling, the
-// block is also staged in shared memory and thread d sums channel d over
-// the slots in slot order in fp32 (the order the coarse stage is defined
-// with), then divides once by the real-token count.
+// Tiling: one CTA per (b, h, 256 tiled rows), i.e. one 256-token block or
+// four 64-token blocks.  A token row of one head is D = 128 bf16 = 256 B,
+// moved as 16 lanes x 16 B, so a warp covers two rows per access and the
+// tiled side is one contiguous 64 KB run per CTA.  When pooling, the rows
+// are also staged in shared memory and thread d sums channel d of a block
+// over its slots in slot order in fp32 (the order the coarse stage is
+// defined with), then divides once by the real-token count.  Untiling: one
+// CTA per (b, h, block).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -28,8 +30,8 @@ using namespace items;
 template <int BS, bool POOL, bool F16>
 __global__ void __launch_bounds__(kTileThreads) tile_kernel(Geo g, int H, const uint4* __restrict__ x,
                                                             uint4* __restrict__ xt, float* __restrict__ pooled) {
-  extern __shared__ __align__(16) uint4 stage[];  // [BS][16] when POOL
-  tile_item<BS, POOL, F16>(g, H, blockIdx.x, blockIdx.y, x, xt, pooled, stage);
+  extern __shared__ __align__(16) uint4 stage[];  // [kItemRows][16] when POOL
+  tile_item<BS, POOL, F16>(g, H, blockIdx.x * item_blocks<BS>(), blockIdx.y, x, xt, pooled, stage);
 }
 
 template <int BS>
@@ -111,9 +113,9 @@ __global__ void __launch_bounds__(kTileThreads) untile_gate_kernel(Geo g, int H,
 
 template <int BS, bool F16>
 cudaError_t launch_tile_t(const Geo& g, int B, int H, const uint4* xi, uint4* xo, float* pooled, cudaStream_t stream) {
-  dim3 grid(g.NB, B * H);
+  dim3 grid((g.NB + item_blocks<BS>() - 1) / item_blocks<BS>(), B * H);
   if (pooled) {
-    const int smem = BS * 256;
+    const int smem = kItemRows * 256;
     cudaError_t e = cudaFuncSetAttribute(tile_kernel<BS, true, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     tile_kernel<BS, true, F16><<<grid, kTileThreads, smem, stream>>>(g, H, xi, xo, pooled);

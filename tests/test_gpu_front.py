@@ -65,6 +65,8 @@ CASES = [
     ("ragged", dict(T=9, Hg=17, Wg=23, B=2, H=2), 5, False, "f16"),
     ("tile64-prefix", dict(T=6, Hg=8, Wg=12, block=(4, 4, 4), n_prefix=100, H=3), 7, True, "bf16"),
     ("tiles-only", dict(T=6, Hg=8, Wg=12, block=(4, 4, 4), n_prefix=100, H=3), 0, False, "bf16"),
+    # 7 blocks: the last tile item of four 64-token blocks holds three
+    ("tile64-odd", dict(T=5, Hg=9, Wg=4, block=(4, 4, 4), n_prefix=10, B=2, H=2), 3, True, "f16"),
     ("compress-only", dict(T=6, Hg=8, Wg=12, block=(4, 4, 4), n_prefix=100, H=3), 0, True, "f16"),
 ]
 
