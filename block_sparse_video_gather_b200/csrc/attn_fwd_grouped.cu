@@ -1,7 +1,7 @@
 // attn_fwd_grouped.cu -- fine stage of VSA for 64-token blocks (the tile-64
 // layout of the FastVideo commit log, examples/inference/basic/README.md:
-// rows of any length, zero included), with four query blocks per work item
-// over the union of their selections.  "FastVideo VSA" (vLLM-Omni user
+// rows of any length, zero included), with four query blocks per work item,
+// two per 128-row Q tile, each Q tile over the union of its two selections.  "FastVideo VSA" (vLLM-Omni user
 // guide), introduction: each query block attends only to the tokens of its
 // selected blocks; non-causal; scale head_size^-1/2.
 #include <cuda.h>
@@ -24,21 +24,25 @@ using namespace fwd;
 //
 // A 64-row query block fills only half of an M = 128 product, and one block
 // per item leaves the second softmax warpgroup idle.  Here a work item is a
-// group of four consecutive query blocks of one head -- two 128-row Q tiles,
-// one per softmax warpgroup, exactly the 256-token kernel's schedule -- and
-// the key stream is the ascending union of the four selections, two 64-key
-// blocks per 128-key tile.  Each softmax warp serves one query block (warps
-// 0-1 of a warpgroup the first, 2-3 the second) and looks up, per key tile,
-// whether its block selected each half: unselected halves are masked, and a
-// warp whose block selected neither half skips the exponentials (P = 0).  The
-// tensor core computes every tile for both Q tiles; the softmax pays only for
-// the selected pairs.
+// group of four consecutive query blocks of one head -- two 128-row Q tiles
+// (query blocks 0-1 and 2-3), one per softmax warpgroup, the 256-token
+// kernel's schedule.  Each Q tile walks its own key stream, two 64-key blocks
+// per 128-key tile: first the blocks both Q tiles selected (ascending), then
+// the blocks only it selected (ascending).  Step t of the group carries tile
+// t of each Q tile that still has one; for t < ns (the shared blocks paired
+// among themselves) the two tiles are the same and are loaded once, later
+// steps load one tile per Q tile.  Each softmax warp serves one query block
+// (warps 0-1 of a warpgroup the first, 2-3 the second) and looks up, per key
+// tile, whether its block selected each half: unselected halves are masked,
+// and a warp whose block selected neither half skips the exponentials (P =
+// 0).  Against one stream over the union of all four selections this cuts
+// the products of a group by the blocks only the other Q tile selected.
 //
 // A fourth role builds the groups: warp 2 reads the four index rows, sets one
 // bit per (query block, selected block) in shared-memory bitmaps (double
 // buffered, two groups ahead), ORs them into the union, counts the tiles and
-// hands the group over on grp_full; the ten consuming warps (producer, MMA,
-// eight softmax warps) release it on grp_free.  Block ids outside [0, NB) are
+// hands the group over on grp_full; the eleven consuming warps (the K and V
+// producers, MMA, eight softmax warps) release it on grp_free.  Block ids outside [0, NB) are
 // skipped and counts outside [0, max_k] clamped (both reported); a list that
 // names a block twice puts the whole group in list order instead ("concat":
 // each query block's list, two ids per tile, only that block's rows unmasked),
@@ -56,21 +60,32 @@ using namespace fwd;
 // ===========================================================================
 constexpr int kGroupBlocks = 4;
 constexpr int kGroupMaxWords = 32;
+// The five 32 KB tile stages after Q: a step that loads one tile per Q tile
+// takes two K and two V stages, and a V stage is held a softmax longer than
+// a K stage (S issues right after its load, P V only after the softmax), so
+// the V ring gets the deeper share.
+constexpr int kStagesKG = 2, kStagesVG = 3;
+static_assert(kStagesKG + kStagesVG == kStagesK + kStagesV, "same shared-memory map as the per-block kernel");
 static_assert(kGroupMaxNB == 32 * kGroupMaxWords, "bitmap capacity");
 
+constexpr int kShared = kGroupBlocks;  // bitmap of the blocks both Q tiles use
+
 struct GroupInfo {
-  int concat;   // 1: walk each list as given (a list repeats an id)
-  int n_tiles;  // 128-key tiles of the group's key stream
-  int nq;       // 128-row query tiles (1 for a group of two query blocks)
+  int concat;  // 1: walk each list as given (a list repeats an id)
+  int ns;      // leading steps whose tile is the same for both Q tiles
+  int len[2];  // 128-key tiles of each Q tile's key stream (0 for an absent Q tile)
+  int nq;      // 128-row query tiles (1 for a group of two query blocks)
   int cnt[kGroupBlocks];
-  int gi;       // the group (b*h * groups per head + query block / 4), -1: no more groups
-  uint32_t bm[kGroupBlocks + 1][kGroupMaxWords];  // selection bitmaps; [kGroupBlocks] = union
+  int gi;      // the group (b*h * groups per head + query block / 4), -1: no more groups
+  // selection bitmaps of the four query blocks; [kShared]: blocks selected
+  // by a query block of each Q tile
+  uint32_t bm[kGroupBlocks + 1][kGroupMaxWords];
 };
 
 struct GroupBarriers {
   uint64_t q_full, q_empty;
-  uint64_t k_full[kStagesK], k_empty[kStagesK];
-  uint64_t v_full[kStagesV], v_empty[kStagesV];
+  uint64_t k_full[kStagesKG], k_empty[kStagesKG];
+  uint64_t v_full[kStagesVG], v_empty[kStagesVG];
   uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
   uint64_t grp_full[2], grp_free[2];
   uint64_t drain;
@@ -82,7 +97,7 @@ static_assert(sizeof(GroupBarriers) <= 256, "barrier block too large");
 constexpr uint32_t kSmemGroups = kSmemBar + 256;
 constexpr uint32_t kSmemTotalG = kSmemGroups + 2 * sizeof(GroupInfo) + 1024;
 static_assert(kSmemTotalG <= 232448, "grouped kernel exceeds the shared memory of one CTA");
-constexpr uint32_t kGroupConsumers = 10;  // producer, MMA, 8 softmax warps: one arrival each
+constexpr uint32_t kGroupConsumers = 11;  // two producers, MMA, 8 softmax warps: one arrival each
 
 __device__ __forceinline__ bool gwarp_wait(uint64_t* bar, uint32_t parity, GroupBarriers* bars,
                                            unsigned int* status) {
@@ -106,31 +121,35 @@ __device__ __forceinline__ int row_block_id(const Params& p, int row, int t) {
   return (kb >= 0 && kb < p.g.NB) ? kb : -1;
 }
 
-// The key stream of one group: 128-key tile after 128-key tile, the two block
-// ids (-1: absent or unusable) and the query blocks of the group that use each.
+// The key stream of Q tile qt of a group: 128-key tile after 128-key tile,
+// the two block ids (-1: absent or unusable) and the query blocks that use
+// each.  Union: the shared blocks ascending, then the blocks only Q tile qt
+// selected ascending.  Concat: the four lists as given, the same stream for
+// both Q tiles.
 struct GroupWalk {
-  int a;       // union: bitmap word; concat: query block j
-  uint32_t b;  // union: bits of word a still to visit; concat: next pair of list j
+  int a;       // union: word a of the shared bitmap, then (a >= W) word a - W of Q tile qt's own
+  uint32_t b;  // union: bits of that word still to visit; concat: next pair of list a
   __device__ __forceinline__ void init(const GroupInfo& gb) {
     a = 0;
-    b = gb.concat ? 0u : gb.bm[kGroupBlocks][0];
+    b = gb.concat ? 0u : gb.bm[kShared][0];
   }
-  __device__ __forceinline__ int pop_union(const GroupInfo& gb, int W) {
+  __device__ __forceinline__ int pop_union(const GroupInfo& gb, int W, int qt) {
     while (b == 0u) {
-      if (++a >= W) return -1;
-      b = gb.bm[kGroupBlocks][a];
+      if (++a >= 2 * W) return -1;
+      const int w = a - W;
+      b = w < 0 ? gb.bm[kShared][a] : (gb.bm[2 * qt][w] | gb.bm[2 * qt + 1][w]) & ~gb.bm[kShared][w];
     }
     const int bit = __ffs(b) - 1;
     b &= b - 1u;
-    return a * 32 + bit;
+    return (a < W ? a : a - W) * 32 + bit;
   }
   // Next tile: ids ka, kb, and the one query block that uses them in list
   // order (owner), or -1 for the union, where each query block's bitmap says.
-  __device__ __forceinline__ void next(const GroupInfo& gb, const Params& p, int row0, int W, int& ka,
+  __device__ __forceinline__ void next(const GroupInfo& gb, const Params& p, int row0, int W, int qt, int& ka,
                                        int& kb, int& owner) {
     if (!gb.concat) {
-      ka = pop_union(gb, W);
-      kb = pop_union(gb, W);
+      ka = pop_union(gb, W, qt);
+      kb = pop_union(gb, W, qt);
       owner = -1;
       return;
     }
@@ -138,7 +157,7 @@ struct GroupWalk {
       ++a;
       b = 0u;
     }
-    if (a >= kGroupBlocks) {  // past the last list (not reached: n_tiles counts the pairs)
+    if (a >= kGroupBlocks) {  // past the last list (not reached: len counts the pairs)
       ka = kb = owner = -1;
       return;
     }
@@ -232,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + kSmemQ;
   uint8_t* sK = smem + kSmemK;
-  uint8_t* sV = smem + kSmemV;
+  uint8_t* sV = sK + kStagesKG * kTileBytes;
   GroupBarriers* bars = reinterpret_cast<GroupBarriers*>(smem + kSmemBar);
   GroupInfo* grp = reinterpret_cast<GroupInfo*>(smem + kSmemGroups);
 
@@ -246,11 +265,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
     mbar_init(&bars->q_empty, 1);
-    for (int s = 0; s < kStagesK; ++s) {
+    for (int s = 0; s < kStagesKG; ++s) {
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->k_empty[s], 1);
     }
-    for (int s = 0; s < kStagesV; ++s) {
+    for (int s = 0; s < kStagesVG; ++s) {
       mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->v_empty[s], 1);
     }
@@ -333,39 +352,58 @@ __global__ void __launch_bounds__(kThreads, 1)
       repeat = __any_sync(0xffffffffu, repeat);
       bad = __any_sync(0xffffffffu, bad);
       if (bad && lane == 0) atomicCAS(p.status, 0u, (unsigned)VSA_ERR_BAD_INDEX);
-      int U = 0;
+      // blocks of both Q tiles, of Q tile 0 only, of Q tile 1 only (a group
+      // of two query blocks has no Q tile 1: all its blocks are Q tile 0's)
+      int cs = 0, c0 = 0, c1 = 0;
       for (int w = lane; w < W; w += 32) {
-        const uint32_t u = gb.bm[0][w] | gb.bm[1][w] | gb.bm[2][w] | gb.bm[3][w];
-        gb.bm[kGroupBlocks][w] = u;
-        U += __popc(u);
+        const uint32_t u0 = gb.bm[0][w] | gb.bm[1][w], u1 = gb.bm[2][w] | gb.bm[3][w], sh = u0 & u1;
+        gb.bm[kShared][w] = sh;
+        cs += __popc(sh);
+        c0 += __popc(u0 & ~sh);
+        c1 += __popc(u1 & ~sh);
       }
-      U = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(U)));
+      cs = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(cs)));
+      c0 = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(c0)));
+      c1 = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(c1)));
       if (lane == 0) {
-        int n = 0;
-        if (repeat) {
+        const int nq = (nqb + 1) / 2;
+        if (repeat) {  // one stream, the lists as given, for every Q tile
+          int n = 0;
 #pragma unroll
           for (int j = 0; j < kGroupBlocks; ++j) n += (cnts[j] + 1) / 2;
+          gb.ns = nq == 2 ? n : 0;
+          gb.len[0] = n;
+          gb.len[1] = nq == 2 ? n : 0;
         } else {
-          n = (U + 1) / 2;
+          gb.ns = cs / 2;
+          gb.len[0] = (cs + c0 + 1) / 2;
+          gb.len[1] = (cs + c1 + 1) / 2;
         }
         gb.gi = gi;
         gb.concat = repeat ? 1 : 0;
-        gb.n_tiles = n;
-        gb.nq = (nqb + 1) / 2;
+        gb.nq = nq;
 #pragma unroll
         for (int j = 0; j < kGroupBlocks; ++j) gb.cnt[j] = cnts[j];
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->grp_full[buf]);
     }
-  } else if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    tma_prefetch_desc(&tm_q);
-    tma_prefetch_desc(&tm_k);
-    tma_prefetch_desc(&tm_v);
+  } else if (warp == 0 || warp == 3) {
+    // ------------------------------------------------------------ producers
+    // Warp 0 loads Q and the K tiles, warp 3 the V tiles: each waits only on
+    // its own ring, so a K load never queues behind a V stage that is still
+    // read (a step may take two stages of each).
+    const bool vside = warp == 3;
+    tma_prefetch_desc(vside ? &tm_v : &tm_k);
+    if (!vside) tma_prefetch_desc(&tm_q);
     const uint64_t pol_kv = policy_evict_last();
     const uint64_t pol_q = policy_evict_first();
-    int kit = 0, vit = 0, qit = 0;
+    const int stages = vside ? kStagesVG : kStagesKG;
+    uint8_t* const ring = vside ? sV : sK;
+    uint64_t* const full = vside ? bars->v_full : bars->k_full;
+    uint64_t* const empty = vside ? bars->v_empty : bars->k_empty;
+    const CUtensorMap* const tm = vside ? &tm_v : &tm_k;
+    int it = 0, qit = 0;
     bool stop = false;
     for (int gl = 0; !stop; ++gl) {
       const int buf = gl & 1;
@@ -373,51 +411,53 @@ __global__ void __launch_bounds__(kThreads, 1)
       const GroupInfo& gb = grp[buf];
       const int gi = gb.gi;
       if (gi < 0) break;
-      const int n = gb.n_tiles, nq = gb.nq;
+      const int ns = gb.ns, len0 = gb.len[0], len1 = gb.len[1], nq = gb.nq;
+      const int n = max(len0, len1);
       const int bh = gi / ngq, qb0 = (gi - bh * ngq) * kGroupBlocks;
       const long long base = static_cast<long long>(bh) * g.Sp;
       const int row0 = bh * g.NB + qb0;
       if (n > 0) {
-        if (!gwarp_wait(&bars->q_empty, (qit & 1) ^ 1, bars, p.status)) break;
-        mbar_arrive_expect_tx_w(&bars->q_full, nq * kTileBytes);
-        const int qrow = static_cast<int>(base + static_cast<long long>(qb0) * 64);
-        for (int i = 0; i < nq; ++i)
-          for (int hf = 0; hf < 2; ++hf)
-            tma_load_2d_w(sQ + i * kTileBytes + hf * kHalfBytes, &tm_q, hf * 64, qrow + i * 128, &bars->q_full,
-                          pol_q);
-        ++qit;
-        GroupWalk walk;
-        walk.init(gb);
-        for (int t = 0; t < n; ++t) {
-          int ka, kb, owner;
-          walk.next(gb, p, row0, W, ka, kb, owner);
-          // absent or unusable blocks load block 0 (finite data, masked by every warp)
-          const int krow0 = static_cast<int>(base + static_cast<long long>(ka < 0 ? 0 : ka) * 64);
-          const int krow1 = static_cast<int>(base + static_cast<long long>(kb < 0 ? 0 : kb) * 64);
-          const int sk = kit % kStagesK;
-          if (!gwarp_wait(&bars->k_empty[sk], ((kit / kStagesK) & 1) ^ 1, bars, p.status)) {
-            stop = true;
-            break;
-          }
-          mbar_arrive_expect_tx_w(&bars->k_full[sk], kTileBytes);
+        if (!vside) {
+          if (!gwarp_wait(&bars->q_empty, (qit & 1) ^ 1, bars, p.status)) break;
+          mbar_arrive_expect_tx_w(&bars->q_full, nq * kTileBytes);
+          const int qrow = static_cast<int>(base + static_cast<long long>(qb0) * 64);
+          for (int i = 0; i < nq; ++i)
+            for (int hf = 0; hf < 2; ++hf)
+              tma_load_2d_w(sQ + i * kTileBytes + hf * kHalfBytes, &tm_q, hf * 64, qrow + i * 128, &bars->q_full,
+                            pol_q);
+          ++qit;
+        }
+        // one stage per distinct tile of a step, Q tile 0's first
+        auto load = [&](int krow0, int krow1) -> bool {
+          const int st = it % stages;
+          if (!gwarp_wait(&empty[st], ((it / stages) & 1) ^ 1, bars, p.status)) return false;
+          mbar_arrive_expect_tx_w(&full[st], kTileBytes);
           for (int hf = 0; hf < 2; ++hf) {
-            uint8_t* dst = sK + sk * kTileBytes + hf * kHalfBytes;
-            tma_load_2d_w(dst, &tm_k, hf * 64, krow0, &bars->k_full[sk], pol_kv);
-            tma_load_2d_w(dst + kHalfBytes / 2, &tm_k, hf * 64, krow1, &bars->k_full[sk], pol_kv);
+            uint8_t* dst = ring + st * kTileBytes + hf * kHalfBytes;
+            tma_load_2d_w(dst, tm, hf * 64, krow0, &full[st], pol_kv);
+            tma_load_2d_w(dst + kHalfBytes / 2, tm, hf * 64, krow1, &full[st], pol_kv);
           }
-          ++kit;
-          const int sv = vit % kStagesV;
-          if (!gwarp_wait(&bars->v_empty[sv], ((vit / kStagesV) & 1) ^ 1, bars, p.status)) {
-            stop = true;
-            break;
+          ++it;
+          return true;
+        };
+        GroupWalk walk[2];
+        walk[0].init(gb);
+        walk[1].init(gb);
+        for (int t = 0; t < n && !stop; ++t) {
+          // the rows of each Q tile's tile (absent or unusable blocks load block 0:
+          // finite data, masked by every warp)
+          int r0[2] = {0, 0}, r1[2] = {0, 0};
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            if (t >= gb.len[j]) continue;
+            int ka, kb, owner;
+            walk[j].next(gb, p, row0, W, j, ka, kb, owner);
+            r0[j] = static_cast<int>(base + static_cast<long long>(ka < 0 ? 0 : ka) * 64);
+            r1[j] = static_cast<int>(base + static_cast<long long>(kb < 0 ? 0 : kb) * 64);
           }
-          mbar_arrive_expect_tx_w(&bars->v_full[sv], kTileBytes);
-          for (int hf = 0; hf < 2; ++hf) {
-            uint8_t* dst = sV + sv * kTileBytes + hf * kHalfBytes;
-            tma_load_2d_w(dst, &tm_v, hf * 64, krow0, &bars->v_full[sv], pol_kv);
-            tma_load_2d_w(dst + kHalfBytes / 2, &tm_v, hf * 64, krow1, &bars->v_full[sv], pol_kv);
-          }
-          ++vit;
+          const bool shared = t < ns;  // both Q tiles' tile t is the same: one stage
+          const bool a0 = t < len0, a1 = t < len1 && !shared;
+          if ((a0 && !load(r0[0], r1[0])) || (a1 && !load(r0[1], r1[1]))) stop = true;
         }
         if (stop) break;
       }
@@ -426,15 +466,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // Drain: every issued copy must land before the CTA's shared memory is released.
     if (qit > 0) mbar_wait_drain(&bars->q_full, (qit - 1) & 1, kTimeoutNs);
-    for (int s = 0; s < kStagesK; ++s)
-      if (kit > s) {
-        const int last = kit - 1 - ((kit - 1 - s) % kStagesK);
-        mbar_wait_drain(&bars->k_full[s], (last / kStagesK) & 1, kTimeoutNs);
-      }
-    for (int s = 0; s < kStagesV; ++s)
-      if (vit > s) {
-        const int last = vit - 1 - ((vit - 1 - s) % kStagesV);
-        mbar_wait_drain(&bars->v_full[s], (last / kStagesV) & 1, kTimeoutNs);
+    for (int st = 0; st < stages; ++st)
+      if (it > st) {
+        const int last = it - 1 - ((it - 1 - st) % stages);
+        mbar_wait_drain(&full[st], (last / stages) & 1, kTimeoutNs);
       }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -443,7 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t dv0 = sdesc_sw128(smem_u32(sV), kHalfBytes, 1024);
     constexpr uint64_t kTileDesc = kTileBytes >> 4;
     int kit = 0, vit = 0, qit = 0;
-    int tiles[2] = {0, 0}, items[2] = {0, 0};
+    int tiles0 = 0, tiles1 = 0, items0 = 0, items1 = 0;  // per Q tile: P V products, groups
     bool ok = true;
     auto issue_s = [&](int i, int sk) {
       const uint32_t d = tmem + i * 128;
@@ -465,67 +500,68 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int buf = gl & 1;
       if (!(ok = gwarp_wait(&bars->grp_full[buf], (gl >> 1) & 1, bars, p.status))) break;
       if (grp[buf].gi < 0) break;
-      const int n = grp[buf].n_tiles, nq = grp[buf].nq;
+      const int ns = grp[buf].ns, len0 = grp[buf].len[0], len1 = grp[buf].len[1];
+      const int n = max(len0, len1);
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->grp_free[buf]);
       if (n == 0) continue;
       if (!(ok = gwarp_wait(&bars->q_full, qit & 1, bars, p.status))) break;
       ++qit;
       tc_fence_after();
-      int sk = kit % kStagesK;
-      if (!(ok = gwarp_wait(&bars->k_full[sk], (kit / kStagesK) & 1, bars, p.status))) break;
-      tc_fence_after();
-      issue_s(0, sk);
-      mma_commit_w(&bars->s_full[0]);
-      if (nq == 2) {
-        issue_s(1, sk);
-        mma_commit_w(&bars->s_full[1]);
-      }
-      mma_commit_w(&bars->k_empty[sk]);
-      // Q is read by the S products only: once the group's last S is issued,
-      // the next group's Q may load while the last P V products run
-      if (n == 1) mma_commit_w(&bars->q_empty);
-      ++kit;
-      for (int t = 0; t < n; ++t) {
-        const int sv = vit % kStagesV;
-        if (!(ok = gwarp_wait(&bars->v_full[sv], (vit / kStagesV) & 1, bars, p.status))) break;
-        if (!(ok = gwarp_wait(&bars->p_full[0], tiles[0] & 1, bars, p.status))) break;
-        if (t == 0 && !(ok = gwarp_wait(&bars->o_empty[0], (items[0] & 1) ^ 1, bars, p.status))) break;
-        tc_fence_after();
-        issue_pv(0, sv, t > 0);
-        ++tiles[0];
-        if (t == n - 1) mma_commit_w(&bars->o_full[0]);
-        const bool more = t + 1 < n;
-        sk = kit % kStagesK;
-        if (more) {
-          if (!(ok = gwarp_wait(&bars->k_full[sk], (kit / kStagesK) & 1, bars, p.status))) break;
-          tc_fence_after();
-          issue_s(0, sk);
-          mma_commit_w(&bars->s_full[0]);
-        }
-        if (nq == 2) {
-          if (!(ok = gwarp_wait(&bars->p_full[1], tiles[1] & 1, bars, p.status))) break;
-          if (t == 0 && !(ok = gwarp_wait(&bars->o_empty[1], (items[1] & 1) ^ 1, bars, p.status))) break;
-          tc_fence_after();
-          issue_pv(1, sv, t > 0);
-          ++tiles[1];
-        }
-        mma_commit_w(&bars->v_empty[sv]);
-        ++vit;
-        if (nq == 2 && t == n - 1) mma_commit_w(&bars->o_full[1]);
-        if (more) {
-          if (nq == 2) {
-            issue_s(1, sk);
-            mma_commit_w(&bars->s_full[1]);
+      // Per step t: PV0(t), S0(t+1), PV1(t), S1(t+1); t = -1 issues the first S
+      // products.  A shared step's tile is one K and one V stage, released by
+      // Q tile 1's product; other steps take one stage per Q tile.  One loop
+      // over the Q tiles (not unrolled), so every product is issued from one
+      // place in the code: the issuing thread stays lean.
+      int sk = 0, sv = 0;
+      for (int t = -1; t < n && ok; ++t) {
+#pragma unroll 1
+        for (int j = 0; j < 2; ++j) {
+          const int lj = j ? len1 : len0;
+          if (t >= 0 && t < lj) {  // P V product of Q tile j at step t
+            const bool shared = t < ns;
+            if (j == 0 || !shared) {
+              sv = vit % kStagesVG;
+              if (!(ok = gwarp_wait(&bars->v_full[sv], (vit / kStagesVG) & 1, bars, p.status))) break;
+            }
+            const int tj = j ? tiles1 : tiles0;
+            if (!(ok = gwarp_wait(&bars->p_full[j], tj & 1, bars, p.status))) break;
+            if (t == 0) {
+              const int ij = j ? items1 : items0;
+              if (!(ok = gwarp_wait(&bars->o_empty[j], (ij & 1) ^ 1, bars, p.status))) break;
+            }
+            tc_fence_after();
+            issue_pv(j, sv, t > 0);
+            if (j) ++tiles1; else ++tiles0;
+            if (t == lj - 1) mma_commit_w(&bars->o_full[j]);
+            if (j == 1 || !shared) {  // the V stage's last reader is issued
+              mma_commit_w(&bars->v_empty[sv]);
+              ++vit;
+            }
           }
-          mma_commit_w(&bars->k_empty[sk]);
-          if (t + 2 == n) mma_commit_w(&bars->q_empty);
-          ++kit;
+          const int u = t + 1;
+          if (u < lj) {  // S product of Q tile j at step t + 1
+            const bool shared = u < ns;
+            if (j == 0 || !shared) {
+              sk = kit % kStagesKG;
+              if (!(ok = gwarp_wait(&bars->k_full[sk], (kit / kStagesKG) & 1, bars, p.status))) break;
+              tc_fence_after();
+            }
+            issue_s(j, sk);
+            mma_commit_w(&bars->s_full[j]);
+            if (j == 1 || !shared) {  // the K stage's last reader is issued
+              mma_commit_w(&bars->k_empty[sk]);
+              ++kit;
+            }
+          }
         }
+        // Q is read by the S products only: once the group's last S is issued,
+        // the next group's Q may load while the last P V products run
+        if (ok && t + 2 == n) mma_commit_w(&bars->q_empty);
       }
       if (!ok) break;
-      ++items[0];
-      if (nq == 2) ++items[1];
+      if (len0 > 0) ++items0;
+      if (len1 > 0) ++items1;
     }
     // Drain: wait for every MMA issued by this thread before TMEM and smem go away.
     mma_commit_w(&bars->drain);
@@ -550,13 +586,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const GroupInfo& gb = grp[buf];
       const int gi = gb.gi;
       if (gi < 0) break;
-      const int n = gb.n_tiles, nq = gb.nq;
+      const int nq = gb.nq;
+      const int n = wg < nq ? gb.len[wg] : 0;  // this Q tile's key tiles
       const int bh = gi / ngq, qb0 = (gi - bh * ngq) * kGroupBlocks;
       const int row0 = bh * g.NB + qb0;  // index row of the group's first query block (NB <= kGroupMaxNB)
-      if (wg >= nq || n == 0) {
+      if (n == 0) {
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->grp_free[buf]);
-        if (wg < nq) {  // nothing selected by any query block of the group
+        if (wg < nq) {  // nothing selected by either query block of this Q tile
           const long long row = static_cast<long long>(bh) * g.Sp + static_cast<long long>(qb0) * 64 + wg * 128 + r;
           uint4* orow = reinterpret_cast<uint4*>(p.o + row * 128);
 #pragma unroll
@@ -570,7 +607,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       walk.init(gb);
       for (int t = 0; t < n; ++t) {
         int ka, kb, owner;
-        walk.next(gb, p, row0, W, ka, kb, owner);
+        walk.next(gb, p, row0, W, wg, ka, kb, owner);
         // this warp's query block: which halves of the tile it selected
         const int sa = group_uses(gb, owner, jq, ka) ? ka : -1;
         const int sb = group_uses(gb, owner, jq, kb) ? kb : -1;

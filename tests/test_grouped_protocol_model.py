@@ -1,17 +1,21 @@
 """A CPU model of the grouped 64-token forward kernel's synchronisation protocol
-(`attn_fwd_grouped64_kernel` in csrc/attn_fwd.cu).
+(`attn_fwd_grouped64_kernel` in csrc/attn_fwd_grouped.cu).
 
 On top of the forward kernels' protocol (modelled in
 tests/test_fwd_protocol_model.py) this kernel adds a group builder warp that
 writes each group's selection bitmaps into one of two shared-memory buffers
-and hands it over on grp_full; ten warps read it (the producer while it
-walks the key stream, the MMA warp once, the eight softmax warps while they
-walk it) and each releases it on grp_free.  (The producer could release
-early without harm: it walks each tile before any softmax warp can reach
-it.  The softmax warps cannot.)  Groups carry their own number of
-key tiles (zero included) and of query tiles (one or two), so the MMA warp
-keeps per-tile counters for the p_full and o_empty phases, and a softmax
-warpgroup sits out the groups that have no second query tile.  With a shared
+and hands it over on grp_full; eleven warps read it (two producers -- Q and
+K tiles, V tiles -- while they walk the key streams, the MMA warp once, the
+eight softmax warps while they walk them) and each releases it on grp_free.
+(The producers could release early without harm: they walk each tile before
+any softmax warp can reach it.  The softmax warps cannot.)  Each query tile of a group walks its own
+key stream: a group carries the number of leading steps whose tile is the
+same for both query tiles (one K and one V stage, released by the second
+query tile's product) and each query tile's number of tiles (zero
+included); later steps load one stage per query tile, and a step past one
+query tile's end runs the other alone.  So the MMA warp keeps per-query-tile
+counters for the p_full and o_empty phases, and a softmax warpgroup sits
+out the groups that have no tile for it.  With a shared
 queue (a caller workspace) the builder takes group tickets and, past the last
 group, publishes an end marker the consumers stop on.  Q is released
 (q_empty) once the group's last S product has been issued, so the next
@@ -32,14 +36,20 @@ from tests.test_fwd_protocol_model import Model as FwdModel
 class GroupedModel(FwdModel):
     def __init__(self, groups, seed, plant=None, skip_every=3, sentinel=False):
         super().__init__([], False, 256, seed, plant)
-        self.groups = groups            # [(key tiles, query tiles)]
+        self.KS, self.VS = 2, 3         # the grouped kernel's K and V ring stages
+        for st in range(self.KS):
+            self.bar(("k_full", st)), self.bar(("k_empty", st))
+        for st in range(self.VS):
+            self.bar(("v_full", st)), self.bar(("v_empty", st))
+        # [(shared steps, key tiles of query tile 0, of query tile 1, query tiles)]
+        self.groups = groups
         self.skip_every = skip_every    # which (warp, tile) pairs select nothing
         # sentinel: the groups come from a shared queue; after the last one the
         # builder publishes an end marker the consumers stop on
         self.sentinel = sentinel
         for b in range(2):
             self.bar(("grp_full", b), 1)
-            self.bar(("grp_free", b), 10)
+            self.bar(("grp_free", b), 11)
         self.grp = [None, None]
 
     def consumer_groups(self):
@@ -57,7 +67,8 @@ class GroupedModel(FwdModel):
             yield ("write_grp", b, gl if gl < len(self.groups) else "end")
             yield ("arrive", ("grp_full", b), 1, gl >> 1)
 
-    def producer(self):
+    def producer(self, side):
+        """side "k": Q and the K tiles; side "v": the V tiles (a warp of its own)."""
         kit = vit = qit = 0
         for gl, grp in self.consumer_groups():
             b = gl & 1
@@ -65,29 +76,37 @@ class GroupedModel(FwdModel):
             if grp is None:
                 yield ("read_grp", b, "end")
                 break
-            n, nq = grp
+            ns, lens, nq = grp[0], grp[1:3], grp[3]
             yield ("read_grp", b, gl)
+            n = max(lens)
             if n > 0:
-                yield ("wait", "q_empty", qit)
-                yield ("tma", "q_full", qit, [(("q", c), gl) for c in range(2 * nq)])
-                qit += 1
+                if side == "k":
+                    yield ("wait", "q_empty", qit)
+                    yield ("tma", "q_full", qit, [(("q", c), gl) for c in range(2 * nq)])
+                    qit += 1
                 for t in range(n):
                     yield ("read_grp", b, gl)
-                    s = kit % self.KS
-                    yield ("wait", ("k_empty", s), kit // self.KS)
-                    yield ("tma", ("k_full", s), kit // self.KS, [(("k", s, c), (gl, t)) for c in range(2)])
-                    kit += 1
-                    s = vit % self.VS
-                    yield ("wait", ("v_empty", s), vit // self.VS)
-                    yield ("tma", ("v_full", s), vit // self.VS, [(("v", s, c), (gl, t)) for c in range(2)])
-                    vit += 1
+                    # one stage per distinct tile of the step, query tile 0's first
+                    tags = ["sh"] if t < ns else [j for j in range(2) if t < lens[j]]
+                    for tag in tags:
+                        if side == "k":
+                            s = kit % self.KS
+                            yield ("wait", ("k_empty", s), kit // self.KS)
+                            yield ("tma", ("k_full", s), kit // self.KS,
+                                   [(("k", s, c), (gl, t, tag)) for c in range(2)])
+                            kit += 1
+                        else:
+                            s = vit % self.VS
+                            yield ("wait", ("v_empty", s), vit // self.VS)
+                            yield ("tma", ("v_full", s), vit // self.VS,
+                                   [(("v", s, c), (gl, t, tag)) for c in range(2)])
+                            vit += 1
             yield ("arrive", ("grp_free", b), 1, gl >> 1)
 
     def mma(self):
-        kit = vit = qit = 0
+        st = dict(kit=0, vit=0, sk=0, sv=0)
+        qit = 0
         tiles, items = [0, 0], [0, 0]
-        if self.plant == "shared_counters":  # one counter for both query tiles, as the ungrouped kernel
-            tiles, items = [0, 0], [0, 0]
         sn = [0, 0]
         for gl, grp in self.consumer_groups():
             b = gl & 1
@@ -95,61 +114,71 @@ class GroupedModel(FwdModel):
             if grp is None:
                 yield ("read_grp", b, "end")
                 break
-            n, nq = grp
+            ns, lens, nq = grp[0], grp[1:3], grp[3]
+            n = max(lens)
             yield ("read_grp", b, gl)
             yield ("arrive", ("grp_free", b), 1, gl >> 1)
             if n == 0:
                 continue
             yield ("wait", "q_full", qit + 1)
             qit += 1
+            if self.plant == "split_as_shared":  # a split step read from one stage, as a shared one
+                ns = n
 
-            def issue_s(i, sk, t):
-                yield ("pipe", ("S", i, sn[i], sk, (gl, t), gl))
-                yield ("pipe", ("commit", ("s_full", i)))
-                sn[i] += 1
+            def s_of(j, u):
+                shared = u < ns
+                if j == 0 or not shared:
+                    st["sk"] = st["kit"] % self.KS
+                    yield ("wait", ("k_full", st["sk"]), st["kit"] // self.KS + 1)
+                tag = "sh" if shared else j
+                yield ("pipe", ("S", j, sn[j], st["sk"], (gl, u, tag), gl))
+                yield ("pipe", ("commit", ("s_full", j)))
+                sn[j] += 1
+                if j == 1 or not shared:
+                    yield ("pipe", ("commit", ("k_empty", st["sk"])))
+                    st["kit"] += 1
 
-            def issue_pv(i, sv, t):
-                yield ("wait", ("p_full", i), tiles[i] + 1)
-                if t == 0:
-                    yield ("wait", ("o_empty", i), items[i])
-                yield ("pipe", ("PV", i, sv, (gl, t)))
-                if t == n - 1:
-                    yield ("pipe", ("commit", ("o_full", i)))
-                tiles[i] += 1
-                if self.plant == "shared_counters" and i == 0:
+            def pv_of(j, u):
+                shared = u < ns
+                if j == 0 or not shared:
+                    st["sv"] = st["vit"] % self.VS
+                    yield ("wait", ("v_full", st["sv"]), st["vit"] // self.VS + 1)
+                yield ("wait", ("p_full", j), tiles[j] + 1)
+                if u == 0:
+                    yield ("wait", ("o_empty", j), items[j])
+                tag = "sh" if shared else j
+                yield ("pipe", ("PV", j, st["sv"], (gl, u, tag)))
+                if u == lens[j] - 1:
+                    yield ("pipe", ("commit", ("o_full", j)))
+                tiles[j] += 1
+                if self.plant == "shared_counters" and j == 0:
                     tiles[1] = tiles[0]
+                release = j == 1 or not shared or self.plant == "v_free_first_pv"
+                if release:
+                    yield ("pipe", ("commit", ("v_empty", st["sv"])))
+                    st["vit"] += 1
 
-            sk = kit % self.KS
-            yield ("wait", ("k_full", sk), kit // self.KS + 1)
-            for i in range(nq):
-                yield from issue_s(i, sk, 0)
-            yield ("pipe", ("commit", ("k_empty", sk)))
+            for j in range(2):
+                if lens[j] > 0:
+                    yield from s_of(j, 0)
             if n == 1 or self.plant == "q_free_first_s":
                 yield ("pipe", ("commit", "q_empty"))  # Q is read by S products only
-            kit += 1
             for t in range(n):
-                sv = vit % self.VS
-                yield ("wait", ("v_full", sv), vit // self.VS + 1)
-                more = t + 1 < n
-                sk = kit % self.KS
-                yield from issue_pv(0, sv, t)
-                if more:
-                    yield ("wait", ("k_full", sk), kit // self.KS + 1)
-                    yield from issue_s(0, sk, t + 1)
-                if nq == 2:
-                    yield from issue_pv(1, sv, t)
-                yield ("pipe", ("commit", ("v_empty", sv)))
-                vit += 1
-                if more:
-                    if nq == 2:
-                        yield from issue_s(1, sk, t + 1)
-                    yield ("pipe", ("commit", ("k_empty", sk)))
-                    if t + 2 == n and self.plant != "q_free_first_s":
-                        yield ("pipe", ("commit", "q_empty"))  # after the group's last S
-                    kit += 1
-            items[0] += 1
-            if nq == 2 or self.plant == "shared_counters":
-                items[1] += 1
+                if t < lens[0]:
+                    yield from pv_of(0, t)
+                if t + 1 < lens[0]:
+                    yield from s_of(0, t + 1)
+                if t < lens[1]:
+                    if self.plant == "v_free_first_pv" and t < ns:
+                        st["vit"] -= 1  # the stage PV0 already released, read again
+                    yield from pv_of(1, t)
+                if t + 1 < lens[1]:
+                    yield from s_of(1, t + 1)
+                if t + 2 == n and self.plant != "q_free_first_s":
+                    yield ("pipe", ("commit", "q_empty"))  # after the group's last S
+            for j in range(2):
+                if lens[j] > 0 or (self.plant == "shared_counters" and lens[0] > 0):
+                    items[j] += 1
 
     def softmax_warp(self, i, w):
         tiles = items = 0
@@ -159,9 +188,10 @@ class GroupedModel(FwdModel):
             if grp is None:
                 yield ("read_grp", b, "end")
                 break
-            n, nq = grp
+            ns, lens, nq = grp[0], grp[1:3], grp[3]
+            n = lens[i] if i < nq else 0
             yield ("read_grp", b, gl)
-            if i >= nq or n == 0:
+            if n == 0:
                 yield ("arrive", ("grp_free", b), 1, gl >> 1)
                 if i < nq:
                     yield ("write_empty_rows", i, w, gl)
@@ -201,6 +231,24 @@ class GroupedModel(FwdModel):
                 raise Hazard(f"S{i}#{u} overwrites P{i} {self.p[i][:3]} before P V read it")
             self.s_val[i], self.s_loaded[i], self.hi[i], self.p[i] = u, set(), ("S", u), None
             return
+        if op[0] == "PV":  # the V stage carries its query tile's tag; P and O as in the base model
+            _, i, sv, (gl, t, tag) = op
+            for c in range(2):
+                self.read_smem(("v", sv, c), (gl, t, tag))
+            op = ("PV_checked", i, sv, (gl, t))
+        if op[0] == "PV_checked":
+            _, i, sv, (it, t) = op
+            if self.p[i] is None or self.p[i][:3] != ["stored", it, t]:
+                raise Hazard(f"P V{i} of {(it, t)} reads P {self.p[i] and self.p[i][:3]}")
+            self.p[i][0] = "read"
+            if t == 0:
+                if self.o[i] is not None and len(self.o_read[i]) < 4:
+                    raise Hazard(f"P V{i} of item {it} restarts O{i} before the epilogue of {self.o[i]} read it")
+                self.o_read[i] = set()
+            elif self.o[i] != (it, t - 1):
+                raise Hazard(f"P V{i} of {(it, t)} accumulates onto O{i} at {self.o[i]}")
+            self.o[i] = (it, t)
+            return
         super().tensor_op(op)
 
     def local_op(self, role, op):
@@ -222,7 +270,8 @@ class GroupedModel(FwdModel):
 
     # ---------------------------------------------------------------- scheduler hooks
     def roles(self):
-        roles = {"builder": self.builder(), "producer": self.producer(), "mma": self.mma()}
+        roles = {"builder": self.builder(), "producer_k": self.producer("k"), "producer_v": self.producer("v"),
+                 "mma": self.mma()}
         for i in range(2):
             for w in range(4):
                 roles[("softmax", i, w)] = self.softmax_warp(i, w)
@@ -231,15 +280,19 @@ class GroupedModel(FwdModel):
     def pipe_readers(self, op):
         if op[0] == "S":
             return [("q", c) for c in (2 * op[1], 2 * op[1] + 1)] + [("k", op[3], c) for c in range(2)]
+        if op[0] == "PV":
+            return [("v", op[2], c) for c in range(2)]
         return super().pipe_readers(op)
 
 
+# (shared steps, key tiles of query tile 0, of query tile 1, query tiles)
 GROUP_SETS = [
-    [(3, 2), (2, 2), (4, 2)],
-    [(5, 2), (0, 2), (1, 2), (0, 1), (3, 1), (2, 2)],   # empty groups, a last group of two blocks
-    [(1, 1), (2, 1), (1, 2), (6, 2), (0, 2), (0, 2), (2, 1)],
-    [(2, 2)] * 7,
-    [(0, 2), (0, 2), (0, 1)],
+    [(3, 3, 3, 2), (0, 2, 2, 2), (1, 4, 2, 2)],                           # shared, split, a tail of tile 0
+    [(2, 5, 2, 2), (0, 0, 0, 2), (0, 1, 0, 1), (0, 0, 0, 1), (0, 3, 0, 1), (1, 1, 2, 2)],
+    [(0, 1, 0, 1), (0, 2, 0, 1), (0, 1, 3, 2), (2, 2, 6, 2), (0, 0, 0, 2), (0, 0, 3, 2), (0, 2, 0, 1)],
+    [(0, 2, 2, 2)] * 7,                                                    # split steps only
+    [(0, 0, 0, 2), (0, 0, 0, 2), (0, 0, 0, 1)],
+    [(0, 4, 1, 2), (0, 1, 4, 2), (0, 3, 0, 2), (4, 4, 4, 2)],              # one query tile empty, tails
 ]
 
 
@@ -262,12 +315,15 @@ def test_queue_with_no_group_for_this_cta_ends_cleanly():
     "softmax_frees_early",    # softmax warps release a group before walking its key stream
     "shared_counters",        # one p_full / o_empty counter for both query tiles
     "q_free_first_s",         # Q released after the group's first S instead of its last
+    "split_as_shared",        # a step with one tile per query tile read from one stage
+    "v_free_first_pv",        # a shared V stage released by the first query tile's P V
 ])
 def test_grouped_planted_mistakes_are_caught(plant):
     caught = 0
     for seed in range(40):
         try:
-            GroupedModel([(3, 2), (2, 1), (4, 2), (1, 1), (2, 2), (3, 1)], seed=seed, plant=plant).run()
+            GroupedModel([(1, 3, 2, 2), (0, 2, 0, 1), (2, 4, 3, 2), (0, 1, 0, 1), (0, 2, 3, 2), (0, 3, 0, 1)],
+                         seed=seed, plant=plant).run()
         except Hazard:
             caught += 1
     assert caught > 0, plant
