@@ -17,10 +17,11 @@
 // runs two independent fused-multiply-add chains in channel order -- the
 // exact fp32 order the selection is defined with.  Scores never reach HBM:
 // they stay in shared memory as order-keys.
-// One warp per query block then finds the k-th largest key by a 32-step
-// bitwise search (each step: count keys >= candidate, warp reduction), and
-// writes the selected ids in ascending order with ballots; ties at the
-// threshold go to the lower block index.
+// One warp per query block then finds the k-th largest key by a bitwise
+// search of at most 32 steps (each step: count keys >= candidate, warp
+// reduction; it stops once exactly k keys pass), and writes the selected ids
+// in ascending order with ballots; ties at the threshold go to the lower
+// block index.
 //
 // Compression branch ("FastVideo VSA", section "Checkpoint behavior": the
 // learned gate_compress projection; FastVideo commit log: the gate-compress

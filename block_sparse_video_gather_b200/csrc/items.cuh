@@ -126,12 +126,12 @@ __device__ __forceinline__ void tile_item(const Geo& g, int H, int blk0, int bh,
 }
 
 
-constexpr int kRows = 8;       // query blocks per score item (one per warp in the selection)
-constexpr int kChunk = 64;     // key blocks per shared-memory chunk
-constexpr int kKStride = 132;  // row stride (floats): 16-byte rows, float4 reads of a warp take 4 wavefronts
+constexpr int kRows = 8;     // query blocks per score item (one per warp in the selection)
 constexpr int kThreads = 256;
-constexpr int kGroups = kThreads / kChunk;      // row groups (4)
-constexpr int kRowsPerGroup = kRows / kGroups;  // rows per thread (2)
+constexpr int kChunk = kThreads;  // key blocks per pass: one per thread
+// One buffer of the key-mean ring: kChunk keys x 16 channels at a row stride
+// of 20 floats (or fewer keys x more channels); two buffers.
+constexpr int kSlabFloats = kChunk * 20;
 
 // fp32 loads: read-only path for inputs of the launch, L2-only for data
 // that other CTAs of the same launch wrote.
@@ -150,9 +150,13 @@ __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc, boo
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
 }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Wait until at most one committed group of this thread is still in flight.
+__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 __host__ __device__ constexpr size_t score_smem_bytes_c(int NB) {
-  return sizeof(float) * (kRows * 128 + kChunk * kKStride) + sizeof(uint32_t) * kRows * static_cast<size_t>(NB) +
+  return sizeof(float) * (kRows * 128 + 2 * kSlabFloats) + sizeof(uint32_t) * kRows * static_cast<size_t>(NB) +
          sizeof(float) * kRows;
 }
 inline size_t score_smem_bytes(int NB) { return score_smem_bytes_c(NB); }
@@ -168,16 +172,53 @@ __device__ __forceinline__ float key_value(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
+// The k-th largest of the order keys key[lo .. NB-1] as the selection's
+// threshold: the largest v with #{key >= v} >= topk, found bit by bit.  Once
+// exactly topk keys are >= v the selection is decided (no tie straddles v,
+// and the selection pass takes every key >= v), so the search stops there.
+// KR > 0: each lane holds its candidates lo + lane + 32 i (i < KR) in
+// registers for the passes (NB - lo <= 32 KR); KR = 0 reads them from
+// shared memory every pass.  Absent candidates count as 0, below every
+// candidate threshold (>= 1).
+template <int KR>
+__device__ __forceinline__ uint32_t select_threshold(const uint32_t* key, int lo, int NB, int topk, int lane) {
+  uint32_t kr[KR > 0 ? KR : 1];
+#pragma unroll
+  for (int i = 0; i < KR; ++i) {
+    const int j = lo + lane + 32 * i;
+    kr[i] = j < NB ? key[j] : 0u;
+  }
+  uint32_t tau = 0;
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t cand = tau | (1u << bit);
+    unsigned cnt = 0;
+    if (KR > 0) {
+#pragma unroll
+      for (int i = 0; i < KR; ++i) cnt += kr[i] >= cand;
+    } else {
+      for (int j = lo + lane; j < NB; j += 32) cnt += key[j] >= cand;
+    }
+    cnt = __reduce_add_sync(0xffffffffu, cnt);
+    if (cnt >= static_cast<unsigned>(topk)) {
+      tau = cand;
+      if (cnt == static_cast<unsigned>(topk)) break;
+    }
+  }
+  return tau;
+}
+
 // Scores, selection and compression branch of query blocks r0 .. r0+7 of
 // head bh.  `sm` is score_smem_bytes(NB) of shared memory.  COHERENT: the
 // block means were written by other CTAs of the same launch, so they are
 // read through L2 only (never the read-only path).
 //
-// A thread owns one key block of the current chunk and kRowsPerGroup query
-// blocks; each score is one fused-multiply-add chain over the channels in
+// A thread owns one key block of the current pass (up to kChunk blocks) and
+// all eight query blocks: eight fused-multiply-add chains over the channels in
 // order (four channels per step: one 16-byte load of the key row, one
-// broadcast 16-byte load per query row).  Block means reach shared memory by
-// cp.async through L2, every copy of a chunk in flight at once.
+// broadcast 16-byte load per query row), so each key row is read from shared
+// memory once.  Key means reach shared memory by cp.async through L2 in
+// slabs of channels (16 for a full pass, more when the pass has fewer keys),
+// two buffers: the next slab loads while the current one is scored.
 //
 // The selection follows `rule` (common.cuh): a forced-empty row writes count
 // 0; a prefix query row under the tile-64 rule lists every block; any other
@@ -188,10 +229,10 @@ __device__ __forceinline__ void score_item(int NB, int topk, const SelectRule& r
                                            const float* qbar, const float* kbar, int32_t* __restrict__ idx,
                                            int32_t* __restrict__ num, const float* vbar,
                                            float* __restrict__ o_compress, float scale, float* sm) {
-  float* q_s = sm;                               // [kRows][128]
-  float* k_s = q_s + kRows * 128;                // [kChunk][kKStride]
-  uint32_t* keys = reinterpret_cast<uint32_t*>(k_s + kChunk * kKStride);  // [kRows][NB]
-  float* wsum = reinterpret_cast<float*>(keys + kRows * NB);              // [kRows]
+  float* q_s = sm;                                                          // [kRows][128]
+  float* k_s = q_s + kRows * 128;                                           // [2][kSlabFloats]
+  uint32_t* keys = reinterpret_cast<uint32_t*>(k_s + 2 * kSlabFloats);     // [kRows][NB]
+  float* wsum = reinterpret_cast<float*>(keys + kRows * NB);                // [kRows]
 
   const int tid = threadIdx.x;
   const float* qh = qbar + static_cast<long long>(bh) * NB * 128;
@@ -204,41 +245,56 @@ __device__ __forceinline__ void score_item(int NB, int topk, const SelectRule& r
     cp_async16(q_s + i, ok ? qh + static_cast<long long>(r0) * 128 + i : qh, ok);  // rows past NB read as 0
   }
 
-  constexpr int kCopies = kChunk * 128 / (4 * kThreads);  // 16-byte copies per thread per chunk (8)
-  const int j_loc = tid % kChunk;
-  const int rg = tid / kChunk;  // owns query rows rg*kRowsPerGroup ..
   for (int c0 = 0; c0 < NB; c0 += kChunk) {
-    const int nrow = min(kChunk, NB - c0);
-    __syncthreads();  // the previous chunk is no longer read
+    const int nk = min(kChunk, NB - c0);
+    int C = 16;  // channels per slab: as many as one buffer holds for this pass
+    while (C < 128 && nk * (2 * C + 4) <= kSlabFloats) C *= 2;
+    const int stride = C + 4;  // 16-byte rows, conflict-free float4 reads
+    const int nslab = 128 / C, units = nk * (C / 4);
+    auto issue = [&](int sl) {  // slab sl into buffer sl & 1, one commit group
+      float* dst = k_s + (sl & 1) * kSlabFloats;
+      const int cpr = C / 4;
+      for (int u = tid; u < units; u += kThreads) {
+        const int key = u / cpr, part = u - key * cpr;
+        cp_async16(dst + key * stride + 4 * part, kh + static_cast<long long>(c0 + key) * 128 + sl * C + 4 * part,
+                   true);
+      }
+      cp_async_commit();
+    };
+    __syncthreads();  // the previous pass no longer reads the buffers
+    issue(0);
+    float acc[kRows];
 #pragma unroll
-    for (int it = 0; it < kCopies; ++it) {
-      const int i4 = tid + it * kThreads;  // 16-byte unit in the chunk; 32 per key row
-      const int jr = i4 >> 5;
-      if (jr < nrow) cp_async16(k_s + jr * kKStride + 4 * (i4 & 31), kh + static_cast<long long>(c0) * 128 + 4 * i4, true);
-    }
-    cp_async_wait();
-    __syncthreads();
-    if (j_loc < nrow) {
-      float acc[kRowsPerGroup];
-#pragma unroll
-      for (int r = 0; r < kRowsPerGroup; ++r) acc[r] = 0.0f;
-      const float* kr = k_s + j_loc * kKStride;
-      const float* q0 = q_s + (rg * kRowsPerGroup) * 128;
+    for (int r = 0; r < kRows; ++r) acc[r] = 0.0f;
+    for (int sl = 0; sl < nslab; ++sl) {
+      if (sl + 1 < nslab) {
+        issue(sl + 1);
+        cp_async_wait_1();
+      } else {
+        cp_async_wait_0();
+      }
+      __syncthreads();  // slab sl (and the query rows) visible to every thread
+      if (tid < nk) {
+        const float* kr = k_s + (sl & 1) * kSlabFloats + tid * stride;
+        const float* qc = q_s + sl * C;
 #pragma unroll 4
-      for (int d = 0; d < 128; d += 4) {
-        const float4 kv = *reinterpret_cast<const float4*>(kr + d);
+        for (int d = 0; d < C; d += 4) {
+          const float4 kv = *reinterpret_cast<const float4*>(kr + d);
 #pragma unroll
-        for (int r = 0; r < kRowsPerGroup; ++r) {
-          const float4 qv = *reinterpret_cast<const float4*>(q0 + r * 128 + d);
-          acc[r] = __fmaf_rn(qv.x, kv.x, acc[r]);
-          acc[r] = __fmaf_rn(qv.y, kv.y, acc[r]);
-          acc[r] = __fmaf_rn(qv.z, kv.z, acc[r]);
-          acc[r] = __fmaf_rn(qv.w, kv.w, acc[r]);
+          for (int r = 0; r < kRows; ++r) {
+            const float4 qv = *reinterpret_cast<const float4*>(qc + r * 128 + d);
+            acc[r] = __fmaf_rn(qv.x, kv.x, acc[r]);
+            acc[r] = __fmaf_rn(qv.y, kv.y, acc[r]);
+            acc[r] = __fmaf_rn(qv.z, kv.z, acc[r]);
+            acc[r] = __fmaf_rn(qv.w, kv.w, acc[r]);
+          }
         }
       }
-      const int j = c0 + j_loc;
+      __syncthreads();  // buffer sl & 1 is free for slab sl + 2
+    }
+    if (tid < nk) {
 #pragma unroll
-      for (int r = 0; r < kRowsPerGroup; ++r) keys[(rg * kRowsPerGroup + r) * NB + j] = order_key(acc[r]);
+      for (int r = 0; r < kRows; ++r) keys[r * NB + c0 + tid] = order_key(acc[r]);
     }
   }
   __syncthreads();
@@ -263,15 +319,10 @@ __device__ __forceinline__ void score_item(int NB, int topk, const SelectRule& r
     const int lo = rule.n_pre;  // candidates lo .. NB-1; blocks 0 .. lo-1 always listed
     for (int j = lane; j < lo; j += 32) out[j] = j;
     const uint32_t* key = keys + r * NB;
-    // k-th largest key: the largest v with #{key >= v} >= topk
-    uint32_t tau = 0;
-    for (int bit = 31; bit >= 0; --bit) {
-      const uint32_t cand = tau | (1u << bit);
-      unsigned cnt = 0;
-      for (int j = lo + lane; j < NB; j += 32) cnt += key[j] >= cand;
-      cnt = __reduce_add_sync(0xffffffffu, cnt);
-      if (cnt >= static_cast<unsigned>(topk)) tau = cand;
-    }
+    const int nc = NB - lo;  // candidates
+    const uint32_t tau = nc <= 32 * 8    ? select_threshold<8>(key, lo, NB, topk, lane)
+                         : nc <= 32 * 20 ? select_threshold<20>(key, lo, NB, topk, lane)
+                                         : select_threshold<0>(key, lo, NB, topk, lane);
     unsigned gt = 0;
     for (int j = lo + lane; j < NB; j += 32) gt += key[j] > tau;
     gt = __reduce_add_sync(0xffffffffu, gt);
