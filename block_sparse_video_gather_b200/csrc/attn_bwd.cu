@@ -749,23 +749,108 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint4* __restrict__
 }
 
 // One CTA per (b*h).  Counts per key block, offsets, then rows in order.
+// Grids up to this many blocks build the transposed selection from a bitmap
+// (NB x NB bits of shared memory: 128 KB at 1024 blocks).
+constexpr int kK2qBitmapMaxNB = 1024;
+
+__host__ __device__ constexpr size_t k2q_smem_bytes(int NB) {
+  return NB <= kK2qBitmapMaxNB
+             ? (static_cast<size_t>(NB) * ((NB + 31) / 32) + 2 * static_cast<size_t>(NB)) * sizeof(int)
+             : 2 * static_cast<size_t>(NB) * sizeof(int);
+}
+
+// The transposed selection of one head: for each key block, the query blocks
+// that list it, ascending.  Grids of at most kK2qBitmapMaxNB blocks set one
+// bit per (key block, query block) and read each key block's list off its
+// bitmap (every step parallel); a head whose lists repeat an id (the repeat is
+// listed again) and larger grids place the rows one query block at a time.
 __global__ void __launch_bounds__(256) k2q_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ num,
                                                   int NB, int max_k, int32_t* __restrict__ k2q_off,
                                                   int32_t* __restrict__ k2q, unsigned int* status) {
   extern __shared__ int kq_sm[];
-  int* cnt = kq_sm;        // [NB]
-  int* cur = kq_sm + NB;   // [NB]
   const int bh = blockIdx.x;
   const int32_t* ih = idx + static_cast<long long>(bh) * NB * max_k;
   const int32_t* nh = num + static_cast<long long>(bh) * NB;
   int32_t* list = k2q + static_cast<long long>(bh) * NB * max_k;
-  for (int c = threadIdx.x; c < NB; c += blockDim.x) {
+  int32_t* off = k2q_off + static_cast<long long>(bh) * (NB + 1);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  bool bad = false;
+  if (NB <= kK2qBitmapMaxNB) {
+    const int W = (NB + 31) >> 5;
+    uint32_t* bits = reinterpret_cast<uint32_t*>(kq_sm);  // [NB key blocks][W words of query blocks]
+    int* cnt = kq_sm + NB * W;                            // [NB]
+    for (int i = tid; i < NB * W; i += blockDim.x) bits[i] = 0u;
+    __syncthreads();
+    bool dup = false;
+    for (long long e = tid; e < static_cast<long long>(NB) * max_k; e += blockDim.x) {
+      const int r = static_cast<int>(e / max_k), t = static_cast<int>(e - static_cast<long long>(r) * max_k);
+      int c = nh[r];
+      if (c < 0 || c > max_k) {
+        bad = true;
+        c = c < 0 ? 0 : max_k;
+      }
+      if (t >= c) continue;
+      const int kb = ih[e];
+      if (kb < 0 || kb >= NB) {
+        bad = true;
+        continue;
+      }
+      const uint32_t bit = 1u << (r & 31);
+      if (atomicOr(&bits[kb * W + (r >> 5)], bit) & bit) dup = true;
+    }
+    if (bad) atomicCAS(status, 0u, (unsigned)VSA_ERR_BAD_INDEX);
+    if (!__syncthreads_or(dup)) {
+      for (int kb = tid; kb < NB; kb += blockDim.x) {
+        int n = 0;
+        for (int w = 0; w < W; ++w) n += __popc(bits[kb * W + w]);
+        cnt[kb] = n;
+      }
+      __syncthreads();
+      if (warp == 0) {  // exclusive scan of the counts: lane l sums a contiguous run
+        const int per = (NB + 31) / 32, lo = lane * per, hi = min(NB, lo + per);
+        int sum = 0;
+        for (int c = lo; c < hi; ++c) sum += cnt[c];
+        int incl = sum;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, d);
+          if (lane >= d) incl += y;
+        }
+        int run = incl - sum;
+        for (int c = lo; c < hi; ++c) {
+          const int x = cnt[c];
+          cnt[c] = run;
+          off[c] = run;
+          run += x;
+        }
+        if (lane == 31) off[NB] = incl;
+      }
+      __syncthreads();
+      for (int kb = tid; kb < NB; kb += blockDim.x) {
+        int pos = cnt[kb];
+        for (int w = 0; w < W; ++w) {
+          uint32_t b = bits[kb * W + w];
+          while (b) {
+            list[pos++] = w * 32 + __ffs(b) - 1;
+            b &= b - 1u;
+          }
+        }
+      }
+      return;
+    }
+    __syncthreads();  // the bitmap is given up; the shared memory is reused below
+  }
+
+  // one query block at a time (repeated ids, or grids beyond the bitmap)
+  int* cnt = kq_sm;        // [NB]
+  int* cur = kq_sm + NB;   // [NB]
+  for (int c = tid; c < NB; c += blockDim.x) {
     cnt[c] = 0;
     cur[c] = 0;
   }
   __syncthreads();
-  bool bad = false;
-  for (long long e = threadIdx.x; e < static_cast<long long>(NB) * max_k; e += blockDim.x) {
+  for (long long e = tid; e < static_cast<long long>(NB) * max_k; e += blockDim.x) {
     const int r = static_cast<int>(e / max_k), t = static_cast<int>(e - static_cast<long long>(r) * max_k);
     int c = nh[r];
     if (c < 0 || c > max_k) {
@@ -782,9 +867,8 @@ __global__ void __launch_bounds__(256) k2q_kernel(const int32_t* __restrict__ id
   }
   if (bad) atomicCAS(status, 0u, (unsigned)VSA_ERR_BAD_INDEX);
   __syncthreads();
-  if (threadIdx.x == 0) {
+  if (tid == 0) {
     int run = 0;
-    int32_t* off = k2q_off + static_cast<long long>(bh) * (NB + 1);
     for (int c = 0; c < NB; ++c) {
       const int x = cnt[c];
       cnt[c] = run;
@@ -797,7 +881,7 @@ __global__ void __launch_bounds__(256) k2q_kernel(const int32_t* __restrict__ id
   for (int r = 0; r < NB; ++r) {
     int c = nh[r];
     c = c < 0 ? 0 : (c > max_k ? max_k : c);
-    for (int t = threadIdx.x; t < c; t += blockDim.x) {
+    for (int t = tid; t < c; t += blockDim.x) {
       const int kb = ih[static_cast<long long>(r) * max_k + t];
       if (kb < 0 || kb >= NB) continue;
       list[cnt[kb] + atomicAdd(&cur[kb], 1)] = r;
@@ -869,9 +953,10 @@ cudaError_t launch_attn_bwd(const Geo& g, const AttnBwdArgs& a, cudaStream_t str
                                                             static_cast<long long>(rows));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  // two int32 per key block of a head (counts, then write positions); above the
-  // default 48 KB the kernel opts in (the API caps NB at kBwdMaxBlocks)
-  const size_t k2q_smem = 2 * static_cast<size_t>(g.NB) * sizeof(int);
+  // the bitmap and counts (or, beyond the bitmap, two int32 per key block:
+  // counts, then write positions); above the default 48 KB the kernel opts in
+  // (the API caps NB at kBwdMaxBlocks)
+  const size_t k2q_smem = k2q_smem_bytes(g.NB);
   if (k2q_smem > 48 * 1024 &&
       (e = cudaFuncSetAttribute(k2q_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 static_cast<int>(k2q_smem))) != cudaSuccess)

@@ -254,3 +254,51 @@ def test_bwd_full_size(name):
         # top-k workloads give every row topk > 0 selections
         np.testing.assert_allclose(dvv[h].sum(axis=0), dov[h].sum(axis=0), rtol=0,
                                    atol=2e-2 * np.abs(dov[h]).sum(axis=0).max())
+
+
+def test_bwd_bad_ids_are_reported_and_skipped():
+    """A block id outside [0, NB) and a count above max_k: VSA_ERR_BAD_INDEX is
+    reported, the bad id is skipped and the count clamped (its list's -1 padding
+    then skipped as well), so the gradients equal the oracle's on the cleaned
+    lists."""
+    wl = workloads.custom(T=8, Hg=8, Wg=16, H=2, topk=1)
+    g, qt, kt, vt, do, idx, num = _problem(wl, "bf16", 4, seed=19, zero_rows=False)
+    bad_idx, bad_num = idx.copy(), num.copy()
+    r = int(np.flatnonzero(num[0, 0] >= 2)[0])
+    bad_idx[0, 0, r, num[0, 0, r] - 1] = g.NB + 3      # the last id of row r: out of range
+    idx[0, 0, r, num[0, 0, r] - 1] = -1                 # cleaned: dropped
+    num[0, 0, r] -= 1
+    bad_num[0, 1, 2] = 99                               # clamped to max_k; the -1 entries past the
+    plan = vsa.Plan.of(wl)                              # real count are skipped
+    q, k, v, d = (_dev(x, "bf16") for x in (qt, kt, vt, do))
+    ti, tn = torch.from_numpy(bad_idx).cuda(), torch.from_numpy(bad_num).cuda()
+    o, lse = vsa.sparse_attn_fwd(plan, q, k, v, ti, tn)
+    assert vsa.get_status() == vsa.VSA_ERR_BAD_INDEX
+    dq, dk, dv = vsa.sparse_attn_bwd(plan, q, k, v, o, lse, d, ti, tn)
+    torch.cuda.synchronize()
+    assert vsa.get_status() == vsa.VSA_ERR_BAD_INDEX
+    assert vsa.get_status() == vsa.VSA_OK
+    real = H.real_rows(wl)
+    rows = np.arange(wl.H * g.Sp, dtype=np.int64)
+    ref_dq = oracle.attn_bwd_q_rows(g, qt, kt, vt, do, idx, num, rows).reshape(dq.shape)
+    ref_dk, ref_dv = oracle.attn_bwd_kv(g, qt, kt, vt, do, idx, num)
+    _check("bad dq", _vals(_host(dq), "bf16")[:, :, real], ref_dq[:, :, real])
+    _check("bad dk", _vals(_host(dk), "bf16")[:, :, real], ref_dk[:, :, real])
+    _check("bad dv", _vals(_host(dv), "bf16")[:, :, real], ref_dv[:, :, real])
+
+
+def test_bwd_grid_beyond_the_transpose_bitmap():
+    """1100 64-token blocks (above the 1024 the transposed selection builds from
+    a bitmap): the lists are placed one query block at a time; dq on sampled
+    rows and dk, dv on sampled key blocks against the oracle."""
+    wl = workloads.custom(T=8, Hg=100, Wg=88, block=(4, 4, 4), H=1, topk=1)
+    g, qt, kt, vt, do, idx, num = _problem(wl, "bf16", 3, seed=21)
+    assert g.NB == 1100
+    dq, dk, dv = _gpu_bwd(wl, "bf16", qt, kt, vt, do, idx, num)
+    rng = np.random.default_rng(22)
+    real = np.flatnonzero(H.real_rows(wl))
+    rows = np.unique(np.concatenate([rng.choice(real, 400, replace=False), real[:3], real[-3:]]))
+    ref_dq = oracle.attn_bwd_q_rows(g, qt, kt, vt, do, idx, num, rows)
+    _check("NB 1100 dq rows", _vals(dq, "bf16").reshape(-1, 128)[rows], ref_dq)
+    picks = [0, 1, 517, g.NB - 2, g.NB - 1] + sorted(rng.choice(g.NB, 3, replace=False).tolist())
+    _check_key_blocks("NB 1100", wl, g, qt, kt, vt, do, idx, num, dk, dv, [0], picks)

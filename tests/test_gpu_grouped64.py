@@ -1,12 +1,15 @@
 """GPU parity of the fine stage for 64-token tiles, whose kernel groups four
-query blocks over the union of their selections (FastVideo commit log,
+query blocks per item, two per 128-row Q tile, each Q tile walking the union
+of its two selections (shared blocks first, loaded once for both Q tiles)
+(FastVideo commit log,
 examples/inference/basic/README.md: the tile-64 layout with non-uniform and
 zero-count rows).  Every case runs the fine stage on oracle-supplied indices
 and compares o / lse with the oracle at the parity tolerances: sorted and
 unsorted lists, lists that repeat an id (the group then walks its lists as
 given), whole groups with nothing selected, a trailing group of two query
-blocks, every block selected, bad ids and counts, B = 2, fp16, and a grid
-beyond the grouped kernel's bitmap capacity (NB > 1024)."""
+blocks, every block selected, bad ids and counts, B = 2, fp16, a grid beyond
+the grouped kernel's bitmap capacity (NB > 1024), and groups built to reach
+every shape of the two Q tiles' streams."""
 import numpy as np
 import pytest
 import torch
@@ -200,3 +203,60 @@ def test_shared_queue_on_small_grids():
     o_ref, lse_ref = oracle.attn_rows(g, qt, kt, vt, idx, num, rows)
     H.compare_o_lse(H.from_dev(o).reshape(-1, 128)[rows], lse.cpu().numpy().reshape(-1)[rows], o_ref, lse_ref,
                     "queue")
+
+
+def _stream_shapes(NB):
+    """Index lists whose groups of four take every shape of the two Q tiles'
+    streams (Q tile 0 = query blocks 0-1 of a group, Q tile 1 = blocks 2-3)."""
+    max_k = 12
+    idx = np.full((1, 1, NB, max_k), -1, dtype=np.int32)
+    num = np.zeros((1, 1, NB), dtype=np.int32)
+
+    def put(row, ids):
+        idx[0, 0, row, :len(ids)] = ids
+        num[0, 0, row] = len(ids)
+
+    # group 0: Q tile 0 selects nothing, Q tile 1 alone
+    put(2, [3, 9, 17, 30]); put(3, [9, 11])
+    # group 1: Q tile 1 selects nothing (two Q tiles, one empty)
+    put(4, [0, 5, 6]); put(5, [31])
+    # group 2: all four select the same 7 blocks (every tile shared, the last
+    # one half empty)
+    for r in range(8, 12):
+        put(r, [1, 4, 8, 13, 21, 25, 29])
+    # group 3: disjoint selections, Q tile 0's stream longer (no shared tile)
+    put(12, [0, 2, 4, 6, 8]); put(13, [10, 12, 14, 16]); put(14, [1, 3]); put(15, [5])
+    # group 4: disjoint, Q tile 1's stream longer
+    put(16, [7]); put(18, [0, 2, 4, 6, 8, 10, 12]); put(19, [14, 16, 18, 20, 22])
+    # group 5: five shared blocks (an odd count: the third tile pairs the last
+    # shared block with each Q tile's first own block), four of Q tile 0's own,
+    # seven of Q tile 1's own
+    sh = [3, 6, 9, 12, 15]
+    put(20, sh[:3] + [0, 1]); put(21, sh[3:] + [2, 4]); put(22, sh + [5, 7, 8, 10]); put(23, [11, 13, 14])
+    # group 6: one query block of each Q tile selects, unsorted, partly shared
+    put(24, [30, 2, 17, 5]); put(27, [5, 30, 19])
+    # group 7: shared blocks only in Q tile 1's second block, with repeats
+    # across query blocks but none inside a list
+    put(28, [0, 31]); put(29, [31, 16]); put(30, [16]); put(31, [0, 8, 31])
+    return idx, num
+
+
+@pytest.mark.parametrize("queue", [False, True], ids=["static", "queue"])
+def test_every_shape_of_the_two_q_tile_streams(queue):
+    """Empty Q tiles, all-shared and no-shared groups, tails on either side, an
+    odd number of shared blocks: against the oracle, static and queued."""
+    wl, g, qt, kt, vt = _setup(8, 16, 16, H_=1)
+    assert g.NB == 32
+    idx, num = _stream_shapes(g.NB)
+    plan = vsa.Plan.of(wl)
+    ws = torch.zeros(4, dtype=torch.int32, device="cuda") if queue else None
+    o, lse = vsa.sparse_attn_fwd(plan, H.to_dev(qt), H.to_dev(kt), H.to_dev(vt), torch.from_numpy(idx).cuda(),
+                                 torch.from_numpy(num).cuda(), workspace=ws)
+    torch.cuda.synchronize()
+    assert vsa.get_status() == vsa.VSA_OK
+    if queue:
+        assert int(ws.abs().sum()) == 0
+    rows = np.flatnonzero(H.real_rows(wl))
+    o_ref, lse_ref = oracle.attn_rows(g, qt, kt, vt, idx, num, rows)
+    H.compare_o_lse(H.from_dev(o).reshape(-1, 128)[rows], lse.cpu().numpy().reshape(-1)[rows], o_ref, lse_ref,
+                    f"stream shapes queue={queue}")
