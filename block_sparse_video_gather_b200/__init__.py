@@ -29,7 +29,7 @@ SYMBOLS = (
     "vsa_sparse_attn_fwd", "vsa_sparse_attn_fwd_ex", "vsa_get_status", "vsa_strerror",
     "vsa_coarse_compress", "vsa_untile_gate", "vsa_tile_coarse", "vsa_tile_coarse_static",
     "vsa_sparse_attn_bwd_workspace", "vsa_sparse_attn_bwd", "vsa_quantize_nvfp4", "vsa_sparse_attn_fwd_nvfp4",
-    "vsa_coarse_topk_prefix", "vsa_tile_coarse_prefix", "vsa_sparse_attn_fwd_ws",
+    "vsa_coarse_topk_prefix", "vsa_tile_coarse_prefix", "vsa_sparse_attn_fwd_ws", "vsa_sparse_attn_fwd_nvfp4_ws",
 )
 
 VSA_BF16 = 0
@@ -86,6 +86,7 @@ def lib():
         L.vsa_sparse_attn_fwd.argtypes = [P, P, P, P, P, P, i, i, i, i, P, P, P]
         L.vsa_quantize_nvfp4.argtypes = [P, i, P, i, i, i, P, P, P]
         L.vsa_sparse_attn_fwd_nvfp4.argtypes = [P, i, P, P, P, P, P, P, P, i, i, i, i, P, P, P]
+        L.vsa_sparse_attn_fwd_nvfp4_ws.argtypes = [P, i, P, P, P, P, P, P, P, i, i, i, i, P, P, P, P]
         L.vsa_get_status.argtypes = [P, P]
         L.vsa_strerror.argtypes = [i]
         L.vsa_strerror.restype = ctypes.c_char_p
@@ -404,8 +405,10 @@ def quantize_nvfp4(plan: Plan, xt, codes=None, scales=None):
 
 
 def sparse_attn_fwd_nvfp4(plan: Plan, q_codes, q_scales, k_codes, k_scales, v, q2k_idx, q2k_num, o_out=None,
-                          lse_out=None):
-    """Fine stage with NVFP4 q, k (from quantize_nvfp4) and 16-bit v (tiled layout) -> (o, lse)."""
+                          lse_out=None, workspace=None):
+    """Fine stage with NVFP4 q, k (from quantize_nvfp4) and 16-bit v (tiled layout) -> (o, lse).
+    workspace: optional zeroed int32 device tensor of >= 2 elements for the 64-token
+    kernel's shared work queue (vsa_sparse_attn_fwd_nvfp4_ws); left zero by every call."""
     torch = _torch()
     B, H, Sp, D = v.shape
     max_k = q2k_idx.shape[-1]
@@ -421,13 +424,17 @@ def sparse_attn_fwd_nvfp4(plan: Plan, q_codes, q_scales, k_codes, k_scales, v, q
     if lse_out is None:
         lse_out = torch.empty((B, H, Sp), dtype=torch.float32, device=v.device)
     u8 = torch.uint8
-    _check(lib().vsa_sparse_attn_fwd_nvfp4(plan.handle, code, _ptr(q_codes, u8, "q_codes"),
-                                           _ptr(q_scales, u8, "q_scales"), _ptr(k_codes, u8, "k_codes"),
-                                           _ptr(k_scales, u8, "k_scales"), _ptr(v, v.dtype, "v"),
-                                           _ptr(q2k_idx, torch.int32, "q2k_idx"), _ptr(q2k_num, torch.int32, "q2k_num"),
-                                           max_k, B, H, D, _ptr(o_out, v.dtype, "o"),
-                                           _ptr(lse_out, torch.float32, "lse"), _stream()),
-           "vsa_sparse_attn_fwd_nvfp4")
+    args = [plan.handle, code, _ptr(q_codes, u8, "q_codes"), _ptr(q_scales, u8, "q_scales"),
+            _ptr(k_codes, u8, "k_codes"), _ptr(k_scales, u8, "k_scales"), _ptr(v, v.dtype, "v"),
+            _ptr(q2k_idx, torch.int32, "q2k_idx"), _ptr(q2k_num, torch.int32, "q2k_num"), max_k, B, H, D,
+            _ptr(o_out, v.dtype, "o"), _ptr(lse_out, torch.float32, "lse")]
+    if workspace is None:
+        _check(lib().vsa_sparse_attn_fwd_nvfp4(*args, _stream()), "vsa_sparse_attn_fwd_nvfp4")
+    else:
+        if workspace.numel() < 2:
+            raise ValueError("workspace needs 2 int32")
+        _check(lib().vsa_sparse_attn_fwd_nvfp4_ws(*args, _ptr(workspace, torch.int32, "workspace"), _stream()),
+               "vsa_sparse_attn_fwd_nvfp4_ws")
     return o_out, lse_out
 
 
@@ -581,7 +588,7 @@ class Forward:
         """The fine-stage attention kernel alone."""
         if self.nvfp4:
             sparse_attn_fwd_nvfp4(self.plan, self.qc, self.qs, self.kc, self.ks, self.vt, self.idx, self.num,
-                                  o_out=self.ot, lse_out=self.lse)
+                                  o_out=self.ot, lse_out=self.lse, workspace=self.fws)
         else:
             sparse_attn_fwd(self.plan, self.qt, self.kt, self.vt, self.idx, self.num, o_out=self.ot,
                             lse_out=self.lse, workspace=self.fws)

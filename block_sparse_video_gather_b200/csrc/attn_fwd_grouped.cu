@@ -10,6 +10,7 @@
 #include "common.cuh"
 #include "fwd_common.cuh"
 #include "kernels.h"
+#include "nvfp4.cuh"
 #include "tiles.cuh"
 
 namespace vsa {
@@ -60,13 +61,38 @@ using namespace fwd;
 // ===========================================================================
 constexpr int kGroupBlocks = 4;
 constexpr int kGroupMaxWords = 32;
-// The five 32 KB tile stages after Q: a step that loads one tile per Q tile
-// takes two K and two V stages, and a V stage is held a softmax longer than
-// a K stage (S issues right after its load, P V only after the softmax), so
-// the V ring gets the deeper share.
-constexpr int kStagesKG = 2, kStagesVG = 3;
-static_assert(kStagesKG + kStagesVG == kStagesK + kStagesV, "same shared-memory map as the per-block kernel");
 static_assert(kGroupMaxNB == 32 * kGroupMaxWords, "bitmap capacity");
+
+// Shared-memory map of the two variants.  16-bit Q and K: the five 32 KB tile
+// stages after Q; a step that loads one tile per Q tile takes two K and two V
+// stages, and a V stage is held a softmax longer than a K stage (S issues
+// right after its load, P V only after the softmax), so the V ring gets the
+// deeper share.  NVFP4 Q and K: a Q tile is 8 KB of codes + a 1 KB scale
+// tile, a key tile 8 KB of codes + a 1 KB scale tile assembled from its two
+// blocks' halves, so both rings get four stages.
+template <bool FP4>
+struct GMap;
+template <>
+struct GMap<false> {
+  static constexpr int kKS = 2, kVS = 3;
+  static constexpr uint32_t kQ = 0, kQsf = 0, kK = kQ + 2 * kTileBytes, kKsf = 0;
+  static constexpr uint32_t kKStage = kTileBytes, kKsfStage = 0, kQTile = kTileBytes;
+  static constexpr uint32_t kV = kK + kKS * kKStage;
+  static constexpr uint32_t kBar = kV + kVS * kTileBytes;
+};
+template <>
+struct GMap<true> {
+  static constexpr int kKS = 4, kVS = 4;
+  static constexpr uint32_t kQTile = nvfp4::kCodeTileBytes;
+  static constexpr uint32_t kQ = 0, kQsf = kQ + 2 * kQTile, kK = kQsf + 2 * nvfp4::kSfTileBytes;
+  static constexpr uint32_t kKStage = nvfp4::kCodeTileBytes, kKsfStage = nvfp4::kSfTileBytes;
+  static constexpr uint32_t kKsf = kK + kKS * kKStage;
+  static constexpr uint32_t kV = kKsf + kKS * kKsfStage;
+  static constexpr uint32_t kBar = kV + kVS * kTileBytes;
+};
+static_assert(GMap<false>::kBar == kSmemBar, "16-bit map: the per-block kernel's");
+static_assert(GMap<true>::kK % 1024 == 0 && GMap<true>::kV % 1024 == 0, "1 KB-aligned rings");
+constexpr int kMaxStages = 4;
 
 constexpr int kShared = kGroupBlocks;  // bitmap of the blocks both Q tiles use
 
@@ -84,19 +110,30 @@ struct GroupInfo {
 
 struct GroupBarriers {
   uint64_t q_full, q_empty;
-  uint64_t k_full[kStagesKG], k_empty[kStagesKG];
-  uint64_t v_full[kStagesVG], v_empty[kStagesVG];
+  uint64_t k_full[kMaxStages], k_empty[kMaxStages];
+  uint64_t v_full[kMaxStages], v_empty[kMaxStages];
   uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
+  uint64_t s_read[2];  // NVFP4: S_i loaded by its softmax (its last 64 columns free for scales)
   uint64_t grp_full[2], grp_free[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
 };
-static_assert(sizeof(GroupBarriers) <= 256, "barrier block too large");
+constexpr uint32_t kBarBytes = 512;
+static_assert(sizeof(GroupBarriers) <= kBarBytes, "barrier block too large");
 
-constexpr uint32_t kSmemGroups = kSmemBar + 256;
-constexpr uint32_t kSmemTotalG = kSmemGroups + 2 * sizeof(GroupInfo) + 1024;
-static_assert(kSmemTotalG <= 232448, "grouped kernel exceeds the shared memory of one CTA");
+template <bool FP4>
+struct GSmem {
+  static constexpr uint32_t kGroups = GMap<FP4>::kBar + kBarBytes;
+  static constexpr uint32_t kTotal = kGroups + 2 * sizeof(GroupInfo) + 1024;
+  static_assert(kTotal <= 232448, "grouped kernel exceeds the shared memory of one CTA");
+};
+
+// Launch parameters: the 16-bit kernel's, plus the NVFP4 scale tiles.
+struct GroupParams : Params {
+  const uint8_t* q_sf;
+  const uint8_t* k_sf;
+};
 constexpr uint32_t kGroupConsumers = 11;  // two producers, MMA, 8 softmax warps: one arrival each
 
 __device__ __forceinline__ bool gwarp_wait(uint64_t* bar, uint32_t parity, GroupBarriers* bars,
@@ -243,17 +280,25 @@ __device__ __forceinline__ float softmax_halves(uint32_t (&sv)[128], bool ha, bo
   return ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
 }
 
-template <bool F16>
+// FP4: Q and K as NVFP4 codes with E4M3 scale tiles (tm_q: 128-row boxes of
+// 64-byte code rows; tm_k: 64-row boxes), S = Q K^T a block-scaled FP4
+// product per 64-token block of the key tile (N = 64), its scales copied into
+// the other Q tile's free S columns once that tile's softmax has loaded its
+// latest S (s_read); V, P and O as in the 16-bit variant.
+template <bool F16, bool FP4>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_grouped64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ Params p) {
+                              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ GroupParams p) {
+  using M = GMap<FP4>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem + kSmemQ;
-  uint8_t* sK = smem + kSmemK;
-  uint8_t* sV = sK + kStagesKG * kTileBytes;
-  GroupBarriers* bars = reinterpret_cast<GroupBarriers*>(smem + kSmemBar);
-  GroupInfo* grp = reinterpret_cast<GroupInfo*>(smem + kSmemGroups);
+  uint8_t* sQ = smem + M::kQ;
+  uint8_t* sQsf = smem + M::kQsf;
+  uint8_t* sK = smem + M::kK;
+  uint8_t* sKsf = smem + M::kKsf;
+  uint8_t* sV = smem + M::kV;
+  GroupBarriers* bars = reinterpret_cast<GroupBarriers*>(smem + M::kBar);
+  GroupInfo* grp = reinterpret_cast<GroupInfo*>(smem + GSmem<FP4>::kGroups);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -265,16 +310,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
     mbar_init(&bars->q_empty, 1);
-    for (int s = 0; s < kStagesKG; ++s) {
+    for (int s = 0; s < M::kKS; ++s) {
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->k_empty[s], 1);
     }
-    for (int s = 0; s < kStagesVG; ++s) {
+    for (int s = 0; s < M::kVS; ++s) {
       mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->v_empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->s_full[i], 1);
+      mbar_init(&bars->s_read[i], 128);
       mbar_init(&bars->p_full[i], 128);
       mbar_init(&bars->o_full[i], 1);
       mbar_init(&bars->o_empty[i], 128);
@@ -398,7 +444,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!vside) tma_prefetch_desc(&tm_q);
     const uint64_t pol_kv = policy_evict_last();
     const uint64_t pol_q = policy_evict_first();
-    const int stages = vside ? kStagesVG : kStagesKG;
+    const int stages = vside ? M::kVS : M::kKS;
+    const long long sf_tiles = g.Sp >> 7;  // NVFP4: 128-row scale tiles per head
     uint8_t* const ring = vside ? sV : sK;
     uint64_t* const full = vside ? bars->v_full : bars->k_full;
     uint64_t* const empty = vside ? bars->v_empty : bars->k_empty;
@@ -419,23 +466,60 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (n > 0) {
         if (!vside) {
           if (!gwarp_wait(&bars->q_empty, (qit & 1) ^ 1, bars, p.status)) break;
-          mbar_arrive_expect_tx_w(&bars->q_full, nq * kTileBytes);
           const int qrow = static_cast<int>(base + static_cast<long long>(qb0) * 64);
-          for (int i = 0; i < nq; ++i)
-            for (int hf = 0; hf < 2; ++hf)
-              tma_load_2d_w(sQ + i * kTileBytes + hf * kHalfBytes, &tm_q, hf * 64, qrow + i * 128, &bars->q_full,
-                            pol_q);
+          if constexpr (FP4) {  // codes + the Q tile's scale tile (qb0 * 64 is 256-row aligned)
+            mbar_arrive_expect_tx_w(&bars->q_full, nq * (M::kQTile + nvfp4::kSfTileBytes));
+            for (int i = 0; i < nq; ++i) {
+              tma_load_2d_w(sQ + i * M::kQTile, &tm_q, 0, qrow + i * 128, &bars->q_full, pol_q);
+              const long long tile = bh * sf_tiles + ((qb0 * 64 + i * 128) >> 7);
+              nvfp4::bulk_load_w(sQsf + i * nvfp4::kSfTileBytes, p.q_sf + tile * nvfp4::kSfTileBytes,
+                                 nvfp4::kSfTileBytes, &bars->q_full);
+            }
+          } else {
+            mbar_arrive_expect_tx_w(&bars->q_full, nq * kTileBytes);
+            for (int i = 0; i < nq; ++i)
+              for (int hf = 0; hf < 2; ++hf)
+                tma_load_2d_w(sQ + i * kTileBytes + hf * kHalfBytes, &tm_q, hf * 64, qrow + i * 128, &bars->q_full,
+                              pol_q);
+          }
           ++qit;
         }
         // one stage per distinct tile of a step, Q tile 0's first
         auto load = [&](int krow0, int krow1) -> bool {
           const int st = it % stages;
           if (!gwarp_wait(&empty[st], ((it / stages) & 1) ^ 1, bars, p.status)) return false;
-          mbar_arrive_expect_tx_w(&full[st], kTileBytes);
-          for (int hf = 0; hf < 2; ++hf) {
-            uint8_t* dst = ring + st * kTileBytes + hf * kHalfBytes;
-            tma_load_2d_w(dst, tm, hf * 64, krow0, &full[st], pol_kv);
-            tma_load_2d_w(dst + kHalfBytes / 2, tm, hf * 64, krow1, &full[st], pol_kv);
+          if (FP4 && !vside) {
+            // K codes: a 64-row box per block, stacked into one 128-row tile.
+            // Scales: a 64-token block is one half of its scale tile, so the
+            // two blocks' halves are assembled into one 128-row scale tile (block
+            // a's rows 0-63, block b's 64-127): in each 16-byte row r%32 of each
+            // channel half, block a's 8 bytes of columns 2 (kb & 1) .. +1, then
+            // block b's.  Generic stores, made visible to the tensor core's copy
+            // by a proxy fence before the stage is announced on k_full.
+            const long long r0h = krow0 - base, r1h = krow1 - base;
+            const uint8_t* ta = p.k_sf + (bh * sf_tiles + (r0h >> 7)) * nvfp4::kSfTileBytes + 8 * ((r0h >> 6) & 1);
+            const uint8_t* tb = p.k_sf + (bh * sf_tiles + (r1h >> 7)) * nvfp4::kSfTileBytes + 8 * ((r1h >> 6) & 1);
+            uint8_t* sfd = sKsf + st * M::kKsfStage;
+#pragma unroll
+            for (int e = lane; e < 128; e += 32) {  // 2 channel halves x 32 rows x 2 blocks of 8 bytes
+              const int kh = e >> 6, rr = (e >> 1) & 31, blk = e & 1;
+              const uint32_t off = kh * 512 + rr * 16;
+              const uint2 v = __ldg(reinterpret_cast<const uint2*>((blk ? tb : ta) + off));
+              *reinterpret_cast<uint2*>(sfd + off + 8 * blk) = v;
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            mbar_arrive_expect_tx_w(&full[st], M::kKStage);
+            uint8_t* kdst = sK + st * M::kKStage;
+            tma_load_2d_w(kdst, &tm_k, 0, krow0, &full[st], pol_kv);
+            tma_load_2d_w(kdst + M::kKStage / 2, &tm_k, 0, krow1, &full[st], pol_kv);
+          } else {
+            mbar_arrive_expect_tx_w(&full[st], kTileBytes);
+            for (int hf = 0; hf < 2; ++hf) {
+              uint8_t* dst = ring + st * kTileBytes + hf * kHalfBytes;
+              tma_load_2d_w(dst, tm, hf * 64, krow0, &full[st], pol_kv);
+              tma_load_2d_w(dst + kHalfBytes / 2, tm, hf * 64, krow1, &full[st], pol_kv);
+            }
           }
           ++it;
           return true;
@@ -473,21 +557,48 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    const uint64_t dq0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
-    const uint64_t dk0 = sdesc_sw128(smem_u32(sK), 16, 1024);
+    const uint64_t dq0 = FP4 ? nvfp4::sdesc_sw64(smem_u32(sQ)) : sdesc_sw128(smem_u32(sQ), 16, 1024);
+    const uint64_t dk0 = FP4 ? nvfp4::sdesc_sw64(smem_u32(sK)) : sdesc_sw128(smem_u32(sK), 16, 1024);
     const uint64_t dv0 = sdesc_sw128(smem_u32(sV), kHalfBytes, 1024);
     constexpr uint64_t kTileDesc = kTileBytes >> 4;
     int kit = 0, vit = 0, qit = 0;
     int tiles0 = 0, tiles1 = 0, items0 = 0, items1 = 0;  // per Q tile: P V products, groups
+    int sn0 = 0, sn1 = 0;                                // NVFP4: S products issued per Q tile
     bool ok = true;
-    auto issue_s = [&](int i, int sk) {
+    // S_i = Q_i K^T for the key tile in K stage sk
+    auto issue_s = [&](int i, int sk) -> bool {
       const uint32_t d = tmem + i * 128;
-      const uint64_t a = dq0 + i * kTileDesc, b = dk0 + sk * kTileDesc;
+      if constexpr (FP4) {
+        // the scales go into the other Q tile's S columns: free once its softmax
+        // has loaded its latest S
+        const int j = 1 - i, nj = j == 0 ? sn0 : sn1;
+        if (nj > 0 && !gwarp_wait(&bars->s_read[j], (nj - 1) & 1, bars, p.status)) return false;
+        tc_fence_after();
+        const uint32_t sf = tmem + nvfp4::sf_col(i);
+        const uint8_t* qsf = sQsf + i * nvfp4::kSfTileBytes;
+        const uint8_t* ksf = sKsf + sk * M::kKsfStage;
+        nvfp4::tmem_cp_32x128_w(sf + 0, nvfp4::sdesc_rows16(smem_u32(qsf)));
+        nvfp4::tmem_cp_32x128_w(sf + 4, nvfp4::sdesc_rows16(smem_u32(qsf + 512)));
+        nvfp4::tmem_cp_32x128_w(sf + 8, nvfp4::sdesc_rows16(smem_u32(ksf)));
+        nvfp4::tmem_cp_32x128_w(sf + 12, nvfp4::sdesc_rows16(smem_u32(ksf + 512)));
+        // the Q tile and the key tile are each one whole scale tile: two N = 128
+        // products (64 channels each)
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t off = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
-        mma_ss_w(d, a + off, b + off, Idesc<F16>::S, kk > 0 ? 1u : 0u);
+        for (int kh = 0; kh < 2; ++kh) {
+          const uint64_t a = dq0 + ((i * M::kQTile + kh * 32) >> 4);
+          const uint64_t b = dk0 + ((sk * M::kKStage + kh * 32) >> 4);
+          nvfp4::mma_fp4_w(d, a, b, nvfp4::idesc_s(128), sf + 4 * kh, sf + 8 + 4 * kh, kh > 0 ? 1u : 0u);
+        }
+        if (i == 0) ++sn0; else ++sn1;
+      } else {
+        const uint64_t a = dq0 + i * kTileDesc, b = dk0 + sk * kTileDesc;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+          mma_ss_w(d, a + off, b + off, Idesc<F16>::S, kk > 0 ? 1u : 0u);
+        }
       }
+      return true;
     };
     auto issue_pv = [&](int i, int sv, bool acc) {
       const uint32_t d = tmem + 256 + i * 128, pa = tmem + i * 128;
@@ -521,8 +632,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (t >= 0 && t < lj) {  // P V product of Q tile j at step t
             const bool shared = t < ns;
             if (j == 0 || !shared) {
-              sv = vit % kStagesVG;
-              if (!(ok = gwarp_wait(&bars->v_full[sv], (vit / kStagesVG) & 1, bars, p.status))) break;
+              sv = vit % M::kVS;
+              if (!(ok = gwarp_wait(&bars->v_full[sv], (vit / M::kVS) & 1, bars, p.status))) break;
             }
             const int tj = j ? tiles1 : tiles0;
             if (!(ok = gwarp_wait(&bars->p_full[j], tj & 1, bars, p.status))) break;
@@ -543,11 +654,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (u < lj) {  // S product of Q tile j at step t + 1
             const bool shared = u < ns;
             if (j == 0 || !shared) {
-              sk = kit % kStagesKG;
-              if (!(ok = gwarp_wait(&bars->k_full[sk], (kit / kStagesKG) & 1, bars, p.status))) break;
+              sk = kit % M::kKS;
+              if (!(ok = gwarp_wait(&bars->k_full[sk], (kit / M::kKS) & 1, bars, p.status))) break;
               tc_fence_after();
             }
-            issue_s(j, sk);
+            if (!(ok = issue_s(j, sk))) break;
             mma_commit_w(&bars->s_full[j]);
             if (j == 1 || !shared) {  // the K stage's last reader is issued
               mma_commit_w(&bars->k_empty[sk]);
@@ -627,6 +738,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
           tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
           tmem_wait_ld();
+          if constexpr (FP4) {  // S is in registers: its last 64 columns may take the other tile's scales
+            tc_fence_before();
+            mbar_arrive(&bars->s_read[wg]);
+          }
           if (st_a == kTilePartial || st_b == kTilePartial) {
             // padded slots of a selected block (an unselected half is skipped below)
             const uint32_t mw[4] = {st_a == kTilePartial ? w0 : 0xffffffffu, st_a == kTilePartial ? w1 : 0xffffffffu,
@@ -636,6 +751,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           lsum = softmax_halves<F16>(sv, ha, hb, sl2, t, m_used, alpha, rescale, pk);
         } else {
           // nothing selected in this tile by this warp's query block
+          if constexpr (FP4) {  // S is not needed: its columns are free now
+            tc_fence_before();
+            mbar_arrive(&bars->s_read[wg]);
+          }
 #pragma unroll
           for (int j = 0; j < 64; ++j) pk[j] = 0u;
         }
@@ -707,18 +826,45 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+template <bool FP4>
+cudaError_t launch_grouped(const Geo& g, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                           const GroupParams& p, int BH, int num_sms, bool f16, cudaStream_t stream) {
+  const long long groups = static_cast<long long>(BH) * ((g.NB + kGroupBlocks - 1) / kGroupBlocks);
+  const int grid = static_cast<int>(groups < num_sms ? groups : num_sms);
+  auto kern = f16 ? attn_fwd_grouped64_kernel<true, FP4> : attn_fwd_grouped64_kernel<false, FP4>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GSmem<FP4>::kTotal);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreads, GSmem<FP4>::kTotal, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_attn_fwd_grouped64(const Geo& g, const CUtensorMap& tq, const CUtensorMap& tk,
                                       const CUtensorMap& tv, const fwd::Params& p, int BH, int num_sms, bool f16,
                                       cudaStream_t stream) {
-  const long long groups = static_cast<long long>(BH) * ((g.NB + kGroupBlocks - 1) / kGroupBlocks);
-  const int grid = static_cast<int>(groups < num_sms ? groups : num_sms);
-  auto kern = f16 ? attn_fwd_grouped64_kernel<true> : attn_fwd_grouped64_kernel<false>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTotalG);
-  if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, kSmemTotalG, stream>>>(tq, tk, tv, p);
-  return cudaGetLastError();
+  GroupParams gp;
+  static_cast<fwd::Params&>(gp) = p;
+  gp.q_sf = gp.k_sf = nullptr;
+  return launch_grouped<false>(g, tq, tk, tv, gp, BH, num_sms, f16, stream);
+}
+
+cudaError_t launch_attn_fwd_grouped64_fp4(const Geo& g, const CUtensorMap& tq, const CUtensorMap& tk,
+                                          const CUtensorMap& tv, const AttnFp4Args& a, cudaStream_t stream) {
+  GroupParams gp;
+  gp.idx = a.idx;
+  gp.num = a.num;
+  gp.max_k = a.max_k;
+  gp.BH = a.BH;
+  gp.o = a.o;
+  gp.lse = a.lse;
+  gp.status = a.status;
+  gp.scale_log2 = static_cast<float>(1.4426950408889634 / 11.313708498984761);  // log2(e) / sqrt(128)
+  gp.g = g;
+  gp.queue = a.queue;  // null: groups go to CTAs statically
+  gp.q_sf = a.q_sf;
+  gp.k_sf = a.k_sf;
+  return launch_grouped<true>(g, tq, tk, tv, gp, a.BH, a.num_sms, a.f16, stream);
 }
 
 }  // namespace vsa

@@ -52,7 +52,9 @@
 #include <cuda_bf16.h>
 
 #include "common.cuh"
+#include "fwd_common.cuh"
 #include "kernels.h"
+#include "nvfp4.cuh"
 #include "tiles.cuh"
 
 namespace vsa {
@@ -60,6 +62,7 @@ namespace vsa {
 namespace {
 
 using namespace tiles;
+using namespace nvfp4;
 
 // ---------------------------------------------------------------------------
 // Conversions
@@ -168,9 +171,8 @@ __global__ void __launch_bounds__(256) quant_nvfp4_kernel(const uint4* __restric
 
 constexpr int kThreads = 384;
 constexpr int kStagesK = 4, kStagesV = 3;
-constexpr uint32_t kQTileBytes = 128 * 64;       // 128 rows x 64 B of codes
-constexpr uint32_t kSfTileBytes = 1024;          // scales of a 128-row tile
-constexpr uint32_t kKTileBytes = 128 * 64;       // 128 keys x 64 B of codes
+constexpr uint32_t kQTileBytes = kCodeTileBytes;  // 128 rows x 64 B of codes
+constexpr uint32_t kKTileBytes = kCodeTileBytes;  // 128 keys x 64 B of codes
 constexpr uint32_t kKSfBytes = 2 * kSfTileBytes;  // a key tile's scale tiles (two for two 64-token blocks)
 constexpr uint32_t kVHalfBytes = 128 * 128;      // 128 keys x 64 channels x 2 B
 constexpr uint32_t kVTileBytes = 2 * kVHalfBytes;
@@ -187,72 +189,12 @@ constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s per wait
 constexpr int kRegsLaunch = 168, kRegsLow = 104, kRegsHigh = 200;
 static_assert(kThreads * kRegsLaunch == 128 * kRegsLow + 256 * kRegsHigh, "register split must match the launch");
 
-// S: E2M1 x E2M1 with UE4M3 block-16 scales, fp32 accumulate, M = 128, both
-// K-major (K = 64 codes per instruction).  Fields: A/B format E2M1 = 1 at bits
-// 7 and 10, N>>3 at 17, scale format UE4M3 = 0 at 23, M>>4 at 24.
-constexpr uint32_t idesc_s(uint32_t n) { return (1u << 7) | (1u << 10) | ((n >> 3) << 17) | ((128u >> 4) << 24); }
 
 template <bool F16>
 struct IdescPV {
   static constexpr uint32_t v = F16 ? idesc_f16_f32(128, 128, 0, 1) : idesc_bf16_f32(128, 128, 0, 1);
 };
 
-// Shared-memory descriptor, K-major with 64-byte swizzle (layout type 4),
-// 8-row atoms of 64 B (SBO 512).
-__device__ __forceinline__ uint64_t sdesc_sw64(uint32_t saddr) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
-  d |= static_cast<uint64_t>(16u >> 4) << 16;
-  d |= static_cast<uint64_t>(512u >> 4) << 32;
-  d |= static_cast<uint64_t>(1) << 46;
-  d |= static_cast<uint64_t>(4) << 61;
-  return d;
-}
-
-// Source of tcgen05.cp.32x128b: 32 rows of 16 B, no swizzle, 8-row core
-// matrices 128 B apart.
-__device__ __forceinline__ uint64_t sdesc_rows16(uint32_t saddr) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
-  d |= static_cast<uint64_t>(128u >> 4) << 16;
-  d |= static_cast<uint64_t>(128u >> 4) << 32;
-  d |= static_cast<uint64_t>(1) << 46;
-  return d;
-}
-
-// D[tmem] (+)= A[smem] * B[smem] with block scales from tensor memory.
-__device__ __forceinline__ void mma_fp4_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                          uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
-          d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
-      : "memory");
-}
-
-// 32 rows x 128 bits of shared memory -> 4 columns of tensor memory, copied
-// into every lane quarter.
-__device__ __forceinline__ void tmem_cp_32x128_w(uint32_t taddr, uint64_t src_desc) {
-  asm volatile(
-      "{\n\t.reg .pred e;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "@e tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;\n\t}" ::"r"(taddr),
-      "l"(src_desc)
-      : "memory");
-}
-
-__device__ __forceinline__ void bulk_load_w(void* smem_dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "{\n\t.reg .pred e;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "@e cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n\t}" ::"r"(
-          smem_u32(smem_dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
 
 struct Barriers {
   uint64_t q_full, q_empty;
@@ -354,8 +296,6 @@ __device__ __forceinline__ uint32_t tile_halves(const Params& p, int item, int n
   return (static_cast<uint32_t>(kb_a < 0 ? 0 : kb_a) & 1u) | ((static_cast<uint32_t>(kb_b < 0 ? 0 : kb_b) & 1u) << 1);
 }
 
-// First scale column of the product S_i (inside the other tile's S).
-__device__ __forceinline__ uint32_t sf_col(int i) { return i == 0 ? 192u : 64u; }
 
 template <int BS, bool F16>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -805,6 +745,9 @@ cudaError_t launch_attn_fwd_nvfp4(const Geo& g, const AttnFp4Args& a, cudaStream
   if (!make_tmap_codes(&tq, a.q, rows, 128) || !make_tmap_codes(&tk, a.k, rows, kv_box) ||
       !make_tmap(&tv, a.v, rows, kv_box, a.f16))
     return cudaErrorInvalidValue;
+  // 64-token blocks: four query blocks per item (two per 128-row Q tile) over
+  // the union of their selections, while the group bitmaps hold the grid
+  if (g.bs == 64 && g.NB <= kGroupMaxNB) return launch_attn_fwd_grouped64_fp4(g, tq, tk, tv, a, stream);
   Params p;
   p.idx = a.idx;
   p.num = a.num;

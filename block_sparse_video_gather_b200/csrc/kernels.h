@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -79,8 +80,14 @@ struct AttnFp4Args {
   unsigned int* status;
   int num_sms;
   bool f16;  // v and o are fp16 (else bf16)
+  int* queue = nullptr;  // 64-token plans: the grouped kernel's shared group queue (2 int32), or null
 };
 cudaError_t launch_attn_fwd_nvfp4(const Geo& g, const AttnFp4Args& a, cudaStream_t stream);
+// attn_fwd_grouped.cu: the grouped 64-token kernel with NVFP4 Q and K (four
+// query blocks per item); launch_attn_fwd_nvfp4 uses it for 64-token plans of
+// up to kGroupMaxNB blocks.  tq: 128-row boxes of codes, tk / tv: 64-row boxes.
+cudaError_t launch_attn_fwd_grouped64_fp4(const Geo& g, const CUtensorMap& tq, const CUtensorMap& tk,
+                                          const CUtensorMap& tv, const AttnFp4Args& a, cudaStream_t stream);
 
 // attn_bwd.cu
 struct AttnBwdArgs {

@@ -486,10 +486,11 @@ int vsa_quantize_nvfp4(vsa_plan_t plan, vsa_dtype_t dtype, const uint16_t* x_til
                                            reinterpret_cast<cudaStream_t>(stream)));
 }
 
-int vsa_sparse_attn_fwd_nvfp4(vsa_plan_t plan, vsa_dtype_t dtype, const uint8_t* q_codes, const uint8_t* q_scales,
-                              const uint8_t* k_codes, const uint8_t* k_scales, const uint16_t* v,
-                              const int32_t* q2k_idx, const int32_t* q2k_num, int max_k, int B, int H, int D,
-                              uint16_t* o, float* lse, vsa_stream_t stream) {
+namespace {
+int sparse_attn_fwd_nvfp4_impl(vsa_plan_t plan, vsa_dtype_t dtype, const uint8_t* q_codes, const uint8_t* q_scales,
+                               const uint8_t* k_codes, const uint8_t* k_scales, const uint16_t* v,
+                               const int32_t* q2k_idx, const int32_t* q2k_num, int max_k, int B, int H, int D,
+                               uint16_t* o, float* lse, int32_t* queue, vsa_stream_t stream) {
   if (dtype != VSA_BF16 && dtype != VSA_F16) return VSA_ERR_INVALID_ARG;
   if (!plan || !aligned16(q_codes) || !aligned16(q_scales) || !aligned16(k_codes) || !aligned16(k_scales) ||
       !aligned16(v) || !aligned16(o) || !aligned16(lse))
@@ -515,7 +516,26 @@ int vsa_sparse_attn_fwd_nvfp4(vsa_plan_t plan, vsa_dtype_t dtype, const uint8_t*
   a.status = ds->status;
   a.num_sms = ds->num_sms;
   a.f16 = dtype == VSA_F16;
+  a.queue = queue;
   return from_cuda(vsa::launch_attn_fwd_nvfp4(g, a, reinterpret_cast<cudaStream_t>(stream)));
+}
+}  // namespace
+
+int vsa_sparse_attn_fwd_nvfp4(vsa_plan_t plan, vsa_dtype_t dtype, const uint8_t* q_codes, const uint8_t* q_scales,
+                              const uint8_t* k_codes, const uint8_t* k_scales, const uint16_t* v,
+                              const int32_t* q2k_idx, const int32_t* q2k_num, int max_k, int B, int H, int D,
+                              uint16_t* o, float* lse, vsa_stream_t stream) {
+  return sparse_attn_fwd_nvfp4_impl(plan, dtype, q_codes, q_scales, k_codes, k_scales, v, q2k_idx, q2k_num, max_k,
+                                    B, H, D, o, lse, nullptr, stream);
+}
+
+int vsa_sparse_attn_fwd_nvfp4_ws(vsa_plan_t plan, vsa_dtype_t dtype, const uint8_t* q_codes, const uint8_t* q_scales,
+                                 const uint8_t* k_codes, const uint8_t* k_scales, const uint16_t* v,
+                                 const int32_t* q2k_idx, const int32_t* q2k_num, int max_k, int B, int H, int D,
+                                 uint16_t* o, float* lse, int32_t* workspace, vsa_stream_t stream) {
+  if (!aligned16(workspace)) return VSA_ERR_INVALID_ARG;
+  return sparse_attn_fwd_nvfp4_impl(plan, dtype, q_codes, q_scales, k_codes, k_scales, v, q2k_idx, q2k_num, max_k,
+                                    B, H, D, o, lse, workspace, stream);
 }
 
 int vsa_sparse_attn_bwd_workspace(vsa_plan_t plan, int B, int H, int max_k, size_t* bytes) {

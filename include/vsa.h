@@ -367,6 +367,24 @@ VSA_API int vsa_sparse_attn_fwd_nvfp4(vsa_plan_t plan, vsa_dtype_t dtype, const 
                                       int B, int H, int D, uint16_t *o, float *lse, vsa_stream_t stream);
 
 /*
+ * vsa_sparse_attn_fwd_nvfp4 with a caller workspace: for 64-token plans of at
+ * most 1024 blocks (four query blocks per work item) the items are handed out
+ * from a shared queue, prefix groups first, as in vsa_sparse_attn_fwd_ws.
+ * Same results bit for bit.
+ *   workspace : 2 int32 of device memory, 16-byte aligned, caller-owned, zero
+ *               before the first call; each call leaves it zero unless it
+ *               reports VSA_ERR_TIMEOUT.  Calls that share a workspace must not
+ *               run concurrently.  Unused by 256-token plans.
+ * Errors: as vsa_sparse_attn_fwd_nvfp4; VSA_ERR_INVALID_ARG for a null or
+ * misaligned workspace.
+ */
+VSA_API int vsa_sparse_attn_fwd_nvfp4_ws(vsa_plan_t plan, vsa_dtype_t dtype, const uint8_t *q_codes,
+                                         const uint8_t *q_scales, const uint8_t *k_codes, const uint8_t *k_scales,
+                                         const uint16_t *v, const int32_t *q2k_idx, const int32_t *q2k_num,
+                                         int max_k, int B, int H, int D, uint16_t *o, float *lse,
+                                         int32_t *workspace, vsa_stream_t stream);
+
+/*
  * Backward of the fine stage with the selection held fixed (the FastVideo
  * commit log keeps the grad path on separate kernels; the pages print no
  * formula, so this is the derivative of the fine stage): with

@@ -261,3 +261,7 @@ def test_fine_stage_with_workspace_checks_it(L):
     assert call(M) == vsa.VSA_ERR_INVALID_ARG
     assert L.vsa_sparse_attn_fwd_ws(p.handle, vsa.VSA_BF16, F, F, F, F, F, 4, 1, 2, 96, F, F, F, None) \
         == vsa.VSA_ERR_UNSUPPORTED
+    call4 = lambda ws: L.vsa_sparse_attn_fwd_nvfp4_ws(p.handle, vsa.VSA_BF16, F, F, F, F, F, F, F, 4, 1, 2, 128,
+                                                     F, F, ws, None)
+    assert call4(None) == vsa.VSA_ERR_INVALID_ARG
+    assert call4(M) == vsa.VSA_ERR_INVALID_ARG

@@ -288,3 +288,45 @@ def test_fp4_cosine_to_bf16_per_call(name):
     cos = float(torch.nn.functional.cosine_similarity(o4.reshape(1, -1), o16.reshape(1, -1)).item())
     print(f"{name}: cosine(o_fp4, o_bf16) = {cos:.5f}")
     assert cos >= 0.99, cos
+
+
+def test_fp4_grouped_every_stream_shape_and_repeats():
+    """64-token tiles run four query blocks per item in the NVFP4 kernel too:
+    crafted groups reaching every shape of the two Q tiles' key streams (empty
+    Q tile on either side, all or no shared blocks, tails on either side, an
+    odd shared count), then lists that repeat an id (those groups walk the
+    lists as given), against the oracle's NVFP4 attention."""
+    from tests.test_gpu_grouped64 import _stream_shapes
+    wl = _wl((8, 16, 16, (4, 4, 4), 0), H_=1)
+    g = oracle.geometry_of(wl)
+    assert g.NB == 32
+    inp = workloads.make_inputs(wl)
+    qt, kt, vt = (oracle.tile(g, inp[n]) for n in ("q", "k", "v"))
+    idx, num = _stream_shapes(g.NB)
+    _fp4_vs_oracle(wl, qt, kt, vt, idx, num, what="fp4 stream shapes")
+    idx[0, 0, 9, :3] = [13, 13, 1]   # group 2: a repeat
+    num[0, 0, 9] = 3
+    idx[0, 0, 30, :2] = [16, 16]     # group 7
+    num[0, 0, 30] = 2
+    _fp4_vs_oracle(wl, qt, kt, vt, idx, num, what="fp4 repeats")
+
+
+def test_fp4_shared_queue_gives_the_static_results():
+    """vsa_sparse_attn_fwd_nvfp4_ws: the 64-token groups handed out from a
+    shared queue give bit for bit the static assignment's results on the full
+    tile64 workload, twice in a row; the workspace is zero after each call."""
+    wl = workloads.WORKLOADS["tile64"]
+    ref = H.oracle_front(wl)
+    plan = vsa.Plan.of(wl)
+    (qc, qs), (kc, ks) = oracle.quant_nvfp4(ref["qt"]), oracle.quant_nvfp4(ref["kt"])
+    args = (plan, _u8(qc), _u8(sf_layout(qs)), _u8(kc), _u8(sf_layout(ks)), H.to_dev(ref["vt"]),
+            torch.from_numpy(ref["idx"]).cuda(), torch.from_numpy(ref["num"]).cuda())
+    o0, l0 = vsa.sparse_attn_fwd_nvfp4(*args)
+    ws = torch.zeros(4, dtype=torch.int32, device="cuda")
+    for _ in range(2):
+        o1, l1 = vsa.sparse_attn_fwd_nvfp4(*args, workspace=ws)
+        torch.cuda.synchronize()
+        assert vsa.get_status() == vsa.VSA_OK
+        assert int(ws.abs().sum()) == 0
+        assert torch.equal(o0.view(torch.int16), o1.view(torch.int16))
+        assert torch.equal(l0.view(torch.int32), l1.view(torch.int32))

@@ -15,7 +15,9 @@ query tile's product) and each query tile's number of tiles (zero
 included); later steps load one stage per query tile, and a step past one
 query tile's end runs the other alone.  So the MMA warp keeps per-query-tile
 counters for the p_full and o_empty phases, and a softmax warpgroup sits
-out the groups that have no tile for it.  With a shared
+out the groups that have no tile for it.  In the NVFP4 variant the scales of
+S_i are copied into the other query tile's S columns (free once that tile's
+softmax has loaded its latest S, signalled on s_read) before S_i is issued.  With a shared
 queue (a caller workspace) the builder takes group tickets and, past the last
 group, publishes an end marker the consumers stop on.  Q is released
 (q_empty) once the group's last S product has been issued, so the next
@@ -34,9 +36,10 @@ from tests.test_fwd_protocol_model import Model as FwdModel
 
 
 class GroupedModel(FwdModel):
-    def __init__(self, groups, seed, plant=None, skip_every=3, sentinel=False):
+    def __init__(self, groups, seed, plant=None, skip_every=3, sentinel=False, fp4=False):
         super().__init__([], False, 256, seed, plant)
-        self.KS, self.VS = 2, 3         # the grouped kernel's K and V ring stages
+        self.fp4 = fp4
+        self.KS, self.VS = (4, 4) if fp4 else (2, 3)  # the grouped kernel's K and V ring stages
         for st in range(self.KS):
             self.bar(("k_full", st)), self.bar(("k_empty", st))
         for st in range(self.VS):
@@ -131,6 +134,10 @@ class GroupedModel(FwdModel):
                     st["sk"] = st["kit"] % self.KS
                     yield ("wait", ("k_full", st["sk"]), st["kit"] // self.KS + 1)
                 tag = "sh" if shared else j
+                if self.fp4:  # scales into the other tile's S columns, once its latest S is loaded
+                    if sn[1 - j] > 0 and self.plant != "no_s_read_wait":
+                        yield ("wait", ("s_read", 1 - j), sn[1 - j])
+                    yield ("pipe", ("cp", j, sn[j]))
                 yield ("pipe", ("S", j, sn[j], st["sk"], (gl, u, tag), gl))
                 yield ("pipe", ("commit", ("s_full", j)))
                 sn[j] += 1
@@ -205,6 +212,8 @@ class GroupedModel(FwdModel):
                     yield ("skip_S", i, w, tiles)  # nothing selected: S is not loaded
                 else:
                     yield ("ld_S", i, w, tiles)
+                if self.fp4:
+                    yield ("arrive", ("s_read", i), 32, tiles)
                 yield ("st_P", i, w, gl, t)
                 if t > 0:
                     yield ("rescale_O", i, gl, t)
@@ -225,10 +234,16 @@ class GroupedModel(FwdModel):
                 self.read_smem(("q", c), gl)
             for c in range(2):
                 self.read_smem(("k", sk, c), kver)
+            if self.fp4:
+                if self.hi[1 - i] != ("sf", i, u):
+                    raise Hazard(f"S{i}#{u} reads scales {self.hi[1 - i]}")
+                self.sf_used.add(("sf", i, u))
             if self.s_val[i] is not None and len(self.s_loaded[i]) < 4:
                 raise Hazard(f"S{i}#{u} overwrites S{i}#{self.s_val[i]} before it was loaded")
             if self.p[i] is not None and self.p[i][0] != "read":
                 raise Hazard(f"S{i}#{u} overwrites P{i} {self.p[i][:3]} before P V read it")
+            if self.hi[i] is not None and self.hi[i][0] == "sf" and self.hi[i] not in self.sf_used:
+                raise Hazard(f"S{i}#{u} overwrites unread scales {self.hi[i]}")
             self.s_val[i], self.s_loaded[i], self.hi[i], self.p[i] = u, set(), ("S", u), None
             return
         if op[0] == "PV":  # the V stage carries its query tile's tag; P and O as in the base model
@@ -296,12 +311,14 @@ GROUP_SETS = [
 ]
 
 
+@pytest.mark.parametrize("fp4", [False, True], ids=["16bit", "nvfp4"])
 @pytest.mark.parametrize("sentinel", [False, True], ids=["static", "queue"])
 @pytest.mark.parametrize("groups", range(len(GROUP_SETS)))
 @pytest.mark.parametrize("skip_every", [2, 3, 5])
-def test_grouped_protocol_has_no_deadlock_alias_or_hazard(groups, skip_every, sentinel):
+def test_grouped_protocol_has_no_deadlock_alias_or_hazard(groups, skip_every, sentinel, fp4):
     for seed in range(8):
-        GroupedModel(GROUP_SETS[groups], seed=100 * groups + seed, skip_every=skip_every, sentinel=sentinel).run()
+        GroupedModel(GROUP_SETS[groups], seed=100 * groups + seed, skip_every=skip_every, sentinel=sentinel,
+                     fp4=fp4).run()
 
 
 def test_queue_with_no_group_for_this_cta_ends_cleanly():
@@ -317,13 +334,14 @@ def test_queue_with_no_group_for_this_cta_ends_cleanly():
     "q_free_first_s",         # Q released after the group's first S instead of its last
     "split_as_shared",        # a step with one tile per query tile read from one stage
     "v_free_first_pv",        # a shared V stage released by the first query tile's P V
+    "no_s_read_wait",         # NVFP4: scales copied before the other tile's softmax loaded its S
 ])
 def test_grouped_planted_mistakes_are_caught(plant):
     caught = 0
     for seed in range(40):
         try:
             GroupedModel([(1, 3, 2, 2), (0, 2, 0, 1), (2, 4, 3, 2), (0, 1, 0, 1), (0, 2, 3, 2), (0, 3, 0, 1)],
-                         seed=seed, plant=plant).run()
+                         seed=seed, plant=plant, fp4=plant == "no_s_read_wait").run()
         except Hazard:
             caught += 1
     assert caught > 0, plant
