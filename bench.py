@@ -38,7 +38,7 @@ PROFILE = os.path.join(ROOT, "profiles", "attn_fwd_fastwan.md")
 ATTN_SOURCES = [os.path.join(ROOT, "block_sparse_video_gather_b200", "csrc", f)
                 for f in ("attn_fwd.cu", "fwd_common.cuh", "common.cuh", "tiles.cuh")]
 GROUPED_SOURCES = [os.path.join(ROOT, "block_sparse_video_gather_b200", "csrc", f)
-                   for f in ("attn_fwd_grouped.cu", "fwd_common.cuh", "common.cuh", "tiles.cuh")]
+                   for f in ("attn_fwd_grouped.cu", "fwd_common.cuh", "nvfp4.cuh", "common.cuh", "tiles.cuh")]
 # committed ncu summaries that carry the DRAM traffic of one fine-stage launch:
 # workload -> (summary, the kernel sources its source_hash covers)
 TRAFFIC_PROFILES = {
@@ -47,7 +47,12 @@ TRAFFIC_PROFILES = {
 }
 FP4_PROFILE = os.path.join(ROOT, "profiles", "attn_fwd_fp4_fastwan.md")
 FP4_SOURCES = [os.path.join(ROOT, "block_sparse_video_gather_b200", "csrc", f)
-               for f in ("fp4.cu", "common.cuh", "tiles.cuh")]
+               for f in ("fp4.cu", "nvfp4.cuh", "common.cuh", "tiles.cuh")]
+# NVFP4 fine stage: workload -> (summary, sources); 64-token plans run the grouped kernel's NVFP4 variant
+FP4_TRAFFIC_PROFILES = {
+    "fastwan": (FP4_PROFILE, FP4_SOURCES),
+    "tile64": (os.path.join(ROOT, "profiles", "attn_fwd_fp4_grouped64_tile64.md"), GROUPED_SOURCES),
+}
 WORKLOAD_TEXT = {
     "tiny": "tiny grid 8x16x16, B1 H2 D128, block 4x8x8, topk 4",
     "fastwan": "FastWan2.2-TI2V-5B latent grid 31x22x40, B1 H24 D128, block 4x8x8, topk 64",
@@ -738,7 +743,9 @@ def main():
         achieved = flops / attn_avg / 1e12
         achieved_real = flops_real / attn_avg / 1e12
         if args.nvfp4:
-            traffic = profile_traffic(args.workload, FP4_PROFILE, FP4_SOURCES)
+            traffic = (profile_traffic(args.workload, *FP4_TRAFFIC_PROFILES[args.workload])
+                       if args.workload in FP4_TRAFFIC_PROFILES and args.heads is None and args.frames is None
+                       else None)
         elif args.workload in TRAFFIC_PROFILES and args.heads is None and args.frames is None:
             traffic = profile_traffic(args.workload, *TRAFFIC_PROFILES[args.workload])
         else:
@@ -778,9 +785,9 @@ def main():
             },
             "roofline": {
                 "bound": "tensor",
-                "kernel": ("attn_fwd_fp4_kernel" if args.nvfp4 else
-                           "attn_fwd_grouped64_kernel" if (wl.block_tokens == 64 and wl.num_blocks <= 1024)
-                           else "attn_fwd_kernel"),
+                "kernel": ("attn_fwd_grouped64_kernel" + ("<nvfp4>" if args.nvfp4 else "")
+                           if (wl.block_tokens == 64 and wl.num_blocks <= 1024)
+                           else "attn_fwd_fp4_kernel" if args.nvfp4 else "attn_fwd_kernel"),
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "achieved_real_tokens": achieved_real, "frac_real_tokens": achieved_real / peak,
                 "peak_source": peak_source,
