@@ -26,6 +26,9 @@
  * fine stage's gradients for a fixed selection.  The _ex calls and
  * vsa_tile_coarse take bf16 or fp16.  For FP4 Q and K, vsa_quantize_nvfp4
  * (tiled q, tiled k) and vsa_sparse_attn_fwd_nvfp4 replace the fine stage.
+ * vsa_tile_coarse_prefix is the one-launch front end with the tile-64
+ * selection.  The _ws fine-stage calls take a caller workspace with which
+ * the 64-token kernel hands out its work items from a shared queue.
  *
  * Conventions shared by every call
  *  - bf16 / fp16 tensors are passed as pointers to their raw 16-bit patterns.
