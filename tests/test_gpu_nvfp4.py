@@ -330,3 +330,18 @@ def test_fp4_shared_queue_gives_the_static_results():
         assert int(ws.abs().sum()) == 0
         assert torch.equal(o0.view(torch.int16), o1.view(torch.int16))
         assert torch.equal(l0.view(torch.int32), l1.view(torch.int32))
+
+
+def test_fp4_beyond_bitmap_capacity_uses_the_per_item_kernel():
+    """NB = 2048 > 1024 64-token blocks: the NVFP4 fine stage runs one query
+    block per item (the per-item kernel's 64-token path) instead of groups."""
+    wl = _wl((32, 64, 64, (4, 4, 4), 0), H_=1)
+    g = oracle.geometry_of(wl)
+    assert g.NB == 2048
+    inp = workloads.make_inputs(wl)
+    qt, kt, vt = (oracle.tile(g, inp[n]) for n in ("q", "k", "v"))
+    idx, num = _random_selection(g, 1, seed=41, max_k=3)
+    rng = np.random.default_rng(42)
+    real = np.flatnonzero(H.real_rows(wl))
+    rows = np.unique(np.concatenate([rng.choice(real, 600, replace=False), real[:4], real[-4:]]))
+    _fp4_vs_oracle(wl, qt, kt, vt, idx, num, rows=rows, what="fp4 NB 2048")
