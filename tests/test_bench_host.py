@@ -50,3 +50,21 @@ def test_real_token_flops_count_real_query_and_key_tokens():
     wl64 = workloads.custom(T=4, Hg=8, Wg=8, block=(4, 4, 4), n_prefix=100, H=1)
     np.testing.assert_array_equal(bench.block_real_tokens(wl64),
                                   oracle.block_valid_counts(oracle.geometry_of(wl64)))
+
+
+def test_committed_traffic_summaries_parse_and_name_their_workload():
+    """Every ncu summary bench.py reads a per-launch DRAM figure from carries the
+    three machine-read lines, for the workload it is filed under; the figure is
+    used only while the hash of the kernel sources matches."""
+    import re
+    entries = list(bench.TRAFFIC_PROFILES.items()) + list(bench.FP4_TRAFFIC_PROFILES.items())
+    for workload, (path, sources) in entries:
+        text = open(path).read()
+        assert re.search(r"source_hash:\s*[0-9a-f]{16}", text), path
+        assert re.search(r"bench_workload:\s*" + workload + r"\b", text), path
+        m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+        assert m and float(m.group(1)) > 0, path
+        got = bench.profile_traffic(workload, path, sources)
+        fresh = re.search(r"source_hash:\s*([0-9a-f]+)", text).group(1) == bench.attn_source_hash(sources)
+        assert (got == float(m.group(1))) if fresh else got is None, path
+        assert bench.profile_traffic("tiny", path, sources) is None  # another workload's summary never applies
