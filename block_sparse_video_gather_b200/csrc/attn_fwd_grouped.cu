@@ -1,9 +1,12 @@
 // attn_fwd_grouped.cu -- fine stage of VSA for 64-token blocks (the tile-64
 // layout of the FastVideo commit log, examples/inference/basic/README.md:
 // rows of any length, zero included), with four query blocks per work item,
-// two per 128-row Q tile, each Q tile over the union of its two selections.  "FastVideo VSA" (vLLM-Omni user
-// guide), introduction: each query block attends only to the tokens of its
-// selected blocks; non-causal; scale head_size^-1/2.
+// two per 128-row Q tile, each Q tile over the union of its two selections;
+// Q and K 16-bit, or NVFP4 (FastVideo "Optimizations" page, section "FP4
+// Flash Attention 4": E2M1 codes with E4M3 scales, V and P 16-bit).
+// "FastVideo VSA" (vLLM-Omni user guide), introduction: each query block
+// attends only to the tokens of its selected blocks; non-causal; scale
+// head_size^-1/2.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -41,13 +44,15 @@ using namespace fwd;
 //
 // A fourth role builds the groups: warp 2 reads the four index rows, sets one
 // bit per (query block, selected block) in shared-memory bitmaps (double
-// buffered, two groups ahead), ORs them into the union, counts the tiles and
-// hands the group over on grp_full; the eleven consuming warps (the K and V
-// producers, MMA, eight softmax warps) release it on grp_free.  Block ids outside [0, NB) are
-// skipped and counts outside [0, max_k] clamped (both reported); a list that
-// names a block twice puts the whole group in list order instead ("concat":
-// each query block's list, two ids per tile, only that block's rows unmasked),
-// so a repeated id counts twice as in the ungrouped kernel.
+// buffered, two groups ahead), forms the bitmap of the blocks both Q tiles
+// selected, counts each Q tile's tiles and hands the group over on grp_full;
+// the eleven consuming warps (the K and V producers, MMA, eight softmax
+// warps) release it on grp_free.  Block ids outside [0, NB) are skipped and
+// counts outside [0, max_k] clamped (both reported); a list that names a
+// block twice puts the whole group in list order instead ("concat": each
+// query block's list, two ids per tile, only that block's rows unmasked, the
+// same stream for both Q tiles), so a repeated id counts twice as in the
+// ungrouped kernel.
 //
 // Groups go to CTAs statically (every gridDim.x-th group) or, with a caller
 // workspace, through a shared queue: the builder takes tickets with an atomic
