@@ -81,7 +81,7 @@ template <>
 struct GMap<false> {
   static constexpr int kKS = 2, kVS = 3;
   static constexpr uint32_t kQ = 0, kQsf = 0, kK = kQ + 2 * kTileBytes, kKsf = 0;
-  static constexpr uint32_t kKStage = kTileBytes, kKsfStage = 0, kQTile = kTileBytes;
+  static constexpr uint32_t kKStage = kTileBytes, kKsfStage = 0;
   static constexpr uint32_t kV = kK + kKS * kKStage;
   static constexpr uint32_t kBar = kV + kVS * kTileBytes;
 };
