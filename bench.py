@@ -87,6 +87,32 @@ def block_real_tokens(wl) -> np.ndarray:
     return np.concatenate([np.array(pre, dtype=np.int64), video])
 
 
+def grouped_products(idx: np.ndarray, num: np.ndarray, NB: int) -> int:
+    """Q-tile products the grouped 64-token fine stage executes (one 128-row Q
+    tile against one 128-key tile, an S and a P V product): per group of four
+    query blocks, each Q tile (blocks 0-1, 2-3) walks the union of its two
+    selections two blocks per tile; a group whose lists repeat an id walks the
+    four lists as given (two ids per tile) for every Q tile.  Ids outside
+    [0, NB) are skipped and counts clamped, as the kernel does."""
+    idx = np.asarray(idx, dtype=np.int64)
+    num = np.clip(np.asarray(num, dtype=np.int64), 0, idx.shape[-1])
+    total = 0
+    for b in range(idx.shape[0]):
+        for h in range(idx.shape[1]):
+            for g0 in range(0, NB, 4):
+                rows = list(range(g0, min(g0 + 4, NB)))
+                cnts = [int(num[b, h, r]) for r in rows]
+                lists = [[int(x) for x in idx[b, h, r, :c] if 0 <= x < NB] for r, c in zip(rows, cnts)]
+                nq = (len(rows) + 1) // 2
+                if any(len(set(lst)) != len(lst) for lst in lists):
+                    total += nq * sum((c + 1) // 2 for c in cnts)
+                    continue
+                for q in range(nq):
+                    union = set().union(*lists[2 * q:2 * q + 2])
+                    total += (len(union) + 1) // 2
+    return total
+
+
 def real_token_flops(wl, idx: np.ndarray, num: np.ndarray) -> float:
     """4 * D * (real query tokens) * (real key tokens) summed over the selected
     (query block, key block) pairs: the work on real tokens only."""
@@ -635,6 +661,11 @@ def main():
     assert vsa.get_status() == vsa.VSA_OK
     flops = selected_flops(wl, fwd.num.cpu().numpy())
     flops_real = real_token_flops(wl, fwd.idx.cpu().numpy(), fwd.num.cpu().numpy())
+    grouped = wl.block_tokens == 64 and wl.num_blocks <= 1024
+    # the grouped 64-token kernel computes whole 128x128 products of which the
+    # selection uses part: its executed FLOPs, 4 D 128^2 per Q-tile product
+    flops_exec = (4.0 * wl.D * 128 * 128 * grouped_products(fwd.idx.cpu().numpy(), fwd.num.cpu().numpy(),
+                                                             wl.num_blocks) if grouped else None)
     fp4_cosine = None
     if args.nvfp4 and not args.gate:
         # the page's quality figure for FP4 attention: per-call cosine similarity of
@@ -790,6 +821,9 @@ def main():
                            else "attn_fwd_fp4_kernel" if args.nvfp4 else "attn_fwd_kernel"),
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "achieved_real_tokens": achieved_real, "frac_real_tokens": achieved_real / peak,
+                **({"executed_tflop_per_launch": flops_exec / 1e12,
+                    "achieved_executed": flops_exec / attn_avg / 1e12,
+                    "frac_executed": flops_exec / attn_avg / 1e12 / peak} if flops_exec else {}),
                 "peak_source": peak_source,
                 "traffic": traffic,
             },

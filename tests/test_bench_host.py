@@ -68,3 +68,26 @@ def test_committed_traffic_summaries_parse_and_name_their_workload():
         fresh = re.search(r"source_hash:\s*([0-9a-f]+)", text).group(1) == bench.attn_source_hash(sources)
         assert (got == float(m.group(1))) if fresh else got is None, path
         assert bench.profile_traffic("tiny", path, sources) is None  # another workload's summary never applies
+
+
+def test_grouped_products_count_each_q_tiles_union():
+    """Executed Q-tile products of the grouped 64-token kernel, on groups built
+    to take every shape of the two Q tiles' streams: each Q tile walks the union
+    of its two query blocks' selections, two blocks per 128-key tile."""
+    import numpy as np
+    from tests.test_gpu_grouped64 import _stream_shapes
+    idx, num = _stream_shapes(32)
+    # per group: ceil(|union of blocks 0-1| / 2) + ceil(|union of blocks 2-3| / 2)
+    assert bench.grouped_products(idx, num, 32) == (0 + 3) + (2 + 0) + (4 + 4) + (5 + 2) + (1 + 6) + (5 + 6) \
+        + (2 + 2) + (2 + 2)
+    # a list that repeats an id: that group walks the four lists as given for both Q tiles
+    idx2, num2 = idx.copy(), num.copy()
+    idx2[0, 0, 9, :3] = [13, 13, 1]
+    num2[0, 0, 9] = 3
+    per_list = sum((int(c) + 1) // 2 for c in num2[0, 0, 8:12])
+    assert bench.grouped_products(idx2, num2, 32) == bench.grouped_products(idx, num, 32) - 8 + 2 * per_list
+    # ids outside [0, NB) are skipped; an all-dense group of two query blocks (NB % 4 == 2)
+    dense = np.broadcast_to(np.arange(6, dtype=np.int32), (1, 1, 6, 6)).copy()
+    assert bench.grouped_products(dense, np.full((1, 1, 6), 6, np.int32), 6) == 3 + 3 + 3
+    dense[0, 0, 5, 0] = 99
+    assert bench.grouped_products(dense, np.full((1, 1, 6), 6, np.int32), 6) == 3 + 3 + 3
