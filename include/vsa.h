@@ -315,8 +315,9 @@ VSA_API int vsa_sparse_attn_fwd_ex(vsa_plan_t plan, vsa_dtype_t dtype, const uin
 
 /*
  * vsa_sparse_attn_fwd_ex with a caller workspace that lets the 64-token
- * fine stage (four query blocks per work item over the union of their
- * selections) hand out its work items from a shared queue -- the items whose
+ * fine stage (four query blocks per work item, two per 128-row query tile,
+ * each query tile over the union of its two selections) hand out its work
+ * items from a shared queue -- the items whose
  * query blocks are prefix tiles (dense under the tile-64 rule) first -- instead
  * of a fixed item-to-CTA assignment.  Same results bit for bit; the schedule
  * is this library's, the pages have no counterpart.
